@@ -1,0 +1,417 @@
+"""Benchmark: one GLM-5.2-shaped MoE layer forward, decode of 1 token.
+
+Workload: hidden 6144, expert inter 2048, 256 routed experts + 1 shared,
+top-8, sigmoid router with correction bias, int4 weights with one F32 scale
+per row, Q8_0 activations; synthetic seeded weights (x ~ N(0,1),
+W_r ~ N(0,0.006), bias ~ U(-0.05,0.05), experts ~ N(0,0.01)).  A step is one
+token through one layer: every step of the hot path (activation Q8, router,
+top-k, bucketing, gate/up + SwiGLU + Q8, down, combine).  Eight distinct
+layers (~39 GB) stay resident and the steps cycle through them, so each
+step streams ~170 MB of expert weights that the 126 MB L2 cannot hold from
+an earlier step.  Steps are replayed from CUDA graphs of up to 64 steps.
+
+Metric: MoE-layer tokens/s (value) and streamed int4 weight GB/s (roofline).
+
+Multi-GPU (torchrun): every rank holds its own replica of the 8 layers and
+runs its own tokens (data parallel, no collective on the data path); the
+step time is the max over ranks.
+
+--impl reference runs the oracle (single-threaded C) on the host cores on the
+same workload, one token through one layer per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s & streamed int4 weight GB/s (% of HBM peak), 1xB200"
+WORKLOAD = ("GLM-5.2-shaped MoE layer decode, 1 token (hidden 6144, expert inter 2048, "
+            "256 routed + 1 shared experts, top-8)")
+N_LAYERS = 8
+N_TOK_POOL = 64
+GRAPH_STEPS = 64
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=16384)
+    p.add_argument("--warmup", type=int, default=512)
+    p.add_argument("--impl", default="coli", choices=["coli", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample-tokens", type=int, default=4)
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except FileNotFoundError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None, "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host (cpu_baseline and --impl reference)
+
+
+def oracle_pool(n_pairs: int):
+    """Oracle inputs for n_pairs (layer, token) decode steps of the workload:
+    (layer l = i % 8, token i); the experts each routing selects are generated
+    and quantised here, outside any timing."""
+    import numpy as np
+
+    import oracle
+    import synth
+    from tests.helpers import oracle_expert
+
+    cfg = synth.config("decode1")
+    xs = synth.tokens(cfg, N_TOK_POOL)
+    jobs = []
+    for i in range(n_pairs):
+        layer = i % N_LAYERS
+        x = xs[i:i + 1]
+        W, b = synth.router_w(cfg, layer), synth.bias(cfg, layer)
+        _, idx, _ = oracle.route(x, W, b, cfg["top_k"], True, cfg["routed_scaling_factor"])
+        experts = {int(e): oracle_expert(cfg, layer, int(e)) for e in np.unique(idx)}
+        shared = [oracle_expert(cfg, layer, 0, shared=True)]
+        jobs.append((W, b, experts, shared, x))
+    return cfg, jobs
+
+
+def oracle_step(cfg, job):
+    import oracle
+    W, b, experts, shared, x = job
+    oracle.moe_layer(cfg, W, b, experts, shared, x)
+
+
+def oracle_token_layer_seconds(n_tokens: int):
+    """Single-threaded oracle seconds per (1 token through 1 layer), over
+    n_tokens distinct tokens and layers."""
+    cfg, jobs = oracle_pool(n_tokens)
+    t0 = time.perf_counter()
+    for job in jobs:
+        oracle_step(cfg, job)
+    dt = time.perf_counter() - t0
+    return dt / n_tokens, (f"{n_tokens} decode tokens, one layer each (layers 0..{min(n_tokens, N_LAYERS) - 1}),"
+                           " full layer forward by the oracle")
+
+
+REF_BUDGET_S = 120.0
+
+
+def run_reference(args):
+    """The oracle on the host cores as the reference arm.  One step = one
+    decode token through one layer, computed in full by the oracle.  The
+    oracle needs ~1-2 s per step, so at most REF_BUDGET_S seconds of steps are
+    run (the count is reported in "steps"); inputs cycle over 2 (layer, token)
+    pairs whose experts are prepared before timing."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg, jobs = oracle_pool(2)
+    t0 = time.perf_counter()
+    for i in range(max(1, min(args.warmup, 1))):
+        oracle_step(cfg, jobs[i % 2])
+    est = time.perf_counter() - t0
+    n = max(1, min(args.steps, int(REF_BUDGET_S / max(est, 1e-3))))
+    t0 = time.perf_counter()
+    for i in range(n):
+        oracle_step(cfg, jobs[i % 2])
+    dt = time.perf_counter() - t0
+    value = n / dt
+    sample = (f"{n} of the requested {args.steps} steps (budget {REF_BUDGET_S:.0f} s); each step one decode "
+              "token through one full layer, single-threaded oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": n, "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": dt / n * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4xint8->f32",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "layers_resident": N_LAYERS, "tokens_per_step": 1},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import int4_weight_only_sigmoid_b200 as coli
+    import synth
+    from synth.layers import device_layer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    coli.load()
+    cfg = synth.config("decode1", seed=rank)  # each rank: its own replica, its own tokens
+    H = cfg["hidden"]
+    staging = torch.empty(cfg["inter"] * H, dtype=torch.float32, device=dev)
+    layers = [device_layer(cfg, l, device=dev, staging=staging) for l in range(N_LAYERS)]
+    del staging
+    cstructs = [L.cstruct() for L in layers]
+    xs = synth.dev_tokens(cfg, N_TOK_POOL, device=dev)
+    outs = torch.empty(2, 1, H, dtype=torch.float32, device=dev)
+    ws = coli.make_workspace(layers[0].cfg, 1, dev)
+    torch.cuda.synchronize()
+
+    # expert bytes actually streamed per step (unique selected experts + shared)
+    mat = cfg["inter"] * H // 2
+    expert_bytes = 3 * mat + (2 * cfg["inter"] + H) * 4
+    gateup_bytes_per_expert = 2 * mat + 2 * cfg["inter"] * 4
+    router_bytes = cfg["n_experts"] * H * 4 + cfg["n_experts"] * 4
+    uniq = []
+    for i in range(N_TOK_POOL):
+        _, idx, _ = coli.moe_route(layers[i % N_LAYERS], xs[i:i + 1])
+        uniq.append(len(torch.unique(idx)))
+    n_exp = [u + cfg["n_shared"] for u in uniq]
+
+    def step(i, stream, evs=None):
+        if evs is not None:
+            coli.arm_phase_events(*evs)
+        coli.moe_layer_forward(layers[i % N_LAYERS], xs[i % N_TOK_POOL:i % N_TOK_POOL + 1], out=outs[i % 2],
+                               workspace=ws, stream=stream, cstruct=cstructs[i % N_LAYERS])
+
+    # warm-up (also sets kernel attributes before any capture)
+    s = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(s):
+        for i in range(max(3, args.warmup)):
+            step(i, s)
+    torch.cuda.synchronize()
+
+    # graphs: a ring of NG graphs of G steps, each with its own phase events
+    K = args.steps
+    G = min(GRAPH_STEPS, K)
+    n_full, rem = divmod(K, G)
+    NG = 3
+
+    def capture(n_steps, base):
+        g = torch.cuda.CUDAGraph()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_steps)]
+        with torch.cuda.graph(g, stream=s):
+            for j in range(n_steps):
+                step(base + j, torch.cuda.current_stream(), evs[j])
+        return g, evs
+
+    ring = [capture(G, r * G) for r in range(NG)]
+    tail = capture(rem, 0) if rem else None
+    # each graph replay starts its steps at a fixed token/layer offset; the ring
+    # rotates over NG*G distinct (layer, token) steps
+    torch.cuda.synchronize()
+    for g, _ in ring:
+        g.replay()
+    torch.cuda.synchronize()
+
+    gate_ms, down_ms, gate_bytes, phase_n = 0.0, 0.0, 0.0, 0
+
+    def harvest(r, base_step):
+        nonlocal gate_ms, down_ms, gate_bytes, phase_n
+        g, evs = r
+        for j, (e0, e1, e2) in enumerate(evs):
+            e2.synchronize()
+            a, b = e0.elapsed_time(e1), e1.elapsed_time(e2)
+            if a <= 0 or b <= 0:
+                continue
+            gate_ms += a
+            down_ms += b
+            gate_bytes += n_exp[(base_step + j) % N_TOK_POOL] * gateup_bytes_per_expert
+            phase_n += 1
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clk = ClockSampler(vis.split(",")[local] if vis else local)
+    clk.start()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    pending = []
+    with torch.cuda.stream(s):
+        start.record(s)
+        for k in range(n_full):
+            r = ring[k % NG]
+            if len(pending) == NG:
+                harvest(*pending.pop(0))
+            r[0].replay()
+            pending.append((r, (k % NG) * G))
+        if tail is not None:
+            tail[0].replay()
+        end.record(s)
+    end.synchronize()
+    while pending:
+        harvest(*pending.pop(0))
+    if tail is not None:
+        harvest(tail, 0)
+    clocks = clk.stop()
+    elapsed_ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / K
+    tokens = K * world
+    value = tokens / (elapsed_ms / 1e3)
+
+    # streamed bytes of the whole step (router + experts) over the step time
+    mean_exp = sum(n_exp) / len(n_exp)
+    step_bytes = mean_exp * expert_bytes + router_bytes
+    peak, peak_kind = peaks()
+    gate_avg_ms = gate_ms / max(1, phase_n)
+    gate_gbs = (gate_bytes / max(1, phase_n)) / (gate_avg_ms * 1e-3) / 1e9 if gate_avg_ms > 0 else 0.0
+    step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host token in, host output back
+    e2e = None
+    if rank == 0 or world > 1:
+        hx = torch.empty(N_TOK_POOL, 1, H, dtype=torch.float32).pin_memory()
+        hx.copy_(xs.view(N_TOK_POOL, 1, H).cpu())
+        hout = torch.empty(2, 1, H, dtype=torch.float32).pin_memory()
+        dx = torch.empty(1, H, dtype=torch.float32, device=dev)
+        Ke = min(K, 1024)
+        ge = torch.cuda.CUDAGraph()
+        Ge = min(GRAPH_STEPS, Ke)
+        with torch.cuda.graph(ge, stream=s):
+            cs = torch.cuda.current_stream()
+            for j in range(Ge):
+                dx.copy_(hx[j % N_TOK_POOL], non_blocking=True)
+                coli.moe_layer_forward(layers[j % N_LAYERS], dx, out=outs[j % 2], workspace=ws, stream=cs,
+                                       cstruct=cstructs[j % N_LAYERS])
+                hout[j % 2].copy_(outs[j % 2], non_blocking=True)
+        ge.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        reps = max(1, Ke // Ge)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(reps):
+                ge.replay()
+            e1.record(s)
+        e1.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": reps * Ge * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": H * 4,
+               "d2h_bytes_per_step": H * 4, "steps": reps * Ge,
+               "note": "pinned H2D of the token, coli_moe_layer_forward, D2H of the output, per step"}
+        del ge
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sec, sample = oracle_token_layer_seconds(args.cpu_sample_tokens)
+        cpu = {"value": 1.0 / sec, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int4xint8->f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "layers_resident": N_LAYERS, "tokens_per_step": 1,
+                       "parallelism": f"dp{world} (replicas, no collective)",
+                       "l2": "inputs larger than L2: 8 resident layers cycled, ~170 MB of weights per step",
+                       "graph_steps": G, "mean_experts_streamed": mean_exp},
+            "streamed_gbs": step_gbs,
+            "streamed_frac_of_hbm": step_gbs / peak,
+            "roofline": {"bound": "hbm", "kernel": "gateup_kernel", "achieved": gate_gbs, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": gate_gbs / peak, "traffic": None,
+                         "avg_launch_ms": gate_avg_ms,
+                         "algorithmic_bytes_per_launch": gate_bytes / max(1, phase_n),
+                         "down_kernel_avg_ms": down_ms / max(1, phase_n)},
+            "e2e": e2e, "gpu_launches": K * 7, "clocks": clocks, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    for g, _ in ring:
+        del g
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * coli.h -- C ABI of libcoli, a B200 (sm_100a) implementation of one
+ * GLM-5.2-shaped MoE layer forward: sigmoid router with correction-bias
+ * top-k, token->expert bucketing, SwiGLU experts with packed int4 weights
+ * (one F32 scale per row) and Q8_0 int8 activations reduced as integer dot
+ * products, and the score-weighted combine plus the shared expert.
+ *
+ * Sources (page title, then section):
+ *  [W] "GLM-5.2-colibri-int4架构解析MoE专家混合与INT4量化原理" (wmrh.cn):
+ *      "GLM-5.2的MoE实现", "MoE的工作原理", "GLM-5.2-colibri-int4的量化流程",
+ *      "高级配置选项 / 路由策略定制", "量化保留模块".
+ *  [C] "Colibri：在笔记本上跑744B参数的AI模型", "关键特性".
+ *  [D] "如何在普通电脑上运行 7440 亿参数神经网络" (devtrends.cc),
+ *      "引擎是如何工作的".
+ *  [H] HN summary (hn.213312.xyz, article 48842459), "已实现的功能".
+ *
+ * Conventions for every entry point:
+ *  - Data pointers are DEVICE pointers (CUDA global memory) owned by the
+ *    caller and 16-byte aligned; the library keeps no reference after the
+ *    call returns.  `stream` is a cudaStream_t (NULL = the legacy stream).
+ *  - Calls are asynchronous and stream-ordered.  A returned COLI_OK means
+ *    the work was validated and enqueued; results are ready once the stream
+ *    has been synchronised.
+ *  - The library allocates no device memory.  Scratch comes from the
+ *    caller's `workspace` (size from coli_moe_workspace_bytes).
+ *  - Host-detectable errors (null or misaligned pointers, unsupported
+ *    shapes, a workspace that is too small) return COLI_EINVAL at once and
+ *    enqueue nothing; a failed launch returns COLI_ECUDA.  coli_last_error()
+ *    then gives a message (per calling thread).
+ *  - n_tok == 0 is a no-op that returns COLI_OK.
+ *  - Weights are row-major [out x in]; an int4 row is in/2 bytes, element
+ *    2j in the low nibble of byte j, two's complement, plus one F32 scale.
+ *  - Results follow the written float-evaluation contracts (router R, row
+ *    fold F, combine C) so they can be compared bit for bit with a second
+ *    implementation: see the design notes.
+ */
+#ifndef COLI_H
+#define COLI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    COLI_OK = 0,
+    COLI_EINVAL = 1,   /* bad argument: nothing was enqueued */
+    COLI_ENOMEM = 2,   /* workspace too small */
+    COLI_ECUDA = 3,    /* a CUDA call or kernel launch failed */
+    COLI_ETIMEOUT = 4, /* a bounded device-side wait gave up */
+    COLI_EDEVICE = 5   /* a device-side check recorded an error */
+} coli_status;
+
+/* Layer shape and routing options ([W] "GLM-5.2的MoE实现": hidden 6144,
+ * expert inter 2048, 256 routed experts, 1 shared, 8 per token;
+ * [W] "路由策略定制": routed_scaling_factor, norm_topk_prob).
+ * Limits: hidden % 128 == 0; inter % 32 == 0; shared_inter % 32 == 0;
+ * 1 <= top_k <= min(n_experts, 16); n_experts <= 512; 0 <= n_shared <= 4. */
+typedef struct {
+    int32_t hidden;
+    int32_t inter;
+    int32_t n_experts;
+    int32_t top_k;
+    int32_t n_shared;
+    int32_t shared_inter;
+    int32_t norm_topk_prob;      /* nonzero: renormalise the selected scores */
+    float routed_scaling_factor; /* multiplies every routed weight */
+} coli_moe_config;
+
+/* One expert's packed weights (device pointers). */
+typedef struct {
+    const uint8_t* gate_q; /* [inter x hidden/2] */
+    const float* gate_s;   /* [inter] */
+    const uint8_t* up_q;   /* [inter x hidden/2] */
+    const float* up_s;     /* [inter] */
+    const uint8_t* down_q; /* [hidden x inter/2] */
+    const float* down_s;   /* [hidden] */
+} coli_expert;
+
+/* One MoE layer.  `experts` and `shared` are HOST arrays (n_experts and
+ * n_shared entries) of device-pointer sets; the router stays F32
+ * ([W] "量化保留模块"). */
+typedef struct {
+    coli_moe_config cfg;
+    const float* w_router;      /* [n_experts x hidden] F32, device */
+    const float* bias;          /* [n_experts] F32 correction bias, device */
+    const coli_expert* experts; /* host array [n_experts] */
+    const coli_expert* shared;  /* host array [n_shared] */
+} coli_moe_layer;
+
+/* Per-row int4 weight quantiser ([W] "GLM-5.2-colibri-int4的量化流程":
+ * rint, one F32 scale per row, packed into U8).  For each row:
+ * scale = absmax/7; q = rint(w/scale) clamped to [-8,7] (half to even); an
+ * all-zero row gets scale 0.  w: [rows x cols] F32; q_out: [rows x cols/2]
+ * bytes; scale_out: [rows] F32.  cols must be a positive multiple of 32. */
+coli_status coli_quantize_rows_int4(const float* w, int64_t rows, int64_t cols, uint8_t* q_out,
+                                    float* scale_out, void* stream);
+
+/* Q8_0-style activation quantiser ([C] "关键特性": Q8_0 风格 int8 激活).
+ * Per 32-element block of each token: d = absmax/127 (F32);
+ * q = rint(x/d) clamped to [-127,127]; an all-zero block gets d = 0.
+ * x: [n_tok x dim] F32; q_out: [n_tok x dim] int8; scale_out: [n_tok x dim/32].
+ * dim must be a positive multiple of 32. */
+coli_status coli_quantize_act_q8(const float* x, int64_t n_tok, int64_t dim, int8_t* q_out,
+                                 float* scale_out, void* stream);
+
+/* Router ([W] "MoE的工作原理", "路由策略定制"; [C] DeepSeek-V3 风格的 sigmoid
+ * 路由器).  scores[t,e] = sigmoid(x_t . W_r[e]) (F32, contract R); the top_k
+ * experts by scores + bias (ties to the lower index) in rank order go to
+ * topk_idx [n_tok x top_k]; topk_w [n_tok x top_k] gets the unbiased scores,
+ * divided by their sum when norm_topk_prob, times routed_scaling_factor.
+ * scores [n_tok x n_experts] is an output too (the caller's buffer). */
+coli_status coli_moe_route(const coli_moe_layer* layer, const float* x, int64_t n_tok, float* scores,
+                           int32_t* topk_idx, float* topk_w, void* stream);
+
+/* Bucketing, the pages' "batched MoE" ([H] "已实现的功能"; [D] 合并对相同
+ * 专家的请求): counts[e] = number of (token, slot) pairs routed to e;
+ * offsets = exclusive prefix sum [n_experts + 1]; perm [n_tok*top_k] lists
+ * the flat pair ids t*top_k + k sorted by (expert, token).  Integer output,
+ * unique.  Needs n_experts <= 512. */
+coli_status coli_moe_bucket(const int32_t* topk_idx, int64_t n_tok, int32_t top_k, int32_t n_experts,
+                            int32_t* counts, int32_t* offsets, int32_t* perm, void* stream);
+
+/* One SwiGLU expert on n_tok Q8 tokens ([C] integer dot kernels):
+ * g = gate.x, u = up.x (int4 x Q8 block dots, contract F), h = SiLU(g)*u,
+ * h re-quantised to Q8_0, y = down.h.  xq [n_tok x hidden] int8,
+ * xs [n_tok x hidden/32] F32, y_out [n_tok x hidden] F32.  `expert` points
+ * to ONE host-side coli_expert.  Workspace: coli_moe_workspace_bytes(cfg,
+ * n_tok) bytes is always enough. */
+coli_status coli_moe_expert_ffn(const coli_moe_config* cfg, const coli_expert* expert, const int8_t* xq,
+                                const float* xs, int64_t n_tok, float* y_out, void* workspace,
+                                size_t ws_bytes, void* stream);
+
+/* The layer: out[t] = sum_k w[t,k] * E_{idx[t,k]}(x_t) + sum_s S_s(x_t)
+ * ([W] "MoE的工作原理" weighted combine; shared experts always on).
+ * x, out: [n_tok x hidden] F32 (may not alias).  Each selected expert's
+ * weights are read once for all the tokens routed to it. */
+coli_status coli_moe_layer_forward(const coli_moe_layer* layer, const float* x, int64_t n_tok,
+                                   float* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* A pre-norm stack of MoE layers: x_{l+1} = x_l + MoE_l(RMSNorm(x_l)), with
+ * RMSNorm(x) = x / sqrt(mean(x^2) + eps) (weight 1).  layers: host array of
+ * n_layers layers with the same cfg.  x, out: [n_tok x hidden]. */
+coli_status coli_moe_stack_forward(const coli_moe_layer* layers, int32_t n_layers, const float* x,
+                                   int64_t n_tok, float eps, float* out, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
+/* RMSNorm alone (weight 1): y = x * (1/sqrtf(sum(x^2)/dim + eps)), the sum
+ * an fmaf chain in ascending element order.  x, y: [n_tok x dim]. */
+coli_status coli_rmsnorm(const float* x, int64_t n_tok, int64_t dim, float eps, float* y, void* stream);
+
+/* Bytes of workspace that coli_moe_layer_forward, coli_moe_stack_forward and
+ * coli_moe_expert_ffn need for up to max_tokens tokens (0 if cfg is
+ * invalid). */
+size_t coli_moe_workspace_bytes(const coli_moe_config* cfg, int64_t max_tokens);
+
+/* Message for the last non-OK status returned on the calling thread. */
+const char* coli_last_error(void);
+
+/* Test hook: the per-32-block int32 partial sums of one expert matrix
+ * (which: 0 gate, 1 up, 2 down) against n_tok Q8 vectors, computed by the
+ * same device routine as the expert kernels:
+ * isum_out[t, r, b] = sum_{j<32} q_w[r, 32b+j] * xq[t, 32b+j],
+ * isum_out is [n_tok x rows x dim_in/32] int32. */
+coli_status coli_debug_block_partials(const coli_expert* expert, int32_t which, const int8_t* xq,
+                                      int64_t n_tok, int64_t dim_in, int64_t rows, int32_t* isum_out,
+                                      void* stream);
+
+/* Profiling hook: arms three cudaEvent_t handles (any may be NULL) that the
+ * NEXT coli_moe_layer_forward call made on this thread records on its
+ * stream: `before_experts` just before the gate/up kernel, `after_gateup`
+ * between the gate/up and the down kernels, `after_down` after the down
+ * kernel.  The events must be created by the caller (with timing enabled);
+ * the call consumes the arming.  Always returns COLI_OK. */
+coli_status coli_debug_phase_events(void* before_experts, void* after_gateup, void* after_down);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COLI_H */

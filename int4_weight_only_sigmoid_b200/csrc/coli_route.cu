@@ -1,0 +1,262 @@
+// coli_route.cu -- router scores, top-k selection and bucketing.
+//
+// Router: "GLM-5.2-colibri-int4架构解析…" (wmrh.cn), sections "MoE的工作原理"
+// (router scores pick 8 experts; weighted sum), "路由策略定制"
+// (routed_scaling_factor, norm_topk_prob), "量化保留模块" (router kept F32);
+// "Colibri：在笔记本上跑744B参数的AI模型", "关键特性" (DeepSeek-V3 style
+// sigmoid router).  Bucketing: "如何在普通电脑上运行 7440 亿参数神经网络",
+// "引擎是如何工作的" (requests for one expert merged) and the HN summary,
+// "已实现的功能" (batched MoE: an expert used by several positions is read
+// once).
+#include <climits>
+
+#include "coli_launch.h"
+
+namespace coli {
+namespace {
+
+// One warp per (token, expert): lane l owns accumulator l of contract R and
+// reads float4 number l + 32j of the row, so each warp load is coalesced.
+__global__ void __launch_bounds__(256) router_scores_kernel(const float* __restrict__ x,
+                                                            const float* __restrict__ wr, int n_tok, int E,
+                                                            int H, float* __restrict__ scores) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (gw >= (int64_t)n_tok * E) return;
+  const int t = (int)(gw / E), e = (int)(gw % E);
+  const float4* xp = reinterpret_cast<const float4*>(x + (int64_t)t * H);
+  const float4* wp = reinterpret_cast<const float4*>(wr + (int64_t)e * H);
+  float acc = 0.0f;
+  for (int j = lane; j < H / 4; j += 32) {
+    const float4 a = xp[j];
+    const float4 b = __ldg(wp + j);
+    acc = __fmaf_rn(a.x, b.x, acc);
+    acc = __fmaf_rn(a.y, b.y, acc);
+    acc = __fmaf_rn(a.z, b.z, acc);
+    acc = __fmaf_rn(a.w, b.w, acc);
+  }
+  const float logit = warp_sum_in_lane_order(acc);
+  if (lane == 0) scores[gw] = sigmoid_cw(logit);
+}
+
+// One warp per token: K rounds of a warp-wide argmax over scores + bias
+// (ties to the lower expert index), then the weights.
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ scores,
+                                                   const float* __restrict__ bias, int n_tok, int E, int K,
+                                                   int norm, float rsf, int32_t* __restrict__ idx,
+                                                   float* __restrict__ wout) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= n_tok) return;
+  const float* st = scores + (int64_t)t * E;
+  float v[kMaxExperts / 32];
+#pragma unroll
+  for (int i = 0; i < kMaxExperts / 32; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? __fadd_rn(st[e], bias[e]) : 0.0f;
+  }
+  uint32_t taken = 0;
+  int sel[kMaxTopK];
+#pragma unroll
+  for (int k = 0; k < kMaxTopK; ++k) {
+    if (k >= K) break;
+    float bv = 0.0f;
+    int be = INT_MAX;
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u)) {
+        if (be == INT_MAX || v[i] > bv) {  // ascending e: strict '>' keeps the lower index
+          bv = v[i];
+          be = e;
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be))) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    sel[k] = be;
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+  }
+  if (lane == 0) {
+    float sk[kMaxTopK];
+    float denom = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kMaxTopK; ++k) {
+      if (k >= K) break;
+      sk[k] = st[sel[k]];
+      denom = (k == 0) ? sk[k] : __fadd_rn(denom, sk[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxTopK; ++k) {
+      if (k >= K) break;
+      idx[(int64_t)t * K + k] = sel[k];
+      wout[(int64_t)t * K + k] = norm ? __fmul_rn(__fdiv_rn(sk[k], denom), rsf) : __fmul_rn(sk[k], rsf);
+    }
+  }
+}
+
+constexpr int kBucketThreads = 1024;
+constexpr int kChunk = 1024;  // tokens per ranking round: one per thread
+
+// Exclusive scan of v[0..n) in place by one warp; returns the total.
+__device__ int warp_exclusive_scan(int* v, int n, int lane) {
+  const int per = (n + 31) / 32;
+  const int lo = lane * per;
+  int local = 0;
+  for (int i = lo; i < lo + per && i < n; ++i) local += v[i];
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int run = incl - local;
+  for (int i = lo; i < lo + per && i < n; ++i) {
+    const int c = v[i];
+    v[i] = run;
+    run += c;
+  }
+  return __shfl_sync(0xffffffffu, incl, 31);
+}
+
+// Single block.  Counts by shared-memory atomics (order-free), offsets by a
+// scan, then a stable scatter: tokens are ranked within each expert through
+// a per-chunk bitmap [E x 32 words] and popcounts, so every output position
+// is a pure function of the input (deterministic, no ordering races).
+__global__ void __launch_bounds__(kBucketThreads) bucket_kernel(const int32_t* __restrict__ idx, int n_tok, int K,
+                                                                int E, int n_shared, int32_t* __restrict__ counts,
+                                                                int32_t* __restrict__ offsets,
+                                                                int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                                Slot* __restrict__ slots,
+                                                                int32_t* __restrict__ n_slots,
+                                                                int32_t* __restrict__ status) {
+  extern __shared__ int sm[];
+  int* cnt = sm;             // [E]
+  int* off = cnt + E;        // [E]
+  int* run = off + E;        // [E]
+  int* tot = run + E;        // [E]
+  int* act = tot + E;        // [E] active-slot index
+  uint32_t* bm = reinterpret_cast<uint32_t*>(act + E);  // [E][32]
+  int* pre = reinterpret_cast<int*>(bm + 32 * E);        // [E][32]
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int64_t n_pairs = (int64_t)n_tok * K;
+
+  for (int e = tid; e < E; e += blockDim.x) {
+    cnt[e] = 0;
+    run[e] = 0;
+  }
+  __syncthreads();
+  for (int64_t i = tid; i < n_pairs; i += blockDim.x) {
+    const int e = idx[i];
+    if (e >= 0 && e < E) {
+      atomicAdd(&cnt[e], 1);
+    } else if (status) {
+      atomicExch(status, 1);
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    for (int e = lane; e < E; e += 32) {
+      off[e] = cnt[e];
+      act[e] = cnt[e] > 0 ? 1 : 0;
+    }
+    __syncwarp();
+    const int total = warp_exclusive_scan(off, E, lane);
+    __syncwarp();
+    const int n_active = warp_exclusive_scan(act, E, lane);
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) {
+      counts[e] = cnt[e];
+      offsets[e] = off[e];
+      if (slots && cnt[e] > 0) slots[act[e]] = Slot{e, off[e], cnt[e], off[e]};
+    }
+    if (lane == 0) {
+      offsets[E] = total;
+      if (slots) {
+        for (int s = 0; s < n_shared; ++s)
+          slots[n_active + s] = Slot{E + s, (int)n_pairs + s * n_tok, n_tok, -1};
+        *n_slots = n_active + n_shared;
+      }
+    }
+  }
+  __syncthreads();
+
+  for (int base = 0; base < n_tok; base += kChunk) {
+    for (int i = tid; i < 32 * E; i += blockDim.x) bm[i] = 0u;
+    __syncthreads();
+    const int j = tid;
+    const int t = base + j;
+    if (j < kChunk && t < n_tok) {
+      for (int k = 0; k < K; ++k) {
+        const int e = idx[(int64_t)t * K + k];
+        if (e >= 0 && e < E) atomicOr(&bm[e * 32 + (j >> 5)], 1u << (j & 31));
+      }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) {
+      int r = 0;
+      for (int wd = 0; wd < 32; ++wd) {
+        pre[e * 32 + wd] = r;
+        r += __popc(bm[e * 32 + wd]);
+      }
+      tot[e] = r;
+    }
+    __syncthreads();
+    if (j < kChunk && t < n_tok) {
+      for (int k = 0; k < K; ++k) {
+        const int e = idx[(int64_t)t * K + k];
+        if (e < 0 || e >= E) continue;
+        const uint32_t below = bm[e * 32 + (j >> 5)] & ((1u << (j & 31)) - 1u);
+        const int pos = off[e] + run[e] + pre[e * 32 + (j >> 5)] + __popc(below);
+        perm[pos] = t * K + k;
+        if (inv) inv[(int64_t)t * K + k] = pos;
+      }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) run[e] += tot[e];
+    __syncthreads();
+  }
+}
+
+size_t bucket_smem_bytes(int E) { return (size_t)E * (5 + 64) * sizeof(int); }
+
+}  // namespace
+
+cudaError_t launch_router_scores(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
+                                 cudaStream_t st) {
+  const int64_t warps = (int64_t)n_tok * E;
+  const int64_t blocks = (warps + 7) / 8;
+  router_scores_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, w_router, n_tok, E, H, scores);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E, int K, int norm, float rsf,
+                        int32_t* idx, float* w, cudaStream_t st) {
+  topk_kernel<<<(n_tok + 7) / 8, 256, 0, st>>>(scores, bias, n_tok, E, K, norm, rsf, idx, w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bucket(const int32_t* idx, int n_tok, int K, int E, int n_shared, int32_t* counts,
+                          int32_t* offsets, int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots,
+                          int32_t* status, cudaStream_t st) {
+  const size_t smem = bucket_smem_bytes(E);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)bucket_smem_bytes(kMaxExperts));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  bucket_kernel<<<1, kBucketThreads, smem, st>>>(idx, n_tok, K, E, n_shared, counts, offsets, perm, inv, slots,
+                                                  n_slots, status);
+  return cudaGetLastError();
+}
+
+}  // namespace coli

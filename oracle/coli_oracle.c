@@ -451,14 +451,15 @@ ORA_API int ora_moe_layer(const ora_layer* L, const float* x, int64_t n_tok, flo
 /* Between layers of a stack: RMSNorm and the residual                       */
 /* ------------------------------------------------------------------------ */
 
-/* RMSNorm with weight 1: ss = sum x^2 (fmaf, ascending h); mean = ss / H;
- * r = 1 / sqrtf(mean + eps); y = x * r.  (A pre-norm reading of "RMSNorm
- * and a residual between layers"; the pages do not describe the norm.) */
+/* RMSNorm with weight 1: ss = sum of x[h]^2 under contract R (the same
+ * 32-accumulator order as the router logit, so a parallel implementation can
+ * reproduce it); mean = ss / H; r = 1 / sqrtf(mean + eps); y = x * r.
+ * (A pre-norm reading of "RMSNorm and a residual between layers"; the pages
+ * do not describe the norm.)  H must be a multiple of 128. */
 ORA_API void ora_rmsnorm(const float* x, int64_t n_tok, int64_t H, float eps, float* y) {
     for (int64_t t = 0; t < n_tok; ++t) {
         const float* xt = x + t * H;
-        float ss = 0.0f;
-        for (int64_t h = 0; h < H; ++h) ss = fmaf(xt[h], xt[h], ss);
+        float ss = ora_router_logit(xt, xt, H);
         float mean = ss / (float)H;
         float r = 1.0f / sqrtf(mean + eps);
         for (int64_t h = 0; h < H; ++h) y[t * H + h] = xt[h] * r;

@@ -1,0 +1,84 @@
+"""The C ABI without a GPU: libcoli.so loads, exports every function that
+include/coli.h declares, and rejects bad arguments on the host (these paths
+return before any CUDA call)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "coli.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(coli_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import int4_weight_only_sigmoid_b200 as m
+    from int4_weight_only_sigmoid_b200 import build
+    build.build()
+    return m.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    import int4_weight_only_sigmoid_b200 as m
+    names = _declared()
+    assert len(names) >= 11
+    assert sorted(m.EXPORTS) == names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_workspace_bytes_host_only(lib):
+    import int4_weight_only_sigmoid_b200 as m
+    cfg = m.make_config(6144, 2048, 256, 8, 1)
+    b1 = m.workspace_bytes(cfg, 1)
+    b2048 = m.workspace_bytes(cfg, 2048)
+    assert 0 < b1 < b2048
+    # y buffer dominates at 2048 tokens: (8 + 1) * 2048 rows of 6144 floats
+    assert b2048 >= 9 * 2048 * 6144 * 4
+    bad = m.make_config(100, 2048, 256, 8, 1)
+    assert m.workspace_bytes(bad, 1) == 0
+    bad = m.make_config(6144, 2048, 256, 17, 1)
+    assert m.workspace_bytes(bad, 1) == 0
+
+
+def test_bad_arguments_rejected_before_any_cuda_call(lib):
+    import int4_weight_only_sigmoid_b200 as m
+    assert lib.coli_quantize_act_q8(None, 1, 64, None, None, None) == m.COLI_EINVAL
+    assert b"null pointer" in lib.coli_last_error()
+    assert lib.coli_quantize_act_q8(C.c_void_p(16), 1, 40, C.c_void_p(16), C.c_void_p(16), None) == m.COLI_EINVAL
+    assert b"multiple of 32" in lib.coli_last_error()
+    assert lib.coli_quantize_rows_int4(C.c_void_p(8), 2, 64, C.c_void_p(16), C.c_void_p(16), None) == m.COLI_EINVAL
+    assert b"aligned" in lib.coli_last_error()
+    assert lib.coli_quantize_rows_int4(None, 0, 64, None, None, None) == m.COLI_OK  # nothing to do
+    cfg = m.make_config(6144, 2048, 256, 8, 1)
+    e = m.Expert()
+    assert lib.coli_moe_expert_ffn(C.byref(cfg), C.byref(e), None, None, 1, None, None, 0, None) == m.COLI_EINVAL
+    L = m.MoeLayerC(cfg, None, None, None, None)
+    assert lib.coli_moe_layer_forward(C.byref(L), None, 1, None, None, 0, None) == m.COLI_EINVAL
+    assert lib.coli_moe_route(None, None, 1, None, None, None, None) == m.COLI_EINVAL
+    assert lib.coli_moe_bucket(None, 1, 8, 1000, None, None, None, None) == m.COLI_EINVAL
+    assert lib.coli_rmsnorm(None, 1, 100, 1e-5, None, None) == m.COLI_EINVAL
+    assert lib.coli_debug_block_partials(None, 0, None, 1, 64, 1, None, None) == m.COLI_EINVAL
+    assert lib.coli_moe_stack_forward(None, 0, None, 1, 1e-5, None, None, 0, None) == m.COLI_EINVAL
+
+
+def test_zero_tokens_is_ok_without_touching_pointers(lib):
+    import int4_weight_only_sigmoid_b200 as m
+    assert lib.coli_quantize_act_q8(None, 0, 64, None, None, None) == m.COLI_OK
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    import int4_weight_only_sigmoid_b200 as m
+    saved = m._lib
+    try:
+        m._lib = None
+        with pytest.raises(ImportError):
+            m.load(str(tmp_path / "nope.so"))
+    finally:
+        m._lib = saved

@@ -1,0 +1,154 @@
+"""GPU parity of the whole MoE layer (coli_moe_layer_forward) and of the
+pre-norm stack against the oracle.
+
+The bar: selected experts identical, and max |out - oracle| <= 2e-3 *
+RMS(oracle out).  The kernels follow the oracle's evaluation contracts, so
+the output is also checked bit for bit (a separate assertion, so that a
+tolerance-only regression is reported as such).  Large batches are checked
+on a seeded sample of tokens: tokens are independent in a MoE layer, so the
+oracle's rows for the sample are exactly the full batch's rows."""
+import numpy as np
+import pytest
+
+from tests.helpers import assert_layer_close, bits_equal, oracle_layer_forward
+
+pytestmark = pytest.mark.gpu
+
+_layers = {}
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _dev_layer(cfg, layer=0):
+    from synth.layers import device_layer
+    key = (cfg["name"], cfg["hidden"], cfg["n_experts"], cfg["top_k"], cfg["n_shared"], layer,
+           cfg["norm_topk_prob"], cfg["routed_scaling_factor"], cfg.get("bias_boost_n", 0))
+    if key not in _layers:
+        if len(_layers) > 3:
+            _layers.clear()
+        _layers[key] = device_layer(cfg, layer)
+    return _layers[key]
+
+
+def _check_layer(coli, syn, cfg, n_tok, sample=None, exact=True):
+    import torch
+    L = _dev_layer(cfg)
+    x = syn.tokens(cfg, n_tok)
+    out = _np(coli.moe_layer_forward(L, torch.from_numpy(x).cuda()))
+    sub = np.arange(n_tok) if sample is None else np.sort(np.random.default_rng(1).choice(n_tok, sample, replace=False))
+    want, idx, w, _ = oracle_layer_forward(cfg, x[sub])
+    _, gidx, gw = coli.moe_route(L, torch.from_numpy(x[sub]).cuda())
+    assert np.array_equal(_np(gidx), idx)
+    assert_layer_close(out[sub], want)
+    if exact:
+        assert bits_equal(out[sub], want)
+    return out
+
+
+@pytest.mark.parametrize("n_tok", [8, 1, 2, 3, 5, 13])
+def test_layer_tiny(coli, syn, n_tok):
+    _check_layer(coli, syn, syn.config("tiny"), n_tok)
+
+
+@pytest.mark.parametrize("over", [dict(norm_topk_prob=False), dict(routed_scaling_factor=1.0),
+                                  dict(top_k=1), dict(top_k=16), dict(n_shared=0), dict(n_shared=2)])
+def test_layer_tiny_variants(coli, syn, over):
+    _check_layer(coli, syn, syn.config("tiny", **over), 8)
+
+
+def test_layer_decode1(coli, syn):
+    _check_layer(coli, syn, syn.config("decode1"), 1)
+
+
+def test_layer_decode4(coli, syn):
+    _check_layer(coli, syn, syn.config("decode4"), 4)
+
+
+def test_layer_decode16(coli, syn):
+    _check_layer(coli, syn, syn.config("decode16"), 16, sample=6)
+
+
+def test_layer_prefill2048_sampled(coli, syn):
+    _check_layer(coli, syn, syn.config("prefill2048"), 2048, sample=4)
+
+
+def test_layer_zero_tokens_is_noop(coli, syn):
+    import torch
+    L = _dev_layer(syn.config("tiny"))
+    x = torch.empty(0, 256, device="cuda")
+    out = coli.moe_layer_forward(L, x)
+    assert out.shape == (0, 256)
+
+
+def test_layer_token_subset_consistency(coli, syn):
+    """Rows of a batch equal the same tokens run alone (batched MoE only
+    changes how often weights are read, never the result)."""
+    import torch
+    cfg = syn.config("tiny")
+    L = _dev_layer(cfg)
+    x = torch.from_numpy(syn.tokens(cfg, 13)).cuda()
+    full = _np(coli.moe_layer_forward(L, x))
+    for t in (0, 6, 12):
+        one = _np(coli.moe_layer_forward(L, x[t:t + 1].contiguous()))
+        assert bits_equal(one[0], full[t])
+
+
+def test_layer_guard_bytes_untouched(coli, syn):
+    """Canary words after the output and around the workspace stay intact."""
+    import torch
+    cfg = syn.config("tiny")
+    L = _dev_layer(cfg)
+    T, H = 5, cfg["hidden"]
+    x = torch.from_numpy(syn.tokens(cfg, T)).cuda()
+    buf = torch.full((T * H + 64,), 12345.0, device="cuda")
+    out = buf[:T * H].view(T, H)
+    nws = coli.workspace_bytes(L.cfg, T)
+    wbuf = torch.full((nws + 4096,), 0x5A, dtype=torch.uint8, device="cuda")
+    coli.moe_layer_forward(L, x, out=out, workspace=wbuf[:nws])
+    torch.cuda.synchronize()
+    assert torch.all(buf[T * H:] == 12345.0)
+    assert torch.all(wbuf[nws:] == 0x5A)
+
+
+def test_stack8_teacher_forced_and_free(coli, ora, syn):
+    """Each layer of the 8-layer stack (GPU) on the oracle's input for that
+    layer: bit-exact indices and output.  Then the free-running stack."""
+    import torch
+    from synth.layers import device_layer
+    cfg = syn.config("stack8")
+    layers = [device_layer(cfg, l) for l in range(8)]
+    x = syn.tokens(cfg, 1)
+    xo = x.copy()
+    for l in range(8):
+        xn = ora.rmsnorm(xo, cfg["rms_eps"])
+        gxn = _np(coli.rmsnorm(torch.from_numpy(xo).cuda(), cfg["rms_eps"]))
+        assert bits_equal(gxn, xn)
+        m, idx, _, _ = oracle_layer_forward(cfg, xn, l)
+        gm = _np(coli.moe_layer_forward(layers[l], torch.from_numpy(xn).cuda()))
+        assert_layer_close(gm, m)
+        assert bits_equal(gm, m)
+        xo = ora.residual_add(xo, m)
+    free = _np(coli.moe_stack_forward(layers, torch.from_numpy(x).cuda(), cfg["rms_eps"]))
+    assert_layer_close(free, xo)
+    assert bits_equal(free, xo)
+    del layers
+    torch.cuda.empty_cache()
+
+
+def test_invalid_arguments_return_einval(coli, syn):
+    import torch
+    cfg = syn.config("tiny")
+    L = _dev_layer(cfg)
+    x = torch.from_numpy(syn.tokens(cfg, 2)).cuda()
+    ws = coli.make_workspace(L.cfg, 2)
+    with pytest.raises(coli.ColiError) as ei:
+        coli.moe_layer_forward(L, x, workspace=ws[:100])
+    assert ei.value.status == coli.COLI_ENOMEM
+    with pytest.raises(coli.ColiError) as ei:
+        coli.moe_layer_forward(L, x, out=x)
+    assert ei.value.status == coli.COLI_EINVAL
+    with pytest.raises(coli.ColiError) as ei:
+        coli.quantize_act_q8(x[:, :40].contiguous())
+    assert ei.value.status == coli.COLI_EINVAL
