@@ -205,6 +205,36 @@ def run_reference(args):
 # the GPU arm
 
 
+class RawEvents:
+    """cudaEvent_t handles from the CUDA runtime that torch already loaded;
+    used for events that the library records (torch's Event objects only
+    report times for events recorded through torch)."""
+
+    def __init__(self):
+        import ctypes as C
+        self.C = C
+        self.rt = C.CDLL("libcudart.so.12")
+        self.rt.cudaEventCreate.argtypes = [C.POINTER(C.c_void_p)]
+        self.rt.cudaEventElapsedTime.argtypes = [C.POINTER(C.c_float), C.c_void_p, C.c_void_p]
+        self.rt.cudaEventSynchronize.argtypes = [C.c_void_p]
+        self.rt.cudaEventDestroy.argtypes = [C.c_void_p]
+
+    def create(self) -> int:
+        h = self.C.c_void_p()
+        rc = self.rt.cudaEventCreate(self.C.byref(h))
+        if rc != 0:
+            raise RuntimeError(f"cudaEventCreate failed ({rc})")
+        return h.value
+
+    def sync(self, e: int):
+        self.rt.cudaEventSynchronize(self.C.c_void_p(e))
+
+    def elapsed_ms(self, a: int, b: int) -> float:
+        ms = self.C.c_float()
+        rc = self.rt.cudaEventElapsedTime(self.C.byref(ms), self.C.c_void_p(a), self.C.c_void_p(b))
+        return ms.value if rc == 0 else -1.0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -263,6 +293,7 @@ def main():
             step(i, s)
     torch.cuda.synchronize()
 
+    raw = RawEvents()
     # graphs: a ring of NG graphs of G steps, each with its own phase events
     K = args.steps
     G = min(GRAPH_STEPS, K)
@@ -271,7 +302,7 @@ def main():
 
     def capture(n_steps, base):
         g = torch.cuda.CUDAGraph()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_steps)]
+        evs = [[raw.create() for _ in range(3)] for _ in range(n_steps)]
         with torch.cuda.graph(g, stream=s):
             for j in range(n_steps):
                 step(base + j, torch.cuda.current_stream(), evs[j])
@@ -292,8 +323,8 @@ def main():
         nonlocal gate_ms, down_ms, gate_bytes, phase_n
         g, evs = r
         for j, (e0, e1, e2) in enumerate(evs):
-            e2.synchronize()
-            a, b = e0.elapsed_time(e1), e1.elapsed_time(e2)
+            raw.sync(e2)
+            a, b = raw.elapsed_ms(e0, e1), raw.elapsed_ms(e1, e2)
             if a <= 0 or b <= 0:
                 continue
             gate_ms += a

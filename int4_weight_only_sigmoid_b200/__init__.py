@@ -267,5 +267,5 @@ def debug_block_partials(expert: QExpert, which: int, xq, rows: int, stream=None
 def arm_phase_events(before_experts=None, after_gateup=None, after_down=None):
     """Arm torch.cuda.Event objects that the next layer forward on this
     thread records around its expert kernels (profiling hook)."""
-    h = lambda e: None if e is None else C.c_void_p(e.cuda_event)
+    h = lambda e: None if e is None else C.c_void_p(e if isinstance(e, int) else e.cuda_event)
     _check(lib().coli_debug_phase_events(h(before_experts), h(after_gateup), h(after_down)))

@@ -145,7 +145,7 @@ def test_route_ties_and_k_equals_e(coli, ora):
 def test_bucket_bit_exact(coli, ora, T, K, E):
     import torch
     rng = np.random.default_rng(T + K + E)
-    idx = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int32).reshape(T, K)
+    idx = np.array([rng.permutation(E)[:K] for _ in range(T)], dtype=np.int32).reshape(T, K)
     if T > 100:  # skew like the prefill workload
         idx[: T // 2, :4] = np.stack([rng.permutation(32)[:4] for _ in range(T // 2)])
         for t in range(T // 2):
