@@ -168,6 +168,28 @@ coli_status coli_debug_block_partials(const coli_expert* expert, int32_t which, 
                                       int64_t n_tok, int64_t dim_in, int64_t rows, int32_t* isum_out,
                                       void* stream);
 
+/* The layer forward for callers that cannot allocate device memory: hosts
+ * that own every device allocation and give a plugin no allocator to fill
+ * `workspace` from, and serving loops that must not call cudaMalloc after
+ * start-up because it can synchronise the device and stall all streams.
+ * (This entry point has no counterpart on the pages: the engine they
+ * describe runs on CPU memory.)
+ * Same arguments and results as coli_moe_layer_forward minus the workspace:
+ * the scratch is a fixed 8 MiB array inside the library, which every GPU
+ * that loads the library holds until the process exits.  A call whose
+ * scratch need (coli_moe_workspace_bytes(&layer->cfg, n_tok)) exceeds 8 MiB
+ * is rejected with COLI_EINVAL and a message naming both sizes -- e.g. the
+ * GLM-5.2 shape (hidden 6144, inter 2048, 256 experts, top-8, 1 shared)
+ * fits up to 25 tokens per call.  The first call on each device
+ * looks up the array's device address with that device current; make that
+ * first call before any stream capture.  Every call shares the one array,
+ * so calls that can overlap on the GPU (different streams, or different
+ * host threads on one device) race: order them on one stream.  The array
+ * keeps the last call's contents; nothing in it needs to start at zero.
+ * Allocates nothing (no cudaMalloc, no cudaFree). */
+coli_status coli_moe_layer_forward_noalloc(const coli_moe_layer* layer, const float* x, int64_t n_tok,
+                                           float* out, void* stream);
+
 /* Profiling hook: arms three cudaEvent_t handles (any may be NULL) that the
  * NEXT coli_moe_layer_forward call made on this thread records on its
  * stream: `before_experts` just before the gate/up kernel, `after_gateup`

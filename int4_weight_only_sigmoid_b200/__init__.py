@@ -24,7 +24,7 @@ EXPORTS = [
     "coli_quantize_rows_int4", "coli_quantize_act_q8", "coli_moe_route", "coli_moe_bucket",
     "coli_moe_expert_ffn", "coli_moe_layer_forward", "coli_moe_stack_forward", "coli_rmsnorm",
     "coli_moe_workspace_bytes", "coli_last_error", "coli_debug_block_partials",
-    "coli_debug_phase_events",
+    "coli_debug_phase_events", "coli_moe_layer_forward_noalloc",
 ]
 
 
@@ -79,6 +79,7 @@ def load(path: str | None = None):
         "coli_last_error": (C.c_char_p, []),
         "coli_debug_block_partials": (st, [C.POINTER(Expert), i32, vp, i64, i64, i64, vp, vp]),
         "coli_debug_phase_events": (st, [vp, vp, vp]),
+        "coli_moe_layer_forward_noalloc": (st, [C.POINTER(MoeLayerC), vp, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -269,3 +270,13 @@ def arm_phase_events(before_experts=None, after_gateup=None, after_down=None):
     thread records around its expert kernels (profiling hook)."""
     h = lambda e: None if e is None else C.c_void_p(e if isinstance(e, int) else e.cuda_event)
     _check(lib().coli_debug_phase_events(h(before_experts), h(after_gateup), h(after_down)))
+
+
+def moe_layer_forward_noalloc(layer: MoeLayer, x, out=None, stream=None, cstruct=None):
+    """Layer forward with the library's fixed internal scratch (no workspace,
+    no device allocation by the library); see coli_moe_layer_forward_noalloc."""
+    import torch
+    o = torch.empty_like(x) if out is None else out
+    Lc = layer.cstruct() if cstruct is None else cstruct
+    _check(lib().coli_moe_layer_forward_noalloc(C.byref(Lc), _ptr(x), x.shape[0], _ptr(o), _stream(stream)))
+    return o

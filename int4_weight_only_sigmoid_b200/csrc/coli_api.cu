@@ -194,6 +194,9 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
 }
 
 }  // namespace
+
+void set_error_message(const char* msg) { g_last_error = msg; }
+
 }  // namespace coli
 
 using namespace coli;

@@ -53,4 +53,7 @@ cudaError_t launch_residual_add(const float* x, const float* m, int64_t n, float
 cudaError_t launch_debug_partials(const uint8_t* wq, const int8_t* xq, int n_tok, int dim_in, int rows,
                                   int32_t* out, cudaStream_t st);
 
+// Sets the message coli_last_error() returns on the calling thread.
+void set_error_message(const char* msg);
+
 }  // namespace coli
