@@ -39,6 +39,7 @@ WORKLOAD = ("GLM-5.2-shaped MoE layer decode, 1 token (hidden 6144, expert inter
 N_LAYERS = 8
 N_TOK_POOL = 64
 GRAPH_STEPS = 64
+KERNELS_PER_STEP = 4  # decode path: router, top-k+bucket, gate/up, down+combine
 
 
 def parse():
@@ -49,17 +50,52 @@ def parse():
     p.add_argument("--impl", default="coli", choices=["coli", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=4)
+    p.add_argument("--layers", type=int, default=N_LAYERS,
+                   help="resident layers cycled by the steps (8 = 39 GB; fewer for profiling captures)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-suite", action="store_true", help="skip the other workloads (decode-4/16, prefill, stack)")
     return p.parse_args()
 
 
-def peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def _load_peaks():
     try:
-        with open(path) as f:
-            d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
     except Exception:
-        return 6650.0, "fallback"
+        return {}
+
+
+MEASURED = _load_peaks()
+
+
+def peaks():
+    if "hbm_gbs" in MEASURED:
+        return float(MEASURED["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# data-parallel plumbing (replicas: no collective on the data path)
+
+
+def rank_token_shard(n_total: int, rank: int, world: int):
+    """Token ids a rank processes when a batch is split across replicas:
+    a contiguous block, earlier ranks taking the remainder."""
+    base, extra = divmod(n_total, world)
+    lo = rank * base + min(rank, extra)
+    return range(lo, lo + base + (1 if rank < extra else 0))
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank number (a device-timed duration) over all ranks;
+    the identity without an initialised process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 # ---------------------------------------------------------------------------
@@ -202,6 +238,101 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# the other workloads (reported beside the metric, not as the metric)
+
+
+def run_suite(layers, cfg, dev, stream, peak_gbs):
+    """decode-4 / decode-16 / prefill-2048 / 8-layer stack (1 and 512 tokens)
+    on the resident layers.  Each entry: per-layer tokens/s, ms per step,
+    unique experts streamed per layer and the weight bytes that implies per
+    second; prefill adds int8-equivalent tensor throughput (2 x MACs / s)."""
+    import torch
+
+    import int4_weight_only_sigmoid_b200 as coli
+    import synth
+
+    H, I, E, K, S = cfg["hidden"], cfg["inter"], cfg["n_experts"], cfg["top_k"], cfg["n_shared"]
+    nl = len(layers)
+    expert_bytes = 3 * (I * H // 2) + (2 * I + H) * 4
+    router_bytes = E * H * 4
+    out = {}
+
+    def uniq(layer, x):
+        _, idx, _ = coli.moe_route(layer, x)
+        return len(torch.unique(idx)) + S
+
+    def time_steps(fn, n_steps, graph):
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for j in range(n_steps):
+                    fn(j, torch.cuda.current_stream())
+            g.replay()
+            torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            if graph:
+                g.replay()
+            else:
+                for j in range(n_steps):
+                    fn(j, stream)
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / n_steps
+
+    for name, T, steps, graph in [("decode4", 4, 256, True), ("decode16", 16, 256, True),
+                                  ("prefill2048", 2048, 16, False)]:
+        c = synth.config(name, seed=cfg["seed"])
+        x = synth.dev_tokens(c, T, device=dev)
+        lys = layers
+        if c.get("bias_boost_n", 0):
+            lys = [coli.MoeLayer(l.cfg, l.w_router, synth.dev_bias(c, li, device=dev), l.experts, l.shared)
+                   for li, l in enumerate(layers)]
+        cs = [l.cstruct() for l in lys]
+        ws = coli.make_workspace(lys[0].cfg, T, dev)
+        o = torch.empty(T, H, dtype=torch.float32, device=dev)
+        with torch.cuda.stream(stream):
+            for j in range(3):
+                coli.moe_layer_forward(lys[j % nl], x, out=o, workspace=ws, stream=stream, cstruct=cs[j % nl])
+        torch.cuda.synchronize()
+        n_exp = [uniq(l, x) for l in lys]
+        fn = lambda j, st: coli.moe_layer_forward(lys[j % nl], x, out=o, workspace=ws, stream=st, cstruct=cs[j % nl])
+        ms = time_steps(fn, steps, graph)
+        ue = sum(n_exp) / len(n_exp)
+        rec = {"tokens": T, "ms_per_layer": ms, "tokens_per_s_per_layer": T / (ms * 1e-3),
+               "unique_experts_streamed": ue,
+               "weight_gbs": (ue * expert_bytes + router_bytes) / (ms * 1e-3) / 1e9}
+        rec["weight_frac_of_hbm"] = rec["weight_gbs"] / peak_gbs
+        if name == "prefill2048":
+            macs = T * (K + S) * 3 * I * H
+            rec["int8_equiv_tops"] = 2 * macs / (ms * 1e-3) / 1e12
+            rec["tensor_note"] = ("operands expanded to exact fp16 (kind::f16, F32 accumulate); fraction vs the "
+                                  "measured bf16/fp16 dense peak")
+            rec["frac_of_fp16_peak"] = rec["int8_equiv_tops"] / float(MEASURED.get("bf16_tflops", 1674.6))
+            rec["routed_tokens_per_expert_max"] = None
+        out[name] = rec
+        del ws
+
+    # the 8-layer pre-norm stack (RMSNorm + residual between layers)
+    for name, T, steps, graph in [("stack8_decode1", 1, 64, True), ("stack8_prefill512", 512, 4, False)]:
+        c = synth.config("stack8_512" if T > 1 else "stack8", seed=cfg["seed"])
+        x = synth.dev_tokens(c, T, device=dev)
+        arr = coli.stack_cstructs(layers)
+        ws = coli.make_workspace(layers[0].cfg, T, dev)
+        o = torch.empty(T, H, dtype=torch.float32, device=dev)
+        with torch.cuda.stream(stream):
+            coli.moe_stack_forward(layers, x, 1e-5, out=o, workspace=ws, stream=stream, carr=arr)
+        torch.cuda.synchronize()
+        fn = lambda j, st: coli.moe_stack_forward(layers, x, 1e-5, out=o, workspace=ws, stream=st, carr=arr)
+        ms = time_steps(fn, steps, graph)
+        out[name] = {"tokens": T, "layers": nl, "ms_per_stack": ms, "ms_per_layer": ms / nl,
+                     "tokens_per_s_per_layer": T * nl / (ms * 1e-3)}
+        del ws
+    return out
+
+
+# ---------------------------------------------------------------------------
 # the GPU arm
 
 
@@ -261,7 +392,8 @@ def main():
     cfg = synth.config("decode1", seed=rank)  # each rank: its own replica, its own tokens
     H = cfg["hidden"]
     staging = torch.empty(cfg["inter"] * H, dtype=torch.float32, device=dev)
-    layers = [device_layer(cfg, l, device=dev, staging=staging) for l in range(N_LAYERS)]
+    n_layers = args.layers
+    layers = [device_layer(cfg, l, device=dev, staging=staging) for l in range(n_layers)]
     del staging
     cstructs = [L.cstruct() for L in layers]
     xs = synth.dev_tokens(cfg, N_TOK_POOL, device=dev)
@@ -276,15 +408,15 @@ def main():
     router_bytes = cfg["n_experts"] * H * 4 + cfg["n_experts"] * 4
     uniq = []
     for i in range(N_TOK_POOL):
-        _, idx, _ = coli.moe_route(layers[i % N_LAYERS], xs[i:i + 1])
+        _, idx, _ = coli.moe_route(layers[i % n_layers], xs[i:i + 1])
         uniq.append(len(torch.unique(idx)))
     n_exp = [u + cfg["n_shared"] for u in uniq]
 
     def step(i, stream, evs=None):
         if evs is not None:
             coli.arm_phase_events(*evs)
-        coli.moe_layer_forward(layers[i % N_LAYERS], xs[i % N_TOK_POOL:i % N_TOK_POOL + 1], out=outs[i % 2],
-                               workspace=ws, stream=stream, cstruct=cstructs[i % N_LAYERS])
+        coli.moe_layer_forward(layers[i % n_layers], xs[i % N_TOK_POOL:i % N_TOK_POOL + 1], out=outs[i % 2],
+                               workspace=ws, stream=stream, cstruct=cstructs[i % n_layers])
 
     # warm-up (also sets kernel attributes before any capture)
     s = torch.cuda.Stream(device=dev)
@@ -294,29 +426,66 @@ def main():
     torch.cuda.synchronize()
 
     raw = RawEvents()
-    # graphs: a ring of NG graphs of G steps, each with its own phase events
     K = args.steps
     G = min(GRAPH_STEPS, K)
     n_full, rem = divmod(K, G)
     NG = 3
 
-    def capture(n_steps, base):
+    def capture(n_steps, base, with_events):
         g = torch.cuda.CUDAGraph()
-        evs = [[raw.create() for _ in range(3)] for _ in range(n_steps)]
+        evs = [[raw.create() for _ in range(3)] for _ in range(n_steps)] if with_events else None
         with torch.cuda.graph(g, stream=s):
             for j in range(n_steps):
-                step(base + j, torch.cuda.current_stream(), evs[j])
+                step(base + j, torch.cuda.current_stream(), evs[j] if with_events else None)
         return g, evs
 
-    ring = [capture(G, r * G) for r in range(NG)]
-    tail = capture(rem, 0) if rem else None
-    # each graph replay starts its steps at a fixed token/layer offset; the ring
-    # rotates over NG*G distinct (layer, token) steps
-    torch.cuda.synchronize()
+    def timed(ring, tail, on_done=None):
+        """Replay the ring of graphs for K steps; returns elapsed ms (events on
+        the replay stream).  on_done(r, base) harvests a finished graph."""
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        pending = []
+        with torch.cuda.stream(s):
+            start.record(s)
+            for k in range(n_full):
+                r = ring[k % NG]
+                if on_done is not None and len(pending) == NG:
+                    on_done(*pending.pop(0))
+                r[0].replay()
+                pending.append((r, (k % NG) * G))
+            if tail is not None:
+                tail[0].replay()
+            end.record(s)
+        end.synchronize()
+        if on_done is not None:
+            while pending:
+                on_done(*pending.pop(0))
+            if tail is not None:
+                on_done(tail, 0)
+        return start.elapsed_time(end)
+
+    # 1) the metric: graphs of plain steps
+    ring = [capture(G, r * G, False) for r in range(NG)]
+    tail = capture(rem, 0, False) if rem else None
     for g, _ in ring:
         g.replay()
     torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clk = ClockSampler(vis.split(",")[local] if vis else local)
+    clk.start()
+    elapsed_ms = timed(ring, tail)
+    clocks = clk.stop()
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
+    ms_per_step = elapsed_ms / K
+    tokens = K * world
+    value = tokens / (elapsed_ms / 1e3)
+    del ring, tail
 
+    # 2) the dominant kernel: the same steps with events the library records
+    #    on its stream around the gate/up and down kernels
     gate_ms, down_ms, gate_bytes, phase_n = 0.0, 0.0, 0.0, 0
 
     def harvest(r, base_step):
@@ -332,40 +501,13 @@ def main():
             gate_bytes += n_exp[(base_step + j) % N_TOK_POOL] * gateup_bytes_per_expert
             phase_n += 1
 
-    if world > 1:
-        dist.barrier()
+    ring = [capture(G, r * G, True) for r in range(NG)]
+    tail = capture(rem, 0, True) if rem else None
+    for g, _ in ring:
+        g.replay()
     torch.cuda.synchronize()
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    clk = ClockSampler(vis.split(",")[local] if vis else local)
-    clk.start()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    pending = []
-    with torch.cuda.stream(s):
-        start.record(s)
-        for k in range(n_full):
-            r = ring[k % NG]
-            if len(pending) == NG:
-                harvest(*pending.pop(0))
-            r[0].replay()
-            pending.append((r, (k % NG) * G))
-        if tail is not None:
-            tail[0].replay()
-        end.record(s)
-    end.synchronize()
-    while pending:
-        harvest(*pending.pop(0))
-    if tail is not None:
-        harvest(tail, 0)
-    clocks = clk.stop()
-    elapsed_ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-    ms_per_step = elapsed_ms / K
-    tokens = K * world
-    value = tokens / (elapsed_ms / 1e3)
+    phase_elapsed_ms = timed(ring, tail, harvest)
+    del ring, tail
 
     # streamed bytes of the whole step (router + experts) over the step time
     mean_exp = sum(n_exp) / len(n_exp)
@@ -377,7 +519,7 @@ def main():
 
     # end to end through the public API: pinned host token in, host output back
     e2e = None
-    if rank == 0 or world > 1:
+    if not args.no_e2e:
         hx = torch.empty(N_TOK_POOL, 1, H, dtype=torch.float32).pin_memory()
         hx.copy_(xs.view(N_TOK_POOL, 1, H).cpu())
         hout = torch.empty(2, 1, H, dtype=torch.float32).pin_memory()
@@ -389,8 +531,8 @@ def main():
             cs = torch.cuda.current_stream()
             for j in range(Ge):
                 dx.copy_(hx[j % N_TOK_POOL], non_blocking=True)
-                coli.moe_layer_forward(layers[j % N_LAYERS], dx, out=outs[j % 2], workspace=ws, stream=cs,
-                                       cstruct=cstructs[j % N_LAYERS])
+                coli.moe_layer_forward(layers[j % n_layers], dx, out=outs[j % 2], workspace=ws, stream=cs,
+                                       cstruct=cstructs[j % n_layers])
                 hout[j % 2].copy_(outs[j % 2], non_blocking=True)
         ge.replay()
         torch.cuda.synchronize()
@@ -404,14 +546,15 @@ def main():
             e1.record(s)
         e1.synchronize()
         e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e_ms, dev)
         e2e = {"value": reps * Ge * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": H * 4,
                "d2h_bytes_per_step": H * 4, "steps": reps * Ge,
                "note": "pinned H2D of the token, coli_moe_layer_forward, D2H of the output, per step"}
         del ge
+
+    suite = None
+    if not args.no_suite:
+        suite = run_suite(layers, cfg, dev, s, peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -423,22 +566,22 @@ def main():
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int4xint8->f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "layers_resident": N_LAYERS, "tokens_per_step": 1,
+            "config": {"workload": WORKLOAD, "layers_resident": n_layers, "tokens_per_step": 1,
                        "parallelism": f"dp{world} (replicas, no collective)",
                        "l2": "inputs larger than L2: 8 resident layers cycled, ~170 MB of weights per step",
                        "graph_steps": G, "mean_experts_streamed": mean_exp},
             "streamed_gbs": step_gbs,
             "streamed_frac_of_hbm": step_gbs / peak,
-            "roofline": {"bound": "hbm", "kernel": "gateup_kernel", "achieved": gate_gbs, "peak": peak,
+            "roofline": {"bound": "hbm", "kernel": "gateup_decode_kernel", "achieved": gate_gbs, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": gate_gbs / peak, "traffic": None,
                          "avg_launch_ms": gate_avg_ms,
                          "algorithmic_bytes_per_launch": gate_bytes / max(1, phase_n),
                          "down_kernel_avg_ms": down_ms / max(1, phase_n)},
-            "e2e": e2e, "gpu_launches": K * 7, "clocks": clocks, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": K * KERNELS_PER_STEP, "clocks": clocks, "cpu_baseline": cpu,
+            "other_workloads": suite,
+            "phase_region_ms_per_step": phase_elapsed_ms / K,
         }
         print(json.dumps(line), flush=True)
-    for g, _ in ring:
-        del g
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

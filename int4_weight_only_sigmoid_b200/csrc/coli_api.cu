@@ -94,7 +94,8 @@ coli_status check_layer(const coli_moe_layer* L, const char* fn) {
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Workspace {
-  size_t xq, xd, scores, idx, w, counts, offsets, perm, inv, slots, n_slots, status, hq, hd, y, xn, xa, xb, total;
+  size_t xq, xd, scores, idx, w, counts, offsets, perm, inv, slots, n_slots, status, tiles, n_tiles, hq, hd, y, xn, xa,
+      xb, total;
 };
 
 Workspace layout(const coli_moe_config& c, int64_t T) {
@@ -119,6 +120,8 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   L.slots = take((size_t)kMaxSlots * sizeof(Slot));
   L.n_slots = take(4);
   L.status = take(4);
+  L.tiles = take(prefill_tile_bytes((int)T, (int)K, (int)E, (int)S));
+  L.n_tiles = take(4);
   L.hq = take(rows * I);
   L.hd = take(rows * (I / 32) * 4);
   L.y = take(rows * H * 4);
@@ -170,6 +173,26 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   static thread_local DownTable dn;
   fill_tables(L, gu, dn);
 
+  cudaEvent_t ev[3] = {g_phase_ev[0], g_phase_ev[1], g_phase_ev[2]};
+  g_phase_ev[0] = g_phase_ev[1] = g_phase_ev[2] = nullptr;
+  auto mark = [&](int i) -> cudaError_t {
+    return ev[i] ? cudaEventRecordWithFlags(ev[i], st, cudaEventRecordExternal) : cudaSuccess;
+  };
+
+  if (T <= kDecodeMaxTok && (size_t)H * 8 <= 200 * 1024) {
+    // decode: 4 kernels, the last three launched with PDL
+    CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, st));
+    CHECK_LAUNCH(launch_topk_bucket_small(scores, L->bias, (int)T, E, K, c.norm_topk_prob, c.routed_scaling_factor,
+                                          idx, wts, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm, inv,
+                                          slots, n_slots, st));
+    CHECK_LAUNCH(mark(0));
+    CHECK_LAUNCH(launch_gateup_decode(gu, slots, n_slots, perm, (int)T, K, E, S, x, H, I, hq, hd, st));
+    CHECK_LAUNCH(mark(1));
+    CHECK_LAUNCH(launch_down_combine(dn, slots, n_slots, (int)T, K, E, S, hq, hd, inv, wts, H, I, out, st));
+    CHECK_LAUNCH(mark(2));
+    return COLI_OK;
+  }
+
   CHECK_LAUNCH(launch_quantize_act_q8(x, T, H, xq, xd, st));
   CHECK_LAUNCH(launch_router_scores(x, L->w_router, (int)T, E, H, scores, st));
   CHECK_LAUNCH(launch_topk(scores, L->bias, (int)T, E, K, c.norm_topk_prob, c.routed_scaling_factor, idx, wts, st));
@@ -182,13 +205,18 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   sl.perm = perm;
   sl.top_k = K;
   const int max_tok = (int)T;
-  cudaEvent_t ev[3] = {g_phase_ev[0], g_phase_ev[1], g_phase_ev[2]};
-  g_phase_ev[0] = g_phase_ev[1] = g_phase_ev[2] = nullptr;
-  if (ev[0]) CHECK_LAUNCH(cudaEventRecordWithFlags(ev[0], st, cudaEventRecordExternal));
-  CHECK_LAUNCH(launch_gateup(gu, sl, xq, xd, H, I, max_tok, hq, hd, st));
-  if (ev[1]) CHECK_LAUNCH(cudaEventRecordWithFlags(ev[1], st, cudaEventRecordExternal));
-  CHECK_LAUNCH(launch_down(dn, sl, hq, hd, H, I, max_tok, y, st));
-  if (ev[2]) CHECK_LAUNCH(cudaEventRecordWithFlags(ev[2], st, cudaEventRecordExternal));
+  CHECK_LAUNCH(mark(0));
+  if (prefill_supported(H, I)) {
+    const int max_tiles = (int)prefill_tiles_bound((int)T, K, E, S);
+    CHECK_LAUNCH(launch_prefill_experts(gu, dn, slots, n_slots, at<void>(ws, W.tiles), at<int32_t>(ws, W.n_tiles),
+                                        max_tiles, perm, K, xq, xd, H, I, hq, hd, y, at<int32_t>(ws, W.status), st,
+                                        ev[1]));
+  } else {
+    CHECK_LAUNCH(launch_gateup(gu, sl, xq, xd, H, I, max_tok, hq, hd, st));
+    CHECK_LAUNCH(mark(1));
+    CHECK_LAUNCH(launch_down(dn, sl, hq, hd, H, I, max_tok, y, st));
+  }
+  CHECK_LAUNCH(mark(2));
   CHECK_LAUNCH(launch_combine(y, inv, wts, (int)T, K, S, H, out, st));
   return COLI_OK;
 }

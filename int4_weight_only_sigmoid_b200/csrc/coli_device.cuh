@@ -117,6 +117,20 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
+// 16-byte asynchronous global -> shared copy (cp.async, L2 only) and the wait
+// for all of this thread's outstanding copies.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Programmatic dependent launch: wait for the grids this one depends on (a
+// no-op when launched without the attribute), and let the next grid in the
+// stream start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Q8_0 of one value given its block scale d (d == 0 -> 0).
 __device__ __forceinline__ int q8_of(float v, float d) {
   if (d == 0.0f) return 0;

@@ -2,11 +2,36 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
+
 #include <cuda_runtime.h>
 
 #include "coli_device.cuh"
 
 namespace coli {
+
+// Largest batch that takes the decode path (router_decode, topk_bucket_small,
+// gateup_decode, down_combine).
+constexpr int kDecodeMaxTok = 16;
+
+// Launch with programmatic stream serialisation (PDL) when `pdl` is set: the
+// kernel may start while its predecessor is still running and must call
+// pdl_wait() before it reads anything the predecessor writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Quantisers
 cudaError_t launch_quantize_rows_int4(const float* w, int64_t rows, int64_t cols, uint8_t* q,
@@ -19,6 +44,14 @@ cudaError_t launch_router_scores(const float* x, const float* w_router, int n_to
                                  float* scores, cudaStream_t st);
 cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E, int K, int norm,
                         float rsf, int32_t* idx, float* w, cudaStream_t st);
+
+// Decode batches: router scores with the router rows staged in shared memory
+// (plain launch), then top-k + weights + bucketing in one CTA (PDL launch).
+cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
+                                 cudaStream_t st);
+cudaError_t launch_topk_bucket_small(const float* scores, const float* bias, int n_tok, int E, int K, int norm,
+                                     float rsf, int32_t* idx, float* w, int32_t* counts, int32_t* offsets,
+                                     int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, cudaStream_t st);
 
 // Bucketing: counts, offsets, perm; optionally the inverse map (pair ->
 // position), the expert slot table (+ shared slots) and its length.
@@ -40,6 +73,29 @@ cudaError_t launch_gateup(const GateUpTable& tbl, const GemvSlots& sl, const int
                           float* hd, cudaStream_t st);
 cudaError_t launch_down(const DownTable& tbl, const GemvSlots& sl, const int8_t* hq, const float* hd,
                         int hidden, int inter, int max_tok_per_slot, float* y, cudaStream_t st);
+
+// Decode expert kernels (PDL launches).  Slot table = the routed experts
+// only; shared expert s is implicit (rows n_tok*K + s*n_tok ..).  gate/up
+// quantises the F32 x itself; down writes `out` through the combine.
+cudaError_t launch_gateup_decode(const GateUpTable& tbl, const Slot* slots, const int32_t* n_slots,
+                                 const int32_t* perm, int n_tok, int K, int E, int n_shared, const float* x,
+                                 int hidden, int inter, int8_t* hq, float* hd, cudaStream_t st);
+cudaError_t launch_down_combine(const DownTable& tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K,
+                                int E, int n_shared, const int8_t* hq, const float* hd, const int32_t* inv,
+                                const float* w, int hidden, int inter, float* out, cudaStream_t st);
+
+// Prefill expert kernels on the tensor cores (tcgen05): build the tile list
+// (<= 64 tokens of one slot per tile) from the slot table, then the gate/up
+// GEMM (+ SwiGLU + Q8 of h) and the down GEMM (-> y).  `tiles` needs
+// prefill_tile_bytes(); grids are sized by prefill_tiles_bound().
+bool prefill_supported(int hidden, int inter);
+size_t prefill_tiles_bound(int n_tok, int K, int E, int n_shared);
+size_t prefill_tile_bytes(int n_tok, int K, int E, int n_shared);
+cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, const Slot* slots,
+                                   const int32_t* n_slots, void* tiles, int32_t* n_tiles, int max_tiles,
+                                   const int32_t* perm, int K, const int8_t* xq, const float* xd, int hidden,
+                                   int inter, int8_t* hq, float* hd, float* y, int32_t* err, cudaStream_t st,
+                                   cudaEvent_t ev_mid);
 
 // out[t] = sum_k w[t,k] y[inv[t,k]] + sum_s y[n_tok*K + s*n_tok + t]  (contract C)
 cudaError_t launch_combine(const float* y, const int32_t* inv, const float* w, int n_tok, int K,

@@ -39,16 +39,31 @@ __global__ void __launch_bounds__(256) router_scores_kernel(const float* __restr
   if (lane == 0) scores[gw] = sigmoid_cw(logit);
 }
 
-// One warp per token: K rounds of a warp-wide argmax over scores + bias
-// (ties to the lower expert index), then the weights.
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ scores,
-                                                   const float* __restrict__ bias, int n_tok, int E, int K,
-                                                   int norm, float rsf, int32_t* __restrict__ idx,
-                                                   float* __restrict__ wout) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= n_tok) return;
-  const float* st = scores + (int64_t)t * E;
+// Exclusive scan of v[0..n) in place by one warp; returns the total.
+__device__ int warp_exclusive_scan(int* v, int n, int lane) {
+  const int per = (n + 31) / 32;
+  const int lo = lane * per;
+  int local = 0;
+  for (int i = lo; i < lo + per && i < n; ++i) local += v[i];
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int run = incl - local;
+  for (int i = lo; i < lo + per && i < n; ++i) {
+    const int c = v[i];
+    v[i] = run;
+    run += c;
+  }
+  return __shfl_sync(0xffffffffu, incl, 31);
+}
+
+// Warp-wide top-k of one token: K rounds of an argmax over scores + bias
+// (ties to the lower expert index).  Every lane returns the same sel[0..K).
+__device__ __forceinline__ void warp_select_topk(const float* __restrict__ st, const float* __restrict__ bias, int E,
+                                                 int K, int lane, int (&sel)[kMaxTopK]) {
   float v[kMaxExperts / 32];
 #pragma unroll
   for (int i = 0; i < kMaxExperts / 32; ++i) {
@@ -56,7 +71,6 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
     v[i] = e < E ? __fadd_rn(st[e], bias[e]) : 0.0f;
   }
   uint32_t taken = 0;
-  int sel[kMaxTopK];
 #pragma unroll
   for (int k = 0; k < kMaxTopK; ++k) {
     if (k >= K) break;
@@ -84,47 +98,149 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
     sel[k] = be;
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
   }
-  if (lane == 0) {
-    float sk[kMaxTopK];
-    float denom = 0.0f;
+}
+
+// Weights of the selected experts (one lane): denom = s_r0 + s_r1 + ...
+// left to right; w_k = (s_rk / denom) * rsf, or s_rk * rsf.
+__device__ __forceinline__ void topk_weights(const float* __restrict__ st, const int (&sel)[kMaxTopK], int K, int norm,
+                                             float rsf, int32_t* __restrict__ idx, float* __restrict__ wout) {
+  float sk[kMaxTopK];
+  float denom = 0.0f;
 #pragma unroll
-    for (int k = 0; k < kMaxTopK; ++k) {
-      if (k >= K) break;
-      sk[k] = st[sel[k]];
-      denom = (k == 0) ? sk[k] : __fadd_rn(denom, sk[k]);
-    }
+  for (int k = 0; k < kMaxTopK; ++k) {
+    if (k >= K) break;
+    sk[k] = st[sel[k]];
+    denom = (k == 0) ? sk[k] : __fadd_rn(denom, sk[k]);
+  }
 #pragma unroll
-    for (int k = 0; k < kMaxTopK; ++k) {
-      if (k >= K) break;
-      idx[(int64_t)t * K + k] = sel[k];
-      wout[(int64_t)t * K + k] = norm ? __fmul_rn(__fdiv_rn(sk[k], denom), rsf) : __fmul_rn(sk[k], rsf);
+  for (int k = 0; k < kMaxTopK; ++k) {
+    if (k >= K) break;
+    idx[k] = sel[k];
+    wout[k] = norm ? __fmul_rn(__fdiv_rn(sk[k], denom), rsf) : __fmul_rn(sk[k], rsf);
+  }
+}
+
+// One warp per token.
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ scores,
+                                                   const float* __restrict__ bias, int n_tok, int E, int K,
+                                                   int norm, float rsf, int32_t* __restrict__ idx,
+                                                   float* __restrict__ wout) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= n_tok) return;
+  const float* st = scores + (int64_t)t * E;
+  int sel[kMaxTopK];
+  warp_select_topk(st, bias, E, K, lane, sel);
+  if (lane == 0) topk_weights(st, sel, K, norm, rsf, idx + (int64_t)t * K, wout + (int64_t)t * K);
+}
+
+// ---------------------------------------------------------------------------
+// Decode batches (n_tok <= kDecodeMaxTok): two kernels.
+
+// Router scores.  A CTA of 8 warps owns 2 experts; their router rows are
+// copied to shared memory with cp.async first (all 48 KB in flight at once),
+// then warp w folds expert (w & 1) for tokens t = w/2, w/2 + 4, ...
+__global__ void __launch_bounds__(256) router_decode_kernel(const float* __restrict__ x,
+                                                            const float* __restrict__ wr, int n_tok, int E, int H,
+                                                            float* __restrict__ scores) {
+  extern __shared__ __align__(16) float4 wsm[];  // [2][H/4]
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e0 = blockIdx.x * 2;
+  const int nq = H / 4;
+  for (int i = threadIdx.x; i < 2 * nq; i += blockDim.x) {
+    const int r = i / nq, j = i - r * nq;
+    if (e0 + r < E) cp_async16(wsm + i, wr + (size_t)(e0 + r) * H + 4 * j);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  const int r = warp & 1, e = e0 + r;
+  if (e >= E) return;
+  const float4* ws = wsm + r * nq;
+  for (int t = warp >> 1; t < n_tok; t += 4) {
+    const float4* xp = reinterpret_cast<const float4*>(x + (size_t)t * H);
+    float acc = 0.0f;
+#pragma unroll 8
+    for (int j = lane; j < nq; j += 32) {
+      const float4 a = __ldg(xp + j);
+      const float4 b = ws[j];
+      acc = __fmaf_rn(a.x, b.x, acc);
+      acc = __fmaf_rn(a.y, b.y, acc);
+      acc = __fmaf_rn(a.z, b.z, acc);
+      acc = __fmaf_rn(a.w, b.w, acc);
     }
+    const float logit = warp_sum_in_lane_order(acc);
+    if (lane == 0) scores[(size_t)t * E + e] = sigmoid_cw(logit);
+  }
+}
+
+// Top-k, weights and bucketing of a decode batch in one CTA: warp t selects
+// token t's experts; counts by shared atomics; offsets and the active-expert
+// list by warp scans; a pair's position within its expert group is the
+// number of earlier tokens that chose the same expert (stable by token).
+// The slot table lists the routed experts in ascending id.
+constexpr int kSmallThreads = 512;
+__global__ void __launch_bounds__(kSmallThreads) topk_bucket_small_kernel(
+    const float* __restrict__ scores, const float* __restrict__ bias, int n_tok, int E, int K, int norm, float rsf,
+    int32_t* __restrict__ idx_out, float* __restrict__ w_out, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv, Slot* __restrict__ slots,
+    int32_t* __restrict__ n_slots) {
+  __shared__ int s_idx[kDecodeMaxTok * kMaxTopK];
+  __shared__ int cnt[kMaxExperts];
+  __shared__ int off[kMaxExperts];
+  __shared__ int act[kMaxExperts];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+  if (warp < n_tok) {
+    const float* st = scores + (size_t)warp * E;
+    int sel[kMaxTopK];
+    warp_select_topk(st, bias, E, K, lane, sel);
+    if (lane == 0) {
+      topk_weights(st, sel, K, norm, rsf, idx_out + (size_t)warp * K, w_out + (size_t)warp * K);
+#pragma unroll
+      for (int k = 0; k < kMaxTopK; ++k)
+        if (k < K) s_idx[warp * K + k] = sel[k];
+    }
+  }
+  __syncthreads();
+  const int n_pairs = n_tok * K;
+  for (int p = tid; p < n_pairs; p += blockDim.x) atomicAdd(&cnt[s_idx[p]], 1);
+  __syncthreads();
+  if (warp == 0) {
+    for (int e = lane; e < E; e += 32) {
+      off[e] = cnt[e];
+      act[e] = cnt[e] > 0 ? 1 : 0;
+    }
+    __syncwarp();
+    const int total = warp_exclusive_scan(off, E, lane);
+    __syncwarp();
+    const int n_active = warp_exclusive_scan(act, E, lane);
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) {
+      counts[e] = cnt[e];
+      offsets[e] = off[e];
+      if (cnt[e] > 0) slots[act[e]] = Slot{e, off[e], cnt[e], off[e]};
+    }
+    if (lane == 0) {
+      offsets[E] = total;
+      *n_slots = n_active;
+    }
+  }
+  __syncthreads();
+  for (int p = tid; p < n_pairs; p += blockDim.x) {
+    const int t = p / K, e = s_idx[p];
+    int rank = 0;
+    for (int q = 0; q < t * K; ++q) rank += (s_idx[q] == e);
+    const int pos = off[e] + rank;
+    perm[pos] = p;
+    inv[p] = pos;
   }
 }
 
 constexpr int kBucketThreads = 1024;
 constexpr int kChunk = 1024;  // tokens per ranking round: one per thread
-
-// Exclusive scan of v[0..n) in place by one warp; returns the total.
-__device__ int warp_exclusive_scan(int* v, int n, int lane) {
-  const int per = (n + 31) / 32;
-  const int lo = lane * per;
-  int local = 0;
-  for (int i = lo; i < lo + per && i < n; ++i) local += v[i];
-  int incl = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  int run = incl - local;
-  for (int i = lo; i < lo + per && i < n; ++i) {
-    const int c = v[i];
-    v[i] = run;
-    run += c;
-  }
-  return __shfl_sync(0xffffffffu, incl, 31);
-}
 
 // Single block.  Counts by shared-memory atomics (order-free), offsets by a
 // scan, then a stable scatter: tokens are ranked within each expert through
@@ -241,6 +357,28 @@ cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E
                         int32_t* idx, float* w, cudaStream_t st) {
   topk_kernel<<<(n_tok + 7) / 8, 256, 0, st>>>(scores, bias, n_tok, E, K, norm, rsf, idx, w);
   return cudaGetLastError();
+}
+
+cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
+                                 cudaStream_t st) {
+  const size_t smem = (size_t)2 * H * sizeof(float);
+  static int attr_dev_mask = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_dev_mask & (1 << (dev & 31)))) {
+    cudaError_t e = cudaFuncSetAttribute(router_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_dev_mask |= 1 << (dev & 31);
+  }
+  router_decode_kernel<<<(E + 1) / 2, 256, smem, st>>>(x, w_router, n_tok, E, H, scores);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_bucket_small(const float* scores, const float* bias, int n_tok, int E, int K, int norm,
+                                     float rsf, int32_t* idx, float* w, int32_t* counts, int32_t* offsets,
+                                     int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, cudaStream_t st) {
+  return launch_pdl(topk_bucket_small_kernel, dim3(1), dim3(kSmallThreads), 0, st, true, scores, bias, n_tok, E, K,
+                    norm, rsf, idx, w, counts, offsets, perm, inv, slots, n_slots);
 }
 
 cudaError_t launch_bucket(const int32_t* idx, int n_tok, int K, int E, int n_shared, int32_t* counts,

@@ -48,9 +48,22 @@ def _check_layer(coli, syn, cfg, n_tok, sample=None, exact=True):
     return out
 
 
-@pytest.mark.parametrize("n_tok", [8, 1, 2, 3, 5, 13])
+@pytest.mark.parametrize("n_tok", [8, 1, 2, 3, 5, 13, 16])
 def test_layer_tiny(coli, syn, n_tok):
+    """Decode path (<= 16 tokens)."""
     _check_layer(coli, syn, syn.config("tiny"), n_tok)
+
+
+@pytest.mark.parametrize("n_tok", [17, 64, 65, 130, 300, 1000])
+def test_layer_tiny_prefill_path(coli, syn, n_tok):
+    """Tensor-core path (> 16 tokens): ragged tiles of <= 64 tokens, several
+    tiles per expert, partial 16-column MMAs."""
+    _check_layer(coli, syn, syn.config("tiny"), n_tok)
+
+
+@pytest.mark.parametrize("over", [dict(top_k=1), dict(n_shared=0), dict(n_shared=2), dict(norm_topk_prob=False)])
+def test_layer_tiny_prefill_variants(coli, syn, over):
+    _check_layer(coli, syn, syn.config("tiny", **over), 200)
 
 
 @pytest.mark.parametrize("over", [dict(norm_topk_prob=False), dict(routed_scaling_factor=1.0),
@@ -73,6 +86,11 @@ def test_layer_decode16(coli, syn):
 
 def test_layer_prefill2048_sampled(coli, syn):
     _check_layer(coli, syn, syn.config("prefill2048"), 2048, sample=4)
+
+
+def test_layer_prefill_glm_ragged(coli, syn):
+    """GLM shape, 100 tokens: every expert gets a partial tile."""
+    _check_layer(coli, syn, syn.config("prefill2048"), 100, sample=3)
 
 
 def test_layer_zero_tokens_is_noop(coli, syn):
