@@ -131,6 +131,15 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Loads of data that an earlier kernel of the same forward writes.  Kernels
+// launched with programmatic dependent launch start while their predecessor
+// still runs, so such data must not be declared __restrict__ (the compiler
+// may then treat it as invariant and load it before the dependency wait) and
+// is read through L2 (ld.global.cg), after pdl_wait().
+__device__ __forceinline__ int32_t ld_dep(const int32_t* p) { return __ldcg(p); }
+__device__ __forceinline__ float ld_dep(const float* p) { return __ldcg(p); }
+__device__ __forceinline__ uint4 ld_dep(const uint4* p) { return __ldcg(p); }
+
 // Q8_0 of one value given its block scale d (d == 0 -> 0).
 __device__ __forceinline__ int q8_of(float v, float d) {
   if (d == 0.0f) return 0;

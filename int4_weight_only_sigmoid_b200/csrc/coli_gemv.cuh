@@ -40,14 +40,14 @@ __device__ __forceinline__ int token_of(const GemvSlots& sl, const Slot& s, int 
 // Stage n_valid activation rows (Q8 bytes + block scales) into shared memory
 // as even/odd byte planes.  act_row(i) gives the source row of token i.
 template <int TT, typename RowFn>
-__device__ __forceinline__ void stage_acts(const int8_t* __restrict__ aq, const float* __restrict__ ad, int dim_in,
+__device__ __forceinline__ void stage_acts(const int8_t* aq, const float* ad, int dim_in,
                                            int n_valid, RowFn act_row, uint4* xe_s, uint4* xo_s, float* xd_s) {
   const int nb = dim_in / 32;
   for (int i = threadIdx.x; i < n_valid * nb; i += kThreads) {
     const int t = i / nb, b = i - t * nb;
     const int64_t row = act_row(t);
     const uint4* src = reinterpret_cast<const uint4*>(aq + row * dim_in + 32 * b);
-    const uint4 a0 = src[0], a1 = src[1];
+    const uint4 a0 = ld_dep(src), a1 = ld_dep(src + 1);
     uint4 e, o;
     split_even_odd(a0.x, a0.y, e.x, o.x);
     split_even_odd(a0.z, a0.w, e.y, o.y);
@@ -55,7 +55,7 @@ __device__ __forceinline__ void stage_acts(const int8_t* __restrict__ aq, const 
     split_even_odd(a1.z, a1.w, e.w, o.w);
     xe_s[t * nb + b] = e;
     xo_s[t * nb + b] = o;
-    xd_s[t * nb + b] = ad[row * nb + b];
+    xd_s[t * nb + b] = ld_dep(ad + row * nb + b);
   }
 }
 

@@ -48,10 +48,11 @@ cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E
 // Decode batches: router scores with the router rows staged in shared memory
 // (plain launch), then top-k + weights + bucketing in one CTA (PDL launch).
 cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
-                                 cudaStream_t st);
+                                 int8_t* xq, float* xd, cudaStream_t st);
 cudaError_t launch_topk_bucket_small(const float* scores, const float* bias, int n_tok, int E, int K, int norm,
                                      float rsf, int32_t* idx, float* w, int32_t* counts, int32_t* offsets,
-                                     int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, cudaStream_t st);
+                                     int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, int32_t* chunk_done,
+                                     int n_chunk, cudaStream_t st);
 
 // Bucketing: counts, offsets, perm; optionally the inverse map (pair ->
 // position), the expert slot table (+ shared slots) and its length.
@@ -74,12 +75,16 @@ cudaError_t launch_gateup(const GateUpTable& tbl, const GemvSlots& sl, const int
 cudaError_t launch_down(const DownTable& tbl, const GemvSlots& sl, const int8_t* hq, const float* hd,
                         int hidden, int inter, int max_tok_per_slot, float* y, cudaStream_t st);
 
-// Decode expert kernels (PDL launches).  Slot table = the routed experts
-// only; shared expert s is implicit (rows n_tok*K + s*n_tok ..).  gate/up
-// quantises the F32 x itself; down writes `out` through the combine.
+// Decode expert kernels (persistent, PDL launches).  Slot table = the routed
+// experts only; shared expert s is implicit (rows n_tok*K + s*n_tok ..).
+// gate/up quantises the F32 x itself for the shared experts (which start
+// before the routing is done) and reads the router kernel's Q8 of x for the
+// routed ones; down computes 16-row chunks of every expert and combines them
+// into `out` in shared memory.
 cudaError_t launch_gateup_decode(const GateUpTable& tbl, const Slot* slots, const int32_t* n_slots,
                                  const int32_t* perm, int n_tok, int K, int E, int n_shared, const float* x,
-                                 int hidden, int inter, int8_t* hq, float* hd, cudaStream_t st);
+                                 const int8_t* xq, const float* xd, int hidden, int inter, int8_t* hq, float* hd,
+                                 cudaStream_t st);
 cudaError_t launch_down_combine(const DownTable& tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K,
                                 int E, int n_shared, const int8_t* hq, const float* hd, const int32_t* inv,
                                 const float* w, int hidden, int inter, float* out, cudaStream_t st);

@@ -20,10 +20,12 @@
 // pipe, is the limit of this layer (one FMA per 32 MACs).  fp16 operands
 // give F32 sums directly.
 //
-// Roles (288 threads): warps 0-3 epilogue (TMEM lanes 0-127 = the tile's
-// rows), warps 4-7 producers (cp.async of packed weights and Q8 activations
-// into a staging ring, expansion to fp16 into the operand ring), warp 8 the
-// MMA issuer (lane 0) and TMEM owner.  All waits are bounded (coli_tc.cuh).
+// Roles (384 threads): warps 0-7 epilogue (warp w reads TMEM lanes
+// 32(w%4).. = 32 of the tile's rows, columns [32(w/4), 32(w/4)+32) = half of
+// the tokens), warps 8-10 producers (cp.async of packed weights and Q8
+// activations into a staging ring, expansion to fp16 into the operand ring),
+// warp 11 the MMA issuer (lane 0) and TMEM owner.  All waits are bounded
+// (coli_tc.cuh).
 //
 // Sources: "Colibri：在笔记本上跑744B参数的AI模型", "关键特性" (integer dot
 // kernels, Q8_0 activations, packed int4); HN summary (hn.213312.xyz),
@@ -43,8 +45,12 @@ constexpr int kM = 128;       // rows per tile (TMEM lanes)
 constexpr int kN = 64;        // tokens per tile (max)
 constexpr int kSB = 4;        // Q8 blocks per packed super-stage
 constexpr int kStages = 3;    // operand ring depth
-constexpr int kThreadsP = 288;
-constexpr int kProd = 128, kMma = 256;  // first producer / MMA thread (epilogue: 0..127)
+constexpr int kEpiWarps = 8;              // 2 per TMEM lane quadrant, each half of the columns
+constexpr int kProdWarps = 3;
+constexpr int kThreadsP = 32 * (kEpiWarps + kProdWarps + 1);  // 384
+constexpr int kProd = 32 * kEpiWarps;                         // first producer thread
+constexpr int kNProd = 32 * kProdWarps;                       // producer threads
+constexpr int kMma = kProd + kNProd;                          // the MMA warp
 
 template <bool GU>
 struct PSmem {
@@ -151,18 +157,18 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_bar[s], 128);
+      mbar_init(&full_bar[s], kNProd);
       mbar_init(&empty_bar[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], 128);
+      mbar_init(&tempty_bar[b], 32 * kEpiWarps);
     }
     mbar_init(&done_bar, 1);
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 8) tmem_alloc(&tmem_s, L::kTmemCols);
+  if (warp == kMma / 32) tmem_alloc(&tmem_s, L::kTmemCols);
   // block scales of the tile's tokens, [kb][64] with the 4-float groups of
   // each row XOR-permuted by (kb & 3) to spread the transposing stores
   for (int i = threadIdx.x; i < kN * nb; i += kThreadsP) {
@@ -194,14 +200,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       unsigned char* pk = pk_ring + (ss & 1) * L::kPkStage;
 #pragma unroll
       for (int m = 0; m < L::kMats; ++m) {
-        for (int i = p; i < kM * kSB; i += 128) {  // 128 rows x kSB 16-byte chunks
+        for (int i = p; i < kM * kSB; i += kNProd) {  // 128 rows x kSB 16-byte chunks
           const int r = i / kSB, c = i % kSB;
           cp_async16(pk + m * L::kPkA + r * (kSB * 16) + ((c ^ ((r >> 1) & 3)) * 16),
                      (m == 0 ? qa0 : qa1) + (size_t)r * rb + (size_t)(ss * kSB + c) * 16);
         }
       }
       unsigned char* pb = pk + L::kMats * L::kPkA;
-      for (int i = p; i < kN * kSB * 2; i += 128) {  // 64 tokens x 2*kSB 16-byte chunks
+      for (int i = p; i < kN * kSB * 2; i += kNProd) {  // 64 tokens x 2*kSB 16-byte chunks
         const int n = i / (kSB * 2), c = i % (kSB * 2);
         if (n < n_valid)
           cp_async16(pb + n * (kSB * 32) + ((c ^ (n & 7)) * 16), aq + act_row(n) * dim_in + ss * kSB * 32 + c * 16);
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       } else {
         asm volatile("cp.async.wait_group 0;" ::: "memory");
       }
-      named_bar(1, 128);  // every producer's copies of super-stage ss are in
+      named_bar(1, kNProd);  // every producer's copies of super-stage ss are in
       const unsigned char* pk = pk_ring + (ss & 1) * L::kPkStage;
       for (int kl = 0; kl < kSB; ++kl) {
         const int kb = ss * kSB + kl;
@@ -227,36 +233,38 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         alive = alive && mbar_wait(&empty_bar[s], ((kb / kStages) & 1) ^ 1, abort, err, 10);
         if (!alive) continue;
         unsigned char* op = op_ring + s * L::kOpStage;
-        // A: row p of each matrix, K-block kb
-#pragma unroll
-        for (int m = 0; m < L::kMats; ++m) {
-          const uint4 w = *reinterpret_cast<const uint4*>(pk + m * L::kPkA + p * (kSB * 16) +
-                                                          ((kl ^ ((p >> 1) & 3)) * 16));
-          unsigned char* dst = op + m * L::kOpA;
-          *reinterpret_cast<uint4*>(dst + op_off(p, 0)) = expand_int4_word(w.x);
-          *reinterpret_cast<uint4*>(dst + op_off(p, 1)) = expand_int4_word(w.y);
-          *reinterpret_cast<uint4*>(dst + op_off(p, 2)) = expand_int4_word(w.z);
-          *reinterpret_cast<uint4*>(dst + op_off(p, 3)) = expand_int4_word(w.w);
-        }
-        // B: token n = p/2, half h = p%2 (16 of the block's 32 values)
-        {
-          const int n = p >> 1, h = p & 1;
-          unsigned char* dst = op + L::kMats * L::kOpA;
-          uint4 e0 = make_uint4(0, 0, 0, 0), e1 = e0;
-          if (n < n_valid) {
-            const int c = 2 * kl + h;
-            const uint4 v = *reinterpret_cast<const uint4*>(pk + L::kMats * L::kPkA + n * (kSB * 32) +
-                                                            ((c ^ (n & 7)) * 16));
-            e0 = expand_int8_pair(v.x, v.y);
-            e1 = expand_int8_pair(v.z, v.w);
+        // work items of this K-block: (matrix m, row r) expansions of A, then
+        // (token n, half h) expansions of B
+        for (int i = p; i < L::kMats * kM + 2 * kN; i += kNProd) {
+          if (i < L::kMats * kM) {
+            const int m = i / kM, r = i % kM;
+            const uint4 w = *reinterpret_cast<const uint4*>(pk + m * L::kPkA + r * (kSB * 16) +
+                                                            ((kl ^ ((r >> 1) & 3)) * 16));
+            unsigned char* dst = op + m * L::kOpA;
+            *reinterpret_cast<uint4*>(dst + op_off(r, 0)) = expand_int4_word(w.x);
+            *reinterpret_cast<uint4*>(dst + op_off(r, 1)) = expand_int4_word(w.y);
+            *reinterpret_cast<uint4*>(dst + op_off(r, 2)) = expand_int4_word(w.z);
+            *reinterpret_cast<uint4*>(dst + op_off(r, 3)) = expand_int4_word(w.w);
+          } else {
+            const int j = i - L::kMats * kM;
+            const int n = j >> 1, h = j & 1;
+            unsigned char* dst = op + L::kMats * L::kOpA;
+            uint4 e0 = make_uint4(0, 0, 0, 0), e1 = e0;
+            if (n < n_valid) {
+              const int c = 2 * kl + h;
+              const uint4 v = *reinterpret_cast<const uint4*>(pk + L::kMats * L::kPkA + n * (kSB * 32) +
+                                                              ((c ^ (n & 7)) * 16));
+              e0 = expand_int8_pair(v.x, v.y);
+              e1 = expand_int8_pair(v.z, v.w);
+            }
+            *reinterpret_cast<uint4*>(dst + op_off(n, 2 * h)) = e0;
+            *reinterpret_cast<uint4*>(dst + op_off(n, 2 * h + 1)) = e1;
           }
-          *reinterpret_cast<uint4*>(dst + op_off(n, 2 * h)) = e0;
-          *reinterpret_cast<uint4*>(dst + op_off(n, 2 * h + 1)) = e1;
         }
         fence_async_smem();
         mbar_arrive(&full_bar[s]);
       }
-      named_bar(1, 128);  // packed buffer ss & 1 may be refilled after this
+      named_bar(1, kNProd);  // packed buffer ss & 1 may be refilled after this
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
   } else if (threadIdx.x >= kMma) {
@@ -292,54 +300,65 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    float acc0[kN], acc1[kN];
+    // warp w: TMEM lanes 32*(w%4).. (rows), columns [cb, cb + 32) (tokens)
+    constexpr int kC = kN / 2;
+    const int quad = warp & 3, cb = (warp >> 2) * kC;
+    float acc0[kC], acc1[kC];
 #pragma unroll
-    for (int n = 0; n < kN; ++n) {
+    for (int n = 0; n < kC; ++n) {
       acc0[n] = 0.0f;
       acc1[n] = 0.0f;
     }
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const bool active = cb < n_pad;  // warp-uniform
     for (int kb = 0; kb < nb; ++kb) {
       const int b = kb & 1;
       if (!mbar_wait(&tfull_bar[b], (kb >> 1) & 1, abort, err, 13)) break;
       fence_after_sync();
-      const float* dxk = xd_s + kb * kN;
-      const int g_x = kb & 3;
+      if (active) {
+        const uint32_t col = tmem + lane_base + b * (L::kMats * kN) + cb;
+        uint32_t r0[kC], r1[kC];
+        // issue every load of the block, then one wait
+        tmem_ld16(col, *reinterpret_cast<uint32_t(*)[16]>(&r0[0]));
+        if (cb + 16 < n_pad) tmem_ld16(col + 16, *reinterpret_cast<uint32_t(*)[16]>(&r0[16]));
+        if constexpr (GU) {
+          tmem_ld16(col + kN, *reinterpret_cast<uint32_t(*)[16]>(&r1[0]));
+          if (cb + 16 < n_pad) tmem_ld16(col + kN + 16, *reinterpret_cast<uint32_t(*)[16]>(&r1[16]));
+        }
+        tmem_ld_wait();
+        fence_before_sync();
+        mbar_arrive(&tempty_bar[b]);  // TMEM buffer b may be rewritten now
+        const float* dxk = xd_s + kb * kN;
+        const int g_x = kb & 3;
 #pragma unroll
-      for (int j = 0; j < kN / 8; ++j) {  // 8 columns at a time (register budget: 9 warps -> 168 regs)
-        if (j * 8 < n_pad) {
-          uint32_t r0[8];
-          tmem_ld8(tmem + lane_base + b * (L::kMats * kN) + j * 8, r0);
-          uint32_t r1[8];
-          if constexpr (GU) tmem_ld8(tmem + lane_base + b * (L::kMats * kN) + kN + j * 8, r1);
-          tmem_ld_wait();
-#pragma unroll
-          for (int gg = 0; gg < 2; ++gg) {
-            const int g = 2 * j + gg;  // absolute group of 4 columns
+        for (int gl = 0; gl < kC / 4; ++gl) {
+          const int g = cb / 4 + gl;  // absolute group of 4 columns
+          if (4 * g < n_pad) {
             const float4 d4 = *reinterpret_cast<const float4*>(dxk + (g & ~3) * 4 + 4 * ((g & 3) ^ g_x));
             const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const int n = 4 * g + i;
-              acc0[n] = __fmaf_rn(dv[i], __uint_as_float(r0[4 * gg + i]), acc0[n]);
-              if constexpr (GU) acc1[n] = __fmaf_rn(dv[i], __uint_as_float(r1[4 * gg + i]), acc1[n]);
+              acc0[4 * gl + i] = __fmaf_rn(dv[i], __uint_as_float(r0[4 * gl + i]), acc0[4 * gl + i]);
+              if constexpr (GU) acc1[4 * gl + i] = __fmaf_rn(dv[i], __uint_as_float(r1[4 * gl + i]), acc1[4 * gl + i]);
             }
           }
         }
+      } else {
+        fence_before_sync();
+        mbar_arrive(&tempty_bar[b]);
       }
-      fence_before_sync();
-      mbar_arrive(&tempty_bar[b]);
     }
-    if (!*abort) {
-      const int o = m0 + threadIdx.x;
+    if (!*abort && active) {
+      const int o = m0 + quad * 32 + lane;
       if constexpr (GU) {
         const float sg = tab.gate_s[slot.table_idx][o];
         const float su = tab.up_s[slot.table_idx][o];
 #pragma unroll
-        for (int n = 0; n < kN; ++n) {
+        for (int j = 0; j < kC; ++j) {
+          const int n = cb + j;
           if (n < n_valid) {
-            const float g = __fmul_rn(sg, acc0[n]);
-            const float u = __fmul_rn(su, acc1[n]);
+            const float g = __fmul_rn(sg, acc0[j]);
+            const float u = __fmul_rn(su, acc1[j]);
             const float h = __fmul_rn(__fmul_rn(g, sigmoid_cw(g)), u);
             const float d = __fdiv_rn(warp_max(fabsf(h)), 127.0f);
             const int64_t row = (int64_t)slot.row_base + tile.n0 + n;
@@ -350,15 +369,16 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       } else {
         const float sd = tab.down_s[slot.table_idx][o];
 #pragma unroll
-        for (int n = 0; n < kN; ++n) {
-          if (n < n_valid) y[((int64_t)slot.row_base + tile.n0 + n) * hidden + o] = __fmul_rn(sd, acc0[n]);
+        for (int j = 0; j < kC; ++j) {
+          const int n = cb + j;
+          if (n < n_valid) y[((int64_t)slot.row_base + tile.n0 + n) * hidden + o] = __fmul_rn(sd, acc0[j]);
         }
       }
     }
   }
   fence_before_sync();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kMma / 32) {
     fence_after_sync();
     tmem_dealloc(tmem, L::kTmemCols);
   }

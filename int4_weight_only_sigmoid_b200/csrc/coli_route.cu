@@ -61,20 +61,22 @@ __device__ int warp_exclusive_scan(int* v, int n, int lane) {
 }
 
 // Warp-wide top-k of one token: K rounds of an argmax over scores + bias
-// (ties to the lower expert index).  Every lane returns the same sel[0..K).
-__device__ __forceinline__ void warp_select_topk(const float* __restrict__ st, const float* __restrict__ bias, int E,
-                                                 int K, int lane, int (&sel)[kMaxTopK]) {
-  float v[kMaxExperts / 32];
+// (ties to the lower expert index).  Every lane returns the same sel[0..K)
+// and the selected unbiased scores ssel[0..K).
+__device__ __forceinline__ void warp_select_topk(const float* st, const float* __restrict__ bias, int E, int K,
+                                                 int lane, int (&sel)[kMaxTopK], float (&ssel)[kMaxTopK]) {
+  float v[kMaxExperts / 32], sv[kMaxExperts / 32];
 #pragma unroll
   for (int i = 0; i < kMaxExperts / 32; ++i) {
     const int e = lane + 32 * i;
-    v[i] = e < E ? __fadd_rn(st[e], bias[e]) : 0.0f;
+    sv[i] = e < E ? ld_dep(st + e) : 0.0f;
+    v[i] = e < E ? __fadd_rn(sv[i], bias[e]) : 0.0f;
   }
   uint32_t taken = 0;
 #pragma unroll
   for (int k = 0; k < kMaxTopK; ++k) {
     if (k >= K) break;
-    float bv = 0.0f;
+    float bv = 0.0f, bs = 0.0f;
     int be = INT_MAX;
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i) {
@@ -82,6 +84,7 @@ __device__ __forceinline__ void warp_select_topk(const float* __restrict__ st, c
       if (e < E && !((taken >> i) & 1u)) {
         if (be == INT_MAX || v[i] > bv) {  // ascending e: strict '>' keeps the lower index
           bv = v[i];
+          bs = sv[i];
           be = e;
         }
       }
@@ -89,27 +92,28 @@ __device__ __forceinline__ void warp_select_topk(const float* __restrict__ st, c
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const float os = __shfl_xor_sync(0xffffffffu, bs, o);
       const int oe = __shfl_xor_sync(0xffffffffu, be, o);
       if (oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be))) {
         bv = ov;
+        bs = os;
         be = oe;
       }
     }
     sel[k] = be;
+    ssel[k] = bs;
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
   }
 }
 
 // Weights of the selected experts (one lane): denom = s_r0 + s_r1 + ...
 // left to right; w_k = (s_rk / denom) * rsf, or s_rk * rsf.
-__device__ __forceinline__ void topk_weights(const float* __restrict__ st, const int (&sel)[kMaxTopK], int K, int norm,
+__device__ __forceinline__ void topk_weights(const int (&sel)[kMaxTopK], const float (&sk)[kMaxTopK], int K, int norm,
                                              float rsf, int32_t* __restrict__ idx, float* __restrict__ wout) {
-  float sk[kMaxTopK];
   float denom = 0.0f;
 #pragma unroll
   for (int k = 0; k < kMaxTopK; ++k) {
     if (k >= K) break;
-    sk[k] = st[sel[k]];
     denom = (k == 0) ? sk[k] : __fadd_rn(denom, sk[k]);
   }
 #pragma unroll
@@ -130,27 +134,42 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
   if (t >= n_tok) return;
   const float* st = scores + (int64_t)t * E;
   int sel[kMaxTopK];
-  warp_select_topk(st, bias, E, K, lane, sel);
-  if (lane == 0) topk_weights(st, sel, K, norm, rsf, idx + (int64_t)t * K, wout + (int64_t)t * K);
+  float ssel[kMaxTopK];
+  warp_select_topk(st, bias, E, K, lane, sel, ssel);
+  if (lane == 0) topk_weights(sel, ssel, K, norm, rsf, idx + (int64_t)t * K, wout + (int64_t)t * K);
 }
 
 // ---------------------------------------------------------------------------
 // Decode batches (n_tok <= kDecodeMaxTok): two kernels.
 
-// Router scores.  A CTA of 8 warps owns 2 experts; their router rows are
-// copied to shared memory with cp.async first (all 48 KB in flight at once),
-// then warp w folds expert (w & 1) for tokens t = w/2, w/2 + 4, ...
+// Router scores.  A CTA of 8 warps owns 2 experts; their router rows and
+// (for up to kStageTok tokens) the token rows are copied to shared memory
+// with cp.async first, so the fold loop below reads only shared memory;
+// warp w folds expert (w & 1) for tokens t = w/2, w/2 + 4, ...  The CTAs
+// also write the Q8_0 of x for the expert kernels.
+constexpr int kStageTok = 2;
 __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restrict__ x,
                                                             const float* __restrict__ wr, int n_tok, int E, int H,
-                                                            float* __restrict__ scores) {
-  extern __shared__ __align__(16) float4 wsm[];  // [2][H/4]
+                                                            float* __restrict__ scores, int8_t* __restrict__ xq,
+                                                            float* __restrict__ xd) {
+  extern __shared__ __align__(16) float4 wsm[];  // [2][H/4] router rows, then [kStageTok][H/4] tokens
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e0 = blockIdx.x * 2;
   const int nq = H / 4;
+  const bool stage_x = n_tok <= kStageTok;
   for (int i = threadIdx.x; i < 2 * nq; i += blockDim.x) {
     const int r = i / nq, j = i - r * nq;
     if (e0 + r < E) cp_async16(wsm + i, wr + (size_t)(e0 + r) * H + 4 * j);
+  }
+  if (stage_x)
+    for (int i = threadIdx.x; i < n_tok * nq; i += blockDim.x) cp_async16(wsm + 2 * nq + i, x + 4 * (size_t)i);
+  // the Q8_0 of x for the expert kernels: one warp per 32-element block
+  for (int j = blockIdx.x * 8 + warp; j < n_tok * (H / 32); j += gridDim.x * 8) {
+    const float v = x[(size_t)j * 32 + lane];
+    const float d = __fdiv_rn(warp_max(fabsf(v)), 127.0f);
+    xq[(size_t)j * 32 + lane] = (int8_t)q8_of(v, d);
+    if (lane == 0) xd[j] = d;
   }
   cp_async_wait_all();
   __syncthreads();
@@ -158,11 +177,11 @@ __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restr
   if (e >= E) return;
   const float4* ws = wsm + r * nq;
   for (int t = warp >> 1; t < n_tok; t += 4) {
-    const float4* xp = reinterpret_cast<const float4*>(x + (size_t)t * H);
+    const float4* xp = stage_x ? wsm + (2 + t) * nq : reinterpret_cast<const float4*>(x + (size_t)t * H);
     float acc = 0.0f;
 #pragma unroll 8
     for (int j = lane; j < nq; j += 32) {
-      const float4 a = __ldg(xp + j);
+      const float4 a = xp[j];
       const float4 b = ws[j];
       acc = __fmaf_rn(a.x, b.x, acc);
       acc = __fmaf_rn(a.y, b.y, acc);
@@ -181,10 +200,10 @@ __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restr
 // The slot table lists the routed experts in ascending id.
 constexpr int kSmallThreads = 512;
 __global__ void __launch_bounds__(kSmallThreads) topk_bucket_small_kernel(
-    const float* __restrict__ scores, const float* __restrict__ bias, int n_tok, int E, int K, int norm, float rsf,
+    const float* scores, const float* __restrict__ bias, int n_tok, int E, int K, int norm, float rsf,
     int32_t* __restrict__ idx_out, float* __restrict__ w_out, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv, Slot* __restrict__ slots,
-    int32_t* __restrict__ n_slots) {
+    int32_t* __restrict__ n_slots, int32_t* __restrict__ chunk_done, int n_chunk) {
   __shared__ int s_idx[kDecodeMaxTok * kMaxTopK];
   __shared__ int cnt[kMaxExperts];
   __shared__ int off[kMaxExperts];
@@ -193,12 +212,14 @@ __global__ void __launch_bounds__(kSmallThreads) topk_bucket_small_kernel(
   pdl_launch_dependents();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+  for (int i = tid; i < n_chunk; i += blockDim.x) chunk_done[i] = 0;  // the down kernel's per-chunk counters
   if (warp < n_tok) {
     const float* st = scores + (size_t)warp * E;
     int sel[kMaxTopK];
-    warp_select_topk(st, bias, E, K, lane, sel);
+    float ssel[kMaxTopK];
+    warp_select_topk(st, bias, E, K, lane, sel, ssel);
     if (lane == 0) {
-      topk_weights(st, sel, K, norm, rsf, idx_out + (size_t)warp * K, w_out + (size_t)warp * K);
+      topk_weights(sel, ssel, K, norm, rsf, idx_out + (size_t)warp * K, w_out + (size_t)warp * K);
 #pragma unroll
       for (int k = 0; k < kMaxTopK; ++k)
         if (k < K) s_idx[warp * K + k] = sel[k];
@@ -360,8 +381,8 @@ cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E
 }
 
 cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
-                                 cudaStream_t st) {
-  const size_t smem = (size_t)2 * H * sizeof(float);
+                                 int8_t* xq, float* xd, cudaStream_t st) {
+  const size_t smem = (size_t)(2 + (n_tok <= kStageTok ? n_tok : 0)) * H * sizeof(float);
   static int attr_dev_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -370,15 +391,16 @@ cudaError_t launch_router_decode(const float* x, const float* w_router, int n_to
     if (e != cudaSuccess) return e;
     attr_dev_mask |= 1 << (dev & 31);
   }
-  router_decode_kernel<<<(E + 1) / 2, 256, smem, st>>>(x, w_router, n_tok, E, H, scores);
+  router_decode_kernel<<<(E + 1) / 2, 256, smem, st>>>(x, w_router, n_tok, E, H, scores, xq, xd);
   return cudaGetLastError();
 }
 
 cudaError_t launch_topk_bucket_small(const float* scores, const float* bias, int n_tok, int E, int K, int norm,
                                      float rsf, int32_t* idx, float* w, int32_t* counts, int32_t* offsets,
-                                     int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, cudaStream_t st) {
+                                     int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, int32_t* chunk_done,
+                                     int n_chunk, cudaStream_t st) {
   return launch_pdl(topk_bucket_small_kernel, dim3(1), dim3(kSmallThreads), 0, st, true, scores, bias, n_tok, E, K,
-                    norm, rsf, idx, w, counts, offsets, perm, inv, slots, n_slots);
+                    norm, rsf, idx, w, counts, offsets, perm, inv, slots, n_slots, chunk_done, n_chunk);
 }
 
 cudaError_t launch_bucket(const int32_t* idx, int n_tok, int K, int E, int n_shared, int32_t* counts,

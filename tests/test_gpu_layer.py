@@ -114,6 +114,24 @@ def test_layer_token_subset_consistency(coli, syn):
         assert bits_equal(one[0], full[t])
 
 
+@pytest.mark.parametrize("name,n_tok", [("decode1", 1), ("decode4", 4), ("tiny", 16), ("tiny", 40)])
+def test_workspace_contents_do_not_matter(coli, syn, name, n_tok):
+    """Repeated forwards on workspaces first memset to 0x00, 0x5A or 0xFF give
+    the same bits: no kernel reads scratch before the forward writes it, and
+    no kernel launched early (programmatic dependent launch) reads a
+    predecessor's output before that output is complete."""
+    import torch
+    cfg = syn.config(name)
+    L = _dev_layer(cfg)
+    x = torch.from_numpy(syn.tokens(cfg, n_tok)).cuda()
+    ref = _np(coli.moe_layer_forward(L, x))
+    for it in range(24):
+        ws = coli.make_workspace(L.cfg, n_tok)
+        ws.fill_((0x00, 0x5A, 0xFF)[it % 3])
+        got = _np(coli.moe_layer_forward(L, x, workspace=ws))
+        assert bits_equal(got, ref), f"iteration {it}"
+
+
 def test_layer_guard_bytes_untouched(coli, syn):
     """Canary words after the output and around the workspace stay intact."""
     import torch
