@@ -94,7 +94,7 @@ coli_status check_layer(const coli_moe_layer* L, const char* fn) {
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Workspace {
-  size_t xq, xd, scores, idx, w, counts, offsets, perm, inv, slots, n_slots, status, tiles, n_tiles, chunk_done, hq, hd,
+  size_t xq, xd, scores, idx, w, counts, offsets, perm, inv, slots, n_slots, status, tiles, n_tiles, hq, hd,
       y, xn, xa, xb, total;
 };
 
@@ -122,7 +122,6 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   L.status = take(4);
   L.tiles = take(prefill_tile_bytes((int)T, (int)K, (int)E, (int)S));
   L.n_tiles = take(4);
-  L.chunk_done = take((size_t)(H / 64 + 1) * 4);
   L.hq = take(rows * I);
   L.hd = take(rows * (I / 32) * 4);
   L.y = take(rows * H * 4);
@@ -180,17 +179,17 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
     return ev[i] ? cudaEventRecordWithFlags(ev[i], st, cudaEventRecordExternal) : cudaSuccess;
   };
 
-  if (T <= kDecodeMaxTok && (size_t)H * 8 <= 200 * 1024) {
-    // decode: 4 kernels, the last three launched with PDL
-    int32_t* chunk_done = at<int32_t>(ws, W.chunk_done);
+  int32_t* status = at<int32_t>(ws, W.status);
+  if (T <= kDecodeMaxTok && decode_supported(H, I)) {
+    // decode: 5 kernels, the last four launched with PDL
     CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, xq, xd, st));
     CHECK_LAUNCH(launch_topk_bucket_small(scores, L->bias, (int)T, E, K, c.norm_topk_prob, c.routed_scaling_factor,
                                           idx, wts, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm, inv,
-                                          slots, n_slots, chunk_done, H / 64, st));
+                                          slots, n_slots, st));
     CHECK_LAUNCH(mark(0));
-    CHECK_LAUNCH(launch_gateup_decode(gu, slots, n_slots, perm, (int)T, K, E, S, x, xq, xd, H, I, hq, hd, st));
+    CHECK_LAUNCH(launch_gateup_decode(gu, slots, n_slots, perm, (int)T, K, E, S, x, xq, xd, H, I, hq, hd, status, st));
     CHECK_LAUNCH(mark(1));
-    CHECK_LAUNCH(launch_down_combine(dn, slots, n_slots, (int)T, K, E, S, hq, hd, inv, wts, H, I, out, st));
+    CHECK_LAUNCH(launch_down_decode(dn, slots, n_slots, (int)T, K, E, S, hq, hd, inv, wts, H, I, y, out, status, st));
     CHECK_LAUNCH(mark(2));
     return COLI_OK;
   }

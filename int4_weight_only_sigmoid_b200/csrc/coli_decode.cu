@@ -2,38 +2,95 @@
 //
 //   router_decode (plain launch; also writes the Q8_0 of x)
 //     -> topk_bucket_small (PDL)
-//     -> gateup_stream (PDL): persistent; the shared experts' items do not
-//        depend on the routing and start at once, the routed items wait
-//     -> down_stream (PDL): persistent; down projection per (64-row chunk,
-//        expert) item, and the last item of each chunk combines the chunk
-//        into `out` (no separate combine kernel).
+//     -> gateup_ring (PDL): persistent 4-warp CTAs; items (expert slot, 64
+//        intermediate outputs), shared experts first: those do not depend on
+//        the routing and start while it runs
+//     -> down_ring (PDL): persistent, every warp on its own; items (expert
+//        slot, 32 output rows, group of <= TT tokens) -> y
+//     -> combine_decode (PDL): out = contract C over y
 //
-// Persistent streaming: a CTA of 4 warps walks a list of items (item i of
-// CTA c is c + i * gridDim.x, so the items of all CTAs are spread evenly);
-// every warp owns 16 weight rows of the current item and streams them
-// through a private ring of kRing steps (a step = 32 consecutive 16-byte
-// blocks of each of its 16 rows = 8 KB), filled by cp.async kRing - 1 steps
-// ahead, across item boundaries, so the weight stream does not drain between
-// items.  A lane copies exactly the 16-byte blocks it later reduces, so a
-// lane's own cp.async.wait_group is the only synchronisation the ring needs.
+// Weight streaming.  Every warp owns a ring of stages of 32 weight rows x 16
+// packed blocks (8 KB; one row per lane, rows 272 B apart so the lanes' reads
+// do not conflict).  The warp fills the stages with cp.async (each
+// instruction copies 256-byte pieces of two rows) one or two steps ahead of
+// the step it computes, across item boundaries, so the stream does not drain
+// between items.  The down kernel fetches a group's h rows with bulk copies
+// on an mbarrier; that wait is bounded (about a second): on expiry the CTA
+// raises its abort flag, records the error in the status word, runs on
+// without waiting (the output is then garbage) and, before it exits, waits
+// (bounded again) for the copies it still has in flight.
 //
-// The integer and float arithmetic is the same as coli_gemv.cu's (dp4a block
-// sums, contract F fold, SwiGLU, Q8_0 of h, contract C combine), so the
-// output is bit-identical to the general path.
+// Arithmetic: lane l holds weight row l; for each block in ascending order it
+// unpacks the 16 bytes once ((w << 4) & 0xF0F0F0F0 and w & 0xF0F0F0F0 are
+// 16*q of the even and odd elements as signed bytes), takes the dp4a block
+// sum against every staged token (even / odd byte planes, read as
+// broadcasts) and folds it into that token's chain (contract F).  SwiGLU,
+// the Q8_0 of h and the combine follow the same contracts as coli_gemv.cu,
+// so the output is bit-identical to the general path.
+//
+// The decode path stores h as "plane" rows: within every 32-element block the
+// 16 even elements come first, then the 16 odd ones, which is the layout the
+// down kernel's dot wants; only the decode kernels read it.
 //
 // Sources: "Colibri：在笔记本上跑744B参数的AI模型", "关键特性" (integer dot
 // kernels, Q8_0 activations); "GLM-5.2-colibri-int4架构解析…", "MoE的工作原理"
 // (weighted combine), "GLM-5.2的MoE实现" (shared expert); HN summary,
 // "已实现的功能" (batched MoE).
 #include "coli_gemv.cuh"
+#include "coli_tc.cuh"
+
 
 namespace coli {
 namespace {
 
 using namespace gemv;
 
-constexpr int kRing = 2;
-constexpr int kStepU4 = kRows * 32;  // uint4 per ring step of one warp
+constexpr int kBlkStep = 16;                     // packed blocks per row per step
+constexpr int kPitch = kBlkStep * 16 + 16;       // stage row pitch (B): rows on lanes read conflict-free
+constexpr int kPitchU4 = kPitch / 16;
+constexpr int kStageBytes = 32 * kPitch;         // 32 rows (one per lane)
+constexpr int kStageU4 = kStageBytes / 16;
+constexpr int kMaxWarpsDown = 8;
+
+// Ring depth: three stages for one token, two otherwise (more CTAs fit).
+template <int TT>
+__host__ __device__ constexpr int ring_depth() {
+  return TT == 1 ? 3 : 2;
+}
+constexpr int kSmemLimit = 227 * 1024;
+constexpr int kErrDownH = 22;  // status word: the down kernel gave up waiting for h rows
+
+// ---------------------------------------------------------------------------
+// bulk copies and mbarriers
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(tc::smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// global -> shared bulk copy completing on `bar` (addresses 16-byte aligned,
+// size a multiple of 16).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   tc::smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+// Wait (bounded, ignoring the abort flag) for a copy the kernel still has in
+// flight before it exits.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!tc::mbar_try_wait(bar, parity))
+    if (clock64() - t0 > tc::kSpinCycles) return;
+}
+
+// ---------------------------------------------------------------------------
+// token staging: xs[2*(t*nb + b)] / [.. + 1] = even / odd byte plane of block b
+// of staged token t; xsd[t*nb + b] = its Q8 scale.
 
 __device__ __forceinline__ Slot shared_slot(int s, int n_tok, int K, int E) {
   return Slot{E + s, n_tok * K + s * n_tok, n_tok, -1};
@@ -45,16 +102,24 @@ __device__ __forceinline__ Slot load_slot_dep(const Slot* p) {
   return Slot{(int32_t)v.x, (int32_t)v.y, (int32_t)v.z, (int32_t)v.w};
 }
 
-// Stage n_valid F32 token rows as Q8_0 (the same arithmetic as
-// quantize_act_q8_kernel: d = absmax/127, q = rint(x/d) in [-127,127]) into
-// even/odd byte planes + block scales.
-template <typename TokFn>
-__device__ __forceinline__ void stage_quantize_f32(const float* x, int dim, int n_valid, TokFn tok,
-                                                   uint4* xe_s, uint4* xo_s, float* xd_s) {
+template <int TT>
+__device__ __forceinline__ int pick(const int (&tok)[TT], int t) {
+  int row = tok[0];
+#pragma unroll
+  for (int j = 1; j < TT; ++j)
+    if (t == j) row = tok[j];
+  return row;
+}
+
+// Q8_0 of F32 token rows (the arithmetic of quantize_act_q8_kernel:
+// d = absmax/127, q = rint(x/d) in [-127,127]).
+template <int TT>
+__device__ __forceinline__ void stage_x_f32(const float* x, int dim, int n_valid, const int (&tok)[TT], uint4* xs,
+                                            float* xsd) {
   const int nb = dim / 32;
   for (int i = threadIdx.x; i < n_valid * nb; i += kThreads) {
     const int t = i / nb, b = i - t * nb;
-    const float4* src = reinterpret_cast<const float4*>(x + (int64_t)tok(t) * dim + 32 * b);
+    const float4* src = reinterpret_cast<const float4*>(x + (int64_t)pick<TT>(tok, t) * dim + 32 * b);
     float v[32];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -81,113 +146,132 @@ __device__ __forceinline__ void stage_quantize_f32(const float* x, int dim, int 
     split_even_odd(w[2], w[3], e.y, o.y);
     split_even_odd(w[4], w[5], e.z, o.z);
     split_even_odd(w[6], w[7], e.w, o.w);
-    xe_s[t * nb + b] = e;
-    xo_s[t * nb + b] = o;
-    xd_s[t * nb + b] = d;
+    xs[2 * (t * nb + b)] = e;
+    xs[2 * (t * nb + b) + 1] = o;
+    xsd[t * nb + b] = d;
   }
 }
 
+// The router kernel's Q8_0 rows of x, split into planes.
 template <int TT>
-struct StreamSmem {
-  __host__ __device__ static size_t ring_bytes() { return (size_t)kWarps * kRing * kStepU4 * 16; }
-  __host__ __device__ static size_t bytes(int dim_in) {
-    const int nb = dim_in / 32;
-    return ring_bytes() + (size_t)TT * nb * 36 + (size_t)kWarps * TT * kRows * kSPad * 4 + (size_t)TT * 32 * 4;
+__device__ __forceinline__ void stage_x_q8(const int8_t* xq, const float* xd, int dim, int n_valid,
+                                           const int (&tok)[TT], uint4* xs, float* xsd) {
+  const int nb = dim / 32;
+  for (int i = threadIdx.x; i < n_valid * nb; i += kThreads) {
+    const int t = i / nb, b = i - t * nb;
+    const int64_t row = pick<TT>(tok, t);
+    const uint4* src = reinterpret_cast<const uint4*>(xq + row * dim + 32 * b);
+    const uint4 a0 = ld_dep(src), a1 = ld_dep(src + 1);
+    uint4 e, o;
+    split_even_odd(a0.x, a0.y, e.x, o.x);
+    split_even_odd(a0.z, a0.w, e.y, o.y);
+    split_even_odd(a1.x, a1.y, e.z, o.z);
+    split_even_odd(a1.z, a1.w, e.w, o.w);
+    xs[2 * (t * nb + b)] = e;
+    xs[2 * (t * nb + b) + 1] = o;
+    xsd[t * nb + b] = ld_dep(xd + row * nb + b);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The dot: lane l holds weight row l of the stage and folds its blocks in
+// ascending order against every staged token (contract F), so no transpose
+// is needed and every lane works whatever the token count.
+
+// (float)i for |i| < 2^22, exactly: 1.5 * 2^23 + i is representable with unit
+// spacing, so building it from the bits and subtracting 1.5 * 2^23 is exact.
+__device__ __forceinline__ float i2f_exact(int i) {
+  return __fsub_rn(__int_as_float(0x4B400000 + i), 12582912.0f);
+}
+
+template <int TT>
+__device__ __forceinline__ void block_fold(const uint4 w, int b, int nb, int n_valid, const uint4* xs,
+                                           const float* xsd, float (&acc)[TT]) {
+  const int e0 = (int)((w.x << 4) & 0xF0F0F0F0u), o0 = (int)(w.x & 0xF0F0F0F0u);
+  const int e1 = (int)((w.y << 4) & 0xF0F0F0F0u), o1 = (int)(w.y & 0xF0F0F0F0u);
+  const int e2 = (int)((w.z << 4) & 0xF0F0F0F0u), o2 = (int)(w.z & 0xF0F0F0F0u);
+  const int e3 = (int)((w.w << 4) & 0xF0F0F0F0u), o3 = (int)(w.w & 0xF0F0F0F0u);
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    if (t < n_valid) {
+      const uint4 xe = xs[2 * (t * nb + b)], xo = xs[2 * (t * nb + b) + 1];
+      int se = __dp4a(e0, (int)xe.x, 0);
+      int so = __dp4a(o0, (int)xo.x, 0);
+      se = __dp4a(e1, (int)xe.y, se);
+      so = __dp4a(o1, (int)xo.y, so);
+      se = __dp4a(e2, (int)xe.z, se);
+      so = __dp4a(o2, (int)xo.z, so);
+      se = __dp4a(e3, (int)xe.w, se);
+      so = __dp4a(o3, (int)xo.w, so);
+      acc[t] = __fmaf_rn(xsd[t * nb + b], i2f_exact((se + so) >> 4), acc[t]);
+    }
+  }
+}
+
+// One ring stage: blocks b0 .. b0 + nblk - 1 of the lane's row.
+template <int TT>
+__device__ __forceinline__ void rows_step(const uint4* stage, int b0, int nblk, int nb, int n_valid, const uint4* xs,
+                                          const float* xsd, float (&acc)[TT]) {
+  const uint4* wrow = stage + (threadIdx.x & 31) * kPitchU4;
+  if (nblk == kBlkStep) {
+#pragma unroll
+    for (int j = 0; j < kBlkStep; ++j) block_fold<TT>(wrow[j], b0 + j, nb, n_valid, xs, xsd, acc);
+  } else {
+    for (int j = 0; j < nblk; ++j) block_fold<TT>(wrow[j], b0 + j, nb, n_valid, xs, xsd, acc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// gate/up + SwiGLU + Q8_0 of h
+
+template <int TT>
+struct GateUpSmem {
+  static constexpr int R = ring_depth<TT>();
+  __host__ __device__ static size_t ring() { return (size_t)kWarps * R * kStageBytes; }
+  __host__ __device__ static size_t xs(int nb) { return (size_t)TT * nb * 32; }
+  __host__ __device__ static size_t xsd(int nb) { return (size_t)TT * nb * 4; }
+  __host__ __device__ static size_t bytes(int hidden) {
+    const int nb = hidden / 32;
+    return ring() + xs(nb) + xsd(nb) + (size_t)TT * 64 * 4;
   }
 };
 
 struct Item {
-  int it;      // item index
+  int it;  // item index
   bool valid;
   Slot slot;
-  int r0;      // first output row of the item
+  int r0;      // first intermediate output of the item
   int groups;  // token groups of <= TT tokens
 };
 
-// Copy this lane's 16-byte block b of 16 rows (row0.. and row8.., rb bytes
-// apart) into ring slot rs; always commits one cp.async group.
-__device__ __forceinline__ void ring_fill(uint4* ring, int rs, const uint8_t* row0, const uint8_t* row8, size_t rb,
-                                          int b, int nb) {
-  const int lane = threadIdx.x & 31;
-  if (b < nb) {
-    uint4* dst = ring + rs * kStepU4 + lane;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) cp_async16(dst + r * 32, row0 + r * rb + 16 * b);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) cp_async16(dst + (8 + r) * 32, row8 + r * rb + 16 * b);
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// One step of the fold from the ring: isums of 16 rows x n_valid tokens
-// parked in shared memory, then each lane's chains (row c % 16, token
-// c / 16 + 2m) advance over the step's blocks in ascending order.
+// Items: (expert slot y, 64 intermediate outputs), slot-major, shared experts
+// first; warp w holds gate rows r0+16w..+15 on lanes 0..15 and the matching
+// up rows on lanes 16..31.  The staged tokens are kept while consecutive
+// groups use the same token list (a 1-token batch stages x once per CTA).
 template <int TT>
-__device__ __forceinline__ void ring_step(const uint4* ring, int rs, int s0, int nb, int n_valid, const uint4* xe_s,
-                                          const uint4* xo_s, const float* xd_s, int32_t* Sw,
-                                          float (&facc)[(TT + 1) / 2]) {
-  const int lane = threadIdx.x & 31;
-  const int cr = lane & 15, ct = lane >> 4;
-  const int b = s0 + lane;
-  const bool valid = b < nb;
-  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  uint4 wv[kRows];
-#pragma unroll
-  for (int r = 0; r < kRows; ++r) wv[r] = valid ? ring[rs * kStepU4 + r * 32 + lane] : zero;
-#pragma unroll
-  for (int t = 0; t < TT; ++t) {
-    if (t < n_valid) {
-      const uint4 xe = valid ? xe_s[t * nb + b] : zero;
-      const uint4 xo = valid ? xo_s[t * nb + b] : zero;
-#pragma unroll
-      for (int r = 0; r < kRows; ++r) Sw[(t * kRows + r) * kSPad + lane] = block_isum(wv[r], xe, xo);
-    }
-  }
-  __syncwarp();
-  const int nst = min(32, nb - s0);
-#pragma unroll
-  for (int m = 0; m < (TT + 1) / 2; ++m) {
-    const int t = ct + 2 * m;
-    if (t < n_valid && t < TT) {
-      const int32_t* srow = Sw + (t * kRows + cr) * kSPad;
-      const float* dsrc = xd_s + t * nb + s0;
-      float a = facc[m];
-      for (int j = 0; j < nst; ++j) a = __fmaf_rn(dsrc[j], (float)srow[j], a);
-      facc[m] = a;
-    }
-  }
-  __syncwarp();
-}
-
-// Gate/up + SwiGLU + Q8_0 of h.  Items: (expert slot y, 32 intermediate
-// outputs), slot-major, shared experts first (y < n_shared: no dependence on
-// the routing); warp w owns gate rows r0+8w..+7 and the matching up rows.
-template <int TT>
-__global__ void __launch_bounds__(kThreads) gateup_stream_kernel(
+__global__ void __launch_bounds__(kThreads) gateup_ring_kernel(
     const __grid_constant__ GateUpTable tbl, const Slot* slots, const int32_t* n_slots, const int32_t* perm, int n_tok,
-    int K, int E, int n_shared, int max_routed, const float* x, const int8_t* xq, const float* xd,
-    int hidden, int inter, int8_t* hq, float* hd) {
-  extern __shared__ __align__(16) unsigned char smem[];
+    int K, int E, int n_shared, int max_routed, const float* x, const int8_t* xq, const float* xd, int hidden,
+    int inter, int8_t* hq, float* hd) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  using SM = GateUpSmem<TT>;
+  constexpr int R = SM::R;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cr = lane & 15, ct = lane >> 4;
-  const int nb = hidden / 32, nsteps = (nb + 31) / 32;
-  const int nchunk = inter / 32;
+  const int nb = hidden / 32, nsteps = (nb + kBlkStep - 1) / kBlkStep;
+  const int nchunk = inter / 64;
   const int n_items = (n_shared + max_routed) * nchunk;
   const size_t rb = (size_t)hidden / 2;
-  uint4* ring = reinterpret_cast<uint4*>(smem) + warp * kRing * kStepU4;
-  uint4* xe_s = reinterpret_cast<uint4*>(smem) + kWarps * kRing * kStepU4;
-  uint4* xo_s = xe_s + TT * nb;
-  float* xd_s = reinterpret_cast<float*>(xo_s + TT * nb);
-  int32_t* Sp = reinterpret_cast<int32_t*>(xd_s + TT * nb);
-  float* Hs = reinterpret_cast<float*>(Sp + kWarps * TT * kRows * kSPad);
-  int32_t* Sw = Sp + warp * TT * kRows * kSPad;
+  uint4* ring = reinterpret_cast<uint4*>(smem) + warp * R * kStageU4;
+  uint4* xs = reinterpret_cast<uint4*>(smem + SM::ring());
+  float* xsd = reinterpret_cast<float*>(smem + SM::ring() + SM::xs(nb));
+  float* Hs = reinterpret_cast<float*>(smem + SM::ring() + SM::xs(nb) + SM::xsd(nb));
 
   bool waited = false;
   auto resolve = [&](Item& c) {
     c.valid = false;
     if (c.it >= n_items) return;
     const int yy = c.it / nchunk;
-    c.r0 = (c.it - yy * nchunk) * 32;
+    c.r0 = (c.it - yy * nchunk) * 64;
     if (yy < n_shared) {
       c.slot = shared_slot(yy, n_tok, K, E);
     } else {
@@ -209,66 +293,101 @@ __global__ void __launch_bounds__(kThreads) gateup_stream_kernel(
   resolve(cur);
   Item pf = cur;
   int pf_step = 0, g_pf = 0, g = 0;
+  // Copy the next step into ring slot g_pf % R: lane l copies block l & 15 of
+  // rows 2k + (l >> 4), k = 0..15 (two 256-byte row pieces per instruction);
+  // every call commits one cp.async group, empty at the end of the work.
   auto prefetch = [&]() {
-    if (pf.valid) {
-      const int st = pf_step % nsteps;
-      const int ti = pf.slot.table_idx;
-      ring_fill(ring, g_pf % kRing, tbl.gate_q[ti] + (size_t)(pf.r0 + 8 * warp) * rb,
-                tbl.up_q[ti] + (size_t)(pf.r0 + 8 * warp) * rb, rb, 32 * st + lane, nb);
-    } else {
+    if (!pf.valid) {
       asm volatile("cp.async.commit_group;" ::: "memory");
+      return;
     }
+    const int st = pf_step % nsteps;
+    const int s = g_pf % R;
+    const int ti = pf.slot.table_idx;
+    const int j = lane & 15, rsub = lane >> 4;
+    const size_t off = (size_t)(pf.r0 + 16 * warp) * rb + (size_t)kBlkStep * 16 * st + 16 * j;
+    const uint8_t* gb = tbl.gate_q[ti] + off;
+    const uint8_t* ub = tbl.up_q[ti] + off;
+    uint4* dst = ring + s * kStageU4 + j;
+    if (j < min(kBlkStep, nb - kBlkStep * st)) {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int r = 2 * k + rsub;
+        cp_async16(dst + r * kPitchU4, (k < 8 ? gb : ub) + (size_t)(r & 15) * rb);
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
     ++g_pf;
-    if (pf.valid && ++pf_step == pf.groups * nsteps) {
+    if (++pf_step == pf.groups * nsteps) {
       pf_step = 0;
       pf.it += gridDim.x;
       resolve(pf);
     }
   };
 #pragma unroll
-  for (int i = 0; i < kRing - 1; ++i) prefetch();
+  for (int i = 0; i < R - 1; ++i) prefetch();
+
+  int staged_n = -1;
+  int staged_tok[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) staged_tok[t] = -1;
 
   while (cur.valid) {
     const int ti = cur.slot.table_idx;
-    const int o_lane = cur.r0 + 8 * warp + (cr & 7);
-    const float s_lane = cr < 8 ? tbl.gate_s[ti][o_lane] : tbl.up_s[ti][o_lane];
+    const int o_lane = cur.r0 + 16 * warp + (lane & 15);
+    const float s_lane = lane < 16 ? tbl.gate_s[ti][o_lane] : tbl.up_s[ti][o_lane];
     const bool is_shared = cur.slot.perm_base < 0;
     for (int grp = 0; grp < cur.groups; ++grp) {
       const int g0 = grp * TT;
       const int n_valid = min(TT, cur.slot.count - g0);
-      __syncthreads();  // the previous group's staging and Hs are consumed
-      if (is_shared) {
-        stage_quantize_f32(x, hidden, n_valid, [=](int t) { return g0 + t; }, xe_s, xo_s, xd_s);
-      } else {
-        const int pb = cur.slot.perm_base;
-        stage_acts<TT>(xq, xd, hidden, n_valid, [=](int t) { return (int64_t)(ld_dep(perm + pb + g0 + t) / K); },
-                       xe_s, xo_s, xd_s);
-      }
-      __syncthreads();
-      float facc[(TT + 1) / 2];
+      int tok[TT];
+      bool same = n_valid == staged_n;
 #pragma unroll
-      for (int m = 0; m < (TT + 1) / 2; ++m) facc[m] = 0.0f;
+      for (int t = 0; t < TT; ++t) {
+        tok[t] = 0;
+        if (t < n_valid) {
+          tok[t] = is_shared ? g0 + t : (n_tok == 1 ? 0 : ld_dep(perm + cur.slot.perm_base + g0 + t) / K);
+          if (tok[t] != staged_tok[t]) same = false;
+        }
+      }
+      if (!same) {  // uniform over the CTA
+        __syncthreads();
+        if (is_shared)
+          stage_x_f32<TT>(x, hidden, n_valid, tok, xs, xsd);
+        else
+          stage_x_q8<TT>(xq, xd, hidden, n_valid, tok, xs, xsd);
+        __syncthreads();
+        staged_n = n_valid;
+#pragma unroll
+        for (int t = 0; t < TT; ++t) staged_tok[t] = tok[t];
+      }
+      float acc[TT];
+#pragma unroll
+      for (int t = 0; t < TT; ++t) acc[t] = 0.0f;
       for (int st = 0; st < nsteps; ++st, ++g) {
         prefetch();
-        asm volatile("cp.async.wait_group %0;" ::"n"(kRing - 1) : "memory");
-        ring_step<TT>(ring, g % kRing, 32 * st, nb, n_valid, xe_s, xo_s, xd_s, Sw, facc);
+        const int s = g % R;
+        asm volatile("cp.async.wait_group %0;" ::"n"(R - 1) : "memory");  // this lane's copies of step g
+        __syncwarp();                                                        // ... and every other lane's
+        rows_step<TT>(ring + s * kStageU4, kBlkStep * st, min(kBlkStep, nb - kBlkStep * st), nb, n_valid, xs, xsd,
+                      acc);
       }
 #pragma unroll
-      for (int m = 0; m < (TT + 1) / 2; ++m) {
-        const int t = ct + 2 * m;
-        const float val = __fmul_rn(s_lane, facc[m]);
-        const float u = __shfl_down_sync(0xffffffffu, val, 8);
-        if (cr < 8 && t < n_valid && t < TT)
-          Hs[t * 32 + 8 * warp + cr] = __fmul_rn(__fmul_rn(val, sigmoid_cw(val)), u);
+      for (int t = 0; t < TT; ++t) {
+        const float val = __fmul_rn(s_lane, acc[t]);
+        const float u = __shfl_down_sync(0xffffffffu, val, 16);
+        if (lane < 16 && t < n_valid) Hs[t * 64 + 16 * warp + lane] = __fmul_rn(__fmul_rn(val, sigmoid_cw(val)), u);
       }
       __syncthreads();
-      for (int t = warp; t < n_valid; t += kWarps) {
-        const float v = Hs[t * 32 + lane];
+      for (int p = warp; p < 2 * n_valid; p += kWarps) {
+        const int t = p >> 1, blk = p & 1;
+        const float v = Hs[t * 64 + 32 * blk + lane];
         const float d = __fdiv_rn(warp_max(fabsf(v)), 127.0f);
         const int64_t row = cur.slot.row_base + g0 + t;
-        hq[row * inter + cur.r0 + lane] = (int8_t)q8_of(v, d);
-        if (lane == 0) hd[row * (inter / 32) + (cur.r0 / 32)] = d;
+        hq[row * inter + cur.r0 + 32 * blk + (lane & 1) * 16 + (lane >> 1)] = (int8_t)q8_of(v, d);
+        if (lane == 0) hd[row * (inter / 32) + (cur.r0 / 32) + blk] = d;
       }
+      __syncthreads();
     }
     cur.it += gridDim.x;
     resolve(cur);
@@ -276,218 +395,286 @@ __global__ void __launch_bounds__(kThreads) gateup_stream_kernel(
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// Stage n_valid Q8 rows of h into one warp's even/odd planes (lane-strided,
-// warp-private staging).
-__device__ __forceinline__ void stage_rows_warp(const int8_t* aq, const float* ad, int dim_in, int64_t row0,
-                                                int n_valid, uint4* xe_s, uint4* xo_s, float* xd_s) {
-  const int nb = dim_in / 32;
-  const int lane = threadIdx.x & 31;
-  for (int i = lane; i < n_valid * nb; i += 32) {
-    const int t = i / nb, b = i - t * nb;
-    const int64_t row = row0 + t;
-    const uint4* src = reinterpret_cast<const uint4*>(aq + row * dim_in + 32 * b);
-    const uint4 a0 = ld_dep(src), a1 = ld_dep(src + 1);
-    uint4 e, o;
-    split_even_odd(a0.x, a0.y, e.x, o.x);
-    split_even_odd(a0.z, a0.w, e.y, o.y);
-    split_even_odd(a1.x, a1.y, e.z, o.z);
-    split_even_odd(a1.z, a1.w, e.w, o.w);
-    xe_s[t * nb + b] = e;
-    xo_s[t * nb + b] = o;
-    xd_s[t * nb + b] = ld_dep(ad + row * nb + b);
-  }
+// ---------------------------------------------------------------------------
+// down projection -> y
+
+// Token groups whose h rows can be in flight at once: the producer runs
+// R - 1 steps ahead and a group lasts nsteps steps.
+template <int TT>
+__host__ __device__ inline int down_h_buffers(int nsteps) {
+  constexpr int R = ring_depth<TT>();
+  const int n = (R - 2 + nsteps) / nsteps + 1;
+  return n < R ? n : R;
 }
 
+// Shared memory of the down kernel: a 128-byte header (the abort flag), then
+// per warp: ring, h mbarriers + group descriptors (256 B), h buffers.
+constexpr int kDownHeader = 128;
 template <int TT>
-struct DownSmem {
-  __host__ __device__ static size_t warp_bytes(int inter) {  // multiple of 16 B
-    const int nb = inter / 32;
-    return ((size_t)kRing * kStepU4 * 16 + (size_t)TT * nb * 36 + (size_t)TT * kRows * kSPad * 4 + 15) & ~size_t(15);
-  }
-  __host__ __device__ static size_t bytes(int inter, int n_tok, int K, int n_shared) {
-    return kWarps * warp_bytes(inter) + (size_t)(n_tok * K + n_tok * n_shared) * kRows * 4;
-  }
-};
+__host__ __device__ inline size_t down_warp_bytes(int inter) {
+  const int nb = inter / 32, nhb = down_h_buffers<TT>((nb + kBlkStep - 1) / kBlkStep);
+  return (size_t)ring_depth<TT>() * kStageBytes + 256 + (size_t)nhb * TT * (inter + nb * 4);
+}
 
-// Down projection + combine.  Items: 16-row chunks of the output; for its
-// item a warp takes expert slots w, w+4, ... (shared experts first) and
-// streams their 16 down rows through its ring; the y values of the chunk
-// land in shared memory by buffer row (perm position, or n_tok*K + s*n_tok
-// + t for shared expert s); then each (token, row) is combined in rank order
-// (contract C) and written to out.
+// Items: unit u = (slot u / n_chunks, 32-row chunk u % n_chunks) in slot-major
+// order, spread over all warps of the grid; in each, the slot's tokens in
+// groups of <= TT; lane l computes output row o0 + l.  The producer writes a
+// descriptor (table index, first h row, token count, first output row) for
+// every group it starts, and the consumer takes its work from those, so it
+// never waits on the slot table.
 template <int TT>
-__global__ void __launch_bounds__(kThreads) down_stream_kernel(
+__global__ void __launch_bounds__(kMaxWarpsDown * 32, 1) down_ring_kernel(
     const __grid_constant__ DownTable tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K, int E,
-    int n_shared, const int8_t* hq, const float* hd, const int32_t* inv, const float* w, int hidden, int inter,
-    float* __restrict__ out) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  pdl_wait();  // h (gate/up kernel) and the slot table are complete
+    int n_shared, const int8_t* hq, const float* hd, int hidden, int inter, float* y, int32_t* status) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  constexpr int R = ring_depth<TT>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cr = lane & 15, ct = lane >> 4;
-  const int nb = inter / 32, nsteps = (nb + 31) / 32;
-  const int n_total = n_shared + ld_dep(n_slots);
-  const int n_items = hidden / kRows;
+  const int W = blockDim.x >> 5;
+  const int nb = inter / 32, nsteps = (nb + kBlkStep - 1) / kBlkStep, nhb = down_h_buffers<TT>(nsteps);
+  const int n_chunks = hidden / 32;
   const size_t rb = (size_t)inter / 2;
-  unsigned char* wbase = smem + warp * DownSmem<TT>::warp_bytes(inter);
-  uint4* ring = reinterpret_cast<uint4*>(wbase);
-  uint4* xe_s = ring + kRing * kStepU4;
-  uint4* xo_s = xe_s + TT * nb;
-  float* xd_s = reinterpret_cast<float*>(xo_s + TT * nb);
-  int32_t* Sw = reinterpret_cast<int32_t*>(xd_s + TT * nb);
-  float* ys = reinterpret_cast<float*>(smem + kWarps * DownSmem<TT>::warp_bytes(inter));
+  unsigned char* base = smem + kDownHeader + (size_t)warp * down_warp_bytes<TT>(inter);
+  uint4* ring = reinterpret_cast<uint4*>(base);
+  uint64_t* hbar = reinterpret_cast<uint64_t*>(base + R * kStageBytes);
+  int4* desc = reinterpret_cast<int4*>(base + R * kStageBytes + 128);
+  int8_t* hbq = reinterpret_cast<int8_t*>(base + R * kStageBytes + 256);
+  float* hbd = reinterpret_cast<float*>(hbq + (size_t)nhb * TT * inter);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem);
 
-  auto slot_of = [&](int si) -> Slot {
-    return si < n_shared ? shared_slot(si, n_tok, K, E) : load_slot_dep(slots + si - n_shared);
-  };
-  // the warp's stream: items it = blockIdx.x + k*gridDim.x; in each, slots
-  // si = warp + 4j < n_total; in each, groups x steps
-  int pf_it = blockIdx.x, pf_si = warp, pf_step = 0, g_pf = 0;
-  Slot pf_slot = (pf_it < n_items && pf_si < n_total) ? slot_of(pf_si) : Slot{0, 0, 0, -1};
-  auto advance_pf = [&]() {  // to the next (slot, item) with work for this warp
-    pf_step = 0;
-    pf_si += kWarps;
-    while (pf_it < n_items && pf_si >= n_total) {
-      pf_it += gridDim.x;
-      pf_si = warp;
+  if (threadIdx.x == 0) *abort_flag = 0;
+  if (lane == 0) {
+    for (int s = 0; s < nhb; ++s) tc::mbar_init(hbar + s, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_wait();  // h (gate/up kernel) and the slot table are complete
+  pdl_launch_dependents();
+  const int n_total = n_shared + ld_dep(n_slots);
+  const int n_units = n_total * n_chunks;
+  const int GW = gridDim.x * W;
+
+  // producer state: unit, group, step; g_pf / h_pf count issued steps / groups.
+  // The weights go through cp.async (lane l copies block l & 15 of rows
+  // 2k + (l >> 4)); a group's h rows and scales through one bulk copy each,
+  // completing on the group's mbarrier.
+  int pu = blockIdx.x * W + warp, pgrp = 0, pngrp = 0, pstep = 0, g_pf = 0, h_pf = 0;
+  Slot ps{0, 0, 0, -1};
+  bool pvalid = false;
+  auto presolve = [&]() {
+    pvalid = pu < n_units;
+    if (!pvalid) {
+      if (lane == 0) desc[h_pf % nhb] = make_int4(0, 0, 0, 0);  // end of this warp's work
+      return;
     }
-    if (pf_it < n_items) pf_slot = slot_of(pf_si);
+    const int si = pu / n_chunks;
+    ps = si < n_shared ? shared_slot(si, n_tok, K, E) : load_slot_dep(slots + si - n_shared);
+    pngrp = (ps.count + TT - 1) / TT;
+    pgrp = 0;
+    pstep = 0;
   };
-  if (pf_it < n_items && pf_si >= n_total) advance_pf();
+  presolve();
   auto prefetch = [&]() {
-    if (pf_it < n_items) {
-      const int st = pf_step % nsteps;
-      const uint8_t* base = tbl.down_q[pf_slot.table_idx] + (size_t)(pf_it * kRows) * rb;
-      ring_fill(ring, g_pf % kRing, base, base + 8 * rb, rb, 32 * st + lane, nb);
-      if (++pf_step == ((pf_slot.count + TT - 1) / TT) * nsteps) advance_pf();
-    } else {
+    if (!pvalid || *abort_flag) {
       asm volatile("cp.async.commit_group;" ::: "memory");
+      return;
     }
-    ++g_pf;
-  };
+    const int o0 = (pu % n_chunks) * 32;
+    if (pstep == 0) {  // a new group: its descriptor and h rows
+      const int hb = h_pf % nhb;
+      const int nv = min(TT, ps.count - pgrp * TT);
+      const int64_t row0 = ps.row_base + pgrp * TT;
+      if (lane == 0) {
+        desc[hb] = make_int4(ps.table_idx, (int)row0, nv, o0);
+        mbar_expect_tx(hbar + hb, (uint32_t)(nv * (inter + nb * 4)));
+        bulk_g2s(hbq + (size_t)hb * TT * inter, hq + row0 * inter, (uint32_t)(nv * inter), hbar + hb);
+        bulk_g2s(hbd + (size_t)hb * TT * nb, hd + row0 * nb, (uint32_t)(nv * nb * 4), hbar + hb);
+      }
+      ++h_pf;
+    }
+    const int s = g_pf % R;
+    const int j = lane & 15, rsub = lane >> 4;
+    const uint8_t* b0p = tbl.down_q[ps.table_idx] + (size_t)o0 * rb + (size_t)kBlkStep * 16 * pstep + 16 * j;
+    uint4* dst = ring + s * kStageU4 + j;
+    if (j < min(kBlkStep, nb - kBlkStep * pstep)) {
 #pragma unroll
-  for (int i = 0; i < kRing - 1; ++i) prefetch();
-
-  int g = 0;
-  for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-    const int o0 = it * kRows;
-    for (int si = warp; si < n_total; si += kWarps) {
-      const Slot slot = slot_of(si);
-      const float s_lane = tbl.down_s[slot.table_idx][o0 + cr];
-      for (int g0 = 0; g0 < slot.count; g0 += TT) {
-        const int n_valid = min(TT, slot.count - g0);
-        stage_rows_warp(hq, hd, inter, (int64_t)slot.row_base + g0, n_valid, xe_s, xo_s, xd_s);
-        __syncwarp();
-        float facc[(TT + 1) / 2];
-#pragma unroll
-        for (int m = 0; m < (TT + 1) / 2; ++m) facc[m] = 0.0f;
-        for (int st = 0; st < nsteps; ++st, ++g) {
-          prefetch();
-          asm volatile("cp.async.wait_group %0;" ::"n"(kRing - 1) : "memory");
-          ring_step<TT>(ring, g % kRing, 32 * st, nb, n_valid, xe_s, xo_s, xd_s, Sw, facc);
-        }
-#pragma unroll
-        for (int m = 0; m < (TT + 1) / 2; ++m) {
-          const int t = ct + 2 * m;
-          if (t < n_valid && t < TT) ys[(slot.row_base + g0 + t) * kRows + cr] = __fmul_rn(s_lane, facc[m]);
-        }
-        __syncwarp();
+      for (int k = 0; k < 16; ++k) {
+        const int r = 2 * k + rsub;
+        cp_async16(dst + r * kPitchU4, b0p + (size_t)r * rb);
       }
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < n_tok * kRows; i += kThreads) {
-      const int t = i / kRows, r = i - t * kRows;
-      float acc = 0.0f;
-      for (int k = 0; k < K; ++k) acc = __fmaf_rn(ld_dep(w + t * K + k), ys[ld_dep(inv + t * K + k) * kRows + r], acc);
-      for (int s2 = 0; s2 < n_shared; ++s2) acc = __fadd_rn(acc, ys[(n_tok * K + s2 * n_tok + t) * kRows + r]);
-      out[(int64_t)t * hidden + o0 + r] = acc;
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    ++g_pf;
+    if (++pstep == nsteps) {
+      pstep = 0;
+      if (++pgrp == pngrp) {
+        pu += GW;
+        presolve();
+      }
     }
-    __syncthreads();
+  };
+#pragma unroll
+  for (int i = 0; i < R - 1; ++i) prefetch();
+
+  int g = 0, hc = 0, first_fail = -1;
+  for (;;) {
+    __syncwarp();
+    const int hb = hc % nhb;
+    const int4 dsc = desc[hb];
+    if (dsc.z == 0) break;
+    const int ti = dsc.x, row0 = dsc.y, nv = dsc.z, o0 = dsc.w;
+    const float s_lane = tbl.down_s[ti][o0 + lane];
+    if (!tc::mbar_wait(hbar + hb, (uint32_t)((hc / nhb) & 1), abort_flag, status, kErrDownH) && first_fail < 0)
+      first_fail = g;
+    ++hc;
+    const uint4* xs = reinterpret_cast<const uint4*>(hbq + (size_t)hb * TT * inter);
+    const float* xsd = hbd + (size_t)hb * TT * nb;
+    float acc[TT];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) acc[t] = 0.0f;
+    for (int st = 0; st < nsteps; ++st, ++g) {
+      prefetch();
+      const int s = g % R;
+      asm volatile("cp.async.wait_group %0;" ::"n"(R - 1) : "memory");  // this lane's copies of step g
+      __syncwarp();                                                        // ... and every other lane's
+      rows_step<TT>(ring + s * kStageU4, kBlkStep * st, min(kBlkStep, nb - kBlkStep * st), nb, nv, xs, xsd, acc);
+    }
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+      if (t < nv) y[(int64_t)(row0 + t) * hidden + o0 + lane] = __fmul_rn(s_lane, acc[t]);
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
+  if (first_fail >= 0)  // h copies this warp may still have in flight
+    for (int k = hc - 1; k < h_pf; ++k)
+      if (k >= 0) mbar_drain(hbar + k % nhb, (uint32_t)((k / nhb) & 1));
 }
 
-template <typename KernelT>
-cudaError_t allow_smem(KernelT* k, int& mask) {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (mask & (1 << (dev & 31))) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  if (e == cudaSuccess) mask |= 1 << (dev & 31);
-  return e;
+// out[t] = sum_k w[t,k] y[inv[t,k]] + sum_s y[shared row s of t] (contract C).
+__global__ void __launch_bounds__(256) combine_decode_kernel(const float* y, const int32_t* inv, const float* w,
+                                                             int n_tok, int K, int n_shared, int H,
+                                                             float* __restrict__ out) {
+  pdl_wait();
+  const int t = blockIdx.y;
+  const int o = blockIdx.x * blockDim.x + threadIdx.x;
+  if (o >= H) return;
+  float acc = 0.0f;
+  for (int k = 0; k < K; ++k) {
+    const int64_t j = ld_dep(inv + t * K + k);
+    acc = __fmaf_rn(ld_dep(w + t * K + k), ld_dep(y + j * H + o), acc);
+  }
+  for (int s = 0; s < n_shared; ++s)
+    acc = __fadd_rn(acc, ld_dep(y + ((int64_t)n_tok * K + (int64_t)s * n_tok + t) * H + o));
+  out[(int64_t)t * H + o] = acc;
 }
 
-// Resident CTAs of a persistent kernel on the current device (cached per
-// kernel instance and device).
+// ---------------------------------------------------------------------------
+// launchers
+
 template <typename KernelT>
-cudaError_t persistent_grid(KernelT* k, size_t smem, int (&cache)[64], int& ctas) {
+cudaError_t allow_smem(KernelT* k, size_t bytes, size_t (&granted)[64]) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (cache[dev] == 0) {
-    int sms = 0, per = 0;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k, kThreads, smem)) != cudaSuccess) return e;
-    cache[dev] = sms * (per > 0 ? per : 1);
-  }
-  ctas = cache[dev];
+  if (granted[dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) granted[dev] = bytes;
+  return e;
+}
+
+cudaError_t sm_count(int& sms) {
+  static int cache[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (cache[dev] == 0 && (e = cudaDeviceGetAttribute(&cache[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  sms = cache[dev];
   return cudaSuccess;
 }
 
 template <int TT>
-cudaError_t gateup_stream_tt(const GateUpTable& tbl, const Slot* slots, const int32_t* n_slots, const int32_t* perm,
-                             int n_tok, int K, int E, int n_shared, const float* x, const int8_t* xq, const float* xd,
-                             int hidden, int inter, int8_t* hq, float* hd, cudaStream_t st) {
-  static int mask = 0;
-  static int cache[64] = {};
-  cudaError_t e = allow_smem(gateup_stream_kernel<TT>, mask);
+cudaError_t gateup_ring_tt(const GateUpTable& tbl, const Slot* slots, const int32_t* n_slots, const int32_t* perm,
+                           int n_tok, int K, int E, int n_shared, const float* x, const int8_t* xq, const float* xd,
+                           int hidden, int inter, int8_t* hq, float* hd, int32_t* status, cudaStream_t st) {
+  static size_t granted[64] = {};
+  static int per_sm[64] = {};
+  const size_t smem = GateUpSmem<TT>::bytes(hidden);
+  cudaError_t e = allow_smem(gateup_ring_kernel<TT>, smem, granted);
   if (e != cudaSuccess) return e;
-  const size_t smem = StreamSmem<TT>::bytes(hidden);
-  int ctas = 0;
-  if ((e = persistent_grid(gateup_stream_kernel<TT>, smem, cache, ctas)) != cudaSuccess) return e;
+  int sms = 0, dev = 0;
+  if ((e = sm_count(sms)) != cudaSuccess || (e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (per_sm[dev] == 0) {
+    int per = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gateup_ring_kernel<TT>, kThreads, smem)) !=
+        cudaSuccess)
+      return e;
+    per_sm[dev] = per > 0 ? per : 1;
+  }
+  const int ctas = sms * per_sm[dev];
   const int max_routed = n_tok * K < E ? n_tok * K : E;
-  const int items = (n_shared + max_routed) * (inter / 32);
-  return launch_pdl(gateup_stream_kernel<TT>, dim3(items < ctas ? items : ctas), dim3(kThreads), smem, st, true,
-                    tbl, slots, n_slots, perm, n_tok, K, E, n_shared, max_routed, x, xq, xd, hidden, inter, hq, hd);
+  const int items = (n_shared + max_routed) * (inter / 64);
+  return launch_pdl(gateup_ring_kernel<TT>, dim3(items < ctas ? items : ctas), dim3(kThreads), smem, st, true, tbl,
+                    slots, n_slots, perm, n_tok, K, E, n_shared, max_routed, x, xq, xd, hidden, inter, hq, hd);
 }
 
 template <int TT>
-cudaError_t down_stream_tt(const DownTable& tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K, int E,
-                           int n_shared, const int8_t* hq, const float* hd, const int32_t* inv, const float* w,
-                           int hidden, int inter, float* out, cudaStream_t st) {
-  static int mask = 0;
-  static int cache[64] = {};
-  cudaError_t e = allow_smem(down_stream_kernel<TT>, mask);
+cudaError_t down_ring_tt(const DownTable& tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K, int E,
+                         int n_shared, const int8_t* hq, const float* hd, int hidden, int inter, float* y,
+                         int32_t* status, cudaStream_t st) {
+  static size_t granted[64] = {};
+  int sms = 0;
+  cudaError_t e = sm_count(sms);
   if (e != cudaSuccess) return e;
-  const size_t smem = DownSmem<TT>::bytes(inter, n_tok, K, n_shared);
-  int ctas = 0;
-  if ((e = persistent_grid(down_stream_kernel<TT>, DownSmem<TT>::bytes(inter, kDecodeMaxTok, kMaxTopK, kMaxShared), cache,
-                           ctas)) != cudaSuccess)
-    return e;
-  const int items = hidden / kRows;
-  return launch_pdl(down_stream_kernel<TT>, dim3(items < ctas ? items : ctas), dim3(kThreads), smem, st, true, tbl,
-                    slots, n_slots, n_tok, K, E, n_shared, hq, hd, inv, w, hidden, inter, out);
+  const size_t per_warp = down_warp_bytes<TT>(inter);
+  int W = (int)((kSmemLimit - kDownHeader) / per_warp);
+  if (W > kMaxWarpsDown) W = kMaxWarpsDown;
+  if (W < 1) return cudaErrorInvalidConfiguration;
+  const size_t smem = kDownHeader + per_warp * W;
+  if ((e = allow_smem(down_ring_kernel<TT>, smem, granted)) != cudaSuccess) return e;
+  const int max_units = (n_shared + (n_tok * K < E ? n_tok * K : E)) * (hidden / 32);
+  int ctas = sms;
+  if (ctas * W > max_units) ctas = (max_units + W - 1) / W;
+  return launch_pdl(down_ring_kernel<TT>, dim3(ctas), dim3(32 * W), smem, st, true, tbl, slots, n_slots, n_tok, K, E,
+                    n_shared, hq, hd, hidden, inter, y, status);
 }
 
 }  // namespace
 
+bool decode_supported(int hidden, int inter) {
+  if (hidden % 128 != 0 || inter % 128 != 0) return false;
+  return GateUpSmem<4>::bytes(hidden) <= (size_t)kSmemLimit &&
+         kDownHeader + down_warp_bytes<4>(inter) <= (size_t)kSmemLimit;
+}
+
 cudaError_t launch_gateup_decode(const GateUpTable& tbl, const Slot* slots, const int32_t* n_slots,
                                  const int32_t* perm, int n_tok, int K, int E, int n_shared, const float* x,
                                  const int8_t* xq, const float* xd, int hidden, int inter, int8_t* hq, float* hd,
-                                 cudaStream_t st) {
+                                 int32_t* status, cudaStream_t st) {
   if (n_tok <= 1)
-    return gateup_stream_tt<1>(tbl, slots, n_slots, perm, n_tok, K, E, n_shared, x, xq, xd, hidden, inter, hq, hd, st);
+    return gateup_ring_tt<1>(tbl, slots, n_slots, perm, n_tok, K, E, n_shared, x, xq, xd, hidden, inter, hq, hd,
+                             status, st);
   if (n_tok <= 2)
-    return gateup_stream_tt<2>(tbl, slots, n_slots, perm, n_tok, K, E, n_shared, x, xq, xd, hidden, inter, hq, hd, st);
-  return gateup_stream_tt<4>(tbl, slots, n_slots, perm, n_tok, K, E, n_shared, x, xq, xd, hidden, inter, hq, hd, st);
+    return gateup_ring_tt<2>(tbl, slots, n_slots, perm, n_tok, K, E, n_shared, x, xq, xd, hidden, inter, hq, hd,
+                             status, st);
+  return gateup_ring_tt<4>(tbl, slots, n_slots, perm, n_tok, K, E, n_shared, x, xq, xd, hidden, inter, hq, hd,
+                           status, st);
 }
 
-cudaError_t launch_down_combine(const DownTable& tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K,
-                                int E, int n_shared, const int8_t* hq, const float* hd, const int32_t* inv,
-                                const float* w, int hidden, int inter, float* out, cudaStream_t st) {
-  if (n_tok <= 1) return down_stream_tt<1>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, inv, w, hidden, inter, out, st);
-  if (n_tok <= 2) return down_stream_tt<2>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, inv, w, hidden, inter, out, st);
-  return down_stream_tt<4>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, inv, w, hidden, inter, out, st);
+cudaError_t launch_down_decode(const DownTable& tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K,
+                               int E, int n_shared, const int8_t* hq, const float* hd, const int32_t* inv,
+                               const float* w, int hidden, int inter, float* y, float* out, int32_t* status,
+                               cudaStream_t st) {
+  cudaError_t e;
+  if (n_tok <= 1)
+    e = down_ring_tt<1>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, hidden, inter, y, status, st);
+  else if (n_tok <= 2)
+    e = down_ring_tt<2>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, hidden, inter, y, status, st);
+  else
+    e = down_ring_tt<4>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, hidden, inter, y, status, st);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(combine_decode_kernel, dim3((hidden + 255) / 256, n_tok), dim3(256), 0, st, true, y, inv, w,
+                    n_tok, K, n_shared, hidden, out);
 }
 
 }  // namespace coli

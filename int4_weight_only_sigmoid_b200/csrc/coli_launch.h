@@ -11,7 +11,7 @@
 namespace coli {
 
 // Largest batch that takes the decode path (router_decode, topk_bucket_small,
-// gateup_decode, down_combine).
+// gate/up, down, combine in coli_decode.cu).
 constexpr int kDecodeMaxTok = 16;
 
 // Launch with programmatic stream serialisation (PDL) when `pdl` is set: the
@@ -51,8 +51,7 @@ cudaError_t launch_router_decode(const float* x, const float* w_router, int n_to
                                  int8_t* xq, float* xd, cudaStream_t st);
 cudaError_t launch_topk_bucket_small(const float* scores, const float* bias, int n_tok, int E, int K, int norm,
                                      float rsf, int32_t* idx, float* w, int32_t* counts, int32_t* offsets,
-                                     int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, int32_t* chunk_done,
-                                     int n_chunk, cudaStream_t st);
+                                     int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, cudaStream_t st);
 
 // Bucketing: counts, offsets, perm; optionally the inverse map (pair ->
 // position), the expert slot table (+ shared slots) and its length.
@@ -79,15 +78,18 @@ cudaError_t launch_down(const DownTable& tbl, const GemvSlots& sl, const int8_t*
 // experts only; shared expert s is implicit (rows n_tok*K + s*n_tok ..).
 // gate/up quantises the F32 x itself for the shared experts (which start
 // before the routing is done) and reads the router kernel's Q8 of x for the
-// routed ones; down computes 16-row chunks of every expert and combines them
-// into `out` in shared memory.
+// routed ones, and writes h as plane rows (per 32-block: 16 even elements,
+// then 16 odd); down writes y and a combine kernel reduces it into `out`.
+// Needs decode_supported(hidden, inter).
+bool decode_supported(int hidden, int inter);
 cudaError_t launch_gateup_decode(const GateUpTable& tbl, const Slot* slots, const int32_t* n_slots,
                                  const int32_t* perm, int n_tok, int K, int E, int n_shared, const float* x,
                                  const int8_t* xq, const float* xd, int hidden, int inter, int8_t* hq, float* hd,
-                                 cudaStream_t st);
-cudaError_t launch_down_combine(const DownTable& tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K,
-                                int E, int n_shared, const int8_t* hq, const float* hd, const int32_t* inv,
-                                const float* w, int hidden, int inter, float* out, cudaStream_t st);
+                                 int32_t* status, cudaStream_t st);
+cudaError_t launch_down_decode(const DownTable& tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K,
+                               int E, int n_shared, const int8_t* hq, const float* hd, const int32_t* inv,
+                               const float* w, int hidden, int inter, float* y, float* out, int32_t* status,
+                               cudaStream_t st);
 
 // Prefill expert kernels on the tensor cores (tcgen05): build the tile list
 // (<= 64 tokens of one slot per tile) from the slot table, then the gate/up

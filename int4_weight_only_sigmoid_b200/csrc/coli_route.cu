@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kSmallThreads) topk_bucket_small_kernel(
     const float* scores, const float* __restrict__ bias, int n_tok, int E, int K, int norm, float rsf,
     int32_t* __restrict__ idx_out, float* __restrict__ w_out, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv, Slot* __restrict__ slots,
-    int32_t* __restrict__ n_slots, int32_t* __restrict__ chunk_done, int n_chunk) {
+    int32_t* __restrict__ n_slots) {
   __shared__ int s_idx[kDecodeMaxTok * kMaxTopK];
   __shared__ int cnt[kMaxExperts];
   __shared__ int off[kMaxExperts];
@@ -212,7 +212,6 @@ __global__ void __launch_bounds__(kSmallThreads) topk_bucket_small_kernel(
   pdl_launch_dependents();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
-  for (int i = tid; i < n_chunk; i += blockDim.x) chunk_done[i] = 0;  // the down kernel's per-chunk counters
   if (warp < n_tok) {
     const float* st = scores + (size_t)warp * E;
     int sel[kMaxTopK];
@@ -397,10 +396,9 @@ cudaError_t launch_router_decode(const float* x, const float* w_router, int n_to
 
 cudaError_t launch_topk_bucket_small(const float* scores, const float* bias, int n_tok, int E, int K, int norm,
                                      float rsf, int32_t* idx, float* w, int32_t* counts, int32_t* offsets,
-                                     int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, int32_t* chunk_done,
-                                     int n_chunk, cudaStream_t st) {
+                                     int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, cudaStream_t st) {
   return launch_pdl(topk_bucket_small_kernel, dim3(1), dim3(kSmallThreads), 0, st, true, scores, bias, n_tok, E, K,
-                    norm, rsf, idx, w, counts, offsets, perm, inv, slots, n_slots, chunk_done, n_chunk);
+                    norm, rsf, idx, w, counts, offsets, perm, inv, slots, n_slots);
 }
 
 cudaError_t launch_bucket(const int32_t* idx, int n_tok, int K, int E, int n_shared, int32_t* counts,
