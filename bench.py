@@ -39,7 +39,7 @@ WORKLOAD = ("GLM-5.2-shaped MoE layer decode, 1 token (hidden 6144, expert inter
 N_LAYERS = 8
 N_TOK_POOL = 64
 GRAPH_STEPS = 64
-KERNELS_PER_STEP = 4  # decode path: router, top-k+bucket, gate/up, down+combine
+KERNELS_PER_STEP = 5  # decode path: router, top-k+bucket, gate/up, down+combine
 
 
 def parse():
@@ -572,7 +572,7 @@ def main():
                        "graph_steps": G, "mean_experts_streamed": mean_exp},
             "streamed_gbs": step_gbs,
             "streamed_frac_of_hbm": step_gbs / peak,
-            "roofline": {"bound": "hbm", "kernel": "gateup_decode_kernel", "achieved": gate_gbs, "peak": peak,
+            "roofline": {"bound": "hbm", "kernel": "gateup_ring_kernel<1>", "achieved": gate_gbs, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": gate_gbs / peak, "traffic": None,
                          "avg_launch_ms": gate_avg_ms,
                          "algorithmic_bytes_per_launch": gate_bytes / max(1, phase_n),

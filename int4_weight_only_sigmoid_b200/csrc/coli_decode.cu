@@ -10,8 +10,8 @@
 //     -> combine_decode (PDL): out = contract C over y
 //
 // Weight streaming.  Every warp owns a ring of stages of 32 weight rows x 16
-// packed blocks (8 KB; one row per lane, rows 272 B apart so the lanes' reads
-// do not conflict).  The warp fills the stages with cp.async (each
+// packed blocks (8 KB; one row per lane, blocks XOR-swizzled within a row so
+// the lanes' reads do not conflict).  The warp fills the stages with cp.async (each
 // instruction copies 256-byte pieces of two rows) one or two steps ahead of
 // the step it computes, across item boundaries, so the stream does not drain
 // between items.  The down kernel fetches a group's h rows with bulk copies
@@ -36,190 +36,16 @@
 // kernels, Q8_0 activations); "GLM-5.2-colibri-int4架构解析…", "MoE的工作原理"
 // (weighted combine), "GLM-5.2的MoE实现" (shared expert); HN summary,
 // "已实现的功能" (batched MoE).
-#include "coli_gemv.cuh"
-#include "coli_tc.cuh"
-
+#include "coli_stream.cuh"
 
 namespace coli {
 namespace {
 
 using namespace gemv;
+using namespace stream;
 
-constexpr int kBlkStep = 16;                     // packed blocks per row per step
-constexpr int kPitch = kBlkStep * 16 + 16;       // stage row pitch (B): rows on lanes read conflict-free
-constexpr int kPitchU4 = kPitch / 16;
-constexpr int kStageBytes = 32 * kPitch;         // 32 rows (one per lane)
-constexpr int kStageU4 = kStageBytes / 16;
 constexpr int kMaxWarpsDown = 8;
-
-// Ring depth: three stages for one token, two otherwise (more CTAs fit).
-template <int TT>
-__host__ __device__ constexpr int ring_depth() {
-  return TT == 1 ? 3 : 2;
-}
-constexpr int kSmemLimit = 227 * 1024;
 constexpr int kErrDownH = 22;  // status word: the down kernel gave up waiting for h rows
-
-// ---------------------------------------------------------------------------
-// bulk copies and mbarriers
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(tc::smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-// global -> shared bulk copy completing on `bar` (addresses 16-byte aligned,
-// size a multiple of 16).
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   tc::smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
-
-// Wait (bounded, ignoring the abort flag) for a copy the kernel still has in
-// flight before it exits.
-__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!tc::mbar_try_wait(bar, parity))
-    if (clock64() - t0 > tc::kSpinCycles) return;
-}
-
-// ---------------------------------------------------------------------------
-// token staging: xs[2*(t*nb + b)] / [.. + 1] = even / odd byte plane of block b
-// of staged token t; xsd[t*nb + b] = its Q8 scale.
-
-__device__ __forceinline__ Slot shared_slot(int s, int n_tok, int K, int E) {
-  return Slot{E + s, n_tok * K + s * n_tok, n_tok, -1};
-}
-
-// A slot-table entry written by the routing kernel (read through L2).
-__device__ __forceinline__ Slot load_slot_dep(const Slot* p) {
-  const uint4 v = ld_dep(reinterpret_cast<const uint4*>(p));
-  return Slot{(int32_t)v.x, (int32_t)v.y, (int32_t)v.z, (int32_t)v.w};
-}
-
-template <int TT>
-__device__ __forceinline__ int pick(const int (&tok)[TT], int t) {
-  int row = tok[0];
-#pragma unroll
-  for (int j = 1; j < TT; ++j)
-    if (t == j) row = tok[j];
-  return row;
-}
-
-// Q8_0 of F32 token rows (the arithmetic of quantize_act_q8_kernel:
-// d = absmax/127, q = rint(x/d) in [-127,127]).
-template <int TT>
-__device__ __forceinline__ void stage_x_f32(const float* x, int dim, int n_valid, const int (&tok)[TT], uint4* xs,
-                                            float* xsd) {
-  const int nb = dim / 32;
-  for (int i = threadIdx.x; i < n_valid * nb; i += kThreads) {
-    const int t = i / nb, b = i - t * nb;
-    const float4* src = reinterpret_cast<const float4*>(x + (int64_t)pick<TT>(tok, t) * dim + 32 * b);
-    float v[32];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 f = __ldcg(src + j);  // x may be a buffer an earlier kernel rewrote
-      v[4 * j] = f.x;
-      v[4 * j + 1] = f.y;
-      v[4 * j + 2] = f.z;
-      v[4 * j + 3] = f.w;
-    }
-    float amax = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
-    const float d = __fdiv_rn(amax, 127.0f);
-    uint32_t w[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) word |= ((uint32_t)q8_of(v[4 * k + j], d) & 0xFFu) << (8 * j);
-      w[k] = word;
-    }
-    uint4 e, o;
-    split_even_odd(w[0], w[1], e.x, o.x);
-    split_even_odd(w[2], w[3], e.y, o.y);
-    split_even_odd(w[4], w[5], e.z, o.z);
-    split_even_odd(w[6], w[7], e.w, o.w);
-    xs[2 * (t * nb + b)] = e;
-    xs[2 * (t * nb + b) + 1] = o;
-    xsd[t * nb + b] = d;
-  }
-}
-
-// The router kernel's Q8_0 rows of x, split into planes.
-template <int TT>
-__device__ __forceinline__ void stage_x_q8(const int8_t* xq, const float* xd, int dim, int n_valid,
-                                           const int (&tok)[TT], uint4* xs, float* xsd) {
-  const int nb = dim / 32;
-  for (int i = threadIdx.x; i < n_valid * nb; i += kThreads) {
-    const int t = i / nb, b = i - t * nb;
-    const int64_t row = pick<TT>(tok, t);
-    const uint4* src = reinterpret_cast<const uint4*>(xq + row * dim + 32 * b);
-    const uint4 a0 = ld_dep(src), a1 = ld_dep(src + 1);
-    uint4 e, o;
-    split_even_odd(a0.x, a0.y, e.x, o.x);
-    split_even_odd(a0.z, a0.w, e.y, o.y);
-    split_even_odd(a1.x, a1.y, e.z, o.z);
-    split_even_odd(a1.z, a1.w, e.w, o.w);
-    xs[2 * (t * nb + b)] = e;
-    xs[2 * (t * nb + b) + 1] = o;
-    xsd[t * nb + b] = ld_dep(xd + row * nb + b);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// The dot: lane l holds weight row l of the stage and folds its blocks in
-// ascending order against every staged token (contract F), so no transpose
-// is needed and every lane works whatever the token count.
-
-// (float)i for |i| < 2^22, exactly: 1.5 * 2^23 + i is representable with unit
-// spacing, so building it from the bits and subtracting 1.5 * 2^23 is exact.
-__device__ __forceinline__ float i2f_exact(int i) {
-  return __fsub_rn(__int_as_float(0x4B400000 + i), 12582912.0f);
-}
-
-template <int TT>
-__device__ __forceinline__ void block_fold(const uint4 w, int b, int nb, int n_valid, const uint4* xs,
-                                           const float* xsd, float (&acc)[TT]) {
-  const int e0 = (int)((w.x << 4) & 0xF0F0F0F0u), o0 = (int)(w.x & 0xF0F0F0F0u);
-  const int e1 = (int)((w.y << 4) & 0xF0F0F0F0u), o1 = (int)(w.y & 0xF0F0F0F0u);
-  const int e2 = (int)((w.z << 4) & 0xF0F0F0F0u), o2 = (int)(w.z & 0xF0F0F0F0u);
-  const int e3 = (int)((w.w << 4) & 0xF0F0F0F0u), o3 = (int)(w.w & 0xF0F0F0F0u);
-#pragma unroll
-  for (int t = 0; t < TT; ++t) {
-    if (t < n_valid) {
-      const uint4 xe = xs[2 * (t * nb + b)], xo = xs[2 * (t * nb + b) + 1];
-      int se = __dp4a(e0, (int)xe.x, 0);
-      int so = __dp4a(o0, (int)xo.x, 0);
-      se = __dp4a(e1, (int)xe.y, se);
-      so = __dp4a(o1, (int)xo.y, so);
-      se = __dp4a(e2, (int)xe.z, se);
-      so = __dp4a(o2, (int)xo.z, so);
-      se = __dp4a(e3, (int)xe.w, se);
-      so = __dp4a(o3, (int)xo.w, so);
-      acc[t] = __fmaf_rn(xsd[t * nb + b], i2f_exact((se + so) >> 4), acc[t]);
-    }
-  }
-}
-
-// One ring stage: blocks b0 .. b0 + nblk - 1 of the lane's row.
-template <int TT>
-__device__ __forceinline__ void rows_step(const uint4* stage, int b0, int nblk, int nb, int n_valid, const uint4* xs,
-                                          const float* xsd, float (&acc)[TT]) {
-  const uint4* wrow = stage + (threadIdx.x & 31) * kPitchU4;
-  if (nblk == kBlkStep) {
-#pragma unroll
-    for (int j = 0; j < kBlkStep; ++j) block_fold<TT>(wrow[j], b0 + j, nb, n_valid, xs, xsd, acc);
-  } else {
-    for (int j = 0; j < nblk; ++j) block_fold<TT>(wrow[j], b0 + j, nb, n_valid, xs, xsd, acc);
-  }
-}
 
 // ---------------------------------------------------------------------------
 // gate/up + SwiGLU + Q8_0 of h
@@ -249,7 +75,7 @@ struct Item {
 // up rows on lanes 16..31.  The staged tokens are kept while consecutive
 // groups use the same token list (a 1-token batch stages x once per CTA).
 template <int TT>
-__global__ void __launch_bounds__(kThreads) gateup_ring_kernel(
+__global__ void __launch_bounds__(kThreads, 3) gateup_ring_kernel(
     const __grid_constant__ GateUpTable tbl, const Slot* slots, const int32_t* n_slots, const int32_t* perm, int n_tok,
     int K, int E, int n_shared, int max_routed, const float* x, const int8_t* xq, const float* xd, int hidden,
     int inter, int8_t* hq, float* hd) {
@@ -308,12 +134,12 @@ __global__ void __launch_bounds__(kThreads) gateup_ring_kernel(
     const size_t off = (size_t)(pf.r0 + 16 * warp) * rb + (size_t)kBlkStep * 16 * st + 16 * j;
     const uint8_t* gb = tbl.gate_q[ti] + off;
     const uint8_t* ub = tbl.up_q[ti] + off;
-    uint4* dst = ring + s * kStageU4 + j;
+    uint4* dst = ring + s * kStageU4;
     if (j < min(kBlkStep, nb - kBlkStep * st)) {
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         const int r = 2 * k + rsub;
-        cp_async16(dst + r * kPitchU4, (k < 8 ? gb : ub) + (size_t)(r & 15) * rb);
+        cp_async16(dst + stage_slot(r, j), (k < 8 ? gb : ub) + (size_t)(r & 15) * rb);
       }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -494,12 +320,12 @@ __global__ void __launch_bounds__(kMaxWarpsDown * 32, 1) down_ring_kernel(
     const int s = g_pf % R;
     const int j = lane & 15, rsub = lane >> 4;
     const uint8_t* b0p = tbl.down_q[ps.table_idx] + (size_t)o0 * rb + (size_t)kBlkStep * 16 * pstep + 16 * j;
-    uint4* dst = ring + s * kStageU4 + j;
+    uint4* dst = ring + s * kStageU4;
     if (j < min(kBlkStep, nb - kBlkStep * pstep)) {
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         const int r = 2 * k + rsub;
-        cp_async16(dst + r * kPitchU4, b0p + (size_t)r * rb);
+        cp_async16(dst + stage_slot(r, j), b0p + (size_t)r * rb);
       }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
