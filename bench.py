@@ -39,7 +39,11 @@ WORKLOAD = ("GLM-5.2-shaped MoE layer decode, 1 token (hidden 6144, expert inter
 N_LAYERS = 8
 N_TOK_POOL = 64
 GRAPH_STEPS = 64
-KERNELS_PER_STEP = 5  # decode path: router, top-k+bucket, gate/up, down+combine
+KERNELS_PER_STEP = 5  # decode path: router, top-k+bucket, gate/up, down, combine
+# dram__bytes_read.sum + dram__bytes_write.sum of one gateup_ring_kernel<1>
+# launch, from one ncu capture of the GLM decode-1 layer; None once that kernel
+# changes.
+GATEUP_TRAFFIC_BYTES = 117.09e6
 
 
 def parse():
@@ -573,7 +577,7 @@ def main():
             "streamed_gbs": step_gbs,
             "streamed_frac_of_hbm": step_gbs / peak,
             "roofline": {"bound": "hbm", "kernel": "gateup_ring_kernel<1>", "achieved": gate_gbs, "peak": peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": gate_gbs / peak, "traffic": None,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": gate_gbs / peak, "traffic": GATEUP_TRAFFIC_BYTES,
                          "avg_launch_ms": gate_avg_ms,
                          "algorithmic_bytes_per_launch": gate_bytes / max(1, phase_n),
                          "down_kernel_avg_ms": down_ms / max(1, phase_n)},
