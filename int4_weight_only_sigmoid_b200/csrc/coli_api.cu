@@ -94,7 +94,7 @@ coli_status check_layer(const coli_moe_layer* L, const char* fn) {
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Workspace {
-  size_t xq, xd, scores, idx, w, counts, offsets, perm, inv, slots, n_slots, status, tiles, n_tiles, hq, hd,
+  size_t xq, xd, scores, idx, w, counts, offsets, perm, inv, slots, n_slots, status, tiles, n_tiles, hq, hd, xf, hf,
       y, xn, xa, xb, total;
 };
 
@@ -123,6 +123,8 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   L.tiles = take(prefill_tile_bytes((int)T, (int)K, (int)E, (int)S));
   L.n_tiles = take(4);
   L.hq = take(rows * I);
+  L.xf = take(T * H * 2);
+  L.hf = take(rows * I * 2);
   L.hd = take(rows * (I / 32) * 4);
   L.y = take(rows * H * 4);
   L.xn = take(T * H * 4);
@@ -208,10 +210,9 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   const int max_tok = (int)T;
   CHECK_LAUNCH(mark(0));
   if (prefill_supported(H, I)) {
-    const int max_tiles = (int)prefill_tiles_bound((int)T, K, E, S);
     CHECK_LAUNCH(launch_prefill_experts(gu, dn, slots, n_slots, at<void>(ws, W.tiles), at<int32_t>(ws, W.n_tiles),
-                                        max_tiles, perm, K, xq, xd, H, I, hq, hd, y, at<int32_t>(ws, W.status), st,
-                                        ev[1]));
+                                        perm, K, xq, xd, (int)T, H, I, at<void>(ws, W.xf), at<void>(ws, W.hf), hd, y,
+                                        at<int32_t>(ws, W.status), st, ev[1]));
   } else {
     CHECK_LAUNCH(launch_gateup(gu, sl, xq, xd, H, I, max_tok, hq, hd, st));
     CHECK_LAUNCH(mark(1));

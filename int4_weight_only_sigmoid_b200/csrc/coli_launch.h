@@ -91,17 +91,19 @@ cudaError_t launch_down_decode(const DownTable& tbl, const Slot* slots, const in
                                const float* w, int hidden, int inter, float* y, float* out, int32_t* status,
                                cudaStream_t st);
 
-// Prefill expert kernels on the tensor cores (tcgen05): build the tile list
-// (<= 64 tokens of one slot per tile) from the slot table, then the gate/up
-// GEMM (+ SwiGLU + Q8 of h) and the down GEMM (-> y).  `tiles` needs
-// prefill_tile_bytes(); grids are sized by prefill_tiles_bound().
+// Prefill expert kernels on the tensor cores (tcgen05): the fp16 operand
+// rows of the Q8 activations (xf: n_tok x hidden halves), the tile list
+// (<= 64 tokens of one slot per tile) built from the slot table, then the
+// persistent gate/up GEMM (+ SwiGLU + Q8 of h, written as fp16 rows hf:
+// rows x inter halves, scales hd) and the persistent down GEMM (-> y).
+// `tiles` needs prefill_tile_bytes().
 bool prefill_supported(int hidden, int inter);
 size_t prefill_tiles_bound(int n_tok, int K, int E, int n_shared);
 size_t prefill_tile_bytes(int n_tok, int K, int E, int n_shared);
 cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, const Slot* slots,
-                                   const int32_t* n_slots, void* tiles, int32_t* n_tiles, int max_tiles,
-                                   const int32_t* perm, int K, const int8_t* xq, const float* xd, int hidden,
-                                   int inter, int8_t* hq, float* hd, float* y, int32_t* err, cudaStream_t st,
+                                   const int32_t* n_slots, void* tiles, int32_t* n_tiles, const int32_t* perm,
+                                   int K, const int8_t* xq, const float* xd, int n_tok, int hidden, int inter,
+                                   void* xf, void* hf, float* hd, float* y, int32_t* err, cudaStream_t st,
                                    cudaEvent_t ev_mid);
 
 // out[t] = sum_k w[t,k] y[inv[t,k]] + sum_s y[n_tok*K + s*n_tok + t]  (contract C)
