@@ -5,8 +5,8 @@
 //     -> gateup_ring (PDL): persistent 4-warp CTAs; items (expert slot, 64
 //        intermediate outputs), shared experts first: those do not depend on
 //        the routing and start while it runs
-//     -> down_ring (PDL): persistent, every warp on its own; items (expert
-//        slot, 32 output rows, group of <= TT tokens) -> y
+//     -> down_cta (PDL): persistent; items (expert slot, 32*W output rows)
+//        for a W-warp CTA, token groups of <= TT -> y
 //     -> combine_decode (PDL): out = contract C over y
 //
 // Weight streaming.  Every warp owns a ring of stages of 32 weight rows x 16
@@ -14,11 +14,11 @@
 // the lanes' reads do not conflict).  The warp fills the stages with cp.async (each
 // instruction copies 256-byte pieces of two rows) one or two steps ahead of
 // the step it computes, across item boundaries, so the stream does not drain
-// between items.  The down kernel fetches a group's h rows with bulk copies
-// on an mbarrier; that wait is bounded (about a second): on expiry the CTA
-// raises its abort flag, records the error in the status word, runs on
-// without waiting (the output is then garbage) and, before it exits, waits
-// (bounded again) for the copies it still has in flight.
+// between items.  The down kernel fetches a group's h rows once per CTA with
+// bulk copies on an mbarrier; that wait is bounded (about a second): on
+// expiry the CTA raises its abort flag, records the error in the status
+// word, runs on without waiting (the output is then garbage) and, before it
+// exits, waits (bounded again) for the copies it still has in flight.
 //
 // Arithmetic: lane l holds weight row l; for each block in ascending order it
 // unpacks the 16 bytes once ((w << 4) & 0xF0F0F0F0 and w & 0xF0F0F0F0 are
@@ -44,7 +44,7 @@ namespace {
 using namespace gemv;
 using namespace stream;
 
-constexpr int kMaxWarpsDown = 8;
+constexpr int kMaxWarpsDown = 12;
 constexpr int kErrDownH = 22;  // status word: the down kernel gave up waiting for h rows
 
 // ---------------------------------------------------------------------------
@@ -224,103 +224,98 @@ __global__ void __launch_bounds__(kThreads, 3) gateup_ring_kernel(
 // ---------------------------------------------------------------------------
 // down projection -> y
 
-// Token groups whose h rows can be in flight at once: the producer runs
-// R - 1 steps ahead and a group lasts nsteps steps.
-template <int TT>
-__host__ __device__ inline int down_h_buffers(int nsteps) {
-  constexpr int R = ring_depth<TT>();
-  const int n = (R - 2 + nsteps) / nsteps + 1;
-  return n < R ? n : R;
-}
-
-// Shared memory of the down kernel: a 128-byte header (the abort flag), then
-// per warp: ring, h mbarriers + group descriptors (256 B), h buffers.
+// Shared memory of the down kernel: a 128-byte header (abort flag, two h
+// mbarriers), two h buffers of one token group each, then one ring per warp.
 constexpr int kDownHeader = 128;
 template <int TT>
-__host__ __device__ inline size_t down_warp_bytes(int inter) {
-  const int nb = inter / 32, nhb = down_h_buffers<TT>((nb + kBlkStep - 1) / kBlkStep);
-  return (size_t)ring_depth<TT>() * kStageBytes + 256 + (size_t)nhb * TT * (inter + nb * 4);
+__host__ __device__ inline size_t down_hbuf_bytes(int inter) {
+  return (size_t)TT * (inter + (inter / 32) * 4);
+}
+template <int TT>
+__host__ __device__ inline size_t down_cta_bytes(int inter, int W) {
+  return kDownHeader + 2 * down_hbuf_bytes<TT>(inter) + (size_t)W * ring_depth<TT>() * kStageBytes;
 }
 
-// Items: unit u = (slot u / n_chunks, 32-row chunk u % n_chunks) in slot-major
-// order, spread over all warps of the grid; in each, the slot's tokens in
-// groups of <= TT; lane l computes output row o0 + l.  The producer writes a
-// descriptor (table index, first h row, token count, first output row) for
-// every group it starts, and the consumer takes its work from those, so it
-// never waits on the slot table.
+// Items: (expert slot, 32*W consecutive output rows), slot-major, shared
+// experts first; the W warps of a CTA take 32 rows each of the same slot, so
+// the slot's h rows are fetched once per CTA (bulk copies on an mbarrier,
+// double-buffered by token group).  Lane l computes output row o0 + l.  A
+// CTA walks its units (item, token group) in order; thread 0 fetches the
+// next unit's h rows while the current one computes, and a CTA barrier ends
+// every unit, so a buffer is refilled only after all warps are done with it.
 template <int TT>
-__global__ void __launch_bounds__(kMaxWarpsDown * 32, 1) down_ring_kernel(
+__global__ void __launch_bounds__(kMaxWarpsDown * 32, 1) down_cta_kernel(
     const __grid_constant__ DownTable tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K, int E,
     int n_shared, const int8_t* hq, const float* hd, int hidden, int inter, float* y, int32_t* status) {
   extern __shared__ __align__(1024) unsigned char smem[];
   constexpr int R = ring_depth<TT>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int W = blockDim.x >> 5;
-  const int nb = inter / 32, nsteps = (nb + kBlkStep - 1) / kBlkStep, nhb = down_h_buffers<TT>(nsteps);
-  const int n_chunks = hidden / 32;
+  const int nb = inter / 32, nsteps = (nb + kBlkStep - 1) / kBlkStep;
+  const int per_slot = hidden / (32 * W);
   const size_t rb = (size_t)inter / 2;
-  unsigned char* base = smem + kDownHeader + (size_t)warp * down_warp_bytes<TT>(inter);
-  uint4* ring = reinterpret_cast<uint4*>(base);
-  uint64_t* hbar = reinterpret_cast<uint64_t*>(base + R * kStageBytes);
-  int4* desc = reinterpret_cast<int4*>(base + R * kStageBytes + 128);
-  int8_t* hbq = reinterpret_cast<int8_t*>(base + R * kStageBytes + 256);
-  float* hbd = reinterpret_cast<float*>(hbq + (size_t)nhb * TT * inter);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem);
+  uint64_t* hbar = reinterpret_cast<uint64_t*>(smem + 64);
+  unsigned char* hbuf = smem + kDownHeader;
+  const size_t hb_bytes = down_hbuf_bytes<TT>(inter);
+  uint4* ring = reinterpret_cast<uint4*>(smem + kDownHeader + 2 * hb_bytes) + (size_t)warp * R * kStageU4;
 
-  if (threadIdx.x == 0) *abort_flag = 0;
-  if (lane == 0) {
-    for (int s = 0; s < nhb; ++s) tc::mbar_init(hbar + s, 1);
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    tc::mbar_init(hbar, 1);
+    tc::mbar_init(hbar + 1, 1);
     fence_mbar_init();
   }
   __syncthreads();
   pdl_wait();  // h (gate/up kernel) and the slot table are complete
   pdl_launch_dependents();
   const int n_total = n_shared + ld_dep(n_slots);
-  const int n_units = n_total * n_chunks;
-  const int GW = gridDim.x * W;
+  const int n_items = n_total * per_slot;
 
-  // producer state: unit, group, step; g_pf / h_pf count issued steps / groups.
-  // The weights go through cp.async (lane l copies block l & 15 of rows
-  // 2k + (l >> 4)); a group's h rows and scales through one bulk copy each,
-  // completing on the group's mbarrier.
-  int pu = blockIdx.x * W + warp, pgrp = 0, pngrp = 0, pstep = 0, g_pf = 0, h_pf = 0;
-  Slot ps{0, 0, 0, -1};
-  bool pvalid = false;
-  auto presolve = [&]() {
-    pvalid = pu < n_units;
-    if (!pvalid) {
-      if (lane == 0) desc[h_pf % nhb] = make_int4(0, 0, 0, 0);  // end of this warp's work
-      return;
-    }
-    const int si = pu / n_chunks;
-    ps = si < n_shared ? shared_slot(si, n_tok, K, E) : load_slot_dep(slots + si - n_shared);
-    pngrp = (ps.count + TT - 1) / TT;
-    pgrp = 0;
-    pstep = 0;
+  // a unit iterator (item, group); every thread walks the same sequence
+  struct Unit {
+    int it, grp, ngrp;
+    Slot slot;
+    bool valid;
   };
-  presolve();
+  auto resolve = [&](Unit& u) {
+    u.valid = u.it < n_items;
+    if (!u.valid) return;
+    const int si = u.it / per_slot;
+    u.slot = si < n_shared ? shared_slot(si, n_tok, K, E) : load_slot_dep(slots + si - n_shared);
+    u.ngrp = (u.slot.count + TT - 1) / TT;
+    u.grp = 0;
+  };
+  auto advance = [&](Unit& u) {
+    if (++u.grp == u.ngrp) {
+      u.it += gridDim.x;
+      resolve(u);
+    }
+  };
+  // thread 0: the h rows of unit k into buffer k & 1
+  auto fetch_h = [&](const Unit& u, int k) {
+    const int nv = min(TT, u.slot.count - u.grp * TT);
+    const int64_t row0 = u.slot.row_base + u.grp * TT;
+    unsigned char* dst = hbuf + (size_t)(k & 1) * hb_bytes;
+    mbar_expect_tx(hbar + (k & 1), (uint32_t)(nv * (inter + nb * 4)));
+    bulk_g2s(dst, hq + row0 * inter, (uint32_t)(nv * inter), hbar + (k & 1));
+    bulk_g2s(dst + (size_t)TT * inter, hd + row0 * nb, (uint32_t)(nv * nb * 4), hbar + (k & 1));
+  };
+
+  // producer (per warp): the weights of the warp's 32 rows, step by step
+  Unit pu;
+  pu.it = blockIdx.x;
+  resolve(pu);
+  int pstep = 0, g_pf = 0;
   auto prefetch = [&]() {
-    if (!pvalid || *abort_flag) {
+    if (!pu.valid || *abort_flag) {
       asm volatile("cp.async.commit_group;" ::: "memory");
       return;
     }
-    const int o0 = (pu % n_chunks) * 32;
-    if (pstep == 0) {  // a new group: its descriptor and h rows
-      const int hb = h_pf % nhb;
-      const int nv = min(TT, ps.count - pgrp * TT);
-      const int64_t row0 = ps.row_base + pgrp * TT;
-      if (lane == 0) {
-        desc[hb] = make_int4(ps.table_idx, (int)row0, nv, o0);
-        mbar_expect_tx(hbar + hb, (uint32_t)(nv * (inter + nb * 4)));
-        bulk_g2s(hbq + (size_t)hb * TT * inter, hq + row0 * inter, (uint32_t)(nv * inter), hbar + hb);
-        bulk_g2s(hbd + (size_t)hb * TT * nb, hd + row0 * nb, (uint32_t)(nv * nb * 4), hbar + hb);
-      }
-      ++h_pf;
-    }
-    const int s = g_pf % R;
+    const int o0 = (pu.it % per_slot) * 32 * W + 32 * warp;
     const int j = lane & 15, rsub = lane >> 4;
-    const uint8_t* b0p = tbl.down_q[ps.table_idx] + (size_t)o0 * rb + (size_t)kBlkStep * 16 * pstep + 16 * j;
-    uint4* dst = ring + s * kStageU4;
+    const uint8_t* b0p = tbl.down_q[pu.slot.table_idx] + (size_t)o0 * rb + (size_t)kBlkStep * 16 * pstep + 16 * j;
+    uint4* dst = ring + (g_pf % R) * kStageU4;
     if (j < min(kBlkStep, nb - kBlkStep * pstep)) {
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
@@ -332,46 +327,51 @@ __global__ void __launch_bounds__(kMaxWarpsDown * 32, 1) down_ring_kernel(
     ++g_pf;
     if (++pstep == nsteps) {
       pstep = 0;
-      if (++pgrp == pngrp) {
-        pu += GW;
-        presolve();
-      }
+      advance(pu);
     }
   };
+
+  Unit cu;
+  cu.it = blockIdx.x;
+  resolve(cu);
+  Unit hu = cu;  // thread 0's fetch iterator, one unit ahead of cu
+  if (threadIdx.x == 0 && hu.valid) fetch_h(hu, 0);
 #pragma unroll
   for (int i = 0; i < R - 1; ++i) prefetch();
 
-  int g = 0, hc = 0, first_fail = -1;
-  for (;;) {
-    __syncwarp();
-    const int hb = hc % nhb;
-    const int4 dsc = desc[hb];
-    if (dsc.z == 0) break;
-    const int ti = dsc.x, row0 = dsc.y, nv = dsc.z, o0 = dsc.w;
-    const float s_lane = tbl.down_s[ti][o0 + lane];
-    if (!tc::mbar_wait(hbar + hb, (uint32_t)((hc / nhb) & 1), abort_flag, status, kErrDownH) && first_fail < 0)
-      first_fail = g;
-    ++hc;
-    const uint4* xs = reinterpret_cast<const uint4*>(hbq + (size_t)hb * TT * inter);
-    const float* xsd = hbd + (size_t)hb * TT * nb;
+  int g = 0, k = 0, first_fail = -1;
+  for (; cu.valid; ++k) {
+    if (threadIdx.x == 0) {  // the next unit's h rows into the other buffer (free since the last barrier)
+      advance(hu);
+      if (hu.valid) fetch_h(hu, k + 1);
+    }
+    if (!tc::mbar_wait(hbar + (k & 1), (uint32_t)((k >> 1) & 1), abort_flag, status, kErrDownH) && first_fail < 0)
+      first_fail = k;
+    const int nv = min(TT, cu.slot.count - cu.grp * TT);
+    const int64_t row0 = cu.slot.row_base + cu.grp * TT;
+    const int o = (cu.it % per_slot) * 32 * W + 32 * warp + lane;
+    const float s_lane = tbl.down_s[cu.slot.table_idx][o];
+    const uint4* xs = reinterpret_cast<const uint4*>(hbuf + (size_t)(k & 1) * hb_bytes);
+    const float* xsd = reinterpret_cast<const float*>(hbuf + (size_t)(k & 1) * hb_bytes + (size_t)TT * inter);
     float acc[TT];
 #pragma unroll
     for (int t = 0; t < TT; ++t) acc[t] = 0.0f;
     for (int st = 0; st < nsteps; ++st, ++g) {
       prefetch();
-      const int s = g % R;
       asm volatile("cp.async.wait_group %0;" ::"n"(R - 1) : "memory");  // this lane's copies of step g
       __syncwarp();                                                        // ... and every other lane's
-      rows_step<TT>(ring + s * kStageU4, kBlkStep * st, min(kBlkStep, nb - kBlkStep * st), nb, nv, xs, xsd, acc);
+      rows_step<TT>(ring + (g % R) * kStageU4, kBlkStep * st, min(kBlkStep, nb - kBlkStep * st), nb, nv, xs, xsd,
+                    acc);
     }
 #pragma unroll
     for (int t = 0; t < TT; ++t)
-      if (t < nv) y[(int64_t)(row0 + t) * hidden + o0 + lane] = __fmul_rn(s_lane, acc[t]);
+      if (t < nv) y[(row0 + t) * hidden + o] = __fmul_rn(s_lane, acc[t]);
+    advance(cu);
+    __syncthreads();  // every warp is done with h buffer k & 1
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
-  if (first_fail >= 0)  // h copies this warp may still have in flight
-    for (int k = hc - 1; k < h_pf; ++k)
-      if (k >= 0) mbar_drain(hbar + k % nhb, (uint32_t)((k / nhb) & 1));
+  if (threadIdx.x == 0 && first_fail >= 0)  // h copies that may still be in flight
+    for (int kk = first_fail; kk <= k; ++kk) mbar_drain(hbar + (kk & 1), (uint32_t)((kk >> 1) & 1));
 }
 
 // out[t] = sum_k w[t,k] y[inv[t,k]] + sum_s y[shared row s of t] (contract C).
@@ -444,24 +444,30 @@ cudaError_t gateup_ring_tt(const GateUpTable& tbl, const Slot* slots, const int3
                     slots, n_slots, perm, n_tok, K, E, n_shared, max_routed, x, xq, xd, hidden, inter, hq, hd);
 }
 
+// Warps per down CTA: the largest W <= kMaxWarpsDown that fits shared
+// memory and divides hidden into 32*W-row items.
 template <int TT>
-cudaError_t down_ring_tt(const DownTable& tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K, int E,
-                         int n_shared, const int8_t* hq, const float* hd, int hidden, int inter, float* y,
-                         int32_t* status, cudaStream_t st) {
+int down_warps(int hidden, int inter) {
+  for (int W = kMaxWarpsDown; W >= 1; --W)
+    if (hidden % (32 * W) == 0 && down_cta_bytes<TT>(inter, W) <= (size_t)kSmemLimit) return W;
+  return 0;
+}
+
+template <int TT>
+cudaError_t down_cta_tt(const DownTable& tbl, const Slot* slots, const int32_t* n_slots, int n_tok, int K, int E,
+                        int n_shared, const int8_t* hq, const float* hd, int hidden, int inter, float* y,
+                        int32_t* status, cudaStream_t st) {
   static size_t granted[64] = {};
   int sms = 0;
   cudaError_t e = sm_count(sms);
   if (e != cudaSuccess) return e;
-  const size_t per_warp = down_warp_bytes<TT>(inter);
-  int W = (int)((kSmemLimit - kDownHeader) / per_warp);
-  if (W > kMaxWarpsDown) W = kMaxWarpsDown;
+  const int W = down_warps<TT>(hidden, inter);
   if (W < 1) return cudaErrorInvalidConfiguration;
-  const size_t smem = kDownHeader + per_warp * W;
-  if ((e = allow_smem(down_ring_kernel<TT>, smem, granted)) != cudaSuccess) return e;
-  const int max_units = (n_shared + (n_tok * K < E ? n_tok * K : E)) * (hidden / 32);
-  int ctas = sms;
-  if (ctas * W > max_units) ctas = (max_units + W - 1) / W;
-  return launch_pdl(down_ring_kernel<TT>, dim3(ctas), dim3(32 * W), smem, st, true, tbl, slots, n_slots, n_tok, K, E,
+  const size_t smem = down_cta_bytes<TT>(inter, W);
+  if ((e = allow_smem(down_cta_kernel<TT>, smem, granted)) != cudaSuccess) return e;
+  const int max_items = (n_shared + (n_tok * K < E ? n_tok * K : E)) * (hidden / (32 * W));
+  const int ctas = max_items < sms ? max_items : sms;
+  return launch_pdl(down_cta_kernel<TT>, dim3(ctas), dim3(32 * W), smem, st, true, tbl, slots, n_slots, n_tok, K, E,
                     n_shared, hq, hd, hidden, inter, y, status);
 }
 
@@ -469,8 +475,7 @@ cudaError_t down_ring_tt(const DownTable& tbl, const Slot* slots, const int32_t*
 
 bool decode_supported(int hidden, int inter) {
   if (hidden % 128 != 0 || inter % 128 != 0) return false;
-  return GateUpSmem<4>::bytes(hidden) <= (size_t)kSmemLimit &&
-         kDownHeader + down_warp_bytes<4>(inter) <= (size_t)kSmemLimit;
+  return GateUpSmem<4>::bytes(hidden) <= (size_t)kSmemLimit && down_warps<4>(hidden, inter) >= 1;
 }
 
 cudaError_t launch_gateup_decode(const GateUpTable& tbl, const Slot* slots, const int32_t* n_slots,
@@ -493,11 +498,11 @@ cudaError_t launch_down_decode(const DownTable& tbl, const Slot* slots, const in
                                cudaStream_t st) {
   cudaError_t e;
   if (n_tok <= 1)
-    e = down_ring_tt<1>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, hidden, inter, y, status, st);
+    e = down_cta_tt<1>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, hidden, inter, y, status, st);
   else if (n_tok <= 2)
-    e = down_ring_tt<2>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, hidden, inter, y, status, st);
+    e = down_cta_tt<2>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, hidden, inter, y, status, st);
   else
-    e = down_ring_tt<4>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, hidden, inter, y, status, st);
+    e = down_cta_tt<4>(tbl, slots, n_slots, n_tok, K, E, n_shared, hq, hd, hidden, inter, y, status, st);
   if (e != cudaSuccess) return e;
   return launch_pdl(combine_decode_kernel, dim3((hidden + 255) / 256, n_tok), dim3(256), 0, st, true, y, inv, w,
                     n_tok, K, n_shared, hidden, out);

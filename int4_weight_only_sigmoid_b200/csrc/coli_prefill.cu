@@ -33,11 +33,12 @@
 // Roles (416 threads): warps 0-3 producers, warp 4 the MMA issuer (lane 0)
 // and TMEM owner, warps 5-12 the fold (warp w reads TMEM lanes
 // 32(w%4).. = 32 of the item's rows, columns [32h, 32h+32) with
-// h = (w-5)/4 = half of the tokens).  Per block g: the producers fill
-// operand stage g % kStages (after `empty`, raised by the MMA's commit) and
-// the block's token scales into scale stage g % kStages (after `dempty`,
-// raised by the fold warps) and arrive on `full`; the MMA writes TMEM buffer
-// g % 2 (after `tempty`) and commits `empty` and `tfull`.  All waits are
+// h = (w-5)/4 = half of the tokens).  Per block g: the producers copy (kLook
+// blocks ahead, all by cp.async) into operand stage g % kStages (after
+// `empty`, raised by the MMA's commit) and the block's token scales into
+// scale stage g % kStages (after `dempty`, raised by the fold warps), expand
+// the weights and arrive on `full`; the MMA writes TMEM buffer g % kTBufs
+// (after `tempty`) and commits `empty` and `tfull`.  All waits are
 // bounded (coli_tc.cuh).
 //
 // Sources: "Colibri：在笔记本上跑744B参数的AI模型", "关键特性" (integer dot
@@ -56,8 +57,9 @@ using namespace tc;
 
 constexpr int kM = 128;        // rows per item (TMEM lanes)
 constexpr int kN = 64;         // tokens per tile (max)
-constexpr int kStages = 4;     // operand / scale ring depth (blocks)
-constexpr int kLook = 2;       // blocks the producers' copies run ahead
+constexpr int kStages = 8;     // operand / scale ring depth (blocks)
+constexpr int kLook = 6;       // blocks the producers' copies run ahead
+constexpr int kTBufs = 4;      // TMEM accumulator buffers (blocks the MMA may run ahead of the fold)
 constexpr int kProdWarps = 4;
 constexpr int kEpiWarps = 8;   // 2 per TMEM lane quadrant, each half of the columns
 constexpr int kMmaWarp = kProdWarps;
@@ -73,7 +75,7 @@ struct PSmem {
   static constexpr int kOpB = kN * 64;                 // 64 tokens x 32 fp16
   static constexpr int kOpStage = kMats * kOpA + kOpB;
   static constexpr int kPk = kMats * kM * 16;          // packed weights of one block
-  static constexpr int kTmemCols = GU ? 256 : 128;     // 2 buffers x (gate, up | down) x 64
+  static constexpr int kTmemCols = kTBufs * kMats * kN;  // 4 buffers x (gate, up | down) x 64
   __host__ __device__ static constexpr size_t bytes() {
     return 1024 + (size_t)kStages * kOpStage + (size_t)(kLook + 1) * kPk + (size_t)kStages * kN * 4;
   }
@@ -181,8 +183,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     const float* ad, int hidden, int inter, __half* hf, float* hd, float* __restrict__ y,
     int32_t* __restrict__ err) {
   using L = PSmem<GU>;
-  __shared__ uint64_t full_bar[kStages], empty_bar[kStages], dempty_bar[kStages], tfull_bar[2], tempty_bar[2],
-      done_bar;
+  __shared__ uint64_t full_bar[kStages], empty_bar[kStages], dempty_bar[kStages], tfull_bar[kTBufs],
+      tempty_bar[kTBufs], done_bar;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
   extern __shared__ unsigned char smem_raw[];
@@ -205,7 +207,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       mbar_init(&empty_bar[s], 1);
       mbar_init(&dempty_bar[s], kNEpi);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kTBufs; ++b) {
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], kNEpi);
     }
@@ -247,10 +249,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       }
       const __half* arow = act + tokB * dim_in;
       // copies of block kb (global block gk): this thread's packed rows into
-      // pk slot kb % (kLook+1), its two B pieces into operand stage gk % kStages
+      // pk slot kb % (kLook+1), its two B pieces into operand stage
+      // gk % kStages and (p < 64) its token's scale into scale stage
+      // gk % kStages, once the MMA and the fold warps are done with them
       auto issue = [&](int kb, int gk) {
         const int s = gk % kStages;
-        if (mbar_wait(&empty_bar[s], ((gk / kStages) & 1) ^ 1, abort, err, 10)) {
+        const bool free_op = mbar_wait(&empty_bar[s], ((gk / kStages) & 1) ^ 1, abort, err, 10);
+        const bool free_d = mbar_wait(&dempty_bar[s], ((gk / kStages) & 1) ^ 1, abort, err, 14);
+        if (free_op && free_d) {
           unsigned char* pk = pk_ring + (kb % (kLook + 1)) * L::kPk;
           cp_async16(pk + p * 16, qa0 + (size_t)kb * 16);
           if constexpr (GU) cp_async16(pk + kM * 16 + p * 16, qa1 + (size_t)kb * 16);
@@ -259,6 +265,15 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
             const int c0 = 2 * (p & 1);
             cp_async16(ob + op_off(nB, c0), arow + (size_t)kb * 32 + c0 * 8);
             cp_async16(ob + op_off(nB, c0 + 1), arow + (size_t)kb * 32 + (c0 + 1) * 8);
+          }
+          if (p < kN) {
+            float* dd = d_ring + s * kN + p;
+            if (vD) {
+              asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dd)), "l"(ad + tokD * nb + kb)
+                           : "memory");
+            } else {
+              *dd = 0.0f;
+            }
           }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
@@ -279,9 +294,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         }
         asm volatile("cp.async.wait_group %0;" ::"n"(kLook) : "memory");  // block kb's copies are in
         const int s = g % kStages;
-        // the block's token scales (the fold warps have read the stage's last ones)
-        if (mbar_wait(&dempty_bar[s], ((g / kStages) & 1) ^ 1, abort, err, 14) && p < kN)
-          d_ring[s * kN + p] = vD ? ad[tokD * nb + kb] : 0.0f;
         if (!*abort) {
           const unsigned char* pk = pk_ring + (kb % (kLook + 1)) * L::kPk;
           unsigned char* op = op_ring + s * L::kOpStage;
@@ -309,12 +321,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         const ItemInfo f = item_info(slots, tiles, item, nm);
         const uint32_t idesc = idesc_f16_f32(kM, f.n_pad);
         for (int kb = 0; kb < nb; ++kb, ++g) {
-          const int s = g % kStages, b = g & 1;
+          const int s = g % kStages, b = g % kTBufs;
           if (!mbar_wait(&full_bar[s], (g / kStages) & 1, abort, err, 11)) {
             ok = false;
             break;
           }
-          if (!mbar_wait(&tempty_bar[b], ((g >> 1) & 1) ^ 1, abort, err, 12)) {
+          if (!mbar_wait(&tempty_bar[b], ((g / kTBufs) & 1) ^ 1, abort, err, 12)) {
             ok = false;
             break;
           }
@@ -359,9 +371,9 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         acc1[n] = 0.0f;
       }
       for (int kb = 0; kb < nb; ++kb, ++g) {
-        const int b = g & 1, s = g % kStages;
+        const int b = g % kTBufs, s = g % kStages;
         // warp-uniform: tcgen05.ld is a warp-wide instruction
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[b], (g >> 1) & 1, abort, err, 13));
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[b], (g / kTBufs) & 1, abort, err, 13));
         fence_after_sync();
         if (active && ok) {
           // two passes of 16 columns each, so that only 16 TMEM values per
