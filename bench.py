@@ -58,6 +58,9 @@ def parse():
                    help="resident layers cycled by the steps (8 = 39 GB; fewer for profiling captures)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-suite", action="store_true", help="skip the other workloads (decode-4/16, prefill, stack)")
+    p.add_argument("--workload", default=None, choices=list(SUITE_WORKLOADS),
+                   help="run only this workload of the suite (a profiling entry point) and print its record")
+    p.add_argument("--tokens", type=int, default=None, help="with --workload: its token count")
     return p.parse_args()
 
 
@@ -245,7 +248,10 @@ def run_reference(args):
 # the other workloads (reported beside the metric, not as the metric)
 
 
-def run_suite(layers, cfg, dev, stream, peak_gbs):
+SUITE_WORKLOADS = ("decode4", "decode16", "prefill2048", "stack8_decode1", "stack8_prefill512")
+
+
+def run_suite(layers, cfg, dev, stream, peak_gbs, only=None, tokens=None):
     """decode-4 / decode-16 / prefill-2048 / 8-layer stack (1 and 512 tokens)
     on the resident layers.  Each entry: per-layer tokens/s, ms per step,
     unique experts streamed per layer and the weight bytes that implies per
@@ -287,6 +293,9 @@ def run_suite(layers, cfg, dev, stream, peak_gbs):
 
     for name, T, steps, graph in [("decode4", 4, 256, True), ("decode16", 16, 256, True),
                                   ("prefill2048", 2048, 16, False)]:
+        if only is not None and name != only:
+            continue
+        T = tokens or T
         c = synth.config(name, seed=cfg["seed"])
         x = synth.dev_tokens(c, T, device=dev)
         lys = layers
@@ -320,6 +329,9 @@ def run_suite(layers, cfg, dev, stream, peak_gbs):
 
     # the 8-layer pre-norm stack (RMSNorm + residual between layers)
     for name, T, steps, graph in [("stack8_decode1", 1, 64, True), ("stack8_prefill512", 512, 4, False)]:
+        if only is not None and name != only:
+            continue
+        T = tokens or T
         c = synth.config("stack8_512" if T > 1 else "stack8", seed=cfg["seed"])
         x = synth.dev_tokens(c, T, device=dev)
         arr = coli.stack_cstructs(layers)
@@ -404,6 +416,16 @@ def main():
     outs = torch.empty(2, 1, H, dtype=torch.float32, device=dev)
     ws = coli.make_workspace(layers[0].cfg, 1, dev)
     torch.cuda.synchronize()
+    if args.workload is not None:
+        peak, _ = peaks()
+        rec = run_suite(layers, cfg, dev, torch.cuda.Stream(device=dev), peak, only=args.workload,
+                        tokens=args.tokens)
+        if rank == 0:
+            print(json.dumps({"workload": args.workload, **rec[args.workload]}), flush=True)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     # expert bytes actually streamed per step (unique selected experts + shared)
     mat = cfg["inter"] * H // 2
@@ -422,8 +444,8 @@ def main():
         coli.moe_layer_forward(layers[i % n_layers], xs[i % N_TOK_POOL:i % N_TOK_POOL + 1], out=outs[i % 2],
                                workspace=ws, stream=stream, cstruct=cstructs[i % n_layers])
 
-    # warm-up (also sets kernel attributes before any capture)
     s = torch.cuda.Stream(device=dev)
+    # warm-up (also sets kernel attributes before any capture)
     with torch.cuda.stream(s):
         for i in range(max(3, args.warmup)):
             step(i, s)
