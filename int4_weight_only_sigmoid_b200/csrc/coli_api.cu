@@ -123,7 +123,7 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   L.tiles = take(prefill_tile_bytes((int)T, (int)K, (int)E, (int)S));
   L.n_tiles = take(4);
   L.hq = take(rows * I);
-  L.xf = take(T * H * 2);
+  L.xf = take(rows * H * 2);
   L.hf = take(rows * I * 2);
   L.hd = take(rows * (I / 32) * 4);
   L.y = take(rows * H * 4);
@@ -211,7 +211,7 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   CHECK_LAUNCH(mark(0));
   if (prefill_supported(H, I)) {
     CHECK_LAUNCH(launch_prefill_experts(gu, dn, slots, n_slots, at<void>(ws, W.tiles), at<int32_t>(ws, W.n_tiles),
-                                        perm, K, xq, xd, (int)T, H, I, at<void>(ws, W.xf), at<void>(ws, W.hf), hd, y,
+                                        perm, K, S, xq, xd, (int)T, H, I, at<void>(ws, W.xf), at<void>(ws, W.hf), hd, y,
                                         at<int32_t>(ws, W.status), st, ev[1]));
   } else {
     CHECK_LAUNCH(launch_gateup(gu, sl, xq, xd, H, I, max_tok, hq, hd, st));

@@ -92,8 +92,9 @@ cudaError_t launch_down_decode(const DownTable& tbl, const Slot* slots, const in
                                cudaStream_t st);
 
 // Prefill expert kernels on the tensor cores (tcgen05): the fp16 operand
-// rows of the Q8 activations (xf: n_tok x hidden halves), the tile list
-// (<= 64 tokens of one slot per tile) built from the slot table, then the
+// rows of the Q8 activations, one per (slot, token) in slot order (xf:
+// n_tok*(K+n_shared) x hidden halves), the tile list (<= 128 tokens of one
+// slot per tile) built from the slot table, then the
 // persistent gate/up GEMM (+ SwiGLU + Q8 of h, written as fp16 rows hf:
 // rows x inter halves, scales hd) and the persistent down GEMM (-> y).
 // `tiles` needs prefill_tile_bytes().
@@ -102,9 +103,9 @@ size_t prefill_tiles_bound(int n_tok, int K, int E, int n_shared);
 size_t prefill_tile_bytes(int n_tok, int K, int E, int n_shared);
 cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, const Slot* slots,
                                    const int32_t* n_slots, void* tiles, int32_t* n_tiles, const int32_t* perm,
-                                   int K, const int8_t* xq, const float* xd, int n_tok, int hidden, int inter,
-                                   void* xf, void* hf, float* hd, float* y, int32_t* err, cudaStream_t st,
-                                   cudaEvent_t ev_mid);
+                                   int K, int n_shared, const int8_t* xq, const float* xd, int n_tok, int hidden,
+                                   int inter, void* xf, void* hf, float* hd, float* y, int32_t* err,
+                                   cudaStream_t st, cudaEvent_t ev_mid);
 
 // out[t] = sum_k w[t,k] y[inv[t,k]] + sum_s y[n_tok*K + s*n_tok + t]  (contract C)
 cudaError_t launch_combine(const float* y, const int32_t* inv, const float* w, int n_tok, int K,

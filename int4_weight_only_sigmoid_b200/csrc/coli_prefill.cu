@@ -1,9 +1,16 @@
 // coli_prefill.cu -- the expert kernels for many tokens per expert (prefill):
 // a grouped GEMM on the 5th-generation tensor cores (tcgen05.mma, F32
-// accumulators in tensor memory).  Work items are (tile of <= 64 of one
-// slot's tokens, 128 output rows); one persistent CTA per SM walks items
+// accumulators in tensor memory).  Work items are (tile of <= 128 of one
+// slot's tokens, 128 output columns); one persistent CTA per SM walks items
 // c, c + G, ... and keeps its pipeline (producers -> MMA -> fold) running
 // from one item to the next.
+//
+// Orientation.  The tokens are the MMA's M dimension (TMEM lanes) and the
+// weight rows its N dimension (TMEM columns), so a fold thread owns one
+// token: the token's Q8 scale d_x[b] is one register per block, and in the
+// gate/up kernel a thread holds its token's 32 consecutive gate rows and the
+// matching up rows, so SwiGLU and the Q8 block of h are thread-local.  The
+// gate/up item's 128 columns are 64 gate rows and the same 64 up rows.
 //
 // Exactness.  Each Q8 block's partial sum must come out exactly, because the
 // row fold (contract F: acc = fmaf(d_x[b], (float)isum[b], acc), b
@@ -18,33 +25,35 @@
 //
 // Why fp16 operands and not kind::i8: the fold costs one F32 FMA per
 // (row, token, block) whatever the MMA kind; with kind::i8 each of those
-// also needs an int32 -> F32 conversion, and the CUDA-core fold, not the
-// tensor pipe, is the limit of this layer (one FMA per 32 MACs).  fp16
-// operands give F32 sums directly.
+// also needs an int32 -> F32 conversion, and the CUDA cores (weight
+// expansion and the fold), not the tensor pipe, are the limit of this layer.
+// fp16 operands give F32 sums directly.
 //
-// Operands.  The activations are converted to fp16 once per forward
-// (act_f16_kernel; the gate/up fold writes h straight as fp16 for the down
-// kernel), in the element order [0,2,4,6,1,3,5,7] of every 8 that the int4
-// expansion produces; a tile's B operand is then a gather of 16-byte pieces
-// by cp.async.  The packed weights of a block are copied by the producer
-// thread that later expands them (each thread owns one row of each matrix),
-// so no producer thread waits for another.
+// Operands.  The activations are converted to fp16 once per forward, one
+// row per (slot, token) in slot order (act_rows_f16_kernel; the gate/up fold
+// writes h straight as fp16 rows in the same order for the down kernel), in
+// the element order [0,4,1,5,2,6,3,7] of every 8 that the int4 expansion
+// produces; a tile's A operand is then 128 consecutive rows, loaded by TMA
+// (128-byte swizzle).  The packed weights are copied by the producer warps
+// with cp.async and expanded into the B operand (K-major, no swizzle).
 //
-// Roles (416 threads): warps 0-3 producers, warp 4 the MMA issuer (lane 0)
-// and TMEM owner, warps 5-12 the fold (warp w reads TMEM lanes
-// 32(w%4).. = 32 of the item's rows, columns [32h, 32h+32) with
-// h = (w-5)/4 = half of the tokens).  Per block g: the producers copy (kLook
-// blocks ahead, all by cp.async) into operand stage g % kStages (after
-// `empty`, raised by the MMA's commit) and the block's token scales into
-// scale stage g % kStages (after `dempty`, raised by the fold warps), expand
-// the weights and arrive on `full`; the MMA writes TMEM buffer g % kTBufs
-// (after `tempty`) and commits `empty` and `tfull`.  All waits are
-// bounded (coli_tc.cuh).
+// Roles (416 threads): warps 0-3 producers (thread p: weight row p and token
+// row p of the tile), warp 4 the MMA issuer (lane 0) and TMEM owner, warps
+// 5-12 the fold (warp w reads TMEM lanes 32(w%4).. = 32 of the tile's
+// tokens, and half of the item's columns).  Per block g: the producers copy
+// (kLook blocks ahead, all by cp.async) into operand stage g % kStages
+// (after `empty`, raised by the MMA's commit, and `dempty`, raised by the
+// fold warps once they have read the stage's token scales), expand the
+// weights and arrive on `full`; the MMA writes TMEM buffer g % kTBufs (after
+// `tempty`) and commits `empty` and `tfull`.  All waits are bounded
+// (coli_tc.cuh).
 //
 // Sources: "Colibri：在笔记本上跑744B参数的AI模型", "关键特性" (integer dot
 // kernels, Q8_0 activations, packed int4); HN summary (hn.213312.xyz),
 // "已实现的功能" (batched MoE: in prefill, an expert used by several
 // positions is read once and shared).
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 
 #include "coli_launch.h"
@@ -55,29 +64,30 @@ namespace {
 
 using namespace tc;
 
-constexpr int kM = 128;        // rows per item (TMEM lanes)
-constexpr int kN = 64;         // tokens per tile (max)
-constexpr int kStages = 8;     // operand / scale ring depth (blocks)
-constexpr int kLook = 6;       // blocks the producers' copies run ahead
-constexpr int kTBufs = 4;      // TMEM accumulator buffers (blocks the MMA may run ahead of the fold)
+constexpr int kM = 128;        // tokens per tile (MMA M, TMEM lanes)
+constexpr int kN = 128;        // output columns per item (MMA N): 64 gate + 64 up rows, or 128 down rows
+constexpr int kBS = 4;         // Q8 blocks per operand stage (K = 128)
+constexpr int kStages = 3;     // operand stages
+constexpr int kLookS = 2;      // stages the producers' copies run ahead
+constexpr int kPkSlots = kLookS + 2;  // packed-weight slots: a slot is rewritten only after every producer expanded it
+constexpr int kHalf = 2;       // Q8 blocks per accumulator hand-off (MMA -> fold)
+constexpr int kTBufs = 4;      // TMEM accumulators (one per block), handed off in pairs
 constexpr int kProdWarps = 4;
 constexpr int kEpiWarps = 8;   // 2 per TMEM lane quadrant, each half of the columns
 constexpr int kMmaWarp = kProdWarps;
 constexpr int kEpi0 = kProdWarps + 1;                          // first fold warp
 constexpr int kThreadsP = 32 * (kProdWarps + 1 + kEpiWarps);  // 416
 constexpr int kNProd = 32 * kProdWarps;                        // 128 producer threads
-constexpr int kNEpi = 32 * kEpiWarps;                          // 256 fold threads
+constexpr int kTmemCols = kTBufs * kN;                         // 512
 
-template <bool GU>
 struct PSmem {
-  static constexpr int kMats = GU ? 2 : 1;
-  static constexpr int kOpA = kM * 64;                 // one matrix: 128 rows x 32 fp16
-  static constexpr int kOpB = kN * 64;                 // 64 tokens x 32 fp16
-  static constexpr int kOpStage = kMats * kOpA + kOpB;
-  static constexpr int kPk = kMats * kM * 16;          // packed weights of one block
-  static constexpr int kTmemCols = kTBufs * kMats * kN;  // 4 buffers x (gate, up | down) x 64
+  static constexpr int kAtomA = kM * 128;           // A: 128 token rows x 64 fp16 (two blocks), 128B-swizzled
+  static constexpr int kStageA = 2 * kAtomA;        // a stage's 4 blocks
+  static constexpr int kSubB = kN * 64;             // B, one block: 128 weight rows x 32 fp16
+  static constexpr int kOpStage = kStageA + kBS * kSubB;
+  static constexpr int kPk = kN * kBS * 16;         // packed weights of one stage (row-major, 64 B per row)
   __host__ __device__ static constexpr size_t bytes() {
-    return 1024 + (size_t)kStages * kOpStage + (size_t)(kLook + 1) * kPk + (size_t)kStages * kN * 4;
+    return 1024 + (size_t)kStages * kOpStage + (size_t)kPkSlots * kPk;
   }
 };
 
@@ -85,27 +95,28 @@ struct Tile {
   int32_t slot, n0;
 };
 
-// fp16 operands from packed int4: 8 nibbles of one 32-bit word -> 8 fp16 in
-// the order [0,2,4,6,1,3,5,7] (the activations use the same order, so the
-// dot product is unchanged).  fp16 bits 0x6400 | u are 1024 + u exactly; with
-// u = q + 8 (offset nibble), subtracting 1032 leaves q exactly.
+// fp16 operands from packed int4: the 8 nibbles of one 32-bit word (element
+// e in bits 4e..4e+3, two's complement) -> 8 fp16 in the order
+// [0,4,1,5,2,6,3,7] (the activations use the same order, so the dot product
+// is unchanged).  (w & 0x000F000F) ^ 0x64086408 is the fp16 pair
+// 1024 + (q + 8) for elements 0 and 4 exactly; the nibbles one position up
+// give 1024 + 16 (q + 8), which x 1/16 - 72 maps to q exactly.
 __device__ __forceinline__ uint4 expand_int4_word(uint32_t w) {
-  const uint32_t u = w ^ 0x88888888u;
-  const uint32_t lo = u & 0x0F0F0F0Fu;
-  const uint32_t hi = (u >> 4) & 0x0F0F0F0Fu;
-  const uint32_t c = 0x64646464u;
-  const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032, 1032
-  uint32_t r[4] = {__byte_perm(lo, c, 0x4140), __byte_perm(lo, c, 0x4342), __byte_perm(hi, c, 0x4140),
-                   __byte_perm(hi, c, 0x4342)};
+  const uint32_t w8 = w >> 8;
+  uint32_t r[4] = {(w & 0x000F000Fu) ^ 0x64086408u, (w & 0x00F000F0u) ^ 0x64806480u,
+                   (w8 & 0x000F000Fu) ^ 0x64086408u, (w8 & 0x00F000F0u) ^ 0x64806480u};
+  const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));        // 1032
+  const __half2 sixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
+  const __half2 m72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));        // -72
   uint4 o;
   __half2 h;
   h = __hsub2(*reinterpret_cast<__half2*>(&r[0]), off);
   o.x = *reinterpret_cast<uint32_t*>(&h);
-  h = __hsub2(*reinterpret_cast<__half2*>(&r[1]), off);
+  h = __hfma2(*reinterpret_cast<__half2*>(&r[1]), sixteenth, m72);
   o.y = *reinterpret_cast<uint32_t*>(&h);
   h = __hsub2(*reinterpret_cast<__half2*>(&r[2]), off);
   o.z = *reinterpret_cast<uint32_t*>(&h);
-  h = __hsub2(*reinterpret_cast<__half2*>(&r[3]), off);
+  h = __hfma2(*reinterpret_cast<__half2*>(&r[3]), sixteenth, m72);
   o.w = *reinterpret_cast<uint32_t*>(&h);
   return o;
 }
@@ -114,10 +125,11 @@ __device__ __forceinline__ uint4 expand_int4_word(uint32_t w) {
 // element order: with u = x + 128, 0x6400 | u is 1024 + u; minus 1152 is x.
 __device__ __forceinline__ uint4 expand_int8_pair(uint32_t a, uint32_t b) {
   const uint32_t ua = a ^ 0x80808080u, ub = b ^ 0x80808080u;
+  const uint32_t t0 = __byte_perm(ua, ub, 0x5140), t1 = __byte_perm(ua, ub, 0x7362);  // u0 u4 u1 u5 | u2 u6 u3 u7
   const uint32_t c = 0x64646464u;
   const __half2 off = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));  // 1152, 1152
-  uint32_t r[4] = {__byte_perm(ua, c, 0x4240), __byte_perm(ub, c, 0x4240), __byte_perm(ua, c, 0x4341),
-                   __byte_perm(ub, c, 0x4341)};
+  uint32_t r[4] = {__byte_perm(t0, c, 0x4140), __byte_perm(t0, c, 0x4342), __byte_perm(t1, c, 0x4140),
+                   __byte_perm(t1, c, 0x4342)};
   uint4 o;
   __half2 h;
   h = __hsub2(*reinterpret_cast<__half2*>(&r[0]), off);
@@ -131,21 +143,54 @@ __device__ __forceinline__ uint4 expand_int8_pair(uint32_t a, uint32_t b) {
   return o;
 }
 
-// Position of element e (0..7) of an 8-group in the operand order.
-__device__ __forceinline__ int op_pos8(int e) { return (e & 1) ? 4 + (e >> 1) : (e >> 1); }
-
 // Byte offset of 16-byte chunk c (0..3) of row r in a K-major, no-swizzle
 // operand tile of 32 fp16 per row: 8-row x 16-byte core matrices, the four
 // K chunks of an 8-row group 128 B apart (LBO), groups 512 B apart (SBO).
 __device__ __forceinline__ uint32_t op_off(int r, int c) { return (r >> 3) * 512 + c * 128 + (r & 7) * 16; }
 
-// Q8 rows (int8) -> fp16 operand rows, 8 values per thread.
-__global__ void __launch_bounds__(256) act_f16_kernel(const int8_t* __restrict__ q, int64_t n8,
-                                                      uint4* __restrict__ out) {
+// fp16 operand rows of the Q8 activations in row order: row r < n_tok*K is
+// token perm[r] / K (the routed slots' rows), row n_tok*K + s*n_tok + t is
+// token t (shared expert s).  8 values per thread.
+__global__ void __launch_bounds__(256) act_rows_f16_kernel(const int8_t* __restrict__ q, const int32_t* perm,
+                                                           int n_tok, int top_k, int64_t rows, int hidden,
+                                                           uint4* __restrict__ out) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n8) return;
-  const uint2 v = reinterpret_cast<const uint2*>(q)[i];
+  const int per_row = hidden / 8;
+  if (i >= rows * per_row) return;
+  const int64_t r = i / per_row;
+  const int c = (int)(i - r * per_row);
+  const int64_t routed = (int64_t)n_tok * top_k;
+  const int64_t tok = r < routed ? (int64_t)(__ldg(perm + r) / top_k) : (r - routed) % n_tok;
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(q + tok * hidden) + c);
   out[i] = expand_int8_pair(v.x, v.y);
+}
+
+// 2D tiled bulk-tensor load (TMA) of box (x, y) into shared memory,
+// completing `bytes` on the mbarrier.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle (the layout a
+// TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes): 8-row x 128-byte atoms,
+// consecutive 8-row groups 1024 B apart; a K step inside the atom advances
+// the start address.
+__device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;             // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset
+  d |= (uint64_t)1 << 46;             // descriptor version for tcgen05
+  d |= (uint64_t)2 << 61;             // SWIZZLE_128B
+  return d;
 }
 
 // fma on two F32 lanes at once (two IEEE fmas, each rounded once).
@@ -160,31 +205,39 @@ __device__ __forceinline__ void fma2(float& a0, float& a1, float d0, float d1, f
 
 struct ItemInfo {
   Slot slot;
-  int n0, n_valid, n_pad, m0;
+  int n0, n_valid, m0;
 };
 
-__device__ __forceinline__ ItemInfo item_info(const Slot* slots, const Tile* tiles, int item, int nm) {
+// Item i: tile i / nm, column group i % nm (rows [m0, m0 + group_rows) of
+// each output matrix).
+__device__ __forceinline__ ItemInfo item_info(const Slot* slots, const Tile* tiles, int item, int nm, int group_rows) {
   ItemInfo f;
   const int t = item / nm;
   const Tile tile = tiles[t];
   f.slot = slots[tile.slot];
   f.n0 = tile.n0;
-  f.n_valid = min(kN, f.slot.count - tile.n0);
-  f.n_pad = (f.n_valid + 15) & ~15;
-  f.m0 = (item - t * nm) * kM;
+  f.n_valid = min(kM, f.slot.count - tile.n0);
+  f.m0 = (item - t * nm) * group_rows;
   return f;
+}
+
+// Source row (into the activation / h rows) of token n of the item's tile.
+__device__ __forceinline__ int64_t item_token_row(const ItemInfo& f, bool gu, const int32_t* perm, int top_k, int n) {
+  if (!gu) return (int64_t)f.slot.row_base + f.n0 + n;
+  return f.slot.perm_base < 0 ? (int64_t)(f.n0 + n) : (int64_t)(perm[f.slot.perm_base + f.n0 + n] / top_k);
 }
 
 // GU: gate/up (+ SwiGLU + Q8 of h -> hf fp16 rows + hd); !GU: down (-> y).
 template <bool GU, typename Tab>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
-    const __grid_constant__ Tab tab, const Slot* __restrict__ slots, const Tile* __restrict__ tiles,
-    const int32_t* __restrict__ n_tiles, const int32_t* __restrict__ perm, int top_k, const __half* act,
-    const float* ad, int hidden, int inter, __half* hf, float* hd, float* __restrict__ y,
-    int32_t* __restrict__ err) {
-  using L = PSmem<GU>;
-  __shared__ uint64_t full_bar[kStages], empty_bar[kStages], dempty_bar[kStages], tfull_bar[kTBufs],
-      tempty_bar[kTBufs], done_bar;
+    const __grid_constant__ Tab tab, const __grid_constant__ CUtensorMap amap, const Slot* __restrict__ slots,
+    const Tile* __restrict__ tiles,
+    const int32_t* __restrict__ n_tiles, const int32_t* __restrict__ perm, int top_k, const float* ad, int hidden,
+    int inter, __half* hf, float* hd, float* __restrict__ y, int32_t* __restrict__ err) {
+  using L = PSmem;
+  constexpr int kGroupRows = GU ? kN / 2 : kN;  // output rows of one matrix per item
+  __shared__ uint64_t full_bar[kStages], empty_bar[kStages], tfull_bar[kTBufs / kHalf], tempty_bar[kTBufs / kHalf],
+      done_bar;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
   extern __shared__ unsigned char smem_raw[];
@@ -192,30 +245,29 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
   const int dim_in = GU ? hidden : inter;
   const int dim_out = GU ? inter : hidden;
   const int nb = dim_in / 32;
-  const int nm = dim_out / kM;
+  const int nst = nb / kBS;  // stages per item
+  const int nm = dim_out / kGroupRows;
   const int n_items = *n_tiles * nm;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1 KB aligned
-  unsigned char* op_ring = smem;
-  unsigned char* pk_ring = op_ring + kStages * L::kOpStage;
-  float* d_ring = reinterpret_cast<float*>(pk_ring + (kLook + 1) * L::kPk);  // [kStages][kN]
+  unsigned char* op_ring = smem;                                  // [kStages][A: 2 atoms | B: kBS x kSubB]
+  unsigned char* pk_ring = op_ring + kStages * L::kOpStage;       // [kPkSlots][128 rows][64 B]
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_bar[s], kNProd);
+      mbar_init(&full_bar[s], kProdWarps + 1);  // + the TMA issuer's expect_tx
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&dempty_bar[s], kNEpi);
     }
-    for (int b = 0; b < kTBufs; ++b) {
+    for (int b = 0; b < kTBufs / kHalf; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], kNEpi);
+      mbar_init(&tempty_bar[b], kEpiWarps);
     }
     mbar_init(&done_bar, 1);
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == kMmaWarp) tmem_alloc(&tmem_s, L::kTmemCols);
+  if (warp == kMmaWarp) tmem_alloc(&tmem_s, kTmemCols);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
@@ -224,127 +276,128 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
 
   if (warp < kProdWarps) {
     // ------------------------------------------------------------ producers
-    const int p = threadIdx.x;  // row p of each matrix; B pieces of token row p >> 1
+    // A stage's A tile (128 rows of the row-ordered fp16 activations / h,
+    // 4 blocks) is one pair of TMA loads issued by thread 0.  Its packed
+    // weights (128 rows x 64 B) are copied 4 lanes per row, so that each
+    // warp instruction touches few cache lines; thread p then expands weight
+    // row p of the stage's 4 blocks.  The copies run kLookS stages ahead
+    // across item boundaries: the issue cursor (item ii, stage ji) moves
+    // ahead of the expansion.
+    const int p = threadIdx.x;
     const size_t rb = (size_t)dim_in / 2;
-    int g = 0;  // global block counter
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const ItemInfo f = item_info(slots, tiles, item, nm);
-      auto tok_of = [&](int n) -> int64_t {
-        if (!GU) return (int64_t)f.slot.row_base + f.n0 + n;
-        return f.slot.perm_base < 0 ? (int64_t)(f.n0 + n) : (int64_t)(perm[f.slot.perm_base + f.n0 + n] / top_k);
-      };
-      const int nB = p >> 1;
-      const bool vB = nB < f.n_valid;
-      const int64_t tokB = vB ? tok_of(nB) : 0;
-      const bool vD = p < f.n_valid;
-      const int64_t tokD = vD ? tok_of(p) : 0;
-      const uint8_t* qa0;
-      const uint8_t* qa1;
-      if constexpr (GU) {
-        qa0 = tab.gate_q[f.slot.table_idx] + (size_t)(f.m0 + p) * rb;
-        qa1 = tab.up_q[f.slot.table_idx] + (size_t)(f.m0 + p) * rb;
-      } else {
-        qa0 = tab.down_q[f.slot.table_idx] + (size_t)(f.m0 + p) * rb;
-        qa1 = qa0;
-      }
-      const __half* arow = act + tokB * dim_in;
-      // copies of block kb (global block gk): this thread's packed rows into
-      // pk slot kb % (kLook+1), its two B pieces into operand stage
-      // gk % kStages and (p < 64) its token's scale into scale stage
-      // gk % kStages, once the MMA and the fold warps are done with them
-      auto issue = [&](int kb, int gk) {
-        const int s = gk % kStages;
-        const bool free_op = mbar_wait(&empty_bar[s], ((gk / kStages) & 1) ^ 1, abort, err, 10);
-        const bool free_d = mbar_wait(&dempty_bar[s], ((gk / kStages) & 1) ^ 1, abort, err, 14);
-        if (free_op && free_d) {
-          unsigned char* pk = pk_ring + (kb % (kLook + 1)) * L::kPk;
-          cp_async16(pk + p * 16, qa0 + (size_t)kb * 16);
-          if constexpr (GU) cp_async16(pk + kM * 16 + p * 16, qa1 + (size_t)kb * 16);
-          if (vB) {
-            unsigned char* ob = op_ring + s * L::kOpStage + L::kMats * L::kOpA;
-            const int c0 = 2 * (p & 1);
-            cp_async16(ob + op_off(nB, c0), arow + (size_t)kb * 32 + c0 * 8);
-            cp_async16(ob + op_off(nB, c0 + 1), arow + (size_t)kb * 32 + (c0 + 1) * 8);
+    const int n_mine = blockIdx.x < n_items ? (n_items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    const int total = n_mine * nst;
+    int ii = blockIdx.x, ji = 0;
+    ItemInfo fi{};
+    auto enter_item = [&]() {
+      if (ii < n_items) fi = item_info(slots, tiles, ii, nm, kGroupRows);
+    };
+    // weight row r of the issue item: GU rows 0..63 gate, 64..127 up
+    auto wrow = [&](int r) -> const uint8_t* {
+      if constexpr (GU)
+        return (r < kGroupRows ? tab.gate_q[fi.slot.table_idx] : tab.up_q[fi.slot.table_idx]) +
+               (size_t)(fi.m0 + (r & (kGroupRows - 1))) * rb;
+      else
+        return tab.down_q[fi.slot.table_idx] + (size_t)(fi.m0 + r) * rb;
+    };
+    // copies of the cursor's stage (global stage gj) into operand stage
+    // gj % kStages and pk slot gj % kPkSlots; then the cursor moves on
+    auto issue = [&](int gj) {
+      if (gj < total) {
+        const int s = gj % kStages;
+        if (mbar_wait(&empty_bar[s], ((gj / kStages) & 1) ^ 1, abort, err, 10)) {
+          const int kb0 = ji * kBS;
+          if (p == 0) {
+            unsigned char* oa = op_ring + s * L::kOpStage;
+            const int row0 = fi.slot.row_base + fi.n0;
+            mbar_arrive_expect_tx(&full_bar[s], L::kStageA);
+            tma_load_2d(oa, &amap, kb0 * 32, row0, &full_bar[s]);
+            tma_load_2d(oa + L::kAtomA, &amap, kb0 * 32 + 64, row0, &full_bar[s]);
           }
-          if (p < kN) {
-            float* dd = d_ring + s * kN + p;
-            if (vD) {
-              asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dd)), "l"(ad + tokD * nb + kb)
-                           : "memory");
-            } else {
-              *dd = 0.0f;
-            }
+          unsigned char* pk = pk_ring + (gj % kPkSlots) * L::kPk;
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {  // W: row it*32 + p/4, chunk p%4 (= block kb0 + p%4)
+            const int q = it * kNProd + p;
+            const int r = q >> 2, c = q & 3;
+            cp_async16(pk + r * 64 + c * 16, wrow(r) + (size_t)(kb0 + c) * 16);
           }
+        } else if (p == 0) {
+          mbar_arrive(&full_bar[s]);  // keep the arrival count; the CTA is aborting
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
-      };
+        if (++ji == nst) {
+          ji = 0;
+          ii += gridDim.x;
+          enter_item();
+        }
+      } else {
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      }
+    };
+    enter_item();
 #pragma unroll
-      for (int i = 0; i < kLook; ++i) {
-        if (i < nb) {
-          issue(i, g + i);
-        } else {
-          asm volatile("cp.async.commit_group;" ::: "memory");
+    for (int i = 0; i < kLookS; ++i) issue(i);
+    for (int gs = 0; gs < total; ++gs) {
+      issue(gs + kLookS);
+      asm volatile("cp.async.wait_group %0;" ::"n"(kLookS) : "memory");  // stage gs's copies (this thread's) are in
+      named_bar(1, kNProd);                                              // ... and every producer's
+      const int s = gs % kStages;
+      if (!*abort) {
+        const uint4* pk = reinterpret_cast<const uint4*>(pk_ring + (gs % kPkSlots) * L::kPk + p * 64);
+        unsigned char* ob = op_ring + s * L::kOpStage + L::kStageA;
+#pragma unroll
+        for (int c = 0; c < kBS; ++c) {
+          const uint4 w = pk[c];
+          unsigned char* dst = ob + c * L::kSubB;
+          *reinterpret_cast<uint4*>(dst + op_off(p, 0)) = expand_int4_word(w.x);
+          *reinterpret_cast<uint4*>(dst + op_off(p, 1)) = expand_int4_word(w.y);
+          *reinterpret_cast<uint4*>(dst + op_off(p, 2)) = expand_int4_word(w.z);
+          *reinterpret_cast<uint4*>(dst + op_off(p, 3)) = expand_int4_word(w.w);
         }
       }
-      for (int kb = 0; kb < nb; ++kb, ++g) {
-        if (kb + kLook < nb) {
-          issue(kb + kLook, g + kLook);
-        } else {
-          asm volatile("cp.async.commit_group;" ::: "memory");
-        }
-        asm volatile("cp.async.wait_group %0;" ::"n"(kLook) : "memory");  // block kb's copies are in
-        const int s = g % kStages;
-        if (!*abort) {
-          const unsigned char* pk = pk_ring + (kb % (kLook + 1)) * L::kPk;
-          unsigned char* op = op_ring + s * L::kOpStage;
-#pragma unroll
-          for (int m = 0; m < L::kMats; ++m) {
-            const uint4 w = *reinterpret_cast<const uint4*>(pk + m * kM * 16 + p * 16);
-            unsigned char* dst = op + m * L::kOpA;
-            *reinterpret_cast<uint4*>(dst + op_off(p, 0)) = expand_int4_word(w.x);
-            *reinterpret_cast<uint4*>(dst + op_off(p, 1)) = expand_int4_word(w.y);
-            *reinterpret_cast<uint4*>(dst + op_off(p, 2)) = expand_int4_word(w.z);
-            *reinterpret_cast<uint4*>(dst + op_off(p, 3)) = expand_int4_word(w.w);
-          }
-        }
-        fence_async_smem();  // this thread's operand writes (stores and cp.async) -> the tensor core
-        mbar_arrive(&full_bar[s]);
-      }
+      fence_async_smem();  // this thread's operand writes (stores and cp.async) -> the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full_bar[s]);
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int g = 0;
+      int gs = 0, gh = 0;
       bool ok = true;
+      constexpr uint32_t idesc = idesc_f16_f32(kM, kN);
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-        const ItemInfo f = item_info(slots, tiles, item, nm);
-        const uint32_t idesc = idesc_f16_f32(kM, f.n_pad);
-        for (int kb = 0; kb < nb; ++kb, ++g) {
-          const int s = g % kStages, b = g % kTBufs;
-          if (!mbar_wait(&full_bar[s], (g / kStages) & 1, abort, err, 11)) {
-            ok = false;
-            break;
-          }
-          if (!mbar_wait(&tempty_bar[b], ((g / kTBufs) & 1) ^ 1, abort, err, 12)) {
+        for (int j = 0; j < nst && ok; ++j, ++gs) {
+          const int s = gs % kStages;
+          if (!mbar_wait(&full_bar[s], (gs / kStages) & 1, abort, err, 11)) {
             ok = false;
             break;
           }
           fence_after_sync();
-          const uint32_t op = smem_u32(op_ring + s * L::kOpStage);
-          const uint32_t opb = op + L::kMats * L::kOpA;
+          const uint32_t opa = smem_u32(op_ring + s * L::kOpStage);
+          const uint32_t opb = opa + L::kStageA;
 #pragma unroll
-          for (int m = 0; m < L::kMats; ++m) {
-            const uint32_t d = tmem + b * (L::kMats * kN) + m * kN;
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {  // two K=16 steps = one Q8 block
-              const uint64_t da = smem_desc_k_noswizzle(op + m * L::kOpA + k * 256, 128, 512);
-              const uint64_t db = smem_desc_k_noswizzle(opb + k * 256, 128, 512);
-              mma_f16(d, da, db, idesc, k);
+          for (int hh = 0; hh < kBS / kHalf; ++hh, ++gh) {
+            const int hb = gh % (kTBufs / kHalf);
+            if (!mbar_wait(&tempty_bar[hb], ((gh / (kTBufs / kHalf)) & 1) ^ 1, abort, err, 12)) {
+              ok = false;
+              break;
             }
+            fence_after_sync();
+#pragma unroll
+            for (int i = 0; i < kHalf; ++i) {
+              const int c = hh * kHalf + i;  // block within the stage
+              const uint32_t d = tmem + (hb * kHalf + i) * kN;
+#pragma unroll
+              for (int k = 0; k < 2; ++k) {  // two K=16 steps = one Q8 block
+                const uint64_t da = smem_desc_k_sw128(opa + (c >> 1) * L::kAtomA + (c & 1) * 64 + k * 32);
+                const uint64_t db = smem_desc_k_noswizzle(opb + c * L::kSubB + k * 256, 128, 512);
+                mma_f16(d, da, db, idesc, k);
+              }
+            }
+            mma_commit(&tfull_bar[hb]);
           }
-          mma_commit(&empty_bar[s]);
-          mma_commit(&tfull_bar[b]);
+          if (ok) mma_commit(&empty_bar[s]);
         }
       }
       // every MMA this thread issued has finished before TMEM is released
@@ -356,99 +409,112 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     __syncwarp();
   } else {
     // ------------------------------------------------------------ fold
-    // warp w: TMEM lanes 32*(w%4).. (rows), columns [cb, cb + 32) (tokens)
-    constexpr int kC = kN / 2;
-    const int quad = warp & 3, cb = ((warp - kEpi0) >> 2) * kC;
+    // warp w: TMEM lanes 32*(w%4).. (tokens); columns c0.. and c1.. (32 each):
+    // gate/up: the gate rows [32 hh, 32 hh + 32) of the group and the same
+    // up rows (64 columns on); down: columns [64 hh, 64 hh + 64)
+    const int quad = warp & 3, hh = (warp - kEpi0) >> 2;
+    const int c0 = GU ? 32 * hh : 64 * hh;
+    const int c1 = GU ? kGroupRows + 32 * hh : 64 * hh + 32;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    int g = 0;
+    const int n = quad * 32 + lane;  // this thread's token within the tile
+    int gh = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const ItemInfo f = item_info(slots, tiles, item, nm);
-      const bool active = cb < f.n_pad;  // warp-uniform
-      float acc0[kC], acc1[kC];
+      const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
+      const bool active = quad * 32 < f.n_valid;  // warp-uniform
+      const bool valid = n < f.n_valid;
+      const float* drow = ad + (valid ? item_token_row(f, GU, perm, top_k, n) : 0) * nb;
+      float acc0[32], acc1[32];
 #pragma unroll
-      for (int n = 0; n < kC; ++n) {
-        acc0[n] = 0.0f;
-        acc1[n] = 0.0f;
+      for (int j = 0; j < 32; ++j) {
+        acc0[j] = 0.0f;
+        acc1[j] = 0.0f;
       }
-      for (int kb = 0; kb < nb; ++kb, ++g) {
-        const int b = g % kTBufs, s = g % kStages;
-        // warp-uniform: tcgen05.ld is a warp-wide instruction
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[b], (g / kTBufs) & 1, abort, err, 13));
-        fence_after_sync();
-        if (active && ok) {
-          // two passes of 16 columns each, so that only 16 TMEM values per
-          // matrix and 16 scales are live at a time
-          const uint32_t col = tmem + lane_base + b * (L::kMats * kN) + cb;
-          mbar_wait(&full_bar[s], (g / kStages) & 1, abort, err, 15);  // the stage's scales are in
+      // this token's scales, one hand-off (2 blocks) per 8-byte load, one hand-off ahead
+      const float2* dp = reinterpret_cast<const float2*>(drow);
+      float2 dnext = valid ? __ldg(dp) : make_float2(0.f, 0.f);
+      for (int j = 0; j < nst; ++j) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const bool live = cb + 16 * h < f.n_pad;  // warp-uniform
-            uint32_t r0[16], r1[16];
-            if (live) {
-              tmem_ld16(col + 16 * h, r0);
-              if constexpr (GU) tmem_ld16(col + kN + 16 * h, r1);
-              tmem_ld_wait();
-            }
-            if (h == 1) {
-              fence_before_sync();
-              mbar_arrive(&tempty_bar[b]);  // TMEM buffer b may be rewritten now
-            }
-            float dv[16];
-            if (live) {
-              const float4* d4p = reinterpret_cast<const float4*>(d_ring + s * kN + cb + 16 * h);
+        for (int hs = 0; hs < kBS / kHalf; ++hs, ++gh) {
+          const float2 dcur = dnext;
+          const int hn = j * (kBS / kHalf) + hs + 1;  // next hand-off of this item
+          if (valid && hn < nst * (kBS / kHalf)) dnext = __ldg(dp + hn);
+          const int hb = gh % (kTBufs / kHalf);
+          // warp-uniform: tcgen05.ld is a warp-wide instruction
+          const bool ok =
+              __all_sync(0xffffffffu, mbar_wait(&tfull_bar[hb], (gh / (kTBufs / kHalf)) & 1, abort, err, 13));
+          fence_after_sync();
+          if (active && ok) {
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float4 d4 = d4p[j];
-                dv[4 * j] = d4.x;
-                dv[4 * j + 1] = d4.y;
-                dv[4 * j + 2] = d4.z;
-                dv[4 * j + 3] = d4.w;
-              }
-            }
-            if (h == 1) mbar_arrive(&dempty_bar[s]);
-            if (live) {
+            for (int i = 0; i < kHalf; ++i) {
+              const float dx = i == 0 ? dcur.x : dcur.y;
+              const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
+              // 8 columns at a time, so that only 8 TMEM values are live
 #pragma unroll
-              for (int j = 0; j < 16; j += 2) {
-                const int jj = 16 * h + j;
-                fma2(acc0[jj], acc0[jj + 1], dv[j], dv[j + 1], __uint_as_float(r0[j]), __uint_as_float(r0[j + 1]));
-                if constexpr (GU)
-                  fma2(acc1[jj], acc1[jj + 1], dv[j], dv[j + 1], __uint_as_float(r1[j]),
-                       __uint_as_float(r1[j + 1]));
+              for (int h = 0; h < 4; ++h) {
+                uint32_t r[8];
+                tmem_ld8(col + c0 + 8 * h, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int jj = 0; jj < 8; jj += 2)
+                  fma2(acc0[8 * h + jj], acc0[8 * h + jj + 1], dx, dx, __uint_as_float(r[jj]),
+                       __uint_as_float(r[jj + 1]));
+                tmem_ld8(col + c1 + 8 * h, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int jj = 0; jj < 8; jj += 2)
+                  fma2(acc1[8 * h + jj], acc1[8 * h + jj + 1], dx, dx, __uint_as_float(r[jj]),
+                       __uint_as_float(r[jj + 1]));
               }
             }
           }
-        } else {
           fence_before_sync();
-          mbar_arrive(&tempty_bar[b]);
-          mbar_arrive(&dempty_bar[s]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty_bar[hb]);  // the pair of TMEM buffers may be rewritten now
         }
       }
-      const bool go = __all_sync(0xffffffffu, !*abort) && active;  // warp-uniform (warp_max below)
-      if (go) {
-        const int o = f.m0 + quad * 32 + lane;
+      const bool go = __all_sync(0xffffffffu, !*abort) && active;  // warp-uniform
+      if (go && valid) {
+        const int64_t row = (int64_t)f.slot.row_base + f.n0 + n;
         if constexpr (GU) {
-          const float sg = tab.gate_s[f.slot.table_idx][o];
-          const float su = tab.up_s[f.slot.table_idx][o];
-          const int pos = (lane & ~7) + op_pos8(lane & 7);
+          const int o = f.m0 + 32 * hh;  // first intermediate row of this thread's Q8 block of h
+          const float* sgp = tab.gate_s[f.slot.table_idx] + o;
+          const float* sup = tab.up_s[f.slot.table_idx] + o;
+          float amax = 0.0f;
 #pragma unroll
-          for (int j = 0; j < kC; ++j) {
-            const int n = cb + j;
-            if (n < f.n_valid) {
-              const float gv = __fmul_rn(sg, acc0[j]);
-              const float u = __fmul_rn(su, acc1[j]);
-              const float h = __fmul_rn(__fmul_rn(gv, sigmoid_cw(gv)), u);
-              const float d = __fdiv_rn(warp_max(fabsf(h)), 127.0f);
-              const int64_t row = (int64_t)f.slot.row_base + f.n0 + n;
-              hf[row * inter + (o - lane) + pos] = __int2half_rn(q8_of(h, d));
-              if (lane == 0) hd[row * (inter / 32) + (o >> 5)] = d;
+          for (int j = 0; j < 32; ++j) {
+            const float gv = __fmul_rn(__ldg(sgp + j), acc0[j]);
+            const float u = __fmul_rn(__ldg(sup + j), acc1[j]);
+            acc0[j] = __fmul_rn(__fmul_rn(gv, sigmoid_cw(gv)), u);
+            amax = fmaxf(amax, fabsf(acc0[j]));
+          }
+          const float d = __fdiv_rn(amax, 127.0f);
+          // fp16 of q in the operand order: position 2(e&3) + (e>>2) of each 8
+          uint32_t pk[16];
+#pragma unroll
+          for (int e8 = 0; e8 < 4; ++e8) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const __half lo = __int2half_rn(q8_of(acc0[8 * e8 + i], d));
+              const __half hi = __int2half_rn(q8_of(acc0[8 * e8 + 4 + i], d));
+              pk[4 * e8 + i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
             }
           }
-        } else {
-          const float sd = tab.down_s[f.slot.table_idx][o];
+          uint4* dst = reinterpret_cast<uint4*>(hf + row * inter + o);
 #pragma unroll
-          for (int j = 0; j < kC; ++j) {
-            const int n = cb + j;
-            if (n < f.n_valid) y[((int64_t)f.slot.row_base + f.n0 + n) * hidden + o] = __fmul_rn(sd, acc0[j]);
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          hd[row * (inter / 32) + (o >> 5)] = d;
+        } else {
+          const float* sdp = tab.down_s[f.slot.table_idx] + f.m0;
+          float4* dst0 = reinterpret_cast<float4*>(y + row * hidden + f.m0 + c0);
+          float4* dst1 = reinterpret_cast<float4*>(y + row * hidden + f.m0 + c1);
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const float4 s0 = __ldg(reinterpret_cast<const float4*>(sdp + c0 + j));
+            const float4 s1 = __ldg(reinterpret_cast<const float4*>(sdp + c1 + j));
+            dst0[j / 4] = make_float4(__fmul_rn(s0.x, acc0[j]), __fmul_rn(s0.y, acc0[j + 1]),
+                                      __fmul_rn(s0.z, acc0[j + 2]), __fmul_rn(s0.w, acc0[j + 3]));
+            dst1[j / 4] = make_float4(__fmul_rn(s1.x, acc1[j]), __fmul_rn(s1.y, acc1[j + 1]),
+                                      __fmul_rn(s1.z, acc1[j + 2]), __fmul_rn(s1.w, acc1[j + 3]));
           }
         }
       }
@@ -458,18 +524,18 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
   __syncthreads();
   if (warp == kMmaWarp) {
     fence_after_sync();
-    tmem_dealloc(tmem, L::kTmemCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
-// Tiles of <= kN tokens over the slot table, in slot order.
+// Tiles of <= kM tokens over the slot table, in slot order.
 __global__ void build_tiles_kernel(const Slot* __restrict__ slots, const int32_t* __restrict__ n_slots,
                                    Tile* __restrict__ tiles, int32_t* __restrict__ n_tiles) {
   if (threadIdx.x != 0) return;
   int j = 0;
   const int ns = *n_slots;
   for (int s = 0; s < ns; ++s)
-    for (int n0 = 0; n0 < slots[s].count; n0 += kN) tiles[j++] = Tile{s, n0};
+    for (int n0 = 0; n0 < slots[s].count; n0 += kM) tiles[j++] = Tile{s, n0};
   *n_tiles = j;
 }
 
@@ -492,7 +558,7 @@ cudaError_t allow_smem(KernelT* k, size_t (&granted)[64], size_t bytes) {
 size_t prefill_tiles_bound(int n_tok, int K, int E, int n_shared) {
   const int64_t pairs = (int64_t)n_tok * (K + n_shared);
   const int64_t slots = (n_tok * (int64_t)K < E ? n_tok * (int64_t)K : E) + n_shared;
-  return (size_t)((pairs + kN - 1) / kN + slots);
+  return (size_t)((pairs + kM - 1) / kM + slots);
 }
 
 size_t prefill_tile_bytes(int n_tok, int K, int E, int n_shared) {
@@ -500,20 +566,53 @@ size_t prefill_tile_bytes(int n_tok, int K, int E, int n_shared) {
 }
 
 bool prefill_supported(int hidden, int inter) {
-  return hidden % kM == 0 && inter % kM == 0 && PSmem<true>::bytes() <= 227 * 1024;
+  // K a whole number of stages (kBS blocks of 32) for both GEMMs; whole column groups
+  return hidden % (32 * kBS) == 0 && inter % (32 * kBS) == 0 && hidden % kN == 0 && inter % (kN / 2) == 0 &&
+         PSmem::bytes() <= 227 * 1024;
 }
+
+namespace {
+
+// A 2D tensor map over `rows` fp16 rows of `cols` values (row-major), box
+// 64 values x kM rows, 128-byte swizzle: the A operand tiles.
+cudaError_t make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int cols) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    cudaDriverEntryPointQueryResult q{};
+    void* fn = nullptr;
+    const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kM};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
 
 cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, const Slot* slots,
                                    const int32_t* n_slots, void* tiles, int32_t* n_tiles, const int32_t* perm,
-                                   int K, const int8_t* xq, const float* xd, int n_tok, int hidden, int inter,
-                                   void* xf, void* hf, float* hd, float* y, int32_t* err, cudaStream_t st,
-                                   cudaEvent_t ev_mid) {
+                                   int K, int n_shared, const int8_t* xq, const float* xd, int n_tok, int hidden,
+                                   int inter, void* xf, void* hf, float* hd, float* y, int32_t* err,
+                                   cudaStream_t st, cudaEvent_t ev_mid) {
   Tile* t = reinterpret_cast<Tile*>(tiles);
-  const int64_t n8 = (int64_t)n_tok * hidden / 8;
-  act_f16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(xq, n8, reinterpret_cast<uint4*>(xf));
+  const int64_t rows = (int64_t)n_tok * (K + n_shared);
+  const int64_t n8 = rows * hidden / 8;
+  act_rows_f16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(xq, perm, n_tok, K, rows, hidden,
+                                                                    reinterpret_cast<uint4*>(xf));
   build_tiles_kernel<<<1, 32, 0, st>>>(slots, n_slots, t, n_tiles);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  CUtensorMap map_x, map_h;
+  if ((e = make_rows_map(&map_x, xf, rows, hidden)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&map_h, hf, rows, inter)) != cudaSuccess) return e;
   static size_t granted_gu[64] = {}, granted_dn[64] = {};
   static int sms_cache[64] = {};
   int dev = 0;
@@ -522,17 +621,17 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
   if (sms_cache[dev] == 0 &&
       (e = cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
-  const size_t sm_gu = PSmem<true>::bytes(), sm_dn = PSmem<false>::bytes();
-  if ((e = allow_smem(prefill_kernel<true, GateUpTable>, granted_gu, sm_gu)) != cudaSuccess) return e;
-  if ((e = allow_smem(prefill_kernel<false, DownTable>, granted_dn, sm_dn)) != cudaSuccess) return e;
+  const size_t smem = PSmem::bytes();
+  if ((e = allow_smem(prefill_kernel<true, GateUpTable>, granted_gu, smem)) != cudaSuccess) return e;
+  if ((e = allow_smem(prefill_kernel<false, DownTable>, granted_dn, smem)) != cudaSuccess) return e;
   const int grid = sms_cache[dev];
   __half* hfh = reinterpret_cast<__half*>(hf);
-  prefill_kernel<true, GateUpTable><<<grid, kThreadsP, sm_gu, st>>>(
-      gu, slots, t, n_tiles, perm, K, reinterpret_cast<const __half*>(xf), xd, hidden, inter, hfh, hd, y, err);
+  prefill_kernel<true, GateUpTable><<<grid, kThreadsP, smem, st>>>(gu, map_x, slots, t, n_tiles, perm, K, xd, hidden,
+                                                                     inter, hfh, hd, y, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecordWithFlags(ev_mid, st, cudaEventRecordExternal)) != cudaSuccess) return e;
-  prefill_kernel<false, DownTable><<<grid, kThreadsP, sm_dn, st>>>(dn, slots, t, n_tiles, perm, K, hfh, hd, hidden,
-                                                                     inter, hfh, hd, y, err);
+  prefill_kernel<false, DownTable><<<grid, kThreadsP, smem, st>>>(dn, map_h, slots, t, n_tiles, perm, K, hd, hidden,
+                                                                    inter, hfh, hd, y, err);
   return cudaGetLastError();
 }
 

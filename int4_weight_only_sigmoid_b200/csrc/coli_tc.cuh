@@ -40,16 +40,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete is suspended
+// until it completes or about `ns` nanoseconds have passed, so waiting
+// threads do not keep polling the shared-memory pipe.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kSleepNs = 20000;  // between checks of the abort flag and the clock
+
 // Wait until the phase with the given parity has completed.  Returns false
 // (after setting *abort and the error word) if it does not complete within
-// kSpinCycles, or at once if another thread of the CTA already aborted.
+// kSpinCycles, or once another thread of the CTA has aborted (seen at the
+// next check, at most ~kSleepNs later).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* err,
                                           int32_t code) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
+    if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
     if (clock64() - t0 > kSpinCycles) {
       *abort = 1;
       if (err) atomicExch(err, code);

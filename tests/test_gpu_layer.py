@@ -56,8 +56,10 @@ def test_layer_tiny(coli, syn, n_tok):
 
 @pytest.mark.parametrize("n_tok", [17, 64, 65, 130, 300, 1000])
 def test_layer_tiny_prefill_path(coli, syn, n_tok):
-    """Tensor-core path (> 16 tokens): ragged tiles of <= 64 tokens, several
-    tiles per expert, partial 16-column MMAs."""
+    """Tensor-core path (> 16 tokens): ragged tiles of <= 128 tokens, several
+    tiles per expert (1000 tokens: ~250 per routed expert, 8 tiles of the
+    shared expert), tiles with a single valid token and with partly filled
+    lane quadrants."""
     _check_layer(coli, syn, syn.config("tiny"), n_tok)
 
 
