@@ -37,16 +37,18 @@
 // (128-byte swizzle).  The packed weights are copied by the producer warps
 // with cp.async and expanded into the B operand (K-major, no swizzle).
 //
-// Roles (416 threads): warps 0-3 producers (thread p: weight row p and token
-// row p of the tile), warp 4 the MMA issuer (lane 0) and TMEM owner, warps
-// 5-12 the fold (warp w reads TMEM lanes 32(w%4).. = 32 of the tile's
-// tokens, and half of the item's columns).  Per block g: the producers copy
-// (kLook blocks ahead, all by cp.async) into operand stage g % kStages
-// (after `empty`, raised by the MMA's commit, and `dempty`, raised by the
-// fold warps once they have read the stage's token scales), expand the
-// weights and arrive on `full`; the MMA writes TMEM buffer g % kTBufs (after
-// `tempty`) and commits `empty` and `tfull`.  All waits are bounded
-// (coli_tc.cuh).
+// Roles (448 threads): warps 0-3 producers (packed-weight copies; thread p
+// expands weight row p), warp 4 the MMA issuer (lane 0) and TMEM owner,
+// warps 5-12 the fold (warp w reads TMEM lanes 32(w%4).. = 32 of the tile's
+// tokens, and half of the item's columns), warp 13 the A-tile TMA loads.
+// An operand stage holds 4 Q8 blocks (K = 128).  Per stage g: the TMA warp
+// loads its A tile into operand stage g % kStages once `empty` (the MMA's
+// commit) says the stage is free; the producers copy its packed weights
+// kLookS stages ahead (cp.async), expand them into the stage's B part and
+// arrive on `full`; the MMA issues two K=16 steps per block into a fresh
+// TMEM accumulator per block (4 of them, handed to the fold two blocks at a
+// time through `tfull` / `tempty`) and commits `empty`.  All waits are
+// bounded (coli_tc.cuh).
 //
 // Sources: "Colibri：在笔记本上跑744B参数的AI模型", "关键特性" (integer dot
 // kernels, Q8_0 activations, packed int4); HN summary (hn.213312.xyz),
@@ -76,7 +78,8 @@ constexpr int kProdWarps = 4;
 constexpr int kEpiWarps = 8;   // 2 per TMEM lane quadrant, each half of the columns
 constexpr int kMmaWarp = kProdWarps;
 constexpr int kEpi0 = kProdWarps + 1;                          // first fold warp
-constexpr int kThreadsP = 32 * (kProdWarps + 1 + kEpiWarps);  // 416
+constexpr int kTmaWarp = kEpi0 + kEpiWarps;                    // A-tile loads
+constexpr int kThreadsP = 32 * (kTmaWarp + 1);                 // 448
 constexpr int kNProd = 32 * kProdWarps;                        // 128 producer threads
 constexpr int kTmemCols = kTBufs * kN;                         // 512
 
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_bar[s], kProdWarps + 1);  // + the TMA issuer's expect_tx
+      mbar_init(&full_bar[s], kProdWarps + 1);  // + the TMA warp's expect_tx
       mbar_init(&empty_bar[s], 1);
     }
     for (int b = 0; b < kTBufs / kHalf; ++b) {
@@ -276,13 +279,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
 
   if (warp < kProdWarps) {
     // ------------------------------------------------------------ producers
-    // A stage's A tile (128 rows of the row-ordered fp16 activations / h,
-    // 4 blocks) is one pair of TMA loads issued by thread 0.  Its packed
-    // weights (128 rows x 64 B) are copied 4 lanes per row, so that each
-    // warp instruction touches few cache lines; thread p then expands weight
-    // row p of the stage's 4 blocks.  The copies run kLookS stages ahead
-    // across item boundaries: the issue cursor (item ii, stage ji) moves
-    // ahead of the expansion.
+    // A stage's packed weights (128 rows x 64 B) are copied 4 lanes per
+    // row, so that each warp instruction touches few cache lines; thread p
+    // then expands weight row p of the stage's 4 blocks into the B operand.
+    // The copies run kLookS stages ahead across item boundaries: the issue
+    // cursor (item ii, stage ji) moves ahead of the expansion.  (The A tiles
+    // come from the TMA warp.)
     const int p = threadIdx.x;
     const size_t rb = (size_t)dim_in / 2;
     const int n_mine = blockIdx.x < n_items ? (n_items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
@@ -300,29 +302,17 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       else
         return tab.down_q[fi.slot.table_idx] + (size_t)(fi.m0 + r) * rb;
     };
-    // copies of the cursor's stage (global stage gj) into operand stage
-    // gj % kStages and pk slot gj % kPkSlots; then the cursor moves on
+    // packed-weight copies of the cursor's stage (global stage gj) into pk
+    // slot gj % kPkSlots; then the cursor moves on
     auto issue = [&](int gj) {
       if (gj < total) {
-        const int s = gj % kStages;
-        if (mbar_wait(&empty_bar[s], ((gj / kStages) & 1) ^ 1, abort, err, 10)) {
-          const int kb0 = ji * kBS;
-          if (p == 0) {
-            unsigned char* oa = op_ring + s * L::kOpStage;
-            const int row0 = fi.slot.row_base + fi.n0;
-            mbar_arrive_expect_tx(&full_bar[s], L::kStageA);
-            tma_load_2d(oa, &amap, kb0 * 32, row0, &full_bar[s]);
-            tma_load_2d(oa + L::kAtomA, &amap, kb0 * 32 + 64, row0, &full_bar[s]);
-          }
-          unsigned char* pk = pk_ring + (gj % kPkSlots) * L::kPk;
+        const int kb0 = ji * kBS;
+        unsigned char* pk = pk_ring + (gj % kPkSlots) * L::kPk;
 #pragma unroll
-          for (int it = 0; it < 4; ++it) {  // W: row it*32 + p/4, chunk p%4 (= block kb0 + p%4)
-            const int q = it * kNProd + p;
-            const int r = q >> 2, c = q & 3;
-            cp_async16(pk + r * 64 + c * 16, wrow(r) + (size_t)(kb0 + c) * 16);
-          }
-        } else if (p == 0) {
-          mbar_arrive(&full_bar[s]);  // keep the arrival count; the CTA is aborting
+        for (int it = 0; it < 4; ++it) {  // W: row it*32 + p/4, chunk p%4 (= block kb0 + p%4)
+          const int q = it * kNProd + p;
+          const int r = q >> 2, c = q & 3;
+          cp_async16(pk + r * 64 + c * 16, wrow(r) + (size_t)(kb0 + c) * 16);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
         if (++ji == nst) {
@@ -342,7 +332,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       asm volatile("cp.async.wait_group %0;" ::"n"(kLookS) : "memory");  // stage gs's copies (this thread's) are in
       named_bar(1, kNProd);                                              // ... and every producer's
       const int s = gs % kStages;
-      if (!*abort) {
+      // the MMA is done with the operand stage's previous contents
+      if (mbar_wait(&empty_bar[s], ((gs / kStages) & 1) ^ 1, abort, err, 10) && !*abort) {
         const uint4* pk = reinterpret_cast<const uint4*>(pk_ring + (gs % kPkSlots) * L::kPk + p * 64);
         unsigned char* ob = op_ring + s * L::kOpStage + L::kStageA;
 #pragma unroll
@@ -404,6 +395,32 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       mma_commit(&done_bar);
       const long long t0 = clock64();
       while (!mbar_try_wait(&done_bar, 0) && clock64() - t0 < kSpinCycles) {
+      }
+    }
+    __syncwarp();
+  } else if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ A tiles
+    // For each stage: once the MMA is done with the operand stage, one
+    // expect_tx arrival on `full` and two TMA loads of 128 rows x 64 fp16
+    // (128-byte swizzle) of the row-ordered activations (gate/up) or h
+    // (down), rows [row_base + n0, +128) of the item's slot.
+    if (lane == 0) {
+      int gs = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
+        const int row0 = f.slot.row_base + f.n0;
+        for (int j = 0; j < nst; ++j, ++gs) {
+          const int s = gs % kStages;
+          if (!mbar_wait(&empty_bar[s], ((gs / kStages) & 1) ^ 1, abort, err, 16)) {
+            ok = false;
+            break;
+          }
+          unsigned char* oa = op_ring + s * L::kOpStage;
+          mbar_arrive_expect_tx(&full_bar[s], L::kStageA);
+          tma_load_2d(oa, &amap, j * kBS * 32, row0, &full_bar[s]);
+          tma_load_2d(oa + L::kAtomA, &amap, j * kBS * 32 + 64, row0, &full_bar[s]);
+        }
       }
     }
     __syncwarp();
