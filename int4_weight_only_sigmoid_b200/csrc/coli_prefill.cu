@@ -38,16 +38,16 @@
 // with cp.async and expanded into the B operand (K-major, no swizzle).
 //
 // Roles (448 threads): warps 0-3 producers (packed-weight copies; thread p
-// expands weight row p), warp 4 the MMA issuer (lane 0) and TMEM owner,
-// warps 5-12 the fold (warp w reads TMEM lanes 32(w%4).. = 32 of the tile's
-// tokens, and half of the item's columns), warp 13 the A-tile TMA loads.
+// expands weight row p), warp 4 the A-tile TMA loads, warps 5-12 the fold
+// (warp w reads TMEM lanes 32(w%4).. = 32 of the tile's tokens, and half of
+// the item's columns), warp 13 the MMA issuer (lane 0) and TMEM owner.
 // An operand stage holds 4 Q8 blocks (K = 128).  Per stage g: the TMA warp
 // loads its A tile into operand stage g % kStages once `empty` (the MMA's
 // commit) says the stage is free; the producers copy its packed weights
 // kLookS stages ahead (cp.async), expand them into the stage's B part and
 // arrive on `full`; the MMA issues two K=16 steps per block into a fresh
-// TMEM accumulator per block (4 of them, handed to the fold two blocks at a
-// time through `tfull` / `tempty`) and commits `empty`.  All waits are
+// TMEM accumulator per block (4 of them, handed to the fold kHalf blocks at
+// a time through `tfull` / `tempty`) and commits `empty`.  All waits are
 // bounded (coli_tc.cuh).
 //
 // Sources: "Colibri：在笔记本上跑744B参数的AI模型", "关键特性" (integer dot
@@ -56,6 +56,7 @@
 // positions is read once and shared).
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <type_traits>
 #include <cuda_fp16.h>
 
 #include "coli_launch.h"
@@ -76,10 +77,13 @@ constexpr int kHalf = 2;       // Q8 blocks per accumulator hand-off (MMA -> fol
 constexpr int kTBufs = 4;      // TMEM accumulators (one per block), handed off in pairs
 constexpr int kProdWarps = 4;
 constexpr int kEpiWarps = 8;   // 2 per TMEM lane quadrant, each half of the columns
-constexpr int kMmaWarp = kProdWarps;
+// Warp w runs on scheduler w % 4 and, as a fold warp, reads TMEM lanes
+// 32 (w % 4)..; the MMA issuer is kept off scheduler 0, which carries the
+// fold of tiles with at most 32 tokens.
+constexpr int kTmaWarp = kProdWarps;                           // A-tile loads
 constexpr int kEpi0 = kProdWarps + 1;                          // first fold warp
-constexpr int kTmaWarp = kEpi0 + kEpiWarps;                    // A-tile loads
-constexpr int kThreadsP = 32 * (kTmaWarp + 1);                 // 448
+constexpr int kMmaWarp = kEpi0 + kEpiWarps;                    // MMA issuer, TMEM owner
+constexpr int kThreadsP = 32 * (kMmaWarp + 1);                 // 448
 constexpr int kNProd = 32 * kProdWarps;                        // 128 producer threads
 constexpr int kTmemCols = kTBufs * kN;                         // 512
 
@@ -205,6 +209,11 @@ __device__ __forceinline__ void fma2(float& a0, float& a1, float d0, float d1, f
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(dd), "l"(xx));
   asm("mov.b64 {%0,%1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
 }
+
+// A fold thread's token scales for one hand-off (kHalf blocks).
+using DVec = std::conditional_t<kHalf == 2, float2, float>;
+[[maybe_unused]] __device__ __forceinline__ float dvec_at(const float2& v, int i) { return i == 0 ? v.x : v.y; }
+[[maybe_unused]] __device__ __forceinline__ float dvec_at(float v, int) { return v; }
 
 struct ItemInfo {
   Slot slot;
@@ -446,13 +455,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         acc0[j] = 0.0f;
         acc1[j] = 0.0f;
       }
-      // this token's scales, one hand-off (2 blocks) per 8-byte load, one hand-off ahead
-      const float2* dp = reinterpret_cast<const float2*>(drow);
-      float2 dnext = valid ? __ldg(dp) : make_float2(0.f, 0.f);
+      // this token's scales, one hand-off (kHalf blocks) per load, one hand-off ahead
+      const DVec* dp = reinterpret_cast<const DVec*>(drow);
+      DVec dnext = valid ? __ldg(dp) : DVec{};
       for (int j = 0; j < nst; ++j) {
 #pragma unroll
         for (int hs = 0; hs < kBS / kHalf; ++hs, ++gh) {
-          const float2 dcur = dnext;
+          const DVec dcur = dnext;
           const int hn = j * (kBS / kHalf) + hs + 1;  // next hand-off of this item
           if (valid && hn < nst * (kBS / kHalf)) dnext = __ldg(dp + hn);
           const int hb = gh % (kTBufs / kHalf);
@@ -463,7 +472,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           if (active && ok) {
 #pragma unroll
             for (int i = 0; i < kHalf; ++i) {
-              const float dx = i == 0 ? dcur.x : dcur.y;
+              const float dx = dvec_at(dcur, i);
               const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
               // 8 columns at a time, so that only 8 TMEM values are live
 #pragma unroll

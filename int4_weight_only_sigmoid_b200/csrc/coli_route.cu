@@ -40,6 +40,91 @@ __global__ void __launch_bounds__(256) router_scores_kernel(const float* __restr
   if (lane == 0) scores[gw] = sigmoid_cw(logit);
 }
 
+// Router scores for many tokens: a CTA of 8 warps owns a tile of 16 tokens
+// x 16 experts and stages both sets of rows through shared memory in
+// chunks of 512 values (cp.async, two chunks in flight), so each row is read
+// from L2 once per tile instead of once per dot product.  Warp w folds 4
+// tokens x 8 experts (32 accumulators per lane); lane l still owns
+// accumulator l of contract R (float4 number l + 32j of the row, ascending
+// j), and the 32 lane partials of each dot are summed left to right by one
+// lane after a transpose through shared memory.
+constexpr int kRtTok = 16, kRtExp = 16, kRtChunk = 128;  // chunk: float4 per row
+__global__ void __launch_bounds__(256) router_tiled_kernel(const float* __restrict__ x,
+                                                           const float* __restrict__ wr, int n_tok, int E, int H,
+                                                           float* __restrict__ scores) {
+  extern __shared__ __align__(16) float4 rsm[];  // [2][(kRtTok + kRtExp) * kRtChunk]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * kRtTok, e0 = blockIdx.y * kRtExp;
+  const int nq = H / 4, n_chunks = nq / kRtChunk;
+  constexpr int kRows = kRtTok + kRtExp;
+  auto load_chunk = [&](int c, int buf) {
+    float4* dst = rsm + buf * kRows * kRtChunk;
+    for (int i = threadIdx.x; i < kRows * kRtChunk; i += blockDim.x) {
+      const int r = i / kRtChunk, j = i - r * kRtChunk;
+      const bool is_x = r < kRtTok;
+      const int g = is_x ? t0 + r : e0 + (r - kRtTok);
+      if (g < (is_x ? n_tok : E)) {
+        const float* src = (is_x ? x : wr) + (int64_t)g * H + 4 * (c * kRtChunk + j);
+        cp_async16(dst + i, src);
+      } else {
+        dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  const int tw = (warp >> 1) * 4, ew = (warp & 1) * 8;  // this warp's 4 tokens, 8 experts within the tile
+  float acc[4][8];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+  load_chunk(0, 0);
+  for (int c = 0; c < n_chunks; ++c) {
+    if (c + 1 < n_chunks) {
+      load_chunk(c + 1, (c + 1) & 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+    const float4* xs = rsm + (c & 1) * kRows * kRtChunk;
+    const float4* ws = xs + kRtTok * kRtChunk;
+#pragma unroll
+    for (int k = 0; k < kRtChunk / 32; ++k) {
+      const int j = 32 * k + lane;
+      float4 xv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) xv[a] = xs[(tw + a) * kRtChunk + j];
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        const float4 wv = ws[(ew + b) * kRtChunk + j];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          acc[a][b] = __fmaf_rn(xv[a].x, wv.x, acc[a][b]);
+          acc[a][b] = __fmaf_rn(xv[a].y, wv.y, acc[a][b]);
+          acc[a][b] = __fmaf_rn(xv[a].z, wv.z, acc[a][b]);
+          acc[a][b] = __fmaf_rn(xv[a].w, wv.w, acc[a][b]);
+        }
+      }
+    }
+    __syncthreads();  // the buffer is refilled by the next iteration's copies
+  }
+  // transpose: red[d][l] = lane l's partial of dot d; lane d then sums its row left to right
+  float* red = reinterpret_cast<float*>(rsm) + warp * 32 * 33;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) red[(a * 8 + b) * 33 + lane] = acc[a][b];
+  __syncwarp();
+  const int t = t0 + tw + (lane >> 3), e = e0 + ew + (lane & 7);
+  float logit = red[lane * 33];
+#pragma unroll
+  for (int l = 1; l < 32; ++l) logit = __fadd_rn(logit, red[lane * 33 + l]);
+  if (t < n_tok && e < E) scores[(int64_t)t * E + e] = sigmoid_cw(logit);
+}
+
+size_t router_tiled_smem() { return (size_t)2 * (kRtTok + kRtExp) * kRtChunk * sizeof(float4); }
+
 // One warp per token.
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ scores,
                                                    const float* __restrict__ bias, int n_tok, int E, int K,
@@ -283,6 +368,21 @@ size_t bucket_smem_bytes(int E) { return (size_t)E * (5 + 64) * sizeof(int); }
 
 cudaError_t launch_router_scores(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
                                  cudaStream_t st) {
+  if (n_tok >= 64 && H % (4 * kRtChunk) == 0) {
+    static int attr_dev_mask = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (!(attr_dev_mask & (1 << (dev & 31)))) {
+      e = cudaFuncSetAttribute(router_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)router_tiled_smem());
+      if (e != cudaSuccess) return e;
+      attr_dev_mask |= 1 << (dev & 31);
+    }
+    const dim3 grid((unsigned)((n_tok + kRtTok - 1) / kRtTok), (unsigned)((E + kRtExp - 1) / kRtExp));
+    router_tiled_kernel<<<grid, 256, router_tiled_smem(), st>>>(x, w_router, n_tok, E, H, scores);
+    return cudaGetLastError();
+  }
   const int64_t warps = (int64_t)n_tok * E;
   const int64_t blocks = (warps + 7) / 8;
   router_scores_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, w_router, n_tok, E, H, scores);
