@@ -474,22 +474,21 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
             for (int i = 0; i < kHalf; ++i) {
               const float dx = dvec_at(dcur, i);
               const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
-              // 8 columns at a time, so that only 8 TMEM values are live
+              // 8 columns of each range at a time (one wait per pair of
+              // loads), so that only 16 TMEM values are live
 #pragma unroll
               for (int h = 0; h < 4; ++h) {
-                uint32_t r[8];
-                tmem_ld8(col + c0 + 8 * h, r);
+                uint32_t r0[8], r1[8];
+                tmem_ld8(col + c0 + 8 * h, r0);
+                tmem_ld8(col + c1 + 8 * h, r1);
                 tmem_ld_wait();
 #pragma unroll
-                for (int jj = 0; jj < 8; jj += 2)
-                  fma2(acc0[8 * h + jj], acc0[8 * h + jj + 1], dx, dx, __uint_as_float(r[jj]),
-                       __uint_as_float(r[jj + 1]));
-                tmem_ld8(col + c1 + 8 * h, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int jj = 0; jj < 8; jj += 2)
-                  fma2(acc1[8 * h + jj], acc1[8 * h + jj + 1], dx, dx, __uint_as_float(r[jj]),
-                       __uint_as_float(r[jj + 1]));
+                for (int jj = 0; jj < 8; jj += 2) {
+                  fma2(acc0[8 * h + jj], acc0[8 * h + jj + 1], dx, dx, __uint_as_float(r0[jj]),
+                       __uint_as_float(r0[jj + 1]));
+                  fma2(acc1[8 * h + jj], acc1[8 * h + jj + 1], dx, dx, __uint_as_float(r1[jj]),
+                       __uint_as_float(r1[jj + 1]));
+                }
               }
             }
           }
