@@ -26,7 +26,9 @@
  *  - Host-detectable errors (null or misaligned pointers, unsupported
  *    shapes, a workspace that is too small) return COLI_EINVAL at once and
  *    enqueue nothing; a failed launch returns COLI_ECUDA.  coli_last_error()
- *    then gives a message (per calling thread).
+ *    then gives a message (per calling thread).  Device-side problems are
+ *    recorded in the workspace's status word and reported by
+ *    coli_sync_status.
  *  - n_tok == 0 is a no-op that returns COLI_OK.
  *  - Weights are row-major [out x in]; an int4 row is in/2 bytes, element
  *    2j in the low nibble of byte j, two's complement, plus one F32 scale.
@@ -197,6 +199,26 @@ coli_status coli_moe_layer_forward_noalloc(const coli_moe_layer* layer, const fl
  * kernel.  The events must be created by the caller (with timing enabled);
  * the call consumes the arming.  Always returns COLI_OK. */
 coli_status coli_debug_phase_events(void* before_experts, void* after_gateup, void* after_down);
+
+/* Device-side errors of the forward calls made on `workspace` (NULL: the
+ * fixed scratch of coli_moe_layer_forward_noalloc on the current device).
+ * The first 4 bytes of a workspace are a status word: each
+ * coli_moe_layer_forward / coli_moe_stack_forward call clears it when its
+ * first kernel starts, and its kernels record the first problem they meet
+ * instead of trapping.  This call synchronises `stream`, reads the word and
+ * returns COLI_OK (0: no problem), COLI_EDEVICE (1..9: a device-side check
+ * failed, e.g. an expert index outside [0, n_experts) in bucketing) or
+ * COLI_ETIMEOUT (>= 10: a bounded wait gave up, about a second after the
+ * awaited data should have arrived; the kernel then finished without the
+ * rest of its work).  coli_last_error() names the code.  The word is left
+ * as it is.  COLI_ECUDA if the synchronisation or the read fails. */
+coli_status coli_sync_status(void* workspace, void* stream);
+
+/* Test hook for the path above: enqueues one thread that waits on a
+ * shared-memory barrier nothing arrives at, for at most `cycles` SM clock
+ * cycles (0 .. 4e9), and then records status code 30 in `workspace`'s
+ * status word.  No fault and no hang: the wait is bounded. */
+coli_status coli_debug_wait_probe(void* workspace, int64_t cycles, void* stream);
 
 #ifdef __cplusplus
 }

@@ -24,7 +24,7 @@ EXPORTS = [
     "coli_quantize_rows_int4", "coli_quantize_act_q8", "coli_moe_route", "coli_moe_bucket",
     "coli_moe_expert_ffn", "coli_moe_layer_forward", "coli_moe_stack_forward", "coli_rmsnorm",
     "coli_moe_workspace_bytes", "coli_last_error", "coli_debug_block_partials",
-    "coli_debug_phase_events", "coli_moe_layer_forward_noalloc",
+    "coli_debug_phase_events", "coli_moe_layer_forward_noalloc", "coli_sync_status", "coli_debug_wait_probe",
 ]
 
 
@@ -80,6 +80,8 @@ def load(path: str | None = None):
         "coli_debug_block_partials": (st, [C.POINTER(Expert), i32, vp, i64, i64, i64, vp, vp]),
         "coli_debug_phase_events": (st, [vp, vp, vp]),
         "coli_moe_layer_forward_noalloc": (st, [C.POINTER(MoeLayerC), vp, i64, vp, vp]),
+        "coli_sync_status": (st, [vp, vp]),
+        "coli_debug_wait_probe": (st, [vp, i64, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -280,3 +282,15 @@ def moe_layer_forward_noalloc(layer: MoeLayer, x, out=None, stream=None, cstruct
     Lc = layer.cstruct() if cstruct is None else cstruct
     _check(lib().coli_moe_layer_forward_noalloc(C.byref(Lc), _ptr(x), x.shape[0], _ptr(o), _stream(stream)))
     return o
+
+
+def sync_status(workspace=None, stream=None) -> int:
+    """Synchronise `stream` and return the coli_status of the device-side
+    status word of `workspace` (None: the no-allocation scratch); the
+    message is in coli_last_error()."""
+    return lib().coli_sync_status(_ptr(workspace), _stream(stream))
+
+
+def debug_wait_probe(workspace, cycles: int, stream=None):
+    """Enqueue the bounded-wait test probe (records status code 30)."""
+    _check(lib().coli_debug_wait_probe(_ptr(workspace), int(cycles), _stream(stream)))

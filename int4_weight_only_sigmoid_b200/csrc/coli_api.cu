@@ -7,6 +7,7 @@
 
 #include "../../include/coli.h"
 #include "coli_launch.h"
+#include "coli_tc.cuh"
 
 #define COLI_EXPORT extern "C" __attribute__((visibility("default")))
 
@@ -108,6 +109,7 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
     off = align256(off + (bytes ? bytes : 1));
     return at;
   };
+  L.status = take(4);  // first, at offset 0: coli_sync_status reads it without knowing T
   L.xq = take(T * H);
   L.xd = take(T * (H / 32) * 4);
   L.scores = take(T * E * 4);
@@ -119,7 +121,6 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   L.inv = take(T * K * 4);
   L.slots = take((size_t)kMaxSlots * sizeof(Slot));
   L.n_slots = take(4);
-  L.status = take(4);
   L.tiles = take(prefill_tile_bytes((int)T, (int)K, (int)E, (int)S));
   L.n_tiles = take(4);
   L.hq = take(rows * I);
@@ -154,8 +155,10 @@ void fill_tables(const coli_moe_layer* L, GateUpTable& gu, DownTable& dn) {
 }
 
 // The layer forward on a validated layer, x -> out, scratch in ws.
+// clear_status: this call starts the workspace's status word afresh (the
+// first layer of a forward call).
 coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, float* out, void* ws,
-                          const Workspace& W, cudaStream_t st, const char* fn) {
+                          const Workspace& W, cudaStream_t st, const char* fn, bool clear_status) {
   const coli_moe_config& c = L->cfg;
   const int H = c.hidden, I = c.inter, E = c.n_experts, K = c.top_k, S = c.n_shared;
   int8_t* xq = at<int8_t>(ws, W.xq);
@@ -184,7 +187,8 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   int32_t* status = at<int32_t>(ws, W.status);
   if (T <= kDecodeMaxTok && decode_supported(H, I)) {
     // decode: 5 kernels, the last four launched with PDL
-    CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, xq, xd, st));
+    CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, xq, xd, clear_status ? status : nullptr,
+                                      st));
     CHECK_LAUNCH(launch_topk_bucket_small(scores, L->bias, (int)T, E, K, c.norm_topk_prob, c.routed_scaling_factor,
                                           idx, wts, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm, inv,
                                           slots, n_slots, st));
@@ -196,6 +200,7 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
     return COLI_OK;
   }
 
+  if (clear_status) CHECK_LAUNCH(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
   CHECK_LAUNCH(launch_quantize_act_q8(x, T, H, xq, xd, st));
   CHECK_LAUNCH(launch_router_scores(x, L->w_router, (int)T, E, H, scores, st));
   CHECK_LAUNCH(launch_topk(scores, L->bias, (int)T, E, K, c.norm_topk_prob, c.routed_scaling_factor, idx, wts, st));
@@ -243,6 +248,67 @@ COLI_EXPORT coli_status coli_debug_phase_events(void* before_experts, void* afte
 COLI_EXPORT size_t coli_moe_workspace_bytes(const coli_moe_config* cfg, int64_t max_tokens) {
   if (check_cfg(cfg, "coli_moe_workspace_bytes") != COLI_OK || max_tokens < 0) return 0;
   return layout(*cfg, max_tokens).total;
+}
+
+namespace coli {
+namespace {
+
+const char* status_meaning(int32_t code) {
+  switch (code) {
+    case kStatusBadExpert: return "bucketing met an expert index outside [0, n_experts)";
+    case 10: return "prefill producers gave up waiting for an operand stage";
+    case 11: return "prefill MMA issuer gave up waiting for operands";
+    case 12: return "prefill MMA issuer gave up waiting for accumulator buffers";
+    case 13: return "prefill fold gave up waiting for accumulators";
+    case 16: return "prefill A-tile loader gave up waiting for an operand stage";
+    case 22: return "decode down kernel gave up waiting for h rows";
+    case kStatusWaitProbe: return "test probe: a wait that nothing completes gave up";
+    default: return code >= kStatusTimeoutFirst ? "a bounded wait gave up" : "a device-side check failed";
+  }
+}
+
+// Test probe: one thread waits on an mbarrier that nothing arrives at, for
+// at most `cycles` clock cycles, then records kStatusWaitProbe.
+__global__ void wait_probe_kernel(int32_t* status, long long cycles) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  tc::mbar_init(&bar, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  const long long t0 = clock64();
+  bool done = false;
+  while (!(done = tc::mbar_try_wait_sleep(&bar, 0, 1000)) && clock64() - t0 < cycles) {
+  }
+  if (!done) atomicExch(status, kStatusWaitProbe);
+}
+
+}  // namespace
+}  // namespace coli
+
+COLI_EXPORT coli_status coli_sync_status(void* workspace, void* stream) {
+  const char* fn = "coli_sync_status";
+  void* ws = workspace;
+  if (ws == nullptr) {
+    coli_status s = cuda_status(noalloc_scratch(&ws), fn);
+    if (s != COLI_OK) return s;
+  } else {
+    CHECK_PTR(workspace);
+  }
+  CHECK_LAUNCH(cudaStreamSynchronize((cudaStream_t)stream));
+  int32_t code = 0;
+  CHECK_LAUNCH(cudaMemcpy(&code, ws, sizeof code, cudaMemcpyDeviceToHost));
+  if (code == 0) return COLI_OK;
+  return fail(code >= kStatusTimeoutFirst ? COLI_ETIMEOUT : COLI_EDEVICE, "%s: device status %d: %s", fn, (int)code,
+              status_meaning(code));
+}
+
+COLI_EXPORT coli_status coli_debug_wait_probe(void* workspace, int64_t cycles, void* stream) {
+  const char* fn = "coli_debug_wait_probe";
+  CHECK_PTR(workspace);
+  if (cycles < 0 || cycles > (int64_t)4000000000LL)
+    return fail(COLI_EINVAL, "%s: cycles=%lld outside [0, 4e9]", fn, (long long)cycles);
+  wait_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(static_cast<int32_t*>(workspace), (long long)cycles);
+  CHECK_LAUNCH(cudaGetLastError());
+  return COLI_OK;
 }
 
 COLI_EXPORT coli_status coli_quantize_rows_int4(const float* w, int64_t rows, int64_t cols, uint8_t* q_out,
@@ -364,7 +430,7 @@ COLI_EXPORT coli_status coli_moe_layer_forward(const coli_moe_layer* layer, cons
   const Workspace W = layout(layer->cfg, n_tok);
   if (ws_bytes < W.total)
     return fail(COLI_ENOMEM, "%s: workspace %zu bytes < %zu needed", fn, ws_bytes, W.total);
-  return layer_forward(layer, x, n_tok, out, workspace, W, (cudaStream_t)stream, fn);
+  return layer_forward(layer, x, n_tok, out, workspace, W, (cudaStream_t)stream, fn, true);
 }
 
 COLI_EXPORT coli_status coli_moe_stack_forward(const coli_moe_layer* layers, int32_t n_layers, const float* x,
@@ -395,7 +461,7 @@ COLI_EXPORT coli_status coli_moe_stack_forward(const coli_moe_layer* layers, int
     // ping[l % 2] never holds `cur` (which is x or ping[(l - 1) % 2])
     float* m = ping[l % 2];
     CHECK_LAUNCH(launch_rmsnorm(cur, (int)n_tok, H, eps, xn, st));
-    if ((s = layer_forward(&layers[l], xn, n_tok, m, workspace, W, st, fn)) != COLI_OK) return s;
+    if ((s = layer_forward(&layers[l], xn, n_tok, m, workspace, W, st, fn, l == 0)) != COLI_OK) return s;
     float* next = (l == n_layers - 1) ? out : m;  // m = cur + m in place, or the final output
     CHECK_LAUNCH(launch_residual_add(cur, m, n_tok * H, next, st));
     cur = next;

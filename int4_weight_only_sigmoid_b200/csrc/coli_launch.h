@@ -48,7 +48,7 @@ cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E
 // Decode batches: router scores with the router rows staged in shared memory
 // (plain launch), then top-k + weights + bucketing in one CTA (PDL launch).
 cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
-                                 int8_t* xq, float* xd, cudaStream_t st);
+                                 int8_t* xq, float* xd, int32_t* status_clear, cudaStream_t st);
 cudaError_t launch_topk_bucket_small(const float* scores, const float* bias, int n_tok, int E, int K, int norm,
                                      float rsf, int32_t* idx, float* w, int32_t* counts, int32_t* offsets,
                                      int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, cudaStream_t st);
@@ -121,5 +121,23 @@ cudaError_t launch_debug_partials(const uint8_t* wq, const int8_t* xq, int n_tok
 
 // Sets the message coli_last_error() returns on the calling thread.
 void set_error_message(const char* msg);
+
+// Device status word: the first 4 bytes of a workspace.  A forward call
+// clears it when it starts; kernels record the first problem they meet.
+//   0            no error
+//   1 .. 9       a device-side check failed (COLI_EDEVICE):
+//                1 = bucketing met an expert index outside [0, E)
+//   10 .. 39     a bounded wait gave up (COLI_ETIMEOUT):
+//                10 prefill producers (operand stage), 11 prefill MMA (operands),
+//                12 prefill MMA (accumulators), 13 prefill fold (accumulators),
+//                16 prefill TMA warp (operand stage), 22 decode down (h rows),
+//                30 the test probe coli_debug_wait_probe
+constexpr int32_t kStatusBadExpert = 1;
+constexpr int32_t kStatusTimeoutFirst = 10;
+constexpr int32_t kStatusWaitProbe = 30;
+
+// Device address of the fixed scratch behind coli_moe_layer_forward_noalloc
+// on the current device.
+cudaError_t noalloc_scratch(void** out);
 
 }  // namespace coli

@@ -150,6 +150,11 @@ __device__ __forceinline__ uint4 expand_int8_pair(uint32_t a, uint32_t b) {
   return o;
 }
 
+// Byte offset of packed block c (0..3) of weight row r in a stage's packed
+// copy: 64 B per row, blocks rotated by (r >> 1) & 3 so that 8 consecutive
+// rows reading the same block hit 8 different bank groups.
+__device__ __forceinline__ uint32_t pk_off(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
+
 // Byte offset of 16-byte chunk c (0..3) of row r in a K-major, no-swizzle
 // operand tile of 32 fp16 per row: 8-row x 16-byte core matrices, the four
 // K chunks of an 8-row group 128 B apart (LBO), groups 512 B apart (SBO).
@@ -321,7 +326,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         for (int it = 0; it < 4; ++it) {  // W: row it*32 + p/4, chunk p%4 (= block kb0 + p%4)
           const int q = it * kNProd + p;
           const int r = q >> 2, c = q & 3;
-          cp_async16(pk + r * 64 + c * 16, wrow(r) + (size_t)(kb0 + c) * 16);
+          cp_async16(pk + pk_off(r, c), wrow(r) + (size_t)(kb0 + c) * 16);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
         if (++ji == nst) {
@@ -343,11 +348,11 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       const int s = gs % kStages;
       // the MMA is done with the operand stage's previous contents
       if (mbar_wait(&empty_bar[s], ((gs / kStages) & 1) ^ 1, abort, err, 10) && !*abort) {
-        const uint4* pk = reinterpret_cast<const uint4*>(pk_ring + (gs % kPkSlots) * L::kPk + p * 64);
+        const unsigned char* pk = pk_ring + (gs % kPkSlots) * L::kPk;
         unsigned char* ob = op_ring + s * L::kOpStage + L::kStageA;
 #pragma unroll
         for (int c = 0; c < kBS; ++c) {
-          const uint4 w = pk[c];
+          const uint4 w = *reinterpret_cast<const uint4*>(pk + pk_off(p, c));
           unsigned char* dst = ob + c * L::kSubB;
           *reinterpret_cast<uint4*>(dst + op_off(p, 0)) = expand_int4_word(w.x);
           *reinterpret_cast<uint4*>(dst + op_off(p, 1)) = expand_int4_word(w.y);

@@ -152,8 +152,11 @@ constexpr int kStageTok = 2;
 __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restrict__ x,
                                                             const float* __restrict__ wr, int n_tok, int E, int H,
                                                             float* __restrict__ scores, int8_t* __restrict__ xq,
-                                                            float* __restrict__ xd) {
+                                                            float* __restrict__ xd, int32_t* status_clear) {
   extern __shared__ __align__(16) float4 wsm[];  // [2][H/4] router rows, then [kStageTok][H/4] tokens
+  // first kernel of a decode forward (launched without PDL, so everything
+  // before it in the stream is complete): start the status word afresh
+  if (status_clear && blockIdx.x == 0 && threadIdx.x == 0) *status_clear = 0;
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e0 = blockIdx.x * 2;
@@ -295,7 +298,7 @@ __global__ void __launch_bounds__(kBucketThreads) bucket_kernel(const int32_t* _
     if (e >= 0 && e < E) {
       atomicAdd(&cnt[e], 1);
     } else if (status) {
-      atomicExch(status, 1);
+      atomicExch(status, kStatusBadExpert);
     }
   }
   __syncthreads();
@@ -396,7 +399,7 @@ cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E
 }
 
 cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
-                                 int8_t* xq, float* xd, cudaStream_t st) {
+                                 int8_t* xq, float* xd, int32_t* status_clear, cudaStream_t st) {
   const size_t smem = (size_t)(2 + (n_tok <= kStageTok ? n_tok : 0)) * H * sizeof(float);
   static int attr_dev_mask = 0;
   int dev = 0;
@@ -406,7 +409,7 @@ cudaError_t launch_router_decode(const float* x, const float* w_router, int n_to
     if (e != cudaSuccess) return e;
     attr_dev_mask |= 1 << (dev & 31);
   }
-  router_decode_kernel<<<(E + 1) / 2, 256, smem, st>>>(x, w_router, n_tok, E, H, scores, xq, xd);
+  router_decode_kernel<<<(E + 1) / 2, 256, smem, st>>>(x, w_router, n_tok, E, H, scores, xq, xd, status_clear);
   return cudaGetLastError();
 }
 

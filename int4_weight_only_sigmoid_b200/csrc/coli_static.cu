@@ -47,6 +47,8 @@ cudaError_t scratch_on_current_device(void** out) {
 
 }  // namespace
 
+cudaError_t coli::noalloc_scratch(void** out) { return scratch_on_current_device(out); }
+
 COLI_EXPORT coli_status coli_moe_layer_forward_noalloc(const coli_moe_layer* layer, const float* x, int64_t n_tok,
                                                        float* out, void* stream) {
   char msg[320];

@@ -66,6 +66,9 @@ def test_bad_arguments_rejected_before_any_cuda_call(lib):
     assert lib.coli_rmsnorm(None, 1, 100, 1e-5, None, None) == m.COLI_EINVAL
     assert lib.coli_debug_block_partials(None, 0, None, 1, 64, 1, None, None) == m.COLI_EINVAL
     assert lib.coli_moe_stack_forward(None, 0, None, 1, 1e-5, None, None, 0, None) == m.COLI_EINVAL
+    assert lib.coli_debug_wait_probe(None, 1000, None) == m.COLI_EINVAL
+    assert lib.coli_debug_wait_probe(C.c_void_p(256), -1, None) == m.COLI_EINVAL
+    assert lib.coli_sync_status(C.c_void_p(8), None) == m.COLI_EINVAL  # misaligned workspace
 
 
 def test_zero_tokens_is_ok_without_touching_pointers(lib):
