@@ -100,6 +100,22 @@ typedef struct {
 coli_status coli_quantize_rows_int4(const float* w, int64_t rows, int64_t cols, uint8_t* q_out,
                                     float* scale_out, void* stream);
 
+/* FP8 -> int4 requantiser, the offline converter's step on the GPU
+ * ([W] "GLM-5.2-colibri-int4的量化流程": the source model is FP8 e4m3,
+ * dequantised to F32, then quantised per row as coli_quantize_rows_int4;
+ * its config gives weight_block_size [128, 128]).
+ * w8 [rows x cols] e4m3 codes (bit 7 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits; 0x7F / 0xFF are NaN); block_factors
+ * [ceil(rows/block) x ceil(cols/block)] F32, row-major: element (r, c) is
+ * e4m3(w8[r, c]) * block_factors[r / block, c / block] (one F32 multiply;
+ * the stored factor multiplies the code's value), and an element whose
+ * product is not finite counts as 0.  Outputs as coli_quantize_rows_int4:
+ * q_out [rows x cols/2] packed int4, scale_out [rows] F32.
+ * cols % 32 == 0; block a positive multiple of 8 (128 for the GLM-5.2 FP8
+ * checkpoint).  Integer and F32 results are exact (bit-reproducible). */
+coli_status coli_requantize_fp8_int4(const uint8_t* w8, const float* block_factors, int64_t rows, int64_t cols,
+                                     int32_t block, uint8_t* q_out, float* scale_out, void* stream);
+
 /* Q8_0-style activation quantiser ([C] "关键特性": Q8_0 风格 int8 激活).
  * Per 32-element block of each token: d = absmax/127 (F32);
  * q = rint(x/d) clamped to [-127,127]; an all-zero block gets d = 0.

@@ -25,6 +25,7 @@ EXPORTS = [
     "coli_moe_expert_ffn", "coli_moe_layer_forward", "coli_moe_stack_forward", "coli_rmsnorm",
     "coli_moe_workspace_bytes", "coli_last_error", "coli_debug_block_partials",
     "coli_debug_phase_events", "coli_moe_layer_forward_noalloc", "coli_sync_status", "coli_debug_wait_probe",
+    "coli_requantize_fp8_int4",
 ]
 
 
@@ -82,6 +83,7 @@ def load(path: str | None = None):
         "coli_moe_layer_forward_noalloc": (st, [C.POINTER(MoeLayerC), vp, i64, vp, vp]),
         "coli_sync_status": (st, [vp, vp]),
         "coli_debug_wait_probe": (st, [vp, i64, vp]),
+        "coli_requantize_fp8_int4": (st, [vp, vp, i64, i64, i32, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -164,6 +166,18 @@ def quantize_rows_int4(w, q_out=None, s_out=None, stream=None):
     q = torch.empty(rows, cols // 2, dtype=torch.uint8, device=w.device) if q_out is None else q_out
     s = torch.empty(rows, dtype=torch.float32, device=w.device) if s_out is None else s_out
     _check(lib().coli_quantize_rows_int4(_ptr(w), rows, cols, _ptr(q), _ptr(s), _stream(stream)))
+    return q, s
+
+
+def requantize_fp8_int4(w8, block_factors, block: int = 128, stream=None):
+    """FP8 e4m3 codes (uint8 [rows x cols], device) with per-tile F32
+    factors -> (packed int4 [rows x cols/2] uint8, row scales [rows] F32)."""
+    import torch
+    rows, cols = w8.shape
+    q = torch.empty(rows, cols // 2, dtype=torch.uint8, device=w8.device)
+    s = torch.empty(rows, dtype=torch.float32, device=w8.device)
+    _check(lib().coli_requantize_fp8_int4(_ptr(w8), _ptr(block_factors), rows, cols, int(block), _ptr(q), _ptr(s),
+                                          _stream(stream)))
     return q, s
 
 

@@ -325,6 +325,25 @@ COLI_EXPORT coli_status coli_quantize_rows_int4(const float* w, int64_t rows, in
   return COLI_OK;
 }
 
+COLI_EXPORT coli_status coli_requantize_fp8_int4(const uint8_t* w8, const float* block_factors, int64_t rows,
+                                                 int64_t cols, int32_t block, uint8_t* q_out, float* scale_out,
+                                                 void* stream) {
+  const char* fn = "coli_requantize_fp8_int4";
+  if (rows < 0 || cols <= 0 || cols % 32 != 0 || rows > (int64_t(1) << 31))
+    return fail(COLI_EINVAL, "%s: rows=%lld cols=%lld (cols must be a positive multiple of 32)", fn,
+                (long long)rows, (long long)cols);
+  if (block < 8 || block % 8 != 0)
+    return fail(COLI_EINVAL, "%s: block=%d (must be a positive multiple of 8)", fn, (int)block);
+  if (rows == 0) return COLI_OK;
+  CHECK_PTR(w8);
+  CHECK_PTR(block_factors);
+  CHECK_PTR(q_out);
+  CHECK_PTR(scale_out);
+  CHECK_LAUNCH(launch_requantize_fp8_int4(w8, block_factors, rows, cols, block, q_out, scale_out,
+                                          (cudaStream_t)stream));
+  return COLI_OK;
+}
+
 COLI_EXPORT coli_status coli_quantize_act_q8(const float* x, int64_t n_tok, int64_t dim, int8_t* q_out,
                                              float* scale_out, void* stream) {
   const char* fn = "coli_quantize_act_q8";

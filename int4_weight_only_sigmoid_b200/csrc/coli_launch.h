@@ -36,6 +36,10 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Quantisers
 cudaError_t launch_quantize_rows_int4(const float* w, int64_t rows, int64_t cols, uint8_t* q,
                                       float* s, cudaStream_t st);
+// FP8 (e4m3 codes, [rows x cols]) with one F32 factor per block x block tile
+// -> packed int4 rows + F32 row scales.  cols % 32 == 0, block % 8 == 0.
+cudaError_t launch_requantize_fp8_int4(const uint8_t* w8, const float* factors, int64_t rows, int64_t cols,
+                                       int block, uint8_t* q, float* s, cudaStream_t st);
 cudaError_t launch_quantize_act_q8(const float* x, int64_t n_tok, int64_t dim, int8_t* q, float* d,
                                    cudaStream_t st);
 

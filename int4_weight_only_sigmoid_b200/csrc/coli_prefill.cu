@@ -558,15 +558,29 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
   }
 }
 
-// Tiles of <= kM tokens over the slot table, in slot order.
+// Tiles of <= kM tokens over the slot table, in slot order.  One warp:
+// rounds of 32 slots, a shuffle scan of their tile counts gives each lane
+// where its slot's tiles go.
 __global__ void build_tiles_kernel(const Slot* __restrict__ slots, const int32_t* __restrict__ n_slots,
                                    Tile* __restrict__ tiles, int32_t* __restrict__ n_tiles) {
-  if (threadIdx.x != 0) return;
-  int j = 0;
+  const int lane = threadIdx.x;
+  if (lane >= 32) return;
   const int ns = *n_slots;
-  for (int s = 0; s < ns; ++s)
-    for (int n0 = 0; n0 < slots[s].count; n0 += kM) tiles[j++] = Tile{s, n0};
-  *n_tiles = j;
+  int base = 0;
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    const int s = s0 + lane;
+    const int cnt = s < ns ? slots[s].count : 0;
+    const int nt = (cnt + kM - 1) / kM;
+    int incl = nt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    for (int i = 0; i < nt; ++i) tiles[base + incl - nt + i] = Tile{s, i * kM};
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) *n_tiles = base;
 }
 
 // Opt the kernel in to `bytes` of dynamic shared memory on the current

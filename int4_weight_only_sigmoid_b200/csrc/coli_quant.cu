@@ -49,6 +49,75 @@ __global__ void __launch_bounds__(256) quantize_rows_int4_kernel(const float* __
   if (lane == 0) s[row] = scale;
 }
 
+// FP8 -> int4 requantiser (the converter: "GLM-5.2-colibri-int4架构解析…",
+// "GLM-5.2-colibri-int4的量化流程": FP8 e4m3 source -> F32 -> int4 per
+// row; config weight_block_size [128, 128]).  e4m3 code -> F32, exact:
+// bit 7 sign, bits 6..3 exponent (bias 7), bits 2..0 mantissa; exponent 0
+// is subnormal (m * 2^-9); 0x7F / 0xFF are NaN (no infinities).
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  float v;
+  if (e == 15u && m == 7u)
+    v = __int_as_float(0x7fc00000);
+  else if (e == 0u)
+    v = __fmul_rn((float)m, 0x1p-9f);
+  else
+    v = __int_as_float((int)(((e + 120u) << 23) | (m << 20)));
+  return (b & 0x80u) ? -v : v;
+}
+
+// Element value: e4m3 * the factor of its block x block tile (one F32
+// multiply); a non-finite product (NaN code, overflow) counts as 0.
+__device__ __forceinline__ float fp8_element(uint32_t code, float factor) {
+  const float v = __fmul_rn(e4m3_value(code), factor);
+  return fabsf(v) <= 3.402823466e38f ? v : 0.0f;
+}
+
+// One warp per row, 8 codes (one 8-byte load, one block factor: block is a
+// multiple of 8) per lane step; absmax pass, then the int4 row rule of
+// quantize_rows_int4_kernel on the same values.
+__global__ void __launch_bounds__(256) requantize_fp8_int4_kernel(const uint8_t* __restrict__ w8,
+                                                                  const float* __restrict__ factors, int64_t rows,
+                                                                  int64_t cols, int block, uint8_t* __restrict__ q,
+                                                                  float* __restrict__ s) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int64_t bcols = (cols + block - 1) / block;
+  const uint2* wr = reinterpret_cast<const uint2*>(w8 + row * cols);
+  const float* fr = factors + (row / block) * bcols;
+  float amax = 0.0f;
+  for (int64_t g = lane; g < cols / 8; g += 32) {
+    const uint2 c = __ldg(wr + g);
+    const float f = __ldg(fr + (8 * g) / block);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      amax = fmaxf(amax, fabsf(fp8_element((c.x >> (8 * i)) & 0xFFu, f)));
+      amax = fmaxf(amax, fabsf(fp8_element((c.y >> (8 * i)) & 0xFFu, f)));
+    }
+  }
+  amax = warp_max(amax);
+  const float scale = __fdiv_rn(amax, 7.0f);
+  uint32_t* qr = reinterpret_cast<uint32_t*>(q + row * (cols / 2));
+  for (int64_t g = lane; g < cols / 8; g += 32) {
+    const uint2 c = __ldg(wr + g);
+    const float f = __ldg(fr + (8 * g) / block);
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t code = ((i < 4 ? c.x : c.y) >> (8 * (i & 3))) & 0xFFu;
+      int qi = 0;
+      if (amax != 0.0f) {
+        qi = (int)rintf(__fdiv_rn(fp8_element(code, f), scale));
+        qi = qi < -8 ? -8 : (qi > 7 ? 7 : qi);
+      }
+      word |= ((uint32_t)qi & 0xFu) << (4 * i);
+    }
+    qr[g] = word;
+  }
+  if (lane == 0) s[row] = scale;
+}
+
 // One warp per 32-element block.
 __global__ void __launch_bounds__(256) quantize_act_q8_kernel(const float* __restrict__ x, int64_t n_blocks,
                                                               int8_t* __restrict__ q, float* __restrict__ d) {
@@ -126,6 +195,13 @@ int blocks_for(int64_t items, int per_block) {
 cudaError_t launch_quantize_rows_int4(const float* w, int64_t rows, int64_t cols, uint8_t* q, float* s,
                                       cudaStream_t st) {
   quantize_rows_int4_kernel<<<blocks_for(rows, 8), 256, 0, st>>>(w, rows, cols, q, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_requantize_fp8_int4(const uint8_t* w8, const float* factors, int64_t rows, int64_t cols,
+                                       int block, uint8_t* q, float* s, cudaStream_t st) {
+  const int64_t blocks = (rows + 7) / 8;
+  requantize_fp8_int4_kernel<<<(unsigned)blocks, 256, 0, st>>>(w8, factors, rows, cols, block, q, s);
   return cudaGetLastError();
 }
 

@@ -56,6 +56,8 @@ def lib():
             ("ora_unpack_int4", None, [vp, i64, vp]),
             ("ora_quantize_rows_int4", None, [vp, i64, i64, vp, vp]),
             ("ora_quantize_act_q8", None, [vp, i64, i64, vp, vp]),
+            ("ora_e4m3_to_f32", f32, [C.c_uint8]),
+            ("ora_requantize_fp8_int4", None, [vp, vp, i64, i64, i64, vp, vp]),
             ("ora_router_logit", f32, [vp, vp, i64]),
             ("ora_route", None, [vp, vp, vp, i64, i64, i64, i32, i32, f32, vp, vp, vp]),
             ("ora_bucket", None, [vp, i64, i32, i32, vp, vp, vp]),
@@ -171,6 +173,26 @@ def quantize_rows_int4(w: np.ndarray):
     q = np.empty((rows, cols // 2), np.uint8)
     s = np.empty(rows, np.float32)
     lib().ora_quantize_rows_int4(_p(w), rows, cols, _p(q), _p(s))
+    return q, s
+
+
+def e4m3_to_f32(codes) -> np.ndarray:
+    """Values of e4m3 byte codes (NaN for 0x7F / 0xFF)."""
+    c = np.asarray(codes, np.uint8).ravel()
+    return np.array([lib().ora_e4m3_to_f32(int(b)) for b in c], np.float32).reshape(np.shape(codes))
+
+
+def requantize_fp8_int4(w8: np.ndarray, block_scale: np.ndarray, block: int = 128):
+    """FP8 (e4m3 codes, [rows x cols] uint8) with per-block F32 factors
+    ([ceil(rows/block) x ceil(cols/block)]) -> packed int4 rows + F32 row
+    scales (the converter's flow: dequantise to F32, then int4 per row)."""
+    w8 = np.ascontiguousarray(w8, np.uint8)
+    rows, cols = w8.shape
+    bs = np.ascontiguousarray(block_scale, np.float32)
+    assert bs.shape == (-(-rows // block), -(-cols // block))
+    q = np.empty((rows, cols // 2), np.uint8)
+    s = np.empty(rows, np.float32)
+    lib().ora_requantize_fp8_int4(_p(w8), _p(bs), rows, cols, block, _p(q), _p(s))
     return q, s
 
 

@@ -62,6 +62,7 @@
  * With those flags every float expression is one binary32 operation,
  * round-to-nearest-even, in the order written.
  */
+#include <float.h>
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -198,6 +199,49 @@ ORA_API void ora_quantize_rows_int4(const float* w, int64_t rows, int64_t cols, 
         ora_pack_int4(q, cols, q_out + r * (cols / 2));
     }
     free(q);
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP8 -> int4 requantiser ([W] "GLM-5.2-colibri-int4的量化流程": the source */
+/* is the FP8 (e4m3) model, dequantised to F32 and then quantised per row as */
+/* above; its config: fmt e4m3, weight_block_size [128, 128])                */
+/* ------------------------------------------------------------------------ */
+
+/* e4m3 ("fn" variant: no infinities): bit 7 sign, bits 6..3 exponent with
+ * bias 7, bits 2..0 mantissa.  Exponent 0: subnormal, (m/8) * 2^-6.
+ * Exponent 15 with mantissa 7: NaN.  Otherwise (1 + m/8) * 2^(e-7).
+ * Every code is exact in F32. */
+ORA_API float ora_e4m3_to_f32(uint8_t b) {
+    const int sign = (b >> 7) & 1, e = (b >> 3) & 15, m = b & 7;
+    float v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexpf((float)m / 8.0f, -6);
+    else
+        v = ldexpf(1.0f + (float)m / 8.0f, e - 7);
+    return sign ? -v : v;
+}
+
+/* Reading (the pages give the flow, not the arithmetic): element (r, c) of
+ * the F32 matrix is e4m3(w8[r, c]) * block_scale[r / block, c / block], one
+ * F32 multiply (DeepSeek-V3's weight_scale_inv convention: the stored factor
+ * multiplies the FP8 value); an element whose product is not finite (a NaN
+ * code, or an overflow) counts as 0; then each row is quantised to int4
+ * exactly as ora_quantize_rows_int4.  block_scale is
+ * [ceil(rows/block) x ceil(cols/block)], row-major. */
+ORA_API void ora_requantize_fp8_int4(const uint8_t* w8, const float* block_scale, int64_t rows, int64_t cols,
+                                     int64_t block, uint8_t* q_out, float* scale_out) {
+    const int64_t bcols = (cols + block - 1) / block;
+    float* row = (float*)malloc((size_t)cols * sizeof(float));
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t c = 0; c < cols; ++c) {
+            float v = ora_e4m3_to_f32(w8[r * cols + c]) * block_scale[(r / block) * bcols + c / block];
+            if (!(fabsf(v) <= FLT_MAX)) v = 0.0f;
+            row[c] = v;
+        }
+        ora_quantize_rows_int4(row, 1, cols, q_out + r * (cols / 2), scale_out + r);
+    }
+    free(row);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -42,6 +42,8 @@ TID_ROUTER = 1
 TID_BIAS = 2
 TID_X = 3
 TID_X_BASE = 4
+TID_FP8_CODES = 5
+TID_FP8_SCALES = 6
 _E_MAX = 4096
 GATE, UP, DOWN = 0, 1, 2
 
@@ -164,6 +166,18 @@ def uniform(n: int, seed: int, layer: int, tid: int, a: float, b: float, i0: int
     out = np.empty(n, np.float32)
     _host().synth_uniform(out.ctypes.data, n, i0, key(seed, layer, tid), a, b)
     return out
+
+
+def fp8_blocks(rows: int, cols: int, block: int = 128, seed: int = 0, lo: float = 1e-4, hi: float = 1e-2):
+    """Synthetic FP8 weights for the FP8 -> int4 converter: e4m3 byte codes
+    uniform over all 256 codes (NaN codes included) and one F32 factor per
+    block x block tile, uniform in [lo, hi) (the scale range of DeepSeek-V3
+    style FP8 checkpoints).  Returns (codes uint8 [rows x cols], factors
+    [ceil(rows/block) x ceil(cols/block)])."""
+    codes = np.floor(uniform(rows * cols, seed, 0, TID_FP8_CODES, 0.0, 256.0)).astype(np.uint8)
+    nb = (-(-rows // block), -(-cols // block))
+    scales = uniform(nb[0] * nb[1], seed, 0, TID_FP8_SCALES, lo, hi)
+    return codes.reshape(rows, cols), scales.reshape(nb)
 
 
 def normal_rows(rows, cols: int, seed: int, layer: int, tid: int, sigma: float) -> np.ndarray:

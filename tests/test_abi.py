@@ -66,6 +66,11 @@ def test_bad_arguments_rejected_before_any_cuda_call(lib):
     assert lib.coli_rmsnorm(None, 1, 100, 1e-5, None, None) == m.COLI_EINVAL
     assert lib.coli_debug_block_partials(None, 0, None, 1, 64, 1, None, None) == m.COLI_EINVAL
     assert lib.coli_moe_stack_forward(None, 0, None, 1, 1e-5, None, None, 0, None) == m.COLI_EINVAL
+    assert lib.coli_requantize_fp8_int4(None, None, 4, 40, 128, None, None, None) == m.COLI_EINVAL
+    assert b"multiple of 32" in lib.coli_last_error()
+    assert lib.coli_requantize_fp8_int4(None, None, 4, 64, 12, None, None, None) == m.COLI_EINVAL
+    assert b"block" in lib.coli_last_error()
+    assert lib.coli_requantize_fp8_int4(None, None, 0, 64, 128, None, None, None) == m.COLI_OK
     assert lib.coli_debug_wait_probe(None, 1000, None) == m.COLI_EINVAL
     assert lib.coli_debug_wait_probe(C.c_void_p(256), -1, None) == m.COLI_EINVAL
     assert lib.coli_sync_status(C.c_void_p(8), None) == m.COLI_EINVAL  # misaligned workspace

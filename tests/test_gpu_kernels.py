@@ -174,3 +174,17 @@ def test_expert_ffn(coli, ora, syn, name, n_tok):
     yo = ora.expert_ffn(oracle_expert(cfg, 0, 0), xq, xd)
     assert_layer_close(y, yo)
     assert bits_equal(y, yo)
+
+
+@pytest.mark.parametrize("rows,cols,block", [(1, 32, 128), (130, 256, 128), (6144, 2048, 128), (257, 160, 64),
+                                             (40, 96, 8)])
+def test_requantize_fp8_int4_bit_exact(coli, ora, syn, rows, cols, block):
+    """The FP8 -> int4 converter step: packed bytes and row scales equal the
+    oracle's bit for bit (ragged tiles, NaN codes and a GLM down-matrix
+    shape included)."""
+    import torch
+    codes, factors = syn.fp8_blocks(rows, cols, block, seed=7 * rows + cols)
+    q, s = coli.requantize_fp8_int4(torch.from_numpy(codes).cuda(), torch.from_numpy(factors).cuda(), block)
+    q_ref, s_ref = ora.requantize_fp8_int4(codes, factors, block)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
