@@ -198,7 +198,7 @@ coli_status coli_debug_block_partials(const coli_expert* expert, int32_t which, 
  * scratch need (coli_moe_workspace_bytes(&layer->cfg, n_tok)) exceeds 8 MiB
  * is rejected with COLI_EINVAL and a message naming both sizes -- e.g. the
  * GLM-5.2 shape (hidden 6144, inter 2048, 256 experts, top-8, 1 shared)
- * fits up to 25 tokens per call.  The first call on each device
+ * fits up to 17 tokens per call.  The first call on each device
  * looks up the array's device address with that device current; make that
  * first call before any stream capture.  Every call shares the one array,
  * so calls that can overlap on the GPU (different streams, or different

@@ -121,11 +121,13 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   L.inv = take(T * K * 4);
   L.slots = take((size_t)kMaxSlots * sizeof(Slot));
   L.n_slots = take(4);
-  L.tiles = take(prefill_tile_bytes((int)T, (int)K, (int)E, (int)S));
+  // the tensor-core prefill path's buffers only when a call of T tokens takes that path
+  const bool tc = (T > kDecodeMaxTok || !decode_supported((int)H, (int)I)) && prefill_supported((int)H, (int)I);
+  L.tiles = take(tc ? prefill_tile_bytes((int)T, (int)K, (int)E, (int)S) : 0);
   L.n_tiles = take(4);
   L.hq = take(rows * I);
-  L.xf = take(rows * H * 2);
-  L.hf = take(rows * I * 2);
+  L.xf = take(tc ? rows * H * 2 : 0);
+  L.hf = take(tc ? rows * I * 2 : 0);
   L.hd = take(rows * (I / 32) * 4);
   L.y = take(rows * H * 4);
   L.xn = take(T * H * 4);
