@@ -21,7 +21,8 @@ def _close(got, want, rel=2e-3):
     assert err <= rel * np.sqrt((want ** 2).mean()), err
 
 
-@pytest.mark.parametrize("name,n_tok", [("tiny", 8), ("tiny", 3), ("decode1", 1), ("decode16", 16)])
+@pytest.mark.parametrize("name,n_tok", [("tiny", 8), ("tiny", 3), ("tiny", 40), ("decode1", 1), ("decode16", 16),
+                                        ("decode16", 17)])  # 17 GLM tokens: the tensor-core path, the documented limit
 def test_noalloc_matches_workspace_forward_twice(coli, syn, name, n_tok):
     import torch
     from synth.layers import device_layer
