@@ -30,6 +30,11 @@
  *    recorded in the workspace's status word and reported by
  *    coli_sync_status.
  *  - n_tok == 0 is a no-op that returns COLI_OK.
+ *  - The first call of a forward path on a device sets kernel attributes
+ *    (shared-memory opt-ins) and looks up the tensor-map encoder; make one
+ *    call of each path (decode: <= 16 tokens, prefill: more) before capturing
+ *    calls into a CUDA graph.  Captured calls replay the device pointers and
+ *    sizes they were captured with.
  *  - Weights are row-major [out x in]; an int4 row is in/2 bytes, element
  *    2j in the low nibble of byte j, two's complement, plus one F32 scale.
  *  - Results follow the written float-evaluation contracts (router R, row
