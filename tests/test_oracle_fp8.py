@@ -64,3 +64,18 @@ def test_requantize_special_rows(ora):
     assert s[1] == 0.0 and not q[1].any()
     assert s[2] == np.float32(224.0) / np.float32(7.0) and q[2, 0] == 0x07 and not q[2, 1:].any()
     assert s[3] == np.float32(0.5) / np.float32(7.0) and (q[3] == 0x77).all()
+
+
+def test_requantize_overflowing_products_count_as_zero(ora):
+    """A tile factor so large that e4m3 * factor overflows F32: those
+    elements count as 0 (the same rule as NaN codes); finite ones keep
+    their values."""
+    codes = np.zeros((1, 64), np.uint8)
+    codes[0, 0] = 0x7E          # 448 * 1e37 = inf in F32 -> 0
+    codes[0, 1] = 0x01          # 2^-9 * 1e37, finite
+    factors = np.array([[1e37]], np.float32)
+    q, s = ora.requantize_fp8_int4(codes, factors, 128)
+    v = np.float32(2.0 ** -9) * np.float32(1e37)
+    assert s[0] == v / np.float32(7.0)
+    assert q[0, 0] == 0x70      # element 0 -> 0 (low nibble), element 1 -> 7 (high nibble)
+    assert not q[0, 1:].any()
