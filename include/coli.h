@@ -134,7 +134,8 @@ coli_status coli_quantize_act_q8(const float* x, int64_t n_tok, int64_t dim, int
  * experts by scores + bias (ties to the lower index) in rank order go to
  * topk_idx [n_tok x top_k]; topk_w [n_tok x top_k] gets the unbiased scores,
  * divided by their sum when norm_topk_prob, times routed_scaling_factor.
- * scores [n_tok x n_experts] is an output too (the caller's buffer). */
+ * scores [n_tok x n_experts] is an optional output: pass NULL to keep the
+ * scores on chip (one kernel; idx and w are the same bits either way). */
 coli_status coli_moe_route(const coli_moe_layer* layer, const float* x, int64_t n_tok, float* scores,
                            int32_t* topk_idx, float* topk_w, void* stream);
 
@@ -151,7 +152,11 @@ coli_status coli_moe_bucket(const int32_t* topk_idx, int64_t n_tok, int32_t top_
  * h re-quantised to Q8_0, y = down.h.  xq [n_tok x hidden] int8,
  * xs [n_tok x hidden/32] F32, y_out [n_tok x hidden] F32.  `expert` points
  * to ONE host-side coli_expert.  Workspace: coli_moe_workspace_bytes(cfg,
- * n_tok) bytes is always enough. */
+ * n_tok) bytes is always enough.  This is the reference-shape entry point:
+ * it runs the general expert kernels (one CTA per 32 outputs), which follow
+ * the same contracts and give the same bits as the layer forward's streaming
+ * and tensor-core kernels, but it is not the tuned path and carries no
+ * performance claim. */
 coli_status coli_moe_expert_ffn(const coli_moe_config* cfg, const coli_expert* expert, const int8_t* xq,
                                 const float* xs, int64_t n_tok, float* y_out, void* workspace,
                                 size_t ws_bytes, void* stream);
@@ -171,7 +176,9 @@ coli_status coli_moe_stack_forward(const coli_moe_layer* layers, int32_t n_layer
                                    size_t ws_bytes, void* stream);
 
 /* RMSNorm alone (weight 1): y = x * (1/sqrtf(sum(x^2)/dim + eps)), the sum
- * an fmaf chain in ascending element order.  x, y: [n_tok x dim]. */
+ * of squares evaluated by contract R (element i feeds accumulator
+ * (i/4) mod 32, each an fmaf chain in ascending i from +0, then the 32
+ * accumulators added left to right); dim % 128 == 0.  x, y: [n_tok x dim]. */
 coli_status coli_rmsnorm(const float* x, int64_t n_tok, int64_t dim, float eps, float* y, void* stream);
 
 /* Bytes of workspace that coli_moe_layer_forward, coli_moe_stack_forward and
@@ -203,9 +210,12 @@ coli_status coli_debug_block_partials(const coli_expert* expert, int32_t which, 
  * scratch need (coli_moe_workspace_bytes(&layer->cfg, n_tok)) exceeds 8 MiB
  * is rejected with COLI_EINVAL and a message naming both sizes -- e.g. the
  * GLM-5.2 shape (hidden 6144, inter 2048, 256 experts, top-8, 1 shared)
- * fits up to 17 tokens per call.  The first call on each device
- * looks up the array's device address with that device current; make that
- * first call before any stream capture.  Every call shares the one array,
+ * fits up to 17 tokens per call.  n_tok outside [0, 2^24] is rejected with
+ * COLI_EINVAL before any size is computed.  The first call on each device
+ * looks up the array's device address with that device current and keeps
+ * it for the life of the process (a device reset invalidates it: do not call
+ * this entry point on a device after cudaDeviceReset); make that first call
+ * before any stream capture.  Every call shares the one array,
  * so calls that can overlap on the GPU (different streams, or different
  * host threads on one device) race: order them on one stream.  The array
  * keeps the last call's contents; nothing in it needs to start at zero.

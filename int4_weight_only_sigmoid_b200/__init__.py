@@ -190,11 +190,13 @@ def quantize_act_q8(x, stream=None):
     return q, d
 
 
-def moe_route(layer: MoeLayer, x, stream=None):
+def moe_route(layer: MoeLayer, x, stream=None, with_scores: bool = True):
+    """(scores, idx, w); with_scores=False passes no scores buffer (the
+    library keeps them on chip) and returns scores=None."""
     import torch
     T = x.shape[0]
     E, K = layer.cfg.n_experts, layer.cfg.top_k
-    scores = torch.empty(T, E, dtype=torch.float32, device=x.device)
+    scores = torch.empty(T, E, dtype=torch.float32, device=x.device) if with_scores else None
     idx = torch.empty(T, K, dtype=torch.int32, device=x.device)
     w = torch.empty(T, K, dtype=torch.float32, device=x.device)
     Lc = layer.cstruct()

@@ -371,11 +371,16 @@ COLI_EXPORT coli_status coli_moe_route(const coli_moe_layer* layer, const float*
   CHECK_PTR(layer->w_router);
   CHECK_PTR(layer->bias);
   CHECK_PTR(x);
-  CHECK_PTR(scores);
   CHECK_PTR(topk_idx);
   CHECK_PTR(topk_w);
   const coli_moe_config& c = layer->cfg;
   cudaStream_t st = (cudaStream_t)stream;
+  if (scores == nullptr) {  // the scores stay on chip
+    CHECK_LAUNCH(launch_route_topk(x, layer->w_router, layer->bias, (int)n_tok, c.n_experts, c.hidden, c.top_k,
+                                   c.norm_topk_prob, c.routed_scaling_factor, topk_idx, topk_w, st));
+    return COLI_OK;
+  }
+  CHECK_PTR(scores);
   CHECK_LAUNCH(launch_router_scores(x, layer->w_router, (int)n_tok, c.n_experts, c.hidden, scores, st));
   CHECK_LAUNCH(launch_topk(scores, layer->bias, (int)n_tok, c.n_experts, c.top_k, c.norm_topk_prob,
                            c.routed_scaling_factor, topk_idx, topk_w, st));

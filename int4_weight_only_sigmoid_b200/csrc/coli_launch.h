@@ -33,6 +33,21 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Set a kernel's dynamic shared-memory opt-in once per device (the
+// attribute belongs to the device's context); `mask` is the caller's
+// per-kernel record of the devices done (devices 0..63).
+template <typename KernelT>
+cudaError_t smem_opt_in_once(KernelT* kernel, int bytes, uint64_t& mask) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (mask & (uint64_t(1) << dev)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) mask |= uint64_t(1) << dev;
+  return e;
+}
+
 // Quantisers
 cudaError_t launch_quantize_rows_int4(const float* w, int64_t rows, int64_t cols, uint8_t* q,
                                       float* s, cudaStream_t st);
@@ -48,6 +63,10 @@ cudaError_t launch_router_scores(const float* x, const float* w_router, int n_to
                                  float* scores, cudaStream_t st);
 cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E, int K, int norm,
                         float rsf, int32_t* idx, float* w, cudaStream_t st);
+// Scores and top-k in one kernel (one CTA per token, scores only in shared
+// memory): the same idx and w as launch_router_scores + launch_topk.
+cudaError_t launch_route_topk(const float* x, const float* w_router, const float* bias, int n_tok, int E, int H, int K,
+                              int norm, float rsf, int32_t* idx, float* w, cudaStream_t st);
 
 // Decode batches: router scores with the router rows staged in shared memory
 // (plain launch), then top-k + weights + bucketing in one CTA (PDL launch).

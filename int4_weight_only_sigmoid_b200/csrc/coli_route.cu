@@ -140,6 +140,44 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
   if (lane == 0) topk_weights(sel, ssel, K, norm, rsf, idx + (int64_t)t * K, wout + (int64_t)t * K);
 }
 
+// Router scores and top-k of one token per CTA, the scores kept in shared
+// memory only (coli_moe_route called without a scores buffer).  Warp w
+// computes experts w, w + 8, ... with the lane mapping and order of
+// router_scores_kernel (contract R), so the scores, and hence the choice,
+// are the same bits.
+constexpr int kRouteThreads = 256;
+__global__ void __launch_bounds__(kRouteThreads) route_topk_kernel(const float* __restrict__ x,
+                                                                   const float* __restrict__ wr,
+                                                                   const float* __restrict__ bias, int E, int H,
+                                                                   int K, int norm, float rsf,
+                                                                   int32_t* __restrict__ idx,
+                                                                   float* __restrict__ wout) {
+  __shared__ float s_sc[kMaxExperts];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x;
+  const float4* xp = reinterpret_cast<const float4*>(x + (int64_t)t * H);
+  for (int e = warp; e < E; e += kRouteThreads / 32) {
+    const float4* wp = reinterpret_cast<const float4*>(wr + (int64_t)e * H);
+    float acc = 0.0f;
+    for (int j = lane; j < H / 4; j += 32) {
+      const float4 a = __ldg(xp + j);
+      const float4 b = __ldg(wp + j);
+      acc = __fmaf_rn(a.x, b.x, acc);
+      acc = __fmaf_rn(a.y, b.y, acc);
+      acc = __fmaf_rn(a.z, b.z, acc);
+      acc = __fmaf_rn(a.w, b.w, acc);
+    }
+    const float logit = warp_sum_in_lane_order(acc);
+    if (lane == 0) s_sc[e] = sigmoid_cw(logit);
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  int sel[kMaxTopK];
+  float ssel[kMaxTopK];
+  warp_select_topk_by([](int e) { return s_sc[e]; }, bias, E, K, lane, sel, ssel);
+  if (lane == 0) topk_weights(sel, ssel, K, norm, rsf, idx + (int64_t)t * K, wout + (int64_t)t * K);
+}
+
 // ---------------------------------------------------------------------------
 // Decode batches (n_tok <= kDecodeMaxTok): two kernels.
 
@@ -372,16 +410,9 @@ size_t bucket_smem_bytes(int E) { return (size_t)E * (5 + 64) * sizeof(int); }
 cudaError_t launch_router_scores(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
                                  cudaStream_t st) {
   if (n_tok >= 64 && H % (4 * kRtChunk) == 0) {
-    static int attr_dev_mask = 0;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static uint64_t attr_dev_mask = 0;
+    const cudaError_t e = smem_opt_in_once(router_tiled_kernel, (int)router_tiled_smem(), attr_dev_mask);
     if (e != cudaSuccess) return e;
-    if (!(attr_dev_mask & (1 << (dev & 31)))) {
-      e = cudaFuncSetAttribute(router_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)router_tiled_smem());
-      if (e != cudaSuccess) return e;
-      attr_dev_mask |= 1 << (dev & 31);
-    }
     const dim3 grid((unsigned)((n_tok + kRtTok - 1) / kRtTok), (unsigned)((E + kRtExp - 1) / kRtExp));
     router_tiled_kernel<<<grid, 256, router_tiled_smem(), st>>>(x, w_router, n_tok, E, H, scores);
     return cudaGetLastError();
@@ -389,6 +420,12 @@ cudaError_t launch_router_scores(const float* x, const float* w_router, int n_to
   const int64_t warps = (int64_t)n_tok * E;
   const int64_t blocks = (warps + 7) / 8;
   router_scores_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, w_router, n_tok, E, H, scores);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_topk(const float* x, const float* w_router, const float* bias, int n_tok, int E, int H, int K,
+                              int norm, float rsf, int32_t* idx, float* w, cudaStream_t st) {
+  route_topk_kernel<<<n_tok, kRouteThreads, 0, st>>>(x, w_router, bias, E, H, K, norm, rsf, idx, w);
   return cudaGetLastError();
 }
 
@@ -401,14 +438,9 @@ cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E
 cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
                                  int8_t* xq, float* xd, int32_t* status_clear, cudaStream_t st) {
   const size_t smem = (size_t)(2 + (n_tok <= kStageTok ? n_tok : 0)) * H * sizeof(float);
-  static int attr_dev_mask = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!(attr_dev_mask & (1 << (dev & 31)))) {
-    cudaError_t e = cudaFuncSetAttribute(router_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_dev_mask |= 1 << (dev & 31);
-  }
+  static uint64_t attr_dev_mask = 0;
+  const cudaError_t e = smem_opt_in_once(router_decode_kernel, 200 * 1024, attr_dev_mask);
+  if (e != cudaSuccess) return e;
   router_decode_kernel<<<(E + 1) / 2, 256, smem, st>>>(x, w_router, n_tok, E, H, scores, xq, xd, status_clear);
   return cudaGetLastError();
 }
@@ -424,13 +456,9 @@ cudaError_t launch_bucket(const int32_t* idx, int n_tok, int K, int E, int n_sha
                           int32_t* offsets, int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots,
                           int32_t* status, cudaStream_t st) {
   const size_t smem = bucket_smem_bytes(E);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)bucket_smem_bytes(kMaxExperts));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static uint64_t attr_dev_mask = 0;  // the opt-in is per device
+  const cudaError_t e = smem_opt_in_once(bucket_kernel, (int)bucket_smem_bytes(kMaxExperts), attr_dev_mask);
+  if (e != cudaSuccess) return e;
   bucket_kernel<<<1, kBucketThreads, smem, st>>>(idx, n_tok, K, E, n_shared, counts, offsets, perm, inv, slots,
                                                   n_slots, status);
   return cudaGetLastError();

@@ -28,7 +28,10 @@ std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch on the current device (looked up once per
-// device, with that device current).
+// device, with that device current).  The cached address assumes that the
+// device's primary context lives as long as the process: after
+// cudaDeviceReset the module is loaded afresh, so a process that resets a
+// device must not call the no-allocation forward on it again.
 cudaError_t scratch_on_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -54,6 +57,13 @@ COLI_EXPORT coli_status coli_moe_layer_forward_noalloc(const coli_moe_layer* lay
   char msg[320];
   if (layer == nullptr) {
     coli::set_error_message("coli_moe_layer_forward_noalloc: null layer");
+    return COLI_EINVAL;
+  }
+  // the token range of coli_moe_layer_forward, checked before the scratch
+  // need is computed (its size arithmetic is only meaningful inside it)
+  if (n_tok < 0 || n_tok > (int64_t(1) << 24)) {
+    snprintf(msg, sizeof msg, "coli_moe_layer_forward_noalloc: n_tok=%lld outside [0, 2^24]", (long long)n_tok);
+    coli::set_error_message(msg);
     return COLI_EINVAL;
   }
   const size_t need = coli_moe_workspace_bytes(&layer->cfg, n_tok);

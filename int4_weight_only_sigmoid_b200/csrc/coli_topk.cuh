@@ -38,14 +38,16 @@ __device__ __forceinline__ int warp_exclusive_scan(int* v, int n, int lane) {
 
 // Warp-wide top-k of one token: K rounds of an argmax over scores + bias
 // (ties to the lower expert index).  Every lane returns the same sel[0..K)
-// and the selected unbiased scores ssel[0..K).
-__device__ __forceinline__ void warp_select_topk(const float* st, const float* __restrict__ bias, int E, int K,
-                                                 int lane, int (&sel)[kMaxTopK], float (&ssel)[kMaxTopK]) {
+// and the selected unbiased scores ssel[0..K).  score(e) gives the token's
+// score of expert e.
+template <typename ScoreAt>
+__device__ __forceinline__ void warp_select_topk_by(ScoreAt score, const float* __restrict__ bias, int E, int K,
+                                                    int lane, int (&sel)[kMaxTopK], float (&ssel)[kMaxTopK]) {
   float v[kMaxExperts / 32], sv[kMaxExperts / 32];
 #pragma unroll
   for (int i = 0; i < kMaxExperts / 32; ++i) {
     const int e = lane + 32 * i;
-    sv[i] = e < E ? ld_dep(st + e) : 0.0f;
+    sv[i] = e < E ? score(e) : 0.0f;
     v[i] = e < E ? __fadd_rn(sv[i], bias[e]) : 0.0f;
   }
   uint32_t taken = 0;
@@ -80,6 +82,13 @@ __device__ __forceinline__ void warp_select_topk(const float* st, const float* _
     ssel[k] = bs;
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
   }
+}
+
+// The same over a score row in global memory that an earlier kernel of the
+// forward wrote (read through L2).
+__device__ __forceinline__ void warp_select_topk(const float* st, const float* __restrict__ bias, int E, int K,
+                                                 int lane, int (&sel)[kMaxTopK], float (&ssel)[kMaxTopK]) {
+  warp_select_topk_by([st](int e) { return ld_dep(st + e); }, bias, E, K, lane, sel, ssel);
 }
 
 // Weights of the selected experts (one lane): denom = s_r0 + s_r1 + ...

@@ -31,6 +31,25 @@ def oracle_layer_forward(cfg: dict, x: np.ndarray, layer: int = 0):
     return out, idx, w, scores
 
 
+def oracle_stack_forward(cfg: dict, x: np.ndarray, n_layers: int, expert_fn=None) -> np.ndarray:
+    """The pre-norm stack by the oracle: for l = 0..n_layers-1,
+    x <- x + MoE_l(RMSNorm(x)) (layer l's seeded weights).  expert_fn(layer,
+    e, shared) may supply the experts instead of the generator."""
+    eps = cfg.get("rms_eps", 1e-5)
+    xo = np.ascontiguousarray(x, np.float32)
+    for l in range(n_layers):
+        xn = oracle.rmsnorm(xo, eps)
+        if expert_fn is None:
+            m, _, _, _ = oracle_layer_forward(cfg, xn, l)
+        else:
+            W, b = synth.router_w(cfg, l), synth.bias(cfg, l)
+            experts = {e: expert_fn(l, e, False) for e in range(cfg["n_experts"])}
+            shared = [expert_fn(l, s, True) for s in range(cfg["n_shared"])]
+            m, _, _ = oracle.moe_layer(cfg, W, b, experts, shared, xn)
+        xo = oracle.residual_add(xo, m)
+    return xo
+
+
 def rms(a) -> float:
     a = np.asarray(a, np.float64)
     return float(np.sqrt((a * a).mean()))

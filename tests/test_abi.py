@@ -89,6 +89,17 @@ def test_bad_arguments_rejected_before_any_cuda_call(lib):
     assert lib.coli_sync_status(C.c_void_p(8), None) == m.COLI_EINVAL  # misaligned workspace
 
 
+def test_noalloc_rejects_token_counts_outside_range_before_sizing(lib):
+    """n_tok < 0 or > 2^24 is refused before the scratch need is computed
+    (whose size arithmetic would otherwise run on absurd counts)."""
+    import int4_weight_only_sigmoid_b200 as m
+    cfg = m.make_config(6144, 2048, 256, 8, 1)
+    L = m.MoeLayerC(cfg, None, None, None, None)
+    for n in (-1, (1 << 24) + 1, 1 << 40, (1 << 62)):
+        assert lib.coli_moe_layer_forward_noalloc(C.byref(L), None, n, None, None) == m.COLI_EINVAL
+        assert b"n_tok" in lib.coli_last_error()
+
+
 def test_zero_tokens_is_ok_without_touching_pointers(lib):
     import int4_weight_only_sigmoid_b200 as m
     assert lib.coli_quantize_act_q8(None, 0, 64, None, None, None) == m.COLI_OK

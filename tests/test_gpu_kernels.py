@@ -121,6 +121,25 @@ def test_route_bit_exact(coli, ora, syn, name, n_tok):
     assert bits_equal(_np(w)[sub], wo)
 
 
+@pytest.mark.parametrize("name,n_tok", [("tiny", 8), ("decode16", 16), ("prefill2048", 300)])
+def test_route_without_scores_buffer(coli, ora, syn, name, n_tok):
+    """coli_moe_route with scores = NULL (scores kept on chip): the same
+    expert indices and weights, bit for bit, as the oracle."""
+    import torch
+    cfg = syn.config(name)
+    ccfg = coli.make_config(cfg["hidden"], cfg["inter"], cfg["n_experts"], cfg["top_k"], cfg["n_shared"],
+                            cfg["shared_inter"], cfg["norm_topk_prob"], cfg["routed_scaling_factor"])
+    L = coli.MoeLayer(ccfg, syn.dev_router_w(cfg), syn.dev_bias(cfg), [], [])
+    x = syn.tokens(cfg, n_tok)
+    scores, idx, w = coli.moe_route(L, torch.from_numpy(x).cuda(), with_scores=False)
+    assert scores is None
+    sub = np.arange(n_tok) if n_tok <= 16 else np.random.default_rng(2).choice(n_tok, 24, replace=False)
+    _, io, wo = ora.route(x[sub], syn.router_w(cfg), syn.bias(cfg), cfg["top_k"], cfg["norm_topk_prob"],
+                          cfg["routed_scaling_factor"])
+    assert np.array_equal(_np(idx)[sub], io)
+    assert bits_equal(_np(w)[sub], wo)
+
+
 def test_route_ties_and_k_equals_e(coli, ora):
     import torch
     E, H = 16, 128
@@ -135,6 +154,8 @@ def test_route_ties_and_k_equals_e(coli, ora):
         s, idx, w = coli.moe_route(L, torch.from_numpy(x).cuda())
         so, io, wo = ora.route(x, W, bias, K, True, 2.5)
         assert np.array_equal(_np(idx), io) and bits_equal(_np(w), wo)
+        _, idx2, w2 = coli.moe_route(L, torch.from_numpy(x).cuda(), with_scores=False)
+        assert np.array_equal(_np(idx2), io) and bits_equal(_np(w2), wo)
 
 
 # --------------------------------------------------------------------------

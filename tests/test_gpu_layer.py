@@ -33,12 +33,18 @@ def _dev_layer(cfg, layer=0):
     return _layers[key]
 
 
-def _check_layer(coli, syn, cfg, n_tok, sample=None, exact=True):
+def _check_layer(coli, syn, cfg, n_tok, sample=None, exact=True, tokens=None):
+    """sample: a seeded random subset of that many tokens; tokens: these."""
     import torch
     L = _dev_layer(cfg)
     x = syn.tokens(cfg, n_tok)
     out = _np(coli.moe_layer_forward(L, torch.from_numpy(x).cuda()))
-    sub = np.arange(n_tok) if sample is None else np.sort(np.random.default_rng(1).choice(n_tok, sample, replace=False))
+    if tokens is not None:
+        sub = np.asarray(sorted(set(int(t) for t in tokens)))
+    elif sample is None:
+        sub = np.arange(n_tok)
+    else:
+        sub = np.sort(np.random.default_rng(1).choice(n_tok, sample, replace=False))
     want, idx, w, _ = oracle_layer_forward(cfg, x[sub])
     _, gidx, gw = coli.moe_route(L, torch.from_numpy(x[sub]).cuda())
     assert np.array_equal(_np(gidx), idx)
@@ -68,6 +74,14 @@ def test_layer_tiny_prefill_variants(coli, syn, over):
     _check_layer(coli, syn, syn.config("tiny", **over), 200)
 
 
+@pytest.mark.parametrize("n_tok", [1, 5, 16, 40])
+def test_layer_inter_not_multiple_of_128(coli, syn, n_tok):
+    """Expert inter 96 (not a multiple of 128): neither the decode streaming
+    kernels nor the tensor-core kernels take it, so the general expert
+    kernels run at layer level, for decode and for prefill batch sizes."""
+    _check_layer(coli, syn, syn.config("tiny", inter=96, shared_inter=96), n_tok)
+
+
 @pytest.mark.parametrize("over", [dict(norm_topk_prob=False), dict(routed_scaling_factor=1.0),
                                   dict(top_k=1), dict(top_k=16), dict(n_shared=0), dict(n_shared=2)])
 def test_layer_tiny_variants(coli, syn, over):
@@ -83,11 +97,45 @@ def test_layer_decode4(coli, syn):
 
 
 def test_layer_decode16(coli, syn):
-    _check_layer(coli, syn, syn.config("decode16"), 16, sample=6)
+    """All 16 tokens of the verify batch."""
+    _check_layer(coli, syn, syn.config("decode16"), 16)
 
 
-def test_layer_prefill2048_sampled(coli, syn):
-    _check_layer(coli, syn, syn.config("prefill2048"), 2048, sample=4)
+def _tile_edge_tokens(coli, syn, cfg, n_tok, tile=128):
+    """Tokens chosen where tiled kernels go wrong first, from the routing of
+    the whole batch: the last token of every tile (and the last token) of
+    the two most loaded experts, the first and last token of the shared
+    expert's last tile, every token of up to four one-token experts, and the
+    first token of the batch."""
+    import torch
+    L = _dev_layer(cfg)
+    x = syn.tokens(cfg, n_tok)
+    _, idx, _ = coli.moe_route(L, torch.from_numpy(x).cuda(), with_scores=False)
+    idx = _np(idx)
+    counts = np.bincount(idx.ravel(), minlength=cfg["n_experts"])
+    chosen = {0, n_tok - 1, (n_tok - 1) // tile * tile}
+    for e in np.argsort(-counts, kind="stable")[:2]:
+        toks = np.flatnonzero((idx == e).any(axis=1))  # the expert's tokens in slot order (ascending)
+        chosen.update(int(toks[i]) for i in range(tile - 1, len(toks), tile))
+        chosen.add(int(toks[-1]))
+    ones = np.flatnonzero(counts == 1)[:4]
+    for e in ones:
+        chosen.add(int(np.flatnonzero((idx == e).any(axis=1))[0]))
+    return sorted(chosen), int(counts.max()), len(ones)
+
+
+def test_layer_prefill2048_tile_edges(coli, syn):
+    """GLM shape, 2048 tokens with the skewed bias: >= 16 tokens picked at
+    tile edges of the heaviest experts (each ~700 tokens = 6 tiles), in the
+    shared expert's last tile and in one-token experts, plus a random
+    sample, all compared with the oracle bit for bit."""
+    cfg = syn.config("prefill2048")
+    edge, cmax, n_ones = _tile_edge_tokens(coli, syn, cfg, 2048)
+    assert cmax > 2 * 128 and n_ones >= 1
+    rand = np.random.default_rng(7).choice(2048, 16, replace=False)
+    chosen = sorted(set(edge) | set(int(t) for t in rand))
+    assert len(chosen) >= 32
+    _check_layer(coli, syn, cfg, 2048, tokens=chosen)
 
 
 def test_layer_prefill_glm_ragged(coli, syn):
@@ -174,6 +222,26 @@ def test_stack8_teacher_forced_and_free(coli, ora, syn):
     assert bits_equal(free, xo)
     del layers
     torch.cuda.empty_cache()
+
+
+def test_stack8_prefill512_sampled_tokens(coli, syn):
+    """The 8-layer stack on 512 tokens (the tensor-core path in every
+    layer), free-running on the GPU; the oracle runs 6 of the tokens through
+    the same 8 layers on its own.  Tokens are independent through the whole
+    stack, so those rows must match bit for bit."""
+    import torch
+    from synth.layers import device_layer
+    from tests.helpers import oracle_stack_forward
+    cfg = syn.config("stack8_512")
+    layers = [device_layer(cfg, l) for l in range(8)]
+    x = syn.tokens(cfg, 512)
+    out = _np(coli.moe_stack_forward(layers, torch.from_numpy(x).cuda(), cfg["rms_eps"]))
+    del layers
+    torch.cuda.empty_cache()
+    sub = np.array([0, 137, 255, 256, 400, 511])
+    want = oracle_stack_forward(cfg, x[sub], 8)
+    assert_layer_close(out[sub], want)
+    assert bits_equal(out[sub], want)
 
 
 def test_invalid_arguments_return_einval(coli, syn):

@@ -51,3 +51,9 @@ def test_noalloc_rejects_more_than_its_scratch(coli, syn):
         coli.moe_layer_forward_noalloc(L, x)
     assert ei.value.status == coli.COLI_EINVAL
     assert "scratch" in str(ei.value)
+    # a token count beyond the forward's range is refused before any sizing
+    Lc = L.cstruct()
+    import ctypes as C
+    rc = coli.lib().coli_moe_layer_forward_noalloc(C.byref(Lc), C.c_void_p(x.data_ptr()), (1 << 40),
+                                                  C.c_void_p(x.data_ptr()), None)
+    assert rc == coli.COLI_EINVAL
