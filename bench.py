@@ -9,6 +9,9 @@ top-k, bucketing, gate/up + SwiGLU + Q8, down, combine).  Eight distinct
 layers (~39 GB) stay resident and the steps cycle through them, so each
 step streams ~170 MB of expert weights that the 126 MB L2 cannot hold from
 an earlier step.  Steps are replayed from CUDA graphs of up to 64 steps.
+Each layer also carries its streaming copy (coli_moe_prepare: the same bytes
+reordered so that each step of the expert kernel is one contiguous 16 KB
+read), which the decode path of <= 4 tokens reads.
 
 Metric: MoE-layer tokens/s (value) and streamed int4 weight GB/s (roofline).
 
@@ -39,11 +42,41 @@ WORKLOAD = ("GLM-5.2-shaped MoE layer decode, 1 token (hidden 6144, expert inter
 N_LAYERS = 8
 N_TOK_POOL = 64
 GRAPH_STEPS = 64
-KERNELS_PER_STEP = 5  # decode path: router, top-k+bucket, gate/up, down, combine
-# dram__bytes_read.sum + dram__bytes_write.sum of one gateup_ring_kernel<1>
-# launch, from one ncu capture of the GLM decode-1 layer; None once that kernel
-# changes.
-GATEUP_TRAFFIC_BYTES = 117.09e6
+KERNELS_PER_STEP = 2  # decode path on a prepared layer: router_decode, expert_stream_kernel<1>
+ROOFLINE_KERNEL = "expert_stream_kernel<1>"
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
+# kernel comes from the ncu summary below, and only while the kernel's
+# source is the one that summary was captured from (its sha256 prefix is
+# recorded there); otherwise traffic is reported as null.
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "expert_stream_glm_decode1.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "int4_weight_only_sigmoid_b200", "csrc", f)
+                  for f in ("coli_expert_stream.cu", "coli_expert_stream.cuh", "coli_stream.cuh")]
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """(bytes per launch, note) from the kept ncu summary when its recorded
+    source hash matches the current kernel sources, else (None, why)."""
+    import re
+    try:
+        text = open(TRAFFIC_PROFILE).read()
+    except OSError:
+        return None, "no ncu summary kept for this kernel"
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", text)
+    if not m or not h:
+        return None, "summary lacks traffic or source hash"
+    if h.group(1) != kernel_source_hash():
+        return None, "kernel changed since the ncu capture"
+    return float(m.group(1)), os.path.relpath(TRAFFIC_PROFILE, ROOT)
 
 
 def parse():
@@ -409,7 +442,7 @@ def main():
     H = cfg["hidden"]
     staging = torch.empty(cfg["inter"] * H, dtype=torch.float32, device=dev)
     n_layers = args.layers
-    layers = [device_layer(cfg, l, device=dev, staging=staging) for l in range(n_layers)]
+    layers = [device_layer(cfg, l, device=dev, staging=staging, prepare=True) for l in range(n_layers)]
     del staging
     cstructs = [L.cstruct() for L in layers]
     xs = synth.dev_tokens(cfg, N_TOK_POOL, device=dev)
@@ -430,7 +463,7 @@ def main():
     # expert bytes actually streamed per step (unique selected experts + shared)
     mat = cfg["inter"] * H // 2
     expert_bytes = 3 * mat + (2 * cfg["inter"] + H) * 4
-    gateup_bytes_per_expert = 2 * mat + 2 * cfg["inter"] * 4
+
     router_bytes = cfg["n_experts"] * H * 4 + cfg["n_experts"] * 4
     uniq = []
     for i in range(N_TOK_POOL):
@@ -512,19 +545,18 @@ def main():
 
     # 2) the dominant kernel: the same steps with events the library records
     #    on its stream around the gate/up and down kernels
-    gate_ms, down_ms, gate_bytes, phase_n = 0.0, 0.0, 0.0, 0
+    kern_ms, kern_bytes, phase_n = 0.0, 0.0, 0
 
     def harvest(r, base_step):
-        nonlocal gate_ms, down_ms, gate_bytes, phase_n
+        nonlocal kern_ms, kern_bytes, phase_n
         g, evs = r
         for j, (e0, e1, e2) in enumerate(evs):
             raw.sync(e2)
-            a, b = raw.elapsed_ms(e0, e1), raw.elapsed_ms(e1, e2)
-            if a <= 0 or b <= 0:
+            a = raw.elapsed_ms(e0, e2)  # the expert kernel (gate/up, down, combine in one launch)
+            if a <= 0:
                 continue
-            gate_ms += a
-            down_ms += b
-            gate_bytes += n_exp[(base_step + j) % N_TOK_POOL] * gateup_bytes_per_expert
+            kern_ms += a
+            kern_bytes += n_exp[(base_step + j) % N_TOK_POOL] * expert_bytes
             phase_n += 1
 
     ring = [capture(G, r * G, True) for r in range(NG)]
@@ -539,8 +571,9 @@ def main():
     mean_exp = sum(n_exp) / len(n_exp)
     step_bytes = mean_exp * expert_bytes + router_bytes
     peak, peak_kind = peaks()
-    gate_avg_ms = gate_ms / max(1, phase_n)
-    gate_gbs = (gate_bytes / max(1, phase_n)) / (gate_avg_ms * 1e-3) / 1e9 if gate_avg_ms > 0 else 0.0
+    kern_avg_ms = kern_ms / max(1, phase_n)
+    kern_gbs = (kern_bytes / max(1, phase_n)) / (kern_avg_ms * 1e-3) / 1e9 if kern_avg_ms > 0 else 0.0
+    traffic, traffic_src = profiled_traffic()
     step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
 
     # end to end through the public API: pinned host token in, host output back
@@ -598,11 +631,11 @@ def main():
                        "graph_steps": G, "mean_experts_streamed": mean_exp},
             "streamed_gbs": step_gbs,
             "streamed_frac_of_hbm": step_gbs / peak,
-            "roofline": {"bound": "hbm", "kernel": "gateup_ring_kernel<1>", "achieved": gate_gbs, "peak": peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": gate_gbs / peak, "traffic": GATEUP_TRAFFIC_BYTES,
-                         "avg_launch_ms": gate_avg_ms,
-                         "algorithmic_bytes_per_launch": gate_bytes / max(1, phase_n),
-                         "down_kernel_avg_ms": down_ms / max(1, phase_n)},
+            "roofline": {"bound": "hbm", "kernel": ROOFLINE_KERNEL, "achieved": kern_gbs, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": kern_gbs / peak, "traffic": traffic,
+                         "traffic_source": traffic_src, "avg_launch_ms": kern_avg_ms,
+                         "algorithmic_bytes_per_launch": kern_bytes / max(1, phase_n),
+                         "source_sha256_16": kernel_source_hash()},
             "e2e": e2e, "gpu_launches": K * KERNELS_PER_STEP, "clocks": clocks, "cpu_baseline": cpu,
             "other_workloads": suite,
             "phase_region_ms_per_step": phase_elapsed_ms / K,

@@ -88,13 +88,17 @@ typedef struct {
 
 /* One MoE layer.  `experts` and `shared` are HOST arrays (n_experts and
  * n_shared entries) of device-pointer sets; the router stays F32
- * ([W] "量化保留模块"). */
+ * ([W] "量化保留模块").  `prepared` is the layer's streaming copy
+ * (coli_moe_prepare) or NULL: with it, decode batches of up to 4 tokens
+ * read the experts from that copy (same results, bit for bit); without it,
+ * or for other batch sizes, the kernels read the row-major weights. */
 typedef struct {
     coli_moe_config cfg;
     const float* w_router;      /* [n_experts x hidden] F32, device */
     const float* bias;          /* [n_experts] F32 correction bias, device */
     const coli_expert* experts; /* host array [n_experts] */
     const coli_expert* shared;  /* host array [n_shared] */
+    const void* prepared;       /* device, 256-byte aligned, or NULL */
 } coli_moe_layer;
 
 /* Per-row int4 weight quantiser ([W] "GLM-5.2-colibri-int4的量化流程":
@@ -180,6 +184,26 @@ coli_status coli_moe_stack_forward(const coli_moe_layer* layers, int32_t n_layer
  * (i/4) mod 32, each an fmaf chain in ascending i from +0, then the 32
  * accumulators added left to right); dim % 128 == 0.  x, y: [n_tok x dim]. */
 coli_status coli_rmsnorm(const float* x, int64_t n_tok, int64_t dim, float eps, float* y, void* stream);
+
+/* The layer's streaming copy ([H] "已实现的功能", batched MoE: one read of
+ * an expert per layer; [D] "引擎是如何工作的": an expert's matrices are
+ * read as one contiguous piece).  The same packed int4 bytes and F32 row
+ * scales as the row-major weights, reordered once so that the decode
+ * kernel moves each step of its work (16 KB: 32 gate + 32 up rows x 16
+ * blocks, or 32 down rows x 32 blocks, the blocks of a row XOR-rotated)
+ * with one bulk copy.  Per expert (routed 0..n_experts-1, then shared):
+ * gate/up units, down units, then the scales; GLM-5.2 shape: 18.9 MB per
+ * expert, 4.86 GB per layer, the size of the row-major weights.
+ * coli_moe_prepared_bytes: bytes for the layer (0 if cfg is invalid or the
+ * shape has no streaming layout: hidden and inter multiples of 128,
+ * hidden/32 a multiple of 16 or 4 or 8, inter/32 a multiple of 32 or 4, 8,
+ * 16).  coli_moe_prepare: writes the copy of `layer`'s weights into
+ * `prepared` (device, 256-byte aligned, `bytes` >= coli_moe_prepared_bytes;
+ * caller-owned), stream-ordered; the row-major weights are only read.
+ * Re-run it after changing the weights.  Store the pointer in
+ * layer->prepared to use it. */
+size_t coli_moe_prepared_bytes(const coli_moe_config* cfg);
+coli_status coli_moe_prepare(const coli_moe_layer* layer, void* prepared, size_t bytes, void* stream);
 
 /* Bytes of workspace that coli_moe_layer_forward, coli_moe_stack_forward and
  * coli_moe_expert_ffn need for up to max_tokens tokens (0 if cfg is

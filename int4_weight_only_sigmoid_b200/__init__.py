@@ -25,7 +25,7 @@ EXPORTS = [
     "coli_moe_expert_ffn", "coli_moe_layer_forward", "coli_moe_stack_forward", "coli_rmsnorm",
     "coli_moe_workspace_bytes", "coli_last_error", "coli_debug_block_partials",
     "coli_debug_phase_events", "coli_moe_layer_forward_noalloc", "coli_sync_status", "coli_debug_wait_probe",
-    "coli_requantize_fp8_int4",
+    "coli_requantize_fp8_int4", "coli_moe_prepared_bytes", "coli_moe_prepare",
 ]
 
 
@@ -48,7 +48,7 @@ class Expert(C.Structure):
 
 class MoeLayerC(C.Structure):
     _fields_ = [("cfg", MoeConfig), ("w_router", C.c_void_p), ("bias", C.c_void_p),
-                ("experts", C.POINTER(Expert)), ("shared", C.POINTER(Expert))]
+                ("experts", C.POINTER(Expert)), ("shared", C.POINTER(Expert)), ("prepared", C.c_void_p)]
 
 
 _lib = None
@@ -84,6 +84,8 @@ def load(path: str | None = None):
         "coli_sync_status": (st, [vp, vp]),
         "coli_debug_wait_probe": (st, [vp, i64, vp]),
         "coli_requantize_fp8_int4": (st, [vp, vp, i64, i64, i32, vp, vp, vp]),
+        "coli_moe_prepared_bytes": (C.c_size_t, [C.POINTER(MoeConfig)]),
+        "coli_moe_prepare": (st, [C.POINTER(MoeLayerC), vp, C.c_size_t, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -140,20 +142,23 @@ class QExpert:
 
 @dataclass
 class MoeLayer:
-    """One MoE layer resident in HBM: router (F32), bias, experts, shared experts."""
+    """One MoE layer resident in HBM: router (F32), bias, experts, shared
+    experts, and optionally its streaming copy (``prepare``)."""
     cfg: MoeConfig
     w_router: object
     bias: object
     experts: list
     shared: list
+    prepared: object = None
     _keep: list = field(default_factory=list, repr=False)
 
-    def cstruct(self) -> MoeLayerC:
+    def cstruct(self, use_prepared: bool = True) -> MoeLayerC:
         ex = (Expert * len(self.experts))(*[e.cstruct() for e in self.experts])
         sh = (Expert * max(1, len(self.shared)))(*[e.cstruct() for e in self.shared])
         self._keep = [ex, sh]
+        prep = self.prepared.data_ptr() if (use_prepared and self.prepared is not None) else None
         return MoeLayerC(self.cfg, self.w_router.data_ptr(), self.bias.data_ptr(),
-                         C.cast(ex, C.POINTER(Expert)), C.cast(sh, C.POINTER(Expert)))
+                         C.cast(ex, C.POINTER(Expert)), C.cast(sh, C.POINTER(Expert)), prep)
 
 
 # ---------------------------------------------------------------------------
@@ -214,6 +219,28 @@ def moe_bucket(idx, n_experts: int, stream=None):
     _check(lib().coli_moe_bucket(_ptr(idx) if T else None, T, K, n_experts, _ptr(counts),
                                  _ptr(offsets), _ptr(perm), _stream(stream)))
     return counts, offsets, perm[:T * K]
+
+
+def prepared_bytes(cfg: MoeConfig) -> int:
+    return int(lib().coli_moe_prepared_bytes(C.byref(cfg)))
+
+
+def prepare(layer: MoeLayer, stream=None):
+    """Make the layer's streaming copy (coli_moe_prepare) in a new device
+    buffer and attach it to the layer (layer.prepared); returns the buffer."""
+    import torch
+    n = prepared_bytes(layer.cfg)
+    if n == 0:
+        raise ColiError(COLI_EINVAL, "this shape has no streaming layout")
+    dev = layer.w_router.device
+    buf = torch.empty(n + 256, dtype=torch.uint8, device=dev)
+    off = (-buf.data_ptr()) % 256
+    view = buf[off:off + n]
+    Lc = layer.cstruct(use_prepared=False)
+    _check(lib().coli_moe_prepare(C.byref(Lc), _ptr(view), n, _stream(stream)))
+    layer.prepared = view
+    layer._prep_storage = buf
+    return view
 
 
 def workspace_bytes(cfg: MoeConfig, max_tokens: int) -> int:

@@ -82,6 +82,8 @@ coli_status check_layer(const coli_moe_layer* L, const char* fn) {
   CHECK_PTR(L->bias);
   if (L->experts == nullptr) return fail(COLI_EINVAL, "%s: null experts array", fn);
   if (L->cfg.n_shared > 0 && L->shared == nullptr) return fail(COLI_EINVAL, "%s: null shared array", fn);
+  if (L->prepared != nullptr && (reinterpret_cast<uintptr_t>(L->prepared) & 255u) != 0)
+    return fail(COLI_EINVAL, "%s: 'prepared' is not 256-byte aligned", fn);
   for (int e = 0; e < L->cfg.n_experts; ++e)
     if ((s = check_expert(&L->experts[e], fn)) != COLI_OK) return s;
   for (int e = 0; e < L->cfg.n_shared; ++e)
@@ -96,7 +98,7 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Workspace {
   size_t xq, xd, scores, idx, w, counts, offsets, perm, inv, slots, n_slots, status, tiles, n_tiles, hq, hd, xf, hf,
-      y, xn, xa, xb, total;
+      hdc, ctr, y, xn, xa, xb, total;
 };
 
 Workspace layout(const coli_moe_config& c, int64_t T) {
@@ -129,6 +131,11 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   L.xf = take(tc ? rows * H * 2 : 0);
   L.hf = take(tc ? rows * I * 2 : 0);
   L.hd = take(rows * (I / 32) * 4);
+  // the streaming decode kernel (prepared layers, <= kStreamMaxTok tokens):
+  // (d, c16) of every h block and its counters
+  const bool sm = T <= kStreamMaxTok;
+  L.hdc = take(sm ? rows * (I / 32) * 8 : 0);
+  L.ctr = take(sm ? (size_t)(kStreamMaxSlots + H / 32) * 4 : 0);
   L.y = take(rows * H * 4);
   L.xn = take(T * H * 4);
   L.xa = take(T * H * 4);
@@ -187,10 +194,41 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   };
 
   int32_t* status = at<int32_t>(ws, W.status);
+  if (L->prepared != nullptr && stream_supported(H, I, (int)T, S, K)) {
+    // decode on the streaming copy: 2 kernels, the second launched with PDL
+    int32_t* ctr = at<int32_t>(ws, W.ctr);
+    CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, xq, xd, clear_status ? status : nullptr,
+                                      ctr, kStreamMaxSlots + H / 32, st));
+    CHECK_LAUNCH(mark(0));
+    StreamArgs a{};
+    a.prep = static_cast<const unsigned char*>(L->prepared);
+    a.g = stream_geom(H, I);
+    a.E = E;
+    a.K = K;
+    a.S = S;
+    a.T = (int)T;
+    a.norm = c.norm_topk_prob;
+    a.rsf = c.routed_scaling_factor;
+    a.scores = scores;
+    a.bias = L->bias;
+    a.xq = xq;
+    a.xd = xd;
+    a.hpl = hq;
+    a.hdc = at<float2>(ws, W.hdc);
+    a.y = y;
+    a.out = out;
+    a.h_ready = ctr;
+    a.dn_done = ctr + kStreamMaxSlots;
+    a.status = status;
+    CHECK_LAUNCH(launch_expert_stream(a, st));
+    CHECK_LAUNCH(mark(1));
+    CHECK_LAUNCH(mark(2));
+    return COLI_OK;
+  }
   if (T <= kDecodeMaxTok && decode_supported(H, I)) {
     // decode: 5 kernels, the last four launched with PDL
     CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, xq, xd, clear_status ? status : nullptr,
-                                      st));
+                                      nullptr, 0, st));
     CHECK_LAUNCH(launch_topk_bucket_small(scores, L->bias, (int)T, E, K, c.norm_topk_prob, c.routed_scaling_factor,
                                           idx, wts, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm, inv,
                                           slots, n_slots, st));
@@ -252,6 +290,35 @@ COLI_EXPORT size_t coli_moe_workspace_bytes(const coli_moe_config* cfg, int64_t 
   return layout(*cfg, max_tokens).total;
 }
 
+COLI_EXPORT size_t coli_moe_prepared_bytes(const coli_moe_config* cfg) {
+  if (check_cfg(cfg, "coli_moe_prepared_bytes") != COLI_OK) return 0;
+  if (!stream_shape_ok(cfg->hidden, cfg->inter)) return 0;
+  return (size_t)(cfg->n_experts + cfg->n_shared) * stream_expert_bytes(cfg->hidden, cfg->inter);
+}
+
+COLI_EXPORT coli_status coli_moe_prepare(const coli_moe_layer* layer, void* prepared, size_t bytes, void* stream) {
+  const char* fn = "coli_moe_prepare";
+  coli_status s = check_layer(layer, fn);
+  if (s != COLI_OK) return s;
+  const coli_moe_config& c = layer->cfg;
+  const size_t need = coli_moe_prepared_bytes(&c);
+  if (need == 0)
+    return fail(COLI_EINVAL, "%s: hidden=%d inter=%d has no streaming layout (both multiples of 128; hidden/32 a "
+                "multiple of 16 or 4, 8; inter/32 a multiple of 32 or 4, 8, 16)", fn, c.hidden, c.inter);
+  if (prepared == nullptr) return fail(COLI_EINVAL, "%s: null pointer 'prepared'", fn);
+  if ((reinterpret_cast<uintptr_t>(prepared) & 255u) != 0)
+    return fail(COLI_EINVAL, "%s: 'prepared' is not 256-byte aligned", fn);
+  if (bytes < need) return fail(COLI_ENOMEM, "%s: %zu bytes < %zu needed", fn, bytes, need);
+  const uint64_t eb = stream_expert_bytes(c.hidden, c.inter);
+  cudaStream_t st = (cudaStream_t)stream;
+  for (int j = 0; j < c.n_experts + c.n_shared; ++j) {
+    const coli_expert& e = j < c.n_experts ? layer->experts[j] : layer->shared[j - c.n_experts];
+    CHECK_LAUNCH(launch_prepare_expert(c.hidden, c.inter, e.gate_q, e.gate_s, e.up_q, e.up_s, e.down_q, e.down_s,
+                                       static_cast<unsigned char*>(prepared) + (size_t)j * eb, st));
+  }
+  return COLI_OK;
+}
+
 namespace coli {
 namespace {
 
@@ -264,6 +331,9 @@ const char* status_meaning(int32_t code) {
     case 13: return "prefill fold gave up waiting for accumulators";
     case 16: return "prefill A-tile loader gave up waiting for an operand stage";
     case 22: return "decode down kernel gave up waiting for h rows";
+    case 24: return "streaming decode kernel gave up waiting for a weight stage";
+    case 25: return "streaming decode kernel gave up waiting for a slot's h rows from other CTAs";
+    case 26: return "streaming decode kernel gave up waiting for staged h rows";
     case kStatusWaitProbe: return "test probe: a wait that nothing completes gave up";
     default: return code >= kStatusTimeoutFirst ? "a bounded wait gave up" : "a device-side check failed";
   }

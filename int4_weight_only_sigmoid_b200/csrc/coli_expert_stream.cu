@@ -1,0 +1,593 @@
+// coli_expert_stream.cu -- the expert part of a decode batch (n_tok <= 4)
+// in one persistent kernel, reading the layer's streaming copy
+// (coli_expert_stream.cuh, made by coli_moe_prepare):
+//
+//   router_decode (plain launch: scores, Q8_0 of x, counters cleared)
+//   -> expert_stream_kernel (PDL):
+//        every CTA takes the top-k and the bucketing of the batch itself
+//        (a few hundred scores; no global round trip), then
+//        gate/up units (32 intermediate outputs of one expert slot: SiLU(g)*u
+//        and the Q8_0 block of h, published with a per-slot counter),
+//        then down units (32 output rows of one slot, waiting for the slot's
+//        h), and the unit that completes a 32-row chunk for every slot
+//        combines it into `out` (contract C).
+//
+// Streaming.  Every warp owns a ring of R 16 KB stages; lane 0 fills a
+// stage with ONE bulk copy (cp.async.bulk, mbarrier completion) of a stage
+// image from the streaming copy, R stages ahead of the one the warp
+// computes, across unit boundaries and from the gate/up phase into the
+// down phase (down weights do not depend on h, so they stream while the
+// last gate/up units finish).  The weights of a warp's gate/up unit
+// (192 KB at GLM-5.2 shapes) are one contiguous range of HBM.
+//
+// Arithmetic (contract F, bit-identical to the oracle).  Lane l holds one
+// weight row (gate/up: gate row l and up row l of the unit); per 16-byte
+// packed block and staged token: (w & 0x0F0F0F0F) ^ 0x08080808 is q + 8 of
+// the even elements (unsigned bytes) and w & 0xF0F0F0F0 is 16 q of the odd
+// ones (signed bytes); with the token's even / odd byte planes xe, xo and
+// c16 = -128 * sum(xe):
+//   A = dp4a.u32.s32(q_e + 8, xe) = sum q_e x_e + 8 sum(xe)
+//   B = dp4a.s32.s32(16 q_o, xo) starting from c16 = 16 sum q_o x_o - 128 sum(xe)
+//   isum = A + (B >> 4)            (B is a multiple of 16: exact)
+// then acc = fmaf(d_x[b], (float)isum, acc) in ascending b.
+//
+// Every wait is bounded (about a second): on expiry the CTA records a
+// status code, stops issuing and computing, drains its copies in flight
+// (bounded again) and exits.
+//
+// Sources: "Colibri：在笔记本上跑744B参数的AI模型", "关键特性" (integer dot
+// kernels, Q8_0 activations, packed int4); "GLM-5.2-colibri-int4架构解析…",
+// "MoE的工作原理" (top-k and the weighted combine), "GLM-5.2的MoE实现" (the
+// shared expert); HN summary, "已实现的功能" (batched MoE: one read of an
+// expert for all of its tokens).
+#include "coli_expert_stream.cuh"
+#include "coli_launch.h"
+#include "coli_stream.cuh"
+#include "coli_topk.cuh"
+
+namespace coli {
+namespace {
+
+constexpr int kSW = 4;                               // warps per CTA (all compute; lane 0 also copies)
+constexpr int kMaxPairsS = kStreamMaxTok * kMaxTopK;  // (token, k) pairs of a batch
+constexpr int kMaxSlotsS = kStreamMaxSlots;          // slots: shared + distinct routed experts
+constexpr int kErrStage = 24;                        // status: gave up waiting for a weight stage
+constexpr int kErrHReady = 25;                       // status: gave up waiting for a slot's h
+constexpr int kErrHStaged = 26;                      // status: gave up waiting for staged h
+
+template <int TT>
+struct StreamRing {
+  static constexpr int R = TT <= 2 ? 3 : 2;  // stages per warp
+};
+
+template <int TT>
+__host__ __device__ inline size_t stream_smem_bytes(const StreamGeom& g) {
+  const size_t ring = (size_t)kSW * StreamRing<TT>::R * kStreamStageMax;
+  const size_t xs = (size_t)TT * g.nbh * 40;        // x planes (32 B) + (d, c16) per block
+  const size_t hs = 2 * (size_t)TT * g.nbi * 40;    // two slots' h rows
+  return 1024 + ring + xs + hs;
+}
+
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// isum of one packed weight block (ue = q_e + 8, so = 16 q_o) against one
+// token's block (planes xe, xo; c16 = -128 * sum of xe's bytes).
+__device__ __forceinline__ int blk_isum(const uint4& ue, const uint4& so, const uint4& xe, const uint4& xo, int c16) {
+  int A = dp4a_us(ue.x, xe.x, 0);
+  int B = __dp4a((int)so.x, (int)xo.x, c16);
+  A = dp4a_us(ue.y, xe.y, A);
+  B = __dp4a((int)so.y, (int)xo.y, B);
+  A = dp4a_us(ue.z, xe.z, A);
+  B = __dp4a((int)so.z, (int)xo.z, B);
+  A = dp4a_us(ue.w, xe.w, A);
+  B = __dp4a((int)so.w, (int)xo.w, B);
+  return A + (B >> 4);
+}
+
+__device__ __forceinline__ void unpack_blk(const uint4& w, uint4& ue, uint4& so) {
+  ue.x = (w.x & 0x0F0F0F0Fu) ^ 0x08080808u;
+  ue.y = (w.y & 0x0F0F0F0Fu) ^ 0x08080808u;
+  ue.z = (w.z & 0x0F0F0F0Fu) ^ 0x08080808u;
+  ue.w = (w.w & 0x0F0F0F0Fu) ^ 0x08080808u;
+  so.x = w.x & 0xF0F0F0F0u;
+  so.y = w.y & 0xF0F0F0F0u;
+  so.z = w.z & 0xF0F0F0F0u;
+  so.w = w.w & 0xF0F0F0F0u;
+}
+
+__device__ __forceinline__ int even_plane_sum(const uint4& e) {
+  int s = __dp4a((int)e.x, 0x01010101, 0);
+  s = __dp4a((int)e.y, 0x01010101, s);
+  s = __dp4a((int)e.z, 0x01010101, s);
+  return __dp4a((int)e.w, 0x01010101, s);
+}
+
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// One gate/up stage: blocks b0 .. b0+G-1 of gate row l and up row l (lane
+// l) against the slot's staged tokens.
+template <int TT>
+__device__ __forceinline__ void gu_stage(const unsigned char* st, int G, int swz, int b0, int nb, int nv,
+                                         const int (&tok)[TT], const uint4* xpl, const float2* xdc, float (&ag)[TT],
+                                         float (&au)[TT]) {
+  const int lane = threadIdx.x & 31;
+  const uint4* rg = reinterpret_cast<const uint4*>(st) + lane * G;
+  const uint4* ru = reinterpret_cast<const uint4*>(st) + (32 + lane) * G;
+  const int sw = lane & swz;
+#pragma unroll 4
+  for (int j = 0; j < G; ++j) {
+    uint4 ge, go, ue, uo;
+    unpack_blk(rg[j ^ sw], ge, go);
+    unpack_blk(ru[j ^ sw], ue, uo);
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      if (t < nv) {
+        const int xi = tok[t] * nb + b0 + j;
+        const uint4 xe = xpl[2 * xi], xo = xpl[2 * xi + 1];
+        const float2 dc = xdc[xi];
+        const int c16 = __float_as_int(dc.y);
+        ag[t] = __fmaf_rn(dc.x, __int2float_rn(blk_isum(ge, go, xe, xo, c16)), ag[t]);
+        au[t] = __fmaf_rn(dc.x, __int2float_rn(blk_isum(ue, uo, xe, xo, c16)), au[t]);
+      }
+    }
+  }
+}
+
+// One down stage: blocks b0 .. b0+G-1 of down row l (lane l) against the
+// slot's staged h rows (token t of the slot at index t).
+template <int TT>
+__device__ __forceinline__ void dn_stage(const unsigned char* st, int G, int swz, int b0, int nb, int nv,
+                                         const uint4* hpl, const float2* hdc, float (&ay)[TT]) {
+  const int lane = threadIdx.x & 31;
+  const uint4* rw = reinterpret_cast<const uint4*>(st) + lane * G;
+  const int sw = lane & swz;
+#pragma unroll 4
+  for (int j = 0; j < G; ++j) {
+    uint4 we, wo;
+    unpack_blk(rw[j ^ sw], we, wo);
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      if (t < nv) {
+        const int hi = t * nb + b0 + j;
+        const uint4 xe = hpl[2 * hi], xo = hpl[2 * hi + 1];
+        const float2 dc = hdc[hi];
+        ay[t] = __fmaf_rn(dc.x, __int2float_rn(blk_isum(we, wo, xe, xo, __float_as_int(dc.y))), ay[t]);
+      }
+    }
+  }
+}
+
+template <int TT>
+__global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid_constant__ StreamArgs a) {
+  constexpr int R = StreamRing<TT>::R;
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ uint64_t full_bar[kSW][R];
+  __shared__ uint64_t hbar[2];
+  __shared__ int abort_s;
+  __shared__ int s_idx[kMaxPairsS], s_row[kMaxPairsS];
+  __shared__ float s_w[kMaxPairsS];
+  __shared__ int s_exp[kMaxSlotsS], s_cnt[kMaxSlotsS], s_base[kMaxSlotsS], s_tok[kMaxSlotsS][TT];
+  __shared__ uint32_t s_bits[kMaxExperts / 32];
+  __shared__ int s_nslots;
+
+  const StreamGeom& g = a.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = a.E, K = a.K, S = a.S, T = a.T;
+  unsigned char* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  unsigned char* ring = smem + (size_t)warp * R * kStreamStageMax;
+  uint4* xpl = reinterpret_cast<uint4*>(smem + (size_t)kSW * R * kStreamStageMax);
+  float2* xdc = reinterpret_cast<float2*>(xpl + 2 * TT * g.nbh);
+  unsigned char* hst = reinterpret_cast<unsigned char*>(xdc + TT * g.nbh);
+  const size_t hbuf_bytes = (size_t)TT * g.nbi * 40;
+  volatile int* abort_f = &abort_s;
+
+  for (int i = threadIdx.x; i < kMaxExperts / 32; i += blockDim.x) s_bits[i] = 0u;
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < kSW; ++w)
+      for (int r = 0; r < R; ++r) tc::mbar_init(&full_bar[w][r], 1);
+    tc::mbar_init(&hbar[0], 32);
+    tc::mbar_init(&hbar[1], 32);
+    abort_s = 0;
+    stream::fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int G = gridDim.x, NW = G * kSW, gw = warp * G + blockIdx.x;
+  const int n_shared_gu = S * g.cpu_gu;
+
+  // The warp's stage sequence: its gate/up units gw, gw + NW, ... then its
+  // down units d0 + warp, d0 + warp + kSW, ... (d0 = this CTA's first down
+  // unit).  Flat stage index i -> (unit, stage).  n_gu_mine / n_dn_mine are
+  // known once the routing is; before that only the first unit, if it is a
+  // shared expert's, can stream.
+  int n_gu_mine = 0, n_dn_mine = 0, d0 = 0;
+  bool routed = false;
+  auto stage_src = [&](int i, uint32_t& bytes) -> const unsigned char* {
+    if (!routed || i < n_gu_mine * g.st_gu) {  // before the routing: the warp's first (shared) unit only
+      const int k = i / g.st_gu, s = i - k * g.st_gu;
+      const int u = gw + k * NW;
+      const int slot = u / g.cpu_gu;
+      const int e = slot < S ? E + slot : s_exp[slot];
+      bytes = g.sb_gu;
+      return a.prep + (uint64_t)e * g.expert_bytes + (uint64_t)(u - slot * g.cpu_gu) * g.ub_gu +
+             (uint64_t)s * g.sb_gu;
+    }
+    const int j = i - n_gu_mine * g.st_gu;
+    const int k = j / g.st_dn, s = j - k * g.st_dn;
+    const int v = d0 + warp + k * kSW;
+    const int slot = v / g.cpu_dn;
+    const int e = slot < S ? E + slot : s_exp[slot];
+    bytes = g.sb_dn;
+    return a.prep + (uint64_t)e * g.expert_bytes + g.dn_off + (uint64_t)(v - slot * g.cpu_dn) * g.ub_dn +
+           (uint64_t)s * g.sb_dn;
+  };
+  int issued = 0;
+  auto issue = [&](int i) {  // lane 0
+    uint32_t bytes;
+    const unsigned char* src = stage_src(i, bytes);
+    uint64_t* bar = &full_bar[warp][i % R];
+    stream::mbar_expect_tx(bar, bytes);
+    stream::bulk_g2s(ring + (size_t)(i % R) * kStreamStageMax, src, bytes, bar);
+  };
+
+  // shared experts' first stages stream while the router finishes
+  if (lane == 0 && gw < n_shared_gu)
+    for (; issued < R && issued < g.st_gu; ++issued) issue(issued);
+
+  pdl_wait();  // scores, the Q8_0 of x and the cleared counters are complete
+  pdl_launch_dependents();
+
+  // ---- routing of the batch (every CTA, identical results) -------------
+  if (warp < T) {
+    int sel[kMaxTopK];
+    float ssel[kMaxTopK];
+    topk::warp_select_topk(a.scores + (size_t)warp * E, a.bias, E, K, lane, sel, ssel);
+    if (lane == 0) topk::topk_weights(sel, ssel, K, a.norm, a.rsf, s_idx + warp * K, s_w + warp * K);
+  }
+  // x planes: block b of token t -> even / odd byte planes and (d, c16)
+  for (int i = threadIdx.x; i < T * g.nbh; i += blockDim.x) {
+    const int t = i / g.nbh, b = i - t * g.nbh;
+    const uint4* src = reinterpret_cast<const uint4*>(a.xq + (size_t)t * g.H + 32 * b);
+    const uint4 a0 = ld_dep(src), a1 = ld_dep(src + 1);
+    uint4 e, o;
+    split_even_odd(a0.x, a0.y, e.x, o.x);
+    split_even_odd(a0.z, a0.w, e.y, o.y);
+    split_even_odd(a1.x, a1.y, e.z, o.z);
+    split_even_odd(a1.z, a1.w, e.w, o.w);
+    xpl[2 * i] = e;
+    xpl[2 * i + 1] = o;
+    xdc[i] = make_float2(ld_dep(a.xd + i), __int_as_float(-128 * even_plane_sum(e)));
+  }
+  __syncthreads();
+  const int n_pairs = T * K;
+  if (warp == 0) {
+    for (int p = lane; p < n_pairs; p += 32) atomicOr(&s_bits[s_idx[p] >> 5], 1u << (s_idx[p] & 31));
+    __syncwarp();
+    // slot of routed expert e: S + (set bits below e); slots in ascending expert id
+    const int nw = (E + 31) / 32;
+    const int c = lane < nw ? __popc(s_bits[lane]) : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int below_word = incl - c;
+    const int n_routed = __shfl_sync(0xffffffffu, incl, 31);
+    if (lane < nw) {
+      uint32_t bits = s_bits[lane];
+      int r = S + below_word;
+      while (bits) {
+        const int bit = __ffs(bits) - 1;
+        bits &= bits - 1;
+        s_exp[r] = 32 * lane + bit;
+        s_cnt[r] = 0;
+        ++r;
+      }
+    }
+    for (int s = lane; s < S; s += 32) {
+      s_exp[s] = E + s;
+      s_cnt[s] = T;
+      for (int t = 0; t < TT; ++t) s_tok[s][t] = t;
+    }
+    __syncwarp();
+    // each pair: its slot, and its position = earlier tokens on the same expert
+    int pslot[2] = {0, 0}, ppos[2] = {0, 0};
+    for (int h = 0; h < 2; ++h) {
+      const int p = lane + 32 * h;
+      if (p < n_pairs) {
+        const int e = s_idx[p], t = p / K;
+        const int w32 = e >> 5;
+        const int lo = __popc(s_bits[w32] & ((1u << (e & 31)) - 1u));
+        int below = 0;  // set bits in the words below w32
+        for (int q = 0; q < w32; ++q) below += __popc(s_bits[q]);
+        pslot[h] = S + below + lo;
+        int pos = 0;
+        for (int q = 0; q < t * K; ++q) pos += (s_idx[q] == e);
+        ppos[h] = pos;
+        atomicAdd(&s_cnt[pslot[h]], 1);
+        s_tok[pslot[h]][pos] = t;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      int base = 0;
+      for (int s = 0; s < S + n_routed; ++s) {
+        s_base[s] = base;
+        base += s_cnt[s];
+      }
+      s_nslots = S + n_routed;
+    }
+    __syncwarp();
+    for (int h = 0; h < 2; ++h) {
+      const int p = lane + 32 * h;
+      if (p < n_pairs) s_row[p] = s_base[pslot[h]] + ppos[h];
+    }
+  }
+  __syncthreads();
+
+  const int n_slots = s_nslots;
+  const int n_gu = n_slots * g.cpu_gu, n_dn = n_slots * g.cpu_dn;
+  n_gu_mine = gw < n_gu ? (n_gu - gw + NW - 1) / NW : 0;
+  d0 = (int)((int64_t)blockIdx.x * n_dn / G);
+  const int d1 = (int)((int64_t)(blockIdx.x + 1) * n_dn / G);
+  n_dn_mine = d0 + warp < d1 ? (d1 - d0 - warp + kSW - 1) / kSW : 0;
+  const int total = n_gu_mine * g.st_gu + n_dn_mine * g.st_dn;
+  routed = true;
+  // the down slots of this CTA's range (at most two: a range never spans
+  // more, since there are at least as many CTAs as slots)
+  const int slotA = d0 / g.cpu_dn;
+  const int slotB = d1 > d0 ? (d1 - 1) / g.cpu_dn : slotA;
+  const int ownerB = slotB != slotA ? ((slotB * g.cpu_dn - d0) % kSW) : -1;
+
+  if (lane == 0) {
+    // a first unit streamed before the routing was known may not exist
+    // (n_gu_mine == 0 only if gw >= n_gu, never for a shared unit)
+    for (; issued < R && issued < total; ++issued) issue(issued);
+  }
+  __syncwarp();
+
+  int consumed = 0;
+  bool ok = true;
+  auto wait_stage = [&]() -> bool {
+    const bool got = tc::mbar_wait(&full_bar[warp][consumed % R], (uint32_t)((consumed / R) & 1), abort_f, a.status,
+                                   kErrStage);
+    return __all_sync(0xffffffffu, got);
+  };
+  auto next_stage = [&]() {  // this stage's ring slot is free again
+    ++consumed;
+    __syncwarp();
+    if (lane == 0 && !*abort_f && issued < total) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // our reads of the slot before the copy's writes
+      issue(issued);
+      ++issued;
+    }
+    __syncwarp();
+  };
+
+  // ---- gate/up units ----------------------------------------------------
+  for (int k = 0; k < n_gu_mine && ok; ++k) {
+    const int u = gw + k * NW;
+    const int slot = u / g.cpu_gu, chunk = u - slot * g.cpu_gu;
+    const int nv = s_cnt[slot];
+    int tok[TT];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) tok[t] = t < nv ? s_tok[slot][t] : 0;
+    float ag[TT], au[TT];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) ag[t] = au[t] = 0.0f;
+    for (int s = 0; s < g.st_gu; ++s) {
+      if (!(ok = wait_stage())) break;
+      gu_stage<TT>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_gu, g.swz_gu, s * g.g_gu, g.nbh, nv, tok,
+                   xpl, xdc, ag, au);
+      next_stage();
+    }
+    if (!ok) break;
+    // SwiGLU, the Q8_0 block of h (these 32 outputs are one block), published
+    const float* sc = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);
+    const int row = chunk * 32 + lane;
+    const float sg = __ldg(sc + row), su = __ldg(sc + g.I + row);
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      if (t < nv) {
+        const float gv = __fmul_rn(sg, ag[t]);
+        const float uv = __fmul_rn(su, au[t]);
+        const float h = __fmul_rn(__fmul_rn(gv, sigmoid_cw(gv)), uv);
+        const float d = __fdiv_rn(warp_max(fabsf(h)), 127.0f);
+        const int q = q8_of(h, d);
+        const int64_t hrow = s_base[slot] + t;
+        a.hpl[(hrow * g.nbi + chunk) * 32 + (lane & 1) * 16 + (lane >> 1)] = (int8_t)q;
+        const int se = warp_sum_int((lane & 1) ? 0 : q);
+        if (lane == 0) a.hdc[hrow * g.nbi + chunk] = make_float2(d, __int_as_float(-128 * se));
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      atomicAdd(a.h_ready + slot, 1);
+    }
+  }
+
+  // ---- down units -------------------------------------------------------
+  int staged_slot = -1;
+  for (int k = 0; k < n_dn_mine && ok; ++k) {
+    const int v = d0 + warp + k * kSW;
+    const int slot = v / g.cpu_dn, chunk = v - slot * g.cpu_dn;
+    const int nv = s_cnt[slot];
+    const int buf = slot == slotA ? 0 : 1;
+    unsigned char* hb = hst + (size_t)buf * hbuf_bytes;
+    if (slot != staged_slot) {
+      const bool owner = buf == 0 ? warp == 0 : warp == ownerB;
+      if (owner) {
+        // wait for every gate/up unit of the slot, then copy its h rows
+        int ready = 0;
+        if (lane == 0) {
+          const long long t0 = clock64();
+          while (!*abort_f) {
+            if (ld_acquire_gpu(a.h_ready + slot) >= g.cpu_gu) {
+              ready = 1;
+              break;
+            }
+            if (clock64() - t0 > tc::kSpinCycles) {
+              *abort_f = 1;
+              atomicExch(a.status, kErrHReady);
+              break;
+            }
+            __nanosleep(256);
+          }
+        }
+        ready = __shfl_sync(0xffffffffu, ready, 0);
+        if (ready) {
+          const uint4* sp = reinterpret_cast<const uint4*>(a.hpl + (size_t)s_base[slot] * g.nbi * 32);
+          uint4* dp = reinterpret_cast<uint4*>(hb);
+          const int n16 = nv * g.nbi * 2;
+          for (int i = lane; i < n16; i += 32) dp[i] = __ldcg(sp + i);
+          const float4* sd = reinterpret_cast<const float4*>(a.hdc + (size_t)s_base[slot] * g.nbi);
+          float4* dd = reinterpret_cast<float4*>(hb + (size_t)TT * g.nbi * 32);
+          for (int i = lane; i < nv * g.nbi / 2; i += 32) dd[i] = __ldcg(sd + i);
+        }
+        tc::mbar_arrive(&hbar[buf]);  // all 32 lanes: the stores above are released to the CTA
+      }
+      const bool got = tc::mbar_wait(&hbar[buf], 0, abort_f, a.status, kErrHStaged);
+      if (!__all_sync(0xffffffffu, got && !*abort_f)) {  // warp-uniform
+        ok = false;
+        break;
+      }
+      staged_slot = slot;
+    }
+    const uint4* hpl = reinterpret_cast<const uint4*>(hb);
+    const float2* hdc = reinterpret_cast<const float2*>(hb + (size_t)TT * g.nbi * 32);
+    float ay[TT];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) ay[t] = 0.0f;
+    for (int s = 0; s < g.st_dn; ++s) {
+      if (!(ok = wait_stage())) break;
+      dn_stage<TT>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_dn, g.swz_dn, s * g.g_dn, g.nbi, nv, hpl,
+                   hdc, ay);
+      next_stage();
+    }
+    if (!ok) break;
+    const float* sc = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);
+    const int o = chunk * 32 + lane;
+    const float sd = __ldg(sc + 2 * g.I + o);
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+      if (t < nv) a.y[((size_t)s_base[slot] + t) * g.H + o] = __fmul_rn(sd, ay[t]);
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      __threadfence();
+      last = atomicAdd(a.dn_done + chunk, 1) == n_slots - 1;
+      if (last) __threadfence();
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      // every slot's y rows of this chunk are written: combine (contract C)
+      for (int t = 0; t < T; ++t) {
+        float acc = 0.0f;
+        for (int kk = 0; kk < K; ++kk)
+          acc = __fmaf_rn(s_w[t * K + kk], __ldcg(a.y + (size_t)s_row[t * K + kk] * g.H + o), acc);
+        for (int s = 0; s < S; ++s) acc = __fadd_rn(acc, __ldcg(a.y + ((size_t)s_base[s] + t) * g.H + o));
+        a.out[(size_t)t * g.H + o] = acc;
+      }
+    }
+  }
+
+  // copies still in flight (only after an abort): wait for them, bounded
+  if (lane == 0)
+    for (int i = consumed; i < issued; ++i) stream::mbar_drain(&full_bar[warp][i % R], (uint32_t)((i / R) & 1));
+  // an owner that gave up before arriving leaves hbar incomplete: waiters give up too (bounded)
+}
+
+// Streaming copy of one expert: one thread per packed 16-byte block, then
+// the scales.
+__global__ void prepare_expert_kernel(StreamGeom g, const uint8_t* __restrict__ gq, const uint8_t* __restrict__ uq,
+                                      const uint8_t* __restrict__ dq, const float* __restrict__ gs,
+                                      const float* __restrict__ us, const float* __restrict__ ds,
+                                      unsigned char* __restrict__ dst) {
+  const int64_t n_gu = (int64_t)g.I * g.nbh, n_dn = (int64_t)g.H * g.nbi;
+  const int64_t total = 2 * n_gu + n_dn;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    int m, r, b;
+    const uint8_t* src;
+    if (i < 2 * n_gu) {
+      m = (int)(i / n_gu);
+      const int64_t j = i - m * n_gu;
+      r = (int)(j / g.nbh);
+      b = (int)(j - (int64_t)r * g.nbh);
+      src = (m == 0 ? gq : uq) + (int64_t)r * (g.H / 2) + 16 * b;
+    } else {
+      m = 2;
+      const int64_t j = i - 2 * n_gu;
+      r = (int)(j / g.nbi);
+      b = (int)(j - (int64_t)r * g.nbi);
+      src = dq + (int64_t)r * (g.I / 2) + 16 * b;
+    }
+    *reinterpret_cast<uint4*>(dst + stream_block_offset(g, m, r, b)) = *reinterpret_cast<const uint4*>(src);
+  }
+  float* sc = reinterpret_cast<float*>(dst + g.sc_off);
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < 2 * g.I + g.H;
+       i += (int64_t)gridDim.x * blockDim.x)
+    sc[i] = i < g.I ? gs[i] : (i < 2 * g.I ? us[i - g.I] : ds[i - 2 * g.I]);
+}
+
+template <int TT>
+cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
+  static uint64_t attr_mask = 0;
+  static int sms[64] = {};
+  const size_t smem = stream_smem_bytes<TT>(a.g);
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+  cudaError_t e = smem_opt_in_once(expert_stream_kernel<TT>, (int)smem, attr_mask);
+  if (e != cudaSuccess) return e;
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (sms[dev] == 0 && (e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  // one CTA per SM, all resident at once (the down units wait for gate/up
+  // units of other CTAs); at least as many CTAs as slots, so that a CTA's
+  // range of down units spans at most two slots
+  if (sms[dev] < kMaxSlotsS) return cudaErrorInvalidConfiguration;
+  return launch_pdl(expert_stream_kernel<TT>, dim3(sms[dev]), dim3(kSW * 32), smem, st, true, a);
+}
+
+}  // namespace
+
+bool stream_supported(int hidden, int inter, int n_tok, int n_shared, int top_k) {
+  if (n_tok < 1 || n_tok > kStreamMaxTok || !stream_shape_ok(hidden, inter)) return false;
+  const StreamGeom g = stream_geom(hidden, inter);
+  (void)n_shared;
+  (void)top_k;
+  return stream_smem_bytes<4>(g) <= 227 * 1024 && stream_smem_bytes<1>(g) <= 227 * 1024;
+}
+
+uint64_t stream_expert_bytes(int hidden, int inter) { return stream_geom(hidden, inter).expert_bytes; }
+
+cudaError_t launch_prepare_expert(int hidden, int inter, const uint8_t* gq, const float* gs, const uint8_t* uq,
+                                  const float* us, const uint8_t* dq, const float* ds, void* dst, cudaStream_t st) {
+  const StreamGeom g = stream_geom(hidden, inter);
+  prepare_expert_kernel<<<592, 256, 0, st>>>(g, gq, uq, dq, gs, us, ds, static_cast<unsigned char*>(dst));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_expert_stream(const StreamArgs& a, cudaStream_t st) {
+  if (a.T <= 1) return stream_tt<1>(a, st);
+  if (a.T <= 2) return stream_tt<2>(a, st);
+  return stream_tt<4>(a, st);
+}
+
+}  // namespace coli

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include "coli_device.cuh"
+#include "coli_expert_stream.cuh"
 
 namespace coli {
 
@@ -70,8 +71,11 @@ cudaError_t launch_route_topk(const float* x, const float* w_router, const float
 
 // Decode batches: router scores with the router rows staged in shared memory
 // (plain launch), then top-k + weights + bucketing in one CTA (PDL launch).
+// The router kernel also clears n_zero words at `zero` (the streaming
+// kernel's counters; may be null).
 cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
-                                 int8_t* xq, float* xd, int32_t* status_clear, cudaStream_t st);
+                                 int8_t* xq, float* xd, int32_t* status_clear, int32_t* zero, int n_zero,
+                                 cudaStream_t st);
 cudaError_t launch_topk_bucket_small(const float* scores, const float* bias, int n_tok, int E, int K, int norm,
                                      float rsf, int32_t* idx, float* w, int32_t* counts, int32_t* offsets,
                                      int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, cudaStream_t st);
@@ -114,6 +118,35 @@ cudaError_t launch_down_decode(const DownTable& tbl, const Slot* slots, const in
                                const float* w, int hidden, int inter, float* y, float* out, int32_t* status,
                                cudaStream_t st);
 
+// Decode batches of <= kStreamMaxTok tokens on a prepared layer: one
+// persistent kernel (PDL launch after router_decode) that routes the batch
+// in every CTA, streams the layer's streaming copy stage by stage (gate/up,
+// SwiGLU, Q8_0 of h; down; combine) and writes `out`.
+constexpr int kStreamMaxTok = 4;
+constexpr int kStreamMaxSlots = kMaxShared + kStreamMaxTok * kMaxTopK;
+struct StreamArgs {
+  const unsigned char* prep;  // the layer's streaming copy (coli_moe_prepare)
+  StreamGeom g;
+  int E, K, S, T, norm;
+  float rsf;
+  const float* scores;  // [T x E] (router_decode)
+  const float* bias;
+  const int8_t* xq;     // [T x H] Q8_0 of x (router_decode)
+  const float* xd;      // [T x H/32]
+  int8_t* hpl;          // [rows x I/32 x 32]: h of every (slot, token) row as even / odd byte planes
+  float2* hdc;          // [rows x I/32]: (d, -128 * sum of the even plane as int bits)
+  float* y;             // [rows x H]
+  float* out;           // [T x H]
+  int32_t* h_ready;     // [kStreamMaxSlots] gate/up units done per slot (zero at launch)
+  int32_t* dn_done;     // [H/32] slots done per 32-row chunk of the output (zero at launch)
+  int32_t* status;
+};
+bool stream_supported(int hidden, int inter, int n_tok, int n_shared, int top_k);
+uint64_t stream_expert_bytes(int hidden, int inter);
+cudaError_t launch_prepare_expert(int hidden, int inter, const uint8_t* gq, const float* gs, const uint8_t* uq,
+                                  const float* us, const uint8_t* dq, const float* ds, void* dst, cudaStream_t st);
+cudaError_t launch_expert_stream(const StreamArgs& a, cudaStream_t st);
+
 // Prefill expert kernels on the tensor cores (tcgen05): the fp16 operand
 // rows of the Q8 activations, one per (slot, token) in slot order (xf:
 // n_tok*(K+n_shared) x hidden halves), the tile list (<= 128 tokens of one
@@ -154,6 +187,8 @@ void set_error_message(const char* msg);
 //                10 prefill producers (operand stage), 11 prefill MMA (operands),
 //                12 prefill MMA (accumulators), 13 prefill fold (accumulators),
 //                16 prefill TMA warp (operand stage), 22 decode down (h rows),
+//                24 streaming kernel (weight stage), 25 streaming kernel (a
+//                slot's h from other CTAs), 26 streaming kernel (staged h),
 //                30 the test probe coli_debug_wait_probe
 constexpr int32_t kStatusBadExpert = 1;
 constexpr int32_t kStatusTimeoutFirst = 10;

@@ -190,11 +190,14 @@ constexpr int kStageTok = 2;
 __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restrict__ x,
                                                             const float* __restrict__ wr, int n_tok, int E, int H,
                                                             float* __restrict__ scores, int8_t* __restrict__ xq,
-                                                            float* __restrict__ xd, int32_t* status_clear) {
+                                                            float* __restrict__ xd, int32_t* status_clear,
+                                                            int32_t* zero, int n_zero) {
   extern __shared__ __align__(16) float4 wsm[];  // [2][H/4] router rows, then [kStageTok][H/4] tokens
   // first kernel of a decode forward (launched without PDL, so everything
   // before it in the stream is complete): start the status word afresh
   if (status_clear && blockIdx.x == 0 && threadIdx.x == 0) *status_clear = 0;
+  if (zero && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e0 = blockIdx.x * 2;
@@ -436,12 +439,14 @@ cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E
 }
 
 cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
-                                 int8_t* xq, float* xd, int32_t* status_clear, cudaStream_t st) {
+                                 int8_t* xq, float* xd, int32_t* status_clear, int32_t* zero, int n_zero,
+                                 cudaStream_t st) {
   const size_t smem = (size_t)(2 + (n_tok <= kStageTok ? n_tok : 0)) * H * sizeof(float);
   static uint64_t attr_dev_mask = 0;
   const cudaError_t e = smem_opt_in_once(router_decode_kernel, 200 * 1024, attr_dev_mask);
   if (e != cudaSuccess) return e;
-  router_decode_kernel<<<(E + 1) / 2, 256, smem, st>>>(x, w_router, n_tok, E, H, scores, xq, xd, status_clear);
+  router_decode_kernel<<<(E + 1) / 2, 256, smem, st>>>(x, w_router, n_tok, E, H, scores, xq, xd, status_clear,
+                                                       zero, n_zero);
   return cudaGetLastError();
 }
 

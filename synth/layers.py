@@ -3,7 +3,8 @@
 F32 weights come from the device generator (``synth_dev.cu``, the same
 numbers as the host generator) and are packed to int4 by the library's own
 quantiser (``coli_quantize_rows_int4``), one matrix at a time through a
-reusable F32 staging buffer.  Each layer's packed weights live in one
+reusable F32 staging buffer (prepare=True also makes the layer's streaming
+copy with coli_moe_prepare).  Each layer's packed weights live in one
 allocation: experts e = 0..E-1 then the shared experts, each as
 [gate | up | down] blocks of inter*hidden/2 bytes (row-major [out x in]).
 """
@@ -12,7 +13,7 @@ from __future__ import annotations
 import synth
 
 
-def device_layer(cfg: dict, layer: int = 0, device="cuda", staging=None):
+def device_layer(cfg: dict, layer: int = 0, device="cuda", staging=None, prepare: bool = False):
     import torch
 
     import int4_weight_only_sigmoid_b200 as coli
@@ -43,4 +44,6 @@ def device_layer(cfg: dict, layer: int = 0, device="cuda", staging=None):
     L = coli.MoeLayer(ccfg, synth.dev_router_w(cfg, layer, device), synth.dev_bias(cfg, layer, device),
                       experts[:E], experts[E:])
     L._storage = (qbuf, s_gu, s_dn)
+    if prepare:
+        coli.prepare(L)
     return L

@@ -100,6 +100,31 @@ def test_noalloc_rejects_token_counts_outside_range_before_sizing(lib):
         assert b"n_tok" in lib.coli_last_error()
 
 
+def test_prepared_bytes_and_prepare_arguments(lib):
+    """The streaming copy is as large as the row-major weights (plus the
+    scales, each expert padded to 256 bytes); shapes without a streaming
+    layout report 0; bad buffers are refused before any CUDA call."""
+    import int4_weight_only_sigmoid_b200 as m
+    cfg = m.make_config(6144, 2048, 256, 8, 1)
+    per_expert = 3 * 2048 * 6144 // 2 + (2 * 2048 + 6144) * 4
+    per_expert = (per_expert + 255) // 256 * 256
+    assert m.prepared_bytes(cfg) == 257 * per_expert
+    tiny = m.make_config(256, 128, 16, 4, 1)
+    assert m.prepared_bytes(tiny) == 17 * ((3 * 128 * 256 // 2 + (2 * 128 + 256) * 4 + 255) // 256 * 256)
+    assert m.prepared_bytes(m.make_config(384, 128, 16, 4, 1)) == 0  # hidden/32 = 12
+    assert m.prepared_bytes(m.make_config(256, 96, 16, 4, 1)) == 0   # inter not a multiple of 128
+    ex = (m.Expert * 17)(*[m.Expert(256, 256, 256, 256, 256, 256) for _ in range(17)])
+    L = m.MoeLayerC(tiny, 256, 256, C.cast(ex, C.POINTER(m.Expert)), C.cast(ex, C.POINTER(m.Expert)), None)
+    n = m.prepared_bytes(tiny)
+    assert lib.coli_moe_prepare(C.byref(L), None, n, None) == m.COLI_EINVAL
+    assert lib.coli_moe_prepare(C.byref(L), C.c_void_p(4096 + 16), n, None) == m.COLI_EINVAL
+    assert b"aligned" in lib.coli_last_error()
+    assert lib.coli_moe_prepare(C.byref(L), C.c_void_p(4096), n - 1, None) == m.COLI_ENOMEM
+    L.prepared = 4096 + 128  # a forward refuses a misaligned copy too
+    assert lib.coli_moe_layer_forward(C.byref(L), C.c_void_p(256), 1, C.c_void_p(512), C.c_void_p(768), 1 << 20,
+                                      None) == m.COLI_EINVAL
+
+
 def test_zero_tokens_is_ok_without_touching_pointers(lib):
     import int4_weight_only_sigmoid_b200 as m
     assert lib.coli_quantize_act_q8(None, 0, 64, None, None, None) == m.COLI_OK

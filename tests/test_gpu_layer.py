@@ -132,9 +132,13 @@ def test_layer_prefill2048_tile_edges(coli, syn):
     cfg = syn.config("prefill2048")
     edge, cmax, n_ones = _tile_edge_tokens(coli, syn, cfg, 2048)
     assert cmax > 2 * 128 and n_ones >= 1
-    rand = np.random.default_rng(7).choice(2048, 16, replace=False)
-    chosen = sorted(set(edge) | set(int(t) for t in rand))
-    assert len(chosen) >= 32
+    chosen = set(edge)
+    for t in np.random.default_rng(7).permutation(2048):  # plus random tokens, up to 36 in all
+        if len(chosen) >= 36:
+            break
+        chosen.add(int(t))
+    chosen = sorted(chosen)
+    assert len(chosen) >= 32 and len(edge) >= 12
     _check_layer(coli, syn, cfg, 2048, tokens=chosen)
 
 

@@ -1,0 +1,142 @@
+"""The streaming decode path (prepared layers, batches of 1..4 tokens):
+the layout that coli_moe_prepare writes, and the layer output of the
+streaming kernel against the oracle, bit for bit, through the C ABI."""
+import numpy as np
+import pytest
+
+from tests.helpers import assert_layer_close, bits_equal, oracle_layer_forward
+
+pytestmark = pytest.mark.gpu
+
+_cache = {}
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _layer(cfg):
+    from synth.layers import device_layer
+    key = tuple(sorted((k, v) for k, v in cfg.items() if not isinstance(v, (list, dict))))
+    if key not in _cache:
+        if len(_cache) > 2:
+            _cache.clear()
+        _cache[key] = device_layer(cfg, 0, prepare=True)
+    return _cache[key]
+
+
+def _layout_offset(H, I, m, r, b):
+    """Byte offset of block b of row r of matrix m (0 gate, 1 up, 2 down) in
+    one expert's streaming copy, as include/coli.h documents it."""
+    nbh, nbi = H // 32, I // 32
+    if m < 2:
+        G = min(16, nbh)
+        swz = min(G, 8) - 1
+        st_bytes = 64 * G * 16
+        unit_bytes = (nbh // G) * st_bytes
+        sr = (0 if m == 0 else 32) + r % 32
+        s, j = divmod(b, G)
+        return (r // 32) * unit_bytes + s * st_bytes + sr * G * 16 + ((j ^ (sr & swz)) * 16)
+    G = min(32, nbi)
+    swz = min(G, 8) - 1
+    st_bytes = 32 * G * 16
+    unit_bytes = (nbi // G) * st_bytes
+    dn_off = (I // 32) * (nbh // min(16, nbh)) * 64 * min(16, nbh) * 16
+    sr = r % 32
+    s, j = divmod(b, G)
+    return dn_off + (r // 32) * unit_bytes + s * st_bytes + sr * G * 16 + ((j ^ (sr & swz)) * 16)
+
+
+def test_prepare_writes_the_documented_layout(coli, syn):
+    cfg = syn.config("tiny")
+    H, I, E, S = cfg["hidden"], cfg["inter"], cfg["n_experts"], cfg["n_shared"]
+    L = _layer(cfg)
+    prep = _np(L.prepared)
+    eb = len(prep) // (E + S)
+    assert eb * (E + S) == len(prep) and eb % 256 == 0
+    for j, ex in enumerate(L.experts + L.shared):
+        base = j * eb
+        mats = [_np(ex.gate_q), _np(ex.up_q), _np(ex.down_q)]
+        for m, q in enumerate(mats):
+            rows, nb = q.shape[0], q.shape[1] // 16
+            for r in range(rows):
+                for b in range(nb):
+                    o = base + _layout_offset(H, I, m, r, b)
+                    assert np.array_equal(prep[o:o + 16], q[r, 16 * b:16 * b + 16]), (j, m, r, b)
+        nbh, nbi = H // 32, I // 32
+        gu_bytes = (I // 32) * (nbh // min(16, nbh)) * 64 * min(16, nbh) * 16
+        dn_bytes = (H // 32) * (nbi // min(32, nbi)) * 32 * min(32, nbi) * 16
+        sc = prep[base + gu_bytes + dn_bytes:base + gu_bytes + dn_bytes + (2 * I + H) * 4].view(np.float32)
+        assert bits_equal(sc[:I], _np(ex.gate_s)) and bits_equal(sc[I:2 * I], _np(ex.up_s))
+        assert bits_equal(sc[2 * I:], _np(ex.down_s))
+
+
+def _check(coli, syn, cfg, n_tok, tokens=None):
+    import torch
+    L = _layer(cfg)
+    x = syn.tokens(cfg, n_tok) if tokens is None else tokens
+    xt = torch.from_numpy(x).cuda()
+    out = _np(coli.moe_layer_forward(L, xt))
+    plain = _np(coli.moe_layer_forward(L, xt, cstruct=L.cstruct(use_prepared=False)))
+    want, idx, _, _ = oracle_layer_forward(cfg, x)
+    assert_layer_close(out, want)
+    assert bits_equal(out, want)
+    assert bits_equal(out, plain)
+    return out
+
+
+@pytest.mark.parametrize("n_tok", [1, 2, 3, 4])
+def test_stream_tiny(coli, syn, n_tok):
+    _check(coli, syn, syn.config("tiny"), n_tok)
+
+
+@pytest.mark.parametrize("over", [dict(norm_topk_prob=False), dict(top_k=1), dict(top_k=16), dict(n_shared=0),
+                                  dict(n_shared=2), dict(routed_scaling_factor=1.0)])
+def test_stream_tiny_variants(coli, syn, over):
+    _check(coli, syn, syn.config("tiny", **over), 4)
+
+
+def test_stream_all_tokens_on_one_expert(coli, syn):
+    """Four identical tokens: every routed slot holds all 4 tokens."""
+    cfg = syn.config("tiny")
+    x = np.repeat(syn.tokens(cfg, 1), 4, axis=0)
+    _check(coli, syn, cfg, 4, tokens=x)
+
+
+@pytest.mark.parametrize("name,n_tok", [("decode1", 1), ("decode4", 4), ("decode4", 2), ("decode4", 3)])
+def test_stream_glm(coli, syn, name, n_tok):
+    _check(coli, syn, syn.config(name), n_tok)
+
+
+@pytest.mark.parametrize("name,n_tok", [("decode1", 1), ("decode4", 4), ("tiny", 3)])
+def test_stream_workspace_contents_do_not_matter(coli, syn, name, n_tok):
+    """Workspaces filled with 0x00 / 0x5A / 0xFF (stale counters, stale h)
+    before each call give the same bits: the router kernel clears the
+    counters and every scratch word is written before it is read."""
+    import torch
+    cfg = syn.config(name)
+    L = _layer(cfg)
+    x = torch.from_numpy(syn.tokens(cfg, n_tok)).cuda()
+    ref = _np(coli.moe_layer_forward(L, x))
+    for it in range(12):
+        ws = coli.make_workspace(L.cfg, n_tok)
+        ws.fill_((0x00, 0x5A, 0xFF)[it % 3])
+        got = _np(coli.moe_layer_forward(L, x, workspace=ws))
+        assert bits_equal(got, ref), f"iteration {it}"
+        assert coli.sync_status(ws) == coli.COLI_OK
+
+
+def test_stream_repeated_calls_one_workspace(coli, syn):
+    """Back-to-back forwards on one stream and one workspace (the counters
+    of one call must not leak into the next)."""
+    import torch
+    cfg = syn.config("decode4")
+    L = _layer(cfg)
+    xs = [torch.from_numpy(syn.tokens(cfg, 4)[::-1].copy()).cuda(), torch.from_numpy(syn.tokens(cfg, 4)).cuda()]
+    ws = coli.make_workspace(L.cfg, 4)
+    refs = [_np(coli.moe_layer_forward(L, x, cstruct=L.cstruct(use_prepared=False))) for x in xs]
+    outs = [torch.empty_like(xs[0]) for _ in range(20)]
+    for i in range(20):
+        coli.moe_layer_forward(L, xs[i % 2], out=outs[i], workspace=ws)
+    for i in range(20):
+        assert bits_equal(_np(outs[i]), refs[i % 2]), i

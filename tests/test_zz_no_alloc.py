@@ -21,13 +21,15 @@ def _close(got, want, rel=2e-3):
     assert err <= rel * np.sqrt((want ** 2).mean()), err
 
 
-@pytest.mark.parametrize("name,n_tok", [("tiny", 8), ("tiny", 3), ("tiny", 40), ("decode1", 1), ("decode16", 16),
-                                        ("decode16", 17)])  # 17 GLM tokens: the tensor-core path, the documented limit
-def test_noalloc_matches_workspace_forward_twice(coli, syn, name, n_tok):
+@pytest.mark.parametrize("name,n_tok,prep", [("tiny", 8, False), ("tiny", 3, False), ("tiny", 40, False),
+                                             ("decode1", 1, False), ("decode16", 16, False),
+                                             ("decode16", 17, False),  # the tensor-core path, the documented limit
+                                             ("decode4", 4, True)])     # the streaming path of a prepared layer
+def test_noalloc_matches_workspace_forward_twice(coli, syn, name, n_tok, prep):
     import torch
     from synth.layers import device_layer
     cfg = syn.config(name)
-    L = device_layer(cfg, 0)
+    L = device_layer(cfg, 0, prepare=prep)
     x = torch.from_numpy(syn.tokens(cfg, n_tok)).cuda()
     want = coli.moe_layer_forward(L, x).cpu().numpy()
     for _ in range(2):
