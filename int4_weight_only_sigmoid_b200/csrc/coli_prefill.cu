@@ -1,9 +1,9 @@
 // coli_prefill.cu -- the expert kernels for many tokens per expert (prefill):
-// a grouped GEMM on the 5th-generation tensor cores (tcgen05.mma, F32
-// accumulators in tensor memory).  Work items are (tile of <= 128 of one
-// slot's tokens, 128 output columns); one persistent CTA per SM walks items
-// c, c + G, ... and keeps its pipeline (producers -> MMA -> fold) running
-// from one item to the next.
+// a grouped int8 GEMM on the 5th-generation tensor cores
+// (tcgen05.mma.kind::i8, int32 accumulators in tensor memory).  Work items
+// are (tile of <= 128 of one slot's tokens, 128 output columns); one
+// persistent CTA per SM walks items c, c + G, ... and keeps its pipeline
+// (producers -> MMA -> fold) running from one item to the next.
 //
 // Orientation.  The tokens are the MMA's M dimension (TMEM lanes) and the
 // weight rows its N dimension (TMEM columns), so a fold thread owns one
@@ -12,30 +12,25 @@
 // matching up rows, so SwiGLU and the Q8 block of h are thread-local.  The
 // gate/up item's 128 columns are 64 gate rows and the same 64 up rows.
 //
+// Operands.  A = the Q8 activations as signed bytes (one row per (slot,
+// token) in slot order, loaded by TMA, 128-byte swizzle); B = the weights as
+// unsigned bytes q + 8 (0..15), expanded from the packed nibbles by the
+// producer warps: for a packed word w, (w & 0x0F0F0F0F) ^ 0x08080808 holds
+// q + 8 of elements 0, 2, 4, 6 and ((w >> 4) & 0x0F0F0F0F) ^ 0x08080808 of
+// elements 1, 3, 5, 7 -- three logic ops per 8 weights, and the A rows are
+// stored in the same order (per 8 elements: 0,2,4,6,1,3,5,7), so the dot
+// product is unchanged.  One MMA (K = 32) is exactly one Q8 block.
+//
 // Exactness.  Each Q8 block's partial sum must come out exactly, because the
 // row fold (contract F: acc = fmaf(d_x[b], (float)isum[b], acc), b
-// ascending) needs it per block.  The operands are therefore fp16, in which
-// every int4 weight (-8..7) and every Q8 activation (-127..127) is exact;
-// the MMA of one 32-element block (two K=16 steps) accumulates products of
-// at most 8*127 into an F32 sum of magnitude at most 32512 < 2^24, so every
-// partial sum is an exact integer in F32 whatever the tensor core's internal
-// order.  The MMA of block b writes a fresh accumulator; the fold warps then
-// fold it with d_x[b] in ascending b.  The results equal the dp4a path's bit
-// for bit.
-//
-// Why fp16 operands and not kind::i8: the fold costs one F32 FMA per
-// (row, token, block) whatever the MMA kind; with kind::i8 each of those
-// also needs an int32 -> F32 conversion, and the CUDA cores (weight
-// expansion and the fold), not the tensor pipe, are the limit of this layer.
-// fp16 operands give F32 sums directly.
-//
-// Operands.  The activations are converted to fp16 once per forward, one
-// row per (slot, token) in slot order (act_rows_f16_kernel; the gate/up fold
-// writes h straight as fp16 rows in the same order for the down kernel), in
-// the element order [0,4,1,5,2,6,3,7] of every 8 that the int4 expansion
-// produces; a tile's A operand is then 128 consecutive rows, loaded by TMA
-// (128-byte swizzle).  The packed weights are copied by the producer warps
-// with cp.async and expanded into the B operand (K-major, no swizzle).
+// ascending) needs it per block.  The MMA of block b adds
+// sum (q + 8) x = isum + 8 * sum(x) to an int32 accumulator that holds
+// M = 0x4B400000 - 8 * sum(x) (the token's block sum, written by the fold
+// before the MMA runs), so the accumulator ends as 0x4B400000 + isum: read as
+// a binary32 that is 1.5 * 2^23 + isum exactly (|isum| <= 32512 < 2^22), and
+// one F32 subtraction gives (float)isum with no integer-to-float
+// conversion.  The fold then applies contract F per block, so prefill equals
+// the dp4a paths bit for bit.
 //
 // Roles (448 threads): warps 0-3 producers (packed-weight copies; thread p
 // expands weight row p), warp 4 the A-tile TMA loads, warps 5-12 the fold
@@ -45,10 +40,12 @@
 // loads its A tile into operand stage g % kStages once `empty` (the MMA's
 // commit) says the stage is free; the producers copy its packed weights
 // kLookS stages ahead (cp.async), expand them into the stage's B part and
-// arrive on `full`; the MMA issues two K=16 steps per block into a fresh
-// TMEM accumulator per block (4 of them, handed to the fold kHalf blocks at
-// a time through `tfull` / `tempty`) and commits `empty`.  All waits are
-// bounded (coli_tc.cuh).
+// arrive on `full`; the MMA issues one K=32 step per block onto a TMEM
+// accumulator per block (4 of them, handed to the fold kHalf blocks at a
+// time through `tfull` / `tempty`) and commits `empty`.  The fold reads a
+// buffer, writes the starting value M of the buffer's next use (the same
+// token slot one stage later, or the CTA's next item) and releases it.  All
+// waits are bounded (coli_tc.cuh).
 //
 // Sources: "Colibri：在笔记本上跑744B参数的AI模型", "关键特性" (integer dot
 // kernels, Q8_0 activations, packed int4); HN summary (hn.213312.xyz),
@@ -56,8 +53,6 @@
 // positions is read once and shared).
 #include <cuda.h>
 #include <cudaTypedefs.h>
-#include <type_traits>
-#include <cuda_fp16.h>
 
 #include "coli_launch.h"
 #include "coli_tc.cuh"
@@ -70,7 +65,7 @@ using namespace tc;
 constexpr int kM = 128;        // tokens per tile (MMA M, TMEM lanes)
 constexpr int kN = 128;        // output columns per item (MMA N): 64 gate + 64 up rows, or 128 down rows
 constexpr int kBS = 4;         // Q8 blocks per operand stage (K = 128)
-constexpr int kStages = 3;     // operand stages
+constexpr int kStages = 4;     // operand stages
 constexpr int kLookS = 2;      // stages the producers' copies run ahead
 constexpr int kPkSlots = kLookS + 2;  // packed-weight slots: a slot is rewritten only after every producer expanded it
 constexpr int kHalf = 2;       // Q8 blocks per accumulator hand-off (MMA -> fold)
@@ -86,11 +81,12 @@ constexpr int kMmaWarp = kEpi0 + kEpiWarps;                    // MMA issuer, TM
 constexpr int kThreadsP = 32 * (kMmaWarp + 1);                 // 448
 constexpr int kNProd = 32 * kProdWarps;                        // 128 producer threads
 constexpr int kTmemCols = kTBufs * kN;                         // 512
+constexpr uint32_t kMagic = 0x4B400000u;                       // binary32 1.5 * 2^23
+constexpr float kMagicF = 12582912.0f;
 
 struct PSmem {
-  static constexpr int kAtomA = kM * 128;           // A: 128 token rows x 64 fp16 (two blocks), 128B-swizzled
-  static constexpr int kStageA = 2 * kAtomA;        // a stage's 4 blocks
-  static constexpr int kSubB = kN * 64;             // B, one block: 128 weight rows x 32 fp16
+  static constexpr int kStageA = kM * 128;          // A: 128 token rows x 128 int8 (4 blocks), 128B-swizzled
+  static constexpr int kSubB = kN * 32;             // B, one block: 128 weight rows x 32 bytes
   static constexpr int kOpStage = kStageA + kBS * kSubB;
   static constexpr int kPk = kN * kBS * 16;         // packed weights of one stage (row-major, 64 B per row)
   __host__ __device__ static constexpr size_t bytes() {
@@ -102,79 +98,61 @@ struct Tile {
   int32_t slot, n0;
 };
 
-// fp16 operands from packed int4: the 8 nibbles of one 32-bit word (element
-// e in bits 4e..4e+3, two's complement) -> 8 fp16 in the order
-// [0,4,1,5,2,6,3,7] (the activations use the same order, so the dot product
-// is unchanged).  (w & 0x000F000F) ^ 0x64086408 is the fp16 pair
-// 1024 + (q + 8) for elements 0 and 4 exactly; the nibbles one position up
-// give 1024 + 16 (q + 8), which x 1/16 - 72 maps to q exactly.
-__device__ __forceinline__ uint4 expand_int4_word(uint32_t w) {
-  const uint32_t w8 = w >> 8;
-  uint32_t r[4] = {(w & 0x000F000Fu) ^ 0x64086408u, (w & 0x00F000F0u) ^ 0x64806480u,
-                   (w8 & 0x000F000Fu) ^ 0x64086408u, (w8 & 0x00F000F0u) ^ 0x64806480u};
-  const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));        // 1032
-  const __half2 sixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
-  const __half2 m72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));        // -72
-  uint4 o;
-  __half2 h;
-  h = __hsub2(*reinterpret_cast<__half2*>(&r[0]), off);
-  o.x = *reinterpret_cast<uint32_t*>(&h);
-  h = __hfma2(*reinterpret_cast<__half2*>(&r[1]), sixteenth, m72);
-  o.y = *reinterpret_cast<uint32_t*>(&h);
-  h = __hsub2(*reinterpret_cast<__half2*>(&r[2]), off);
-  o.z = *reinterpret_cast<uint32_t*>(&h);
-  h = __hfma2(*reinterpret_cast<__half2*>(&r[3]), sixteenth, m72);
-  o.w = *reinterpret_cast<uint32_t*>(&h);
-  return o;
-}
-
-// fp16 operands from 8 int8 values (words a = x0..x3, b = x4..x7), same
-// element order: with u = x + 128, 0x6400 | u is 1024 + u; minus 1152 is x.
-__device__ __forceinline__ uint4 expand_int8_pair(uint32_t a, uint32_t b) {
-  const uint32_t ua = a ^ 0x80808080u, ub = b ^ 0x80808080u;
-  const uint32_t t0 = __byte_perm(ua, ub, 0x5140), t1 = __byte_perm(ua, ub, 0x7362);  // u0 u4 u1 u5 | u2 u6 u3 u7
-  const uint32_t c = 0x64646464u;
-  const __half2 off = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));  // 1152, 1152
-  uint32_t r[4] = {__byte_perm(t0, c, 0x4140), __byte_perm(t0, c, 0x4342), __byte_perm(t1, c, 0x4140),
-                   __byte_perm(t1, c, 0x4342)};
-  uint4 o;
-  __half2 h;
-  h = __hsub2(*reinterpret_cast<__half2*>(&r[0]), off);
-  o.x = *reinterpret_cast<uint32_t*>(&h);
-  h = __hsub2(*reinterpret_cast<__half2*>(&r[1]), off);
-  o.y = *reinterpret_cast<uint32_t*>(&h);
-  h = __hsub2(*reinterpret_cast<__half2*>(&r[2]), off);
-  o.z = *reinterpret_cast<uint32_t*>(&h);
-  h = __hsub2(*reinterpret_cast<__half2*>(&r[3]), off);
-  o.w = *reinterpret_cast<uint32_t*>(&h);
-  return o;
-}
-
 // Byte offset of packed block c (0..3) of weight row r in a stage's packed
 // copy: 64 B per row, blocks rotated by (r >> 1) & 3 so that 8 consecutive
 // rows reading the same block hit 8 different bank groups.
 __device__ __forceinline__ uint32_t pk_off(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
 
-// Byte offset of 16-byte chunk c (0..3) of row r in a K-major, no-swizzle
-// operand tile of 32 fp16 per row: 8-row x 16-byte core matrices, the four
-// K chunks of an 8-row group 128 B apart (LBO), groups 512 B apart (SBO).
-__device__ __forceinline__ uint32_t op_off(int r, int c) { return (r >> 3) * 512 + c * 128 + (r & 7) * 16; }
+// Byte offset of 16-byte chunk c (0..1) of row r in a K-major, no-swizzle
+// operand tile of 32 bytes per row: 8-row x 16-byte core matrices, the two
+// K chunks of an 8-row group 128 B apart (LBO), groups 256 B apart (SBO).
+__device__ __forceinline__ uint32_t op_off(int r, int c) { return (r >> 3) * 256 + c * 128 + (r & 7) * 16; }
 
-// fp16 operand rows of the Q8 activations in row order: row r < n_tok*K is
+// q + 8 of the 8 nibbles of a packed word, as unsigned bytes in the order
+// 0,2,4,6 (lo) then 1,3,5,7 (hi).
+__device__ __forceinline__ void expand_word(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
+  hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+}
+
+// Operand rows of the Q8 activations in row order: row r < n_tok*K is
 // token perm[r] / K (the routed slots' rows), row n_tok*K + s*n_tok + t is
-// token t (shared expert s).  8 values per thread.
-__global__ void __launch_bounds__(256) act_rows_f16_kernel(const int8_t* __restrict__ q, const int32_t* perm,
-                                                           int n_tok, int top_k, int64_t rows, int hidden,
-                                                           uint4* __restrict__ out) {
+// token t (shared expert s); within every 8 elements the order 0,2,4,6,1,3,5,7.
+// 16 values per thread.
+__global__ void __launch_bounds__(256) act_rows_i8_kernel(const int8_t* __restrict__ q, const int32_t* perm,
+                                                          int n_tok, int top_k, int64_t rows, int hidden,
+                                                          uint4* __restrict__ out) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int per_row = hidden / 8;
+  const int per_row = hidden / 16;
   if (i >= rows * per_row) return;
   const int64_t r = i / per_row;
   const int c = (int)(i - r * per_row);
   const int64_t routed = (int64_t)n_tok * top_k;
   const int64_t tok = r < routed ? (int64_t)(__ldg(perm + r) / top_k) : (r - routed) % n_tok;
-  const uint2 v = __ldg(reinterpret_cast<const uint2*>(q + tok * hidden) + c);
-  out[i] = expand_int8_pair(v.x, v.y);
+  const uint4 v = __ldg(reinterpret_cast<const uint4*>(q + tok * hidden) + c);
+  uint4 o;
+  split_even_odd(v.x, v.y, o.x, o.y);
+  split_even_odd(v.z, v.w, o.z, o.w);
+  out[i] = o;
+}
+
+// Starting accumulator value of every (token, block): 0x4B400000 - 8 * sum
+// of the block's 32 values.  One thread per block.
+__global__ void __launch_bounds__(256) act_magic_kernel(const int8_t* __restrict__ q, int64_t n_blocks,
+                                                        int32_t* __restrict__ mag) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_blocks) return;
+  const uint4* p = reinterpret_cast<const uint4*>(q + 32 * i);
+  const uint4 a = __ldg(p), b = __ldg(p + 1);
+  int s = __dp4a((int)a.x, 0x01010101, 0);
+  s = __dp4a((int)a.y, 0x01010101, s);
+  s = __dp4a((int)a.z, 0x01010101, s);
+  s = __dp4a((int)a.w, 0x01010101, s);
+  s = __dp4a((int)b.x, 0x01010101, s);
+  s = __dp4a((int)b.y, 0x01010101, s);
+  s = __dp4a((int)b.z, 0x01010101, s);
+  s = __dp4a((int)b.w, 0x01010101, s);
+  mag[i] = (int32_t)(kMagic - (uint32_t)(8 * s));
 }
 
 // 2D tiled bulk-tensor load (TMA) of box (x, y) into shared memory,
@@ -205,7 +183,37 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
   return d;
 }
 
-// fma on two F32 lanes at once (two IEEE fmas, each rounded once).
+// Instruction descriptor of kind::i8: signed A (activations), unsigned B
+// (weights + 8), int32 accumulator, shape M x N, both K-major.
+__host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N) {
+  return (2u << 4)                       // D format: S32
+         | (1u << 7)                     // A format: S8
+         | (0u << 10)                    // B format: U8
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// D[tmem] += A[smem] * B[smem]^T (int8, int32 accumulate), issued by one thread.
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, 1, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc)
+      : "memory");
+}
+
+// 16 consecutive 32-bit TMEM columns of this warp's 32 lanes <- v (each
+// lane writes its own value in all 16 columns).
+__device__ __forceinline__ void tmem_st16_same(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(v)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// fma / add on two F32 lanes at once (each lane one IEEE operation, rounded once).
 __device__ __forceinline__ void fma2(float& a0, float& a1, float d0, float d1, float x0, float x1) {
   unsigned long long acc, dd, xx;
   asm("mov.b64 %0, {%1,%2};" : "=l"(acc) : "f"(a0), "f"(a1));
@@ -214,11 +222,13 @@ __device__ __forceinline__ void fma2(float& a0, float& a1, float d0, float d1, f
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(dd), "l"(xx));
   asm("mov.b64 {%0,%1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
 }
-
-// A fold thread's token scales for one hand-off (kHalf blocks).
-using DVec = std::conditional_t<kHalf == 2, float2, float>;
-[[maybe_unused]] __device__ __forceinline__ float dvec_at(const float2& v, int i) { return i == 0 ? v.x : v.y; }
-[[maybe_unused]] __device__ __forceinline__ float dvec_at(float v, int) { return v; }
+__device__ __forceinline__ void sub2(float& x0, float& x1, float c) {
+  unsigned long long xx, cc;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(xx) : "f"(x0), "f"(x1));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(cc) : "f"(c));
+  asm("sub.rn.f32x2 %0, %0, %1;" : "+l"(xx) : "l"(cc));
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(x0), "=f"(x1) : "l"(xx));
+}
 
 struct ItemInfo {
   Slot slot;
@@ -238,19 +248,21 @@ __device__ __forceinline__ ItemInfo item_info(const Slot* slots, const Tile* til
   return f;
 }
 
-// Source row (into the activation / h rows) of token n of the item's tile.
+// Row of token n of the item's tile in the per-token arrays: gate/up: the
+// token itself (x's scales and block sums); down: the (slot, token) row.
 __device__ __forceinline__ int64_t item_token_row(const ItemInfo& f, bool gu, const int32_t* perm, int top_k, int n) {
   if (!gu) return (int64_t)f.slot.row_base + f.n0 + n;
   return f.slot.perm_base < 0 ? (int64_t)(f.n0 + n) : (int64_t)(perm[f.slot.perm_base + f.n0 + n] / top_k);
 }
 
-// GU: gate/up (+ SwiGLU + Q8 of h -> hf fp16 rows + hd); !GU: down (-> y).
+// GU: gate/up (+ SwiGLU + Q8 of h -> hr int8 rows + hd + hm); !GU: down (-> y).
+// ad / am: the A rows' Q8 scales and starting values, [row x nb].
 template <bool GU, typename Tab>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     const __grid_constant__ Tab tab, const __grid_constant__ CUtensorMap amap, const Slot* __restrict__ slots,
-    const Tile* __restrict__ tiles,
-    const int32_t* __restrict__ n_tiles, const int32_t* __restrict__ perm, int top_k, const float* ad, int hidden,
-    int inter, __half* hf, float* hd, float* __restrict__ y, int32_t* __restrict__ err) {
+    const Tile* __restrict__ tiles, const int32_t* __restrict__ n_tiles, const int32_t* __restrict__ perm, int top_k,
+    const float* ad, const int32_t* am, int hidden, int inter, int8_t* hr, float* hd, int32_t* hm,
+    float* __restrict__ y, int32_t* __restrict__ err) {
   using L = PSmem;
   constexpr int kGroupRows = GU ? kN / 2 : kN;  // output rows of one matrix per item
   __shared__ uint64_t full_bar[kStages], empty_bar[kStages], tfull_bar[kTBufs / kHalf], tempty_bar[kTBufs / kHalf],
@@ -268,7 +280,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1 KB aligned
-  unsigned char* op_ring = smem;                                  // [kStages][A: 2 atoms | B: kBS x kSubB]
+  unsigned char* op_ring = smem;                                  // [kStages][A | B: kBS x kSubB]
   unsigned char* pk_ring = op_ring + kStages * L::kOpStage;       // [kPkSlots][128 rows][64 B]
 
   if (threadIdx.x == 0) {
@@ -354,10 +366,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         for (int c = 0; c < kBS; ++c) {
           const uint4 w = *reinterpret_cast<const uint4*>(pk + pk_off(p, c));
           unsigned char* dst = ob + c * L::kSubB;
-          *reinterpret_cast<uint4*>(dst + op_off(p, 0)) = expand_int4_word(w.x);
-          *reinterpret_cast<uint4*>(dst + op_off(p, 1)) = expand_int4_word(w.y);
-          *reinterpret_cast<uint4*>(dst + op_off(p, 2)) = expand_int4_word(w.z);
-          *reinterpret_cast<uint4*>(dst + op_off(p, 3)) = expand_int4_word(w.w);
+          uint4 o0, o1;
+          expand_word(w.x, o0.x, o0.y);
+          expand_word(w.y, o0.z, o0.w);
+          expand_word(w.z, o1.x, o1.y);
+          expand_word(w.w, o1.z, o1.w);
+          *reinterpret_cast<uint4*>(dst + op_off(p, 0)) = o0;
+          *reinterpret_cast<uint4*>(dst + op_off(p, 1)) = o1;
         }
       }
       fence_async_smem();  // this thread's operand writes (stores and cp.async) -> the tensor core
@@ -370,7 +385,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     if (lane == 0) {
       int gs = 0, gh = 0;
       bool ok = true;
-      constexpr uint32_t idesc = idesc_f16_f32(kM, kN);
+      constexpr uint32_t idesc = idesc_i8_s32(kM, kN);
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
         for (int j = 0; j < nst && ok; ++j, ++gs) {
           const int s = gs % kStages;
@@ -384,21 +399,19 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
 #pragma unroll
           for (int hh = 0; hh < kBS / kHalf; ++hh, ++gh) {
             const int hb = gh % (kTBufs / kHalf);
-            if (!mbar_wait(&tempty_bar[hb], ((gh / (kTBufs / kHalf)) & 1) ^ 1, abort, err, 12)) {
+            // the fold has read the pair's previous values and written their starting values
+            if (!mbar_wait(&tempty_bar[hb], (gh / (kTBufs / kHalf)) & 1, abort, err, 12)) {
               ok = false;
               break;
             }
             fence_after_sync();
 #pragma unroll
             for (int i = 0; i < kHalf; ++i) {
-              const int c = hh * kHalf + i;  // block within the stage
+              const int c = hh * kHalf + i;  // block within the stage: one K=32 step
               const uint32_t d = tmem + (hb * kHalf + i) * kN;
-#pragma unroll
-              for (int k = 0; k < 2; ++k) {  // two K=16 steps = one Q8 block
-                const uint64_t da = smem_desc_k_sw128(opa + (c >> 1) * L::kAtomA + (c & 1) * 64 + k * 32);
-                const uint64_t db = smem_desc_k_noswizzle(opb + c * L::kSubB + k * 256, 128, 512);
-                mma_f16(d, da, db, idesc, k);
-              }
+              const uint64_t da = smem_desc_k_sw128(opa + c * 32);
+              const uint64_t db = smem_desc_k_noswizzle(opb + c * L::kSubB, 128, 256);
+              mma_i8(d, da, db, idesc);
             }
             mma_commit(&tfull_bar[hb]);
           }
@@ -415,7 +428,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
   } else if (warp == kTmaWarp) {
     // ------------------------------------------------------------ A tiles
     // For each stage: once the MMA is done with the operand stage, one
-    // expect_tx arrival on `full` and two TMA loads of 128 rows x 64 fp16
+    // expect_tx arrival on `full` and one TMA load of 128 rows x 128 bytes
     // (128-byte swizzle) of the row-ordered activations (gate/up) or h
     // (down), rows [row_base + n0, +128) of the item's slot.
     if (lane == 0) {
@@ -433,7 +446,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           unsigned char* oa = op_ring + s * L::kOpStage;
           mbar_arrive_expect_tx(&full_bar[s], L::kStageA);
           tma_load_2d(oa, &amap, j * kBS * 32, row0, &full_bar[s]);
-          tma_load_2d(oa + L::kAtomA, &amap, j * kBS * 32 + 64, row0, &full_bar[s]);
         }
       }
     }
@@ -448,37 +460,67 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     const int c1 = GU ? kGroupRows + 32 * hh : 64 * hh + 32;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const int n = quad * 32 + lane;  // this thread's token within the tile
+    constexpr int kHandPerStage = kBS / kHalf;
+    // starting value of this thread's lane for block b of item `it` (0 if
+    // the lane holds no token there: that lane's result is never read)
+    auto start_value = [&](int it, int b) -> uint32_t {
+      if (it >= n_items) return kMagic;
+      const ItemInfo f = item_info(slots, tiles, it, nm, kGroupRows);
+      if (n >= f.n_valid) return kMagic;
+      return (uint32_t)__ldg(am + item_token_row(f, GU, perm, top_k, n) * nb + b);
+    };
+    auto write_start = [&](int buf, uint32_t v) {
+      const uint32_t col = tmem + lane_base + buf * kN;
+      tmem_st16_same(col + c0, v);
+      tmem_st16_same(col + c0 + 16, v);
+      tmem_st16_same(col + c1, v);
+      tmem_st16_same(col + c1 + 16, v);
+    };
+    // first use of every buffer: blocks 0..3 of the CTA's first item
+    if ((int)blockIdx.x < n_items) {
+#pragma unroll
+      for (int b = 0; b < kTBufs; ++b) write_start(b, start_value(blockIdx.x, b));
+      tmem_st_wait();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0)
+        for (int h = 0; h < kTBufs / kHalf; ++h) mbar_arrive(&tempty_bar[h]);
+    }
     int gh = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
       const bool active = quad * 32 < f.n_valid;  // warp-uniform
       const bool valid = n < f.n_valid;
-      const float* drow = ad + (valid ? item_token_row(f, GU, perm, top_k, n) : 0) * nb;
+      const int64_t trow = valid ? item_token_row(f, GU, perm, top_k, n) : 0;
+      const float* drow = ad + trow * nb;
+      const int32_t* mrow = am + trow * nb;
+      // the next item's starting values for its first stage (this thread's lane)
+      const int nxt = item + gridDim.x;
+      int64_t nrow = -1;
+      if (nxt < n_items) {
+        const ItemInfo fn = item_info(slots, tiles, nxt, nm, kGroupRows);
+        if (n < fn.n_valid) nrow = item_token_row(fn, GU, perm, top_k, n);
+      }
       float acc0[32], acc1[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         acc0[j] = 0.0f;
         acc1[j] = 0.0f;
       }
-      // this token's scales, one hand-off (kHalf blocks) per load, one hand-off ahead
-      const DVec* dp = reinterpret_cast<const DVec*>(drow);
-      DVec dnext = valid ? __ldg(dp) : DVec{};
       for (int j = 0; j < nst; ++j) {
 #pragma unroll
-        for (int hs = 0; hs < kBS / kHalf; ++hs, ++gh) {
-          const DVec dcur = dnext;
-          const int hn = j * (kBS / kHalf) + hs + 1;  // next hand-off of this item
-          if (valid && hn < nst * (kBS / kHalf)) dnext = __ldg(dp + hn);
+        for (int hs = 0; hs < kHandPerStage; ++hs, ++gh) {
           const int hb = gh % (kTBufs / kHalf);
           // warp-uniform: tcgen05.ld is a warp-wide instruction
           const bool ok =
               __all_sync(0xffffffffu, mbar_wait(&tfull_bar[hb], (gh / (kTBufs / kHalf)) & 1, abort, err, 13));
           fence_after_sync();
-          if (active && ok) {
 #pragma unroll
-            for (int i = 0; i < kHalf; ++i) {
-              const float dx = dvec_at(dcur, i);
-              const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
+          for (int i = 0; i < kHalf; ++i) {
+            const int b = j * kBS + hs * kHalf + i;  // block of this item
+            const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
+            if (active && ok) {
+              const float dx = valid ? __ldg(drow + b) : 0.0f;
               // 8 columns of each range at a time (one wait per pair of
               // loads), so that only 16 TMEM values are live
 #pragma unroll
@@ -489,14 +531,26 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
                 tmem_ld_wait();
 #pragma unroll
                 for (int jj = 0; jj < 8; jj += 2) {
-                  fma2(acc0[8 * h + jj], acc0[8 * h + jj + 1], dx, dx, __uint_as_float(r0[jj]),
-                       __uint_as_float(r0[jj + 1]));
-                  fma2(acc1[8 * h + jj], acc1[8 * h + jj + 1], dx, dx, __uint_as_float(r1[jj]),
-                       __uint_as_float(r1[jj + 1]));
+                  float v0 = __uint_as_float(r0[jj]), v1 = __uint_as_float(r0[jj + 1]);
+                  float u0 = __uint_as_float(r1[jj]), u1 = __uint_as_float(r1[jj + 1]);
+                  sub2(v0, v1, kMagicF);  // exact: (float)isum
+                  sub2(u0, u1, kMagicF);
+                  fma2(acc0[8 * h + jj], acc0[8 * h + jj + 1], dx, dx, v0, v1);
+                  fma2(acc1[8 * h + jj], acc1[8 * h + jj + 1], dx, dx, u0, u1);
                 }
               }
             }
+            // the buffer's next use: block b + kBS of this item, else block
+            // b + kBS - nb of the next item
+            uint32_t v = kMagic;
+            if (b + kBS < nb) {
+              if (valid) v = (uint32_t)__ldg(mrow + b + kBS);
+            } else if (nrow >= 0) {
+              v = (uint32_t)__ldg(am + nrow * nb + (b + kBS - nb));
+            }
+            write_start(hb * kHalf + i, v);
           }
+          tmem_st_wait();
           fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty_bar[hb]);  // the pair of TMEM buffers may be rewritten now
@@ -518,21 +572,27 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
             amax = fmaxf(amax, fabsf(acc0[j]));
           }
           const float d = __fdiv_rn(amax, 127.0f);
-          // fp16 of q in the operand order: position 2(e&3) + (e>>2) of each 8
-          uint32_t pk[16];
+          // q in the operand order (per 8 elements: 0,2,4,6,1,3,5,7) and the block sum
+          uint32_t pk[8];
+          int sum = 0;
 #pragma unroll
           for (int e8 = 0; e8 < 4; ++e8) {
+            uint32_t lo = 0, hi = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const __half lo = __int2half_rn(q8_of(acc0[8 * e8 + i], d));
-              const __half hi = __int2half_rn(q8_of(acc0[8 * e8 + 4 + i], d));
-              pk[4 * e8 + i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+              const int qe = q8_of(acc0[8 * e8 + 2 * i], d), qo = q8_of(acc0[8 * e8 + 2 * i + 1], d);
+              sum += qe + qo;
+              lo |= ((uint32_t)qe & 0xFFu) << (8 * i);
+              hi |= ((uint32_t)qo & 0xFFu) << (8 * i);
             }
+            pk[2 * e8] = lo;
+            pk[2 * e8 + 1] = hi;
           }
-          uint4* dst = reinterpret_cast<uint4*>(hf + row * inter + o);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          uint4* dst = reinterpret_cast<uint4*>(hr + row * inter + o);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           hd[row * (inter / 32) + (o >> 5)] = d;
+          hm[row * (inter / 32) + (o >> 5)] = (int32_t)(kMagic - (uint32_t)(8 * sum));
         } else {
           const float* sdp = tab.down_s[f.slot.table_idx] + f.m0;
           float4* dst0 = reinterpret_cast<float4*>(y + row * hidden + f.m0 + c0);
@@ -583,20 +643,6 @@ __global__ void build_tiles_kernel(const Slot* __restrict__ slots, const int32_t
   if (lane == 0) *n_tiles = base;
 }
 
-// Opt the kernel in to `bytes` of dynamic shared memory on the current
-// device (raised when a larger shape needs more than the last setting).
-template <typename KernelT>
-cudaError_t allow_smem(KernelT* k, size_t (&granted)[64], size_t bytes) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (granted[dev] >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess) granted[dev] = bytes;
-  return e;
-}
-
 }  // namespace
 
 size_t prefill_tiles_bound(int n_tok, int K, int E, int n_shared) {
@@ -617,8 +663,8 @@ bool prefill_supported(int hidden, int inter) {
 
 namespace {
 
-// A 2D tensor map over `rows` fp16 rows of `cols` values (row-major), box
-// 64 values x kM rows, 128-byte swizzle: the A operand tiles.
+// A 2D tensor map over `rows` int8 rows of `cols` bytes (row-major), box
+// 128 bytes x kM rows, 128-byte swizzle: the A operand tiles.
 cudaError_t make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int cols) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
@@ -630,10 +676,10 @@ cudaError_t make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int co
     encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)kM};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols};
+  const cuuint32_t box[2] = {128, (cuuint32_t)kM};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -644,20 +690,22 @@ cudaError_t make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int co
 cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, const Slot* slots,
                                    const int32_t* n_slots, void* tiles, int32_t* n_tiles, const int32_t* perm,
                                    int K, int n_shared, const int8_t* xq, const float* xd, int n_tok, int hidden,
-                                   int inter, void* xf, void* hf, float* hd, float* y, int32_t* err,
-                                   cudaStream_t st, cudaEvent_t ev_mid) {
+                                   int inter, void* xr, int32_t* xm, void* hr, float* hd, int32_t* hm, float* y,
+                                   int32_t* err, cudaStream_t st, cudaEvent_t ev_mid) {
   Tile* t = reinterpret_cast<Tile*>(tiles);
   const int64_t rows = (int64_t)n_tok * (K + n_shared);
-  const int64_t n8 = rows * hidden / 8;
-  act_rows_f16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(xq, perm, n_tok, K, rows, hidden,
-                                                                    reinterpret_cast<uint4*>(xf));
+  const int64_t n16 = rows * hidden / 16;
+  act_rows_i8_kernel<<<(unsigned)((n16 + 255) / 256), 256, 0, st>>>(xq, perm, n_tok, K, rows, hidden,
+                                                                    reinterpret_cast<uint4*>(xr));
+  const int64_t nblk = (int64_t)n_tok * (hidden / 32);
+  act_magic_kernel<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(xq, nblk, xm);
   build_tiles_kernel<<<1, 32, 0, st>>>(slots, n_slots, t, n_tiles);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap map_x, map_h;
-  if ((e = make_rows_map(&map_x, xf, rows, hidden)) != cudaSuccess) return e;
-  if ((e = make_rows_map(&map_h, hf, rows, inter)) != cudaSuccess) return e;
-  static size_t granted_gu[64] = {}, granted_dn[64] = {};
+  if ((e = make_rows_map(&map_x, xr, rows, hidden)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&map_h, hr, rows, inter)) != cudaSuccess) return e;
+  static uint64_t mask_gu = 0, mask_dn = 0;
   static int sms_cache[64] = {};
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -666,16 +714,16 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
       (e = cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
   const size_t smem = PSmem::bytes();
-  if ((e = allow_smem(prefill_kernel<true, GateUpTable>, granted_gu, smem)) != cudaSuccess) return e;
-  if ((e = allow_smem(prefill_kernel<false, DownTable>, granted_dn, smem)) != cudaSuccess) return e;
+  if ((e = smem_opt_in_once(prefill_kernel<true, GateUpTable>, (int)smem, mask_gu)) != cudaSuccess) return e;
+  if ((e = smem_opt_in_once(prefill_kernel<false, DownTable>, (int)smem, mask_dn)) != cudaSuccess) return e;
   const int grid = sms_cache[dev];
-  __half* hfh = reinterpret_cast<__half*>(hf);
-  prefill_kernel<true, GateUpTable><<<grid, kThreadsP, smem, st>>>(gu, map_x, slots, t, n_tiles, perm, K, xd, hidden,
-                                                                     inter, hfh, hd, y, err);
+  int8_t* hri = reinterpret_cast<int8_t*>(hr);
+  prefill_kernel<true, GateUpTable><<<grid, kThreadsP, smem, st>>>(gu, map_x, slots, t, n_tiles, perm, K, xd, xm,
+                                                                     hidden, inter, hri, hd, hm, y, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecordWithFlags(ev_mid, st, cudaEventRecordExternal)) != cudaSuccess) return e;
-  prefill_kernel<false, DownTable><<<grid, kThreadsP, smem, st>>>(dn, map_h, slots, t, n_tiles, perm, K, hd, hidden,
-                                                                    inter, hfh, hd, y, err);
+  prefill_kernel<false, DownTable><<<grid, kThreadsP, smem, st>>>(dn, map_h, slots, t, n_tiles, perm, K, hd, hm,
+                                                                    hidden, inter, hri, hd, hm, y, err);
   return cudaGetLastError();
 }
 
