@@ -55,6 +55,8 @@ def lib():
             ("ora_pack_int4", None, [vp, i64, vp]),
             ("ora_unpack_int4", None, [vp, i64, vp]),
             ("ora_quantize_rows_int4", None, [vp, i64, i64, vp, vp]),
+            ("ora_quantize_rows_int8", None, [vp, i64, i64, vp, vp]),
+            ("ora_block_isums_int8", None, [vp, vp, i64, vp]),
             ("ora_quantize_act_q8", None, [vp, i64, i64, vp, vp]),
             ("ora_e4m3_to_f32", f32, [C.c_uint8]),
             ("ora_requantize_fp8_int4", None, [vp, vp, i64, i64, i64, vp, vp]),
@@ -89,7 +91,7 @@ def _f32(a) -> np.ndarray:
 
 class _Expert(C.Structure):
     _fields_ = [("gate_q", C.c_void_p), ("gate_s", C.c_void_p), ("up_q", C.c_void_p),
-                ("up_s", C.c_void_p), ("down_q", C.c_void_p), ("down_s", C.c_void_p)]
+                ("up_s", C.c_void_p), ("down_q", C.c_void_p), ("down_s", C.c_void_p), ("bits", C.c_int32)]
 
 
 class _Layer(C.Structure):
@@ -102,17 +104,19 @@ class _Layer(C.Structure):
 
 @dataclass
 class QExpert:
-    """One expert's packed int4 weights (row-major [out x in], in/2 bytes per row)."""
+    """One expert's weights, row-major [out x in]: packed int4 (in/2 bytes
+    per row, bits=4) or int8 (in bytes per row, bits=8), one F32 scale per row."""
     gate_q: np.ndarray
     gate_s: np.ndarray
     up_q: np.ndarray
     up_s: np.ndarray
     down_q: np.ndarray
     down_s: np.ndarray
+    bits: int = 4
 
     def _struct(self) -> _Expert:
         return _Expert(_p(self.gate_q), _p(self.gate_s), _p(self.up_q), _p(self.up_s),
-                       _p(self.down_q), _p(self.down_s))
+                       _p(self.down_q), _p(self.down_s), int(self.bits))
 
 
 # ---------------------------------------------------------------------------
@@ -174,6 +178,24 @@ def quantize_rows_int4(w: np.ndarray):
     s = np.empty(rows, np.float32)
     lib().ora_quantize_rows_int4(_p(w), rows, cols, _p(q), _p(s))
     return q, s
+
+
+def quantize_rows_int8(w: np.ndarray):
+    """Per-row int8 weights: (q int8 [rows x cols], scale F32 [rows])."""
+    w = _f32(w)
+    rows, cols = w.shape
+    q = np.empty((rows, cols), np.int8)
+    s = np.empty(rows, np.float32)
+    lib().ora_quantize_rows_int8(_p(w), rows, cols, _p(q), _p(s))
+    return q, s
+
+
+def block_isums_int8(qrow: np.ndarray, xq: np.ndarray) -> np.ndarray:
+    qrow = np.ascontiguousarray(qrow, np.int8)
+    xq = np.ascontiguousarray(xq, np.int8)
+    out = np.empty(len(xq) // 32, np.int32)
+    lib().ora_block_isums_int8(_p(qrow), _p(xq), len(xq), _p(out))
+    return out
 
 
 def e4m3_to_f32(codes) -> np.ndarray:

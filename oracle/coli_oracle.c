@@ -201,6 +201,27 @@ ORA_API void ora_quantize_rows_int4(const float* w, int64_t rows, int64_t cols, 
     free(q);
 }
 
+/* Per-row int8 weight quantiser, the int8 variant of the expert weights
+ * ([C] "关键特性": quantisation kernels int8 / packed int4 / packed int2).
+ * Reading: the int4 recipe with the int8 range -- scale = absmax/127 (F32
+ * division), q = rint(w/scale) clamped to [-127,127] (round half to even),
+ * one byte per element; an all-zero row gets scale 0 and q = 0. */
+ORA_API void ora_quantize_rows_int8(const float* w, int64_t rows, int64_t cols, int8_t* q_out,
+                                    float* scale_out) {
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* row = w + r * cols;
+        float amax = 0.0f;
+        for (int64_t c = 0; c < cols; ++c) {
+            float a = fabsf(row[c]);
+            if (a > amax) amax = a;
+        }
+        float scale = amax / 127.0f;
+        for (int64_t c = 0; c < cols; ++c)
+            q_out[r * cols + c] = (amax == 0.0f) ? 0 : (int8_t)ora_clampi((int)rintf(row[c] / scale), -127, 127);
+        scale_out[r] = scale;
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* FP8 -> int4 requantiser ([W] "GLM-5.2-colibri-int4的量化流程": the source */
 /* is the FP8 (e4m3) model, dequantised to F32 and then quantised per row as */
@@ -372,6 +393,31 @@ ORA_API void ora_block_isums(const uint8_t* qrow, const int8_t* xq, int64_t dim_
     }
 }
 
+/* The same for an int8 weight row (one signed byte per element). */
+ORA_API void ora_block_isums_int8(const int8_t* qrow, const int8_t* xq, int64_t dim_in, int32_t* isum) {
+    for (int64_t b = 0; b < dim_in / 32; ++b) {
+        int32_t acc = 0;
+        for (int j = 0; j < 32; ++j) acc += (int32_t)qrow[b * 32 + j] * (int32_t)xq[b * 32 + j];
+        isum[b] = acc;
+    }
+}
+
+/* One output of a weight x Q8 matrix-vector product, contract F: the weight
+ * row is packed int4 (bits 4) or int8 (bits 8). */
+static float ora_row_dot_bits(const uint8_t* qrow, int bits, float s_w, const int8_t* xq, const float* xd,
+                              int64_t dim_in) {
+    int64_t nb = dim_in / 32;
+    int32_t* isum = (int32_t*)malloc((size_t)nb * sizeof(int32_t));
+    if (bits == 8)
+        ora_block_isums_int8((const int8_t*)qrow, xq, dim_in, isum);
+    else
+        ora_block_isums(qrow, xq, dim_in, isum);
+    float acc = 0.0f;
+    for (int64_t b = 0; b < nb; ++b) acc = fmaf(xd[b], (float)isum[b], acc);
+    free(isum);
+    return s_w * acc;
+}
+
 /* One output of an int4 x Q8 matrix-vector product, contract F. */
 ORA_API float ora_row_dot(const uint8_t* qrow, float s_w, const int8_t* xq, const float* xd,
                           int64_t dim_in) {
@@ -384,14 +430,16 @@ ORA_API float ora_row_dot(const uint8_t* qrow, float s_w, const int8_t* xq, cons
     return s_w * acc;
 }
 
-/* One expert's packed weights, row-major [out x in] matrices. */
+/* One expert's weights, row-major [out x in] matrices: packed int4 (in/2
+ * bytes per row) when bits is 4 (or 0), int8 (in bytes per row) when 8. */
 typedef struct {
-    const uint8_t* gate_q; /* [inter x hidden/2] */
+    const uint8_t* gate_q; /* [inter x hidden*bits/8] */
     const float* gate_s;   /* [inter] */
-    const uint8_t* up_q;   /* [inter x hidden/2] */
+    const uint8_t* up_q;   /* [inter x hidden*bits/8] */
     const float* up_s;     /* [inter] */
-    const uint8_t* down_q; /* [hidden x inter/2] */
+    const uint8_t* down_q; /* [hidden x inter*bits/8] */
     const float* down_s;   /* [hidden] */
+    int32_t bits;
 } ora_expert;
 
 /* SwiGLU expert on one Q8 token:
@@ -406,15 +454,17 @@ ORA_API void ora_expert_ffn_token(const ora_expert* ex, int64_t hidden, int64_t 
     float* h = (float*)malloc((size_t)inter * sizeof(float));
     int8_t* hq = (int8_t*)malloc((size_t)inter);
     float* hd = (float*)malloc((size_t)(inter / 32) * sizeof(float));
+    const int bits = ex->bits == 8 ? 8 : 4;
+    const int64_t rb_in = hidden * bits / 8, rb_h = inter * bits / 8; /* bytes per weight row */
     for (int64_t o = 0; o < inter; ++o) {
-        float g = ora_row_dot(ex->gate_q + o * (hidden / 2), ex->gate_s[o], xq, xd, hidden);
-        float u = ora_row_dot(ex->up_q + o * (hidden / 2), ex->up_s[o], xq, xd, hidden);
+        float g = ora_row_dot_bits(ex->gate_q + o * rb_in, bits, ex->gate_s[o], xq, xd, hidden);
+        float u = ora_row_dot_bits(ex->up_q + o * rb_in, bits, ex->up_s[o], xq, xd, hidden);
         float sg = ora_sigmoid(g);
         h[o] = (g * sg) * u;
     }
     ora_quantize_act_q8(h, 1, inter, hq, hd);
     for (int64_t o = 0; o < hidden; ++o)
-        y[o] = ora_row_dot(ex->down_q + o * (inter / 2), ex->down_s[o], hq, hd, inter);
+        y[o] = ora_row_dot_bits(ex->down_q + o * rb_h, bits, ex->down_s[o], hq, hd, inter);
     if (hq_out) memcpy(hq_out, hq, (size_t)inter);
     if (hd_out) memcpy(hd_out, hd, (size_t)(inter / 32) * sizeof(float));
     free(h);
