@@ -552,7 +552,8 @@ cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
   static int sms[64] = {};
   const size_t smem = stream_smem_bytes<TT>(a.g);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
-  cudaError_t e = smem_opt_in_once(expert_stream_kernel<TT>, (int)smem, attr_mask);
+  // the opt-in is set once per device, so to the largest size any shape needs
+  cudaError_t e = smem_opt_in_once(expert_stream_kernel<TT>, 227 * 1024, attr_mask);
   if (e != cudaSuccess) return e;
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;

@@ -36,7 +36,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // Set a kernel's dynamic shared-memory opt-in once per device (the
 // attribute belongs to the device's context); `mask` is the caller's
-// per-kernel record of the devices done (devices 0..63).
+// per-kernel record of the devices done (devices 0..63).  Pass the largest
+// size the kernel is ever launched with: later calls do not raise it.
 template <typename KernelT>
 cudaError_t smem_opt_in_once(KernelT* kernel, int bytes, uint64_t& mask) {
   int dev = 0;
