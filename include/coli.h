@@ -63,8 +63,12 @@ typedef enum {
 /* Layer shape and routing options ([W] "GLM-5.2的MoE实现": hidden 6144,
  * expert inter 2048, 256 routed experts, 1 shared, 8 per token;
  * [W] "路由策略定制": routed_scaling_factor, norm_topk_prob).
+ * weight_bits: 4 (packed int4, also when 0) or 8 (int8 expert weights, the
+ * pages' int8 kernel variant, [C] "关键特性"; same per-row F32 scale).
  * Limits: hidden % 128 == 0; inter % 32 == 0; shared_inter % 32 == 0;
- * 1 <= top_k <= min(n_experts, 16); n_experts <= 512; 0 <= n_shared <= 4. */
+ * 1 <= top_k <= min(n_experts, 16); n_experts <= 512; 0 <= n_shared <= 4.
+ * int8 weights need inter % 128 == 0 (they run on the streaming kernel of
+ * a prepared layer for <= 4 tokens, else on the tensor-core kernels). */
 typedef struct {
     int32_t hidden;
     int32_t inter;
@@ -74,15 +78,17 @@ typedef struct {
     int32_t shared_inter;
     int32_t norm_topk_prob;      /* nonzero: renormalise the selected scores */
     float routed_scaling_factor; /* multiplies every routed weight */
+    int32_t weight_bits;         /* 4 (or 0) or 8 */
 } coli_moe_config;
 
-/* One expert's packed weights (device pointers). */
+/* One expert's weights (device pointers): packed int4 rows of in/2 bytes
+ * (weight_bits 4) or int8 rows of `in` bytes (weight_bits 8). */
 typedef struct {
-    const uint8_t* gate_q; /* [inter x hidden/2] */
+    const uint8_t* gate_q; /* [inter x hidden*bits/8] */
     const float* gate_s;   /* [inter] */
-    const uint8_t* up_q;   /* [inter x hidden/2] */
+    const uint8_t* up_q;   /* [inter x hidden*bits/8] */
     const float* up_s;     /* [inter] */
-    const uint8_t* down_q; /* [hidden x inter/2] */
+    const uint8_t* down_q; /* [hidden x inter*bits/8] */
     const float* down_s;   /* [hidden] */
 } coli_expert;
 
@@ -108,6 +114,15 @@ typedef struct {
  * bytes; scale_out: [rows] F32.  cols must be a positive multiple of 32. */
 coli_status coli_quantize_rows_int4(const float* w, int64_t rows, int64_t cols, uint8_t* q_out,
                                     float* scale_out, void* stream);
+
+/* Per-row int8 weight quantiser, the int8 variant of the expert weights
+ * ([C] "关键特性": quantisation kernels int8 / packed int4 / packed int2;
+ * the int4 recipe of [W] "GLM-5.2-colibri-int4的量化流程" with the int8
+ * range): scale = absmax/127; q = rint(w/scale) clamped to [-127,127] (half
+ * to even); an all-zero row gets scale 0.  w: [rows x cols] F32; q_out:
+ * [rows x cols] int8; scale_out: [rows] F32.  cols a positive multiple of 32. */
+coli_status coli_quantize_rows_int8(const float* w, int64_t rows, int64_t cols, int8_t* q_out, float* scale_out,
+                                    void* stream);
 
 /* FP8 -> int4 requantiser, the offline converter's step on the GPU
  * ([W] "GLM-5.2-colibri-int4的量化流程": the source model is FP8 e4m3,
@@ -156,7 +171,8 @@ coli_status coli_moe_bucket(const int32_t* topk_idx, int64_t n_tok, int32_t top_
  * h re-quantised to Q8_0, y = down.h.  xq [n_tok x hidden] int8,
  * xs [n_tok x hidden/32] F32, y_out [n_tok x hidden] F32.  `expert` points
  * to ONE host-side coli_expert.  Workspace: coli_moe_workspace_bytes(cfg,
- * n_tok) bytes is always enough.  This is the reference-shape entry point:
+ * n_tok) bytes is always enough.  int4 weights only (weight_bits 4).  This
+ * is the reference-shape entry point:
  * it runs the general expert kernels (one CTA per 32 outputs), which follow
  * the same contracts and give the same bits as the layer forward's streaming
  * and tensor-core kernels, but it is not the tuned path and carries no
@@ -213,7 +229,7 @@ size_t coli_moe_workspace_bytes(const coli_moe_config* cfg, int64_t max_tokens);
 /* Message for the last non-OK status returned on the calling thread. */
 const char* coli_last_error(void);
 
-/* Test hook: the per-32-block int32 partial sums of one expert matrix
+/* Test hook (packed int4 weights): the per-32-block int32 partial sums of one expert matrix
  * (which: 0 gate, 1 up, 2 down) against n_tok Q8 vectors, computed by the
  * same device routine as the expert kernels:
  * isum_out[t, r, b] = sum_{j<32} q_w[r, 32b+j] * xq[t, 32b+j],

@@ -25,7 +25,7 @@ EXPORTS = [
     "coli_moe_expert_ffn", "coli_moe_layer_forward", "coli_moe_stack_forward", "coli_rmsnorm",
     "coli_moe_workspace_bytes", "coli_last_error", "coli_debug_block_partials",
     "coli_debug_phase_events", "coli_moe_layer_forward_noalloc", "coli_sync_status", "coli_debug_wait_probe",
-    "coli_requantize_fp8_int4", "coli_moe_prepared_bytes", "coli_moe_prepare",
+    "coli_requantize_fp8_int4", "coli_moe_prepared_bytes", "coli_moe_prepare", "coli_quantize_rows_int8",
 ]
 
 
@@ -38,7 +38,7 @@ class ColiError(RuntimeError):
 class MoeConfig(C.Structure):
     _fields_ = [("hidden", C.c_int32), ("inter", C.c_int32), ("n_experts", C.c_int32),
                 ("top_k", C.c_int32), ("n_shared", C.c_int32), ("shared_inter", C.c_int32),
-                ("norm_topk_prob", C.c_int32), ("routed_scaling_factor", C.c_float)]
+                ("norm_topk_prob", C.c_int32), ("routed_scaling_factor", C.c_float), ("weight_bits", C.c_int32)]
 
 
 class Expert(C.Structure):
@@ -85,6 +85,7 @@ def load(path: str | None = None):
         "coli_debug_wait_probe": (st, [vp, i64, vp]),
         "coli_requantize_fp8_int4": (st, [vp, vp, i64, i64, i32, vp, vp, vp]),
         "coli_moe_prepared_bytes": (C.c_size_t, [C.POINTER(MoeConfig)]),
+        "coli_quantize_rows_int8": (st, [vp, i64, i64, vp, vp, vp]),
         "coli_moe_prepare": (st, [C.POINTER(MoeLayerC), vp, C.c_size_t, vp]),
     }
     for name, (res, args) in sig.items():
@@ -119,15 +120,16 @@ def _ptr(t):
 
 
 def make_config(hidden, inter, n_experts, top_k, n_shared=1, shared_inter=None, norm_topk_prob=True,
-                routed_scaling_factor=2.5) -> MoeConfig:
+                routed_scaling_factor=2.5, weight_bits=4) -> MoeConfig:
     return MoeConfig(hidden, inter, n_experts, top_k, n_shared,
                      inter if shared_inter is None else shared_inter, int(bool(norm_topk_prob)),
-                     float(routed_scaling_factor))
+                     float(routed_scaling_factor), int(weight_bits))
 
 
 @dataclass
 class QExpert:
-    """Packed int4 weights of one expert (torch CUDA tensors, row-major [out x in])."""
+    """One expert's weights (torch CUDA tensors, row-major [out x in]): packed
+    int4 rows of in/2 bytes, or int8 rows of `in` bytes (weight_bits 8)."""
     gate_q: object
     gate_s: object
     up_q: object
@@ -171,6 +173,16 @@ def quantize_rows_int4(w, q_out=None, s_out=None, stream=None):
     q = torch.empty(rows, cols // 2, dtype=torch.uint8, device=w.device) if q_out is None else q_out
     s = torch.empty(rows, dtype=torch.float32, device=w.device) if s_out is None else s_out
     _check(lib().coli_quantize_rows_int4(_ptr(w), rows, cols, _ptr(q), _ptr(s), _stream(stream)))
+    return q, s
+
+
+def quantize_rows_int8(w, q_out=None, s_out=None, stream=None):
+    """Per-row int8 weights: (q int8 [rows x cols], scale F32 [rows])."""
+    import torch
+    rows, cols = w.shape
+    q = torch.empty(rows, cols, dtype=torch.int8, device=w.device) if q_out is None else q_out
+    s = torch.empty(rows, dtype=torch.float32, device=w.device) if s_out is None else s_out
+    _check(lib().coli_quantize_rows_int8(_ptr(w), rows, cols, _ptr(q), _ptr(s), _stream(stream)))
     return q, s
 
 

@@ -60,8 +60,14 @@ coli_status check_cfg(const coli_moe_config* c, const char* fn) {
     return fail(COLI_EINVAL, "%s: n_shared=%d outside [0, %d]", fn, c->n_shared, kMaxShared);
   if (c->n_shared > 0 && c->shared_inter != c->inter)
     return fail(COLI_EINVAL, "%s: shared_inter=%d must equal inter=%d", fn, c->shared_inter, c->inter);
+  if (c->weight_bits != 0 && c->weight_bits != 4 && c->weight_bits != 8)
+    return fail(COLI_EINVAL, "%s: weight_bits=%d (4 or 8)", fn, c->weight_bits);
+  if (c->weight_bits == 8 && !prefill_supported(c->hidden, c->inter))
+    return fail(COLI_EINVAL, "%s: int8 weights need hidden and inter multiples of 128", fn);
   return COLI_OK;
 }
+
+int bits_of(const coli_moe_config& c) { return c.weight_bits == 8 ? 8 : 4; }
 
 coli_status check_expert(const coli_expert* e, const char* fn) {
   if (e == nullptr) return fail(COLI_EINVAL, "%s: null expert", fn);
@@ -123,8 +129,10 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   L.inv = take(T * K * 4);
   L.slots = take((size_t)kMaxSlots * sizeof(Slot));
   L.n_slots = take(4);
-  // the tensor-core prefill path's buffers only when a call of T tokens takes that path
-  const bool tc = (T > kDecodeMaxTok || !decode_supported((int)H, (int)I)) && prefill_supported((int)H, (int)I);
+  // the tensor-core prefill path's buffers only when a call of T tokens can take that path
+  // (int8 weights: whenever the layer is not prepared or T > kStreamMaxTok)
+  const bool tc = (T > kDecodeMaxTok || !decode_supported((int)H, (int)I) || bits_of(c) == 8) &&
+                  prefill_supported((int)H, (int)I);
   L.tiles = take(tc ? prefill_tile_bytes((int)T, (int)K, (int)E, (int)S) : 0);
   L.n_tiles = take(4);
   L.hq = take(rows * I);  // h as int8 rows (Q8 of h; the tensor-core path's down operand)
@@ -195,7 +203,8 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   };
 
   int32_t* status = at<int32_t>(ws, W.status);
-  if (L->prepared != nullptr && stream_supported(H, I, (int)T, S, K)) {
+  const int bits = bits_of(c);
+  if (L->prepared != nullptr && stream_supported(H, I, bits, (int)T)) {
     // decode on the streaming copy: 2 kernels, the second launched with PDL
     int32_t* ctr = at<int32_t>(ws, W.ctr);
     CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, xq, xd, clear_status ? status : nullptr,
@@ -203,7 +212,7 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
     CHECK_LAUNCH(mark(0));
     StreamArgs a{};
     a.prep = static_cast<const unsigned char*>(L->prepared);
-    a.g = stream_geom(H, I);
+    a.g = stream_geom(H, I, bits);
     a.E = E;
     a.K = K;
     a.S = S;
@@ -226,7 +235,7 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
     CHECK_LAUNCH(mark(2));
     return COLI_OK;
   }
-  if (T <= kDecodeMaxTok && decode_supported(H, I)) {
+  if (bits == 4 && T <= kDecodeMaxTok && decode_supported(H, I)) {
     // decode: 5 kernels, the last four launched with PDL
     CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, xq, xd, clear_status ? status : nullptr,
                                       nullptr, 0, st));
@@ -257,8 +266,9 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   CHECK_LAUNCH(mark(0));
   if (prefill_supported(H, I)) {
     CHECK_LAUNCH(launch_prefill_experts(gu, dn, slots, n_slots, at<void>(ws, W.tiles), at<int32_t>(ws, W.n_tiles),
-                                        perm, K, S, xq, xd, (int)T, H, I, at<void>(ws, W.xr), at<int32_t>(ws, W.xm), hq,
-                                        hd, at<int32_t>(ws, W.hm), y, at<int32_t>(ws, W.status), st, ev[1]));
+                                        perm, K, S, bits, xq, xd, (int)T, H, I, at<void>(ws, W.xr),
+                                        at<int32_t>(ws, W.xm), hq, hd, at<int32_t>(ws, W.hm), y,
+                                        at<int32_t>(ws, W.status), st, ev[1]));
   } else {
     CHECK_LAUNCH(launch_gateup(gu, sl, xq, xd, H, I, max_tok, hq, hd, st));
     CHECK_LAUNCH(mark(1));
@@ -293,8 +303,8 @@ COLI_EXPORT size_t coli_moe_workspace_bytes(const coli_moe_config* cfg, int64_t 
 
 COLI_EXPORT size_t coli_moe_prepared_bytes(const coli_moe_config* cfg) {
   if (check_cfg(cfg, "coli_moe_prepared_bytes") != COLI_OK) return 0;
-  if (!stream_shape_ok(cfg->hidden, cfg->inter)) return 0;
-  return (size_t)(cfg->n_experts + cfg->n_shared) * stream_expert_bytes(cfg->hidden, cfg->inter);
+  if (!stream_shape_ok(cfg->hidden, cfg->inter, bits_of(*cfg))) return 0;
+  return (size_t)(cfg->n_experts + cfg->n_shared) * stream_expert_bytes(cfg->hidden, cfg->inter, bits_of(*cfg));
 }
 
 COLI_EXPORT coli_status coli_moe_prepare(const coli_moe_layer* layer, void* prepared, size_t bytes, void* stream) {
@@ -304,18 +314,19 @@ COLI_EXPORT coli_status coli_moe_prepare(const coli_moe_layer* layer, void* prep
   const coli_moe_config& c = layer->cfg;
   const size_t need = coli_moe_prepared_bytes(&c);
   if (need == 0)
-    return fail(COLI_EINVAL, "%s: hidden=%d inter=%d has no streaming layout (both multiples of 128; hidden/32 a "
-                "multiple of 16 or 4, 8; inter/32 a multiple of 32 or 4, 8, 16)", fn, c.hidden, c.inter);
+    return fail(COLI_EINVAL, "%s: hidden=%d inter=%d has no streaming layout (both multiples of 128; int4: hidden/32 "
+                "a multiple of 16 or 4, 8; inter/32 a multiple of 32 or 4, 8, 16; int8: hidden/32 a multiple of 8 or "
+                "4; inter/32 a multiple of 16 or 4, 8)", fn, c.hidden, c.inter);
   if (prepared == nullptr) return fail(COLI_EINVAL, "%s: null pointer 'prepared'", fn);
   if ((reinterpret_cast<uintptr_t>(prepared) & 255u) != 0)
     return fail(COLI_EINVAL, "%s: 'prepared' is not 256-byte aligned", fn);
   if (bytes < need) return fail(COLI_ENOMEM, "%s: %zu bytes < %zu needed", fn, bytes, need);
-  const uint64_t eb = stream_expert_bytes(c.hidden, c.inter);
+  const uint64_t eb = stream_expert_bytes(c.hidden, c.inter, bits_of(c));
   cudaStream_t st = (cudaStream_t)stream;
   for (int j = 0; j < c.n_experts + c.n_shared; ++j) {
     const coli_expert& e = j < c.n_experts ? layer->experts[j] : layer->shared[j - c.n_experts];
-    CHECK_LAUNCH(launch_prepare_expert(c.hidden, c.inter, e.gate_q, e.gate_s, e.up_q, e.up_s, e.down_q, e.down_s,
-                                       static_cast<unsigned char*>(prepared) + (size_t)j * eb, st));
+    CHECK_LAUNCH(launch_prepare_expert(c.hidden, c.inter, bits_of(c), e.gate_q, e.gate_s, e.up_q, e.up_s, e.down_q,
+                                       e.down_s, static_cast<unsigned char*>(prepared) + (size_t)j * eb, st));
   }
   return COLI_OK;
 }
@@ -395,6 +406,20 @@ COLI_EXPORT coli_status coli_quantize_rows_int4(const float* w, int64_t rows, in
   CHECK_PTR(q_out);
   CHECK_PTR(scale_out);
   CHECK_LAUNCH(launch_quantize_rows_int4(w, rows, cols, q_out, scale_out, (cudaStream_t)stream));
+  return COLI_OK;
+}
+
+COLI_EXPORT coli_status coli_quantize_rows_int8(const float* w, int64_t rows, int64_t cols, int8_t* q_out,
+                                                float* scale_out, void* stream) {
+  const char* fn = "coli_quantize_rows_int8";
+  if (rows < 0 || cols <= 0 || cols % 32 != 0)
+    return fail(COLI_EINVAL, "%s: rows=%lld cols=%lld (cols must be a positive multiple of 32)", fn,
+                (long long)rows, (long long)cols);
+  if (rows == 0) return COLI_OK;
+  CHECK_PTR(w);
+  CHECK_PTR(q_out);
+  CHECK_PTR(scale_out);
+  CHECK_LAUNCH(launch_quantize_rows_int8(w, rows, cols, q_out, scale_out, (cudaStream_t)stream));
   return COLI_OK;
 }
 
@@ -482,6 +507,7 @@ COLI_EXPORT coli_status coli_moe_expert_ffn(const coli_moe_config* cfg, const co
   const char* fn = "coli_moe_expert_ffn";
   coli_status s = check_cfg(cfg, fn);
   if (s != COLI_OK) return s;
+  if (bits_of(*cfg) != 4) return fail(COLI_EINVAL, "%s: int4 weights only (weight_bits 4)", fn);
   if (n_tok < 0 || n_tok > (1 << 24)) return fail(COLI_EINVAL, "%s: n_tok=%lld", fn, (long long)n_tok);
   if (n_tok == 0) return COLI_OK;
   if ((s = check_expert(expert, fn)) != COLI_OK) return s;

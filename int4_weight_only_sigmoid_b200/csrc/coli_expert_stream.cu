@@ -21,8 +21,10 @@
 // (192 KB at GLM-5.2 shapes) are one contiguous range of HBM.
 //
 // Arithmetic (contract F, bit-identical to the oracle).  Lane l holds one
-// weight row (gate/up: gate row l and up row l of the unit); per 16-byte
-// packed block and staged token: (w & 0x0F0F0F0F) ^ 0x08080808 is q + 8 of
+// weight row (gate/up: gate row l and up row l of the unit); int8 weights
+// (stored as even / odd element planes) take 8 dp4a per block and staged
+// token against the token's planes; per 16-byte packed int4 block and
+// staged token: (w & 0x0F0F0F0F) ^ 0x08080808 is q + 8 of
 // the even elements (unsigned bytes) and w & 0xF0F0F0F0 is 16 q of the odd
 // ones (signed bytes); with the token's even / odd byte planes xe, xo and
 // c16 = -128 * sum(xe):
@@ -118,21 +120,54 @@ __device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
   return v;
 }
 
+// isum of one int8 weight block (even / odd element planes we, wo) against
+// one token's block (planes xe, xo).
+__device__ __forceinline__ int blk_isum8(const uint4& we, const uint4& wo, const uint4& xe, const uint4& xo) {
+  int A = __dp4a((int)we.x, (int)xe.x, 0);
+  int B = __dp4a((int)wo.x, (int)xo.x, 0);
+  A = __dp4a((int)we.y, (int)xe.y, A);
+  B = __dp4a((int)wo.y, (int)xo.y, B);
+  A = __dp4a((int)we.z, (int)xe.z, A);
+  B = __dp4a((int)wo.z, (int)xo.z, B);
+  A = __dp4a((int)we.w, (int)xe.w, A);
+  B = __dp4a((int)wo.w, (int)xo.w, B);
+  return A + B;
+}
+
+// One weight block of a stage row: the two operand halves for blk_isum
+// (int4: q + 8 of the even elements, 16 q of the odd ones) or blk_isum8.
+template <int BITS>
+__device__ __forceinline__ void load_blk(const uint4* row, int j, int sw, uint4& a, uint4& b) {
+  if constexpr (BITS == 4) {
+    unpack_blk(row[j ^ sw], a, b);
+  } else {
+    a = row[(2 * j) ^ sw];
+    b = row[(2 * j + 1) ^ sw];
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ int isum_of(const uint4& a, const uint4& b, const uint4& xe, const uint4& xo, int c16) {
+  if constexpr (BITS == 4) return blk_isum(a, b, xe, xo, c16);
+  return blk_isum8(a, b, xe, xo);
+}
+
 // One gate/up stage: blocks b0 .. b0+G-1 of gate row l and up row l (lane
 // l) against the slot's staged tokens.
-template <int TT>
+template <int TT, int BITS>
 __device__ __forceinline__ void gu_stage(const unsigned char* st, int G, int swz, int b0, int nb, int nv,
                                          const int (&tok)[TT], const uint4* xpl, const float2* xdc, float (&ag)[TT],
                                          float (&au)[TT]) {
   const int lane = threadIdx.x & 31;
-  const uint4* rg = reinterpret_cast<const uint4*>(st) + lane * G;
-  const uint4* ru = reinterpret_cast<const uint4*>(st) + (32 + lane) * G;
+  constexpr int cpb = BITS / 4;  // 16-byte chunks per block
+  const uint4* rg = reinterpret_cast<const uint4*>(st) + lane * G * cpb;
+  const uint4* ru = reinterpret_cast<const uint4*>(st) + (32 + lane) * G * cpb;
   const int sw = lane & swz;
 #pragma unroll 4
   for (int j = 0; j < G; ++j) {
     uint4 ge, go, ue, uo;
-    unpack_blk(rg[j ^ sw], ge, go);
-    unpack_blk(ru[j ^ sw], ue, uo);
+    load_blk<BITS>(rg, j, sw, ge, go);
+    load_blk<BITS>(ru, j, sw, ue, uo);
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
       if (t < nv) {
@@ -140,8 +175,8 @@ __device__ __forceinline__ void gu_stage(const unsigned char* st, int G, int swz
         const uint4 xe = xpl[2 * xi], xo = xpl[2 * xi + 1];
         const float2 dc = xdc[xi];
         const int c16 = __float_as_int(dc.y);
-        ag[t] = __fmaf_rn(dc.x, __int2float_rn(blk_isum(ge, go, xe, xo, c16)), ag[t]);
-        au[t] = __fmaf_rn(dc.x, __int2float_rn(blk_isum(ue, uo, xe, xo, c16)), au[t]);
+        ag[t] = __fmaf_rn(dc.x, __int2float_rn(isum_of<BITS>(ge, go, xe, xo, c16)), ag[t]);
+        au[t] = __fmaf_rn(dc.x, __int2float_rn(isum_of<BITS>(ue, uo, xe, xo, c16)), au[t]);
       }
     }
   }
@@ -149,29 +184,30 @@ __device__ __forceinline__ void gu_stage(const unsigned char* st, int G, int swz
 
 // One down stage: blocks b0 .. b0+G-1 of down row l (lane l) against the
 // slot's staged h rows (token t of the slot at index t).
-template <int TT>
+template <int TT, int BITS>
 __device__ __forceinline__ void dn_stage(const unsigned char* st, int G, int swz, int b0, int nb, int nv,
                                          const uint4* hpl, const float2* hdc, float (&ay)[TT]) {
   const int lane = threadIdx.x & 31;
-  const uint4* rw = reinterpret_cast<const uint4*>(st) + lane * G;
+  constexpr int cpb = BITS / 4;
+  const uint4* rw = reinterpret_cast<const uint4*>(st) + lane * G * cpb;
   const int sw = lane & swz;
 #pragma unroll 4
   for (int j = 0; j < G; ++j) {
     uint4 we, wo;
-    unpack_blk(rw[j ^ sw], we, wo);
+    load_blk<BITS>(rw, j, sw, we, wo);
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
       if (t < nv) {
         const int hi = t * nb + b0 + j;
         const uint4 xe = hpl[2 * hi], xo = hpl[2 * hi + 1];
         const float2 dc = hdc[hi];
-        ay[t] = __fmaf_rn(dc.x, __int2float_rn(blk_isum(we, wo, xe, xo, __float_as_int(dc.y))), ay[t]);
+        ay[t] = __fmaf_rn(dc.x, __int2float_rn(isum_of<BITS>(we, wo, xe, xo, __float_as_int(dc.y))), ay[t]);
       }
     }
   }
 }
 
-template <int TT>
+template <int TT, int BITS>
 __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid_constant__ StreamArgs a) {
   constexpr int R = StreamRing<TT>::R;
   extern __shared__ unsigned char smem_raw[];
@@ -392,8 +428,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     for (int t = 0; t < TT; ++t) ag[t] = au[t] = 0.0f;
     for (int s = 0; s < g.st_gu; ++s) {
       if (!(ok = wait_stage())) break;
-      gu_stage<TT>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_gu, g.swz_gu, s * g.g_gu, g.nbh, nv, tok,
-                   xpl, xdc, ag, au);
+      gu_stage<TT, BITS>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_gu, g.swz_gu, s * g.g_gu, g.nbh, nv,
+                         tok, xpl, xdc, ag, au);
       next_stage();
     }
     if (!ok) break;
@@ -476,8 +512,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     for (int t = 0; t < TT; ++t) ay[t] = 0.0f;
     for (int s = 0; s < g.st_dn; ++s) {
       if (!(ok = wait_stage())) break;
-      dn_stage<TT>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_dn, g.swz_dn, s * g.g_dn, g.nbi, nv, hpl,
-                   hdc, ay);
+      dn_stage<TT, BITS>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_dn, g.swz_dn, s * g.g_dn, g.nbi, nv,
+                         hpl, hdc, ay);
       next_stage();
     }
     if (!ok) break;
@@ -513,7 +549,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   // an owner that gave up before arriving leaves hbar incomplete: waiters give up too (bounded)
 }
 
-// Streaming copy of one expert: one thread per packed 16-byte block, then
+// Streaming copy of one expert: one thread per weight block (16 bytes of
+// int4, or 32 bytes of int8 split into its even / odd element planes), then
 // the scales.
 __global__ void prepare_expert_kernel(StreamGeom g, const uint8_t* __restrict__ gq, const uint8_t* __restrict__ uq,
                                       const uint8_t* __restrict__ dq, const float* __restrict__ gs,
@@ -530,15 +567,27 @@ __global__ void prepare_expert_kernel(StreamGeom g, const uint8_t* __restrict__ 
       const int64_t j = i - m * n_gu;
       r = (int)(j / g.nbh);
       b = (int)(j - (int64_t)r * g.nbh);
-      src = (m == 0 ? gq : uq) + (int64_t)r * (g.H / 2) + 16 * b;
+      src = (m == 0 ? gq : uq) + (int64_t)r * (g.H / 32) * g.bpb + (int64_t)g.bpb * b;
     } else {
       m = 2;
       const int64_t j = i - 2 * n_gu;
       r = (int)(j / g.nbi);
       b = (int)(j - (int64_t)r * g.nbi);
-      src = dq + (int64_t)r * (g.I / 2) + 16 * b;
+      src = dq + (int64_t)r * (g.I / 32) * g.bpb + (int64_t)g.bpb * b;
     }
-    *reinterpret_cast<uint4*>(dst + stream_block_offset(g, m, r, b)) = *reinterpret_cast<const uint4*>(src);
+    const uint4 w0 = *reinterpret_cast<const uint4*>(src);
+    if (g.bits == 4) {
+      *reinterpret_cast<uint4*>(dst + stream_chunk_offset(g, m, r, b, 0)) = w0;
+    } else {
+      const uint4 w1 = *reinterpret_cast<const uint4*>(src + 16);
+      uint4 e, o;
+      split_even_odd(w0.x, w0.y, e.x, o.x);
+      split_even_odd(w0.z, w0.w, e.y, o.y);
+      split_even_odd(w1.x, w1.y, e.z, o.z);
+      split_even_odd(w1.z, w1.w, e.w, o.w);
+      *reinterpret_cast<uint4*>(dst + stream_chunk_offset(g, m, r, b, 0)) = e;
+      *reinterpret_cast<uint4*>(dst + stream_chunk_offset(g, m, r, b, 1)) = o;
+    }
   }
   float* sc = reinterpret_cast<float*>(dst + g.sc_off);
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < 2 * g.I + g.H;
@@ -546,14 +595,14 @@ __global__ void prepare_expert_kernel(StreamGeom g, const uint8_t* __restrict__ 
     sc[i] = i < g.I ? gs[i] : (i < 2 * g.I ? us[i - g.I] : ds[i - 2 * g.I]);
 }
 
-template <int TT>
+template <int TT, int BITS>
 cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
   static uint64_t attr_mask = 0;
   static int sms[64] = {};
   const size_t smem = stream_smem_bytes<TT>(a.g);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   // the opt-in is set once per device, so to the largest size any shape needs
-  cudaError_t e = smem_opt_in_once(expert_stream_kernel<TT>, 227 * 1024, attr_mask);
+  cudaError_t e = smem_opt_in_once(expert_stream_kernel<TT, BITS>, 227 * 1024, attr_mask);
   if (e != cudaSuccess) return e;
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -563,32 +612,37 @@ cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
   // units of other CTAs); at least as many CTAs as slots, so that a CTA's
   // range of down units spans at most two slots
   if (sms[dev] < kMaxSlotsS) return cudaErrorInvalidConfiguration;
-  return launch_pdl(expert_stream_kernel<TT>, dim3(sms[dev]), dim3(kSW * 32), smem, st, true, a);
+  return launch_pdl(expert_stream_kernel<TT, BITS>, dim3(sms[dev]), dim3(kSW * 32), smem, st, true, a);
 }
 
 }  // namespace
 
-bool stream_supported(int hidden, int inter, int n_tok, int n_shared, int top_k) {
-  if (n_tok < 1 || n_tok > kStreamMaxTok || !stream_shape_ok(hidden, inter)) return false;
-  const StreamGeom g = stream_geom(hidden, inter);
-  (void)n_shared;
-  (void)top_k;
-  return stream_smem_bytes<4>(g) <= 227 * 1024 && stream_smem_bytes<1>(g) <= 227 * 1024;
+bool stream_supported(int hidden, int inter, int bits, int n_tok) {
+  if (n_tok < 1 || n_tok > kStreamMaxTok || !stream_shape_ok(hidden, inter, bits)) return false;
+  const StreamGeom g = stream_geom(hidden, inter, bits);
+  return stream_smem_bytes<4>(g) <= 227 * 1024 && stream_smem_bytes<1>(g) <= 227 * 1024 &&
+         stream_smem_bytes<2>(g) <= 227 * 1024;
 }
 
-uint64_t stream_expert_bytes(int hidden, int inter) { return stream_geom(hidden, inter).expert_bytes; }
+uint64_t stream_expert_bytes(int hidden, int inter, int bits) { return stream_geom(hidden, inter, bits).expert_bytes; }
 
-cudaError_t launch_prepare_expert(int hidden, int inter, const uint8_t* gq, const float* gs, const uint8_t* uq,
-                                  const float* us, const uint8_t* dq, const float* ds, void* dst, cudaStream_t st) {
-  const StreamGeom g = stream_geom(hidden, inter);
+cudaError_t launch_prepare_expert(int hidden, int inter, int bits, const uint8_t* gq, const float* gs,
+                                  const uint8_t* uq, const float* us, const uint8_t* dq, const float* ds, void* dst,
+                                  cudaStream_t st) {
+  const StreamGeom g = stream_geom(hidden, inter, bits);
   prepare_expert_kernel<<<592, 256, 0, st>>>(g, gq, uq, dq, gs, us, ds, static_cast<unsigned char*>(dst));
   return cudaGetLastError();
 }
 
 cudaError_t launch_expert_stream(const StreamArgs& a, cudaStream_t st) {
-  if (a.T <= 1) return stream_tt<1>(a, st);
-  if (a.T <= 2) return stream_tt<2>(a, st);
-  return stream_tt<4>(a, st);
+  if (a.g.bits == 8) {
+    if (a.T <= 1) return stream_tt<1, 8>(a, st);
+    if (a.T <= 2) return stream_tt<2, 8>(a, st);
+    return stream_tt<4, 8>(a, st);
+  }
+  if (a.T <= 1) return stream_tt<1, 4>(a, st);
+  if (a.T <= 2) return stream_tt<2, 4>(a, st);
+  return stream_tt<4, 4>(a, st);
 }
 
 }  // namespace coli

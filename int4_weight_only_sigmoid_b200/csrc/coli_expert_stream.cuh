@@ -1,23 +1,27 @@
 // coli_expert_stream.cuh -- the streaming layout of a layer's expert weights
-// (host and device): where every packed 16-byte Q8 block of every expert
-// row sits in the private copy that coli_moe_prepare writes and the
-// streaming decode kernel reads.
+// (host and device): where every Q8 block of every expert row sits in the
+// private copy that coli_moe_prepare writes and the streaming decode kernel
+// reads.
 //
 // The copy is made of "stages": the exact shared-memory image of one step
 // of a warp's work, so that one bulk copy moves a stage from HBM to shared
-// memory with no gather.
+// memory with no gather.  A weight block (32 weights) is 16 bytes of packed
+// int4 or 32 bytes of int8; an int8 block is stored as its even elements
+// (16 bytes: 0, 2, .., 30) then its odd elements, so both widths meet the
+// activations as even / odd byte planes.  The 16-byte chunks of a stage row
+// are XOR-rotated: chunk c of stage row r sits in slot c ^ (r & swz) (rows
+// on lanes: lane l reads row l, and the XOR spreads the 8 lanes of each
+// shared-memory phase over 8 bank groups).
 //  - gate/up unit u of an expert (intermediate outputs 32u .. 32u+31):
-//    stages s = 0 .. nbh/G - 1 of 64 stage rows x G blocks; stage row
-//    r < 32 is gate row 32u + r, r >= 32 is up row 32u + r - 32; block j of
-//    stage s is Q8 block sG + j of the row, stored in 16-byte slot
-//    j ^ (r & swz) of the stage row (rows on lanes: lane l reads row l, and
-//    the XOR spreads the 8 lanes of each shared-memory phase over 8 bank
-//    groups).  G = min(16, nbh).
+//    stages of 64 stage rows x G blocks; stage row r < 32 is gate row
+//    32u + r, r >= 32 is up row 32u + r - 32; block j of stage s is Q8 block
+//    sG + j of the row.  G = min(16, nbh) for int4, min(8, nbh) for int8.
 //  - down unit v (output rows 32v .. 32v+31): stages of 32 rows x G blocks,
-//    G = min(32, nbi), the same slot rule.
+//    G = min(32, nbi) for int4, min(16, nbi) for int8.
 //  - then the F32 row scales: gate [I], up [I], down [H].
 // Per expert: gate/up units | down units | scales, each expert padded to
 // 256 bytes; expert j (routed 0..E-1, then shared) at j * expert_bytes.
+// Every stage is 16 KB at GLM-5.2 shapes.
 #pragma once
 
 #include <cstddef>
@@ -29,6 +33,8 @@ constexpr int kStreamStageMax = 16 * 1024;  // bytes of the largest stage (and o
 
 struct StreamGeom {
   int H, I;          // hidden, expert inter
+  int bits;          // 4 (packed int4) or 8 (int8)
+  int bpb;           // bytes per weight block: 16 or 32
   int nbh, nbi;      // Q8 blocks per gate/up row (H/32) and per down row (I/32)
   int g_gu, g_dn;    // blocks per stage row
   int swz_gu, swz_dn;
@@ -39,30 +45,40 @@ struct StreamGeom {
   uint64_t dn_off, sc_off, expert_bytes;
 };
 
-__host__ __device__ inline bool stream_shape_ok(int H, int I) {
-  if (H <= 0 || I <= 0 || H % 128 != 0 || I % 128 != 0) return false;
-  const int nbh = H / 32, nbi = I / 32;
-  const bool gu = nbh % 16 == 0 || nbh == 4 || nbh == 8;
-  const bool dn = nbi % 32 == 0 || nbi == 4 || nbi == 8 || nbi == 16;
-  return gu && dn;
+__host__ __device__ inline bool stream_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+// A row of nb blocks splits into stages of gmax blocks, or is one stage of
+// a power-of-two number of 16-byte chunks.
+__host__ __device__ inline bool stream_row_ok(int nb, int gmax, int bpb) {
+  return nb % gmax == 0 || (nb < gmax && stream_pow2(nb * bpb / 16));
 }
 
-__host__ __device__ inline StreamGeom stream_geom(int H, int I) {
+__host__ __device__ inline bool stream_shape_ok(int H, int I, int bits) {
+  if (H <= 0 || I <= 0 || H % 128 != 0 || I % 128 != 0 || (bits != 4 && bits != 8)) return false;
+  const int bpb = bits == 8 ? 32 : 16;
+  return stream_row_ok(H / 32, 256 / bpb, bpb) && stream_row_ok(I / 32, 512 / bpb, bpb);
+}
+
+__host__ __device__ inline StreamGeom stream_geom(int H, int I, int bits) {
   StreamGeom g{};
   g.H = H;
   g.I = I;
+  g.bits = bits;
+  g.bpb = bits == 8 ? 32 : 16;
   g.nbh = H / 32;
   g.nbi = I / 32;
-  g.g_gu = g.nbh < 16 ? g.nbh : 16;
-  g.g_dn = g.nbi < 32 ? g.nbi : 32;
-  g.swz_gu = (g.g_gu < 8 ? g.g_gu : 8) - 1;
-  g.swz_dn = (g.g_dn < 8 ? g.g_dn : 8) - 1;
+  const int gmax_gu = 256 / g.bpb, gmax_dn = 512 / g.bpb;
+  g.g_gu = g.nbh < gmax_gu ? g.nbh : gmax_gu;
+  g.g_dn = g.nbi < gmax_dn ? g.nbi : gmax_dn;
+  const int ch_gu = g.g_gu * g.bpb / 16, ch_dn = g.g_dn * g.bpb / 16;  // 16-byte chunks per stage row
+  g.swz_gu = (ch_gu < 8 ? ch_gu : 8) - 1;
+  g.swz_dn = (ch_dn < 8 ? ch_dn : 8) - 1;
   g.st_gu = g.nbh / g.g_gu;
   g.st_dn = g.nbi / g.g_dn;
   g.cpu_gu = I / 32;
   g.cpu_dn = H / 32;
-  g.sb_gu = (uint32_t)(64 * g.g_gu * 16);
-  g.sb_dn = (uint32_t)(32 * g.g_dn * 16);
+  g.sb_gu = (uint32_t)(64 * g.g_gu * g.bpb);
+  g.sb_dn = (uint32_t)(32 * g.g_dn * g.bpb);
   g.ub_gu = (uint64_t)g.st_gu * g.sb_gu;
   g.ub_dn = (uint64_t)g.st_dn * g.sb_dn;
   g.dn_off = (uint64_t)g.cpu_gu * g.ub_gu;
@@ -71,19 +87,23 @@ __host__ __device__ inline StreamGeom stream_geom(int H, int I) {
   return g;
 }
 
-// Byte offset, within an expert's streaming copy, of Q8 block b of row r of
-// matrix m (0 gate, 1 up, 2 down).
-__host__ __device__ inline uint64_t stream_block_offset(const StreamGeom& g, int m, int r, int b) {
+// Byte offset, within an expert's streaming copy, of 16-byte chunk h of Q8
+// block b of row r of matrix m (0 gate, 1 up, 2 down).  int4: h = 0 (the
+// whole block); int8: h = 0 the even elements, h = 1 the odd ones.
+__host__ __device__ inline uint64_t stream_chunk_offset(const StreamGeom& g, int m, int r, int b, int h) {
+  const int cpb = g.bpb / 16;  // chunks per block
   if (m < 2) {
     const int u = r / 32, sr = (m == 0 ? 0 : 32) + (r & 31);
     const int s = b / g.g_gu, j = b - s * g.g_gu;
-    return (uint64_t)u * g.ub_gu + (uint64_t)s * g.sb_gu + (uint64_t)sr * g.g_gu * 16 +
-           (uint64_t)((j ^ (sr & g.swz_gu)) * 16);
+    const int c = j * cpb + h;
+    return (uint64_t)u * g.ub_gu + (uint64_t)s * g.sb_gu + (uint64_t)sr * g.g_gu * g.bpb +
+           (uint64_t)((c ^ (sr & g.swz_gu)) * 16);
   }
   const int v = r / 32, sr = r & 31;
   const int s = b / g.g_dn, j = b - s * g.g_dn;
-  return g.dn_off + (uint64_t)v * g.ub_dn + (uint64_t)s * g.sb_dn + (uint64_t)sr * g.g_dn * 16 +
-         (uint64_t)((j ^ (sr & g.swz_dn)) * 16);
+  const int c = j * cpb + h;
+  return g.dn_off + (uint64_t)v * g.ub_dn + (uint64_t)s * g.sb_dn + (uint64_t)sr * g.g_dn * g.bpb +
+         (uint64_t)((c ^ (sr & g.swz_dn)) * 16);
 }
 
 }  // namespace coli

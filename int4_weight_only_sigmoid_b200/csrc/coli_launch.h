@@ -59,6 +59,8 @@ cudaError_t launch_requantize_fp8_int4(const uint8_t* w8, const float* factors, 
                                        int block, uint8_t* q, float* s, cudaStream_t st);
 cudaError_t launch_quantize_act_q8(const float* x, int64_t n_tok, int64_t dim, int8_t* q, float* d,
                                    cudaStream_t st);
+cudaError_t launch_quantize_rows_int8(const float* w, int64_t rows, int64_t cols, int8_t* q, float* s,
+                                      cudaStream_t st);
 
 // Router: scores[t,e] = sigmoid(logit) (contract R), then top-k + weights.
 cudaError_t launch_router_scores(const float* x, const float* w_router, int n_tok, int E, int H,
@@ -142,10 +144,11 @@ struct StreamArgs {
   int32_t* dn_done;     // [H/32] slots done per 32-row chunk of the output (zero at launch)
   int32_t* status;
 };
-bool stream_supported(int hidden, int inter, int n_tok, int n_shared, int top_k);
-uint64_t stream_expert_bytes(int hidden, int inter);
-cudaError_t launch_prepare_expert(int hidden, int inter, const uint8_t* gq, const float* gs, const uint8_t* uq,
-                                  const float* us, const uint8_t* dq, const float* ds, void* dst, cudaStream_t st);
+bool stream_supported(int hidden, int inter, int bits, int n_tok);
+uint64_t stream_expert_bytes(int hidden, int inter, int bits);
+cudaError_t launch_prepare_expert(int hidden, int inter, int bits, const uint8_t* gq, const float* gs,
+                                  const uint8_t* uq, const float* us, const uint8_t* dq, const float* ds, void* dst,
+                                  cudaStream_t st);
 cudaError_t launch_expert_stream(const StreamArgs& a, cudaStream_t st);
 
 // Prefill expert kernels on the tensor cores (tcgen05.mma.kind::i8): the
@@ -162,9 +165,9 @@ size_t prefill_tiles_bound(int n_tok, int K, int E, int n_shared);
 size_t prefill_tile_bytes(int n_tok, int K, int E, int n_shared);
 cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, const Slot* slots,
                                    const int32_t* n_slots, void* tiles, int32_t* n_tiles, const int32_t* perm,
-                                   int K, int n_shared, const int8_t* xq, const float* xd, int n_tok, int hidden,
-                                   int inter, void* xr, int32_t* xm, void* hr, float* hd, int32_t* hm, float* y,
-                                   int32_t* err, cudaStream_t st, cudaEvent_t ev_mid);
+                                   int K, int n_shared, int bits, const int8_t* xq, const float* xd, int n_tok,
+                                   int hidden, int inter, void* xr, int32_t* xm, void* hr, float* hd, int32_t* hm,
+                                   float* y, int32_t* err, cudaStream_t st, cudaEvent_t ev_mid);
 
 // out[t] = sum_k w[t,k] y[inv[t,k]] + sum_s y[n_tok*K + s*n_tok + t]  (contract C)
 cudaError_t launch_combine(const float* y, const int32_t* inv, const float* w, int n_tok, int K,

@@ -12,6 +12,10 @@
 // matching up rows, so SwiGLU and the Q8 block of h are thread-local.  The
 // gate/up item's 128 columns are 64 gate rows and the same 64 up rows.
 //
+// int8 expert weights (the pages' int8 variant) take the same kernel with
+// B signed and copied as it is, A in the elements' own order, and no
+// per-block correction (every accumulator starts at 0x4B400000).
+//
 // Operands.  A = the Q8 activations as signed bytes (one row per (slot,
 // token) in slot order, loaded by TMA, 128-byte swizzle); B = the weights as
 // unsigned bytes q + 8 (0..15), expanded from the packed nibbles by the
@@ -88,7 +92,7 @@ struct PSmem {
   static constexpr int kStageA = kM * 128;          // A: 128 token rows x 128 int8 (4 blocks), 128B-swizzled
   static constexpr int kSubB = kN * 32;             // B, one block: 128 weight rows x 32 bytes
   static constexpr int kOpStage = kStageA + kBS * kSubB;
-  static constexpr int kPk = kN * kBS * 16;         // packed weights of one stage (row-major, 64 B per row)
+  static constexpr int kPk = kN * kBS * 32;         // weights of one stage as copied (64 B per row int4, 128 B int8)
   __host__ __device__ static constexpr size_t bytes() {
     return 1024 + (size_t)kStages * kOpStage + (size_t)kPkSlots * kPk;
   }
@@ -98,10 +102,16 @@ struct Tile {
   int32_t slot, n0;
 };
 
-// Byte offset of packed block c (0..3) of weight row r in a stage's packed
-// copy: 64 B per row, blocks rotated by (r >> 1) & 3 so that 8 consecutive
-// rows reading the same block hit 8 different bank groups.
-__device__ __forceinline__ uint32_t pk_off(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
+// Byte offset of 16-byte chunk c of weight row r in a stage's copy of the
+// weights: int4 rows are 64 B (4 chunks, one per block), rotated by
+// (r >> 1) & 3; int8 rows are 128 B (8 chunks, two per block), rotated by
+// r & 7; either way 8 consecutive rows reading the same chunk hit 8
+// different bank groups.
+template <int BITS>
+__device__ __forceinline__ uint32_t pk_off(int r, int c) {
+  if constexpr (BITS == 4) return r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+  return r * 128 + ((c ^ (r & 7)) << 4);
+}
 
 // Byte offset of 16-byte chunk c (0..1) of row r in a K-major, no-swizzle
 // operand tile of 32 bytes per row: 8-row x 16-byte core matrices, the two
@@ -117,8 +127,10 @@ __device__ __forceinline__ void expand_word(uint32_t w, uint32_t& lo, uint32_t& 
 
 // Operand rows of the Q8 activations in row order: row r < n_tok*K is
 // token perm[r] / K (the routed slots' rows), row n_tok*K + s*n_tok + t is
-// token t (shared expert s); within every 8 elements the order 0,2,4,6,1,3,5,7.
-// 16 values per thread.
+// token t (shared expert s).  With int4 weights, within every 8 elements the
+// order 0,2,4,6,1,3,5,7 (the order of the expanded weights); with int8
+// weights the elements' own order.  16 values per thread.
+template <int BITS>
 __global__ void __launch_bounds__(256) act_rows_i8_kernel(const int8_t* __restrict__ q, const int32_t* perm,
                                                           int n_tok, int top_k, int64_t rows, int hidden,
                                                           uint4* __restrict__ out) {
@@ -130,10 +142,14 @@ __global__ void __launch_bounds__(256) act_rows_i8_kernel(const int8_t* __restri
   const int64_t routed = (int64_t)n_tok * top_k;
   const int64_t tok = r < routed ? (int64_t)(__ldg(perm + r) / top_k) : (r - routed) % n_tok;
   const uint4 v = __ldg(reinterpret_cast<const uint4*>(q + tok * hidden) + c);
-  uint4 o;
-  split_even_odd(v.x, v.y, o.x, o.y);
-  split_even_odd(v.z, v.w, o.z, o.w);
-  out[i] = o;
+  if constexpr (BITS == 8) {
+    out[i] = v;
+  } else {
+    uint4 o;
+    split_even_odd(v.x, v.y, o.x, o.y);
+    split_even_odd(v.z, v.w, o.z, o.w);
+    out[i] = o;
+  }
 }
 
 // Starting accumulator value of every (token, block): 0x4B400000 - 8 * sum
@@ -183,12 +199,13 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor of kind::i8: signed A (activations), unsigned B
-// (weights + 8), int32 accumulator, shape M x N, both K-major.
-__host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N) {
+// Instruction descriptor of kind::i8: signed A (activations), B unsigned
+// (int4 weights + 8) or signed (int8 weights), int32 accumulator, shape
+// M x N, both K-major.
+__host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N, bool b_signed) {
   return (2u << 4)                       // D format: S32
          | (1u << 7)                     // A format: S8
-         | (0u << 10)                    // B format: U8
+         | ((b_signed ? 1u : 0u) << 10)  // B format: U8 / S8
          | ((uint32_t)(N >> 3) << 17)    // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
@@ -256,8 +273,9 @@ __device__ __forceinline__ int64_t item_token_row(const ItemInfo& f, bool gu, co
 }
 
 // GU: gate/up (+ SwiGLU + Q8 of h -> hr int8 rows + hd + hm); !GU: down (-> y).
-// ad / am: the A rows' Q8 scales and starting values, [row x nb].
-template <bool GU, typename Tab>
+// ad / am: the A rows' Q8 scales and starting values, [row x nb] (int8
+// weights need no per-block correction: every start value is 0x4B400000).
+template <bool GU, int BITS, typename Tab>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     const __grid_constant__ Tab tab, const __grid_constant__ CUtensorMap amap, const Slot* __restrict__ slots,
     const Tile* __restrict__ tiles, const int32_t* __restrict__ n_tiles, const int32_t* __restrict__ perm, int top_k,
@@ -312,7 +330,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     // cursor (item ii, stage ji) moves ahead of the expansion.  (The A tiles
     // come from the TMA warp.)
     const int p = threadIdx.x;
-    const size_t rb = (size_t)dim_in / 2;
+    const size_t rb = (size_t)dim_in * BITS / 8;  // bytes per weight row
+    constexpr int kChunks = BITS == 4 ? 4 : 8;      // 16-byte chunks per row per stage
     const int n_mine = blockIdx.x < n_items ? (n_items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
     const int total = n_mine * nst;
     int ii = blockIdx.x, ji = 0;
@@ -335,10 +354,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         const int kb0 = ji * kBS;
         unsigned char* pk = pk_ring + (gj % kPkSlots) * L::kPk;
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {  // W: row it*32 + p/4, chunk p%4 (= block kb0 + p%4)
+        for (int it = 0; it < kChunks; ++it) {  // row q / kChunks, chunk q % kChunks of the stage's bytes
           const int q = it * kNProd + p;
-          const int r = q >> 2, c = q & 3;
-          cp_async16(pk + pk_off(r, c), wrow(r) + (size_t)(kb0 + c) * 16);
+          const int r = q / kChunks, c = q % kChunks;
+          cp_async16(pk + pk_off<BITS>(r, c), wrow(r) + (size_t)kb0 * (BITS * 4) + (size_t)c * 16);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
         if (++ji == nst) {
@@ -364,13 +383,18 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         unsigned char* ob = op_ring + s * L::kOpStage + L::kStageA;
 #pragma unroll
         for (int c = 0; c < kBS; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(pk + pk_off(p, c));
           unsigned char* dst = ob + c * L::kSubB;
           uint4 o0, o1;
-          expand_word(w.x, o0.x, o0.y);
-          expand_word(w.y, o0.z, o0.w);
-          expand_word(w.z, o1.x, o1.y);
-          expand_word(w.w, o1.z, o1.w);
+          if constexpr (BITS == 4) {
+            const uint4 w = *reinterpret_cast<const uint4*>(pk + pk_off<4>(p, c));
+            expand_word(w.x, o0.x, o0.y);
+            expand_word(w.y, o0.z, o0.w);
+            expand_word(w.z, o1.x, o1.y);
+            expand_word(w.w, o1.z, o1.w);
+          } else {  // int8 rows are the operand as they are
+            o0 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(p, 2 * c));
+            o1 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(p, 2 * c + 1));
+          }
           *reinterpret_cast<uint4*>(dst + op_off(p, 0)) = o0;
           *reinterpret_cast<uint4*>(dst + op_off(p, 1)) = o1;
         }
@@ -385,7 +409,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     if (lane == 0) {
       int gs = 0, gh = 0;
       bool ok = true;
-      constexpr uint32_t idesc = idesc_i8_s32(kM, kN);
+      constexpr uint32_t idesc = idesc_i8_s32(kM, kN, BITS == 8);
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
         for (int j = 0; j < nst && ok; ++j, ++gs) {
           const int s = gs % kStages;
@@ -464,7 +488,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     // starting value of this thread's lane for block b of item `it` (0 if
     // the lane holds no token there: that lane's result is never read)
     auto start_value = [&](int it, int b) -> uint32_t {
-      if (it >= n_items) return kMagic;
+      if (BITS == 8 || it >= n_items) return kMagic;
       const ItemInfo f = item_info(slots, tiles, it, nm, kGroupRows);
       if (n >= f.n_valid) return kMagic;
       return (uint32_t)__ldg(am + item_token_row(f, GU, perm, top_k, n) * nb + b);
@@ -543,10 +567,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
             // the buffer's next use: block b + kBS of this item, else block
             // b + kBS - nb of the next item
             uint32_t v = kMagic;
-            if (b + kBS < nb) {
-              if (valid) v = (uint32_t)__ldg(mrow + b + kBS);
-            } else if (nrow >= 0) {
-              v = (uint32_t)__ldg(am + nrow * nb + (b + kBS - nb));
+            if constexpr (BITS == 4) {
+              if (b + kBS < nb) {
+                if (valid) v = (uint32_t)__ldg(mrow + b + kBS);
+              } else if (nrow >= 0) {
+                v = (uint32_t)__ldg(am + nrow * nb + (b + kBS - nb));
+              }
             }
             write_start(hb * kHalf + i, v);
           }
@@ -572,7 +598,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
             amax = fmaxf(amax, fabsf(acc0[j]));
           }
           const float d = __fdiv_rn(amax, 127.0f);
-          // q in the operand order (per 8 elements: 0,2,4,6,1,3,5,7) and the block sum
+          // q in the operand order (int4 weights: per 8 elements 0,2,4,6,1,3,5,7;
+          // int8: the elements' order) and the block sum
           uint32_t pk[8];
           int sum = 0;
 #pragma unroll
@@ -585,8 +612,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
               lo |= ((uint32_t)qe & 0xFFu) << (8 * i);
               hi |= ((uint32_t)qo & 0xFFu) << (8 * i);
             }
-            pk[2 * e8] = lo;
-            pk[2 * e8 + 1] = hi;
+            if constexpr (BITS == 4) {
+              pk[2 * e8] = lo;
+              pk[2 * e8 + 1] = hi;
+            } else {  // back to element order: even / odd bytes interleaved
+              pk[2 * e8] = __byte_perm(lo, hi, 0x5140);
+              pk[2 * e8 + 1] = __byte_perm(lo, hi, 0x7362);
+            }
           }
           uint4* dst = reinterpret_cast<uint4*>(hr + row * inter + o);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -689,16 +721,20 @@ cudaError_t make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int co
 
 cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, const Slot* slots,
                                    const int32_t* n_slots, void* tiles, int32_t* n_tiles, const int32_t* perm,
-                                   int K, int n_shared, const int8_t* xq, const float* xd, int n_tok, int hidden,
-                                   int inter, void* xr, int32_t* xm, void* hr, float* hd, int32_t* hm, float* y,
-                                   int32_t* err, cudaStream_t st, cudaEvent_t ev_mid) {
+                                   int K, int n_shared, int bits, const int8_t* xq, const float* xd, int n_tok,
+                                   int hidden, int inter, void* xr, int32_t* xm, void* hr, float* hd, int32_t* hm,
+                                   float* y, int32_t* err, cudaStream_t st, cudaEvent_t ev_mid) {
   Tile* t = reinterpret_cast<Tile*>(tiles);
   const int64_t rows = (int64_t)n_tok * (K + n_shared);
   const int64_t n16 = rows * hidden / 16;
-  act_rows_i8_kernel<<<(unsigned)((n16 + 255) / 256), 256, 0, st>>>(xq, perm, n_tok, K, rows, hidden,
-                                                                    reinterpret_cast<uint4*>(xr));
+  if (bits == 8)
+    act_rows_i8_kernel<8><<<(unsigned)((n16 + 255) / 256), 256, 0, st>>>(xq, perm, n_tok, K, rows, hidden,
+                                                                         reinterpret_cast<uint4*>(xr));
+  else
+    act_rows_i8_kernel<4><<<(unsigned)((n16 + 255) / 256), 256, 0, st>>>(xq, perm, n_tok, K, rows, hidden,
+                                                                         reinterpret_cast<uint4*>(xr));
   const int64_t nblk = (int64_t)n_tok * (hidden / 32);
-  act_magic_kernel<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(xq, nblk, xm);
+  if (bits == 4) act_magic_kernel<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(xq, nblk, xm);
   build_tiles_kernel<<<1, 32, 0, st>>>(slots, n_slots, t, n_tiles);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -714,16 +750,28 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
       (e = cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
   const size_t smem = PSmem::bytes();
-  if ((e = smem_opt_in_once(prefill_kernel<true, GateUpTable>, (int)smem, mask_gu)) != cudaSuccess) return e;
-  if ((e = smem_opt_in_once(prefill_kernel<false, DownTable>, (int)smem, mask_dn)) != cudaSuccess) return e;
   const int grid = sms_cache[dev];
   int8_t* hri = reinterpret_cast<int8_t*>(hr);
-  prefill_kernel<true, GateUpTable><<<grid, kThreadsP, smem, st>>>(gu, map_x, slots, t, n_tiles, perm, K, xd, xm,
-                                                                     hidden, inter, hri, hd, hm, y, err);
+  if (bits == 8) {
+    static uint64_t mask_gu8 = 0, mask_dn8 = 0;
+    if ((e = smem_opt_in_once(prefill_kernel<true, 8, GateUpTable>, (int)smem, mask_gu8)) != cudaSuccess) return e;
+    if ((e = smem_opt_in_once(prefill_kernel<false, 8, DownTable>, (int)smem, mask_dn8)) != cudaSuccess) return e;
+    prefill_kernel<true, 8, GateUpTable><<<grid, kThreadsP, smem, st>>>(gu, map_x, slots, t, n_tiles, perm, K, xd,
+                                                                          xm, hidden, inter, hri, hd, hm, y, err);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev_mid && (e = cudaEventRecordWithFlags(ev_mid, st, cudaEventRecordExternal)) != cudaSuccess) return e;
+    prefill_kernel<false, 8, DownTable><<<grid, kThreadsP, smem, st>>>(dn, map_h, slots, t, n_tiles, perm, K, hd,
+                                                                         hm, hidden, inter, hri, hd, hm, y, err);
+    return cudaGetLastError();
+  }
+  if ((e = smem_opt_in_once(prefill_kernel<true, 4, GateUpTable>, (int)smem, mask_gu)) != cudaSuccess) return e;
+  if ((e = smem_opt_in_once(prefill_kernel<false, 4, DownTable>, (int)smem, mask_dn)) != cudaSuccess) return e;
+  prefill_kernel<true, 4, GateUpTable><<<grid, kThreadsP, smem, st>>>(gu, map_x, slots, t, n_tiles, perm, K, xd, xm,
+                                                                        hidden, inter, hri, hd, hm, y, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecordWithFlags(ev_mid, st, cudaEventRecordExternal)) != cudaSuccess) return e;
-  prefill_kernel<false, DownTable><<<grid, kThreadsP, smem, st>>>(dn, map_h, slots, t, n_tiles, perm, K, hd, hm,
-                                                                    hidden, inter, hri, hd, hm, y, err);
+  prefill_kernel<false, 4, DownTable><<<grid, kThreadsP, smem, st>>>(dn, map_h, slots, t, n_tiles, perm, K, hd, hm,
+                                                                       hidden, inter, hri, hd, hm, y, err);
   return cudaGetLastError();
 }
 

@@ -49,6 +49,42 @@ __global__ void __launch_bounds__(256) quantize_rows_int4_kernel(const float* __
   if (lane == 0) s[row] = scale;
 }
 
+// One warp per row.  int8 weights: scale = absmax/127; q = rint(w/scale)
+// in [-127,127], one byte per element ("Colibri：在笔记本上跑744B参数的AI
+// 模型", "关键特性": the int8 kernel variant).
+__global__ void __launch_bounds__(256) quantize_rows_int8_kernel(const float* __restrict__ w, int64_t rows,
+                                                                 int64_t cols, int8_t* __restrict__ q,
+                                                                 float* __restrict__ s) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float* wr = w + row * cols;
+  float amax = 0.0f;
+  for (int64_t c = lane * 4; c < cols; c += 128) {
+    const float4 v = *reinterpret_cast<const float4*>(wr + c);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+  amax = warp_max(amax);
+  const float scale = __fdiv_rn(amax, 127.0f);
+  uint32_t* qr = reinterpret_cast<uint32_t*>(q + row * cols);
+  for (int64_t g = lane; g < cols / 4; g += 32) {
+    const float4 a = *reinterpret_cast<const float4*>(wr + 4 * g);
+    const float e[4] = {a.x, a.y, a.z, a.w};
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int qi = 0;
+      if (amax != 0.0f) {
+        qi = (int)rintf(__fdiv_rn(e[i], scale));
+        qi = qi < -127 ? -127 : (qi > 127 ? 127 : qi);
+      }
+      word |= ((uint32_t)qi & 0xFFu) << (8 * i);
+    }
+    qr[g] = word;
+  }
+  if (lane == 0) s[row] = scale;
+}
+
 // FP8 -> int4 requantiser (the converter: "GLM-5.2-colibri-int4架构解析…",
 // "GLM-5.2-colibri-int4的量化流程": FP8 e4m3 source -> F32 -> int4 per
 // row; config weight_block_size [128, 128]).  e4m3 code -> F32, exact:
@@ -195,6 +231,12 @@ int blocks_for(int64_t items, int per_block) {
 cudaError_t launch_quantize_rows_int4(const float* w, int64_t rows, int64_t cols, uint8_t* q, float* s,
                                       cudaStream_t st) {
   quantize_rows_int4_kernel<<<blocks_for(rows, 8), 256, 0, st>>>(w, rows, cols, q, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_rows_int8(const float* w, int64_t rows, int64_t cols, int8_t* q, float* s,
+                                      cudaStream_t st) {
+  quantize_rows_int8_kernel<<<blocks_for(rows, 8), 256, 0, st>>>(w, rows, cols, q, s);
   return cudaGetLastError();
 }
 

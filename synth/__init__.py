@@ -59,7 +59,7 @@ def tid_shared(s: int, m: int) -> int:
 _GLM = dict(hidden=6144, inter=2048, n_experts=256, top_k=8, n_shared=1, shared_inter=2048,
             norm_topk_prob=True, routed_scaling_factor=2.5, sigma_router=0.006,
             bias_lo=-0.05, bias_hi=0.05, sigma_expert=0.01, x_kind="normal",
-            bias_boost_n=0, bias_boost=0.0, n_layers=1, seed=0)
+            bias_boost_n=0, bias_boost=0.0, n_layers=1, seed=0, weight_bits=4)
 
 CONFIGS = {
     "tiny": dict(_GLM, hidden=256, inter=128, n_experts=16, top_k=4, shared_inter=128,
@@ -70,6 +70,7 @@ CONFIGS = {
     "prefill2048": dict(_GLM, n_tok=2048, bias_boost_n=32, bias_boost=0.2),
     "stack8": dict(_GLM, n_tok=1, n_layers=8, rms_eps=1e-5),
     "stack8_512": dict(_GLM, n_tok=512, n_layers=8, rms_eps=1e-5),
+    "decode1_int8": dict(_GLM, n_tok=1, weight_bits=8),
 }
 
 

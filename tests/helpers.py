@@ -11,12 +11,14 @@ _qcache: dict = {}
 
 
 def oracle_expert(cfg: dict, layer: int, e: int, shared: bool = False) -> oracle.QExpert:
-    key = (cfg["name"], cfg["seed"], cfg["hidden"], cfg["inter"], layer, e, shared)
+    bits = cfg.get("weight_bits", 4)
+    key = (cfg["name"], cfg["seed"], cfg["hidden"], cfg["inter"], layer, e, shared, bits, cfg["sigma_expert"])
     if key not in _qcache:
+        quant = oracle.quantize_rows_int4 if bits == 4 else oracle.quantize_rows_int8
         mats = []
         for m in (synth.GATE, synth.UP, synth.DOWN):
-            mats.extend(oracle.quantize_rows_int4(synth.expert_matrix(cfg, layer, e, m, shared)))
-        _qcache[key] = oracle.QExpert(*mats)
+            mats.extend(quant(synth.expert_matrix(cfg, layer, e, m, shared)))
+        _qcache[key] = oracle.QExpert(*mats, bits=bits)
     return _qcache[key]
 
 

@@ -125,6 +125,22 @@ def test_prepared_bytes_and_prepare_arguments(lib):
                                       None) == m.COLI_EINVAL
 
 
+def test_int8_weight_config_checks(lib):
+    """weight_bits 8: the streaming copy holds one byte per weight; other
+    widths are refused; the reference-shape expert call is int4 only."""
+    import int4_weight_only_sigmoid_b200 as m
+    c8 = m.make_config(6144, 2048, 256, 8, 1, weight_bits=8)
+    per_expert = (3 * 2048 * 6144 + (2 * 2048 + 6144) * 4 + 255) // 256 * 256
+    assert m.prepared_bytes(c8) == 257 * per_expert
+    assert m.workspace_bytes(m.make_config(6144, 2048, 256, 8, 1, weight_bits=5), 1) == 0
+    assert m.workspace_bytes(m.make_config(256, 96, 16, 4, 1, weight_bits=8), 1) == 0  # inter % 128
+    e = m.Expert(256, 256, 256, 256, 256, 256)
+    rc = lib.coli_moe_expert_ffn(C.byref(c8), C.byref(e), C.c_void_p(256), C.c_void_p(256), 1, C.c_void_p(256),
+                                 C.c_void_p(256), 1 << 30, None)
+    assert rc == m.COLI_EINVAL and b"int4" in lib.coli_last_error()
+    assert lib.coli_quantize_rows_int8(C.c_void_p(16), 2, 40, C.c_void_p(16), C.c_void_p(16), None) == m.COLI_EINVAL
+
+
 def test_zero_tokens_is_ok_without_touching_pointers(lib):
     import int4_weight_only_sigmoid_b200 as m
     assert lib.coli_quantize_act_q8(None, 0, 64, None, None, None) == m.COLI_OK

@@ -25,7 +25,7 @@ def _dev_layer(cfg, layer=0):
     from synth.layers import device_layer
     key = (cfg["hidden"], cfg["inter"], cfg["n_experts"], cfg["top_k"], cfg["n_shared"], layer, cfg["seed"],
            cfg["norm_topk_prob"], cfg["routed_scaling_factor"], cfg.get("bias_boost_n", 0),
-           cfg["sigma_expert"], cfg["sigma_router"], cfg["bias_lo"], cfg["bias_hi"])
+           cfg["sigma_expert"], cfg["sigma_router"], cfg["bias_lo"], cfg["bias_hi"], cfg.get("weight_bits", 4))
     if key not in _layers:
         if len(_layers) > 3:
             _layers.clear()
