@@ -597,12 +597,11 @@ __global__ void prepare_expert_kernel(StreamGeom g, const uint8_t* __restrict__ 
 
 template <int TT, int BITS>
 cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
-  static uint64_t attr_mask = 0;
+  static int granted[64] = {};
   static int sms[64] = {};
   const size_t smem = stream_smem_bytes<TT>(a.g);
-  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
-  // the opt-in is set once per device, so to the largest size any shape needs
-  cudaError_t e = smem_opt_in_once(expert_stream_kernel<TT, BITS>, 227 * 1024, attr_mask);
+  if (smem > 224 * 1024) return cudaErrorInvalidConfiguration;
+  cudaError_t e = smem_opt_in(expert_stream_kernel<TT, BITS>, (int)smem, granted);
   if (e != cudaSuccess) return e;
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -620,8 +619,8 @@ cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
 bool stream_supported(int hidden, int inter, int bits, int n_tok) {
   if (n_tok < 1 || n_tok > kStreamMaxTok || !stream_shape_ok(hidden, inter, bits)) return false;
   const StreamGeom g = stream_geom(hidden, inter, bits);
-  return stream_smem_bytes<4>(g) <= 227 * 1024 && stream_smem_bytes<1>(g) <= 227 * 1024 &&
-         stream_smem_bytes<2>(g) <= 227 * 1024;
+  constexpr size_t kDyn = 224 * 1024;  // 227 KB per block, less the kernel's static shared memory
+  return stream_smem_bytes<4>(g) <= kDyn && stream_smem_bytes<1>(g) <= kDyn && stream_smem_bytes<2>(g) <= kDyn;
 }
 
 uint64_t stream_expert_bytes(int hidden, int inter, int bits) { return stream_geom(hidden, inter, bits).expert_bytes; }

@@ -149,8 +149,8 @@ template <int TT>
 cudaError_t gateup_tt(const GateUpTable& tbl, const GemvSlots& sl, const int8_t* xq, const float* xd, int hidden,
                       int inter, int8_t* hq, float* hd, cudaStream_t st) {
   const size_t smem = GemvSmem<TT>::bytes(hidden);
-  static uint64_t attr_dev_mask = 0;
-  const cudaError_t e = smem_opt_in_once(gateup_kernel<TT>, 200 * 1024, attr_dev_mask);
+  static int granted[64] = {};
+  const cudaError_t e = smem_opt_in(gateup_kernel<TT>, 200 * 1024, granted);
   if (e != cudaSuccess) return e;
   dim3 grid(inter / 32, sl.max_slots);
   gateup_kernel<TT><<<grid, kThreads, smem, st>>>(tbl, sl, xq, xd, hidden, inter, hq, hd);
@@ -161,8 +161,8 @@ template <int TT>
 cudaError_t down_tt(const DownTable& tbl, const GemvSlots& sl, const int8_t* hq, const float* hd, int hidden,
                     int inter, float* y, cudaStream_t st) {
   const size_t smem = GemvSmem<TT>::bytes(inter);
-  static uint64_t attr_dev_mask = 0;
-  const cudaError_t e = smem_opt_in_once(down_kernel<TT>, 200 * 1024, attr_dev_mask);
+  static int granted[64] = {};
+  const cudaError_t e = smem_opt_in(down_kernel<TT>, 200 * 1024, granted);
   if (e != cudaSuccess) return e;
   dim3 grid(hidden / 64, sl.max_slots);
   down_kernel<TT><<<grid, kThreads, smem, st>>>(tbl, sl, hq, hd, hidden, inter, y);

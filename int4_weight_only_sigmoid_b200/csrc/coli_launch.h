@@ -34,19 +34,20 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Set a kernel's dynamic shared-memory opt-in once per device (the
-// attribute belongs to the device's context); `mask` is the caller's
-// per-kernel record of the devices done (devices 0..63).  Pass the largest
-// size the kernel is ever launched with: later calls do not raise it.
+// Raise a kernel's dynamic shared-memory opt-in on the current device to
+// `bytes` when the last setting there is lower (the attribute belongs to the
+// device's context; `granted` is the caller's per-kernel record for devices
+// 0..63).  The opt-in plus the kernel's static shared memory must stay
+// within the device's per-block limit, so ask for what the launch needs.
 template <typename KernelT>
-cudaError_t smem_opt_in_once(KernelT* kernel, int bytes, uint64_t& mask) {
+cudaError_t smem_opt_in(KernelT* kernel, int bytes, int (&granted)[64]) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (mask & (uint64_t(1) << dev)) return cudaSuccess;
+  if (granted[dev] >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) mask |= uint64_t(1) << dev;
+  if (e == cudaSuccess) granted[dev] = bytes;
   return e;
 }
 

@@ -741,7 +741,7 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
   CUtensorMap map_x, map_h;
   if ((e = make_rows_map(&map_x, xr, rows, hidden)) != cudaSuccess) return e;
   if ((e = make_rows_map(&map_h, hr, rows, inter)) != cudaSuccess) return e;
-  static uint64_t mask_gu = 0, mask_dn = 0;
+  static int mask_gu[64] = {}, mask_dn[64] = {};
   static int sms_cache[64] = {};
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -753,9 +753,9 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
   const int grid = sms_cache[dev];
   int8_t* hri = reinterpret_cast<int8_t*>(hr);
   if (bits == 8) {
-    static uint64_t mask_gu8 = 0, mask_dn8 = 0;
-    if ((e = smem_opt_in_once(prefill_kernel<true, 8, GateUpTable>, (int)smem, mask_gu8)) != cudaSuccess) return e;
-    if ((e = smem_opt_in_once(prefill_kernel<false, 8, DownTable>, (int)smem, mask_dn8)) != cudaSuccess) return e;
+    static int mask_gu8[64] = {}, mask_dn8[64] = {};
+    if ((e = smem_opt_in(prefill_kernel<true, 8, GateUpTable>, (int)smem, mask_gu8)) != cudaSuccess) return e;
+    if ((e = smem_opt_in(prefill_kernel<false, 8, DownTable>, (int)smem, mask_dn8)) != cudaSuccess) return e;
     prefill_kernel<true, 8, GateUpTable><<<grid, kThreadsP, smem, st>>>(gu, map_x, slots, t, n_tiles, perm, K, xd,
                                                                           xm, hidden, inter, hri, hd, hm, y, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -764,8 +764,8 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
                                                                          hm, hidden, inter, hri, hd, hm, y, err);
     return cudaGetLastError();
   }
-  if ((e = smem_opt_in_once(prefill_kernel<true, 4, GateUpTable>, (int)smem, mask_gu)) != cudaSuccess) return e;
-  if ((e = smem_opt_in_once(prefill_kernel<false, 4, DownTable>, (int)smem, mask_dn)) != cudaSuccess) return e;
+  if ((e = smem_opt_in(prefill_kernel<true, 4, GateUpTable>, (int)smem, mask_gu)) != cudaSuccess) return e;
+  if ((e = smem_opt_in(prefill_kernel<false, 4, DownTable>, (int)smem, mask_dn)) != cudaSuccess) return e;
   prefill_kernel<true, 4, GateUpTable><<<grid, kThreadsP, smem, st>>>(gu, map_x, slots, t, n_tiles, perm, K, xd, xm,
                                                                         hidden, inter, hri, hd, hm, y, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -413,8 +413,8 @@ size_t bucket_smem_bytes(int E) { return (size_t)E * (5 + 64) * sizeof(int); }
 cudaError_t launch_router_scores(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
                                  cudaStream_t st) {
   if (n_tok >= 64 && H % (4 * kRtChunk) == 0) {
-    static uint64_t attr_dev_mask = 0;
-    const cudaError_t e = smem_opt_in_once(router_tiled_kernel, (int)router_tiled_smem(), attr_dev_mask);
+    static int granted[64] = {};
+    const cudaError_t e = smem_opt_in(router_tiled_kernel, (int)router_tiled_smem(), granted);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((n_tok + kRtTok - 1) / kRtTok), (unsigned)((E + kRtExp - 1) / kRtExp));
     router_tiled_kernel<<<grid, 256, router_tiled_smem(), st>>>(x, w_router, n_tok, E, H, scores);
@@ -442,8 +442,8 @@ cudaError_t launch_router_decode(const float* x, const float* w_router, int n_to
                                  int8_t* xq, float* xd, int32_t* status_clear, int32_t* zero, int n_zero,
                                  cudaStream_t st) {
   const size_t smem = (size_t)(2 + (n_tok <= kStageTok ? n_tok : 0)) * H * sizeof(float);
-  static uint64_t attr_dev_mask = 0;
-  const cudaError_t e = smem_opt_in_once(router_decode_kernel, 200 * 1024, attr_dev_mask);
+  static int granted[64] = {};
+  const cudaError_t e = smem_opt_in(router_decode_kernel, 200 * 1024, granted);
   if (e != cudaSuccess) return e;
   router_decode_kernel<<<(E + 1) / 2, 256, smem, st>>>(x, w_router, n_tok, E, H, scores, xq, xd, status_clear,
                                                        zero, n_zero);
@@ -461,8 +461,8 @@ cudaError_t launch_bucket(const int32_t* idx, int n_tok, int K, int E, int n_sha
                           int32_t* offsets, int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots,
                           int32_t* status, cudaStream_t st) {
   const size_t smem = bucket_smem_bytes(E);
-  static uint64_t attr_dev_mask = 0;  // the opt-in is per device
-  const cudaError_t e = smem_opt_in_once(bucket_kernel, (int)bucket_smem_bytes(kMaxExperts), attr_dev_mask);
+  static int granted[64] = {};  // the opt-in is per device
+  const cudaError_t e = smem_opt_in(bucket_kernel, (int)bucket_smem_bytes(kMaxExperts), granted);
   if (e != cudaSuccess) return e;
   bucket_kernel<<<1, kBucketThreads, smem, st>>>(idx, n_tok, K, E, n_shared, counts, offsets, perm, inv, slots,
                                                   n_slots, status);
