@@ -263,6 +263,20 @@ coli_status coli_debug_block_partials(const coli_expert* expert, int32_t which, 
 coli_status coli_moe_layer_forward_noalloc(const coli_moe_layer* layer, const float* x, int64_t n_tok,
                                            float* out, void* stream);
 
+/* Test hook: arms a capture of every per-32-block int32 partial sum that the
+ * NEXT coli_moe_layer_forward call on this thread computes, taken inside the
+ * expert kernels that run (the streaming kernel of a prepared layer, or the
+ * tensor-core kernels: the same kernels with the sums also stored; other
+ * calls return COLI_EINVAL and consume the arming).  isum_out (device,
+ * 16-byte aligned, n_words int32) receives, for token t and rank k of its
+ * routed experts (row t*(K+S) + k) and for shared expert s (row
+ * t*(K+S) + K + s), P = 2*inter*(hidden/32) + hidden*(inter/32) words:
+ * gate [inter][hidden/32], up [inter][hidden/32], down [hidden][inter/32],
+ * where entry [o][b] = sum_{j<32} q_w[o, 32b+j] * q_in[32b+j] (q_in: the
+ * token's Q8 x for gate/up, its Q8 h for down).  The forward fails with
+ * COLI_EINVAL if n_words < n_tok*(K+S)*P. */
+coli_status coli_debug_capture_partials(int32_t* isum_out, size_t n_words);
+
 /* Profiling hook: arms three cudaEvent_t handles (any may be NULL) that the
  * NEXT coli_moe_layer_forward call made on this thread records on its
  * stream: `before_experts` just before the gate/up kernel, `after_gateup`

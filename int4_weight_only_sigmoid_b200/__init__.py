@@ -26,6 +26,7 @@ EXPORTS = [
     "coli_moe_workspace_bytes", "coli_last_error", "coli_debug_block_partials",
     "coli_debug_phase_events", "coli_moe_layer_forward_noalloc", "coli_sync_status", "coli_debug_wait_probe",
     "coli_requantize_fp8_int4", "coli_moe_prepared_bytes", "coli_moe_prepare", "coli_quantize_rows_int8",
+    "coli_debug_capture_partials",
 ]
 
 
@@ -86,6 +87,7 @@ def load(path: str | None = None):
         "coli_requantize_fp8_int4": (st, [vp, vp, i64, i64, i32, vp, vp, vp]),
         "coli_moe_prepared_bytes": (C.c_size_t, [C.POINTER(MoeConfig)]),
         "coli_quantize_rows_int8": (st, [vp, i64, i64, vp, vp, vp]),
+        "coli_debug_capture_partials": (st, [vp, C.c_size_t]),
         "coli_moe_prepare": (st, [C.POINTER(MoeLayerC), vp, C.c_size_t, vp]),
     }
     for name, (res, args) in sig.items():
@@ -320,6 +322,20 @@ def debug_block_partials(expert: QExpert, which: int, xq, rows: int, stream=None
     _check(lib().coli_debug_block_partials(C.byref(e), which, _ptr(xq), T, dim_in, rows, _ptr(out),
                                            _stream(stream)))
     return out
+
+
+def capture_partials(layer: MoeLayer, x, cstruct=None, stream=None):
+    """Run one layer forward with the partials capture armed; returns
+    (out, isum) with isum [T, K+S, P] int32 (coli_debug_capture_partials)."""
+    import torch
+    c = layer.cfg
+    H, I, K, S = c.hidden, c.inter, c.top_k, c.n_shared
+    P = 2 * I * (H // 32) + H * (I // 32)
+    T = x.shape[0]
+    buf = torch.full((T, K + S, P), -(2 ** 31), dtype=torch.int32, device=x.device)
+    _check(lib().coli_debug_capture_partials(_ptr(buf), buf.numel()))
+    out = moe_layer_forward(layer, x, cstruct=cstruct, stream=stream)
+    return out, buf
 
 
 def arm_phase_events(before_experts=None, after_gateup=None, after_down=None):

@@ -16,6 +16,8 @@ namespace {
 
 thread_local std::string g_last_error;
 thread_local cudaEvent_t g_phase_ev[3] = {nullptr, nullptr, nullptr};
+thread_local int32_t* g_capture = nullptr;  // armed partials capture (coli_debug_capture_partials)
+thread_local size_t g_capture_words = 0;
 
 coli_status fail(coli_status st, const char* fmt, ...) {
   char buf[512];
@@ -198,6 +200,16 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
 
   cudaEvent_t ev[3] = {g_phase_ev[0], g_phase_ev[1], g_phase_ev[2]};
   g_phase_ev[0] = g_phase_ev[1] = g_phase_ev[2] = nullptr;
+  int32_t* capture = g_capture;
+  const size_t capture_words = g_capture_words;
+  g_capture = nullptr;
+  g_capture_words = 0;
+  if (capture != nullptr) {
+    const size_t P = 2 * (size_t)I * (H / 32) + (size_t)H * (I / 32);
+    const size_t need = (size_t)T * (K + S) * P;
+    if (capture_words < need)
+      return fail(COLI_EINVAL, "%s: the partials capture needs %zu int32 words, %zu given", fn, need, capture_words);
+  }
   auto mark = [&](int i) -> cudaError_t {
     return ev[i] ? cudaEventRecordWithFlags(ev[i], st, cudaEventRecordExternal) : cudaSuccess;
   };
@@ -230,12 +242,16 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
     a.h_ready = ctr;
     a.dn_done = ctr + kStreamMaxSlots;
     a.status = status;
+    a.dbg = capture;
     CHECK_LAUNCH(launch_expert_stream(a, st));
     CHECK_LAUNCH(mark(1));
     CHECK_LAUNCH(mark(2));
     return COLI_OK;
   }
   if (bits == 4 && T <= kDecodeMaxTok && decode_supported(H, I)) {
+    if (capture != nullptr)
+      return fail(COLI_EINVAL, "%s: the partials capture covers the streaming (prepared layer, <= %d tokens) and "
+                  "tensor-core kernels, not this call's decode kernels", fn, kStreamMaxTok);
     // decode: 5 kernels, the last four launched with PDL
     CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, xq, xd, clear_status ? status : nullptr,
                                       nullptr, 0, st));
@@ -268,8 +284,10 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
     CHECK_LAUNCH(launch_prefill_experts(gu, dn, slots, n_slots, at<void>(ws, W.tiles), at<int32_t>(ws, W.n_tiles),
                                         perm, K, S, bits, xq, xd, (int)T, H, I, at<void>(ws, W.xr),
                                         at<int32_t>(ws, W.xm), hq, hd, at<int32_t>(ws, W.hm), y,
-                                        at<int32_t>(ws, W.status), st, ev[1]));
+                                        at<int32_t>(ws, W.status), st, ev[1], capture, E));
   } else {
+    if (capture != nullptr)
+      return fail(COLI_EINVAL, "%s: the partials capture covers the streaming and tensor-core kernels only", fn);
     CHECK_LAUNCH(launch_gateup(gu, sl, xq, xd, H, I, max_tok, hq, hd, st));
     CHECK_LAUNCH(mark(1));
     CHECK_LAUNCH(launch_down(dn, sl, hq, hd, H, I, max_tok, y, st));
@@ -288,6 +306,15 @@ void set_error_message(const char* msg) { g_last_error = msg; }
 using namespace coli;
 
 COLI_EXPORT const char* coli_last_error(void) { return g_last_error.c_str(); }
+
+COLI_EXPORT coli_status coli_debug_capture_partials(int32_t* isum_out, size_t n_words) {
+  const char* fn = "coli_debug_capture_partials";
+  if (isum_out == nullptr || (reinterpret_cast<uintptr_t>(isum_out) & 15u) != 0)
+    return fail(COLI_EINVAL, "%s: isum_out must be a 16-byte aligned device pointer", fn);
+  g_capture = isum_out;
+  g_capture_words = n_words;
+  return COLI_OK;
+}
 
 COLI_EXPORT coli_status coli_debug_phase_events(void* before_experts, void* after_gateup, void* after_down) {
   g_phase_ev[0] = (cudaEvent_t)before_experts;

@@ -154,10 +154,10 @@ __device__ __forceinline__ int isum_of(const uint4& a, const uint4& b, const uin
 
 // One gate/up stage: blocks b0 .. b0+G-1 of gate row l and up row l (lane
 // l) against the slot's staged tokens.
-template <int TT, int BITS>
+template <int TT, int BITS, bool DBG>
 __device__ __forceinline__ void gu_stage(const unsigned char* st, int G, int swz, int b0, int nb, int nv,
                                          const int (&tok)[TT], const uint4* xpl, const float2* xdc, float (&ag)[TT],
-                                         float (&au)[TT]) {
+                                         float (&au)[TT], int32_t* const (&dg)[TT], int32_t* const (&du)[TT]) {
   const int lane = threadIdx.x & 31;
   constexpr int cpb = BITS / 4;  // 16-byte chunks per block
   const uint4* rg = reinterpret_cast<const uint4*>(st) + lane * G * cpb;
@@ -175,8 +175,13 @@ __device__ __forceinline__ void gu_stage(const unsigned char* st, int G, int swz
         const uint4 xe = xpl[2 * xi], xo = xpl[2 * xi + 1];
         const float2 dc = xdc[xi];
         const int c16 = __float_as_int(dc.y);
-        ag[t] = __fmaf_rn(dc.x, __int2float_rn(isum_of<BITS>(ge, go, xe, xo, c16)), ag[t]);
-        au[t] = __fmaf_rn(dc.x, __int2float_rn(isum_of<BITS>(ue, uo, xe, xo, c16)), au[t]);
+        const int ig = isum_of<BITS>(ge, go, xe, xo, c16), iu = isum_of<BITS>(ue, uo, xe, xo, c16);
+        if constexpr (DBG) {
+          dg[t][b0 + j] = ig;
+          du[t][b0 + j] = iu;
+        }
+        ag[t] = __fmaf_rn(dc.x, __int2float_rn(ig), ag[t]);
+        au[t] = __fmaf_rn(dc.x, __int2float_rn(iu), au[t]);
       }
     }
   }
@@ -184,9 +189,10 @@ __device__ __forceinline__ void gu_stage(const unsigned char* st, int G, int swz
 
 // One down stage: blocks b0 .. b0+G-1 of down row l (lane l) against the
 // slot's staged h rows (token t of the slot at index t).
-template <int TT, int BITS>
+template <int TT, int BITS, bool DBG>
 __device__ __forceinline__ void dn_stage(const unsigned char* st, int G, int swz, int b0, int nb, int nv,
-                                         const uint4* hpl, const float2* hdc, float (&ay)[TT]) {
+                                         const uint4* hpl, const float2* hdc, float (&ay)[TT],
+                                         int32_t* const (&dd)[TT]) {
   const int lane = threadIdx.x & 31;
   constexpr int cpb = BITS / 4;
   const uint4* rw = reinterpret_cast<const uint4*>(st) + lane * G * cpb;
@@ -201,13 +207,15 @@ __device__ __forceinline__ void dn_stage(const unsigned char* st, int G, int swz
         const int hi = t * nb + b0 + j;
         const uint4 xe = hpl[2 * hi], xo = hpl[2 * hi + 1];
         const float2 dc = hdc[hi];
-        ay[t] = __fmaf_rn(dc.x, __int2float_rn(isum_of<BITS>(we, wo, xe, xo, __float_as_int(dc.y))), ay[t]);
+        const int iy = isum_of<BITS>(we, wo, xe, xo, __float_as_int(dc.y));
+        if constexpr (DBG) dd[t][b0 + j] = iy;
+        ay[t] = __fmaf_rn(dc.x, __int2float_rn(iy), ay[t]);
       }
     }
   }
 }
 
-template <int TT, int BITS>
+template <int TT, int BITS, bool DBG>
 __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid_constant__ StreamArgs a) {
   constexpr int R = StreamRing<TT>::R;
   extern __shared__ unsigned char smem_raw[];
@@ -219,6 +227,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   __shared__ int s_exp[kMaxSlotsS], s_cnt[kMaxSlotsS], s_base[kMaxSlotsS], s_tok[kMaxSlotsS][TT];
   __shared__ uint32_t s_bits[kMaxExperts / 32];
   __shared__ int s_nslots;
+  __shared__ int s_drow[DBG ? kMaxSlotsS : 1][TT];  // capture row of (slot, position): token * (K + S) + rank
 
   const StreamGeom& g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -338,7 +347,10 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     for (int s = lane; s < S; s += 32) {
       s_exp[s] = E + s;
       s_cnt[s] = T;
-      for (int t = 0; t < TT; ++t) s_tok[s][t] = t;
+      for (int t = 0; t < TT; ++t) {
+        s_tok[s][t] = t;
+        if constexpr (DBG) s_drow[s][t] = t * (K + S) + K + s;
+      }
     }
     __syncwarp();
     // each pair: its slot, and its position = earlier tokens on the same expert
@@ -357,6 +369,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
         ppos[h] = pos;
         atomicAdd(&s_cnt[pslot[h]], 1);
         s_tok[pslot[h]][pos] = t;
+        if constexpr (DBG) s_drow[pslot[h]][pos] = t * (K + S) + (p - t * K);  // rank p - tK of token t
+
       }
     }
     __syncwarp();
@@ -424,12 +438,24 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
 #pragma unroll
     for (int t = 0; t < TT; ++t) tok[t] = t < nv ? s_tok[slot][t] : 0;
     float ag[TT], au[TT];
+    int32_t* dg[TT];
+    int32_t* du[TT];
 #pragma unroll
-    for (int t = 0; t < TT; ++t) ag[t] = au[t] = 0.0f;
+    for (int t = 0; t < TT; ++t) {
+      ag[t] = au[t] = 0.0f;
+      dg[t] = du[t] = nullptr;
+      if constexpr (DBG) {
+        if (t < nv) {
+          const int64_t P = 2 * (int64_t)g.I * g.nbh + (int64_t)g.H * g.nbi;
+          dg[t] = a.dbg + s_drow[slot][t] * P + (int64_t)(chunk * 32 + lane) * g.nbh;
+          du[t] = dg[t] + (int64_t)g.I * g.nbh;
+        }
+      }
+    }
     for (int s = 0; s < g.st_gu; ++s) {
       if (!(ok = wait_stage())) break;
-      gu_stage<TT, BITS>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_gu, g.swz_gu, s * g.g_gu, g.nbh, nv,
-                         tok, xpl, xdc, ag, au);
+      gu_stage<TT, BITS, DBG>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_gu, g.swz_gu, s * g.g_gu, g.nbh,
+                              nv, tok, xpl, xdc, ag, au, dg, du);
       next_stage();
     }
     if (!ok) break;
@@ -508,12 +534,22 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     const uint4* hpl = reinterpret_cast<const uint4*>(hb);
     const float2* hdc = reinterpret_cast<const float2*>(hb + (size_t)TT * g.nbi * 32);
     float ay[TT];
+    int32_t* dd[TT];
 #pragma unroll
-    for (int t = 0; t < TT; ++t) ay[t] = 0.0f;
+    for (int t = 0; t < TT; ++t) {
+      ay[t] = 0.0f;
+      dd[t] = nullptr;
+      if constexpr (DBG) {
+        if (t < nv) {
+          const int64_t P = 2 * (int64_t)g.I * g.nbh + (int64_t)g.H * g.nbi;
+          dd[t] = a.dbg + s_drow[slot][t] * P + 2 * (int64_t)g.I * g.nbh + (int64_t)(chunk * 32 + lane) * g.nbi;
+        }
+      }
+    }
     for (int s = 0; s < g.st_dn; ++s) {
       if (!(ok = wait_stage())) break;
-      dn_stage<TT, BITS>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_dn, g.swz_dn, s * g.g_dn, g.nbi, nv,
-                         hpl, hdc, ay);
+      dn_stage<TT, BITS, DBG>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_dn, g.swz_dn, s * g.g_dn, g.nbi,
+                              nv, hpl, hdc, ay, dd);
       next_stage();
     }
     if (!ok) break;
@@ -595,13 +631,13 @@ __global__ void prepare_expert_kernel(StreamGeom g, const uint8_t* __restrict__ 
     sc[i] = i < g.I ? gs[i] : (i < 2 * g.I ? us[i - g.I] : ds[i - 2 * g.I]);
 }
 
-template <int TT, int BITS>
+template <int TT, int BITS, bool DBG>
 cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
   static int granted[64] = {};
   static int sms[64] = {};
   const size_t smem = stream_smem_bytes<TT>(a.g);
   if (smem > 224 * 1024) return cudaErrorInvalidConfiguration;
-  cudaError_t e = smem_opt_in(expert_stream_kernel<TT, BITS>, (int)smem, granted);
+  cudaError_t e = smem_opt_in(expert_stream_kernel<TT, BITS, DBG>, (int)smem, granted);
   if (e != cudaSuccess) return e;
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -611,7 +647,7 @@ cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
   // units of other CTAs); at least as many CTAs as slots, so that a CTA's
   // range of down units spans at most two slots
   if (sms[dev] < kMaxSlotsS) return cudaErrorInvalidConfiguration;
-  return launch_pdl(expert_stream_kernel<TT, BITS>, dim3(sms[dev]), dim3(kSW * 32), smem, st, true, a);
+  return launch_pdl(expert_stream_kernel<TT, BITS, DBG>, dim3(sms[dev]), dim3(kSW * 32), smem, st, true, a);
 }
 
 }  // namespace
@@ -633,15 +669,17 @@ cudaError_t launch_prepare_expert(int hidden, int inter, int bits, const uint8_t
   return cudaGetLastError();
 }
 
+template <int BITS, bool DBG>
+cudaError_t stream_bits(const StreamArgs& a, cudaStream_t st) {
+  if (a.T <= 1) return stream_tt<1, BITS, DBG>(a, st);
+  if (a.T <= 2) return stream_tt<2, BITS, DBG>(a, st);
+  return stream_tt<4, BITS, DBG>(a, st);
+}
+
 cudaError_t launch_expert_stream(const StreamArgs& a, cudaStream_t st) {
-  if (a.g.bits == 8) {
-    if (a.T <= 1) return stream_tt<1, 8>(a, st);
-    if (a.T <= 2) return stream_tt<2, 8>(a, st);
-    return stream_tt<4, 8>(a, st);
-  }
-  if (a.T <= 1) return stream_tt<1, 4>(a, st);
-  if (a.T <= 2) return stream_tt<2, 4>(a, st);
-  return stream_tt<4, 4>(a, st);
+  // the capture is the same kernel with the partial sums also stored
+  if (a.dbg != nullptr) return a.g.bits == 8 ? stream_bits<8, true>(a, st) : stream_bits<4, true>(a, st);
+  return a.g.bits == 8 ? stream_bits<8, false>(a, st) : stream_bits<4, false>(a, st);
 }
 
 }  // namespace coli

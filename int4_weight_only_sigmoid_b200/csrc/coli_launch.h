@@ -144,6 +144,7 @@ struct StreamArgs {
   int32_t* h_ready;     // [kStreamMaxSlots] gate/up units done per slot (zero at launch)
   int32_t* dn_done;     // [H/32] slots done per 32-row chunk of the output (zero at launch)
   int32_t* status;
+  int32_t* dbg;         // null, or the partials capture (coli_debug_capture_partials layout)
 };
 bool stream_supported(int hidden, int inter, int bits, int n_tok);
 uint64_t stream_expert_bytes(int hidden, int inter, int bits);
@@ -168,7 +169,8 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
                                    const int32_t* n_slots, void* tiles, int32_t* n_tiles, const int32_t* perm,
                                    int K, int n_shared, int bits, const int8_t* xq, const float* xd, int n_tok,
                                    int hidden, int inter, void* xr, int32_t* xm, void* hr, float* hd, int32_t* hm,
-                                   float* y, int32_t* err, cudaStream_t st, cudaEvent_t ev_mid);
+                                   float* y, int32_t* err, cudaStream_t st, cudaEvent_t ev_mid, int32_t* dbg_buf,
+                                   int n_experts);
 
 // out[t] = sum_k w[t,k] y[inv[t,k]] + sum_s y[n_tok*K + s*n_tok + t]  (contract C)
 cudaError_t launch_combine(const float* y, const int32_t* inv, const float* w, int n_tok, int K,

@@ -252,6 +252,13 @@ struct ItemInfo {
   int n0, n_valid, m0;
 };
 
+// The partials capture (coli_debug_capture_partials): buffer, and what maps a
+// slot row to its capture row token * (K + S) + rank (shared s: rank K + s).
+struct DbgArgs {
+  int32_t* buf;
+  int E, S;
+};
+
 // Item i: tile i / nm, column group i % nm (rows [m0, m0 + group_rows) of
 // each output matrix).
 __device__ __forceinline__ ItemInfo item_info(const Slot* slots, const Tile* tiles, int item, int nm, int group_rows) {
@@ -275,12 +282,12 @@ __device__ __forceinline__ int64_t item_token_row(const ItemInfo& f, bool gu, co
 // GU: gate/up (+ SwiGLU + Q8 of h -> hr int8 rows + hd + hm); !GU: down (-> y).
 // ad / am: the A rows' Q8 scales and starting values, [row x nb] (int8
 // weights need no per-block correction: every start value is 0x4B400000).
-template <bool GU, int BITS, typename Tab>
+template <bool GU, int BITS, bool DBG, typename Tab>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     const __grid_constant__ Tab tab, const __grid_constant__ CUtensorMap amap, const Slot* __restrict__ slots,
     const Tile* __restrict__ tiles, const int32_t* __restrict__ n_tiles, const int32_t* __restrict__ perm, int top_k,
     const float* ad, const int32_t* am, int hidden, int inter, int8_t* hr, float* hd, int32_t* hm,
-    float* __restrict__ y, int32_t* __restrict__ err) {
+    float* __restrict__ y, int32_t* __restrict__ err, DbgArgs dbg) {
   using L = PSmem;
   constexpr int kGroupRows = GU ? kN / 2 : kN;  // output rows of one matrix per item
   __shared__ uint64_t full_bar[kStages], empty_bar[kStages], tfull_bar[kTBufs / kHalf], tempty_bar[kTBufs / kHalf],
@@ -531,6 +538,30 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         acc0[j] = 0.0f;
         acc1[j] = 0.0f;
       }
+      // capture: this token's row and the first output row of each column range
+      int32_t* dbg0 = nullptr;
+      int32_t* dbg1 = nullptr;
+      if constexpr (DBG) {
+        if (valid) {
+          const int nbh = hidden / 32, nbi = inter / 32;
+          const int64_t P = 2 * (int64_t)inter * nbh + (int64_t)hidden * nbi;
+          int64_t crow;
+          if (f.slot.perm_base < 0) {
+            crow = (int64_t)(f.n0 + n) * (top_k + dbg.S) + top_k + (f.slot.table_idx - dbg.E);
+          } else {
+            const int pr = perm[f.slot.perm_base + f.n0 + n];
+            crow = (int64_t)(pr / top_k) * (top_k + dbg.S) + pr % top_k;
+          }
+          int32_t* base = dbg.buf + crow * P;
+          if constexpr (GU) {
+            dbg0 = base + (int64_t)(f.m0 + 32 * hh) * nbh;                            // gate rows
+            dbg1 = base + (int64_t)inter * nbh + (int64_t)(f.m0 + 32 * hh) * nbh;     // up rows
+          } else {
+            dbg0 = base + 2 * (int64_t)inter * nbh + (int64_t)(f.m0 + c0) * nbi;
+            dbg1 = base + 2 * (int64_t)inter * nbh + (int64_t)(f.m0 + c1) * nbi;
+          }
+        }
+      }
       for (int j = 0; j < nst; ++j) {
 #pragma unroll
         for (int hs = 0; hs < kHandPerStage; ++hs, ++gh) {
@@ -559,6 +590,15 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
                   float u0 = __uint_as_float(r1[jj]), u1 = __uint_as_float(r1[jj + 1]);
                   sub2(v0, v1, kMagicF);  // exact: (float)isum
                   sub2(u0, u1, kMagicF);
+                  if constexpr (DBG) {
+                    if (valid) {
+                      const int col = 8 * h + jj;
+                      dbg0[(int64_t)col * nb + b] = (int32_t)v0;
+                      dbg0[(int64_t)(col + 1) * nb + b] = (int32_t)v1;
+                      dbg1[(int64_t)col * nb + b] = (int32_t)u0;
+                      dbg1[(int64_t)(col + 1) * nb + b] = (int32_t)u1;
+                    }
+                  }
                   fma2(acc0[8 * h + jj], acc0[8 * h + jj + 1], dx, dx, v0, v1);
                   fma2(acc1[8 * h + jj], acc1[8 * h + jj + 1], dx, dx, u0, u1);
                 }
@@ -719,11 +759,37 @@ cudaError_t make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int co
 
 }  // namespace
 
+namespace {
+
+// The two GEMMs of one weight width; DBG: the capture instantiation.
+template <int BITS, bool DBG>
+cudaError_t prefill_pair(const GateUpTable& gu, const DownTable& dn, const CUtensorMap& map_x,
+                         const CUtensorMap& map_h, const Slot* slots, const Tile* t, const int32_t* n_tiles,
+                         const int32_t* perm, int K, const float* xd, const int32_t* xm, int hidden, int inter,
+                         int8_t* hri, float* hd, int32_t* hm, float* y, int32_t* err, int grid, DbgArgs dbg,
+                         cudaStream_t st, cudaEvent_t ev_mid) {
+  static int mask_gu[64] = {}, mask_dn[64] = {};
+  const size_t smem = PSmem::bytes();
+  cudaError_t e;
+  if ((e = smem_opt_in(prefill_kernel<true, BITS, DBG, GateUpTable>, (int)smem, mask_gu)) != cudaSuccess) return e;
+  if ((e = smem_opt_in(prefill_kernel<false, BITS, DBG, DownTable>, (int)smem, mask_dn)) != cudaSuccess) return e;
+  prefill_kernel<true, BITS, DBG, GateUpTable><<<grid, kThreadsP, smem, st>>>(
+      gu, map_x, slots, t, n_tiles, perm, K, xd, xm, hidden, inter, hri, hd, hm, y, err, dbg);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (ev_mid && (e = cudaEventRecordWithFlags(ev_mid, st, cudaEventRecordExternal)) != cudaSuccess) return e;
+  prefill_kernel<false, BITS, DBG, DownTable><<<grid, kThreadsP, smem, st>>>(
+      dn, map_h, slots, t, n_tiles, perm, K, hd, hm, hidden, inter, hri, hd, hm, y, err, dbg);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, const Slot* slots,
                                    const int32_t* n_slots, void* tiles, int32_t* n_tiles, const int32_t* perm,
                                    int K, int n_shared, int bits, const int8_t* xq, const float* xd, int n_tok,
                                    int hidden, int inter, void* xr, int32_t* xm, void* hr, float* hd, int32_t* hm,
-                                   float* y, int32_t* err, cudaStream_t st, cudaEvent_t ev_mid) {
+                                   float* y, int32_t* err, cudaStream_t st, cudaEvent_t ev_mid, int32_t* dbg_buf,
+                                   int n_experts) {
   Tile* t = reinterpret_cast<Tile*>(tiles);
   const int64_t rows = (int64_t)n_tok * (K + n_shared);
   const int64_t n16 = rows * hidden / 16;
@@ -741,7 +807,6 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
   CUtensorMap map_x, map_h;
   if ((e = make_rows_map(&map_x, xr, rows, hidden)) != cudaSuccess) return e;
   if ((e = make_rows_map(&map_h, hr, rows, inter)) != cudaSuccess) return e;
-  static int mask_gu[64] = {}, mask_dn[64] = {};
   static int sms_cache[64] = {};
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -749,30 +814,18 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
   if (sms_cache[dev] == 0 &&
       (e = cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
-  const size_t smem = PSmem::bytes();
   const int grid = sms_cache[dev];
   int8_t* hri = reinterpret_cast<int8_t*>(hr);
-  if (bits == 8) {
-    static int mask_gu8[64] = {}, mask_dn8[64] = {};
-    if ((e = smem_opt_in(prefill_kernel<true, 8, GateUpTable>, (int)smem, mask_gu8)) != cudaSuccess) return e;
-    if ((e = smem_opt_in(prefill_kernel<false, 8, DownTable>, (int)smem, mask_dn8)) != cudaSuccess) return e;
-    prefill_kernel<true, 8, GateUpTable><<<grid, kThreadsP, smem, st>>>(gu, map_x, slots, t, n_tiles, perm, K, xd,
-                                                                          xm, hidden, inter, hri, hd, hm, y, err);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (ev_mid && (e = cudaEventRecordWithFlags(ev_mid, st, cudaEventRecordExternal)) != cudaSuccess) return e;
-    prefill_kernel<false, 8, DownTable><<<grid, kThreadsP, smem, st>>>(dn, map_h, slots, t, n_tiles, perm, K, hd,
-                                                                         hm, hidden, inter, hri, hd, hm, y, err);
-    return cudaGetLastError();
-  }
-  if ((e = smem_opt_in(prefill_kernel<true, 4, GateUpTable>, (int)smem, mask_gu)) != cudaSuccess) return e;
-  if ((e = smem_opt_in(prefill_kernel<false, 4, DownTable>, (int)smem, mask_dn)) != cudaSuccess) return e;
-  prefill_kernel<true, 4, GateUpTable><<<grid, kThreadsP, smem, st>>>(gu, map_x, slots, t, n_tiles, perm, K, xd, xm,
-                                                                        hidden, inter, hri, hd, hm, y, err);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (ev_mid && (e = cudaEventRecordWithFlags(ev_mid, st, cudaEventRecordExternal)) != cudaSuccess) return e;
-  prefill_kernel<false, 4, DownTable><<<grid, kThreadsP, smem, st>>>(dn, map_h, slots, t, n_tiles, perm, K, hd, hm,
-                                                                       hidden, inter, hri, hd, hm, y, err);
-  return cudaGetLastError();
+  const DbgArgs dbg{dbg_buf, n_experts, n_shared};
+  if (bits == 8)
+    return dbg_buf ? prefill_pair<8, true>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, xm, hidden, inter,
+                                           hri, hd, hm, y, err, grid, dbg, st, ev_mid)
+                   : prefill_pair<8, false>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, xm, hidden, inter,
+                                            hri, hd, hm, y, err, grid, dbg, st, ev_mid);
+  return dbg_buf ? prefill_pair<4, true>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, xm, hidden, inter, hri,
+                                         hd, hm, y, err, grid, dbg, st, ev_mid)
+                 : prefill_pair<4, false>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, xm, hidden, inter, hri,
+                                          hd, hm, y, err, grid, dbg, st, ev_mid);
 }
 
 }  // namespace coli

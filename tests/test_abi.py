@@ -84,6 +84,8 @@ def test_bad_arguments_rejected_before_any_cuda_call(lib):
     assert lib.coli_requantize_fp8_int4(None, None, 4, 64, 12, None, None, None) == m.COLI_EINVAL
     assert b"block" in lib.coli_last_error()
     assert lib.coli_requantize_fp8_int4(None, None, 0, 64, 128, None, None, None) == m.COLI_OK
+    assert lib.coli_debug_capture_partials(None, 100) == m.COLI_EINVAL
+    assert lib.coli_debug_capture_partials(C.c_void_p(8), 100) == m.COLI_EINVAL
     assert lib.coli_debug_wait_probe(None, 1000, None) == m.COLI_EINVAL
     assert lib.coli_debug_wait_probe(C.c_void_p(256), -1, None) == m.COLI_EINVAL
     assert lib.coli_sync_status(C.c_void_p(8), None) == m.COLI_EINVAL  # misaligned workspace
