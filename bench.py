@@ -94,6 +94,8 @@ def parse():
     p.add_argument("--workload", default=None, choices=list(SUITE_WORKLOADS),
                    help="run only this workload of the suite (a profiling entry point) and print its record")
     p.add_argument("--tokens", type=int, default=None, help="with --workload: its token count")
+    p.add_argument("--experts", type=int, default=256,
+                   help="routed experts per layer (256 = GLM-5.2; fewer only for small profiling captures)")
     return p.parse_args()
 
 
@@ -329,7 +331,7 @@ def run_suite(layers, cfg, dev, stream, peak_gbs, only=None, tokens=None):
         if only is not None and name != only:
             continue
         T = tokens or T
-        c = synth.config(name, seed=cfg["seed"])
+        c = synth.config(name, seed=cfg["seed"], n_experts=cfg["n_experts"])
         x = synth.dev_tokens(c, T, device=dev)
         lys = layers
         if c.get("bias_boost_n", 0):
@@ -365,7 +367,7 @@ def run_suite(layers, cfg, dev, stream, peak_gbs, only=None, tokens=None):
         if only is not None and name != only:
             continue
         T = tokens or T
-        c = synth.config("stack8_512" if T > 1 else "stack8", seed=cfg["seed"])
+        c = synth.config("stack8_512" if T > 1 else "stack8", seed=cfg["seed"], n_experts=cfg["n_experts"])
         x = synth.dev_tokens(c, T, device=dev)
         arr = coli.stack_cstructs(layers)
         ws = coli.make_workspace(layers[0].cfg, T, dev)
@@ -438,7 +440,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
     coli.load()
-    cfg = synth.config("decode1", seed=rank)  # each rank: its own replica, its own tokens
+    cfg = synth.config("decode1", seed=rank, n_experts=args.experts)  # each rank: its own replica, its own tokens
     H = cfg["hidden"]
     staging = torch.empty(cfg["inter"] * H, dtype=torch.float32, device=dev)
     n_layers = args.layers

@@ -268,7 +268,7 @@ def dev_bias(cfg: dict, layer: int = 0, device="cuda"):
     import torch
     out = torch.empty(cfg["n_experts"], dtype=torch.float32, device=device)
     dev_uniform(out, cfg["seed"], layer, TID_BIAS, cfg["bias_lo"], cfg["bias_hi"])
-    nb = cfg.get("bias_boost_n", 0)
+    nb = min(cfg.get("bias_boost_n", 0), cfg["n_experts"])
     if nb:
         _check(_dev().synth_dev_add_range(out.data_ptr(), nb, cfg["bias_boost"], _stream()), "add")
     return out
