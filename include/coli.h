@@ -250,7 +250,7 @@ coli_status coli_debug_block_partials(const coli_expert* expert, int32_t which, 
  * scratch need (coli_moe_workspace_bytes(&layer->cfg, n_tok)) exceeds 8 MiB
  * is rejected with COLI_EINVAL and a message naming both sizes -- e.g. the
  * GLM-5.2 shape (hidden 6144, inter 2048, 256 experts, top-8, 1 shared)
- * fits up to 21 tokens per call.  n_tok outside [0, 2^24] is rejected with
+ * fits up to 22 tokens per call.  n_tok outside [0, 2^24] is rejected with
  * COLI_EINVAL before any size is computed.  The first call on each device
  * looks up the array's device address with that device current and keeps
  * it for the life of the process (a device reset invalidates it: do not call

@@ -105,8 +105,8 @@ coli_status check_layer(const coli_moe_layer* L, const char* fn) {
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Workspace {
-  size_t xq, xd, scores, idx, w, counts, offsets, perm, inv, slots, n_slots, status, tiles, n_tiles, hq, hd, xr, xm,
-      hm, hdc, ctr, y, xn, xa, xb, total;
+  size_t xq, xd, scores, idx, w, counts, offsets, perm, inv, slots, n_slots, status, tiles, n_tiles, hq, hd, xr, hdc,
+      ctr, y, xn, xa, xb, total;
 };
 
 Workspace layout(const coli_moe_config& c, int64_t T) {
@@ -139,8 +139,6 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   L.n_tiles = take(4);
   L.hq = take(rows * I);  // h as int8 rows (Q8 of h; the tensor-core path's down operand)
   L.xr = take(tc ? rows * H : 0);
-  L.xm = take(tc ? T * (H / 32) * 4 : 0);
-  L.hm = take(tc ? rows * (I / 32) * 4 : 0);
   L.hd = take(rows * (I / 32) * 4);
   // the streaming decode kernel (prepared layers, <= kStreamMaxTok tokens):
   // (d, c16) of every h block and its counters
@@ -282,8 +280,7 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   CHECK_LAUNCH(mark(0));
   if (prefill_supported(H, I)) {
     CHECK_LAUNCH(launch_prefill_experts(gu, dn, slots, n_slots, at<void>(ws, W.tiles), at<int32_t>(ws, W.n_tiles),
-                                        perm, K, S, bits, xq, xd, (int)T, H, I, at<void>(ws, W.xr),
-                                        at<int32_t>(ws, W.xm), hq, hd, at<int32_t>(ws, W.hm), y,
+                                        perm, K, S, bits, xq, xd, (int)T, H, I, at<void>(ws, W.xr), hq, hd, y,
                                         at<int32_t>(ws, W.status), st, ev[1], capture, E));
   } else {
     if (capture != nullptr)

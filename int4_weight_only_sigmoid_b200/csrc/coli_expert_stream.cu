@@ -50,7 +50,7 @@
 namespace coli {
 namespace {
 
-constexpr int kSW = 4;                               // warps per CTA (all compute; lane 0 also copies)
+constexpr int kSW = 8;                               // warps per CTA (all compute; lane 0 also copies)
 constexpr int kMaxPairsS = kStreamMaxTok * kMaxTopK;  // (token, k) pairs of a batch
 constexpr int kMaxSlotsS = kStreamMaxSlots;          // slots: shared + distinct routed experts
 constexpr int kErrStage = 24;                        // status: gave up waiting for a weight stage
@@ -64,7 +64,7 @@ struct StreamRing {
 
 template <int TT>
 __host__ __device__ inline size_t stream_smem_bytes(const StreamGeom& g) {
-  const size_t ring = (size_t)kSW * StreamRing<TT>::R * kStreamStageMax;
+  const size_t ring = (size_t)kSW * StreamRing<TT>::R * kStreamStageMax;  // 8 KB stages
   const size_t xs = (size_t)TT * g.nbh * 40;        // x planes (32 B) + (d, c16) per block
   const size_t hs = 2 * (size_t)TT * g.nbi * 40;    // two slots' h rows
   return 1024 + ring + xs + hs;
@@ -152,64 +152,31 @@ __device__ __forceinline__ int isum_of(const uint4& a, const uint4& b, const uin
   return blk_isum8(a, b, xe, xo);
 }
 
-// One gate/up stage: blocks b0 .. b0+G-1 of gate row l and up row l (lane
-// l) against the slot's staged tokens.
+// One stage of rows on lanes: blocks b0 .. b0+G-1 of the lane's weight row
+// (gate/up halves: lanes 0-15 gate rows, 16-31 the matching up rows; down:
+// 32 output rows) against the staged activation planes of the tokens tok[t]
+// (row tok[t] of the plane arrays xpl / xdc, nb blocks per row).
 template <int TT, int BITS, bool DBG>
-__device__ __forceinline__ void gu_stage(const unsigned char* st, int G, int swz, int b0, int nb, int nv,
-                                         const int (&tok)[TT], const uint4* xpl, const float2* xdc, float (&ag)[TT],
-                                         float (&au)[TT], int32_t* const (&dg)[TT], int32_t* const (&du)[TT]) {
+__device__ __forceinline__ void rows_stage(const unsigned char* st, int G, int swz, int b0, int nb, int nv,
+                                           const int (&tok)[TT], const uint4* xpl, const float2* xdc,
+                                           float (&acc)[TT], int32_t* const (&dbg)[TT]) {
   const int lane = threadIdx.x & 31;
   constexpr int cpb = BITS / 4;  // 16-byte chunks per block
-  const uint4* rg = reinterpret_cast<const uint4*>(st) + lane * G * cpb;
-  const uint4* ru = reinterpret_cast<const uint4*>(st) + (32 + lane) * G * cpb;
+  const uint4* rw = reinterpret_cast<const uint4*>(st) + lane * G * cpb;
   const int sw = lane & swz;
 #pragma unroll 4
   for (int j = 0; j < G; ++j) {
-    uint4 ge, go, ue, uo;
-    load_blk<BITS>(rg, j, sw, ge, go);
-    load_blk<BITS>(ru, j, sw, ue, uo);
+    uint4 wa, wb;
+    load_blk<BITS>(rw, j, sw, wa, wb);
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
       if (t < nv) {
         const int xi = tok[t] * nb + b0 + j;
         const uint4 xe = xpl[2 * xi], xo = xpl[2 * xi + 1];
         const float2 dc = xdc[xi];
-        const int c16 = __float_as_int(dc.y);
-        const int ig = isum_of<BITS>(ge, go, xe, xo, c16), iu = isum_of<BITS>(ue, uo, xe, xo, c16);
-        if constexpr (DBG) {
-          dg[t][b0 + j] = ig;
-          du[t][b0 + j] = iu;
-        }
-        ag[t] = __fmaf_rn(dc.x, __int2float_rn(ig), ag[t]);
-        au[t] = __fmaf_rn(dc.x, __int2float_rn(iu), au[t]);
-      }
-    }
-  }
-}
-
-// One down stage: blocks b0 .. b0+G-1 of down row l (lane l) against the
-// slot's staged h rows (token t of the slot at index t).
-template <int TT, int BITS, bool DBG>
-__device__ __forceinline__ void dn_stage(const unsigned char* st, int G, int swz, int b0, int nb, int nv,
-                                         const uint4* hpl, const float2* hdc, float (&ay)[TT],
-                                         int32_t* const (&dd)[TT]) {
-  const int lane = threadIdx.x & 31;
-  constexpr int cpb = BITS / 4;
-  const uint4* rw = reinterpret_cast<const uint4*>(st) + lane * G * cpb;
-  const int sw = lane & swz;
-#pragma unroll 4
-  for (int j = 0; j < G; ++j) {
-    uint4 we, wo;
-    load_blk<BITS>(rw, j, sw, we, wo);
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      if (t < nv) {
-        const int hi = t * nb + b0 + j;
-        const uint4 xe = hpl[2 * hi], xo = hpl[2 * hi + 1];
-        const float2 dc = hdc[hi];
-        const int iy = isum_of<BITS>(we, wo, xe, xo, __float_as_int(dc.y));
-        if constexpr (DBG) dd[t][b0 + j] = iy;
-        ay[t] = __fmaf_rn(dc.x, __int2float_rn(iy), ay[t]);
+        const int is = isum_of<BITS>(wa, wb, xe, xo, __float_as_int(dc.y));
+        if constexpr (DBG) dbg[t][b0 + j] = is;
+        acc[t] = __fmaf_rn(dc.x, __int2float_rn(is), acc[t]);
       }
     }
   }
@@ -218,6 +185,7 @@ __device__ __forceinline__ void dn_stage(const unsigned char* st, int G, int swz
 template <int TT, int BITS, bool DBG>
 __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid_constant__ StreamArgs a) {
   constexpr int R = StreamRing<TT>::R;
+  constexpr int kPairs = kSW / 2;
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint64_t full_bar[kSW][R];
   __shared__ uint64_t hbar[2];
@@ -227,6 +195,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   __shared__ int s_exp[kMaxSlotsS], s_cnt[kMaxSlotsS], s_base[kMaxSlotsS], s_tok[kMaxSlotsS][TT];
   __shared__ uint32_t s_bits[kMaxExperts / 32];
   __shared__ int s_nslots;
+  __shared__ float s_h[kPairs][2][TT][32];  // a warp pair's h block, double-buffered by unit
+  __shared__ int s_pair_ok[kPairs][2][2];   // each half's "no wait gave up", double-buffered by unit
   __shared__ int s_drow[DBG ? kMaxSlotsS : 1][TT];  // capture row of (slot, position): token * (K + S) + rank
 
   const StreamGeom& g = a.g;
@@ -251,24 +221,27 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   }
   __syncthreads();
 
-  const int G = gridDim.x, NW = G * kSW, gw = warp * G + blockIdx.x;
+  // Gate/up work goes to warp pairs: pair p of this CTA takes units
+  // gp, gp + NP, ... (gp = p * G + blockIdx.x), warp 2p the first half of
+  // each unit, warp 2p + 1 the second.  Down units: this CTA's contiguous
+  // range [d0, d1), warp w takes d0 + w, d0 + w + kSW, ...
+  const int G = gridDim.x, NP = G * kPairs;
+  const int pair = warp >> 1, half = warp & 1, gp = pair * G + blockIdx.x;
   const int n_shared_gu = S * g.cpu_gu;
 
-  // The warp's stage sequence: its gate/up units gw, gw + NW, ... then its
-  // down units d0 + warp, d0 + warp + kSW, ... (d0 = this CTA's first down
-  // unit).  Flat stage index i -> (unit, stage).  n_gu_mine / n_dn_mine are
-  // known once the routing is; before that only the first unit, if it is a
-  // shared expert's, can stream.
+  // The warp's stage sequence (flat index i -> unit, stage): its gate/up
+  // half units, then its down units.  Before the routing is known only the
+  // first unit, if it is a shared expert's, can stream.
   int n_gu_mine = 0, n_dn_mine = 0, d0 = 0;
   bool routed = false;
   auto stage_src = [&](int i, uint32_t& bytes) -> const unsigned char* {
-    if (!routed || i < n_gu_mine * g.st_gu) {  // before the routing: the warp's first (shared) unit only
+    if (!routed || i < n_gu_mine * g.st_gu) {
       const int k = i / g.st_gu, s = i - k * g.st_gu;
-      const int u = gw + k * NW;
+      const int u = gp + k * NP;
       const int slot = u / g.cpu_gu;
       const int e = slot < S ? E + slot : s_exp[slot];
       bytes = g.sb_gu;
-      return a.prep + (uint64_t)e * g.expert_bytes + (uint64_t)(u - slot * g.cpu_gu) * g.ub_gu +
+      return a.prep + (uint64_t)e * g.expert_bytes + (uint64_t)((u - slot * g.cpu_gu) * 2 + half) * g.ub_gu +
              (uint64_t)s * g.sb_gu;
     }
     const int j = i - n_gu_mine * g.st_gu;
@@ -281,7 +254,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
            (uint64_t)s * g.sb_dn;
   };
   int issued = 0;
-  auto issue = [&](int i) {  // lane 0
+  auto issue = [&](int i) {  // lane 0: one bulk copy of a stage image
     uint32_t bytes;
     const unsigned char* src = stage_src(i, bytes);
     uint64_t* bar = &full_bar[warp][i % R];
@@ -290,7 +263,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   };
 
   // shared experts' first stages stream while the router finishes
-  if (lane == 0 && gw < n_shared_gu)
+  if (lane == 0 && gp < n_shared_gu)
     for (; issued < R && issued < g.st_gu; ++issued) issue(issued);
 
   pdl_wait();  // scores, the Q8_0 of x and the cleared counters are complete
@@ -370,7 +343,6 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
         atomicAdd(&s_cnt[pslot[h]], 1);
         s_tok[pslot[h]][pos] = t;
         if constexpr (DBG) s_drow[pslot[h]][pos] = t * (K + S) + (p - t * K);  // rank p - tK of token t
-
       }
     }
     __syncwarp();
@@ -392,7 +364,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
 
   const int n_slots = s_nslots;
   const int n_gu = n_slots * g.cpu_gu, n_dn = n_slots * g.cpu_dn;
-  n_gu_mine = gw < n_gu ? (n_gu - gw + NW - 1) / NW : 0;
+  n_gu_mine = gp < n_gu ? (n_gu - gp + NP - 1) / NP : 0;
   d0 = (int)((int64_t)blockIdx.x * n_dn / G);
   const int d1 = (int)((int64_t)(blockIdx.x + 1) * n_dn / G);
   n_dn_mine = d0 + warp < d1 ? (d1 - d0 - warp + kSW - 1) / kSW : 0;
@@ -404,11 +376,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   const int slotB = d1 > d0 ? (d1 - 1) / g.cpu_dn : slotA;
   const int ownerB = slotB != slotA ? ((slotB * g.cpu_dn - d0) % kSW) : -1;
 
-  if (lane == 0) {
-    // a first unit streamed before the routing was known may not exist
-    // (n_gu_mine == 0 only if gw >= n_gu, never for a shared unit)
+  if (lane == 0)
     for (; issued < R && issued < total; ++issued) issue(issued);
-  }
   __syncwarp();
 
   int consumed = 0;
@@ -418,69 +387,75 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
                                    kErrStage);
     return __all_sync(0xffffffffu, got);
   };
-  auto next_stage = [&]() {  // this stage's ring slot is free again
+  // The slot's reads of the stage are done (their values are consumed);
+  // the mbarrier orders the next copy into it after them.
+  auto next_stage = [&]() {
     ++consumed;
     __syncwarp();
     if (lane == 0 && !*abort_f && issued < total) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // our reads of the slot before the copy's writes
       issue(issued);
       ++issued;
     }
-    __syncwarp();
   };
+  const int64_t P = 2 * (int64_t)g.I * g.nbh + (int64_t)g.H * g.nbi;  // capture words per (token, expert)
 
-  // ---- gate/up units ----------------------------------------------------
+  // ---- gate/up half units -----------------------------------------------
   for (int k = 0; k < n_gu_mine && ok; ++k) {
-    const int u = gw + k * NW;
+    const int u = gp + k * NP;
     const int slot = u / g.cpu_gu, chunk = u - slot * g.cpu_gu;
     const int nv = s_cnt[slot];
+    const int orow = chunk * 32 + 16 * half + (lane & 15);  // the lane's intermediate output
     int tok[TT];
-#pragma unroll
-    for (int t = 0; t < TT; ++t) tok[t] = t < nv ? s_tok[slot][t] : 0;
-    float ag[TT], au[TT];
-    int32_t* dg[TT];
-    int32_t* du[TT];
+    float acc[TT];
+    int32_t* dbg[TT];
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
-      ag[t] = au[t] = 0.0f;
-      dg[t] = du[t] = nullptr;
-      if constexpr (DBG) {
-        if (t < nv) {
-          const int64_t P = 2 * (int64_t)g.I * g.nbh + (int64_t)g.H * g.nbi;
-          dg[t] = a.dbg + s_drow[slot][t] * P + (int64_t)(chunk * 32 + lane) * g.nbh;
-          du[t] = dg[t] + (int64_t)g.I * g.nbh;
-        }
-      }
+      tok[t] = t < nv ? s_tok[slot][t] : 0;
+      acc[t] = 0.0f;
+      dbg[t] = nullptr;
+      if constexpr (DBG)
+        if (t < nv) dbg[t] = a.dbg + s_drow[slot][t] * P + (int64_t)(lane < 16 ? 0 : g.I) * g.nbh + (int64_t)orow * g.nbh;
     }
     for (int s = 0; s < g.st_gu; ++s) {
       if (!(ok = wait_stage())) break;
-      gu_stage<TT, BITS, DBG>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_gu, g.swz_gu, s * g.g_gu, g.nbh,
-                              nv, tok, xpl, xdc, ag, au, dg, du);
+      rows_stage<TT, BITS, DBG>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_gu, g.swz_gu, s * g.g_gu,
+                                g.nbh, nv, tok, xpl, xdc, acc, dbg);
       next_stage();
     }
-    if (!ok) break;
-    // SwiGLU, the Q8_0 block of h (these 32 outputs are one block), published
+    // the partner half must reach the barrier even if this warp gave up: no early exit before it
     const float* sc = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);
-    const int row = chunk * 32 + lane;
-    const float sg = __ldg(sc + row), su = __ldg(sc + g.I + row);
+    const float sv = __ldg(sc + (lane < 16 ? 0 : g.I) + orow);
+    float* hb = &s_h[pair][k & 1][0][0];
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
-      if (t < nv) {
-        const float gv = __fmul_rn(sg, ag[t]);
-        const float uv = __fmul_rn(su, au[t]);
-        const float h = __fmul_rn(__fmul_rn(gv, sigmoid_cw(gv)), uv);
-        const float d = __fdiv_rn(warp_max(fabsf(h)), 127.0f);
-        const int q = q8_of(h, d);
-        const int64_t hrow = s_base[slot] + t;
-        a.hpl[(hrow * g.nbi + chunk) * 32 + (lane & 1) * 16 + (lane >> 1)] = (int8_t)q;
-        const int se = warp_sum_int((lane & 1) ? 0 : q);
-        if (lane == 0) a.hdc[hrow * g.nbi + chunk] = make_float2(d, __int_as_float(-128 * se));
-      }
+      const float v = __fmul_rn(sv, acc[t]);
+      const float uv = __shfl_down_sync(0xffffffffu, v, 16);
+      if (lane < 16 && t < nv) hb[t * 32 + 16 * half + lane] = __fmul_rn(__fmul_rn(v, sigmoid_cw(v)), uv);
     }
-    __syncwarp();
-    if (lane == 0) {
-      __threadfence();
-      atomicAdd(a.h_ready + slot, 1);
+    if (lane == 0) s_pair_ok[pair][k & 1][half] = (ok && !*abort_f) ? 1 : 0;
+    tc::named_bar(1 + pair, 64);  // both halves of the h block are in shared memory
+    // one decision for both warps of the pair (each meets the barrier of
+    // every unit, so neither may leave the loop alone)
+    ok = s_pair_ok[pair][k & 1][0] && s_pair_ok[pair][k & 1][1];
+    if (half == 0 && ok) {
+      // the Q8_0 block of h (these 32 outputs) for every token, published
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        if (t < nv) {
+          const float h = hb[t * 32 + lane];
+          const float d = __fdiv_rn(warp_max(fabsf(h)), 127.0f);
+          const int q = q8_of(h, d);
+          const int64_t hrow = s_base[slot] + t;
+          a.hpl[(hrow * g.nbi + chunk) * 32 + (lane & 1) * 16 + (lane >> 1)] = (int8_t)q;
+          const int se = warp_sum_int((lane & 1) ? 0 : q);
+          if (lane == 0) a.hdc[hrow * g.nbi + chunk] = make_float2(d, __int_as_float(-128 * se));
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence();
+        atomicAdd(a.h_ready + slot, 1);
+      }
     }
   }
 
@@ -509,7 +484,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
               atomicExch(a.status, kErrHReady);
               break;
             }
-            __nanosleep(256);
+            __nanosleep(128);
           }
         }
         ready = __shfl_sync(0xffffffffu, ready, 0);
@@ -533,32 +508,30 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     }
     const uint4* hpl = reinterpret_cast<const uint4*>(hb);
     const float2* hdc = reinterpret_cast<const float2*>(hb + (size_t)TT * g.nbi * 32);
-    float ay[TT];
-    int32_t* dd[TT];
+    int tok[TT];
+    float acc[TT];
+    int32_t* dbg[TT];
+    const int o = chunk * 32 + lane;
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
-      ay[t] = 0.0f;
-      dd[t] = nullptr;
-      if constexpr (DBG) {
-        if (t < nv) {
-          const int64_t P = 2 * (int64_t)g.I * g.nbh + (int64_t)g.H * g.nbi;
-          dd[t] = a.dbg + s_drow[slot][t] * P + 2 * (int64_t)g.I * g.nbh + (int64_t)(chunk * 32 + lane) * g.nbi;
-        }
-      }
+      tok[t] = t;  // the staged h rows are the slot's tokens in order
+      acc[t] = 0.0f;
+      dbg[t] = nullptr;
+      if constexpr (DBG)
+        if (t < nv) dbg[t] = a.dbg + s_drow[slot][t] * P + 2 * (int64_t)g.I * g.nbh + (int64_t)o * g.nbi;
     }
     for (int s = 0; s < g.st_dn; ++s) {
       if (!(ok = wait_stage())) break;
-      dn_stage<TT, BITS, DBG>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_dn, g.swz_dn, s * g.g_dn, g.nbi,
-                              nv, hpl, hdc, ay, dd);
+      rows_stage<TT, BITS, DBG>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_dn, g.swz_dn, s * g.g_dn,
+                                g.nbi, nv, tok, hpl, hdc, acc, dbg);
       next_stage();
     }
     if (!ok) break;
     const float* sc = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);
-    const int o = chunk * 32 + lane;
     const float sd = __ldg(sc + 2 * g.I + o);
 #pragma unroll
     for (int t = 0; t < TT; ++t)
-      if (t < nv) a.y[((size_t)s_base[slot] + t) * g.H + o] = __fmul_rn(sd, ay[t]);
+      if (t < nv) a.y[((size_t)s_base[slot] + t) * g.H + o] = __fmul_rn(sd, acc[t]);
     __syncwarp();
     int last = 0;
     if (lane == 0) {
@@ -570,11 +543,11 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     if (last) {
       // every slot's y rows of this chunk are written: combine (contract C)
       for (int t = 0; t < T; ++t) {
-        float acc = 0.0f;
+        float accc = 0.0f;
         for (int kk = 0; kk < K; ++kk)
-          acc = __fmaf_rn(s_w[t * K + kk], __ldcg(a.y + (size_t)s_row[t * K + kk] * g.H + o), acc);
-        for (int s = 0; s < S; ++s) acc = __fadd_rn(acc, __ldcg(a.y + ((size_t)s_base[s] + t) * g.H + o));
-        a.out[(size_t)t * g.H + o] = acc;
+          accc = __fmaf_rn(s_w[t * K + kk], __ldcg(a.y + (size_t)s_row[t * K + kk] * g.H + o), accc);
+        for (int s = 0; s < S; ++s) accc = __fadd_rn(accc, __ldcg(a.y + ((size_t)s_base[s] + t) * g.H + o));
+        a.out[(size_t)t * g.H + o] = accc;
       }
     }
   }

@@ -4,24 +4,25 @@
 // reads.
 //
 // The copy is made of "stages": the exact shared-memory image of one step
-// of a warp's work, so that one bulk copy moves a stage from HBM to shared
-// memory with no gather.  A weight block (32 weights) is 16 bytes of packed
-// int4 or 32 bytes of int8; an int8 block is stored as its even elements
-// (16 bytes: 0, 2, .., 30) then its odd elements, so both widths meet the
-// activations as even / odd byte planes.  The 16-byte chunks of a stage row
-// are XOR-rotated: chunk c of stage row r sits in slot c ^ (r & swz) (rows
-// on lanes: lane l reads row l, and the XOR spreads the 8 lanes of each
-// shared-memory phase over 8 bank groups).
-//  - gate/up unit u of an expert (intermediate outputs 32u .. 32u+31):
-//    stages of 64 stage rows x G blocks; stage row r < 32 is gate row
-//    32u + r, r >= 32 is up row 32u + r - 32; block j of stage s is Q8 block
-//    sG + j of the row.  G = min(16, nbh) for int4, min(8, nbh) for int8.
-//  - down unit v (output rows 32v .. 32v+31): stages of 32 rows x G blocks,
-//    G = min(32, nbi) for int4, min(16, nbi) for int8.
+// of a warp's work (32 weight rows x 256 bytes, 8 KB), so that one bulk copy
+// moves a stage from HBM to shared memory with no gather.  A weight block
+// (32 weights) is 16 bytes of packed int4 or 32 bytes of int8; an int8
+// block is stored as its even elements (16 bytes: 0, 2, .., 30) then its odd
+// elements, so both widths meet the activations as even / odd byte planes.
+// The 16-byte chunks of a stage row are XOR-rotated: chunk c of stage row r
+// sits in slot c ^ (r & swz) (rows on lanes: lane l reads row l, and the XOR
+// spreads the 8 lanes of each shared-memory phase over 8 bank groups).
+//  - gate/up unit u of an expert (intermediate outputs 32u .. 32u+31) is
+//    two halves h = 0, 1 (outputs 32u + 16h .. +15); a half's stage row
+//    r < 16 is gate row 32u + 16h + r, r >= 16 the up row of the same
+//    output; block j of stage s is Q8 block sG + j of the row.
+//  - down unit v (output rows 32v .. 32v+31): stage row r is down row 32v + r.
+//  - G = 16 blocks per stage row for int4, 8 for int8 (fewer when a row is
+//    shorter than one stage).
 //  - then the F32 row scales: gate [I], up [I], down [H].
-// Per expert: gate/up units | down units | scales, each expert padded to
-// 256 bytes; expert j (routed 0..E-1, then shared) at j * expert_bytes.
-// Every stage is 16 KB at GLM-5.2 shapes.
+// Per expert: gate/up halves (unit-major) | down units | scales, each expert
+// padded to 256 bytes; expert j (routed 0..E-1, then shared) at
+// j * expert_bytes.
 #pragma once
 
 #include <cstddef>
@@ -29,7 +30,7 @@
 
 namespace coli {
 
-constexpr int kStreamStageMax = 16 * 1024;  // bytes of the largest stage (and of a ring slot)
+constexpr int kStreamStageMax = 8 * 1024;  // bytes of the largest stage (and of a ring slot)
 
 struct StreamGeom {
   int H, I;          // hidden, expert inter
@@ -41,7 +42,7 @@ struct StreamGeom {
   int st_gu, st_dn;  // stages per unit
   int cpu_gu, cpu_dn;  // units per expert (I/32 gate/up, H/32 down)
   uint32_t sb_gu, sb_dn;  // stage bytes
-  uint64_t ub_gu, ub_dn;  // unit bytes
+  uint64_t ub_gu, ub_dn;  // bytes of a gate/up half unit, of a down unit
   uint64_t dn_off, sc_off, expert_bytes;
 };
 
@@ -56,7 +57,7 @@ __host__ __device__ inline bool stream_row_ok(int nb, int gmax, int bpb) {
 __host__ __device__ inline bool stream_shape_ok(int H, int I, int bits) {
   if (H <= 0 || I <= 0 || H % 128 != 0 || I % 128 != 0 || (bits != 4 && bits != 8)) return false;
   const int bpb = bits == 8 ? 32 : 16;
-  return stream_row_ok(H / 32, 256 / bpb, bpb) && stream_row_ok(I / 32, 512 / bpb, bpb);
+  return stream_row_ok(H / 32, 256 / bpb, bpb) && stream_row_ok(I / 32, 256 / bpb, bpb);
 }
 
 __host__ __device__ inline StreamGeom stream_geom(int H, int I, int bits) {
@@ -67,9 +68,9 @@ __host__ __device__ inline StreamGeom stream_geom(int H, int I, int bits) {
   g.bpb = bits == 8 ? 32 : 16;
   g.nbh = H / 32;
   g.nbi = I / 32;
-  const int gmax_gu = 256 / g.bpb, gmax_dn = 512 / g.bpb;
-  g.g_gu = g.nbh < gmax_gu ? g.nbh : gmax_gu;
-  g.g_dn = g.nbi < gmax_dn ? g.nbi : gmax_dn;
+  const int gmax = 256 / g.bpb;  // blocks in a 256-byte stage row
+  g.g_gu = g.nbh < gmax ? g.nbh : gmax;
+  g.g_dn = g.nbi < gmax ? g.nbi : gmax;
   const int ch_gu = g.g_gu * g.bpb / 16, ch_dn = g.g_dn * g.bpb / 16;  // 16-byte chunks per stage row
   g.swz_gu = (ch_gu < 8 ? ch_gu : 8) - 1;
   g.swz_dn = (ch_dn < 8 ? ch_dn : 8) - 1;
@@ -77,11 +78,11 @@ __host__ __device__ inline StreamGeom stream_geom(int H, int I, int bits) {
   g.st_dn = g.nbi / g.g_dn;
   g.cpu_gu = I / 32;
   g.cpu_dn = H / 32;
-  g.sb_gu = (uint32_t)(64 * g.g_gu * g.bpb);
+  g.sb_gu = (uint32_t)(32 * g.g_gu * g.bpb);
   g.sb_dn = (uint32_t)(32 * g.g_dn * g.bpb);
-  g.ub_gu = (uint64_t)g.st_gu * g.sb_gu;
+  g.ub_gu = (uint64_t)g.st_gu * g.sb_gu;  // one half of a gate/up unit
   g.ub_dn = (uint64_t)g.st_dn * g.sb_dn;
-  g.dn_off = (uint64_t)g.cpu_gu * g.ub_gu;
+  g.dn_off = (uint64_t)g.cpu_gu * 2 * g.ub_gu;
   g.sc_off = g.dn_off + (uint64_t)g.cpu_dn * g.ub_dn;
   g.expert_bytes = (g.sc_off + (uint64_t)(2 * I + H) * 4 + 255) & ~uint64_t(255);
   return g;
@@ -93,10 +94,10 @@ __host__ __device__ inline StreamGeom stream_geom(int H, int I, int bits) {
 __host__ __device__ inline uint64_t stream_chunk_offset(const StreamGeom& g, int m, int r, int b, int h) {
   const int cpb = g.bpb / 16;  // chunks per block
   if (m < 2) {
-    const int u = r / 32, sr = (m == 0 ? 0 : 32) + (r & 31);
+    const int u = r / 32, half = (r / 16) & 1, sr = (m == 0 ? 0 : 16) + (r & 15);
     const int s = b / g.g_gu, j = b - s * g.g_gu;
     const int c = j * cpb + h;
-    return (uint64_t)u * g.ub_gu + (uint64_t)s * g.sb_gu + (uint64_t)sr * g.g_gu * g.bpb +
+    return (uint64_t)(u * 2 + half) * g.ub_gu + (uint64_t)s * g.sb_gu + (uint64_t)sr * g.g_gu * g.bpb +
            (uint64_t)((c ^ (sr & g.swz_gu)) * 16);
   }
   const int v = r / 32, sr = r & 31;

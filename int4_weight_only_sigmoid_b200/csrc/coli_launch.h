@@ -155,12 +155,11 @@ cudaError_t launch_expert_stream(const StreamArgs& a, cudaStream_t st);
 
 // Prefill expert kernels on the tensor cores (tcgen05.mma.kind::i8): the
 // int8 operand rows of the Q8 activations, one per (slot, token) in slot
-// order (xr: n_tok*(K+n_shared) x hidden bytes, per 8 elements in the order
-// 0,2,4,6,1,3,5,7) and the accumulator starting value of every (token, block)
-// (xm: n_tok x hidden/32 int32), the tile list (<= 128 tokens of one slot per
-// tile) built from the slot table, then the persistent gate/up GEMM (+ SwiGLU
-// + Q8 of h, written as int8 rows hr: rows x inter, scales hd, starting values
-// hm: rows x inter/32) and the persistent down GEMM (-> y).
+// order (xr: n_tok*(K+n_shared) x hidden bytes; with int4 weights per 8
+// elements in the order 0,2,4,6,1,3,5,7), the tile list (<= 128 tokens of
+// one slot per tile) built from the slot table, then the persistent gate/up
+// GEMM (+ SwiGLU + Q8 of h, written as int8 rows hr: rows x inter, scales hd)
+// and the persistent down GEMM (-> y).
 // `tiles` needs prefill_tile_bytes().
 bool prefill_supported(int hidden, int inter);
 size_t prefill_tiles_bound(int n_tok, int K, int E, int n_shared);
@@ -168,9 +167,8 @@ size_t prefill_tile_bytes(int n_tok, int K, int E, int n_shared);
 cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, const Slot* slots,
                                    const int32_t* n_slots, void* tiles, int32_t* n_tiles, const int32_t* perm,
                                    int K, int n_shared, int bits, const int8_t* xq, const float* xd, int n_tok,
-                                   int hidden, int inter, void* xr, int32_t* xm, void* hr, float* hd, int32_t* hm,
-                                   float* y, int32_t* err, cudaStream_t st, cudaEvent_t ev_mid, int32_t* dbg_buf,
-                                   int n_experts);
+                                   int hidden, int inter, void* xr, void* hr, float* hd, float* y, int32_t* err,
+                                   cudaStream_t st, cudaEvent_t ev_mid, int32_t* dbg_buf, int n_experts);
 
 // out[t] = sum_k w[t,k] y[inv[t,k]] + sum_s y[n_tok*K + s*n_tok + t]  (contract C)
 cudaError_t launch_combine(const float* y, const int32_t* inv, const float* w, int n_tok, int K,

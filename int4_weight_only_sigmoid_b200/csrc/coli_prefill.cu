@@ -118,11 +118,12 @@ __device__ __forceinline__ uint32_t pk_off(int r, int c) {
 // K chunks of an 8-row group 128 B apart (LBO), groups 256 B apart (SBO).
 __device__ __forceinline__ uint32_t op_off(int r, int c) { return (r >> 3) * 256 + c * 128 + (r & 7) * 16; }
 
-// q + 8 of the 8 nibbles of a packed word, as unsigned bytes in the order
-// 0,2,4,6 (lo) then 1,3,5,7 (hi).
+// 16 q of the 8 nibbles of a packed word, as signed bytes in the order
+// 0,2,4,6 (lo) then 1,3,5,7 (hi): each nibble moved to the high half of its
+// byte.
 __device__ __forceinline__ void expand_word(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
-  hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+  lo = (w << 4) & 0xF0F0F0F0u;
+  hi = w & 0xF0F0F0F0u;
 }
 
 // Operand rows of the Q8 activations in row order: row r < n_tok*K is
@@ -150,25 +151,6 @@ __global__ void __launch_bounds__(256) act_rows_i8_kernel(const int8_t* __restri
     split_even_odd(v.z, v.w, o.z, o.w);
     out[i] = o;
   }
-}
-
-// Starting accumulator value of every (token, block): 0x4B400000 - 8 * sum
-// of the block's 32 values.  One thread per block.
-__global__ void __launch_bounds__(256) act_magic_kernel(const int8_t* __restrict__ q, int64_t n_blocks,
-                                                        int32_t* __restrict__ mag) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n_blocks) return;
-  const uint4* p = reinterpret_cast<const uint4*>(q + 32 * i);
-  const uint4 a = __ldg(p), b = __ldg(p + 1);
-  int s = __dp4a((int)a.x, 0x01010101, 0);
-  s = __dp4a((int)a.y, 0x01010101, s);
-  s = __dp4a((int)a.z, 0x01010101, s);
-  s = __dp4a((int)a.w, 0x01010101, s);
-  s = __dp4a((int)b.x, 0x01010101, s);
-  s = __dp4a((int)b.y, 0x01010101, s);
-  s = __dp4a((int)b.z, 0x01010101, s);
-  s = __dp4a((int)b.w, 0x01010101, s);
-  mag[i] = (int32_t)(kMagic - (uint32_t)(8 * s));
 }
 
 // 2D tiled bulk-tensor load (TMA) of box (x, y) into shared memory,
@@ -199,13 +181,13 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor of kind::i8: signed A (activations), B unsigned
-// (int4 weights + 8) or signed (int8 weights), int32 accumulator, shape
-// M x N, both K-major.
-__host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N, bool b_signed) {
+// Instruction descriptor of kind::i8: signed A (activations) and B
+// (weights: 16 q for int4, q for int8), int32 accumulator, shape M x N,
+// both K-major.
+__host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N) {
   return (2u << 4)                       // D format: S32
          | (1u << 7)                     // A format: S8
-         | ((b_signed ? 1u : 0u) << 10)  // B format: U8 / S8
+         | (1u << 10)                    // B format: S8
          | ((uint32_t)(N >> 3) << 17)    // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
@@ -239,11 +221,13 @@ __device__ __forceinline__ void fma2(float& a0, float& a1, float d0, float d1, f
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(dd), "l"(xx));
   asm("mov.b64 {%0,%1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
 }
-__device__ __forceinline__ void sub2(float& x0, float& x1, float c) {
-  unsigned long long xx, cc;
+// x = fma(x, a, c) on two F32 lanes with the same a and c.
+__device__ __forceinline__ void fma2c(float& x0, float& x1, float a, float c) {
+  unsigned long long xx, aa, cc;
   asm("mov.b64 %0, {%1,%2};" : "=l"(xx) : "f"(x0), "f"(x1));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(aa) : "f"(a));
   asm("mov.b64 %0, {%1,%1};" : "=l"(cc) : "f"(c));
-  asm("sub.rn.f32x2 %0, %0, %1;" : "+l"(xx) : "l"(cc));
+  asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(xx) : "l"(aa), "l"(cc));
   asm("mov.b64 {%0,%1}, %2;" : "=f"(x0), "=f"(x1) : "l"(xx));
 }
 
@@ -279,15 +263,14 @@ __device__ __forceinline__ int64_t item_token_row(const ItemInfo& f, bool gu, co
   return f.slot.perm_base < 0 ? (int64_t)(f.n0 + n) : (int64_t)(perm[f.slot.perm_base + f.n0 + n] / top_k);
 }
 
-// GU: gate/up (+ SwiGLU + Q8 of h -> hr int8 rows + hd + hm); !GU: down (-> y).
-// ad / am: the A rows' Q8 scales and starting values, [row x nb] (int8
-// weights need no per-block correction: every start value is 0x4B400000).
+// GU: gate/up (+ SwiGLU + Q8 of h -> hr int8 rows + hd); !GU: down (-> y).
+// ad: the A rows' Q8 scales, [row x nb].
 template <bool GU, int BITS, bool DBG, typename Tab>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     const __grid_constant__ Tab tab, const __grid_constant__ CUtensorMap amap, const Slot* __restrict__ slots,
     const Tile* __restrict__ tiles, const int32_t* __restrict__ n_tiles, const int32_t* __restrict__ perm, int top_k,
-    const float* ad, const int32_t* am, int hidden, int inter, int8_t* hr, float* hd, int32_t* hm,
-    float* __restrict__ y, int32_t* __restrict__ err, DbgArgs dbg) {
+    const float* ad, int hidden, int inter, int8_t* hr, float* hd, float* __restrict__ y, int32_t* __restrict__ err,
+    DbgArgs dbg) {
   using L = PSmem;
   constexpr int kGroupRows = GU ? kN / 2 : kN;  // output rows of one matrix per item
   __shared__ uint64_t full_bar[kStages], empty_bar[kStages], tfull_bar[kTBufs / kHalf], tempty_bar[kTBufs / kHalf],
@@ -416,7 +399,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     if (lane == 0) {
       int gs = 0, gh = 0;
       bool ok = true;
-      constexpr uint32_t idesc = idesc_i8_s32(kM, kN, BITS == 8);
+      constexpr uint32_t idesc = idesc_i8_s32(kM, kN);
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
         for (int j = 0; j < nst && ok; ++j, ++gs) {
           const int s = gs % kStages;
@@ -492,25 +475,22 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const int n = quad * 32 + lane;  // this thread's token within the tile
     constexpr int kHandPerStage = kBS / kHalf;
-    // starting value of this thread's lane for block b of item `it` (0 if
-    // the lane holds no token there: that lane's result is never read)
-    auto start_value = [&](int it, int b) -> uint32_t {
-      if (BITS == 8 || it >= n_items) return kMagic;
-      const ItemInfo f = item_info(slots, tiles, it, nm, kGroupRows);
-      if (n >= f.n_valid) return kMagic;
-      return (uint32_t)__ldg(am + item_token_row(f, GU, perm, top_k, n) * nb + b);
-    };
-    auto write_start = [&](int buf, uint32_t v) {
+    // isum from an accumulator read as binary32: int4 (B = 16 q): the value
+    // is 0x4B400000 + 16 isum, so fma(v, 1/16, -C/16) = isum exactly (the
+    // exact result is an integer below 2^22); int8 (B = q): v - C.
+    constexpr float kIsumScale = BITS == 4 ? 0.0625f : 1.0f;
+    constexpr float kIsumOffset = -kMagicF * kIsumScale;
+    auto write_start = [&](int buf) {  // every accumulator starts at 0x4B400000
       const uint32_t col = tmem + lane_base + buf * kN;
-      tmem_st16_same(col + c0, v);
-      tmem_st16_same(col + c0 + 16, v);
-      tmem_st16_same(col + c1, v);
-      tmem_st16_same(col + c1 + 16, v);
+      tmem_st16_same(col + c0, kMagic);
+      tmem_st16_same(col + c0 + 16, kMagic);
+      tmem_st16_same(col + c1, kMagic);
+      tmem_st16_same(col + c1 + 16, kMagic);
     };
-    // first use of every buffer: blocks 0..3 of the CTA's first item
+    // first use of every buffer
     if ((int)blockIdx.x < n_items) {
 #pragma unroll
-      for (int b = 0; b < kTBufs; ++b) write_start(b, start_value(blockIdx.x, b));
+      for (int b = 0; b < kTBufs; ++b) write_start(b);
       tmem_st_wait();
       fence_before_sync();
       __syncwarp();
@@ -519,19 +499,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     }
     int gh = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
-      const bool active = quad * 32 < f.n_valid;  // warp-uniform
-      const bool valid = n < f.n_valid;
-      const int64_t trow = valid ? item_token_row(f, GU, perm, top_k, n) : 0;
-      const float* drow = ad + trow * nb;
-      const int32_t* mrow = am + trow * nb;
-      // the next item's starting values for its first stage (this thread's lane)
-      const int nxt = item + gridDim.x;
-      int64_t nrow = -1;
-      if (nxt < n_items) {
-        const ItemInfo fn = item_info(slots, tiles, nxt, nm, kGroupRows);
-        if (n < fn.n_valid) nrow = item_token_row(fn, GU, perm, top_k, n);
-      }
+      bool active, valid;
+      const float2* drow;
       float acc0[32], acc1[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
@@ -541,6 +510,11 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       // capture: this token's row and the first output row of each column range
       int32_t* dbg0 = nullptr;
       int32_t* dbg1 = nullptr;
+      {  // the item's description is read again for the epilogue: fewer live registers in the block loop
+        const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
+        active = quad * 32 < f.n_valid;  // warp-uniform
+        valid = n < f.n_valid;
+        drow = reinterpret_cast<const float2*>(ad + (valid ? item_token_row(f, GU, perm, top_k, n) : 0) * nb);
       if constexpr (DBG) {
         if (valid) {
           const int nbh = hidden / 32, nbi = inter / 32;
@@ -562,9 +536,15 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           }
         }
       }
+      }
+      // the token's Q8 scales of a hand-off (kHalf = 2 blocks), one hand-off ahead
+      float2 dnext = valid ? __ldg(drow) : make_float2(0.f, 0.f);
       for (int j = 0; j < nst; ++j) {
 #pragma unroll
         for (int hs = 0; hs < kHandPerStage; ++hs, ++gh) {
+          const float2 dcur = dnext;
+          const int hn = j * kHandPerStage + hs + 1;  // next hand-off of this item
+          if (valid && hn < nst * kHandPerStage) dnext = __ldg(drow + hn);
           const int hb = gh % (kTBufs / kHalf);
           // warp-uniform: tcgen05.ld is a warp-wide instruction
           const bool ok =
@@ -575,7 +555,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
             const int b = j * kBS + hs * kHalf + i;  // block of this item
             const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
             if (active && ok) {
-              const float dx = valid ? __ldg(drow + b) : 0.0f;
+              const float dx = i == 0 ? dcur.x : dcur.y;
               // 8 columns of each range at a time (one wait per pair of
               // loads), so that only 16 TMEM values are live
 #pragma unroll
@@ -588,15 +568,15 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
                 for (int jj = 0; jj < 8; jj += 2) {
                   float v0 = __uint_as_float(r0[jj]), v1 = __uint_as_float(r0[jj + 1]);
                   float u0 = __uint_as_float(r1[jj]), u1 = __uint_as_float(r1[jj + 1]);
-                  sub2(v0, v1, kMagicF);  // exact: (float)isum
-                  sub2(u0, u1, kMagicF);
+                  fma2c(v0, v1, kIsumScale, kIsumOffset);  // exact: (float)isum
+                  fma2c(u0, u1, kIsumScale, kIsumOffset);
                   if constexpr (DBG) {
                     if (valid) {
-                      const int col = 8 * h + jj;
-                      dbg0[(int64_t)col * nb + b] = (int32_t)v0;
-                      dbg0[(int64_t)(col + 1) * nb + b] = (int32_t)v1;
-                      dbg1[(int64_t)col * nb + b] = (int32_t)u0;
-                      dbg1[(int64_t)(col + 1) * nb + b] = (int32_t)u1;
+                      const int colw = 8 * h + jj;
+                      dbg0[(int64_t)colw * nb + b] = (int32_t)v0;
+                      dbg0[(int64_t)(colw + 1) * nb + b] = (int32_t)v1;
+                      dbg1[(int64_t)colw * nb + b] = (int32_t)u0;
+                      dbg1[(int64_t)(colw + 1) * nb + b] = (int32_t)u1;
                     }
                   }
                   fma2(acc0[8 * h + jj], acc0[8 * h + jj + 1], dx, dx, v0, v1);
@@ -604,17 +584,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
                 }
               }
             }
-            // the buffer's next use: block b + kBS of this item, else block
-            // b + kBS - nb of the next item
-            uint32_t v = kMagic;
-            if constexpr (BITS == 4) {
-              if (b + kBS < nb) {
-                if (valid) v = (uint32_t)__ldg(mrow + b + kBS);
-              } else if (nrow >= 0) {
-                v = (uint32_t)__ldg(am + nrow * nb + (b + kBS - nb));
-              }
-            }
-            write_start(hb * kHalf + i, v);
+            write_start(hb * kHalf + i);  // the buffer's next use starts at 0x4B400000 again
           }
           tmem_st_wait();
           fence_before_sync();
@@ -624,6 +594,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       }
       const bool go = __all_sync(0xffffffffu, !*abort) && active;  // warp-uniform
       if (go && valid) {
+        const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
         const int64_t row = (int64_t)f.slot.row_base + f.n0 + n;
         if constexpr (GU) {
           const int o = f.m0 + 32 * hh;  // first intermediate row of this thread's Q8 block of h
@@ -639,16 +610,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           }
           const float d = __fdiv_rn(amax, 127.0f);
           // q in the operand order (int4 weights: per 8 elements 0,2,4,6,1,3,5,7;
-          // int8: the elements' order) and the block sum
+          // int8: the elements' order)
           uint32_t pk[8];
-          int sum = 0;
 #pragma unroll
           for (int e8 = 0; e8 < 4; ++e8) {
             uint32_t lo = 0, hi = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int qe = q8_of(acc0[8 * e8 + 2 * i], d), qo = q8_of(acc0[8 * e8 + 2 * i + 1], d);
-              sum += qe + qo;
               lo |= ((uint32_t)qe & 0xFFu) << (8 * i);
               hi |= ((uint32_t)qo & 0xFFu) << (8 * i);
             }
@@ -664,7 +633,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           hd[row * (inter / 32) + (o >> 5)] = d;
-          hm[row * (inter / 32) + (o >> 5)] = (int32_t)(kMagic - (uint32_t)(8 * sum));
         } else {
           const float* sdp = tab.down_s[f.slot.table_idx] + f.m0;
           float4* dst0 = reinterpret_cast<float4*>(y + row * hidden + f.m0 + c0);
@@ -765,20 +733,19 @@ namespace {
 template <int BITS, bool DBG>
 cudaError_t prefill_pair(const GateUpTable& gu, const DownTable& dn, const CUtensorMap& map_x,
                          const CUtensorMap& map_h, const Slot* slots, const Tile* t, const int32_t* n_tiles,
-                         const int32_t* perm, int K, const float* xd, const int32_t* xm, int hidden, int inter,
-                         int8_t* hri, float* hd, int32_t* hm, float* y, int32_t* err, int grid, DbgArgs dbg,
-                         cudaStream_t st, cudaEvent_t ev_mid) {
+                         const int32_t* perm, int K, const float* xd, int hidden, int inter, int8_t* hri, float* hd,
+                         float* y, int32_t* err, int grid, DbgArgs dbg, cudaStream_t st, cudaEvent_t ev_mid) {
   static int mask_gu[64] = {}, mask_dn[64] = {};
   const size_t smem = PSmem::bytes();
   cudaError_t e;
   if ((e = smem_opt_in(prefill_kernel<true, BITS, DBG, GateUpTable>, (int)smem, mask_gu)) != cudaSuccess) return e;
   if ((e = smem_opt_in(prefill_kernel<false, BITS, DBG, DownTable>, (int)smem, mask_dn)) != cudaSuccess) return e;
   prefill_kernel<true, BITS, DBG, GateUpTable><<<grid, kThreadsP, smem, st>>>(
-      gu, map_x, slots, t, n_tiles, perm, K, xd, xm, hidden, inter, hri, hd, hm, y, err, dbg);
+      gu, map_x, slots, t, n_tiles, perm, K, xd, hidden, inter, hri, hd, y, err, dbg);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecordWithFlags(ev_mid, st, cudaEventRecordExternal)) != cudaSuccess) return e;
   prefill_kernel<false, BITS, DBG, DownTable><<<grid, kThreadsP, smem, st>>>(
-      dn, map_h, slots, t, n_tiles, perm, K, hd, hm, hidden, inter, hri, hd, hm, y, err, dbg);
+      dn, map_h, slots, t, n_tiles, perm, K, hd, hidden, inter, hri, hd, y, err, dbg);
   return cudaGetLastError();
 }
 
@@ -787,9 +754,8 @@ cudaError_t prefill_pair(const GateUpTable& gu, const DownTable& dn, const CUten
 cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, const Slot* slots,
                                    const int32_t* n_slots, void* tiles, int32_t* n_tiles, const int32_t* perm,
                                    int K, int n_shared, int bits, const int8_t* xq, const float* xd, int n_tok,
-                                   int hidden, int inter, void* xr, int32_t* xm, void* hr, float* hd, int32_t* hm,
-                                   float* y, int32_t* err, cudaStream_t st, cudaEvent_t ev_mid, int32_t* dbg_buf,
-                                   int n_experts) {
+                                   int hidden, int inter, void* xr, void* hr, float* hd, float* y, int32_t* err,
+                                   cudaStream_t st, cudaEvent_t ev_mid, int32_t* dbg_buf, int n_experts) {
   Tile* t = reinterpret_cast<Tile*>(tiles);
   const int64_t rows = (int64_t)n_tok * (K + n_shared);
   const int64_t n16 = rows * hidden / 16;
@@ -799,8 +765,6 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
   else
     act_rows_i8_kernel<4><<<(unsigned)((n16 + 255) / 256), 256, 0, st>>>(xq, perm, n_tok, K, rows, hidden,
                                                                          reinterpret_cast<uint4*>(xr));
-  const int64_t nblk = (int64_t)n_tok * (hidden / 32);
-  if (bits == 4) act_magic_kernel<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(xq, nblk, xm);
   build_tiles_kernel<<<1, 32, 0, st>>>(slots, n_slots, t, n_tiles);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -818,14 +782,14 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
   int8_t* hri = reinterpret_cast<int8_t*>(hr);
   const DbgArgs dbg{dbg_buf, n_experts, n_shared};
   if (bits == 8)
-    return dbg_buf ? prefill_pair<8, true>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, xm, hidden, inter,
-                                           hri, hd, hm, y, err, grid, dbg, st, ev_mid)
-                   : prefill_pair<8, false>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, xm, hidden, inter,
-                                            hri, hd, hm, y, err, grid, dbg, st, ev_mid);
-  return dbg_buf ? prefill_pair<4, true>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, xm, hidden, inter, hri,
-                                         hd, hm, y, err, grid, dbg, st, ev_mid)
-                 : prefill_pair<4, false>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, xm, hidden, inter, hri,
-                                          hd, hm, y, err, grid, dbg, st, ev_mid);
+    return dbg_buf ? prefill_pair<8, true>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, hidden, inter, hri,
+                                           hd, y, err, grid, dbg, st, ev_mid)
+                   : prefill_pair<8, false>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, hidden, inter, hri,
+                                            hd, y, err, grid, dbg, st, ev_mid);
+  return dbg_buf ? prefill_pair<4, true>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, hidden, inter, hri, hd,
+                                         y, err, grid, dbg, st, ev_mid)
+                 : prefill_pair<4, false>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, hidden, inter, hri, hd,
+                                          y, err, grid, dbg, st, ev_mid);
 }
 
 }  // namespace coli

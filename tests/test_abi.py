@@ -51,13 +51,13 @@ def test_workspace_holds_prefill_buffers_only_for_that_path(lib):
     """Calls of <= 16 tokens take the decode path and need no int8 operand
     rows of x; above that the tensor-core path keeps one int8 row of x per
     (slot, token) and the accumulator starting values.  The documented
-    no-allocation limit (8 MiB of scratch) is 21 GLM tokens."""
+    no-allocation limit (8 MiB of scratch) is 22 GLM tokens."""
     import int4_weight_only_sigmoid_b200 as m
     cfg = m.make_config(6144, 2048, 256, 8, 1)
     b16, b17 = (m.workspace_bytes(cfg, t) for t in (16, 17))
     rows17 = 17 * (8 + 1)
     assert b17 - b16 >= rows17 * 6144
-    assert m.workspace_bytes(cfg, 21) <= 8 << 20 < m.workspace_bytes(cfg, 22)
+    assert m.workspace_bytes(cfg, 22) <= 8 << 20 < m.workspace_bytes(cfg, 23)
 
 
 def test_bad_arguments_rejected_before_any_cuda_call(lib):

@@ -25,47 +25,63 @@ def _layer(cfg):
     return _cache[key]
 
 
-def _layout_offset(H, I, m, r, b):
-    """Byte offset of block b of row r of matrix m (0 gate, 1 up, 2 down) in
-    one expert's streaming copy, as include/coli.h documents it."""
-    nbh, nbi = H // 32, I // 32
+def _geom(H, I, bits):
+    bpb = 16 if bits == 4 else 32
+    gmax = 256 // bpb
+    g_gu, g_dn = min(gmax, H // 32), min(gmax, I // 32)
+    st_gu, st_dn = (H // 32) // g_gu, (I // 32) // g_dn
+    stage_gu, stage_dn = 32 * g_gu * bpb, 32 * g_dn * bpb
+    gu_bytes = (I // 32) * 2 * st_gu * stage_gu
+    dn_bytes = (H // 32) * st_dn * stage_dn
+    return bpb, g_gu, g_dn, st_gu, st_dn, stage_gu, stage_dn, gu_bytes, dn_bytes
+
+
+def _layout_offset(H, I, m, r, b, bits=4, h=0):
+    """Byte offset of 16-byte chunk h of block b of row r of matrix m (0 gate,
+    1 up, 2 down) in one expert's streaming copy, as include/coli.h and the
+    layout header document it."""
+    bpb, g_gu, g_dn, st_gu, st_dn, stage_gu, stage_dn, gu_bytes, _ = _geom(H, I, bits)
+    cpb = bpb // 16
     if m < 2:
-        G = min(16, nbh)
-        swz = min(G, 8) - 1
-        st_bytes = 64 * G * 16
-        unit_bytes = (nbh // G) * st_bytes
-        sr = (0 if m == 0 else 32) + r % 32
-        s, j = divmod(b, G)
-        return (r // 32) * unit_bytes + s * st_bytes + sr * G * 16 + ((j ^ (sr & swz)) * 16)
-    G = min(32, nbi)
-    swz = min(G, 8) - 1
-    st_bytes = 32 * G * 16
-    unit_bytes = (nbi // G) * st_bytes
-    dn_off = (I // 32) * (nbh // min(16, nbh)) * 64 * min(16, nbh) * 16
+        swz = min(g_gu * cpb, 8) - 1
+        u, half = r // 32, (r // 16) % 2
+        sr = (0 if m == 0 else 16) + r % 16
+        s, j = divmod(b, g_gu)
+        c = j * cpb + h
+        return ((u * 2 + half) * st_gu + s) * stage_gu + sr * g_gu * bpb + ((c ^ (sr & swz)) * 16)
+    swz = min(g_dn * cpb, 8) - 1
     sr = r % 32
-    s, j = divmod(b, G)
-    return dn_off + (r // 32) * unit_bytes + s * st_bytes + sr * G * 16 + ((j ^ (sr & swz)) * 16)
+    s, j = divmod(b, g_dn)
+    c = j * cpb + h
+    return gu_bytes + ((r // 32) * st_dn + s) * stage_dn + sr * g_dn * bpb + ((c ^ (sr & swz)) * 16)
 
 
-def test_prepare_writes_the_documented_layout(coli, syn):
-    cfg = syn.config("tiny")
+@pytest.mark.parametrize("bits", [4, 8])
+def test_prepare_writes_the_documented_layout(coli, syn, bits):
+    cfg = syn.config("tiny", weight_bits=bits)
     H, I, E, S = cfg["hidden"], cfg["inter"], cfg["n_experts"], cfg["n_shared"]
     L = _layer(cfg)
     prep = _np(L.prepared)
     eb = len(prep) // (E + S)
     assert eb * (E + S) == len(prep) and eb % 256 == 0
+    _, _, _, _, _, _, _, gu_bytes, dn_bytes = _geom(H, I, bits)
     for j, ex in enumerate(L.experts + L.shared):
         base = j * eb
-        mats = [_np(ex.gate_q), _np(ex.up_q), _np(ex.down_q)]
+        mats = [_np(ex.gate_q).view(np.uint8), _np(ex.up_q).view(np.uint8), _np(ex.down_q).view(np.uint8)]
         for m, q in enumerate(mats):
-            rows, nb = q.shape[0], q.shape[1] // 16
+            bpb = 16 if bits == 4 else 32
+            rows, nb = q.shape[0], q.shape[1] // bpb
             for r in range(rows):
                 for b in range(nb):
-                    o = base + _layout_offset(H, I, m, r, b)
-                    assert np.array_equal(prep[o:o + 16], q[r, 16 * b:16 * b + 16]), (j, m, r, b)
-        nbh, nbi = H // 32, I // 32
-        gu_bytes = (I // 32) * (nbh // min(16, nbh)) * 64 * min(16, nbh) * 16
-        dn_bytes = (H // 32) * (nbi // min(32, nbi)) * 32 * min(32, nbi) * 16
+                    blk = q[r, bpb * b:bpb * (b + 1)]
+                    if bits == 4:
+                        o = base + _layout_offset(H, I, m, r, b)
+                        assert np.array_equal(prep[o:o + 16], blk), (j, m, r, b)
+                    else:  # even elements, then odd elements
+                        o0 = base + _layout_offset(H, I, m, r, b, 8, 0)
+                        o1 = base + _layout_offset(H, I, m, r, b, 8, 1)
+                        assert np.array_equal(prep[o0:o0 + 16], blk[0::2]), (j, m, r, b)
+                        assert np.array_equal(prep[o1:o1 + 16], blk[1::2]), (j, m, r, b)
         sc = prep[base + gu_bytes + dn_bytes:base + gu_bytes + dn_bytes + (2 * I + H) * 4].view(np.float32)
         assert bits_equal(sc[:I], _np(ex.gate_s)) and bits_equal(sc[I:2 * I], _np(ex.up_s))
         assert bits_equal(sc[2 * I:], _np(ex.down_s))

@@ -23,7 +23,7 @@ def _close(got, want, rel=2e-3):
 
 @pytest.mark.parametrize("name,n_tok,prep", [("tiny", 8, False), ("tiny", 3, False), ("tiny", 40, False),
                                              ("decode1", 1, False), ("decode16", 16, False),
-                                             ("decode16", 21, False),  # the tensor-core path, the documented limit
+                                             ("decode16", 22, False),  # the tensor-core path, the documented limit
                                              ("decode4", 4, True)])     # the streaming path of a prepared layer
 def test_noalloc_matches_workspace_forward_twice(coli, syn, name, n_tok, prep):
     import torch
