@@ -53,7 +53,6 @@ namespace {
 constexpr int kSW = 8;                               // warps per CTA (all compute; lane 0 also copies)
 constexpr int kMaxPairsS = kStreamMaxTok * kMaxTopK;  // (token, k) pairs of a batch
 constexpr int kMaxSlotsS = kStreamMaxSlots;          // slots: shared + distinct routed experts
-constexpr int kErrStage = 24;                        // status: gave up waiting for a weight stage
 constexpr int kErrHReady = 25;                       // status: gave up waiting for a slot's h
 constexpr int kErrHStaged = 26;                      // status: gave up waiting for staged h
 
@@ -187,7 +186,6 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   constexpr int R = StreamRing<TT>::R;
   constexpr int kPairs = kSW / 2;
   extern __shared__ unsigned char smem_raw[];
-  __shared__ uint64_t full_bar[kSW][R];
   __shared__ uint64_t hbar[2];
   __shared__ int abort_s;
   __shared__ int s_idx[kMaxPairsS], s_row[kMaxPairsS];
@@ -212,8 +210,6 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
 
   for (int i = threadIdx.x; i < kMaxExperts / 32; i += blockDim.x) s_bits[i] = 0u;
   if (threadIdx.x == 0) {
-    for (int w = 0; w < kSW; ++w)
-      for (int r = 0; r < R; ++r) tc::mbar_init(&full_bar[w][r], 1);
     tc::mbar_init(&hbar[0], 32);
     tc::mbar_init(&hbar[1], 32);
     abort_s = 0;
@@ -229,42 +225,69 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   const int pair = warp >> 1, half = warp & 1, gp = pair * G + blockIdx.x;
   const int n_shared_gu = S * g.cpu_gu;
 
-  // The warp's stage sequence (flat index i -> unit, stage): its gate/up
-  // half units, then its down units.  Before the routing is known only the
-  // first unit, if it is a shared expert's, can stream.
+  // The warp's stage sequence: its gate/up half units, then its down units.
+  // A cursor walks it R stages ahead of the compute: (phase, unit index k,
+  // stage s, the unit's base address); the divisions happen once per unit.
+  // Before the routing is known only the first unit, if it is a shared
+  // expert's, can stream.
   int n_gu_mine = 0, n_dn_mine = 0, d0 = 0;
-  bool routed = false;
-  auto stage_src = [&](int i, uint32_t& bytes) -> const unsigned char* {
-    if (!routed || i < n_gu_mine * g.st_gu) {
-      const int k = i / g.st_gu, s = i - k * g.st_gu;
-      const int u = gp + k * NP;
+  struct Cursor {
+    int phase, k, s;  // phase 0 gate/up, 1 down, 2 done
+    const unsigned char* base;
+  };
+  auto unit_base = [&](Cursor& c) {
+    if (c.phase == 0 && c.k >= n_gu_mine) {
+      c.phase = 1;
+      c.k = 0;
+    }
+    if (c.phase == 1 && c.k >= n_dn_mine) c.phase = 2;
+    if (c.phase == 0) {
+      const int u = gp + c.k * NP;
       const int slot = u / g.cpu_gu;
       const int e = slot < S ? E + slot : s_exp[slot];
-      bytes = g.sb_gu;
-      return a.prep + (uint64_t)e * g.expert_bytes + (uint64_t)((u - slot * g.cpu_gu) * 2 + half) * g.ub_gu +
-             (uint64_t)s * g.sb_gu;
+      c.base = a.prep + (uint64_t)e * g.expert_bytes + (uint64_t)((u - slot * g.cpu_gu) * 2 + half) * g.ub_gu;
+    } else if (c.phase == 1) {
+      const int v = d0 + warp + c.k * kSW;
+      const int slot = v / g.cpu_dn;
+      const int e = slot < S ? E + slot : s_exp[slot];
+      c.base = a.prep + (uint64_t)e * g.expert_bytes + g.dn_off + (uint64_t)(v - slot * g.cpu_dn) * g.ub_dn;
     }
-    const int j = i - n_gu_mine * g.st_gu;
-    const int k = j / g.st_dn, s = j - k * g.st_dn;
-    const int v = d0 + warp + k * kSW;
-    const int slot = v / g.cpu_dn;
-    const int e = slot < S ? E + slot : s_exp[slot];
-    bytes = g.sb_dn;
-    return a.prep + (uint64_t)e * g.expert_bytes + g.dn_off + (uint64_t)(v - slot * g.cpu_dn) * g.ub_dn +
-           (uint64_t)s * g.sb_dn;
   };
+  Cursor pc{0, 0, 0, nullptr};
   int issued = 0;
-  auto issue = [&](int i) {  // lane 0: one bulk copy of a stage image
-    uint32_t bytes;
-    const unsigned char* src = stage_src(i, bytes);
-    uint64_t* bar = &full_bar[warp][i % R];
-    stream::mbar_expect_tx(bar, bytes);
-    stream::bulk_g2s(ring + (size_t)(i % R) * kStreamStageMax, src, bytes, bar);
+  // all lanes: the cursor's stage into ring slot issued % R with cp.async
+  // (lane l copies 16-byte chunks l, l + 32, ...: each instruction moves 512
+  // contiguous bytes), one commit group per stage (empty past the end)
+  auto copy_stage = [&]() {
+    if (pc.phase < 2) {
+      const uint32_t bytes = pc.phase == 0 ? g.sb_gu : g.sb_dn;
+      const unsigned char* src = pc.base + (uint64_t)pc.s * bytes;
+      unsigned char* dst = ring + (size_t)(issued % R) * kStreamStageMax;
+      for (uint32_t off = 16 * lane; off < bytes; off += 512) cp_async16(dst + off, src + off);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    ++issued;
+  };
+  auto issue = [&]() {  // copy, then move the cursor on
+    copy_stage();
+    if (pc.phase < 2 && ++pc.s == (pc.phase == 0 ? g.st_gu : g.st_dn)) {
+      pc.s = 0;
+      ++pc.k;
+      unit_base(pc);
+    }
   };
 
-  // shared experts' first stages stream while the router finishes
-  if (lane == 0 && gp < n_shared_gu)
-    for (; issued < R && issued < g.st_gu; ++issued) issue(issued);
+  // shared experts' first stages stream while the router finishes (within
+  // the warp's first unit: what follows depends on the routing)
+  int pre = 0;
+  if (gp < n_shared_gu) {
+    n_gu_mine = 1;  // provisional: the first unit
+    unit_base(pc);
+    for (; pre < R && pre < g.st_gu; ++pre) {
+      copy_stage();
+      ++pc.s;
+    }
+  }
 
   pdl_wait();  // scores, the Q8_0 of x and the cleared counters are complete
   pdl_launch_dependents();
@@ -368,34 +391,34 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   d0 = (int)((int64_t)blockIdx.x * n_dn / G);
   const int d1 = (int)((int64_t)(blockIdx.x + 1) * n_dn / G);
   n_dn_mine = d0 + warp < d1 ? (d1 - d0 - warp + kSW - 1) / kSW : 0;
-  const int total = n_gu_mine * g.st_gu + n_dn_mine * g.st_dn;
-  routed = true;
   // the down slots of this CTA's range (at most two: a range never spans
   // more, since there are at least as many CTAs as slots)
   const int slotA = d0 / g.cpu_dn;
   const int slotB = d1 > d0 ? (d1 - 1) / g.cpu_dn : slotA;
   const int ownerB = slotB != slotA ? ((slotB * g.cpu_dn - d0) % kSW) : -1;
 
-  if (lane == 0)
-    for (; issued < R && issued < total; ++issued) issue(issued);
-  __syncwarp();
+  if (pre == 0) {
+    unit_base(pc);  // the cursor's first unit, now that the counts are known
+  } else if (pc.s == g.st_gu) {
+    pc.s = 0;  // the first unit was streamed whole before the routing: on to the next
+    pc.k = 1;
+    unit_base(pc);
+  }
+  for (int i = pre; i < R; ++i) issue();
 
   int consumed = 0;
   bool ok = true;
-  auto wait_stage = [&]() -> bool {
-    const bool got = tc::mbar_wait(&full_bar[warp][consumed % R], (uint32_t)((consumed / R) & 1), abort_f, a.status,
-                                   kErrStage);
-    return __all_sync(0xffffffffu, got);
+  // this lane's copies of the oldest stage are in (R - 1 newer groups may
+  // still be in flight), then every lane's
+  auto wait_stage = [&]() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(R - 1) : "memory");
+    __syncwarp();
   };
-  // The slot's reads of the stage are done (their values are consumed);
-  // the mbarrier orders the next copy into it after them.
+  // the ring slot of the stage just computed is free again: copy the stage R ahead into it
   auto next_stage = [&]() {
     ++consumed;
     __syncwarp();
-    if (lane == 0 && !*abort_f && issued < total) {
-      issue(issued);
-      ++issued;
-    }
+    issue();
   };
   const int64_t P = 2 * (int64_t)g.I * g.nbh + (int64_t)g.H * g.nbi;  // capture words per (token, expert)
 
@@ -417,7 +440,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
         if (t < nv) dbg[t] = a.dbg + s_drow[slot][t] * P + (int64_t)(lane < 16 ? 0 : g.I) * g.nbh + (int64_t)orow * g.nbh;
     }
     for (int s = 0; s < g.st_gu; ++s) {
-      if (!(ok = wait_stage())) break;
+      wait_stage();
       rows_stage<TT, BITS, DBG>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_gu, g.swz_gu, s * g.g_gu,
                                 g.nbh, nv, tok, xpl, xdc, acc, dbg);
       next_stage();
@@ -521,12 +544,11 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
         if (t < nv) dbg[t] = a.dbg + s_drow[slot][t] * P + 2 * (int64_t)g.I * g.nbh + (int64_t)o * g.nbi;
     }
     for (int s = 0; s < g.st_dn; ++s) {
-      if (!(ok = wait_stage())) break;
+      wait_stage();
       rows_stage<TT, BITS, DBG>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_dn, g.swz_dn, s * g.g_dn,
                                 g.nbi, nv, tok, hpl, hdc, acc, dbg);
       next_stage();
     }
-    if (!ok) break;
     const float* sc = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);
     const float sd = __ldg(sc + 2 * g.I + o);
 #pragma unroll
@@ -552,9 +574,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     }
   }
 
-  // copies still in flight (only after an abort): wait for them, bounded
-  if (lane == 0)
-    for (int i = consumed; i < issued; ++i) stream::mbar_drain(&full_bar[warp][i % R], (uint32_t)((i / R) & 1));
+  // copies still in flight (after an abort, the stages never computed)
+  asm volatile("cp.async.wait_all;" ::: "memory");
   // an owner that gave up before arriving leaves hbar incomplete: waiters give up too (bounded)
 }
 
