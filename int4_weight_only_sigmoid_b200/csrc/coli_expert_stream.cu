@@ -133,18 +133,6 @@ __device__ __forceinline__ int blk_isum8(const uint4& we, const uint4& wo, const
   return A + B;
 }
 
-// One weight block of a stage row: the two operand halves for blk_isum
-// (int4: q + 8 of the even elements, 16 q of the odd ones) or blk_isum8.
-template <int BITS>
-__device__ __forceinline__ void load_blk(const uint4* row, int j, int sw, uint4& a, uint4& b) {
-  if constexpr (BITS == 4) {
-    unpack_blk(row[j ^ sw], a, b);
-  } else {
-    a = row[(2 * j) ^ sw];
-    b = row[(2 * j + 1) ^ sw];
-  }
-}
-
 template <int BITS>
 __device__ __forceinline__ int isum_of(const uint4& a, const uint4& b, const uint4& xe, const uint4& xo, int c16) {
   if constexpr (BITS == 4) return blk_isum(a, b, xe, xo, c16);
@@ -154,31 +142,63 @@ __device__ __forceinline__ int isum_of(const uint4& a, const uint4& b, const uin
 // One stage of rows on lanes: blocks b0 .. b0+G-1 of the lane's weight row
 // (gate/up halves: lanes 0-15 gate rows, 16-31 the matching up rows; down:
 // 32 output rows) against the staged activation planes of the tokens tok[t]
-// (row tok[t] of the plane arrays xpl / xdc, nb blocks per row).
-template <int TT, int BITS, bool DBG>
-__device__ __forceinline__ void rows_stage(const unsigned char* st, int G, int swz, int b0, int nb, int nv,
+// (row tok[t] of the plane arrays xpl / xdc, nb blocks per row).  G is a
+// compile-time stage width, so the block loop is straight-line code: the
+// row's chunk c sits at (row base | rotation) ^ (c << 4) (the row is aligned
+// to its length) and every activation load has an immediate offset.
+template <int TT, int BITS, bool DBG, int G>
+__device__ __forceinline__ void rows_stage(const unsigned char* st, int swz, int b0, int nb, int nv,
                                            const int (&tok)[TT], const uint4* xpl, const float2* xdc,
                                            float (&acc)[TT], int32_t* const (&dbg)[TT]) {
   const int lane = threadIdx.x & 31;
-  constexpr int cpb = BITS / 4;  // 16-byte chunks per block
-  const uint4* rw = reinterpret_cast<const uint4*>(st) + lane * G * cpb;
-  const int sw = lane & swz;
-#pragma unroll 4
+  constexpr int cpb = BITS / 4;             // 16-byte chunks per block
+  constexpr int kRowBytes = G * cpb * 16;
+  const uintptr_t rb = reinterpret_cast<uintptr_t>(st + lane * kRowBytes) | (uintptr_t)((lane & swz) << 4);
+  const uint4* xp[TT];
+  const float2* xd[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    xp[t] = xpl + 2 * (tok[t] * nb + b0);
+    xd[t] = xdc + tok[t] * nb + b0;
+  }
+#pragma unroll
   for (int j = 0; j < G; ++j) {
     uint4 wa, wb;
-    load_blk<BITS>(rw, j, sw, wa, wb);
+    if constexpr (BITS == 4) {
+      unpack_blk(*reinterpret_cast<const uint4*>(rb ^ (uintptr_t)(j << 4)), wa, wb);
+    } else {
+      wa = *reinterpret_cast<const uint4*>(rb ^ (uintptr_t)((2 * j) << 4));
+      wb = *reinterpret_cast<const uint4*>(rb ^ (uintptr_t)((2 * j + 1) << 4));
+    }
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
-      if (t < nv) {
-        const int xi = tok[t] * nb + b0 + j;
-        const uint4 xe = xpl[2 * xi], xo = xpl[2 * xi + 1];
-        const float2 dc = xdc[xi];
+      if (TT == 1 || t < nv) {
+        const uint4 xe = xp[t][2 * j], xo = xp[t][2 * j + 1];
+        const float2 dc = xd[t][j];
         const int is = isum_of<BITS>(wa, wb, xe, xo, __float_as_int(dc.y));
         if constexpr (DBG) dbg[t][b0 + j] = is;
         acc[t] = __fmaf_rn(dc.x, __int2float_rn(is), acc[t]);
       }
     }
   }
+}
+
+// A stage of runtime width G (a power of two, 1 .. 16 blocks) through the
+// compile-time instances.
+template <int TT, int BITS, bool DBG>
+__device__ __forceinline__ void rows_stage_any(int G, const unsigned char* st, int swz, int b0, int nb, int nv,
+                                               const int (&tok)[TT], const uint4* xpl, const float2* xdc,
+                                               float (&acc)[TT], int32_t* const (&dbg)[TT]) {
+  if (G == 16)
+    rows_stage<TT, BITS, DBG, 16>(st, swz, b0, nb, nv, tok, xpl, xdc, acc, dbg);
+  else if (G == 8)
+    rows_stage<TT, BITS, DBG, 8>(st, swz, b0, nb, nv, tok, xpl, xdc, acc, dbg);
+  else if (G == 4)
+    rows_stage<TT, BITS, DBG, 4>(st, swz, b0, nb, nv, tok, xpl, xdc, acc, dbg);
+  else if (G == 2)
+    rows_stage<TT, BITS, DBG, 2>(st, swz, b0, nb, nv, tok, xpl, xdc, acc, dbg);
+  else
+    rows_stage<TT, BITS, DBG, 1>(st, swz, b0, nb, nv, tok, xpl, xdc, acc, dbg);
 }
 
 template <int TT, int BITS, bool DBG>
@@ -441,8 +461,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     }
     for (int s = 0; s < g.st_gu; ++s) {
       wait_stage();
-      rows_stage<TT, BITS, DBG>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_gu, g.swz_gu, s * g.g_gu,
-                                g.nbh, nv, tok, xpl, xdc, acc, dbg);
+      rows_stage_any<TT, BITS, DBG>(g.g_gu, ring + (size_t)(consumed % R) * kStreamStageMax, g.swz_gu, s * g.g_gu,
+                                    g.nbh, nv, tok, xpl, xdc, acc, dbg);
       next_stage();
     }
     // the partner half must reach the barrier even if this warp gave up: no early exit before it
@@ -545,8 +565,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     }
     for (int s = 0; s < g.st_dn; ++s) {
       wait_stage();
-      rows_stage<TT, BITS, DBG>(ring + (size_t)(consumed % R) * kStreamStageMax, g.g_dn, g.swz_dn, s * g.g_dn,
-                                g.nbi, nv, tok, hpl, hdc, acc, dbg);
+      rows_stage_any<TT, BITS, DBG>(g.g_dn, ring + (size_t)(consumed % R) * kStreamStageMax, g.swz_dn, s * g.g_dn,
+                                    g.nbi, nv, tok, hpl, hdc, acc, dbg);
       next_stage();
     }
     const float* sc = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);

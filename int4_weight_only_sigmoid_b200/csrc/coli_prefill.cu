@@ -36,10 +36,13 @@
 // conversion.  The fold then applies contract F per block, so prefill equals
 // the dp4a paths bit for bit.
 //
-// Roles (448 threads): warps 0-3 producers (packed-weight copies; thread p
-// expands weight row p), warp 4 the A-tile TMA loads, warps 5-12 the fold
-// (warp w reads TMEM lanes 32(w%4).. = 32 of the tile's tokens, and half of
-// the item's columns), warp 13 the MMA issuer (lane 0) and TMEM owner.
+// Roles (704 threads): warps 0-3 producers (packed-weight copies; thread p
+// expands weight row p), warp 4 the A-tile TMA loads, warps 5-20 the fold
+// (warp w reads TMEM lanes 32(w%4).. = 32 of the tile's tokens, and a
+// quarter of the item's columns: gate/up 16 gate rows and the same 16 up
+// rows, down 32 rows), warp 21 the MMA issuer (lane 0) and TMEM owner.  The
+// two fold warps that hold one Q8 block of h (32 intermediate rows) meet at
+// a named barrier to share the block's absmax.
 // An operand stage holds 4 Q8 blocks (K = 128).  Per stage g: the TMA warp
 // loads its A tile into operand stage g % kStages once `empty` (the MMA's
 // commit) says the stage is free; the producers copy its packed weights
@@ -75,14 +78,14 @@ constexpr int kPkSlots = kLookS + 2;  // packed-weight slots: a slot is rewritte
 constexpr int kHalf = 2;       // Q8 blocks per accumulator hand-off (MMA -> fold)
 constexpr int kTBufs = 4;      // TMEM accumulators (one per block), handed off in pairs
 constexpr int kProdWarps = 4;
-constexpr int kEpiWarps = 8;   // 2 per TMEM lane quadrant, each half of the columns
+constexpr int kEpiWarps = 16;  // 4 per TMEM lane quadrant, each a quarter of the columns
 // Warp w runs on scheduler w % 4 and, as a fold warp, reads TMEM lanes
 // 32 (w % 4)..; the MMA issuer is kept off scheduler 0, which carries the
 // fold of tiles with at most 32 tokens.
 constexpr int kTmaWarp = kProdWarps;                           // A-tile loads
 constexpr int kEpi0 = kProdWarps + 1;                          // first fold warp
 constexpr int kMmaWarp = kEpi0 + kEpiWarps;                    // MMA issuer, TMEM owner
-constexpr int kThreadsP = 32 * (kMmaWarp + 1);                 // 448
+constexpr int kThreadsP = 32 * (kMmaWarp + 1);                 // 704
 constexpr int kNProd = 32 * kProdWarps;                        // 128 producer threads
 constexpr int kTmemCols = kTBufs * kN;                         // 512
 constexpr uint32_t kMagic = 0x4B400000u;                       // binary32 1.5 * 2^23
@@ -277,6 +280,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       done_bar;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
+  __shared__ float s_amax[2][kEpiWarps][32];  // gate/up fold: half-block absmax per (warp, token), by item parity
   extern __shared__ unsigned char smem_raw[];
 
   const int dim_in = GU ? hidden : inter;
@@ -466,12 +470,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     __syncwarp();
   } else {
     // ------------------------------------------------------------ fold
-    // warp w: TMEM lanes 32*(w%4).. (tokens); columns c0.. and c1.. (32 each):
-    // gate/up: the gate rows [32 hh, 32 hh + 32) of the group and the same
-    // up rows (64 columns on); down: columns [64 hh, 64 hh + 64)
-    const int quad = warp & 3, hh = (warp - kEpi0) >> 2;
-    const int c0 = GU ? 32 * hh : 64 * hh;
-    const int c1 = GU ? kGroupRows + 32 * hh : 64 * hh + 32;
+    // warp w: TMEM lanes 32*(w%4).. (tokens); columns c0.. and c1.. (16 each):
+    // gate/up: gate rows [16 c4, 16 c4 + 16) of the group and the same up
+    // rows (64 columns on); down: columns [32 c4, 32 c4 + 32)
+    const int quad = warp & 3, c4 = (warp - kEpi0) >> 2;
+    const int c0 = GU ? 16 * c4 : 32 * c4;
+    const int c1 = GU ? kGroupRows + 16 * c4 : 32 * c4 + 16;
+    int n_done = 0;  // items this warp has folded (parity of the absmax exchange buffer)
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const int n = quad * 32 + lane;  // this thread's token within the tile
     constexpr int kHandPerStage = kBS / kHalf;
@@ -483,9 +488,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     auto write_start = [&](int buf) {  // every accumulator starts at 0x4B400000
       const uint32_t col = tmem + lane_base + buf * kN;
       tmem_st16_same(col + c0, kMagic);
-      tmem_st16_same(col + c0 + 16, kMagic);
       tmem_st16_same(col + c1, kMagic);
-      tmem_st16_same(col + c1 + 16, kMagic);
     };
     // first use of every buffer
     if ((int)blockIdx.x < n_items) {
@@ -501,9 +504,9 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       bool active, valid;
       const float2* drow;
-      float acc0[32], acc1[32];
+      float acc0[16], acc1[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
+      for (int j = 0; j < 16; ++j) {
         acc0[j] = 0.0f;
         acc1[j] = 0.0f;
       }
@@ -528,8 +531,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           }
           int32_t* base = dbg.buf + crow * P;
           if constexpr (GU) {
-            dbg0 = base + (int64_t)(f.m0 + 32 * hh) * nbh;                            // gate rows
-            dbg1 = base + (int64_t)inter * nbh + (int64_t)(f.m0 + 32 * hh) * nbh;     // up rows
+            dbg0 = base + (int64_t)(f.m0 + c0) * nbh;                            // gate rows
+            dbg1 = base + (int64_t)inter * nbh + (int64_t)(f.m0 + c0) * nbh;     // up rows
           } else {
             dbg0 = base + 2 * (int64_t)inter * nbh + (int64_t)(f.m0 + c0) * nbi;
             dbg1 = base + 2 * (int64_t)inter * nbh + (int64_t)(f.m0 + c1) * nbi;
@@ -559,7 +562,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
               // 8 columns of each range at a time (one wait per pair of
               // loads), so that only 16 TMEM values are live
 #pragma unroll
-              for (int h = 0; h < 4; ++h) {
+              for (int h = 0; h < 2; ++h) {
                 uint32_t r0[8], r1[8];
                 tmem_ld8(col + c0 + 8 * h, r0);
                 tmem_ld8(col + c1 + 8 * h, r1);
@@ -592,53 +595,58 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           if (lane == 0) mbar_arrive(&tempty_bar[hb]);  // the pair of TMEM buffers may be rewritten now
         }
       }
-      const bool go = __all_sync(0xffffffffu, !*abort) && active;  // warp-uniform
-      if (go && valid) {
+      if (active) {  // warp-uniform, and the same for both warps of a pair (one quadrant)
+        const bool go = !*abort;  // this warp's writes only: both warps meet the barrier regardless
         const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
         const int64_t row = (int64_t)f.slot.row_base + f.n0 + n;
         if constexpr (GU) {
-          const int o = f.m0 + 32 * hh;  // first intermediate row of this thread's Q8 block of h
+          const int o = f.m0 + c0;  // this thread's 16 intermediate rows (half of a Q8 block of h)
           const float* sgp = tab.gate_s[f.slot.table_idx] + o;
           const float* sup = tab.up_s[f.slot.table_idx] + o;
           float amax = 0.0f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const float gv = __fmul_rn(__ldg(sgp + j), acc0[j]);
             const float u = __fmul_rn(__ldg(sup + j), acc1[j]);
             acc0[j] = __fmul_rn(__fmul_rn(gv, sigmoid_cw(gv)), u);
             amax = fmaxf(amax, fabsf(acc0[j]));
           }
+          // the block's absmax: this half's and the partner warp's (c4 ^ 1)
+          float* xa = &s_amax[n_done & 1][0][0];
+          xa[(warp - kEpi0) * 32 + lane] = valid ? amax : 0.0f;
+          named_bar(2 + quad * 2 + (c4 >> 1), 64);
+          amax = fmaxf(amax, xa[(warp - kEpi0 + 4 * ((c4 ^ 1) - c4)) * 32 + lane]);
           const float d = __fdiv_rn(amax, 127.0f);
-          // q in the operand order (int4 weights: per 8 elements 0,2,4,6,1,3,5,7;
-          // int8: the elements' order)
-          uint32_t pk[8];
+          if (go && valid) {
+            // q in the operand order (int4 weights: per 8 elements 0,2,4,6,1,3,5,7;
+            // int8: the elements' order)
+            uint32_t pk[4];
 #pragma unroll
-          for (int e8 = 0; e8 < 4; ++e8) {
-            uint32_t lo = 0, hi = 0;
+            for (int e8 = 0; e8 < 2; ++e8) {
+              uint32_t lo = 0, hi = 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int qe = q8_of(acc0[8 * e8 + 2 * i], d), qo = q8_of(acc0[8 * e8 + 2 * i + 1], d);
-              lo |= ((uint32_t)qe & 0xFFu) << (8 * i);
-              hi |= ((uint32_t)qo & 0xFFu) << (8 * i);
+              for (int i = 0; i < 4; ++i) {
+                const int qe = q8_of(acc0[8 * e8 + 2 * i], d), qo = q8_of(acc0[8 * e8 + 2 * i + 1], d);
+                lo |= ((uint32_t)qe & 0xFFu) << (8 * i);
+                hi |= ((uint32_t)qo & 0xFFu) << (8 * i);
+              }
+              if constexpr (BITS == 4) {
+                pk[2 * e8] = lo;
+                pk[2 * e8 + 1] = hi;
+              } else {  // back to element order: even / odd bytes interleaved
+                pk[2 * e8] = __byte_perm(lo, hi, 0x5140);
+                pk[2 * e8 + 1] = __byte_perm(lo, hi, 0x7362);
+              }
             }
-            if constexpr (BITS == 4) {
-              pk[2 * e8] = lo;
-              pk[2 * e8 + 1] = hi;
-            } else {  // back to element order: even / odd bytes interleaved
-              pk[2 * e8] = __byte_perm(lo, hi, 0x5140);
-              pk[2 * e8 + 1] = __byte_perm(lo, hi, 0x7362);
-            }
+            *reinterpret_cast<uint4*>(hr + row * inter + o) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            if ((c4 & 1) == 0) hd[row * (inter / 32) + (o >> 5)] = d;
           }
-          uint4* dst = reinterpret_cast<uint4*>(hr + row * inter + o);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          hd[row * (inter / 32) + (o >> 5)] = d;
-        } else {
+        } else if (go && valid) {
           const float* sdp = tab.down_s[f.slot.table_idx] + f.m0;
           float4* dst0 = reinterpret_cast<float4*>(y + row * hidden + f.m0 + c0);
           float4* dst1 = reinterpret_cast<float4*>(y + row * hidden + f.m0 + c1);
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
+          for (int j = 0; j < 16; j += 4) {
             const float4 s0 = __ldg(reinterpret_cast<const float4*>(sdp + c0 + j));
             const float4 s1 = __ldg(reinterpret_cast<const float4*>(sdp + c1 + j));
             dst0[j / 4] = make_float4(__fmul_rn(s0.x, acc0[j]), __fmul_rn(s0.y, acc0[j + 1]),
@@ -648,6 +656,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           }
         }
       }
+      ++n_done;
     }
   }
   fence_before_sync();
