@@ -367,9 +367,9 @@ const char* status_meaning(int32_t code) {
     case 13: return "prefill fold gave up waiting for accumulators";
     case 16: return "prefill A-tile loader gave up waiting for an operand stage";
     case 22: return "decode down kernel gave up waiting for h rows";
-    case 24: return "streaming decode kernel gave up waiting for a weight stage";
     case 25: return "streaming decode kernel gave up waiting for a slot's h rows from other CTAs";
     case 26: return "streaming decode kernel gave up waiting for staged h rows";
+    case 27: return "streaming decode kernel gave up waiting for its warp pair's h buffer";
     case kStatusWaitProbe: return "test probe: a wait that nothing completes gave up";
     default: return code >= kStatusTimeoutFirst ? "a bounded wait gave up" : "a device-side check failed";
   }

@@ -55,6 +55,7 @@ constexpr int kMaxPairsS = kStreamMaxTok * kMaxTopK;  // (token, k) pairs of a b
 constexpr int kMaxSlotsS = kStreamMaxSlots;          // slots: shared + distinct routed experts
 constexpr int kErrHReady = 25;                       // status: gave up waiting for a slot's h
 constexpr int kErrHStaged = 26;                      // status: gave up waiting for staged h
+constexpr int kErrHPair = 27;                        // status: gave up waiting for a pair's h buffer
 
 template <int TT>
 struct StreamRing {
@@ -142,18 +143,19 @@ __device__ __forceinline__ int isum_of(const uint4& a, const uint4& b, const uin
 // One stage of rows on lanes: blocks b0 .. b0+G-1 of the lane's weight row
 // (gate/up halves: lanes 0-15 gate rows, 16-31 the matching up rows; down:
 // 32 output rows) against the staged activation planes of the tokens tok[t]
-// (row tok[t] of the plane arrays xpl / xdc, nb blocks per row).  G is a
-// compile-time stage width, so the block loop is straight-line code: the
-// row's chunk c sits at (row base | rotation) ^ (c << 4) (the row is aligned
-// to its length) and every activation load has an immediate offset.
-template <int TT, int BITS, bool DBG, int G>
-__device__ __forceinline__ void rows_stage(const unsigned char* st, int swz, int b0, int nb, int nv,
+// (row tok[t] of the plane arrays xpl / xdc, nb blocks per row).  The row's
+// chunk c sits at (row base | rotation) ^ (c << 4) (the row is aligned to its
+// length) and the activation loads are offsets from per-stage bases.  GC > 0
+// is a compile-time stage width (straight-line code); GC == 0 takes G at run
+// time.
+template <int TT, int BITS, bool DBG, int GC>
+__device__ __forceinline__ void rows_stage(int Grt, const unsigned char* st, int swz, int b0, int nb, int nv,
                                            const int (&tok)[TT], const uint4* xpl, const float2* xdc,
                                            float (&acc)[TT], int32_t* const (&dbg)[TT]) {
   const int lane = threadIdx.x & 31;
-  constexpr int cpb = BITS / 4;             // 16-byte chunks per block
-  constexpr int kRowBytes = G * cpb * 16;
-  const uintptr_t rb = reinterpret_cast<uintptr_t>(st + lane * kRowBytes) | (uintptr_t)((lane & swz) << 4);
+  constexpr int cpb = BITS / 4;  // 16-byte chunks per block
+  const int G = GC > 0 ? GC : Grt;
+  const uintptr_t rb = reinterpret_cast<uintptr_t>(st + lane * (G * cpb * 16)) | (uintptr_t)((lane & swz) << 4);
   const uint4* xp[TT];
   const float2* xd[TT];
 #pragma unroll
@@ -161,8 +163,7 @@ __device__ __forceinline__ void rows_stage(const unsigned char* st, int swz, int
     xp[t] = xpl + 2 * (tok[t] * nb + b0);
     xd[t] = xdc + tok[t] * nb + b0;
   }
-#pragma unroll
-  for (int j = 0; j < G; ++j) {
+  auto block = [&](int j) {
     uint4 wa, wb;
     if constexpr (BITS == 4) {
       unpack_blk(*reinterpret_cast<const uint4*>(rb ^ (uintptr_t)(j << 4)), wa, wb);
@@ -180,28 +181,17 @@ __device__ __forceinline__ void rows_stage(const unsigned char* st, int swz, int
         acc[t] = __fmaf_rn(dc.x, __int2float_rn(is), acc[t]);
       }
     }
+  };
+  if constexpr (GC > 0) {
+#pragma unroll
+    for (int j = 0; j < GC; ++j) block(j);
+  } else {
+#pragma unroll 4
+    for (int j = 0; j < G; ++j) block(j);
   }
 }
 
-// A stage of runtime width G (a power of two, 1 .. 16 blocks) through the
-// compile-time instances.
-template <int TT, int BITS, bool DBG>
-__device__ __forceinline__ void rows_stage_any(int G, const unsigned char* st, int swz, int b0, int nb, int nv,
-                                               const int (&tok)[TT], const uint4* xpl, const float2* xdc,
-                                               float (&acc)[TT], int32_t* const (&dbg)[TT]) {
-  if (G == 16)
-    rows_stage<TT, BITS, DBG, 16>(st, swz, b0, nb, nv, tok, xpl, xdc, acc, dbg);
-  else if (G == 8)
-    rows_stage<TT, BITS, DBG, 8>(st, swz, b0, nb, nv, tok, xpl, xdc, acc, dbg);
-  else if (G == 4)
-    rows_stage<TT, BITS, DBG, 4>(st, swz, b0, nb, nv, tok, xpl, xdc, acc, dbg);
-  else if (G == 2)
-    rows_stage<TT, BITS, DBG, 2>(st, swz, b0, nb, nv, tok, xpl, xdc, acc, dbg);
-  else
-    rows_stage<TT, BITS, DBG, 1>(st, swz, b0, nb, nv, tok, xpl, xdc, acc, dbg);
-}
-
-template <int TT, int BITS, bool DBG>
+template <int TT, int BITS, bool DBG, int GC>
 __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid_constant__ StreamArgs a) {
   constexpr int R = StreamRing<TT>::R;
   constexpr int kPairs = kSW / 2;
@@ -214,7 +204,10 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   __shared__ uint32_t s_bits[kMaxExperts / 32];
   __shared__ int s_nslots;
   __shared__ float s_h[kPairs][2][TT][32];  // a warp pair's h block, double-buffered by unit
-  __shared__ int s_pair_ok[kPairs][2][2];   // each half's "no wait gave up", double-buffered by unit
+  // per unit parity (unit k uses k & 1, like s_h): halves of the pair's
+  // units finished, and 1 + the last unit whose Q8 block of h is published
+  __shared__ int s_arrive[kPairs][2];
+  __shared__ int s_qdone[kPairs][2];
   __shared__ int s_drow[DBG ? kMaxSlotsS : 1][TT];  // capture row of (slot, position): token * (K + S) + rank
 
   const StreamGeom& g = a.g;
@@ -229,6 +222,10 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   volatile int* abort_f = &abort_s;
 
   for (int i = threadIdx.x; i < kMaxExperts / 32; i += blockDim.x) s_bits[i] = 0u;
+  if (threadIdx.x < 2 * kPairs) {
+    s_arrive[threadIdx.x >> 1][threadIdx.x & 1] = 0;
+    s_qdone[threadIdx.x >> 1][threadIdx.x & 1] = 0;
+  }
   if (threadIdx.x == 0) {
     tc::mbar_init(&hbar[0], 32);
     tc::mbar_init(&hbar[1], 32);
@@ -442,154 +439,184 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   };
   const int64_t P = 2 * (int64_t)g.I * g.nbh + (int64_t)g.H * g.nbi;  // capture words per (token, expert)
 
-  // ---- gate/up half units -----------------------------------------------
-  for (int k = 0; k < n_gu_mine && ok; ++k) {
-    const int u = gp + k * NP;
-    const int slot = u / g.cpu_gu, chunk = u - slot * g.cpu_gu;
-    const int nv = s_cnt[slot];
-    const int orow = chunk * 32 + 16 * half + (lane & 15);  // the lane's intermediate output
+  // ---- the warp's units: gate/up halves, then down units --------------
+  // One loop with one stage-compute call, so that the kernel holds a single
+  // copy of the unrolled block loop.
+  int staged_slot = -1;
+  const int n_units = n_gu_mine + n_dn_mine;
+  for (int k = 0; k < n_units && ok; ++k) {
+    const bool gu = k < n_gu_mine;
+    int slot, chunk, nv, nst, Gs, swz, nb;
+    const uint4* ap;
+    const float2* adc;
     int tok[TT];
-    float acc[TT];
     int32_t* dbg[TT];
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      tok[t] = t < nv ? s_tok[slot][t] : 0;
-      acc[t] = 0.0f;
-      dbg[t] = nullptr;
-      if constexpr (DBG)
-        if (t < nv) dbg[t] = a.dbg + s_drow[slot][t] * P + (int64_t)(lane < 16 ? 0 : g.I) * g.nbh + (int64_t)orow * g.nbh;
-    }
-    for (int s = 0; s < g.st_gu; ++s) {
-      wait_stage();
-      rows_stage_any<TT, BITS, DBG>(g.g_gu, ring + (size_t)(consumed % R) * kStreamStageMax, g.swz_gu, s * g.g_gu,
-                                    g.nbh, nv, tok, xpl, xdc, acc, dbg);
-      next_stage();
-    }
-    // the partner half must reach the barrier even if this warp gave up: no early exit before it
-    const float* sc = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);
-    const float sv = __ldg(sc + (lane < 16 ? 0 : g.I) + orow);
-    float* hb = &s_h[pair][k & 1][0][0];
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      const float v = __fmul_rn(sv, acc[t]);
-      const float uv = __shfl_down_sync(0xffffffffu, v, 16);
-      if (lane < 16 && t < nv) hb[t * 32 + 16 * half + lane] = __fmul_rn(__fmul_rn(v, sigmoid_cw(v)), uv);
-    }
-    if (lane == 0) s_pair_ok[pair][k & 1][half] = (ok && !*abort_f) ? 1 : 0;
-    tc::named_bar(1 + pair, 64);  // both halves of the h block are in shared memory
-    // one decision for both warps of the pair (each meets the barrier of
-    // every unit, so neither may leave the loop alone)
-    ok = s_pair_ok[pair][k & 1][0] && s_pair_ok[pair][k & 1][1];
-    if (half == 0 && ok) {
-      // the Q8_0 block of h (these 32 outputs) for every token, published
+    if (gu) {
+      const int u = gp + k * NP;
+      slot = u / g.cpu_gu;
+      chunk = u - slot * g.cpu_gu;
+      nv = s_cnt[slot];
+      nst = g.st_gu;
+      Gs = g.g_gu;
+      swz = g.swz_gu;
+      nb = g.nbh;
+      ap = xpl;
+      adc = xdc;
+      const int orow = chunk * 32 + 16 * half + (lane & 15);
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
-        if (t < nv) {
-          const float h = hb[t * 32 + lane];
-          const float d = __fdiv_rn(warp_max(fabsf(h)), 127.0f);
-          const int q = q8_of(h, d);
-          const int64_t hrow = s_base[slot] + t;
-          a.hpl[(hrow * g.nbi + chunk) * 32 + (lane & 1) * 16 + (lane >> 1)] = (int8_t)q;
-          const int se = warp_sum_int((lane & 1) ? 0 : q);
-          if (lane == 0) a.hdc[hrow * g.nbi + chunk] = make_float2(d, __int_as_float(-128 * se));
-        }
+        tok[t] = t < nv ? s_tok[slot][t] : 0;
+        dbg[t] = nullptr;
+        if constexpr (DBG)
+          if (t < nv)
+            dbg[t] = a.dbg + s_drow[slot][t] * P + (int64_t)(lane < 16 ? 0 : g.I) * g.nbh + (int64_t)orow * g.nbh;
       }
-      __syncwarp();
-      if (lane == 0) {
-        __threadfence();
-        atomicAdd(a.h_ready + slot, 1);
-      }
-    }
-  }
-
-  // ---- down units -------------------------------------------------------
-  int staged_slot = -1;
-  for (int k = 0; k < n_dn_mine && ok; ++k) {
-    const int v = d0 + warp + k * kSW;
-    const int slot = v / g.cpu_dn, chunk = v - slot * g.cpu_dn;
-    const int nv = s_cnt[slot];
-    const int buf = slot == slotA ? 0 : 1;
-    unsigned char* hb = hst + (size_t)buf * hbuf_bytes;
-    if (slot != staged_slot) {
-      const bool owner = buf == 0 ? warp == 0 : warp == ownerB;
-      if (owner) {
-        // wait for every gate/up unit of the slot, then copy its h rows
-        int ready = 0;
-        if (lane == 0) {
-          const long long t0 = clock64();
-          while (!*abort_f) {
-            if (ld_acquire_gpu(a.h_ready + slot) >= g.cpu_gu) {
-              ready = 1;
-              break;
+    } else {
+      const int v = d0 + warp + (k - n_gu_mine) * kSW;
+      slot = v / g.cpu_dn;
+      chunk = v - slot * g.cpu_dn;
+      nv = s_cnt[slot];
+      nst = g.st_dn;
+      Gs = g.g_dn;
+      swz = g.swz_dn;
+      nb = g.nbi;
+      const int buf = slot == slotA ? 0 : 1;
+      unsigned char* hb = hst + (size_t)buf * hbuf_bytes;
+      if (slot != staged_slot) {
+        const bool owner = buf == 0 ? warp == 0 : warp == ownerB;
+        if (owner) {
+          // wait for every gate/up unit of the slot, then copy its h rows
+          int ready = 0;
+          if (lane == 0) {
+            const long long t0 = clock64();
+            while (!*abort_f) {
+              if (ld_acquire_gpu(a.h_ready + slot) >= g.cpu_gu) {
+                ready = 1;
+                break;
+              }
+              if (clock64() - t0 > tc::kSpinCycles) {
+                *abort_f = 1;
+                atomicExch(a.status, kErrHReady);
+                break;
+              }
+              __nanosleep(128);
             }
-            if (clock64() - t0 > tc::kSpinCycles) {
-              *abort_f = 1;
-              atomicExch(a.status, kErrHReady);
-              break;
-            }
-            __nanosleep(128);
           }
+          ready = __shfl_sync(0xffffffffu, ready, 0);
+          if (ready) {
+            const uint4* sp = reinterpret_cast<const uint4*>(a.hpl + (size_t)s_base[slot] * g.nbi * 32);
+            uint4* dp = reinterpret_cast<uint4*>(hb);
+            const int n16 = nv * g.nbi * 2;
+            for (int i = lane; i < n16; i += 32) dp[i] = __ldcg(sp + i);
+            const float4* sd = reinterpret_cast<const float4*>(a.hdc + (size_t)s_base[slot] * g.nbi);
+            float4* dd = reinterpret_cast<float4*>(hb + (size_t)TT * g.nbi * 32);
+            for (int i = lane; i < nv * g.nbi / 2; i += 32) dd[i] = __ldcg(sd + i);
+          }
+          tc::mbar_arrive(&hbar[buf]);  // all 32 lanes: the stores above are released to the CTA
         }
-        ready = __shfl_sync(0xffffffffu, ready, 0);
-        if (ready) {
-          const uint4* sp = reinterpret_cast<const uint4*>(a.hpl + (size_t)s_base[slot] * g.nbi * 32);
-          uint4* dp = reinterpret_cast<uint4*>(hb);
-          const int n16 = nv * g.nbi * 2;
-          for (int i = lane; i < n16; i += 32) dp[i] = __ldcg(sp + i);
-          const float4* sd = reinterpret_cast<const float4*>(a.hdc + (size_t)s_base[slot] * g.nbi);
-          float4* dd = reinterpret_cast<float4*>(hb + (size_t)TT * g.nbi * 32);
-          for (int i = lane; i < nv * g.nbi / 2; i += 32) dd[i] = __ldcg(sd + i);
+        const bool got = tc::mbar_wait(&hbar[buf], 0, abort_f, a.status, kErrHStaged);
+        if (!__all_sync(0xffffffffu, got && !*abort_f)) {  // warp-uniform
+          ok = false;
+          break;
         }
-        tc::mbar_arrive(&hbar[buf]);  // all 32 lanes: the stores above are released to the CTA
+        staged_slot = slot;
       }
-      const bool got = tc::mbar_wait(&hbar[buf], 0, abort_f, a.status, kErrHStaged);
-      if (!__all_sync(0xffffffffu, got && !*abort_f)) {  // warp-uniform
-        ok = false;
-        break;
-      }
-      staged_slot = slot;
-    }
-    const uint4* hpl = reinterpret_cast<const uint4*>(hb);
-    const float2* hdc = reinterpret_cast<const float2*>(hb + (size_t)TT * g.nbi * 32);
-    int tok[TT];
-    float acc[TT];
-    int32_t* dbg[TT];
-    const int o = chunk * 32 + lane;
+      ap = reinterpret_cast<const uint4*>(hb);
+      adc = reinterpret_cast<const float2*>(hb + (size_t)TT * g.nbi * 32);
+      const int o = chunk * 32 + lane;
 #pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      tok[t] = t;  // the staged h rows are the slot's tokens in order
-      acc[t] = 0.0f;
-      dbg[t] = nullptr;
-      if constexpr (DBG)
-        if (t < nv) dbg[t] = a.dbg + s_drow[slot][t] * P + 2 * (int64_t)g.I * g.nbh + (int64_t)o * g.nbi;
+      for (int t = 0; t < TT; ++t) {
+        tok[t] = t;  // the staged h rows are the slot's tokens in order
+        dbg[t] = nullptr;
+        if constexpr (DBG)
+          if (t < nv) dbg[t] = a.dbg + s_drow[slot][t] * P + 2 * (int64_t)g.I * g.nbh + (int64_t)o * g.nbi;
+      }
     }
-    for (int s = 0; s < g.st_dn; ++s) {
+    float acc[TT];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) acc[t] = 0.0f;
+    for (int s = 0; s < nst; ++s) {
       wait_stage();
-      rows_stage_any<TT, BITS, DBG>(g.g_dn, ring + (size_t)(consumed % R) * kStreamStageMax, g.swz_dn, s * g.g_dn,
-                                    g.nbi, nv, tok, hpl, hdc, acc, dbg);
+      rows_stage<TT, BITS, DBG, GC>(Gs, ring + (size_t)(consumed % R) * kStreamStageMax, swz, s * Gs, nb, nv, tok,
+                                    ap, adc, acc, dbg);
       next_stage();
     }
     const float* sc = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);
-    const float sd = __ldg(sc + 2 * g.I + o);
+    if (gu) {
+      // SwiGLU of the half's 16 outputs into shared memory; the second warp
+      // of the pair to finish quantises the whole Q8_0 block of h and
+      // publishes it (no warp waits for the other)
+      const int orow = chunk * 32 + 16 * half + (lane & 15);
+      const float sv = __ldg(sc + (lane < 16 ? 0 : g.I) + orow);
+      float* hbuf = &s_h[pair][k & 1][0][0];
+      // the buffer was last used by unit k - 2: its block must be published
+      if (k >= 2) {
+        const long long t0 = clock64();
+        while (*(volatile int*)&s_qdone[pair][k & 1] < k - 1 && !*abort_f) {
+          if (clock64() - t0 > tc::kSpinCycles) {
+            *abort_f = 1;
+            atomicExch(a.status, kErrHPair);
+          }
+        }
+      }
 #pragma unroll
-    for (int t = 0; t < TT; ++t)
-      if (t < nv) a.y[((size_t)s_base[slot] + t) * g.H + o] = __fmul_rn(sd, acc[t]);
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) {
-      __threadfence();
-      last = atomicAdd(a.dn_done + chunk, 1) == n_slots - 1;
-      if (last) __threadfence();
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (last) {
-      // every slot's y rows of this chunk are written: combine (contract C)
-      for (int t = 0; t < T; ++t) {
-        float accc = 0.0f;
-        for (int kk = 0; kk < K; ++kk)
-          accc = __fmaf_rn(s_w[t * K + kk], __ldcg(a.y + (size_t)s_row[t * K + kk] * g.H + o), accc);
-        for (int s = 0; s < S; ++s) accc = __fadd_rn(accc, __ldcg(a.y + ((size_t)s_base[s] + t) * g.H + o));
-        a.out[(size_t)t * g.H + o] = accc;
+      for (int t = 0; t < TT; ++t) {
+        const float v = __fmul_rn(sv, acc[t]);
+        const float uv = __shfl_down_sync(0xffffffffu, v, 16);
+        if (lane < 16 && t < nv) hbuf[t * 32 + 16 * half + lane] = __fmul_rn(__fmul_rn(v, sigmoid_cw(v)), uv);
+      }
+      __syncwarp();
+      int second = 0;
+      if (lane == 0) {
+        __threadfence_block();
+        second = atomicAdd(&s_arrive[pair][k & 1], 1) & 1;
+        if (second) __threadfence_block();
+      }
+      second = __shfl_sync(0xffffffffu, second, 0);
+      if (second && !*abort_f) {
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+          if (t < nv) {
+            const float h = *(volatile float*)&hbuf[t * 32 + lane];
+            const float d = __fdiv_rn(warp_max(fabsf(h)), 127.0f);
+            const int q = q8_of(h, d);
+            const int64_t hrow = s_base[slot] + t;
+            a.hpl[(hrow * g.nbi + chunk) * 32 + (lane & 1) * 16 + (lane >> 1)] = (int8_t)q;
+            const int se = warp_sum_int((lane & 1) ? 0 : q);
+            if (lane == 0) a.hdc[hrow * g.nbi + chunk] = make_float2(d, __int_as_float(-128 * se));
+          }
+        }
+        __syncwarp();
+        if (lane == 0) {
+          *(volatile int*)&s_qdone[pair][k & 1] = k + 1;
+          __threadfence();
+          atomicAdd(a.h_ready + slot, 1);
+        }
+      }
+      ok = !*abort_f;
+    } else {
+      const int o = chunk * 32 + lane;
+      const float sd = __ldg(sc + 2 * g.I + o);
+#pragma unroll
+      for (int t = 0; t < TT; ++t)
+        if (t < nv) a.y[((size_t)s_base[slot] + t) * g.H + o] = __fmul_rn(sd, acc[t]);
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) {
+        __threadfence();
+        last = atomicAdd(a.dn_done + chunk, 1) == n_slots - 1;
+        if (last) __threadfence();
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        // every slot's y rows of this chunk are written: combine (contract C)
+        for (int t = 0; t < T; ++t) {
+          float accc = 0.0f;
+          for (int kk = 0; kk < K; ++kk)
+            accc = __fmaf_rn(s_w[t * K + kk], __ldcg(a.y + (size_t)s_row[t * K + kk] * g.H + o), accc);
+          for (int s = 0; s < S; ++s) accc = __fadd_rn(accc, __ldcg(a.y + ((size_t)s_base[s] + t) * g.H + o));
+          a.out[(size_t)t * g.H + o] = accc;
+        }
       }
     }
   }
@@ -645,13 +672,13 @@ __global__ void prepare_expert_kernel(StreamGeom g, const uint8_t* __restrict__ 
     sc[i] = i < g.I ? gs[i] : (i < 2 * g.I ? us[i - g.I] : ds[i - 2 * g.I]);
 }
 
-template <int TT, int BITS, bool DBG>
+template <int TT, int BITS, bool DBG, int GC>
 cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
   static int granted[64] = {};
   static int sms[64] = {};
   const size_t smem = stream_smem_bytes<TT>(a.g);
   if (smem > 224 * 1024) return cudaErrorInvalidConfiguration;
-  cudaError_t e = smem_opt_in(expert_stream_kernel<TT, BITS, DBG>, (int)smem, granted);
+  cudaError_t e = smem_opt_in(expert_stream_kernel<TT, BITS, DBG, GC>, (int)smem, granted);
   if (e != cudaSuccess) return e;
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -661,7 +688,7 @@ cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
   // units of other CTAs); at least as many CTAs as slots, so that a CTA's
   // range of down units spans at most two slots
   if (sms[dev] < kMaxSlotsS) return cudaErrorInvalidConfiguration;
-  return launch_pdl(expert_stream_kernel<TT, BITS, DBG>, dim3(sms[dev]), dim3(kSW * 32), smem, st, true, a);
+  return launch_pdl(expert_stream_kernel<TT, BITS, DBG, GC>, dim3(sms[dev]), dim3(kSW * 32), smem, st, true, a);
 }
 
 }  // namespace
@@ -683,11 +710,20 @@ cudaError_t launch_prepare_expert(int hidden, int inter, int bits, const uint8_t
   return cudaGetLastError();
 }
 
+template <int BITS, bool DBG, int GC>
+cudaError_t stream_g(const StreamArgs& a, cudaStream_t st) {
+  if (a.T <= 1) return stream_tt<1, BITS, DBG, GC>(a, st);
+  if (a.T <= 2) return stream_tt<2, BITS, DBG, GC>(a, st);
+  return stream_tt<4, BITS, DBG, GC>(a, st);
+}
+
+// Full stages (256-byte rows for gate/up and down) take the compile-time
+// width; other shapes the run-time loop.
 template <int BITS, bool DBG>
 cudaError_t stream_bits(const StreamArgs& a, cudaStream_t st) {
-  if (a.T <= 1) return stream_tt<1, BITS, DBG>(a, st);
-  if (a.T <= 2) return stream_tt<2, BITS, DBG>(a, st);
-  return stream_tt<4, BITS, DBG>(a, st);
+  constexpr int kFull = BITS == 4 ? 16 : 8;
+  if (a.g.g_gu == kFull && a.g.g_dn == kFull) return stream_g<BITS, DBG, kFull>(a, st);
+  return stream_g<BITS, DBG, 0>(a, st);
 }
 
 cudaError_t launch_expert_stream(const StreamArgs& a, cudaStream_t st) {

@@ -194,8 +194,9 @@ void set_error_message(const char* msg);
 //                10 prefill producers (operand stage), 11 prefill MMA (operands),
 //                12 prefill MMA (accumulators), 13 prefill fold (accumulators),
 //                16 prefill TMA warp (operand stage), 22 decode down (h rows),
-//                24 streaming kernel (weight stage), 25 streaming kernel (a
-//                slot's h from other CTAs), 26 streaming kernel (staged h),
+//                25 streaming kernel (a slot's h from other CTAs),
+//                26 streaming kernel (staged h), 27 streaming kernel (its warp
+//                pair's h buffer),
 //                30 the test probe coli_debug_wait_probe
 constexpr int32_t kStatusBadExpert = 1;
 constexpr int32_t kStatusTimeoutFirst = 10;
