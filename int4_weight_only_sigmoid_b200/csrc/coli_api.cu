@@ -144,7 +144,7 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   // (d, c16) of every h block and its counters
   const bool sm = T <= kStreamMaxTok;
   L.hdc = take(sm ? rows * (I / 32) * 8 : 0);
-  L.ctr = take(sm ? (size_t)(kStreamMaxSlots + H / 32) * 4 : 0);
+  L.ctr = take(sm ? (size_t)kStreamMaxSlots * 4 : 0);
   L.y = take(rows * H * 4);
   L.xn = take(T * H * 4);
   L.xa = take(T * H * 4);
@@ -214,11 +214,11 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
 
   int32_t* status = at<int32_t>(ws, W.status);
   const int bits = bits_of(c);
-  if (L->prepared != nullptr && stream_supported(H, I, bits, (int)T)) {
+  if (L->prepared != nullptr && stream_supported(H, I, bits, (int)T, K, S)) {
     // decode on the streaming copy: 2 kernels, the second launched with PDL
     int32_t* ctr = at<int32_t>(ws, W.ctr);
     CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, xq, xd, clear_status ? status : nullptr,
-                                      ctr, kStreamMaxSlots + H / 32, st));
+                                      ctr, kStreamMaxSlots, st));
     CHECK_LAUNCH(mark(0));
     StreamArgs a{};
     a.prep = static_cast<const unsigned char*>(L->prepared);
@@ -235,10 +235,8 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
     a.xd = xd;
     a.hpl = hq;
     a.hdc = at<float2>(ws, W.hdc);
-    a.y = y;
     a.out = out;
     a.h_ready = ctr;
-    a.dn_done = ctr + kStreamMaxSlots;
     a.status = status;
     a.dbg = capture;
     CHECK_LAUNCH(launch_expert_stream(a, st));
@@ -368,8 +366,10 @@ const char* status_meaning(int32_t code) {
     case 16: return "prefill A-tile loader gave up waiting for an operand stage";
     case 22: return "decode down kernel gave up waiting for h rows";
     case 25: return "streaming decode kernel gave up waiting for a slot's h rows from other CTAs";
-    case 26: return "streaming decode kernel gave up waiting for staged h rows";
+    case 26: return "streaming decode kernel gave up waiting for a slot's h rows in shared memory";
     case 27: return "streaming decode kernel gave up waiting for its warp pair's h buffer";
+    case 28: return "streaming decode kernel gave up waiting for a weight stage copy";
+
     case kStatusWaitProbe: return "test probe: a wait that nothing completes gave up";
     default: return code >= kStatusTimeoutFirst ? "a bounded wait gave up" : "a device-side check failed";
   }

@@ -54,20 +54,33 @@ constexpr int kSW = 8;                               // warps per CTA (all compu
 constexpr int kMaxPairsS = kStreamMaxTok * kMaxTopK;  // (token, k) pairs of a batch
 constexpr int kMaxSlotsS = kStreamMaxSlots;          // slots: shared + distinct routed experts
 constexpr int kErrHReady = 25;                       // status: gave up waiting for a slot's h
-constexpr int kErrHStaged = 26;                      // status: gave up waiting for staged h
+constexpr int kErrHStaged = 26;                      // status: gave up waiting for a slot's staged h
 constexpr int kErrHPair = 27;                        // status: gave up waiting for a pair's h buffer
+constexpr int kErrStage = 28;                        // status: gave up waiting for a weight stage
+constexpr int kR = 2;                                // ring stages per warp (8 KB each)
+constexpr int kQ = 4;                                // a warp's queue of down units (> kR)
 
+// y rows of a CTA's down chunks in shared memory: rows = T * (K + S) of the
+// batch (slot order), rpu floats per (chunk, row)
+__host__ __device__ inline size_t stream_y_bytes(const StreamGeom& g, int n_sms, int n_rows) {
+  const int nch = (g.cpu_dn + n_sms - 1) / n_sms;
+  return (size_t)nch * n_rows * g.rpu_dn * 4;
+}
+
+// Batches of up to two tokens stage each slot's h rows in shared memory
+// (one bulk copy per slot, made by the first warp that needs it); larger
+// batches read them through L1.
 template <int TT>
-struct StreamRing {
-  static constexpr int R = TT <= 2 ? 3 : 2;  // stages per warp
+struct StreamHStaged {
+  static constexpr bool value = TT <= 2;
 };
 
 template <int TT>
-__host__ __device__ inline size_t stream_smem_bytes(const StreamGeom& g) {
-  const size_t ring = (size_t)kSW * StreamRing<TT>::R * kStreamStageMax;  // 8 KB stages
-  const size_t xs = (size_t)TT * g.nbh * 40;        // x planes (32 B) + (d, c16) per block
-  const size_t hs = 2 * (size_t)TT * g.nbi * 40;    // two slots' h rows
-  return 1024 + ring + xs + hs;
+__host__ __device__ inline size_t stream_smem_bytes(const StreamGeom& g, int n_sms, int n_rows) {
+  const size_t ring = (size_t)kSW * kR * kStreamStageMax;  // 8 KB stages
+  const size_t xs = (size_t)TT * g.nbh * 40;               // x planes (32 B) + (d, c16) per block
+  const size_t hs = StreamHStaged<TT>::value ? (size_t)n_rows * g.nbi * 40 : 0;  // h planes + (d, c16)
+  return 1024 + ring + xs + stream_y_bytes(g, n_sms, n_rows) + hs;
 }
 
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
@@ -140,51 +153,101 @@ __device__ __forceinline__ int isum_of(const uint4& a, const uint4& b, const uin
   return blk_isum8(a, b, xe, xo);
 }
 
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ float2 lds64f(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
 // One stage of rows on lanes: blocks b0 .. b0+G-1 of the lane's weight row
 // (gate/up halves: lanes 0-15 gate rows, 16-31 the matching up rows; down:
-// 32 output rows) against the staged activation planes of the tokens tok[t]
-// (row tok[t] of the plane arrays xpl / xdc, nb blocks per row).  The row's
-// chunk c sits at (row base | rotation) ^ (c << 4) (the row is aligned to its
-// length) and the activation loads are offsets from per-stage bases.  GC > 0
-// is a compile-time stage width (straight-line code); GC == 0 takes G at run
-// time.
-template <int TT, int BITS, bool DBG, int GC>
+// 32 output rows) against the activation planes of the tokens tok[t] (row
+// tok[t] of the plane arrays xpl / xdc, nb blocks per row: shared memory
+// when XS, else global memory read through L1).  The stage sits in shared
+// memory; the row's chunk c is at (row base | rotation) ^ (c << 4) (the row
+// is aligned to its length).  GC > 0 is a compile-time stage width
+// (straight-line code); GC == 0 takes G at run time.  pair (GC > 0 only):
+// lanes l and l + 16 hold the two pieces of one row (blocks b0 .. of lane l,
+// then those of lane l + 16): lanes 16-31 fold their blocks again from lane
+// l - 16's result, and both lanes keep the row's sum.
+template <int TT, int BITS, bool DBG, int GC, bool XS>
 __device__ __forceinline__ void rows_stage(int Grt, const unsigned char* st, int swz, int b0, int nb, int nv,
-                                           const int (&tok)[TT], const uint4* xpl, const float2* xdc,
+                                           bool pair, const int (&tok)[TT], const uint4* xpl, const float2* xdc,
                                            float (&acc)[TT], int32_t* const (&dbg)[TT]) {
   const int lane = threadIdx.x & 31;
   constexpr int cpb = BITS / 4;  // 16-byte chunks per block
   const int G = GC > 0 ? GC : Grt;
-  const uintptr_t rb = reinterpret_cast<uintptr_t>(st + lane * (G * cpb * 16)) | (uintptr_t)((lane & swz) << 4);
+  const uint32_t rb = (tc::smem_u32(st) + (uint32_t)(lane * (G * cpb * 16))) | (uint32_t)((lane & swz) << 4);
   const uint4* xp[TT];
   const float2* xd[TT];
+  uint32_t xps[TT], xds[TT];
 #pragma unroll
   for (int t = 0; t < TT; ++t) {
     xp[t] = xpl + 2 * (tok[t] * nb + b0);
     xd[t] = xdc + tok[t] * nb + b0;
+    if constexpr (XS) {
+      xps[t] = tc::smem_u32(xp[t]);
+      xds[t] = tc::smem_u32(xd[t]);
+    }
   }
+  auto xload = [&](int t, int j, uint4& xe, uint4& xo, float2& dc) {
+    if constexpr (XS) {
+      xe = lds128(xps[t] + 32 * j);
+      xo = lds128(xps[t] + 32 * j + 16);
+      dc = lds64f(xds[t] + 8 * j);
+    } else {
+      xe = xp[t][2 * j];
+      xo = xp[t][2 * j + 1];
+      dc = xd[t][j];
+    }
+  };
+  float fis[TT][GC > 0 ? GC : 1];  // the blocks' sums, for the second piece of a lane pair
   auto block = [&](int j) {
     uint4 wa, wb;
     if constexpr (BITS == 4) {
-      unpack_blk(*reinterpret_cast<const uint4*>(rb ^ (uintptr_t)(j << 4)), wa, wb);
+      unpack_blk(lds128(rb ^ (uint32_t)(j << 4)), wa, wb);
     } else {
-      wa = *reinterpret_cast<const uint4*>(rb ^ (uintptr_t)((2 * j) << 4));
-      wb = *reinterpret_cast<const uint4*>(rb ^ (uintptr_t)((2 * j + 1) << 4));
+      wa = lds128(rb ^ (uint32_t)((2 * j) << 4));
+      wb = lds128(rb ^ (uint32_t)((2 * j + 1) << 4));
     }
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
       if (TT == 1 || t < nv) {
-        const uint4 xe = xp[t][2 * j], xo = xp[t][2 * j + 1];
-        const float2 dc = xd[t][j];
+        uint4 xe, xo;
+        float2 dc;
+        xload(t, j, xe, xo, dc);
         const int is = isum_of<BITS>(wa, wb, xe, xo, __float_as_int(dc.y));
         if constexpr (DBG) dbg[t][b0 + j] = is;
-        acc[t] = __fmaf_rn(dc.x, __int2float_rn(is), acc[t]);
+        const float f = __int2float_rn(is);
+        if constexpr (GC > 0) fis[t][j] = f;
+        acc[t] = __fmaf_rn(dc.x, f, acc[t]);
       }
     }
   };
   if constexpr (GC > 0) {
 #pragma unroll
     for (int j = 0; j < GC; ++j) block(j);
+    if (pair) {
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        if (TT == 1 || t < nv) {
+          float a2 = __shfl_xor_sync(0xffffffffu, acc[t], 16);
+#pragma unroll
+          for (int j = 0; j < GC; ++j) {
+            const float d = XS ? lds64f(xds[t] + 8 * j).x : xd[t][j].x;
+            a2 = __fmaf_rn(d, fis[t][j], a2);
+          }
+          const float o2 = __shfl_xor_sync(0xffffffffu, a2, 16);
+          acc[t] = lane >= 16 ? a2 : o2;
+        }
+      }
+    }
   } else {
 #pragma unroll 4
     for (int j = 0; j < G; ++j) block(j);
@@ -193,61 +256,82 @@ __device__ __forceinline__ void rows_stage(int Grt, const unsigned char* st, int
 
 template <int TT, int BITS, bool DBG, int GC>
 __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid_constant__ StreamArgs a) {
-  constexpr int R = StreamRing<TT>::R;
+  constexpr int R = kR;
   constexpr int kPairs = kSW / 2;
   extern __shared__ unsigned char smem_raw[];
-  __shared__ uint64_t hbar[2];
+  __shared__ uint64_t s_full[kSW][kR];  // one mbarrier per ring slot of each warp
   __shared__ int abort_s;
   __shared__ int s_idx[kMaxPairsS], s_row[kMaxPairsS];
   __shared__ float s_w[kMaxPairsS];
   __shared__ int s_exp[kMaxSlotsS], s_cnt[kMaxSlotsS], s_base[kMaxSlotsS], s_tok[kMaxSlotsS][TT];
-  __shared__ uint32_t s_bits[kMaxExperts / 32];
+  __shared__ uint32_t s_bits[kMaxExperts / 32], s_tm[kMaxExperts / 4];
+  __shared__ int s_bpre[kMaxExperts / 32];
   __shared__ int s_nslots;
+  __shared__ int s_dn_next;     // the next of this CTA's down units to hand out
+  __shared__ int s_q[kSW][kQ];  // per warp: the down units its cursor took, in order (-1: no more)
   __shared__ float s_h[kPairs][2][TT][32];  // a warp pair's h block, double-buffered by unit
   // per unit parity (unit k uses k & 1, like s_h): halves of the pair's
   // units finished, and 1 + the last unit whose Q8 block of h is published
   __shared__ int s_arrive[kPairs][2];
   __shared__ int s_qdone[kPairs][2];
   __shared__ int s_drow[DBG ? kMaxSlotsS : 1][TT];  // capture row of (slot, position): token * (K + S) + rank
+  constexpr bool HS = StreamHStaged<TT>::value;
+  __shared__ int s_hclaim[HS ? kMaxSlotsS : 1];      // a warp has issued the slot's h copy
+  __shared__ uint64_t s_hbar[HS ? kMaxSlotsS : 1];   // the slot's h rows are in shared memory
 
   const StreamGeom& g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = a.E, K = a.K, S = a.S, T = a.T;
+  const int n_rows = T * (K + S);  // y rows of the batch (slot order)
   unsigned char* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   unsigned char* ring = smem + (size_t)warp * R * kStreamStageMax;
   uint4* xpl = reinterpret_cast<uint4*>(smem + (size_t)kSW * R * kStreamStageMax);
   float2* xdc = reinterpret_cast<float2*>(xpl + 2 * TT * g.nbh);
-  unsigned char* hst = reinterpret_cast<unsigned char*>(xdc + TT * g.nbh);
-  const size_t hbuf_bytes = (size_t)TT * g.nbi * 40;
+  float* s_y = reinterpret_cast<float*>(xdc + TT * g.nbh);  // [chunk of this CTA][y row][rpu_dn]
+  // staged h (HS): the batch's rows in global order, planes then (d, c16)
+  unsigned char* hst = reinterpret_cast<unsigned char*>(s_y) + stream_y_bytes(g, gridDim.x, n_rows);
+  unsigned char* hst_dc = hst + (size_t)n_rows * g.nbi * 32;
   volatile int* abort_f = &abort_s;
 
-  for (int i = threadIdx.x; i < kMaxExperts / 32; i += blockDim.x) s_bits[i] = 0u;
+  for (int i = threadIdx.x; i < kMaxExperts / 4; i += blockDim.x) {
+    if (i < kMaxExperts / 32) s_bits[i] = 0u;
+    s_tm[i] = 0u;
+  }
   if (threadIdx.x < 2 * kPairs) {
     s_arrive[threadIdx.x >> 1][threadIdx.x & 1] = 0;
     s_qdone[threadIdx.x >> 1][threadIdx.x & 1] = 0;
   }
+  if constexpr (HS)
+    for (int i = threadIdx.x; i < kMaxSlotsS; i += blockDim.x) s_hclaim[i] = 0;
   if (threadIdx.x == 0) {
-    tc::mbar_init(&hbar[0], 32);
-    tc::mbar_init(&hbar[1], 32);
+    for (int i = 0; i < kSW * kR; ++i) tc::mbar_init(&s_full[i / kR][i % kR], 1);
+    if constexpr (HS)
+      for (int i = 0; i < kMaxSlotsS; ++i) tc::mbar_init(&s_hbar[i], 1);
     abort_s = 0;
+    s_dn_next = 0;
     stream::fence_mbar_init();
   }
   __syncthreads();
 
   // Gate/up work goes to warp pairs: pair p of this CTA takes units
   // gp, gp + NP, ... (gp = p * G + blockIdx.x), warp 2p the first half of
-  // each unit, warp 2p + 1 the second.  Down units: this CTA's contiguous
-  // range [d0, d1), warp w takes d0 + w, d0 + w + kSW, ...
+  // each unit, warp 2p + 1 the second.  Down work: this CTA owns the output
+  // chunks [c0, c1) (rpu_dn rows each) of every slot, i.e. the units
+  // id = slot * nch + (chunk - c0), handed out in that order (slot by slot)
+  // to whichever warp's cursor asks next; their y rows stay in shared memory
+  // and the CTA combines its own chunks at the end.
   const int G = gridDim.x, NP = G * kPairs;
   const int pair = warp >> 1, half = warp & 1, gp = pair * G + blockIdx.x;
   const int n_shared_gu = S * g.cpu_gu;
+  const int c0 = (int)((int64_t)blockIdx.x * g.cpu_dn / G), c1 = (int)((int64_t)(blockIdx.x + 1) * g.cpu_dn / G);
+  const int nch = c1 - c0;
 
-  // The warp's stage sequence: its gate/up half units, then its down units.
-  // A cursor walks it R stages ahead of the compute: (phase, unit index k,
-  // stage s, the unit's base address); the divisions happen once per unit.
-  // Before the routing is known only the first unit, if it is a shared
-  // expert's, can stream.
-  int n_gu_mine = 0, n_dn_mine = 0, d0 = 0;
+  // The warp's stage sequence: its gate/up half units, then the down units
+  // it takes.  A cursor walks it R stages ahead of the compute: (phase, unit
+  // index k, stage s, the unit's base address); the divisions happen once
+  // per unit.  Before the routing is known only the first unit, if it is a
+  // shared expert's, can stream.
+  int n_gu_mine = 0, n_dn_cta = 0;
   struct Cursor {
     int phase, k, s;  // phase 0 gate/up, 1 down, 2 done
     const unsigned char* base;
@@ -257,32 +341,41 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       c.phase = 1;
       c.k = 0;
     }
-    if (c.phase == 1 && c.k >= n_dn_mine) c.phase = 2;
     if (c.phase == 0) {
       const int u = gp + c.k * NP;
       const int slot = u / g.cpu_gu;
       const int e = slot < S ? E + slot : s_exp[slot];
       c.base = a.prep + (uint64_t)e * g.expert_bytes + (uint64_t)((u - slot * g.cpu_gu) * 2 + half) * g.ub_gu;
     } else if (c.phase == 1) {
-      const int v = d0 + warp + c.k * kSW;
-      const int slot = v / g.cpu_dn;
-      const int e = slot < S ? E + slot : s_exp[slot];
-      c.base = a.prep + (uint64_t)e * g.expert_bytes + g.dn_off + (uint64_t)(v - slot * g.cpu_dn) * g.ub_dn;
+      int id = 0;
+      if (lane == 0) id = atomicAdd(&s_dn_next, 1);
+      id = __shfl_sync(0xffffffffu, id, 0);
+      if (id >= n_dn_cta) {
+        id = -1;
+        c.phase = 2;
+      }
+      s_q[warp][c.k & (kQ - 1)] = id;
+      if (id >= 0) {
+        const int slot = id / nch, chunk = c0 + (id - slot * nch);
+        const int e = slot < S ? E + slot : s_exp[slot];
+        c.base = a.prep + (uint64_t)e * g.expert_bytes + g.dn_off + (uint64_t)chunk * g.ub_dn;
+      }
     }
   };
   Cursor pc{0, 0, 0, nullptr};
-  int issued = 0;
-  // all lanes: the cursor's stage into ring slot issued % R with cp.async
-  // (lane l copies 16-byte chunks l, l + 32, ...: each instruction moves 512
-  // contiguous bytes), one commit group per stage (empty past the end)
+  int issued = 0, n_real = 0;  // stages issued (past the end: empty), and real copies among them
+  // lane 0: the cursor's stage into ring slot issued % R, one bulk copy
+  // completing on the slot's mbarrier
   auto copy_stage = [&]() {
     if (pc.phase < 2) {
       const uint32_t bytes = pc.phase == 0 ? g.sb_gu : g.sb_dn;
-      const unsigned char* src = pc.base + (uint64_t)pc.s * bytes;
-      unsigned char* dst = ring + (size_t)(issued % R) * kStreamStageMax;
-      for (uint32_t off = 16 * lane; off < bytes; off += 512) cp_async16(dst + off, src + off);
+      if (lane == 0) {
+        uint64_t* bar = &s_full[warp][issued % R];
+        stream::mbar_expect_tx(bar, bytes);
+        stream::bulk_g2s(ring + (size_t)(issued % R) * kStreamStageMax, pc.base + (uint64_t)pc.s * bytes, bytes, bar);
+      }
+      ++n_real;
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
     ++issued;
   };
   auto issue = [&]() {  // copy, then move the cursor on
@@ -306,15 +399,26 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     }
   }
 
+  // the correction bias is a layer constant: into registers before the wait
+  float bias_r[kMaxExperts / 32];
+#pragma unroll
+  for (int i = 0; i < kMaxExperts / 32; ++i) {
+    const int e = lane + 32 * i;
+    bias_r[i] = warp < T && e < E ? __ldg(a.bias + e) : 0.0f;
+  }
+
   pdl_wait();  // scores, the Q8_0 of x and the cleared counters are complete
   pdl_launch_dependents();
 
   // ---- routing of the batch (every CTA, identical results) -------------
   if (warp < T) {
-    int sel[kMaxTopK];
-    float ssel[kMaxTopK];
-    topk::warp_select_topk(a.scores + (size_t)warp * E, a.bias, E, K, lane, sel, ssel);
-    if (lane == 0) topk::topk_weights(sel, ssel, K, a.norm, a.rsf, s_idx + warp * K, s_w + warp * K);
+    const float* st = a.scores + (size_t)warp * E;
+    auto sc = [st](int e) { return ld_dep(st + e); };
+    if (E <= 256)
+      topk::warp_route_token<8>(sc, bias_r, E, K, a.norm, a.rsf, lane, s_idx + warp * K, s_w + warp * K);
+    else
+      topk::warp_route_token<kMaxExperts / 32>(sc, bias_r, E, K, a.norm, a.rsf, lane, s_idx + warp * K,
+                                               s_w + warp * K);
   }
   // x planes: block b of token t -> even / odd byte planes and (d, c16)
   for (int i = threadIdx.x; i < T * g.nbh; i += blockDim.x) {
@@ -331,88 +435,74 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     xdc[i] = make_float2(ld_dep(a.xd + i), __int_as_float(-128 * even_plane_sum(e)));
   }
   __syncthreads();
-  const int n_pairs = T * K;
   if (warp == 0) {
-    for (int p = lane; p < n_pairs; p += 32) atomicOr(&s_bits[s_idx[p] >> 5], 1u << (s_idx[p] & 31));
+    // bucketing: the chosen experts (bit e of s_bits) and, per expert, the
+    // tokens that chose it (byte e & 3 of s_tm[e >> 2], bit t)
+    const int n_pairs = T * K;
+    for (int p = lane; p < n_pairs; p += 32) {
+      const int e = s_idx[p], t = p / K;
+      atomicOr(&s_bits[e >> 5], 1u << (e & 31));
+      atomicOr(&s_tm[e >> 2], 1u << ((e & 3) * 8 + t));
+    }
     __syncwarp();
-    // slot of routed expert e: S + (set bits below e); slots in ascending expert id
+    auto tm_of = [&](int e) { return (s_tm[e >> 2] >> ((e & 3) * 8)) & 0xFFu; };
+    // lane l: the experts 32l .. 32l+31; slots in ascending expert id after
+    // the shared ones, rows in slot order, a slot's rows in token order
     const int nw = (E + 31) / 32;
-    const int c = lane < nw ? __popc(s_bits[lane]) : 0;
-    int incl = c;
+    const uint32_t bits = lane < nw ? s_bits[lane] : 0u;
+    int rows = 0;
+    for (uint32_t bb = bits; bb; bb &= bb - 1) rows += __popc(tm_of(32 * lane + __ffs(bb) - 1));
+    const int c = __popc(bits);
+    int ci = c, ri = rows;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const int below_word = incl - c;
-    const int n_routed = __shfl_sync(0xffffffffu, incl, 31);
-    if (lane < nw) {
-      uint32_t bits = s_bits[lane];
-      int r = S + below_word;
-      while (bits) {
-        const int bit = __ffs(bits) - 1;
-        bits &= bits - 1;
-        s_exp[r] = 32 * lane + bit;
-        s_cnt[r] = 0;
-        ++r;
+      const int yc = __shfl_up_sync(0xffffffffu, ci, o), yr = __shfl_up_sync(0xffffffffu, ri, o);
+      if (lane >= o) {
+        ci += yc;
+        ri += yr;
       }
     }
-    for (int s = lane; s < S; s += 32) {
-      s_exp[s] = E + s;
-      s_cnt[s] = T;
+    if (lane < nw) s_bpre[lane] = ci - c;
+    if (lane == 31) s_nslots = S + ci;
+    int r = S + ci - c, base = S * T + ri - rows;
+    for (uint32_t bb = bits; bb; bb &= bb - 1) {
+      const int e = 32 * lane + __ffs(bb) - 1;
+      const uint32_t m = tm_of(e);
+      s_exp[r] = e;
+      s_cnt[r] = __popc(m);
+      s_base[r] = base;
+      int pos = 0;
+#pragma unroll
+      for (int t = 0; t < TT; ++t)
+        if ((m >> t) & 1u) s_tok[r][pos++] = t;
+      base += __popc(m);
+      ++r;
+    }
+    for (int sh = lane; sh < S; sh += 32) {
+      s_exp[sh] = E + sh;
+      s_cnt[sh] = T;
+      s_base[sh] = sh * T;
       for (int t = 0; t < TT; ++t) {
-        s_tok[s][t] = t;
-        if constexpr (DBG) s_drow[s][t] = t * (K + S) + K + s;
+        s_tok[sh][t] = t;
+        if constexpr (DBG) s_drow[sh][t] = t * (K + S) + K + sh;
       }
     }
     __syncwarp();
-    // each pair: its slot, and its position = earlier tokens on the same expert
-    int pslot[2] = {0, 0}, ppos[2] = {0, 0};
-    for (int h = 0; h < 2; ++h) {
-      const int p = lane + 32 * h;
-      if (p < n_pairs) {
-        const int e = s_idx[p], t = p / K;
-        const int w32 = e >> 5;
-        const int lo = __popc(s_bits[w32] & ((1u << (e & 31)) - 1u));
-        int below = 0;  // set bits in the words below w32
-        for (int q = 0; q < w32; ++q) below += __popc(s_bits[q]);
-        pslot[h] = S + below + lo;
-        int pos = 0;
-        for (int q = 0; q < t * K; ++q) pos += (s_idx[q] == e);
-        ppos[h] = pos;
-        atomicAdd(&s_cnt[pslot[h]], 1);
-        s_tok[pslot[h]][pos] = t;
-        if constexpr (DBG) s_drow[pslot[h]][pos] = t * (K + S) + (p - t * K);  // rank p - tK of token t
-      }
-    }
-    __syncwarp();
-    if (lane == 0) {
-      int base = 0;
-      for (int s = 0; s < S + n_routed; ++s) {
-        s_base[s] = base;
-        base += s_cnt[s];
-      }
-      s_nslots = S + n_routed;
-    }
-    __syncwarp();
-    for (int h = 0; h < 2; ++h) {
-      const int p = lane + 32 * h;
-      if (p < n_pairs) s_row[p] = s_base[pslot[h]] + ppos[h];
+    // each (token, rank) pair: the row of its expert's output
+    for (int p = lane; p < n_pairs; p += 32) {
+      const int e = s_idx[p], t = p / K, w32 = e >> 5;
+      const int slot = S + s_bpre[w32] + __popc(s_bits[w32] & ((1u << (e & 31)) - 1u));
+      const int pos = __popc(tm_of(e) & ((1u << t) - 1u));
+      s_row[p] = s_base[slot] + pos;
+      if constexpr (DBG) s_drow[slot][pos] = t * (K + S) + (p - t * K);  // rank p - tK of token t
     }
   }
   __syncthreads();
 
   const int n_slots = s_nslots;
-  const int n_gu = n_slots * g.cpu_gu, n_dn = n_slots * g.cpu_dn;
+  const int n_gu = n_slots * g.cpu_gu;
   n_gu_mine = gp < n_gu ? (n_gu - gp + NP - 1) / NP : 0;
-  d0 = (int)((int64_t)blockIdx.x * n_dn / G);
-  const int d1 = (int)((int64_t)(blockIdx.x + 1) * n_dn / G);
-  n_dn_mine = d0 + warp < d1 ? (d1 - d0 - warp + kSW - 1) / kSW : 0;
-  // the down slots of this CTA's range (at most two: a range never spans
-  // more, since there are at least as many CTAs as slots)
-  const int slotA = d0 / g.cpu_dn;
-  const int slotB = d1 > d0 ? (d1 - 1) / g.cpu_dn : slotA;
-  const int ownerB = slotB != slotA ? ((slotB * g.cpu_dn - d0) % kSW) : -1;
+  n_dn_cta = n_slots * nch;
 
   if (pre == 0) {
     unit_base(pc);  // the cursor's first unit, now that the counts are known
@@ -425,11 +515,10 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
 
   int consumed = 0;
   bool ok = true;
-  // this lane's copies of the oldest stage are in (R - 1 newer groups may
-  // still be in flight), then every lane's
-  auto wait_stage = [&]() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(R - 1) : "memory");
-    __syncwarp();
+  auto wait_stage = [&]() -> bool {
+    const bool got = tc::mbar_wait(&s_full[warp][consumed % R], (uint32_t)((consumed / R) & 1), abort_f, a.status,
+                                   kErrStage);
+    return __all_sync(0xffffffffu, got);
   };
   // the ring slot of the stage just computed is free again: copy the stage R ahead into it
   auto next_stage = [&]() {
@@ -442,11 +531,10 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   // ---- the warp's units: gate/up halves, then down units --------------
   // One loop with one stage-compute call, so that the kernel holds a single
   // copy of the unrolled block loop.
-  int staged_slot = -1;
-  const int n_units = n_gu_mine + n_dn_mine;
-  for (int k = 0; k < n_units && ok; ++k) {
+  int acq_slot = -1;  // the last slot whose h this warp has acquired
+  for (int k = 0; ok; ++k) {
     const bool gu = k < n_gu_mine;
-    int slot, chunk, nv, nst, Gs, swz, nb;
+    int slot, chunk, nv, nst, Gs, swz, nb, lpr = 1;
     const uint4* ap;
     const float2* adc;
     int tok[TT];
@@ -472,82 +560,104 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
             dbg[t] = a.dbg + s_drow[slot][t] * P + (int64_t)(lane < 16 ? 0 : g.I) * g.nbh + (int64_t)orow * g.nbh;
       }
     } else {
-      const int v = d0 + warp + (k - n_gu_mine) * kSW;
-      slot = v / g.cpu_dn;
-      chunk = v - slot * g.cpu_dn;
+      const int id = s_q[warp][(k - n_gu_mine) & (kQ - 1)];
+      if (id < 0) break;  // the CTA's down units are all taken
+      slot = id / nch;
+      chunk = c0 + (id - slot * nch);
       nv = s_cnt[slot];
       nst = g.st_dn;
       Gs = g.g_dn;
       swz = g.swz_dn;
       nb = g.nbi;
-      const int buf = slot == slotA ? 0 : 1;
-      unsigned char* hb = hst + (size_t)buf * hbuf_bytes;
-      if (slot != staged_slot) {
-        const bool owner = buf == 0 ? warp == 0 : warp == ownerB;
-        if (owner) {
-          // wait for every gate/up unit of the slot, then copy its h rows
-          int ready = 0;
-          if (lane == 0) {
-            const long long t0 = clock64();
-            while (!*abort_f) {
-              if (ld_acquire_gpu(a.h_ready + slot) >= g.cpu_gu) {
-                ready = 1;
-                break;
-              }
-              if (clock64() - t0 > tc::kSpinCycles) {
-                *abort_f = 1;
-                atomicExch(a.status, kErrHReady);
-                break;
-              }
-              __nanosleep(128);
+      lpr = g.lpr_dn;
+      if (slot != acq_slot) {
+        // every gate/up unit of the slot is counted: its h rows are complete,
+        // and the acquire orders the reads of them after their stores.  HS:
+        // the first warp of the CTA to get here copies the rows into shared
+        // memory (one bulk copy for the planes, one for (d, c16)); every
+        // warp waits for that copy.
+        bool claim = true;
+        if constexpr (HS) {
+          int c = 0;
+          if (lane == 0) c = atomicCAS(&s_hclaim[slot], 0, 1) == 0;
+          claim = __shfl_sync(0xffffffffu, c, 0) != 0;
+        }
+        bool ready = !claim;
+        if (claim) {
+          const long long t0 = clock64();
+          while (!*abort_f) {
+            if (ld_acquire_gpu(a.h_ready + slot) >= g.cpu_gu) {
+              ready = true;
+              break;
+            }
+            if (clock64() - t0 > tc::kSpinCycles) {
+              *abort_f = 1;
+              atomicExch(a.status, kErrHReady);
+              break;
+            }
+            __nanosleep(64);
+          }
+          if constexpr (HS) {
+            if (lane == 0 && ready) {
+              const size_t r0 = s_base[slot];
+              const uint32_t pl = (uint32_t)(nv * g.nbi * 32), dc = (uint32_t)(nv * g.nbi * 8);
+              stream::fence_proxy_async_global();
+              stream::mbar_expect_tx(&s_hbar[slot], pl + dc);
+              stream::bulk_g2s(hst + r0 * g.nbi * 32, a.hpl + r0 * g.nbi * 32, pl, &s_hbar[slot]);
+              stream::bulk_g2s(hst_dc + r0 * g.nbi * 8, a.hdc + r0 * g.nbi, dc, &s_hbar[slot]);
             }
           }
-          ready = __shfl_sync(0xffffffffu, ready, 0);
-          if (ready) {
-            const uint4* sp = reinterpret_cast<const uint4*>(a.hpl + (size_t)s_base[slot] * g.nbi * 32);
-            uint4* dp = reinterpret_cast<uint4*>(hb);
-            const int n16 = nv * g.nbi * 2;
-            for (int i = lane; i < n16; i += 32) dp[i] = __ldcg(sp + i);
-            const float4* sd = reinterpret_cast<const float4*>(a.hdc + (size_t)s_base[slot] * g.nbi);
-            float4* dd = reinterpret_cast<float4*>(hb + (size_t)TT * g.nbi * 32);
-            for (int i = lane; i < nv * g.nbi / 2; i += 32) dd[i] = __ldcg(sd + i);
-          }
-          tc::mbar_arrive(&hbar[buf]);  // all 32 lanes: the stores above are released to the CTA
         }
-        const bool got = tc::mbar_wait(&hbar[buf], 0, abort_f, a.status, kErrHStaged);
-        if (!__all_sync(0xffffffffu, got && !*abort_f)) {  // warp-uniform
+        if constexpr (HS) ready = tc::mbar_wait(&s_hbar[slot], 0, abort_f, a.status, kErrHStaged);
+        if (!__all_sync(0xffffffffu, ready)) {
           ok = false;
           break;
         }
-        staged_slot = slot;
+        acq_slot = slot;
       }
-      ap = reinterpret_cast<const uint4*>(hb);
-      adc = reinterpret_cast<const float2*>(hb + (size_t)TT * g.nbi * 32);
-      const int o = chunk * 32 + lane;
+      if constexpr (HS) {
+        ap = reinterpret_cast<const uint4*>(hst + (size_t)s_base[slot] * g.nbi * 32);
+        adc = reinterpret_cast<const float2*>(hst_dc + (size_t)s_base[slot] * g.nbi * 8);
+      } else {
+        // the slot's h rows are read through L1 (every lane loads the same block)
+        ap = reinterpret_cast<const uint4*>(a.hpl + (size_t)s_base[slot] * g.nbi * 32);
+        adc = a.hdc + (size_t)s_base[slot] * g.nbi;
+      }
+      const int o = chunk * g.rpu_dn + (lane & (g.rpu_dn - 1));
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
-        tok[t] = t;  // the staged h rows are the slot's tokens in order
+        tok[t] = t;  // the slot's h rows are its tokens in order
         dbg[t] = nullptr;
         if constexpr (DBG)
           if (t < nv) dbg[t] = a.dbg + s_drow[slot][t] * P + 2 * (int64_t)g.I * g.nbh + (int64_t)o * g.nbi;
       }
     }
+    // the row scale of this lane's output, loaded ahead of the stages
+    const float* sc = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);
+    const float rs =
+        gu ? __ldg(sc + (lane < 16 ? 0 : g.I) + chunk * 32 + 16 * half + (lane & 15))
+           : __ldg(sc + 2 * g.I + chunk * g.rpu_dn + (lane & (g.rpu_dn - 1)));
     float acc[TT];
 #pragma unroll
     for (int t = 0; t < TT; ++t) acc[t] = 0.0f;
-    for (int s = 0; s < nst; ++s) {
-      wait_stage();
-      rows_stage<TT, BITS, DBG, GC>(Gs, ring + (size_t)(consumed % R) * kStreamStageMax, swz, s * Gs, nb, nv, tok,
-                                    ap, adc, acc, dbg);
+    // a lane's first block in stage s (lane pairs: lanes 16-31 the second piece)
+    const int span = lpr * Gs, piece0 = lpr == 2 ? (lane >> 4) * Gs : 0;
+    for (int s = 0; s < nst && ok; ++s) {
+      ok = wait_stage();
+      if (!ok) break;
+      const unsigned char* stg = ring + (size_t)(consumed % R) * kStreamStageMax;
+      if (HS || gu)
+        rows_stage<TT, BITS, DBG, GC, true>(Gs, stg, swz, s * span + piece0, nb, nv, lpr == 2, tok, ap, adc, acc, dbg);
+      else
+        rows_stage<TT, BITS, DBG, GC, false>(Gs, stg, swz, s * span + piece0, nb, nv, lpr == 2, tok, ap, adc, acc,
+                                             dbg);
       next_stage();
     }
-    const float* sc = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);
+    if (!ok) break;
     if (gu) {
       // SwiGLU of the half's 16 outputs into shared memory; the second warp
       // of the pair to finish quantises the whole Q8_0 block of h and
       // publishes it (no warp waits for the other)
-      const int orow = chunk * 32 + 16 * half + (lane & 15);
-      const float sv = __ldg(sc + (lane < 16 ? 0 : g.I) + orow);
       float* hbuf = &s_h[pair][k & 1][0][0];
       // the buffer was last used by unit k - 2: its block must be published
       if (k >= 2) {
@@ -561,7 +671,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       }
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
-        const float v = __fmul_rn(sv, acc[t]);
+        const float v = __fmul_rn(rs, acc[t]);
         const float uv = __shfl_down_sync(0xffffffffu, v, 16);
         if (lane < 16 && t < nv) hbuf[t * 32 + 16 * half + lane] = __fmul_rn(__fmul_rn(v, sigmoid_cw(v)), uv);
       }
@@ -586,44 +696,48 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
             if (lane == 0) a.hdc[hrow * g.nbi + chunk] = make_float2(d, __int_as_float(-128 * se));
           }
         }
+        __threadfence();  // every lane: its h stores are visible before the count moves
         __syncwarp();
         if (lane == 0) {
           *(volatile int*)&s_qdone[pair][k & 1] = k + 1;
-          __threadfence();
           atomicAdd(a.h_ready + slot, 1);
         }
       }
       ok = !*abort_f;
     } else {
-      const int o = chunk * 32 + lane;
-      const float sd = __ldg(sc + 2 * g.I + o);
+      // lanes 0 .. rpu_dn - 1: the unit's rows (lane pairs hold the same sum)
+      const int rpu = g.rpu_dn;
+      if (lane < rpu) {
+        float* yc = s_y + ((size_t)(chunk - c0) * n_rows + s_base[slot]) * rpu + lane;
 #pragma unroll
-      for (int t = 0; t < TT; ++t)
-        if (t < nv) a.y[((size_t)s_base[slot] + t) * g.H + o] = __fmul_rn(sd, acc[t]);
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) {
-        __threadfence();
-        last = atomicAdd(a.dn_done + chunk, 1) == n_slots - 1;
-        if (last) __threadfence();
-      }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        // every slot's y rows of this chunk are written: combine (contract C)
-        for (int t = 0; t < T; ++t) {
-          float accc = 0.0f;
-          for (int kk = 0; kk < K; ++kk)
-            accc = __fmaf_rn(s_w[t * K + kk], __ldcg(a.y + (size_t)s_row[t * K + kk] * g.H + o), accc);
-          for (int s = 0; s < S; ++s) accc = __fadd_rn(accc, __ldcg(a.y + ((size_t)s_base[s] + t) * g.H + o));
-          a.out[(size_t)t * g.H + o] = accc;
-        }
+        for (int t = 0; t < TT; ++t)
+          if (t < nv) yc[(size_t)t * rpu] = __fmul_rn(rs, acc[t]);
       }
     }
   }
 
   // copies still in flight (after an abort, the stages never computed)
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  // an owner that gave up before arriving leaves hbar incomplete: waiters give up too (bounded)
+  for (int i = consumed; i < n_real; ++i) stream::mbar_drain(&s_full[warp][i % R], (uint32_t)((i / R) & 1));
+  __syncthreads();
+  if constexpr (HS) {
+    if (*abort_f && threadIdx.x == 0)  // h copies issued, perhaps never waited for
+      for (int i = 0; i < n_slots; ++i)
+        if (s_hclaim[i]) stream::mbar_drain(&s_hbar[i], 0);
+  }
+
+  // ---- combine of this CTA's output chunks (contract C): every slot's y
+  // rows of them are in shared memory
+  if (!*abort_f) {
+    const int rpu = g.rpu_dn, n = T * nch * rpu;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const int t = i / (nch * rpu), rem = i - t * nch * rpu, cl = rem / rpu, rr = rem - cl * rpu;
+      const float* yc = s_y + (size_t)cl * n_rows * rpu + rr;
+      float accc = 0.0f;
+      for (int kk = 0; kk < K; ++kk) accc = __fmaf_rn(s_w[t * K + kk], yc[(size_t)s_row[t * K + kk] * rpu], accc);
+      for (int s = 0; s < S; ++s) accc = __fadd_rn(accc, yc[(size_t)(s_base[s] + t) * rpu]);
+      a.out[(size_t)t * g.H + (size_t)(c0 + cl) * rpu + rr] = accc;
+    }
+  }
 }
 
 // Streaming copy of one expert: one thread per weight block (16 bytes of
@@ -672,32 +786,48 @@ __global__ void prepare_expert_kernel(StreamGeom g, const uint8_t* __restrict__ 
     sc[i] = i < g.I ? gs[i] : (i < 2 * g.I ? us[i - g.I] : ds[i - 2 * g.I]);
 }
 
+// SMs of the current device (cached per device)
+cudaError_t device_sms(int* n) {
+  static int sms[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (sms[dev] == 0 && (e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  *n = sms[dev];
+  return cudaSuccess;
+}
+
+constexpr size_t kStreamDynMax = 224 * 1024;  // 227 KB per block, less the kernel's static shared memory
+
 template <int TT, int BITS, bool DBG, int GC>
 cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
   static int granted[64] = {};
-  static int sms[64] = {};
-  const size_t smem = stream_smem_bytes<TT>(a.g);
-  if (smem > 224 * 1024) return cudaErrorInvalidConfiguration;
-  cudaError_t e = smem_opt_in(expert_stream_kernel<TT, BITS, DBG, GC>, (int)smem, granted);
+  int n_sms = 0;
+  cudaError_t e = device_sms(&n_sms);
   if (e != cudaSuccess) return e;
-  int dev = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if (sms[dev] == 0 && (e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-    return e;
-  // one CTA per SM, all resident at once (the down units wait for gate/up
-  // units of other CTAs); at least as many CTAs as slots, so that a CTA's
-  // range of down units spans at most two slots
-  if (sms[dev] < kMaxSlotsS) return cudaErrorInvalidConfiguration;
-  return launch_pdl(expert_stream_kernel<TT, BITS, DBG, GC>, dim3(sms[dev]), dim3(kSW * 32), smem, st, true, a);
+  const size_t smem = stream_smem_bytes<TT>(a.g, n_sms, a.T * (a.K + a.S));
+  if (smem > kStreamDynMax) return cudaErrorInvalidConfiguration;
+  if ((e = smem_opt_in(expert_stream_kernel<TT, BITS, DBG, GC>, (int)smem, granted)) != cudaSuccess) return e;
+  // one CTA per SM, all resident at once (down units wait for gate/up units
+  // of other CTAs)
+  return launch_pdl(expert_stream_kernel<TT, BITS, DBG, GC>, dim3(n_sms), dim3(kSW * 32), smem, st, true, a);
 }
 
 }  // namespace
 
-bool stream_supported(int hidden, int inter, int bits, int n_tok) {
+bool stream_supported(int hidden, int inter, int bits, int n_tok, int top_k, int n_shared) {
   if (n_tok < 1 || n_tok > kStreamMaxTok || !stream_shape_ok(hidden, inter, bits)) return false;
+  if (top_k < 1 || top_k > kMaxTopK || n_shared < 0 || n_shared > kMaxShared) return false;
+  int n_sms = 0;
+  if (device_sms(&n_sms) != cudaSuccess) return false;
   const StreamGeom g = stream_geom(hidden, inter, bits);
-  constexpr size_t kDyn = 224 * 1024;  // 227 KB per block, less the kernel's static shared memory
-  return stream_smem_bytes<4>(g) <= kDyn && stream_smem_bytes<1>(g) <= kDyn && stream_smem_bytes<2>(g) <= kDyn;
+  const int rows = n_tok * (top_k + n_shared);  // y (and h) rows of the batch
+  const size_t need = n_tok <= 1   ? stream_smem_bytes<1>(g, n_sms, rows)
+                      : n_tok <= 2 ? stream_smem_bytes<2>(g, n_sms, rows)
+                                   : stream_smem_bytes<4>(g, n_sms, rows);
+  return need <= kStreamDynMax;
 }
 
 uint64_t stream_expert_bytes(int hidden, int inter, int bits) { return stream_geom(hidden, inter, bits).expert_bytes; }

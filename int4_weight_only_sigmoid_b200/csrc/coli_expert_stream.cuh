@@ -16,7 +16,12 @@
 //    two halves h = 0, 1 (outputs 32u + 16h .. +15); a half's stage row
 //    r < 16 is gate row 32u + 16h + r, r >= 16 the up row of the same
 //    output; block j of stage s is Q8 block sG + j of the row.
-//  - down unit v (output rows 32v .. 32v+31): stage row r is down row 32v + r.
+//  - down unit v: 32 rows, or 16 rows on lane pairs when every row spans an
+//    even number of whole stages (and so do the gate/up rows).  Single rows:
+//    stage row r is down row 32v + r, block j of stage s is block sG + j.
+//    Lane pairs (unit rows 16v .. 16v+15): stage row p * 16 + r holds piece
+//    p = 0, 1 of down row 16v + r, block j of it is block 2sG + pG + j (the
+//    two lanes of a row fold its blocks in order, piece 0 first).
 //  - G = 16 blocks per stage row for int4, 8 for int8 (fewer when a row is
 //    shorter than one stage).
 //  - then the F32 row scales: gate [I], up [I], down [H].
@@ -40,7 +45,8 @@ struct StreamGeom {
   int g_gu, g_dn;    // blocks per stage row
   int swz_gu, swz_dn;
   int st_gu, st_dn;  // stages per unit
-  int cpu_gu, cpu_dn;  // units per expert (I/32 gate/up, H/32 down)
+  int cpu_gu, cpu_dn;  // units per expert (I/32 gate/up, H/rpu_dn down)
+  int lpr_dn, rpu_dn;  // lanes per down row (1 or 2), down rows per unit (32 / lpr_dn)
   uint32_t sb_gu, sb_dn;  // stage bytes
   uint64_t ub_gu, ub_dn;  // bytes of a gate/up half unit, of a down unit
   uint64_t dn_off, sc_off, expert_bytes;
@@ -74,10 +80,12 @@ __host__ __device__ inline StreamGeom stream_geom(int H, int I, int bits) {
   const int ch_gu = g.g_gu * g.bpb / 16, ch_dn = g.g_dn * g.bpb / 16;  // 16-byte chunks per stage row
   g.swz_gu = (ch_gu < 8 ? ch_gu : 8) - 1;
   g.swz_dn = (ch_dn < 8 ? ch_dn : 8) - 1;
+  g.lpr_dn = (g.nbh % gmax == 0 && g.nbi % (2 * gmax) == 0) ? 2 : 1;
+  g.rpu_dn = 32 / g.lpr_dn;
   g.st_gu = g.nbh / g.g_gu;
-  g.st_dn = g.nbi / g.g_dn;
+  g.st_dn = g.nbi / (g.lpr_dn * g.g_dn);
   g.cpu_gu = I / 32;
-  g.cpu_dn = H / 32;
+  g.cpu_dn = H / g.rpu_dn;
   g.sb_gu = (uint32_t)(32 * g.g_gu * g.bpb);
   g.sb_dn = (uint32_t)(32 * g.g_dn * g.bpb);
   g.ub_gu = (uint64_t)g.st_gu * g.sb_gu;  // one half of a gate/up unit
@@ -100,8 +108,11 @@ __host__ __device__ inline uint64_t stream_chunk_offset(const StreamGeom& g, int
     return (uint64_t)(u * 2 + half) * g.ub_gu + (uint64_t)s * g.sb_gu + (uint64_t)sr * g.g_gu * g.bpb +
            (uint64_t)((c ^ (sr & g.swz_gu)) * 16);
   }
-  const int v = r / 32, sr = r & 31;
-  const int s = b / g.g_dn, j = b - s * g.g_dn;
+  const int v = r / g.rpu_dn, rr = r - v * g.rpu_dn;
+  const int span = g.lpr_dn * g.g_dn;  // blocks of a row in one stage
+  const int s = b / span, jj = b - s * span;
+  const int piece = jj / g.g_dn, j = jj - piece * g.g_dn;
+  const int sr = piece * g.rpu_dn + rr;
   const int c = j * cpb + h;
   return g.dn_off + (uint64_t)v * g.ub_dn + (uint64_t)s * g.sb_dn + (uint64_t)sr * g.g_dn * g.bpb +
          (uint64_t)((c ^ (sr & g.swz_dn)) * 16);

@@ -139,14 +139,12 @@ struct StreamArgs {
   const float* xd;      // [T x H/32]
   int8_t* hpl;          // [rows x I/32 x 32]: h of every (slot, token) row as even / odd byte planes
   float2* hdc;          // [rows x I/32]: (d, -128 * sum of the even plane as int bits)
-  float* y;             // [rows x H]
   float* out;           // [T x H]
   int32_t* h_ready;     // [kStreamMaxSlots] gate/up units done per slot (zero at launch)
-  int32_t* dn_done;     // [H/32] slots done per 32-row chunk of the output (zero at launch)
   int32_t* status;
   int32_t* dbg;         // null, or the partials capture (coli_debug_capture_partials layout)
 };
-bool stream_supported(int hidden, int inter, int bits, int n_tok);
+bool stream_supported(int hidden, int inter, int bits, int n_tok, int top_k, int n_shared);
 uint64_t stream_expert_bytes(int hidden, int inter, int bits);
 cudaError_t launch_prepare_expert(int hidden, int inter, int bits, const uint8_t* gq, const float* gs,
                                   const uint8_t* uq, const float* us, const uint8_t* dq, const float* ds, void* dst,

@@ -53,6 +53,18 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                : "memory");
 }
 
+// Orders this thread's earlier (generic-proxy) view of global memory before
+// its later async-proxy reads of it (a bulk copy of data that other CTAs
+// stored and this thread acquired).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Hint: bring [src, src + bytes) into L2 (16-byte aligned, a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 
 // Wait (bounded, ignoring the abort flag) for a copy the kernel still has in

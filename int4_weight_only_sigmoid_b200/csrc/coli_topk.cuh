@@ -109,5 +109,72 @@ __device__ __forceinline__ void topk_weights(const int (&sel)[kMaxTopK], const f
   }
 }
 
+// Order key of a selection value: a larger float gives a larger unsigned key
+// (-0 and +0 share a key, so that equal floats tie).
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v == 0.0f ? 0.0f : v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The top-k of one token and its weights, by one warp.  Lane l holds the
+// experts l, l + 32, .. (M per lane, E <= 32 M; bias_r[i] = bias of expert
+// l + 32 i, loaded ahead by the caller); each of the K rounds is a warp max
+// of the order keys of score + bias and a warp min of the expert ids that
+// hold it (ties to the lower expert index), so the selection equals
+// warp_select_topk_by's.  Lane k < K writes idx[k] and w[k] (topk_weights'
+// arithmetic: the left-to-right sum of the selected unbiased scores, then
+// w_k = (s_k / denom) * rsf, or s_k * rsf).
+template <int M, int MB, typename ScoreAt>
+__device__ __forceinline__ void warp_route_token(ScoreAt score, const float (&bias_r)[MB], int E, int K, int norm,
+                                                 float rsf, int lane, int32_t* __restrict__ idx,
+                                                 float* __restrict__ w) {
+  static_assert(M <= MB, "bias registers");
+  float sv[M];
+  uint32_t key[M];
+#pragma unroll
+  for (int i = 0; i < M; ++i) {
+    const int e = lane + 32 * i;
+    sv[i] = e < E ? score(e) : 0.0f;
+    key[i] = e < E ? order_key(__fadd_rn(sv[i], bias_r[i])) : 0u;  // 0: below every real key
+  }
+  int mine = 0;
+  for (int k = 0; k < K; ++k) {
+    uint32_t m[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) m[i] = key[i];
+#pragma unroll
+    for (int h = M / 2; h > 0; h >>= 1)
+#pragma unroll
+      for (int i = 0; i < h; ++i) m[i] = max(m[i], m[i + h]);
+    const uint32_t mx = __reduce_max_sync(0xffffffffu, m[0]);
+    int ce = INT_MAX;
+#pragma unroll
+    for (int i = M - 1; i >= 0; --i)
+      if (key[i] == mx) ce = lane + 32 * i;
+    const int ew = __reduce_min_sync(0xffffffffu, ce);
+    if (lane == k) mine = ew;
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+      if (ew == lane + 32 * i) key[i] = 0u;
+  }
+  // the unbiased score of this lane's pick, from the lane that holds it
+  float sk = 0.0f;
+#pragma unroll
+  for (int i = 0; i < M; ++i) {
+    const float v = __shfl_sync(0xffffffffu, sv[i], mine & 31);
+    if ((mine >> 5) == i) sk = v;
+  }
+  if (lane >= K) sk = 0.0f;
+  float denom = 0.0f;
+  for (int j = 0; j < K; ++j) {
+    const float s = __shfl_sync(0xffffffffu, sk, j);
+    denom = j == 0 ? s : __fadd_rn(denom, s);
+  }
+  if (lane < K) {
+    idx[lane] = mine;
+    w[lane] = norm ? __fmul_rn(__fdiv_rn(sk, denom), rsf) : __fmul_rn(sk, rsf);
+  }
+}
+
 }  // namespace topk
 }  // namespace coli

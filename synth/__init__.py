@@ -11,6 +11,8 @@ experts + 1 shared, top-8, from "GLM-5.2-colibri-int4架构解析…", section
 "GLM-5.2的MoE实现"):
 
 * ``tiny``        hidden 256, inter 128, 16 experts, top-4, 1 shared, 8 tokens;
+* ``mid``         hidden 512, inter 1024, 16 experts, top-4, 1 shared, 4 tokens
+                  (rows that span whole 256-byte stages, as in the GLM shape);
                   x ~ N(0,1), W_r ~ N(0,0.02), bias ~ U(-0.1,0.1),
                   experts ~ N(0,0.02); norm_topk_prob, routed_scaling_factor 2.5.
 * ``decode1``     GLM shape, 1 token; W_r ~ N(0,0.006), bias ~ U(-0.05,0.05),
@@ -64,6 +66,8 @@ _GLM = dict(hidden=6144, inter=2048, n_experts=256, top_k=8, n_shared=1, shared_
 CONFIGS = {
     "tiny": dict(_GLM, hidden=256, inter=128, n_experts=16, top_k=4, shared_inter=128,
                  sigma_router=0.02, bias_lo=-0.1, bias_hi=0.1, sigma_expert=0.02, n_tok=8),
+    "mid": dict(_GLM, hidden=512, inter=1024, n_experts=16, top_k=4, shared_inter=1024,
+                sigma_router=0.02, bias_lo=-0.1, bias_hi=0.1, sigma_expert=0.02, n_tok=4),
     "decode1": dict(_GLM, n_tok=1),
     "decode4": dict(_GLM, n_tok=4, x_kind="base+0.5n"),
     "decode16": dict(_GLM, n_tok=16, x_kind="base+0.5n"),

@@ -28,19 +28,21 @@ def _layer(cfg):
 def _geom(H, I, bits):
     bpb = 16 if bits == 4 else 32
     gmax = 256 // bpb
-    g_gu, g_dn = min(gmax, H // 32), min(gmax, I // 32)
-    st_gu, st_dn = (H // 32) // g_gu, (I // 32) // g_dn
+    nbh, nbi = H // 32, I // 32
+    g_gu, g_dn = min(gmax, nbh), min(gmax, nbi)
+    lpr = 2 if nbh % gmax == 0 and nbi % (2 * gmax) == 0 else 1  # lanes per down row
+    st_gu, st_dn = nbh // g_gu, nbi // (lpr * g_dn)
     stage_gu, stage_dn = 32 * g_gu * bpb, 32 * g_dn * bpb
     gu_bytes = (I // 32) * 2 * st_gu * stage_gu
-    dn_bytes = (H // 32) * st_dn * stage_dn
-    return bpb, g_gu, g_dn, st_gu, st_dn, stage_gu, stage_dn, gu_bytes, dn_bytes
+    dn_bytes = (H // (32 // lpr)) * st_dn * stage_dn
+    return bpb, g_gu, g_dn, st_gu, st_dn, stage_gu, stage_dn, gu_bytes, dn_bytes, lpr
 
 
 def _layout_offset(H, I, m, r, b, bits=4, h=0):
     """Byte offset of 16-byte chunk h of block b of row r of matrix m (0 gate,
     1 up, 2 down) in one expert's streaming copy, as include/coli.h and the
     layout header document it."""
-    bpb, g_gu, g_dn, st_gu, st_dn, stage_gu, stage_dn, gu_bytes, _ = _geom(H, I, bits)
+    bpb, g_gu, g_dn, st_gu, st_dn, stage_gu, stage_dn, gu_bytes, _, lpr = _geom(H, I, bits)
     cpb = bpb // 16
     if m < 2:
         swz = min(g_gu * cpb, 8) - 1
@@ -50,38 +52,40 @@ def _layout_offset(H, I, m, r, b, bits=4, h=0):
         c = j * cpb + h
         return ((u * 2 + half) * st_gu + s) * stage_gu + sr * g_gu * bpb + ((c ^ (sr & swz)) * 16)
     swz = min(g_dn * cpb, 8) - 1
-    sr = r % 32
-    s, j = divmod(b, g_dn)
+    rpu = 32 // lpr
+    v, rr = divmod(r, rpu)
+    s, jj = divmod(b, lpr * g_dn)
+    piece, j = divmod(jj, g_dn)
+    sr = piece * rpu + rr
     c = j * cpb + h
-    return gu_bytes + ((r // 32) * st_dn + s) * stage_dn + sr * g_dn * bpb + ((c ^ (sr & swz)) * 16)
+    return gu_bytes + (v * st_dn + s) * stage_dn + sr * g_dn * bpb + ((c ^ (sr & swz)) * 16)
 
 
+@pytest.mark.parametrize("name", ["tiny", "mid"])
 @pytest.mark.parametrize("bits", [4, 8])
-def test_prepare_writes_the_documented_layout(coli, syn, bits):
-    cfg = syn.config("tiny", weight_bits=bits)
+def test_prepare_writes_the_documented_layout(coli, syn, name, bits):
+    cfg = syn.config(name, weight_bits=bits)
     H, I, E, S = cfg["hidden"], cfg["inter"], cfg["n_experts"], cfg["n_shared"]
     L = _layer(cfg)
     prep = _np(L.prepared)
     eb = len(prep) // (E + S)
     assert eb * (E + S) == len(prep) and eb % 256 == 0
-    _, _, _, _, _, _, _, gu_bytes, dn_bytes = _geom(H, I, bits)
+    _, _, _, _, _, _, _, gu_bytes, dn_bytes, lpr = _geom(H, I, bits)
+    assert lpr == (2 if name == "mid" else 1)
+    bpb = 16 if bits == 4 else 32
     for j, ex in enumerate(L.experts + L.shared):
         base = j * eb
         mats = [_np(ex.gate_q).view(np.uint8), _np(ex.up_q).view(np.uint8), _np(ex.down_q).view(np.uint8)]
         for m, q in enumerate(mats):
-            bpb = 16 if bits == 4 else 32
             rows, nb = q.shape[0], q.shape[1] // bpb
-            for r in range(rows):
-                for b in range(nb):
-                    blk = q[r, bpb * b:bpb * (b + 1)]
-                    if bits == 4:
-                        o = base + _layout_offset(H, I, m, r, b)
-                        assert np.array_equal(prep[o:o + 16], blk), (j, m, r, b)
-                    else:  # even elements, then odd elements
-                        o0 = base + _layout_offset(H, I, m, r, b, 8, 0)
-                        o1 = base + _layout_offset(H, I, m, r, b, 8, 1)
-                        assert np.array_equal(prep[o0:o0 + 16], blk[0::2]), (j, m, r, b)
-                        assert np.array_equal(prep[o1:o1 + 16], blk[1::2]), (j, m, r, b)
+            r, b = np.meshgrid(np.arange(rows), np.arange(nb), indexing="ij")
+            blk = q.reshape(rows, nb, bpb)
+            # int4: the block; int8: even elements, then odd elements
+            chunks = [blk] if bits == 4 else [blk[:, :, 0::2], blk[:, :, 1::2]]
+            for h, want in enumerate(chunks):
+                o = base + _layout_offset(H, I, m, r, b, bits, h)
+                got = prep[o[:, :, None] + np.arange(16)]
+                assert np.array_equal(got, want), (j, m, h)
         sc = prep[base + gu_bytes + dn_bytes:base + gu_bytes + dn_bytes + (2 * I + H) * 4].view(np.float32)
         assert bits_equal(sc[:I], _np(ex.gate_s)) and bits_equal(sc[I:2 * I], _np(ex.up_s))
         assert bits_equal(sc[2 * I:], _np(ex.down_s))
@@ -104,6 +108,13 @@ def _check(coli, syn, cfg, n_tok, tokens=None):
 @pytest.mark.parametrize("n_tok", [1, 2, 3, 4])
 def test_stream_tiny(coli, syn, n_tok):
     _check(coli, syn, syn.config("tiny"), n_tok)
+
+
+@pytest.mark.parametrize("n_tok", [1, 2, 3, 4])
+@pytest.mark.parametrize("bits", [4, 8])
+def test_stream_mid_lane_pairs(coli, syn, n_tok, bits):
+    """Down rows split over lane pairs (rows of whole stages)."""
+    _check(coli, syn, syn.config("mid", weight_bits=bits), n_tok)
 
 
 @pytest.mark.parametrize("over", [dict(norm_topk_prob=False), dict(top_k=1), dict(top_k=16), dict(n_shared=0),
