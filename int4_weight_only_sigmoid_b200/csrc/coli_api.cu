@@ -214,11 +214,12 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
 
   int32_t* status = at<int32_t>(ws, W.status);
   const int bits = bits_of(c);
-  if (L->prepared != nullptr && stream_supported(H, I, bits, (int)T, K, S)) {
+  const bool aligned16 = ((uintptr_t)x & 15) == 0;
+  if (L->prepared != nullptr && aligned16 && stream_supported(H, I, bits, (int)T, K, S, E)) {
     // decode on the streaming copy: 2 kernels, the second launched with PDL
     int32_t* ctr = at<int32_t>(ws, W.ctr);
-    CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, xq, xd, clear_status ? status : nullptr,
-                                      ctr, kStreamMaxSlots, st));
+    CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, nullptr, nullptr,
+                                      clear_status ? status : nullptr, ctr, kStreamMaxSlots, st));
     CHECK_LAUNCH(mark(0));
     StreamArgs a{};
     a.prep = static_cast<const unsigned char*>(L->prepared);
@@ -231,8 +232,7 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
     a.rsf = c.routed_scaling_factor;
     a.scores = scores;
     a.bias = L->bias;
-    a.xq = xq;
-    a.xd = xd;
+    a.x = x;
     a.hpl = hq;
     a.hdc = at<float2>(ws, W.hdc);
     a.out = out;
@@ -369,6 +369,7 @@ const char* status_meaning(int32_t code) {
     case 26: return "streaming decode kernel gave up waiting for a slot's h rows in shared memory";
     case 27: return "streaming decode kernel gave up waiting for its warp pair's h buffer";
     case 28: return "streaming decode kernel gave up waiting for a weight stage copy";
+    case 29: return "streaming decode kernel gave up waiting for the routing of the batch";
 
     case kStatusWaitProbe: return "test probe: a wait that nothing completes gave up";
     default: return code >= kStatusTimeoutFirst ? "a bounded wait gave up" : "a device-side check failed";

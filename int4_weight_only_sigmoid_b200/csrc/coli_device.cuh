@@ -123,6 +123,21 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
 }
+// An L2 policy whose lines go first when L2 needs room (data read once).
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// cp_async16 under an L2 policy
+__device__ __forceinline__ void cp_async16_hint(void* smem, const void* gmem, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(smem)),
+               "l"(gmem), "l"(policy)
+               : "memory");
+}
+
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Programmatic dependent launch: wait for the grids this one depends on (a
@@ -144,6 +159,31 @@ __device__ __forceinline__ uint4 ld_dep(const uint4* p) { return __ldcg(p); }
 __device__ __forceinline__ int q8_of(float v, float d) {
   if (d == 0.0f) return 0;
   int q = (int)rintf(__fdiv_rn(v, d));
+  return q < -127 ? -127 : (q > 127 ? 127 : q);
+}
+
+// v / d rounded to nearest from r = RN(1 / d), by Markstein's theorem (P. W.
+// Markstein, "Computation of elementary functions on the IBM RISC System/
+// 6000 processor", IBM J. Res. Dev. 34(1), 1990): with q0 = RN(v r) the
+// remainder v - q0 d is exact in one FMA, and RN(q0 + (v - q0 d) r) is the
+// correctly rounded quotient when nothing overflows or underflows, which
+// holds for 2^-100 <= d <= 2^100 and |v| <= 127 d (a quotient below 1/4 in
+// magnitude, the only case where the remainder can be subnormal, rounds to
+// the integer 0 either way).
+__device__ __forceinline__ bool div_by_recip_ok(float d) { return d >= 0x1p-100f && d <= 0x1p100f; }
+__device__ __forceinline__ float div_by_recip(float v, float d, float r) {
+  const float q0 = __fmul_rn(v, r);
+  return __fmaf_rn(__fmaf_rn(-q0, d, v), r, q0);
+}
+
+// (kept out of line: one copy of the division, off the common path)
+static __device__ __noinline__ float div_rn_outlined(float v, float d) { return __fdiv_rn(v, d); }
+
+// q8_of with one reciprocal per block: r = __frcp_rn(d) (unused unless
+// div_by_recip_ok(d)); the same integer as q8_of(v, d).
+__device__ __forceinline__ int q8_of_r(float v, float d, float r) {
+  if (d == 0.0f) return 0;
+  int q = (int)rintf(div_by_recip_ok(d) ? div_by_recip(v, d, r) : div_rn_outlined(v, d));
   return q < -127 ? -127 : (q > 127 ? 127 : q);
 }
 

@@ -57,6 +57,7 @@ constexpr int kErrHReady = 25;                       // status: gave up waiting 
 constexpr int kErrHStaged = 26;                      // status: gave up waiting for a slot's staged h
 constexpr int kErrHPair = 27;                        // status: gave up waiting for a pair's h buffer
 constexpr int kErrStage = 28;                        // status: gave up waiting for a weight stage
+constexpr int kErrRouting = 29;                      // status: gave up waiting for the routing of the batch
 constexpr int kR = 2;                                // ring stages per warp (8 KB each)
 constexpr int kQ = 4;                                // a warp's queue of down units (> kR)
 
@@ -267,6 +268,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   __shared__ uint32_t s_bits[kMaxExperts / 32], s_tm[kMaxExperts / 4];
   __shared__ int s_bpre[kMaxExperts / 32];
   __shared__ int s_nslots;
+  __shared__ int s_routed;      // the routing tables below are complete
+  __shared__ int s_xready;      // the x planes are complete
   __shared__ int s_dn_next;     // the next of this CTA's down units to hand out
   __shared__ int s_q[kSW][kQ];  // per warp: the down units its cursor took, in order (-1: no more)
   __shared__ float s_h[kPairs][2][TT][32];  // a warp pair's h block, double-buffered by unit
@@ -303,16 +306,35 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   }
   if constexpr (HS)
     for (int i = threadIdx.x; i < kMaxSlotsS; i += blockDim.x) s_hclaim[i] = 0;
+  // the shared slots come first and need no routing: slot s < S is shared
+  // expert s, with all T tokens (rows s T .. s T + T - 1)
+  for (int s = threadIdx.x; s < S; s += blockDim.x) {
+    s_exp[s] = E + s;
+    s_cnt[s] = T;
+    s_base[s] = s * T;
+    for (int t = 0; t < TT; ++t) {
+      s_tok[s][t] = t;
+      if constexpr (DBG) s_drow[s][t] = t * (K + S) + K + s;
+    }
+  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSW * kR; ++i) tc::mbar_init(&s_full[i / kR][i % kR], 1);
     if constexpr (HS)
       for (int i = 0; i < kMaxSlotsS; ++i) tc::mbar_init(&s_hbar[i], 1);
     abort_s = 0;
     s_dn_next = 0;
+    s_routed = 0;
+    s_xready = 0;
     stream::fence_mbar_init();
   }
   __syncthreads();
 
+  // The first T warps route the batch (one token each; warp 0 also
+  // buckets) while the others quantise x and start: a warp whose first unit
+  // is a shared expert's computes that unit before the routing is known.
+  // (The routing is a short serial chain on the critical path: the low warp
+  // ids, which the schedulers favour, take it.)
+  const bool router = warp < T;
   // Gate/up work goes to warp pairs: pair p of this CTA takes units
   // gp, gp + NP, ... (gp = p * G + blockIdx.x), warp 2p the first half of
   // each unit, warp 2p + 1 the second.  Down work: this CTA owns the output
@@ -321,19 +343,23 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   // to whichever warp's cursor asks next; their y rows stay in shared memory
   // and the CTA combines its own chunks at the end.
   const int G = gridDim.x, NP = G * kPairs;
-  const int pair = warp >> 1, half = warp & 1, gp = pair * G + blockIdx.x;
+  // pairs from the top warp down, so that the router warps form the last pairs
+  const int pw = kSW - 1 - warp;
+  const int pair = pw >> 1, half = pw & 1, gp = pair * G + blockIdx.x;
   const int n_shared_gu = S * g.cpu_gu;
   const int c0 = (int)((int64_t)blockIdx.x * g.cpu_dn / G), c1 = (int)((int64_t)(blockIdx.x + 1) * g.cpu_dn / G);
   const int nch = c1 - c0;
+  const bool shared_first = !router && gp < n_shared_gu;
 
   // The warp's stage sequence: its gate/up half units, then the down units
   // it takes.  A cursor walks it R stages ahead of the compute: (phase, unit
   // index k, stage s, the unit's base address); the divisions happen once
-  // per unit.  Before the routing is known only the first unit, if it is a
-  // shared expert's, can stream.
-  int n_gu_mine = 0, n_dn_cta = 0;
+  // per unit.  Until the routing is known a shared-first warp's cursor stops
+  // at the end of its first unit (phase 3) and owes the stages it skipped.
+  int n_gu_mine = shared_first ? 1 : 0, n_dn_cta = 0;  // shared-first: the shared unit, until the routing
+  bool routed = false;
   struct Cursor {
-    int phase, k, s;  // phase 0 gate/up, 1 down, 2 done
+    int phase, k, s;  // phase 0 gate/up, 1 down, 2 done, 3 waiting for the routing
     const unsigned char* base;
   };
   auto unit_base = [&](Cursor& c) {
@@ -363,7 +389,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     }
   };
   Cursor pc{0, 0, 0, nullptr};
-  int issued = 0, n_real = 0;  // stages issued (past the end: empty), and real copies among them
+  const uint64_t l2pol = l2_evict_first();  // the weights are read once per forward: first out of L2
+  int issued = 0, n_real = 0, owed = 0;  // stages issued (past the end: empty), real copies, stages owed
   // lane 0: the cursor's stage into ring slot issued % R, one bulk copy
   // completing on the slot's mbarrier
   auto copy_stage = [&]() {
@@ -372,146 +399,180 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       if (lane == 0) {
         uint64_t* bar = &s_full[warp][issued % R];
         stream::mbar_expect_tx(bar, bytes);
-        stream::bulk_g2s(ring + (size_t)(issued % R) * kStreamStageMax, pc.base + (uint64_t)pc.s * bytes, bytes, bar);
+        stream::bulk_g2s_hint(ring + (size_t)(issued % R) * kStreamStageMax, pc.base + (uint64_t)pc.s * bytes, bytes,
+                              bar, l2pol);
       }
       ++n_real;
     }
     ++issued;
   };
   auto issue = [&]() {  // copy, then move the cursor on
+    if (pc.phase == 3) {
+      ++owed;
+      return;
+    }
     copy_stage();
     if (pc.phase < 2 && ++pc.s == (pc.phase == 0 ? g.st_gu : g.st_dn)) {
       pc.s = 0;
       ++pc.k;
-      unit_base(pc);
+      if (!routed)
+        pc.phase = 3;  // the routing is not known yet
+      else
+        unit_base(pc);
     }
   };
 
-  // shared experts' first stages stream while the router finishes (within
-  // the warp's first unit: what follows depends on the routing)
-  int pre = 0;
-  if (gp < n_shared_gu) {
-    n_gu_mine = 1;  // provisional: the first unit
-    unit_base(pc);
-    for (; pre < R && pre < g.st_gu; ++pre) {
-      copy_stage();
-      ++pc.s;
+  if (!router) {
+    // x planes, from the layer input (the Q8_0 of the router kernel,
+    // quotients from one reciprocal per block): block b of token t ->
+    // even / odd byte planes and (d, c16 = -128 * sum of the even plane)
+    // eight lanes per block (lane m: elements 4m .. 4m + 3), four blocks per
+    // warp and step; lane m writes bytes 2m, 2m + 1 of both planes
+    const int sub = lane >> 3, m = lane & 7;
+    for (int i = (warp - T) * 4 + sub; i < T * g.nbh; i += (kSW - T) * 4) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(a.x + (size_t)i * 32) + m);
+      float amax = fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w)));
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float d = __fdiv_rn(amax, 127.0f), r = __frcp_rn(d);
+      const int q0 = q8_of_r(f.x, d, r), q1 = q8_of_r(f.y, d, r), q2 = q8_of_r(f.z, d, r), q3 = q8_of_r(f.w, d, r);
+      unsigned short* pl = reinterpret_cast<unsigned short*>(xpl + 2 * i);
+      pl[m] = (unsigned short)((q0 & 0xFF) | (q2 & 0xFF) << 8);      // even plane
+      pl[8 + m] = (unsigned short)((q1 & 0xFF) | (q3 & 0xFF) << 8);  // odd plane
+      int se = q0 + q2;
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
+      if (m == 0) xdc[i] = make_float2(d, __int_as_float(-128 * se));
+    }
+    asm volatile("bar.sync 2, %0;" ::"r"((kSW - T) * 32) : "memory");  // the non-router warps
+    if (threadIdx.x == T * 32) {
+      __threadfence_block();
+      *(volatile int*)&s_xready = 1;
     }
   }
 
-  // the correction bias is a layer constant: into registers before the wait
-  float bias_r[kMaxExperts / 32];
-#pragma unroll
-  for (int i = 0; i < kMaxExperts / 32; ++i) {
-    const int e = lane + 32 * i;
-    bias_r[i] = warp < T && e < E ? __ldg(a.bias + e) : 0.0f;
-  }
 
-  pdl_wait();  // scores, the Q8_0 of x and the cleared counters are complete
-  pdl_launch_dependents();
+  if (shared_first) {
+    unit_base(pc);  // k = 0: the warp's shared unit
+    for (int i = 0; i < R; ++i) issue();
+  }
 
   // ---- routing of the batch (every CTA, identical results) -------------
-  if (warp < T) {
-    const float* st = a.scores + (size_t)warp * E;
+  if (router) {
+    const int tr = warp;  // this warp's token
+    // the correction bias is a layer constant: into registers before the wait
+    float bias_r[kMaxExperts / 32];
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+      const int e = lane + 32 * i;
+      bias_r[i] = e < E ? __ldg(a.bias + e) : 0.0f;
+    }
+    pdl_wait();  // the scores and the cleared counters are complete
+    const float* st = a.scores + (size_t)tr * E;
     auto sc = [st](int e) { return ld_dep(st + e); };
     if (E <= 256)
-      topk::warp_route_token<8>(sc, bias_r, E, K, a.norm, a.rsf, lane, s_idx + warp * K, s_w + warp * K);
+      topk::warp_route_token<8>(sc, bias_r, E, K, a.norm, a.rsf, lane, s_idx + tr * K, s_w + tr * K);
     else
-      topk::warp_route_token<kMaxExperts / 32>(sc, bias_r, E, K, a.norm, a.rsf, lane, s_idx + warp * K,
-                                               s_w + warp * K);
-  }
-  // x planes: block b of token t -> even / odd byte planes and (d, c16)
-  for (int i = threadIdx.x; i < T * g.nbh; i += blockDim.x) {
-    const int t = i / g.nbh, b = i - t * g.nbh;
-    const uint4* src = reinterpret_cast<const uint4*>(a.xq + (size_t)t * g.H + 32 * b);
-    const uint4 a0 = ld_dep(src), a1 = ld_dep(src + 1);
-    uint4 e, o;
-    split_even_odd(a0.x, a0.y, e.x, o.x);
-    split_even_odd(a0.z, a0.w, e.y, o.y);
-    split_even_odd(a1.x, a1.y, e.z, o.z);
-    split_even_odd(a1.z, a1.w, e.w, o.w);
-    xpl[2 * i] = e;
-    xpl[2 * i + 1] = o;
-    xdc[i] = make_float2(ld_dep(a.xd + i), __int_as_float(-128 * even_plane_sum(e)));
-  }
-  __syncthreads();
-  if (warp == 0) {
-    // bucketing: the chosen experts (bit e of s_bits) and, per expert, the
-    // tokens that chose it (byte e & 3 of s_tm[e >> 2], bit t)
-    const int n_pairs = T * K;
-    for (int p = lane; p < n_pairs; p += 32) {
-      const int e = s_idx[p], t = p / K;
+      topk::warp_route_token<kMaxExperts / 32>(sc, bias_r, E, K, a.norm, a.rsf, lane, s_idx + tr * K,
+                                               s_w + tr * K);
+    __syncwarp();
+    // the chosen experts (bit e of s_bits) and, per expert, the tokens that
+    // chose it (byte e & 3 of s_tm[e >> 2], bit t)
+    if (lane < K) {
+      const int e = s_idx[tr * K + lane];
       atomicOr(&s_bits[e >> 5], 1u << (e & 31));
-      atomicOr(&s_tm[e >> 2], 1u << ((e & 3) * 8 + t));
+      atomicOr(&s_tm[e >> 2], 1u << ((e & 3) * 8 + tr));
     }
-    __syncwarp();
-    auto tm_of = [&](int e) { return (s_tm[e >> 2] >> ((e & 3) * 8)) & 0xFFu; };
-    // lane l: the experts 32l .. 32l+31; slots in ascending expert id after
-    // the shared ones, rows in slot order, a slot's rows in token order
-    const int nw = (E + 31) / 32;
-    const uint32_t bits = lane < nw ? s_bits[lane] : 0u;
-    int rows = 0;
-    for (uint32_t bb = bits; bb; bb &= bb - 1) rows += __popc(tm_of(32 * lane + __ffs(bb) - 1));
-    const int c = __popc(bits);
-    int ci = c, ri = rows;
+    if (T > 1) asm volatile("bar.sync 1, %0;" ::"r"(T * 32) : "memory");  // the router warps
+    if (warp == 0) {
+      __syncwarp();
+      auto tm_of = [&](int e) { return (s_tm[e >> 2] >> ((e & 3) * 8)) & 0xFFu; };
+      // lane l: the experts 32l .. 32l+31; slots in ascending expert id after
+      // the shared ones, rows in slot order, a slot's rows in token order
+      const int nw = (E + 31) / 32;
+      const uint32_t bits = lane < nw ? s_bits[lane] : 0u;
+      int rows = 0;
+      for (uint32_t bb = bits; bb; bb &= bb - 1) rows += __popc(tm_of(32 * lane + __ffs(bb) - 1));
+      const int c = __popc(bits);
+      int ci = c, ri = rows;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int yc = __shfl_up_sync(0xffffffffu, ci, o), yr = __shfl_up_sync(0xffffffffu, ri, o);
-      if (lane >= o) {
-        ci += yc;
-        ri += yr;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yc = __shfl_up_sync(0xffffffffu, ci, o), yr = __shfl_up_sync(0xffffffffu, ri, o);
+        if (lane >= o) {
+          ci += yc;
+          ri += yr;
+        }
+      }
+      if (lane < nw) s_bpre[lane] = ci - c;
+      if (lane == 31) s_nslots = S + ci;
+      int r = S + ci - c, base = S * T + ri - rows;
+      for (uint32_t bb = bits; bb; bb &= bb - 1) {
+        const int e = 32 * lane + __ffs(bb) - 1;
+        const uint32_t m = tm_of(e);
+        s_exp[r] = e;
+        s_cnt[r] = __popc(m);
+        s_base[r] = base;
+        int pos = 0;
+#pragma unroll
+        for (int t = 0; t < TT; ++t)
+          if ((m >> t) & 1u) s_tok[r][pos++] = t;
+        base += __popc(m);
+        ++r;
+      }
+      __syncwarp();
+      // each (token, rank) pair: the row of its expert's output
+      for (int p = lane; p < T * K; p += 32) {
+        const int e = s_idx[p], t = p / K, w32 = e >> 5;
+        const int slot = S + s_bpre[w32] + __popc(s_bits[w32] & ((1u << (e & 31)) - 1u));
+        const int pos = __popc(tm_of(e) & ((1u << t) - 1u));
+        s_row[p] = s_base[slot] + pos;
+        if constexpr (DBG) s_drow[slot][pos] = t * (K + S) + (p - t * K);  // rank p - tK of token t
+      }
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        *(volatile int*)&s_routed = 1;
       }
     }
-    if (lane < nw) s_bpre[lane] = ci - c;
-    if (lane == 31) s_nslots = S + ci;
-    int r = S + ci - c, base = S * T + ri - rows;
-    for (uint32_t bb = bits; bb; bb &= bb - 1) {
-      const int e = 32 * lane + __ffs(bb) - 1;
-      const uint32_t m = tm_of(e);
-      s_exp[r] = e;
-      s_cnt[r] = __popc(m);
-      s_base[r] = base;
-      int pos = 0;
-#pragma unroll
-      for (int t = 0; t < TT; ++t)
-        if ((m >> t) & 1u) s_tok[r][pos++] = t;
-      base += __popc(m);
-      ++r;
-    }
-    for (int sh = lane; sh < S; sh += 32) {
-      s_exp[sh] = E + sh;
-      s_cnt[sh] = T;
-      s_base[sh] = sh * T;
-      for (int t = 0; t < TT; ++t) {
-        s_tok[sh][t] = t;
-        if constexpr (DBG) s_drow[sh][t] = t * (K + S) + K + sh;
+  }
+  // The routing is known to this warp once s_routed is set (bounded wait);
+  // then the counts, and the cursor's next unit.
+  auto await_routing = [&]() -> bool {
+    pdl_wait();
+    pdl_launch_dependents();
+    int got = 0;
+    if (lane == 0) {
+      const long long t0 = clock64();
+      while (!*abort_f) {
+        if (*(volatile int*)&s_routed && *(volatile int*)&s_xready) {
+          got = 1;
+          break;
+        }
+        if (clock64() - t0 > tc::kSpinCycles) {
+          *abort_f = 1;
+          atomicExch(a.status, kErrRouting);
+          break;
+        }
+        __nanosleep(32);
       }
+      __threadfence_block();
     }
-    __syncwarp();
-    // each (token, rank) pair: the row of its expert's output
-    for (int p = lane; p < n_pairs; p += 32) {
-      const int e = s_idx[p], t = p / K, w32 = e >> 5;
-      const int slot = S + s_bpre[w32] + __popc(s_bits[w32] & ((1u << (e & 31)) - 1u));
-      const int pos = __popc(tm_of(e) & ((1u << t) - 1u));
-      s_row[p] = s_base[slot] + pos;
-      if constexpr (DBG) s_drow[slot][pos] = t * (K + S) + (p - t * K);  // rank p - tK of token t
+    if (!__shfl_sync(0xffffffffu, got, 0)) return false;
+    const int n_slots = s_nslots;
+    const int n_gu = n_slots * g.cpu_gu;
+    n_gu_mine = gp < n_gu ? (n_gu - gp + NP - 1) / NP : 0;
+    n_dn_cta = n_slots * nch;
+    routed = true;
+    if (!shared_first) {
+      unit_base(pc);  // the cursor's first unit
+      for (int i = 0; i < R; ++i) issue();
+    } else if (pc.phase == 3) {
+      pc.phase = 0;  // past the shared unit: on to the next
+      unit_base(pc);
+      for (; owed > 0; --owed) issue();
     }
-  }
-  __syncthreads();
-
-  const int n_slots = s_nslots;
-  const int n_gu = n_slots * g.cpu_gu;
-  n_gu_mine = gp < n_gu ? (n_gu - gp + NP - 1) / NP : 0;
-  n_dn_cta = n_slots * nch;
-
-  if (pre == 0) {
-    unit_base(pc);  // the cursor's first unit, now that the counts are known
-  } else if (pc.s == g.st_gu) {
-    pc.s = 0;  // the first unit was streamed whole before the routing: on to the next
-    pc.k = 1;
-    unit_base(pc);
-  }
-  for (int i = pre; i < R; ++i) issue();
+    return true;
+  };
 
   int consumed = 0;
   bool ok = true;
@@ -533,6 +594,10 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   // copy of the unrolled block loop.
   int acq_slot = -1;  // the last slot whose h this warp has acquired
   for (int k = 0; ok; ++k) {
+    if (!routed && (k > 0 || !shared_first) && !await_routing()) {
+      ok = false;
+      break;
+    }
     const bool gu = k < n_gu_mine;
     int slot, chunk, nv, nst, Gs, swz, nb, lpr = 1;
     const uint4* ap;
@@ -698,6 +763,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
         }
         __threadfence();  // every lane: its h stores are visible before the count moves
         __syncwarp();
+        pdl_wait();  // (a shared unit done before the routing) the router kernel has cleared the counts
         if (lane == 0) {
           *(volatile int*)&s_qdone[pair][k & 1] = k + 1;
           atomicAdd(a.h_ready + slot, 1);
@@ -721,7 +787,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   __syncthreads();
   if constexpr (HS) {
     if (*abort_f && threadIdx.x == 0)  // h copies issued, perhaps never waited for
-      for (int i = 0; i < n_slots; ++i)
+      for (int i = 0; i < kMaxSlotsS; ++i)
         if (s_hclaim[i]) stream::mbar_drain(&s_hbar[i], 0);
   }
 
@@ -817,7 +883,7 @@ cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-bool stream_supported(int hidden, int inter, int bits, int n_tok, int top_k, int n_shared) {
+bool stream_supported(int hidden, int inter, int bits, int n_tok, int top_k, int n_shared, int n_experts) {
   if (n_tok < 1 || n_tok > kStreamMaxTok || !stream_shape_ok(hidden, inter, bits)) return false;
   if (top_k < 1 || top_k > kMaxTopK || n_shared < 0 || n_shared > kMaxShared) return false;
   int n_sms = 0;
@@ -827,6 +893,7 @@ bool stream_supported(int hidden, int inter, int bits, int n_tok, int top_k, int
   const size_t need = n_tok <= 1   ? stream_smem_bytes<1>(g, n_sms, rows)
                       : n_tok <= 2 ? stream_smem_bytes<2>(g, n_sms, rows)
                                    : stream_smem_bytes<4>(g, n_sms, rows);
+  (void)n_experts;
   return need <= kStreamDynMax;
 }
 

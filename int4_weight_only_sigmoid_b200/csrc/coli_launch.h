@@ -135,8 +135,7 @@ struct StreamArgs {
   float rsf;
   const float* scores;  // [T x E] (router_decode)
   const float* bias;
-  const int8_t* xq;     // [T x H] Q8_0 of x (router_decode)
-  const float* xd;      // [T x H/32]
+  const float* x;       // [T x H] the layer input
   int8_t* hpl;          // [rows x I/32 x 32]: h of every (slot, token) row as even / odd byte planes
   float2* hdc;          // [rows x I/32]: (d, -128 * sum of the even plane as int bits)
   float* out;           // [T x H]
@@ -144,7 +143,8 @@ struct StreamArgs {
   int32_t* status;
   int32_t* dbg;         // null, or the partials capture (coli_debug_capture_partials layout)
 };
-bool stream_supported(int hidden, int inter, int bits, int n_tok, int top_k, int n_shared);
+bool stream_supported(int hidden, int inter, int bits, int n_tok, int top_k, int n_shared, int n_experts);
+
 uint64_t stream_expert_bytes(int hidden, int inter, int bits);
 cudaError_t launch_prepare_expert(int hidden, int inter, int bits, const uint8_t* gq, const float* gs,
                                   const uint8_t* uq, const float* us, const uint8_t* dq, const float* ds, void* dst,

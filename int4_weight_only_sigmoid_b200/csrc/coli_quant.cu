@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(256) quantize_act_q8_kernel(const float* __res
   const float v = x[blk * 32 + lane];
   const float amax = warp_max(fabsf(v));
   const float dd = __fdiv_rn(amax, 127.0f);
-  q[blk * 32 + lane] = (int8_t)q8_of(v, dd);
+  q[blk * 32 + lane] = (int8_t)q8_of_r(v, dd, __frcp_rn(dd));  // the quotient the streaming kernel uses
   if (lane == 0) d[blk] = dd;
 }
 

@@ -203,14 +203,19 @@ __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restr
   const int e0 = blockIdx.x * 2;
   const int nq = H / 4;
   const bool stage_x = n_tok <= kStageTok;
-  for (int i = threadIdx.x; i < 2 * nq; i += blockDim.x) {
-    const int r = i / nq, j = i - r * nq;
-    if (e0 + r < E) cp_async16(wsm + i, wr + (size_t)(e0 + r) * H + 4 * j);
+  {
+    // the router rows are read once per forward: first out of L2
+    const uint64_t pol = l2_evict_first();
+    for (int i = threadIdx.x; i < 2 * nq; i += blockDim.x) {
+      const int r = i / nq, j = i - r * nq;
+      if (e0 + r < E) cp_async16_hint(wsm + i, wr + (size_t)(e0 + r) * H + 4 * j, pol);
+    }
   }
   if (stage_x)
     for (int i = threadIdx.x; i < n_tok * nq; i += blockDim.x) cp_async16(wsm + 2 * nq + i, x + 4 * (size_t)i);
-  // the Q8_0 of x for the expert kernels: one warp per 32-element block
-  for (int j = blockIdx.x * 8 + warp; j < n_tok * (H / 32); j += gridDim.x * 8) {
+  // the Q8_0 of x for the expert kernels (unless they make their own): one
+  // warp per 32-element block
+  for (int j = blockIdx.x * 8 + warp; xq != nullptr && j < n_tok * (H / 32); j += gridDim.x * 8) {
     const float v = x[(size_t)j * 32 + lane];
     const float d = __fdiv_rn(warp_max(fabsf(v)), 127.0f);
     xq[(size_t)j * 32 + lane] = (int8_t)q8_of(v, d);

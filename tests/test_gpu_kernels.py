@@ -78,6 +78,30 @@ def test_quantize_act_q8_bit_exact(coli, ora, syn, n, dim):
     assert bits_equal(_np(d), do)
 
 
+def test_quantize_act_q8_quotients_near_half_integers(coli, ora):
+    """Blocks whose elements sit a few ulps either side of (k + 1/2) d, so
+    that the integer codes hang on the last bit of each quotient v / d; the
+    scales span 2^-90 .. 2^90 (the quotient from one reciprocal per block is
+    exact there) plus subnormal-range blocks (plain division)."""
+    import torch
+    rng = np.random.default_rng(0x51)
+    blocks = []
+    for b in range(4096):
+        e = int(rng.integers(-90, 91)) if b % 8 else int(rng.integers(-140, -120))
+        amax = np.float32(np.ldexp(1.0 + rng.random(), e))
+        d = np.float32(amax / np.float32(127.0))
+        k = rng.integers(-127, 127, size=31).astype(np.float32) + np.float32(0.5)
+        v = (k * d).astype(np.float32)
+        v = (v.view(np.int32) + rng.integers(-3, 4, size=31).astype(np.int32)).view(np.float32)
+        v = np.clip(v, -amax, amax).astype(np.float32)
+        blocks.append(np.concatenate([[amax], v]).astype(np.float32))
+    x = np.stack(blocks).reshape(64, -1).astype(np.float32)
+    q, d = coli.quantize_act_q8(torch.from_numpy(x).cuda())
+    qo, do = ora.quantize_act_q8(x)
+    assert bits_equal(_np(d), do)
+    assert bits_equal(_np(q), qo)
+
+
 # --------------------------------------------------------------------------
 # integer partial sums
 
