@@ -203,21 +203,27 @@ coli_status coli_rmsnorm(const float* x, int64_t n_tok, int64_t dim, float eps, 
 
 /* The layer's streaming copy ([H] "已实现的功能", batched MoE: one read of
  * an expert per layer; [D] "引擎是如何工作的": an expert's matrices are
- * read as one contiguous piece).  The same packed int4 bytes and F32 row
- * scales as the row-major weights, reordered once so that the decode
- * kernel moves each step of its work (16 KB: 32 gate + 32 up rows x 16
- * blocks, or 32 down rows x 32 blocks, the blocks of a row XOR-rotated)
- * with one bulk copy.  Per expert (routed 0..n_experts-1, then shared):
- * gate/up units, down units, then the scales; GLM-5.2 shape: 18.9 MB per
- * expert, 4.86 GB per layer, the size of the row-major weights.
- * coli_moe_prepared_bytes: bytes for the layer (0 if cfg is invalid or the
- * shape has no streaming layout: hidden and inter multiples of 128,
- * hidden/32 a multiple of 16 or 4 or 8, inter/32 a multiple of 32 or 4, 8,
- * 16).  coli_moe_prepare: writes the copy of `layer`'s weights into
- * `prepared` (device, 256-byte aligned, `bytes` >= coli_moe_prepared_bytes;
- * caller-owned), stream-ordered; the row-major weights are only read.
- * Re-run it after changing the weights.  Store the pointer in
- * layer->prepared to use it. */
+ * read as one contiguous piece).  The same weight bytes and F32 row scales
+ * as the row-major weights, reordered once so that the decode kernel moves
+ * each step of a warp's work with one bulk copy: a step ("stage") is 32
+ * rows x 256 bytes (8 KB: 16 blocks of packed int4, or 8 blocks of int8
+ * stored as their even then odd elements), the 16-byte chunks of a stage row
+ * XOR-rotated by the row index.  Gate/up: half units of 16 gate rows and
+ * the 16 matching up rows, hidden/32/16 stages each.  Down: units of 32
+ * rows, or of 16 rows whose two 256-byte pieces per stage sit in stage rows
+ * r and r + 16 when every row spans an even number of whole stages (the
+ * GLM-5.2 shape).  Per expert (routed 0..n_experts-1, then shared): gate/up
+ * half units, down units, then the scales (gate, up, down), padded to 256
+ * bytes; GLM-5.2 shape: 18.9 MB per expert, 4.86 GB per layer, the size of
+ * the row-major weights.  coli_moe_prepared_bytes: bytes for the layer (0
+ * if cfg is invalid or the shape has no streaming layout: hidden and inter
+ * multiples of 128, and each of hidden/32 and inter/32 either a multiple of
+ * the blocks of a 256-byte row (16 int4, 8 int8) or a power-of-two number
+ * of 16-byte chunks below it).  coli_moe_prepare: writes the copy of
+ * `layer`'s weights into `prepared` (device, 256-byte aligned, `bytes` >=
+ * coli_moe_prepared_bytes; caller-owned), stream-ordered; the row-major
+ * weights are only read.  Re-run it after changing the weights.  Store the
+ * pointer in layer->prepared to use it. */
 size_t coli_moe_prepared_bytes(const coli_moe_config* cfg);
 coli_status coli_moe_prepare(const coli_moe_layer* layer, void* prepared, size_t bytes, void* stream);
 
