@@ -106,7 +106,7 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Workspace {
   size_t xq, xd, scores, idx, w, counts, offsets, perm, inv, slots, n_slots, status, tiles, n_tiles, hq, hd, xr, hdc,
-      ctr, y, xn, xa, xb, total;
+      xdc, ctr, y, xn, xa, xb, total;
 };
 
 Workspace layout(const coli_moe_config& c, int64_t T) {
@@ -144,6 +144,7 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   // (d, c16) of every h block and its counters
   const bool sm = T <= kStreamMaxTok;
   L.hdc = take(sm ? rows * (I / 32) * 8 : 0);
+  L.xdc = take(sm ? T * (H / 32) * 8 : 0);  // with xq: the x planes the router kernel writes for > 2 tokens
   L.ctr = take(sm ? (size_t)kStreamMaxSlots * 4 : 0);
   L.y = take(rows * H * 4);
   L.xn = take(T * H * 4);
@@ -218,8 +219,13 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   if (L->prepared != nullptr && aligned16 && stream_supported(H, I, bits, (int)T, K, S, E)) {
     // decode on the streaming copy: 2 kernels, the second launched with PDL
     int32_t* ctr = at<int32_t>(ws, W.ctr);
+    // up to 2 tokens the streaming kernel quantises x itself (so that the
+    // shared expert starts before the router kernel ends); more tokens take
+    // the router kernel's planes
+    int8_t* xpl = T > 2 ? xq : nullptr;
+    float2* xdcp = T > 2 ? at<float2>(ws, W.xdc) : nullptr;
     CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, nullptr, nullptr,
-                                      clear_status ? status : nullptr, ctr, kStreamMaxSlots, st));
+                                      clear_status ? status : nullptr, ctr, kStreamMaxSlots, st, xpl, xdcp));
     CHECK_LAUNCH(mark(0));
     StreamArgs a{};
     a.prep = static_cast<const unsigned char*>(L->prepared);
@@ -233,6 +239,8 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
     a.scores = scores;
     a.bias = L->bias;
     a.x = x;
+    a.xpl_g = xpl;
+    a.xdc_g = xdcp;
     a.hpl = hq;
     a.hdc = at<float2>(ws, W.hdc);
     a.out = out;

@@ -1,4 +1,4 @@
-// coli_expert_stream.cu -- the expert part of a decode batch (n_tok <= 4)
+// coli_expert_stream.cu -- the expert part of a decode batch (n_tok <= 8)
 // in one persistent kernel, reading the layer's streaming copy
 // (coli_expert_stream.cuh, made by coli_moe_prepare):
 //
@@ -75,12 +75,20 @@ template <int TT>
 struct StreamHStaged {
   static constexpr bool value = TT <= 2;
 };
+// Batches of 3-4 tokens stage each slot's h rows too, in a ring of kHRing
+// slot buffers (the slots of a CTA's down units come in ascending order).
+constexpr int kHRing = 4;
+template <int TT>
+struct StreamHRing {
+  static constexpr bool value = TT == 4;
+};
 
 template <int TT>
 __host__ __device__ inline size_t stream_smem_bytes(const StreamGeom& g, int n_sms, int n_rows) {
   const size_t ring = (size_t)kSW * kR * kStreamStageMax;  // 8 KB stages
   const size_t xs = (size_t)TT * g.nbh * 40;               // x planes (32 B) + (d, c16) per block
-  const size_t hs = StreamHStaged<TT>::value ? (size_t)n_rows * g.nbi * 40 : 0;  // h planes + (d, c16)
+  const size_t hs = StreamHStaged<TT>::value ? (size_t)n_rows * g.nbi * 40              // h planes + (d, c16)
+                    : StreamHRing<TT>::value  ? (size_t)kHRing * TT * g.nbi * 40 : 0;  // per slot buffer
   return 1024 + ring + xs + stream_y_bytes(g, n_sms, n_rows) + hs;
 }
 
@@ -255,6 +263,121 @@ __device__ __forceinline__ void rows_stage(int Grt, const unsigned char* st, int
   }
 }
 
+// Batches of more than two tokens fold on the tensor cores: mma.sync
+// m16n8k32 (s8 x s8 -> s32) over 16 weight rows x one Q8 block x 8 token
+// columns.  Lane (g, c) = (lane / 4, lane % 4) supplies word c of rows g and
+// g + 8 of the block: for int4 its even nibbles as 16 q (a0, a1: the k slots
+// 4c .. 4c + 3 are elements 8c, 8c + 2, 8c + 4, 8c + 6) and its odd nibbles
+// (a2, a3: k slots 16 + 4c .. are elements 8c + 1, ..); for int8 the words
+// c of the block's even and odd planes.  The activation columns in the same
+// k order are word c of the token's even and odd byte planes, i.e. the
+// staged planes as they are.  The accumulators start at 0x4B400000, so that
+// D read as a float is 1.5 2^23 + 16 isum (int4) or + isum (int8), exact.
+template <int TT>
+struct StreamMma {
+  static constexpr bool value = TT >= 4;
+};
+
+__device__ __forceinline__ void mma_s8_16x8x32(uint32_t (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  constexpr uint32_t m = 0x4B400000u;
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %11, %12, %13};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(m), "r"(m), "r"(m), "r"(m));
+}
+
+template <int BITS>
+__device__ __forceinline__ float isum_of_acc(uint32_t d) {
+  if constexpr (BITS == 4) return __fmaf_rn(__uint_as_float(d), 0.0625f, -786432.0f);  // (1.5 2^23 + 16 s) / 16 - 1.5 2^19
+  return __fadd_rn(__uint_as_float(d), -12582912.0f);
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// One stage of the tensor-core fold.  Stage rows 16 rg + g and 16 rg + g + 8
+// (rg = 0, 1) of block j against token columns; acc[rg][i]: i = 0 (row g,
+// column 2c), 1 (g, 2c + 1), 2 (g + 8, 2c), 3 (g + 8, 2c + 1).  mode 0: the
+// two row groups are separate rows (gate / up, or 32 down rows); mode 1:
+// they are the two pieces of the same 16 rows (blocks b0 .. b0 + G - 1, then
+// b0 + G ..), folded in that order into acc[0].  Activations: row rB of the
+// plane array for the lane's B column (g), rows rF0, rF1 for its fold
+// columns (2c, 2c + 1); XS: shared memory, else global through L1.
+template <int BITS, bool DBG, int GC, bool XS>
+__device__ __forceinline__ void rows_stage_mma(int Grt, const unsigned char* st, int swz, int b0, int nb, int mode,
+                                               int rB, int rF0, int rF1, const uint4* xpl, const float2* xdc,
+                                               float (&acc)[2][4], int32_t* const (&dbg)[2][4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  constexpr int cpb = BITS / 4;
+  const int G = GC > 0 ? GC : Grt;
+  const uint32_t sbase = tc::smem_u32(st);
+  const uint32_t rowb = (uint32_t)(G * cpb * 16);  // bytes of a stage row
+  auto wload = [&](int r, int chunk) -> uint32_t {   // word c of 16-byte chunk `chunk` of stage row r
+    return lds32(sbase + (uint32_t)r * rowb + (uint32_t)((chunk ^ (r & swz)) << 4) + 4u * c);
+  };
+  auto xw = [&](int row, int b, int h) -> uint32_t {  // word c of plane h of block b of activation row `row`
+    const uint4* p = xpl + 2 * ((size_t)row * nb + b) + h;
+    if constexpr (XS) return lds32(tc::smem_u32(p) + 4u * c);
+    return reinterpret_cast<const uint32_t*>(p)[c];
+  };
+  auto xd = [&](int row, int b) -> float {
+    const float2* p = xdc + (size_t)row * nb + b;
+    if constexpr (XS) return lds64f(tc::smem_u32(p)).x;
+    return p->x;
+  };
+  auto step = [&](int rg, int j, int b, float (&ac)[4], int32_t* const (&db)[4]) {
+    uint32_t a0, a1, a2, a3;
+    const int r0 = 16 * rg + g, r1 = r0 + 8;
+    if constexpr (BITS == 4) {
+      const uint32_t w0 = wload(r0, j), w1 = wload(r1, j);
+      a0 = (w0 << 4) & 0xF0F0F0F0u;
+      a1 = (w1 << 4) & 0xF0F0F0F0u;
+      a2 = w0 & 0xF0F0F0F0u;
+      a3 = w1 & 0xF0F0F0F0u;
+    } else {
+      a0 = wload(r0, 2 * j);
+      a1 = wload(r1, 2 * j);
+      a2 = wload(r0, 2 * j + 1);
+      a3 = wload(r1, 2 * j + 1);
+    }
+    uint32_t d[4];
+    mma_s8_16x8x32(d, a0, a1, a2, a3, xw(rB, b, 0), xw(rB, b, 1));
+    const float dx0 = xd(rF0, b), dx1 = xd(rF1, b);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float s = isum_of_acc<BITS>(d[i]);
+      if constexpr (DBG)
+        if (db[i] != nullptr) db[i][b] = (int32_t)s;
+      ac[i] = __fmaf_rn((i & 1) ? dx1 : dx0, s, ac[i]);
+    }
+  };
+  if (mode == 0) {
+    if constexpr (GC > 0) {
+#pragma unroll
+      for (int j = 0; j < GC; ++j) {
+        step(0, j, b0 + j, acc[0], dbg[0]);
+        step(1, j, b0 + j, acc[1], dbg[1]);
+      }
+    } else {
+#pragma unroll 2
+      for (int j = 0; j < G; ++j) {
+        step(0, j, b0 + j, acc[0], dbg[0]);
+        step(1, j, b0 + j, acc[1], dbg[1]);
+      }
+    }
+  } else {
+#pragma unroll 4
+    for (int j = 0; j < G; ++j) step(0, j, b0 + j, acc[0], dbg[0]);
+#pragma unroll 4
+    for (int j = 0; j < G; ++j) step(1, j, b0 + G + j, acc[0], dbg[0]);
+  }
+}
+
 template <int TT, int BITS, bool DBG, int GC>
 __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid_constant__ StreamArgs a) {
   constexpr int R = kR;
@@ -270,6 +393,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   __shared__ int s_nslots;
   __shared__ int s_routed;      // the routing tables below are complete
   __shared__ int s_xready;      // the x planes are complete
+  __shared__ uint64_t s_xbar;   // the x planes' bulk copies (from the router kernel) have landed
   __shared__ int s_dn_next;     // the next of this CTA's down units to hand out
   __shared__ int s_q[kSW][kQ];  // per warp: the down units its cursor took, in order (-1: no more)
   __shared__ float s_h[kPairs][2][TT][32];  // a warp pair's h block, double-buffered by unit
@@ -279,8 +403,12 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   __shared__ int s_qdone[kPairs][2];
   __shared__ int s_drow[DBG ? kMaxSlotsS : 1][TT];  // capture row of (slot, position): token * (K + S) + rank
   constexpr bool HS = StreamHStaged<TT>::value;
-  __shared__ int s_hclaim[HS ? kMaxSlotsS : 1];      // a warp has issued the slot's h copy
-  __shared__ uint64_t s_hbar[HS ? kMaxSlotsS : 1];   // the slot's h rows are in shared memory
+  constexpr bool MMA = StreamMma<TT>::value;
+  constexpr bool HR = StreamHRing<TT>::value;
+  __shared__ int s_hclaim[HS || HR ? kMaxSlotsS : 1];   // a warp has taken the staging of the slot's h
+  __shared__ int s_hissued[HR ? kMaxSlotsS : 1];        // ... and issued its copy (ring: the buffer's phase is set)
+  __shared__ uint64_t s_hbar[HS ? kMaxSlotsS : (HR ? kHRing : 1)];  // the slot's (ring: the buffer's) h rows landed
+  __shared__ int s_hused[HR ? kHRing : 1];              // ring: down units finished on each buffer, in total
 
   const StreamGeom& g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -304,8 +432,13 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     s_arrive[threadIdx.x >> 1][threadIdx.x & 1] = 0;
     s_qdone[threadIdx.x >> 1][threadIdx.x & 1] = 0;
   }
-  if constexpr (HS)
-    for (int i = threadIdx.x; i < kMaxSlotsS; i += blockDim.x) s_hclaim[i] = 0;
+  if constexpr (HS || HR)
+    for (int i = threadIdx.x; i < kMaxSlotsS; i += blockDim.x) {
+      s_hclaim[i] = 0;
+      if constexpr (HR) s_hissued[i] = 0;
+    }
+  if constexpr (HR)
+    if (threadIdx.x < kHRing) s_hused[threadIdx.x] = 0;
   // the shared slots come first and need no routing: slot s < S is shared
   // expert s, with all T tokens (rows s T .. s T + T - 1)
   for (int s = threadIdx.x; s < S; s += blockDim.x) {
@@ -319,8 +452,11 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSW * kR; ++i) tc::mbar_init(&s_full[i / kR][i % kR], 1);
+    tc::mbar_init(&s_xbar, 1);
     if constexpr (HS)
       for (int i = 0; i < kMaxSlotsS; ++i) tc::mbar_init(&s_hbar[i], 1);
+    if constexpr (HR)
+      for (int i = 0; i < kHRing; ++i) tc::mbar_init(&s_hbar[i], 1);
     abort_s = 0;
     s_dn_next = 0;
     s_routed = 0;
@@ -334,7 +470,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   // is a shared expert's computes that unit before the routing is known.
   // (The routing is a short serial chain on the critical path: the low warp
   // ids, which the schedulers favour, take it.)
-  const bool router = warp < T;
+  const int n_router = T < 4 ? T : 4;  // router warps: token warp, warp + 4
+  const bool router = warp < n_router;
   // Gate/up work goes to warp pairs: pair p of this CTA takes units
   // gp, gp + NP, ... (gp = p * G + blockIdx.x), warp 2p the first half of
   // each unit, warp 2p + 1 the second.  Down work: this CTA owns the output
@@ -422,30 +559,61 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     }
   };
 
-  if (!router) {
+  if (!router && a.xpl_g != nullptr) {
+    // the x planes from the router kernel: two bulk copies after the PDL wait
+    if (threadIdx.x == n_router * 32) {
+      pdl_wait();
+      const uint32_t pb = (uint32_t)(T * g.nbh * 32), db = (uint32_t)(T * g.nbh * 8);
+      stream::fence_proxy_async_global();
+      stream::mbar_expect_tx(&s_xbar, pb + db);
+      stream::bulk_g2s(xpl, a.xpl_g, pb, &s_xbar);
+      stream::bulk_g2s(xdc, a.xdc_g, db, &s_xbar);
+    }
+    tc::mbar_wait(&s_xbar, 0, abort_f, a.status, kErrRouting);
+    asm volatile("bar.sync 2, %0;" ::"r"((kSW - n_router) * 32) : "memory");  // the non-router warps
+    if (threadIdx.x == n_router * 32) {
+      __threadfence_block();
+      *(volatile int*)&s_xready = 1;
+    }
+  } else if (!router) {
     // x planes, from the layer input (the Q8_0 of the router kernel,
     // quotients from one reciprocal per block): block b of token t ->
     // even / odd byte planes and (d, c16 = -128 * sum of the even plane)
     // eight lanes per block (lane m: elements 4m .. 4m + 3), four blocks per
     // warp and step; lane m writes bytes 2m, 2m + 1 of both planes
-    const int sub = lane >> 3, m = lane & 7;
-    for (int i = (warp - T) * 4 + sub; i < T * g.nbh; i += (kSW - T) * 4) {
-      const float4 f = __ldg(reinterpret_cast<const float4*>(a.x + (size_t)i * 32) + m);
-      float amax = fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w)));
+    // (the loads of eight steps go out together: the loop is bound by their latency)
+    const int sub = lane >> 3, m = lane & 7, nblk = T * g.nbh, stride = (kSW - n_router) * 4;
+    for (int i0 = (warp - n_router) * 4 + sub; i0 < nblk; i0 += 8 * stride) {
+      float4 fv[8];
 #pragma unroll
-      for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const float d = __fdiv_rn(amax, 127.0f), r = __frcp_rn(d);
-      const int q0 = q8_of_r(f.x, d, r), q1 = q8_of_r(f.y, d, r), q2 = q8_of_r(f.z, d, r), q3 = q8_of_r(f.w, d, r);
-      unsigned short* pl = reinterpret_cast<unsigned short*>(xpl + 2 * i);
-      pl[m] = (unsigned short)((q0 & 0xFF) | (q2 & 0xFF) << 8);      // even plane
-      pl[8 + m] = (unsigned short)((q1 & 0xFF) | (q3 & 0xFF) << 8);  // odd plane
-      int se = q0 + q2;
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * stride;
+        fv[u] = i < nblk ? __ldg(reinterpret_cast<const float4*>(a.x + (size_t)i * 32) + m)
+                         : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      }
+      // (eight independent chains: unrolled, so that they overlap)
 #pragma unroll
-      for (int o = 4; o > 0; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
-      if (m == 0) xdc[i] = make_float2(d, __int_as_float(-128 * se));
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * stride;
+        const float4 f = fv[u];
+        float amax = fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w)));
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float d = __fdiv_rn(amax, 127.0f), r = __frcp_rn(d);
+        const int q0 = q8_of_r(f.x, d, r), q1 = q8_of_r(f.y, d, r), q2 = q8_of_r(f.z, d, r), q3 = q8_of_r(f.w, d, r);
+        int se = q0 + q2;
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
+        if (i < nblk) {
+          unsigned short* pl = reinterpret_cast<unsigned short*>(xpl + 2 * i);
+          pl[m] = (unsigned short)((q0 & 0xFF) | (q2 & 0xFF) << 8);      // even plane
+          pl[8 + m] = (unsigned short)((q1 & 0xFF) | (q3 & 0xFF) << 8);  // odd plane
+          if (m == 0) xdc[i] = make_float2(d, __int_as_float(-128 * se));
+        }
+      }
     }
-    asm volatile("bar.sync 2, %0;" ::"r"((kSW - T) * 32) : "memory");  // the non-router warps
-    if (threadIdx.x == T * 32) {
+    asm volatile("bar.sync 2, %0;" ::"r"((kSW - n_router) * 32) : "memory");  // the non-router warps
+    if (threadIdx.x == n_router * 32) {
       __threadfence_block();
       *(volatile int*)&s_xready = 1;
     }
@@ -459,7 +627,6 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
 
   // ---- routing of the batch (every CTA, identical results) -------------
   if (router) {
-    const int tr = warp;  // this warp's token
     // the correction bias is a layer constant: into registers before the wait
     float bias_r[kMaxExperts / 32];
 #pragma unroll
@@ -468,22 +635,24 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       bias_r[i] = e < E ? __ldg(a.bias + e) : 0.0f;
     }
     pdl_wait();  // the scores and the cleared counters are complete
-    const float* st = a.scores + (size_t)tr * E;
-    auto sc = [st](int e) { return ld_dep(st + e); };
-    if (E <= 256)
-      topk::warp_route_token<8>(sc, bias_r, E, K, a.norm, a.rsf, lane, s_idx + tr * K, s_w + tr * K);
-    else
-      topk::warp_route_token<kMaxExperts / 32>(sc, bias_r, E, K, a.norm, a.rsf, lane, s_idx + tr * K,
-                                               s_w + tr * K);
-    __syncwarp();
-    // the chosen experts (bit e of s_bits) and, per expert, the tokens that
-    // chose it (byte e & 3 of s_tm[e >> 2], bit t)
-    if (lane < K) {
-      const int e = s_idx[tr * K + lane];
-      atomicOr(&s_bits[e >> 5], 1u << (e & 31));
-      atomicOr(&s_tm[e >> 2], 1u << ((e & 3) * 8 + tr));
+    for (int tr = warp; tr < T; tr += n_router) {  // this warp's tokens
+      const float* st = a.scores + (size_t)tr * E;
+      auto sc = [st](int e) { return ld_dep(st + e); };
+      if (E <= 256)
+        topk::warp_route_token<8>(sc, bias_r, E, K, a.norm, a.rsf, lane, s_idx + tr * K, s_w + tr * K);
+      else
+        topk::warp_route_token<kMaxExperts / 32>(sc, bias_r, E, K, a.norm, a.rsf, lane, s_idx + tr * K,
+                                                 s_w + tr * K);
+      __syncwarp();
+      // the chosen experts (bit e of s_bits) and, per expert, the tokens that
+      // chose it (byte e & 3 of s_tm[e >> 2], bit t)
+      if (lane < K) {
+        const int e = s_idx[tr * K + lane];
+        atomicOr(&s_bits[e >> 5], 1u << (e & 31));
+        atomicOr(&s_tm[e >> 2], 1u << ((e & 3) * 8 + tr));
+      }
     }
-    if (T > 1) asm volatile("bar.sync 1, %0;" ::"r"(T * 32) : "memory");  // the router warps
+    if (n_router > 1) asm volatile("bar.sync 1, %0;" ::"r"(n_router * 32) : "memory");  // the router warps
     if (warp == 0) {
       __syncwarp();
       auto tm_of = [&](int e) { return (s_tm[e >> 2] >> ((e & 3) * 8)) & 0xFFu; };
@@ -642,7 +811,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
         // memory (one bulk copy for the planes, one for (d, c16)); every
         // warp waits for that copy.
         bool claim = true;
-        if constexpr (HS) {
+        if constexpr (HS || HR) {
           int c = 0;
           if (lane == 0) c = atomicCAS(&s_hclaim[slot], 0, 1) == 0;
           claim = __shfl_sync(0xffffffffu, c, 0) != 0;
@@ -672,8 +841,49 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
               stream::bulk_g2s(hst_dc + r0 * g.nbi * 8, a.hdc + r0 * g.nbi, dc, &s_hbar[slot]);
             }
           }
+          if constexpr (HR) {
+            // ring buffer slot % kHRing: free once every down unit of its
+            // previous slot (slot - kHRing) has finished here
+            if (lane == 0 && ready) {
+              const int b = slot % kHRing;
+              const int need = (slot / kHRing) * nch;
+              const long long t1 = clock64();
+              while (*(volatile int*)&s_hused[b] < need && !*abort_f)
+                if (clock64() - t1 > tc::kSpinCycles) {
+                  *abort_f = 1;
+                  atomicExch(a.status, kErrHStaged);
+                }
+              if (!*abort_f) {
+                const size_t r0 = s_base[slot];
+                unsigned char* hb = hst + (size_t)b * TT * g.nbi * 40;
+                const uint32_t pl = (uint32_t)(nv * g.nbi * 32), dc = (uint32_t)(nv * g.nbi * 8);
+                stream::fence_proxy_async_global();
+                stream::mbar_expect_tx(&s_hbar[b], pl + dc);
+                stream::bulk_g2s(hb, a.hpl + r0 * g.nbi * 32, pl, &s_hbar[b]);
+                stream::bulk_g2s(hb + (size_t)TT * g.nbi * 32, a.hdc + r0 * g.nbi, dc, &s_hbar[b]);
+                __threadfence_block();
+                *(volatile int*)&s_hissued[slot] = 1;
+              }
+            }
+          }
         }
         if constexpr (HS) ready = tc::mbar_wait(&s_hbar[slot], 0, abort_f, a.status, kErrHStaged);
+        if constexpr (HR) {
+          // the copy is issued (so the buffer's phase is this slot's), then landed
+          int is = 1;
+          if (lane == 0) {
+            const long long t1 = clock64();
+            while (!*(volatile int*)&s_hissued[slot] && !*abort_f)
+              if (clock64() - t1 > tc::kSpinCycles) {
+                *abort_f = 1;
+                atomicExch(a.status, kErrHStaged);
+              }
+            is = !*abort_f;
+          }
+          is = __shfl_sync(0xffffffffu, is, 0);
+          ready = is && tc::mbar_wait(&s_hbar[slot % kHRing], (uint32_t)((slot / kHRing) & 1), abort_f, a.status,
+                                      kErrHStaged);
+        }
         if (!__all_sync(0xffffffffu, ready)) {
           ok = false;
           break;
@@ -683,6 +893,10 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       if constexpr (HS) {
         ap = reinterpret_cast<const uint4*>(hst + (size_t)s_base[slot] * g.nbi * 32);
         adc = reinterpret_cast<const float2*>(hst_dc + (size_t)s_base[slot] * g.nbi * 8);
+      } else if constexpr (HR) {
+        const unsigned char* hb = hst + (size_t)(slot % kHRing) * TT * g.nbi * 40;
+        ap = reinterpret_cast<const uint4*>(hb);
+        adc = reinterpret_cast<const float2*>(hb + (size_t)TT * g.nbi * 32);
       } else {
         // the slot's h rows are read through L1 (every lane loads the same block)
         ap = reinterpret_cast<const uint4*>(a.hpl + (size_t)s_base[slot] * g.nbi * 32);
@@ -696,6 +910,46 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
         if constexpr (DBG)
           if (t < nv) dbg[t] = a.dbg + s_drow[slot][t] * P + 2 * (int64_t)g.I * g.nbh + (int64_t)o * g.nbi;
       }
+    }
+    // tensor-core fold (batches of more than two tokens): lane (gq, cq) =
+    // (lane / 4, lane % 4) feeds token column gq and folds columns 2cq,
+    // 2cq + 1 of rows gq, gq + 8 (and 16 + .. of the second row group);
+    // mode 0: the row groups are separate rows, 1: the two pieces of the
+    // same 16 down rows
+    const int gq = lane >> 2, cq = lane & 3;
+    const int mmode = gu ? 0 : (lpr == 2 ? 1 : 0);
+    int rB = 0, rF0 = 0, rF1 = 0;
+    float accm[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+    float rsm[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
+    int32_t* dbgm[2][4] = {{nullptr, nullptr, nullptr, nullptr}, {nullptr, nullptr, nullptr, nullptr}};
+    if constexpr (MMA) {
+      const int last = nv - 1;
+      const int cB = gq < nv ? gq : last, cF0 = 2 * cq < nv ? 2 * cq : last, cF1 = 2 * cq + 1 < nv ? 2 * cq + 1 : last;
+      rB = gu ? s_tok[slot][cB] : cB;
+      rF0 = gu ? s_tok[slot][cF0] : cF0;
+      rF1 = gu ? s_tok[slot][cF1] : cF1;
+      const float* scm = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);
+#pragma unroll
+      for (int rg = 0; rg < 2; ++rg)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          // the output row of (rg, h) within the unit, and its scale
+          const int orow = gu ? chunk * 32 + 16 * half + gq + 8 * h
+                              : chunk * g.rpu_dn + (mmode == 1 ? 0 : 16 * rg) + gq + 8 * h;
+          if (gu || mmode == 0 || rg == 0)
+            rsm[rg][h] = __ldg(scm + (gu ? (rg == 0 ? 0 : g.I) : 2 * g.I) + orow);
+          if constexpr (DBG) {
+#pragma unroll
+            for (int ti = 0; ti < 2; ++ti) {
+              const int t = 2 * cq + ti;
+              if (t < nv)
+                dbgm[rg][2 * h + ti] = gu ? a.dbg + s_drow[slot][t] * P + (int64_t)(rg == 0 ? 0 : g.I) * g.nbh +
+                                                (int64_t)orow * g.nbh
+                                          : a.dbg + s_drow[slot][t] * P + 2 * (int64_t)g.I * g.nbh +
+                                                (int64_t)orow * g.nbi;
+            }
+          }
+        }
     }
     // the row scale of this lane's output, loaded ahead of the stages
     const float* sc = reinterpret_cast<const float*>(a.prep + (uint64_t)s_exp[slot] * g.expert_bytes + g.sc_off);
@@ -711,14 +965,28 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       ok = wait_stage();
       if (!ok) break;
       const unsigned char* stg = ring + (size_t)(consumed % R) * kStreamStageMax;
-      if (HS || gu)
-        rows_stage<TT, BITS, DBG, GC, true>(Gs, stg, swz, s * span + piece0, nb, nv, lpr == 2, tok, ap, adc, acc, dbg);
-      else
-        rows_stage<TT, BITS, DBG, GC, false>(Gs, stg, swz, s * span + piece0, nb, nv, lpr == 2, tok, ap, adc, acc,
-                                             dbg);
+      if constexpr (MMA) {
+        if (HS || HR || gu)
+          rows_stage_mma<BITS, DBG, GC, true>(Gs, stg, swz, s * span, nb, mmode, rB, rF0, rF1, ap, adc, accm, dbgm);
+        else
+          rows_stage_mma<BITS, DBG, GC, false>(Gs, stg, swz, s * span, nb, mmode, rB, rF0, rF1, ap, adc, accm, dbgm);
+      } else {
+        if (HS || HR || gu)
+          rows_stage<TT, BITS, DBG, GC, true>(Gs, stg, swz, s * span + piece0, nb, nv, lpr == 2, tok, ap, adc, acc,
+                                              dbg);
+        else
+          rows_stage<TT, BITS, DBG, GC, false>(Gs, stg, swz, s * span + piece0, nb, nv, lpr == 2, tok, ap, adc, acc,
+                                               dbg);
+      }
       next_stage();
     }
     if (!ok) break;
+    if constexpr (HR) {
+      if (!gu) {  // this unit's reads of its ring buffer are done
+        __syncwarp();
+        if (lane == 0) atomicAdd(&s_hused[slot % kHRing], 1);
+      }
+    }
     if (gu) {
       // SwiGLU of the half's 16 outputs into shared memory; the second warp
       // of the pair to finish quantises the whole Q8_0 block of h and
@@ -734,11 +1002,20 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
           }
         }
       }
+      if constexpr (MMA) {
 #pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        const float v = __fmul_rn(rs, acc[t]);
-        const float uv = __shfl_down_sync(0xffffffffu, v, 16);
-        if (lane < 16 && t < nv) hbuf[t * 32 + 16 * half + lane] = __fmul_rn(__fmul_rn(v, sigmoid_cw(v)), uv);
+        for (int i = 0; i < 4; ++i) {
+          const int t = 2 * cq + (i & 1), o = gq + 8 * (i >> 1);
+          const float v = __fmul_rn(rsm[0][i >> 1], accm[0][i]), uv = __fmul_rn(rsm[1][i >> 1], accm[1][i]);
+          if (t < nv) hbuf[t * 32 + 16 * half + o] = __fmul_rn(__fmul_rn(v, sigmoid_cw(v)), uv);
+        }
+      } else {
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+          const float v = __fmul_rn(rs, acc[t]);
+          const float uv = __shfl_down_sync(0xffffffffu, v, 16);
+          if (lane < 16 && t < nv) hbuf[t * 32 + 16 * half + lane] = __fmul_rn(__fmul_rn(v, sigmoid_cw(v)), uv);
+        }
       }
       __syncwarp();
       int second = 0;
@@ -773,7 +1050,16 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     } else {
       // lanes 0 .. rpu_dn - 1: the unit's rows (lane pairs hold the same sum)
       const int rpu = g.rpu_dn;
-      if (lane < rpu) {
+      if constexpr (MMA) {
+        float* yc = s_y + ((size_t)(chunk - c0) * n_rows + s_base[slot]) * rpu;
+#pragma unroll
+        for (int rg = 0; rg < 2; ++rg)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int t = 2 * cq + (i & 1), rr = (mmode == 1 ? 0 : 16 * rg) + gq + 8 * (i >> 1);
+            if (t < nv && (rg == 0 || mmode == 0)) yc[(size_t)t * rpu + rr] = __fmul_rn(rsm[rg][i >> 1], accm[rg][i]);
+          }
+      } else if (lane < rpu) {
         float* yc = s_y + ((size_t)(chunk - c0) * n_rows + s_base[slot]) * rpu + lane;
 #pragma unroll
         for (int t = 0; t < TT; ++t)
@@ -789,6 +1075,11 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     if (*abort_f && threadIdx.x == 0)  // h copies issued, perhaps never waited for
       for (int i = 0; i < kMaxSlotsS; ++i)
         if (s_hclaim[i]) stream::mbar_drain(&s_hbar[i], 0);
+  }
+  if constexpr (HR) {
+    if (*abort_f && threadIdx.x == 0)
+      for (int i = 0; i < kMaxSlotsS; ++i)
+        if (s_hissued[i]) stream::mbar_drain(&s_hbar[i % kHRing], (uint32_t)((i / kHRing) & 1));
   }
 
   // ---- combine of this CTA's output chunks (contract C): every slot's y
@@ -892,7 +1183,8 @@ bool stream_supported(int hidden, int inter, int bits, int n_tok, int top_k, int
   const int rows = n_tok * (top_k + n_shared);  // y (and h) rows of the batch
   const size_t need = n_tok <= 1   ? stream_smem_bytes<1>(g, n_sms, rows)
                       : n_tok <= 2 ? stream_smem_bytes<2>(g, n_sms, rows)
-                                   : stream_smem_bytes<4>(g, n_sms, rows);
+                      : n_tok <= 4 ? stream_smem_bytes<4>(g, n_sms, rows)
+                                   : stream_smem_bytes<8>(g, n_sms, rows);
   (void)n_experts;
   return need <= kStreamDynMax;
 }
@@ -911,7 +1203,8 @@ template <int BITS, bool DBG, int GC>
 cudaError_t stream_g(const StreamArgs& a, cudaStream_t st) {
   if (a.T <= 1) return stream_tt<1, BITS, DBG, GC>(a, st);
   if (a.T <= 2) return stream_tt<2, BITS, DBG, GC>(a, st);
-  return stream_tt<4, BITS, DBG, GC>(a, st);
+  if (a.T <= 4) return stream_tt<4, BITS, DBG, GC>(a, st);
+  return stream_tt<8, BITS, DBG, GC>(a, st);
 }
 
 // Full stages (256-byte rows for gate/up and down) take the compile-time

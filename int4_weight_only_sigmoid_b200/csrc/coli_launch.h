@@ -79,7 +79,7 @@ cudaError_t launch_route_topk(const float* x, const float* w_router, const float
 // kernel's counters; may be null).
 cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
                                  int8_t* xq, float* xd, int32_t* status_clear, int32_t* zero, int n_zero,
-                                 cudaStream_t st);
+                                 cudaStream_t st, int8_t* xpl = nullptr, float2* xdc = nullptr);
 cudaError_t launch_topk_bucket_small(const float* scores, const float* bias, int n_tok, int E, int K, int norm,
                                      float rsf, int32_t* idx, float* w, int32_t* counts, int32_t* offsets,
                                      int32_t* perm, int32_t* inv, Slot* slots, int32_t* n_slots, cudaStream_t st);
@@ -126,7 +126,7 @@ cudaError_t launch_down_decode(const DownTable& tbl, const Slot* slots, const in
 // persistent kernel (PDL launch after router_decode) that routes the batch
 // in every CTA, streams the layer's streaming copy stage by stage (gate/up,
 // SwiGLU, Q8_0 of h; down; combine) and writes `out`.
-constexpr int kStreamMaxTok = 4;
+constexpr int kStreamMaxTok = 8;
 constexpr int kStreamMaxSlots = kMaxShared + kStreamMaxTok * kMaxTopK;
 struct StreamArgs {
   const unsigned char* prep;  // the layer's streaming copy (coli_moe_prepare)
@@ -136,6 +136,8 @@ struct StreamArgs {
   const float* scores;  // [T x E] (router_decode)
   const float* bias;
   const float* x;       // [T x H] the layer input
+  const int8_t* xpl_g;  // null (the kernel quantises x itself), or [T x H/32 x 32] planes of Q8(x) (router_decode)
+  const float2* xdc_g;  // [T x H/32] (d, -128 * sum of the even plane) with xpl_g
   int8_t* hpl;          // [rows x I/32 x 32]: h of every (slot, token) row as even / odd byte planes
   float2* hdc;          // [rows x I/32]: (d, -128 * sum of the even plane as int bits)
   float* out;           // [T x H]

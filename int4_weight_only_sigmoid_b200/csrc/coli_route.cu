@@ -190,7 +190,8 @@ constexpr int kStageTok = 2;
 __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restrict__ x,
                                                             const float* __restrict__ wr, int n_tok, int E, int H,
                                                             float* __restrict__ scores, int8_t* __restrict__ xq,
-                                                            float* __restrict__ xd, int32_t* status_clear,
+                                                            float* __restrict__ xd, int8_t* __restrict__ xpl,
+                                                            float2* __restrict__ xdc, int32_t* status_clear,
                                                             int32_t* zero, int n_zero) {
   extern __shared__ __align__(16) float4 wsm[];  // [2][H/4] router rows, then [kStageTok][H/4] tokens
   // first kernel of a decode forward (launched without PDL, so everything
@@ -213,13 +214,25 @@ __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restr
   }
   if (stage_x)
     for (int i = threadIdx.x; i < n_tok * nq; i += blockDim.x) cp_async16(wsm + 2 * nq + i, x + 4 * (size_t)i);
-  // the Q8_0 of x for the expert kernels (unless they make their own): one
-  // warp per 32-element block
-  for (int j = blockIdx.x * 8 + warp; xq != nullptr && j < n_tok * (H / 32); j += gridDim.x * 8) {
+  // the Q8_0 of x for the expert kernels: one warp per 32-element block,
+  // as rows (xq, xd) and / or as the streaming kernel's even / odd byte
+  // planes with (d, -128 * sum of the even plane) (xpl, xdc)
+  for (int j = blockIdx.x * 8 + warp; (xq != nullptr || xpl != nullptr) && j < n_tok * (H / 32);
+       j += gridDim.x * 8) {
     const float v = x[(size_t)j * 32 + lane];
     const float d = __fdiv_rn(warp_max(fabsf(v)), 127.0f);
-    xq[(size_t)j * 32 + lane] = (int8_t)q8_of(v, d);
-    if (lane == 0) xd[j] = d;
+    const int q = q8_of(v, d);
+    if (xq != nullptr) {
+      xq[(size_t)j * 32 + lane] = (int8_t)q;
+      if (lane == 0) xd[j] = d;
+    }
+    if (xpl != nullptr) {
+      xpl[(size_t)j * 32 + (lane & 1) * 16 + (lane >> 1)] = (int8_t)q;
+      int se = (lane & 1) ? 0 : q;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
+      if (lane == 0) xdc[j] = make_float2(d, __int_as_float(-128 * se));
+    }
   }
   cp_async_wait_all();
   __syncthreads();
@@ -445,13 +458,13 @@ cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E
 
 cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
                                  int8_t* xq, float* xd, int32_t* status_clear, int32_t* zero, int n_zero,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, int8_t* xpl, float2* xdc) {
   const size_t smem = (size_t)(2 + (n_tok <= kStageTok ? n_tok : 0)) * H * sizeof(float);
   static int granted[64] = {};
   const cudaError_t e = smem_opt_in(router_decode_kernel, 200 * 1024, granted);
   if (e != cudaSuccess) return e;
-  router_decode_kernel<<<(E + 1) / 2, 256, smem, st>>>(x, w_router, n_tok, E, H, scores, xq, xd, status_clear,
-                                                       zero, n_zero);
+  router_decode_kernel<<<(E + 1) / 2, 256, smem, st>>>(x, w_router, n_tok, E, H, scores, xq, xd, xpl, xdc,
+                                                       status_clear, zero, n_zero);
   return cudaGetLastError();
 }
 

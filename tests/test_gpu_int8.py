@@ -53,7 +53,7 @@ def _check(coli, syn, cfg, n_tok, prepare, sample=None):
     return out
 
 
-@pytest.mark.parametrize("n_tok", [1, 2, 3, 4])
+@pytest.mark.parametrize("n_tok", [1, 2, 3, 4, 6])
 def test_int8_tiny_streaming(coli, syn, n_tok):
     _check(coli, syn, syn.config("tiny", weight_bits=8), n_tok, prepare=True)
 

@@ -105,12 +105,12 @@ def _check(coli, syn, cfg, n_tok, tokens=None):
     return out
 
 
-@pytest.mark.parametrize("n_tok", [1, 2, 3, 4])
+@pytest.mark.parametrize("n_tok", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_stream_tiny(coli, syn, n_tok):
     _check(coli, syn, syn.config("tiny"), n_tok)
 
 
-@pytest.mark.parametrize("n_tok", [1, 2, 3, 4])
+@pytest.mark.parametrize("n_tok", [1, 2, 3, 4, 8])
 @pytest.mark.parametrize("bits", [4, 8])
 def test_stream_mid_lane_pairs(coli, syn, n_tok, bits):
     """Down rows split over lane pairs (rows of whole stages)."""
@@ -130,7 +130,8 @@ def test_stream_all_tokens_on_one_expert(coli, syn):
     _check(coli, syn, cfg, 4, tokens=x)
 
 
-@pytest.mark.parametrize("name,n_tok", [("decode1", 1), ("decode4", 4), ("decode4", 2), ("decode4", 3)])
+@pytest.mark.parametrize("name,n_tok", [("decode1", 1), ("decode4", 4), ("decode4", 2), ("decode4", 3),
+                                        ("decode16", 5), ("decode16", 8)])
 def test_stream_glm(coli, syn, name, n_tok):
     _check(coli, syn, syn.config(name), n_tok)
 
