@@ -126,7 +126,8 @@ cudaError_t launch_down_decode(const DownTable& tbl, const Slot* slots, const in
 // persistent kernel (PDL launch after router_decode) that routes the batch
 // in every CTA, streams the layer's streaming copy stage by stage (gate/up,
 // SwiGLU, Q8_0 of h; down; combine) and writes `out`.
-constexpr int kStreamMaxTok = 8;
+constexpr int kStreamMaxTok = 8;   // tokens of one streaming kernel launch
+constexpr int kStreamChunked = 16;  // a prepared layer's batches up to this run as launches of <= kStreamMaxTok
 constexpr int kStreamMaxSlots = kMaxShared + kStreamMaxTok * kMaxTopK;
 struct StreamArgs {
   const unsigned char* prep;  // the layer's streaming copy (coli_moe_prepare)

@@ -54,7 +54,7 @@ def _run(coli, ora, syn, cfg, n_tok, prepare, rows_per_matrix=None):
     _check_partials(ora, syn, cfg, x, _np(isum), _np(idx), rows_per_matrix)
 
 
-@pytest.mark.parametrize("n_tok", [1, 3, 4, 8])
+@pytest.mark.parametrize("n_tok", [1, 3, 4, 8, 11])
 def test_partials_streaming_kernel_tiny(coli, ora, syn, n_tok):
     _run(coli, ora, syn, syn.config("tiny"), n_tok, prepare=True)
 

@@ -105,7 +105,7 @@ def _check(coli, syn, cfg, n_tok, tokens=None):
     return out
 
 
-@pytest.mark.parametrize("n_tok", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("n_tok", [1, 2, 3, 4, 5, 6, 7, 8, 12, 16])
 def test_stream_tiny(coli, syn, n_tok):
     _check(coli, syn, syn.config("tiny"), n_tok)
 
@@ -131,7 +131,7 @@ def test_stream_all_tokens_on_one_expert(coli, syn):
 
 
 @pytest.mark.parametrize("name,n_tok", [("decode1", 1), ("decode4", 4), ("decode4", 2), ("decode4", 3),
-                                        ("decode16", 5), ("decode16", 8)])
+                                        ("decode16", 5), ("decode16", 8), ("decode16", 16)])
 def test_stream_glm(coli, syn, name, n_tok):
     _check(coli, syn, syn.config(name), n_tok)
 
