@@ -653,7 +653,28 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       }
     }
     if (n_router > 1) asm volatile("bar.sync 1, %0;" ::"r"(n_router * 32) : "memory");  // the router warps
-    if (warp == 0) {
+    if (warp == 0 && T == 1) {
+      // one token: every chosen expert is a slot of one row; slot of rank k
+      // = S + the number of chosen experts with a lower id
+      const int e = lane < K ? s_idx[lane] : INT_MAX;
+      int below = 0;
+      for (int j = 0; j < K; ++j) below += __shfl_sync(0xffffffffu, e, j) < e;
+      if (lane < K) {
+        const int r = S + below;
+        s_exp[r] = e;
+        s_cnt[r] = 1;
+        s_base[r] = r;
+        s_tok[r][0] = 0;
+        s_row[lane] = r;
+        if constexpr (DBG) s_drow[r][0] = lane;  // token 0, rank lane
+      }
+      if (lane == 0) s_nslots = S + K;
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        *(volatile int*)&s_routed = 1;
+      }
+    } else if (warp == 0) {
       __syncwarp();
       auto tm_of = [&](int e) { return (s_tm[e >> 2] >> ((e & 3) * 8)) & 0xFFu; };
       // lane l: the experts 32l .. 32l+31; slots in ascending expert id after
