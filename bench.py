@@ -307,6 +307,12 @@ def run_suite(layers, cfg, dev, stream, peak_gbs, only=None, tokens=None):
         _, idx, _ = coli.moe_route(layer, x)
         return len(torch.unique(idx)) + S
 
+    def issued(layer, x):
+        """Experts streamed by the prepared decode path: once per launch of
+        at most 8 tokens (a 16-token batch is two launches)."""
+        _, idx, _ = coli.moe_route(layer, x)
+        return sum(len(torch.unique(idx[i:i + 8])) + S for i in range(0, idx.shape[0], 8))
+
     def time_steps(fn, n_steps, graph):
         if graph:
             g = torch.cuda.CUDAGraph()
@@ -346,11 +352,13 @@ def run_suite(layers, cfg, dev, stream, peak_gbs, only=None, tokens=None):
                 coli.moe_layer_forward(lys[j % nl], x, out=o, workspace=ws, stream=stream, cstruct=cs[j % nl])
         torch.cuda.synchronize()
         n_exp = [uniq(l, x) for l in lys]
+        n_iss = [issued(l, x) for l in lys] if T <= 16 else n_exp
         fn = lambda j, st: coli.moe_layer_forward(lys[j % nl], x, out=o, workspace=ws, stream=st, cstruct=cs[j % nl])
         ms = time_steps(fn, steps, graph)
         ue = sum(n_exp) / len(n_exp)
         rec = {"tokens": T, "ms_per_layer": ms, "tokens_per_s_per_layer": T / (ms * 1e-3),
                "unique_experts_streamed": ue,
+               "issued_experts_streamed": sum(n_iss) / len(n_iss),
                "weight_gbs": (ue * expert_bytes + router_bytes) / (ms * 1e-3) / 1e9}
         rec["weight_frac_of_hbm"] = rec["weight_gbs"] / peak_gbs
         if name == "prefill2048":
