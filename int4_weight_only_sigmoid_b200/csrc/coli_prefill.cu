@@ -13,36 +13,35 @@
 // gate/up item's 128 columns are 64 gate rows and the same 64 up rows.
 //
 // int8 expert weights (the pages' int8 variant) take the same kernel with
-// B signed and copied as it is, A in the elements' own order, and no
-// per-block correction (every accumulator starts at 0x4B400000).
+// B = q copied as it is and A in the elements' own order.
 //
 // Operands.  A = the Q8 activations as signed bytes (one row per (slot,
 // token) in slot order, loaded by TMA, 128-byte swizzle); B = the weights as
-// unsigned bytes q + 8 (0..15), expanded from the packed nibbles by the
-// producer warps: for a packed word w, (w & 0x0F0F0F0F) ^ 0x08080808 holds
-// q + 8 of elements 0, 2, 4, 6 and ((w >> 4) & 0x0F0F0F0F) ^ 0x08080808 of
-// elements 1, 3, 5, 7 -- three logic ops per 8 weights, and the A rows are
-// stored in the same order (per 8 elements: 0,2,4,6,1,3,5,7), so the dot
-// product is unchanged.  One MMA (K = 32) is exactly one Q8 block.
+// signed bytes 16 q, expanded from the packed nibbles by the producer warps:
+// for a packed word w, (w << 4) & 0xF0F0F0F0 holds 16 q of elements
+// 0, 2, 4, 6 and w & 0xF0F0F0F0 of elements 1, 3, 5, 7 -- two logic ops per
+// 8 weights, and the A rows are stored in the same order (per 8 elements:
+// 0,2,4,6,1,3,5,7), so the dot product is 16 times the block's.  One MMA
+// (K = 32) is exactly one Q8 block.
 //
 // Exactness.  Each Q8 block's partial sum must come out exactly, because the
 // row fold (contract F: acc = fmaf(d_x[b], (float)isum[b], acc), b
-// ascending) needs it per block.  The MMA of block b adds
-// sum (q + 8) x = isum + 8 * sum(x) to an int32 accumulator that holds
-// M = 0x4B400000 - 8 * sum(x) (the token's block sum, written by the fold
-// before the MMA runs), so the accumulator ends as 0x4B400000 + isum: read as
-// a binary32 that is 1.5 * 2^23 + isum exactly (|isum| <= 32512 < 2^22), and
-// one F32 subtraction gives (float)isum with no integer-to-float
-// conversion.  The fold then applies contract F per block, so prefill equals
-// the dp4a paths bit for bit.
+// ascending) needs it per block.  The MMA of block b writes S = 16 isum
+// (int8 weights: isum) into a fresh int32 accumulator (the previous contents
+// are not read).  |S| < 2^22, so S + 0x4B400000 read as a binary32 is
+// 1.5 * 2^23 + S exactly: one integer add and one FMA (x 1/16, - 1.5 * 2^19)
+// give (float)isum with no integer-to-float conversion.  The fold then
+// applies contract F per block, so prefill equals the dp4a paths bit for
+// bit.
 //
-// Roles (704 threads): warps 0-3 producers (packed-weight copies; thread p
-// expands weight row p), warp 4 the A-tile TMA loads, warps 5-20 the fold
-// (warp w reads TMEM lanes 32(w%4).. = 32 of the tile's tokens, and a
-// quarter of the item's columns: gate/up 16 gate rows and the same 16 up
-// rows, down 32 rows), warp 21 the MMA issuer (lane 0) and TMEM owner.  The
+// Roles (640 threads): warps 0-1 producers (packed-weight copies; thread p
+// expands weight rows p and p + 64), warp 2 the A-tile TMA loads, warps 3-18
+// the fold (warp w reads TMEM lanes 32(w%4).. = 32 of the tile's tokens, and
+// a quarter of the item's columns: gate/up 16 gate rows and the same 16 up
+// rows, down 32 rows), warp 19 the MMA issuer (lane 0) and TMEM owner.  The
 // two fold warps that hold one Q8 block of h (32 intermediate rows) meet at
-// a named barrier to share the block's absmax.
+// a named barrier to share the block's absmax.  (20 warps, 5 per scheduler,
+// leave 96 registers per thread.)
 // An operand stage holds 4 Q8 blocks (K = 128).  Per stage g: the TMA warp
 // loads its A tile into operand stage g % kStages once `empty` (the MMA's
 // commit) says the stage is free; the producers copy its packed weights
@@ -50,9 +49,7 @@
 // arrive on `full`; the MMA issues one K=32 step per block onto a TMEM
 // accumulator per block (4 of them, handed to the fold kHalf blocks at a
 // time through `tfull` / `tempty`) and commits `empty`.  The fold reads a
-// buffer, writes the starting value M of the buffer's next use (the same
-// token slot one stage later, or the CTA's next item) and releases it.  All
-// waits are bounded (coli_tc.cuh).
+// buffer and releases it.  All waits are bounded (coli_tc.cuh).
 //
 // Sources: "Colibri：在笔记本上跑744B参数的AI模型", "关键特性" (integer dot
 // kernels, Q8_0 activations, packed int4); HN summary (hn.213312.xyz),
@@ -60,6 +57,8 @@
 // positions is read once and shared).
 #include <cuda.h>
 #include <cudaTypedefs.h>
+
+#include <type_traits>
 
 #include "coli_launch.h"
 #include "coli_tc.cuh"
@@ -75,9 +74,9 @@ constexpr int kBS = 4;         // Q8 blocks per operand stage (K = 128)
 constexpr int kStages = 4;     // operand stages
 constexpr int kLookS = 2;      // stages the producers' copies run ahead
 constexpr int kPkSlots = kLookS + 2;  // packed-weight slots: a slot is rewritten only after every producer expanded it
-constexpr int kHalf = 2;       // Q8 blocks per accumulator hand-off (MMA -> fold)
+constexpr int kHalf = 2;       // Q8 blocks per accumulator hand-off (MMA -> fold): 1 or 2
 constexpr int kTBufs = 4;      // TMEM accumulators (one per block), handed off in pairs
-constexpr int kProdWarps = 4;
+constexpr int kProdWarps = 2;
 constexpr int kEpiWarps = 16;  // 4 per TMEM lane quadrant, each a quarter of the columns
 // Warp w runs on scheduler w % 4 and, as a fold warp, reads TMEM lanes
 // 32 (w % 4)..; the MMA issuer is kept off scheduler 0, which carries the
@@ -85,8 +84,9 @@ constexpr int kEpiWarps = 16;  // 4 per TMEM lane quadrant, each a quarter of th
 constexpr int kTmaWarp = kProdWarps;                           // A-tile loads
 constexpr int kEpi0 = kProdWarps + 1;                          // first fold warp
 constexpr int kMmaWarp = kEpi0 + kEpiWarps;                    // MMA issuer, TMEM owner
-constexpr int kThreadsP = 32 * (kMmaWarp + 1);                 // 704
-constexpr int kNProd = 32 * kProdWarps;                        // 128 producer threads
+constexpr int kThreadsP = 32 * (kMmaWarp + 1);                 // 640
+constexpr int kNProd = 32 * kProdWarps;                        // producer threads
+static_assert(kN % kNProd == 0, "each producer thread expands whole weight rows");
 constexpr int kTmemCols = kTBufs * kN;                         // 512
 constexpr uint32_t kMagic = 0x4B400000u;                       // binary32 1.5 * 2^23
 constexpr float kMagicF = 12582912.0f;
@@ -195,25 +195,17 @@ __host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
 
-// D[tmem] += A[smem] * B[smem]^T (int8, int32 accumulate), issued by one thread.
+// D[tmem] = A[smem] * B[smem]^T (int8 operands, int32 result; the
+// accumulator's previous contents are not read), issued by one thread.
 __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, 1, 0;\n\t"
+      "setp.ne.b32 p, 0, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc)
       : "memory");
 }
 
-// 16 consecutive 32-bit TMEM columns of this warp's 32 lanes <- v (each
-// lane writes its own value in all 16 columns).
-__device__ __forceinline__ void tmem_st16_same(uint32_t taddr, uint32_t v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(v)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // fma / add on two F32 lanes at once (each lane one IEEE operation, rounded once).
 __device__ __forceinline__ void fma2(float& a0, float& a1, float d0, float d1, float x0, float x1) {
@@ -270,7 +262,8 @@ __device__ __forceinline__ int64_t item_token_row(const ItemInfo& f, bool gu, co
 // ad: the A rows' Q8 scales, [row x nb].
 template <bool GU, int BITS, bool DBG, typename Tab>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
-    const __grid_constant__ Tab tab, const __grid_constant__ CUtensorMap amap, const Slot* __restrict__ slots,
+    const __grid_constant__ Tab tab, const __grid_constant__ CUtensorMap amap,
+    const __grid_constant__ CUtensorMap amap32, const Slot* __restrict__ slots,
     const Tile* __restrict__ tiles, const int32_t* __restrict__ n_tiles, const int32_t* __restrict__ perm, int top_k,
     const float* ad, int hidden, int inter, int8_t* hr, float* hd, float* __restrict__ y, int32_t* __restrict__ err,
     DbgArgs dbg) {
@@ -319,7 +312,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     // ------------------------------------------------------------ producers
     // A stage's packed weights (128 rows x 64 B) are copied 4 lanes per
     // row, so that each warp instruction touches few cache lines; thread p
-    // then expands weight row p of the stage's 4 blocks into the B operand.
+    // then expands weight rows p, p + kNProd, ... of the stage's 4 blocks
+    // into the B operand.
     // The copies run kLookS stages ahead across item boundaries: the issue
     // cursor (item ii, stage ji) moves ahead of the expansion.  (The A tiles
     // come from the TMA warp.)
@@ -348,7 +342,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         const int kb0 = ji * kBS;
         unsigned char* pk = pk_ring + (gj % kPkSlots) * L::kPk;
 #pragma unroll
-        for (int it = 0; it < kChunks; ++it) {  // row q / kChunks, chunk q % kChunks of the stage's bytes
+        for (int it = 0; it < kChunks * kN / kNProd; ++it) {  // row q / kChunks, chunk q % kChunks of the stage's bytes
           const int q = it * kNProd + p;
           const int r = q / kChunks, c = q % kChunks;
           cp_async16(pk + pk_off<BITS>(r, c), wrow(r) + (size_t)kb0 * (BITS * 4) + (size_t)c * 16);
@@ -376,21 +370,25 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         const unsigned char* pk = pk_ring + (gs % kPkSlots) * L::kPk;
         unsigned char* ob = op_ring + s * L::kOpStage + L::kStageA;
 #pragma unroll
+        for (int rr = 0; rr < kN / kNProd; ++rr) {
+        const int pr = p + rr * kNProd;  // the weight row this thread expands
+#pragma unroll
         for (int c = 0; c < kBS; ++c) {
           unsigned char* dst = ob + c * L::kSubB;
           uint4 o0, o1;
           if constexpr (BITS == 4) {
-            const uint4 w = *reinterpret_cast<const uint4*>(pk + pk_off<4>(p, c));
+            const uint4 w = *reinterpret_cast<const uint4*>(pk + pk_off<4>(pr, c));
             expand_word(w.x, o0.x, o0.y);
             expand_word(w.y, o0.z, o0.w);
             expand_word(w.z, o1.x, o1.y);
             expand_word(w.w, o1.z, o1.w);
           } else {  // int8 rows are the operand as they are
-            o0 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(p, 2 * c));
-            o1 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(p, 2 * c + 1));
+            o0 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(pr, 2 * c));
+            o1 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(pr, 2 * c + 1));
           }
-          *reinterpret_cast<uint4*>(dst + op_off(p, 0)) = o0;
-          *reinterpret_cast<uint4*>(dst + op_off(p, 1)) = o1;
+          *reinterpret_cast<uint4*>(dst + op_off(pr, 0)) = o0;
+          *reinterpret_cast<uint4*>(dst + op_off(pr, 1)) = o1;
+        }
         }
       }
       fence_async_smem();  // this thread's operand writes (stores and cp.async) -> the tensor core
@@ -448,13 +446,16 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     // For each stage: once the MMA is done with the operand stage, one
     // expect_tx arrival on `full` and one TMA load of 128 rows x 128 bytes
     // (128-byte swizzle) of the row-ordered activations (gate/up) or h
-    // (down), rows [row_base + n0, +128) of the item's slot.
+    // (down), rows [row_base + n0, +128) of the item's slot; a light item (at
+    // most 32 tokens): rows [row_base + n0, +32) four times, into rows 0, 32,
+    // 64 and 96 of the tile (one per TMEM lane quadrant).
     if (lane == 0) {
       int gs = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
         const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
         const int row0 = f.slot.row_base + f.n0;
+        const bool light = f.n_valid <= 32;
         for (int j = 0; j < nst; ++j, ++gs) {
           const int s = gs % kStages;
           if (!mbar_wait(&empty_bar[s], ((gs / kStages) & 1) ^ 1, abort, err, 16)) {
@@ -463,7 +464,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           }
           unsigned char* oa = op_ring + s * L::kOpStage;
           mbar_arrive_expect_tx(&full_bar[s], L::kStageA);
-          tma_load_2d(oa, &amap, j * kBS * 32, row0, &full_bar[s]);
+          if (light) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tma_load_2d(oa + q * 32 * 128, &amap32, j * kBS * 32, row0, &full_bar[s]);
+          } else {
+            tma_load_2d(oa, &amap, j * kBS * 32, row0, &full_bar[s]);
+          }
         }
       }
     }
@@ -472,38 +478,66 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     // ------------------------------------------------------------ fold
     // warp w: TMEM lanes 32*(w%4).. (tokens); columns c0.. and c1.. (16 each):
     // gate/up: gate rows [16 c4, 16 c4 + 16) of the group and the same up
-    // rows (64 columns on); down: columns [32 c4, 32 c4 + 32)
+    // rows (64 columns on); down: columns [32 c4, 32 c4 + 32).
+    // A light item (at most 32 tokens) holds its tokens in every lane
+    // quadrant (the A tile carries them four times), and the 16 warps split
+    // the columns instead: warp (quad q, c4) takes 4 of each range,
+    // c0 + 4 q and c1 + 4 q, so the fold runs on all four schedulers.
     const int quad = warp & 3, c4 = (warp - kEpi0) >> 2;
-    const int c0 = GU ? 16 * c4 : 32 * c4;
-    const int c1 = GU ? kGroupRows + 16 * c4 : 32 * c4 + 16;
+    const int c0n = GU ? 16 * c4 : 32 * c4;
+    const int c1n = GU ? kGroupRows + 16 * c4 : 32 * c4 + 16;
     int n_done = 0;  // items this warp has folded (parity of the absmax exchange buffer)
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    const int n = quad * 32 + lane;  // this thread's token within the tile
     constexpr int kHandPerStage = kBS / kHalf;
     // isum from an accumulator read as binary32: int4 (B = 16 q): the value
     // is 0x4B400000 + 16 isum, so fma(v, 1/16, -C/16) = isum exactly (the
     // exact result is an integer below 2^22); int8 (B = q): v - C.
     constexpr float kIsumScale = BITS == 4 ? 0.0625f : 1.0f;
     constexpr float kIsumOffset = -kMagicF * kIsumScale;
-    auto write_start = [&](int buf) {  // every accumulator starts at 0x4B400000
-      const uint32_t col = tmem + lane_base + buf * kN;
-      tmem_st16_same(col + c0, kMagic);
-      tmem_st16_same(col + c1, kMagic);
-    };
-    // first use of every buffer
+    // every buffer is free for its first use
     if ((int)blockIdx.x < n_items) {
-#pragma unroll
-      for (int b = 0; b < kTBufs; ++b) write_start(b);
-      tmem_st_wait();
-      fence_before_sync();
       __syncwarp();
       if (lane == 0)
         for (int h = 0; h < kTBufs / kHalf; ++h) mbar_arrive(&tempty_bar[h]);
     }
+    // fold of nc (8 or 4) columns of each range from TMEM column col, block b
+    auto fold_cols = [&](auto ncw, uint32_t col, int c0, int c1, float dx, int b, float (&acc0)[16],
+                         float (&acc1)[16], int32_t* dbg0, int32_t* dbg1, bool valid, int h) {
+      constexpr int nc = decltype(ncw)::value;
+      uint32_t r0[nc], r1[nc];
+      if constexpr (nc == 8) {
+        tmem_ld8(col + c0 + 8 * h, r0);
+        tmem_ld8(col + c1 + 8 * h, r1);
+      } else {
+        tmem_ld4(col + c0, r0);
+        tmem_ld4(col + c1, r1);
+      }
+      tmem_ld_wait();
+#pragma unroll
+      for (int jj = 0; jj < nc; jj += 2) {
+        // S + 0x4B400000 read as binary32 is 1.5 * 2^23 + S (|S| < 2^22)
+        float v0 = __uint_as_float(r0[jj] + kMagic), v1 = __uint_as_float(r0[jj + 1] + kMagic);
+        float u0 = __uint_as_float(r1[jj] + kMagic), u1 = __uint_as_float(r1[jj + 1] + kMagic);
+        fma2c(v0, v1, kIsumScale, kIsumOffset);  // exact: (float)isum
+        fma2c(u0, u1, kIsumScale, kIsumOffset);
+        const int colw = nc * h + jj;
+        if constexpr (DBG) {
+          if (valid) {
+            dbg0[(int64_t)colw * nb + b] = (int32_t)v0;
+            dbg0[(int64_t)(colw + 1) * nb + b] = (int32_t)v1;
+            dbg1[(int64_t)colw * nb + b] = (int32_t)u0;
+            dbg1[(int64_t)(colw + 1) * nb + b] = (int32_t)u1;
+          }
+        }
+        fma2(acc0[colw], acc0[colw + 1], dx, dx, v0, v1);
+        fma2(acc1[colw], acc1[colw + 1], dx, dx, u0, u1);
+      }
+    };
     int gh = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      bool active, valid;
-      const float2* drow;
+      bool active, valid, light;
+      int n, c0, c1;
+      const float* drow;  // the token's Q8 scales, one per block
       float acc0[16], acc1[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -515,9 +549,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       int32_t* dbg1 = nullptr;
       {  // the item's description is read again for the epilogue: fewer live registers in the block loop
         const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
-        active = quad * 32 < f.n_valid;  // warp-uniform
+        light = f.n_valid <= 32;  // CTA-uniform
+        n = light ? lane : quad * 32 + lane;  // this thread's token within the tile
+        c0 = light ? c0n + 4 * quad : c0n;
+        c1 = light ? c1n + 4 * quad : c1n;
+        active = light || quad * 32 < f.n_valid;  // warp-uniform
         valid = n < f.n_valid;
-        drow = reinterpret_cast<const float2*>(ad + (valid ? item_token_row(f, GU, perm, top_k, n) : 0) * nb);
+        drow = ad + (valid ? item_token_row(f, GU, perm, top_k, n) : 0) * nb;
       if constexpr (DBG) {
         if (valid) {
           const int nbh = hidden / 32, nbi = inter / 32;
@@ -540,14 +578,19 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         }
       }
       }
-      // the token's Q8 scales of a hand-off (kHalf = 2 blocks), one hand-off ahead
-      float2 dnext = valid ? __ldg(drow) : make_float2(0.f, 0.f);
+      // the token's Q8 scales of a hand-off (kHalf blocks), one hand-off ahead
+      float dnext[kHalf], dcur[kHalf];
+#pragma unroll
+      for (int i = 0; i < kHalf; ++i) dnext[i] = valid ? __ldg(drow + i) : 0.0f;
       for (int j = 0; j < nst; ++j) {
 #pragma unroll
         for (int hs = 0; hs < kHandPerStage; ++hs, ++gh) {
-          const float2 dcur = dnext;
           const int hn = j * kHandPerStage + hs + 1;  // next hand-off of this item
-          if (valid && hn < nst * kHandPerStage) dnext = __ldg(drow + hn);
+#pragma unroll
+          for (int i = 0; i < kHalf; ++i) {
+            dcur[i] = dnext[i];
+            if (valid && hn < nst * kHandPerStage) dnext[i] = __ldg(drow + hn * kHalf + i);
+          }
           const int hb = gh % (kTBufs / kHalf);
           // warp-uniform: tcgen05.ld is a warp-wide instruction
           const bool ok =
@@ -558,88 +601,100 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
             const int b = j * kBS + hs * kHalf + i;  // block of this item
             const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
             if (active && ok) {
-              const float dx = i == 0 ? dcur.x : dcur.y;
-              // 8 columns of each range at a time (one wait per pair of
-              // loads), so that only 16 TMEM values are live
+              if (light) {
+                fold_cols(std::integral_constant<int, 4>{}, col, c0, c1, dcur[i], b, acc0, acc1, dbg0, dbg1, valid, 0);
+              } else {
+                // 8 columns of each range at a time (16 TMEM values live)
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                uint32_t r0[8], r1[8];
-                tmem_ld8(col + c0 + 8 * h, r0);
-                tmem_ld8(col + c1 + 8 * h, r1);
-                tmem_ld_wait();
-#pragma unroll
-                for (int jj = 0; jj < 8; jj += 2) {
-                  float v0 = __uint_as_float(r0[jj]), v1 = __uint_as_float(r0[jj + 1]);
-                  float u0 = __uint_as_float(r1[jj]), u1 = __uint_as_float(r1[jj + 1]);
-                  fma2c(v0, v1, kIsumScale, kIsumOffset);  // exact: (float)isum
-                  fma2c(u0, u1, kIsumScale, kIsumOffset);
-                  if constexpr (DBG) {
-                    if (valid) {
-                      const int colw = 8 * h + jj;
-                      dbg0[(int64_t)colw * nb + b] = (int32_t)v0;
-                      dbg0[(int64_t)(colw + 1) * nb + b] = (int32_t)v1;
-                      dbg1[(int64_t)colw * nb + b] = (int32_t)u0;
-                      dbg1[(int64_t)(colw + 1) * nb + b] = (int32_t)u1;
-                    }
-                  }
-                  fma2(acc0[8 * h + jj], acc0[8 * h + jj + 1], dx, dx, v0, v1);
-                  fma2(acc1[8 * h + jj], acc1[8 * h + jj + 1], dx, dx, u0, u1);
-                }
+                for (int h = 0; h < 2; ++h)
+                  fold_cols(std::integral_constant<int, 8>{}, col, c0, c1, dcur[i], b, acc0, acc1, dbg0, dbg1, valid,
+                            h);
               }
             }
-            write_start(hb * kHalf + i);  // the buffer's next use starts at 0x4B400000 again
           }
-          tmem_st_wait();
           fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty_bar[hb]);  // the pair of TMEM buffers may be rewritten now
+          if (lane == 0) mbar_arrive(&tempty_bar[hb]);  // the hand-off's TMEM buffers may be rewritten now
         }
       }
-      if (active) {  // warp-uniform, and the same for both warps of a pair (one quadrant)
-        const bool go = !*abort;  // this warp's writes only: both warps meet the barrier regardless
+      if (active) {  // warp-uniform; the same for all warps that share a Q8 block of h
+        const bool go = !*abort;  // this warp's writes only: the warps meet the barrier regardless
         const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
         const int64_t row = (int64_t)f.slot.row_base + f.n0 + n;
+        const int nr = light ? 4 : 16;  // rows of each range this thread holds
         if constexpr (GU) {
-          const int o = f.m0 + c0;  // this thread's 16 intermediate rows (half of a Q8 block of h)
+          const int o = f.m0 + c0;  // this thread's first intermediate row
           const float* sgp = tab.gate_s[f.slot.table_idx] + o;
           const float* sup = tab.up_s[f.slot.table_idx] + o;
           float amax = 0.0f;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float gv = __fmul_rn(__ldg(sgp + j), acc0[j]);
-            const float u = __fmul_rn(__ldg(sup + j), acc1[j]);
-            acc0[j] = __fmul_rn(__fmul_rn(gv, sigmoid_cw(gv)), u);
-            amax = fmaxf(amax, fabsf(acc0[j]));
+            if (j < nr) {
+              const float gv = __fmul_rn(__ldg(sgp + j), acc0[j]);
+              const float u = __fmul_rn(__ldg(sup + j), acc1[j]);
+              acc0[j] = __fmul_rn(__fmul_rn(gv, sigmoid_cw(gv)), u);
+              amax = fmaxf(amax, fabsf(acc0[j]));
+            }
           }
-          // the block's absmax: this half's and the partner warp's (c4 ^ 1)
+          // the block's absmax over the warps that hold its 32 rows: the
+          // partner warp (c4 ^ 1) of this quadrant, or (light) the 8 warps
+          // c4 in {c4 & ~1, c4 | 1} of all quadrants
           float* xa = &s_amax[n_done & 1][0][0];
           xa[(warp - kEpi0) * 32 + lane] = valid ? amax : 0.0f;
-          named_bar(2 + quad * 2 + (c4 >> 1), 64);
-          amax = fmaxf(amax, xa[(warp - kEpi0 + 4 * ((c4 ^ 1) - c4)) * 32 + lane]);
+          if (light) {
+            named_bar(10 + (c4 >> 1), 256);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int cc = (c4 & ~1) + (k >> 2), qq = k & 3;  // fold warp with c4 = cc in quadrant qq
+              amax = fmaxf(amax, xa[(4 * cc + ((qq - kEpi0) & 3)) * 32 + lane]);
+            }
+          } else {
+            named_bar(2 + quad * 2 + (c4 >> 1), 64);
+            amax = fmaxf(amax, xa[(warp - kEpi0 + 4 * ((c4 ^ 1) - c4)) * 32 + lane]);
+          }
           const float d = __fdiv_rn(amax, 127.0f);
           if (go && valid) {
-            // q in the operand order (int4 weights: per 8 elements 0,2,4,6,1,3,5,7;
-            // int8: the elements' order)
-            uint32_t pk[4];
+            if (!light) {
+              // q in the operand order (int4 weights: per 8 elements 0,2,4,6,1,3,5,7;
+              // int8: the elements' order)
+              uint32_t pk[4];
 #pragma unroll
-            for (int e8 = 0; e8 < 2; ++e8) {
-              uint32_t lo = 0, hi = 0;
+              for (int e8 = 0; e8 < 2; ++e8) {
+                uint32_t lo = 0, hi = 0;
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int qe = q8_of(acc0[8 * e8 + 2 * i], d), qo = q8_of(acc0[8 * e8 + 2 * i + 1], d);
-                lo |= ((uint32_t)qe & 0xFFu) << (8 * i);
-                hi |= ((uint32_t)qo & 0xFFu) << (8 * i);
+                for (int i = 0; i < 4; ++i) {
+                  const int qe = q8_of(acc0[8 * e8 + 2 * i], d), qo = q8_of(acc0[8 * e8 + 2 * i + 1], d);
+                  lo |= ((uint32_t)qe & 0xFFu) << (8 * i);
+                  hi |= ((uint32_t)qo & 0xFFu) << (8 * i);
+                }
+                if constexpr (BITS == 4) {
+                  pk[2 * e8] = lo;
+                  pk[2 * e8 + 1] = hi;
+                } else {  // back to element order: even / odd bytes interleaved
+                  pk[2 * e8] = __byte_perm(lo, hi, 0x5140);
+                  pk[2 * e8 + 1] = __byte_perm(lo, hi, 0x7362);
+                }
               }
+              *reinterpret_cast<uint4*>(hr + row * inter + o) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            } else {
+              // 4 rows o.. (o % 8 is 0 or 4): int8 weights, 4 bytes in element
+              // order; int4 weights, element e of the group of 8 at byte
+              // e / 2 (even e) or 4 + e / 2 (odd e)
+              int8_t* hg = hr + row * inter + (o & ~7);
               if constexpr (BITS == 4) {
-                pk[2 * e8] = lo;
-                pk[2 * e8 + 1] = hi;
-              } else {  // back to element order: even / odd bytes interleaved
-                pk[2 * e8] = __byte_perm(lo, hi, 0x5140);
-                pk[2 * e8 + 1] = __byte_perm(lo, hi, 0x7362);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const int e = (o & 7) + j;
+                  hg[(e & 1) ? 4 + (e >> 1) : (e >> 1)] = (int8_t)q8_of(acc0[j], d);
+                }
+              } else {
+                uint32_t w = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) w |= ((uint32_t)q8_of(acc0[j], d) & 0xFFu) << (8 * j);
+                *reinterpret_cast<uint32_t*>(hr + row * inter + o) = w;
               }
             }
-            *reinterpret_cast<uint4*>(hr + row * inter + o) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            if ((c4 & 1) == 0) hd[row * (inter / 32) + (o >> 5)] = d;
+            if ((c4 & 1) == 0 && (!light || quad == 0)) hd[row * (inter / 32) + (o >> 5)] = d;
           }
         } else if (go && valid) {
           const float* sdp = tab.down_s[f.slot.table_idx] + f.m0;
@@ -647,12 +702,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           float4* dst1 = reinterpret_cast<float4*>(y + row * hidden + f.m0 + c1);
 #pragma unroll
           for (int j = 0; j < 16; j += 4) {
-            const float4 s0 = __ldg(reinterpret_cast<const float4*>(sdp + c0 + j));
-            const float4 s1 = __ldg(reinterpret_cast<const float4*>(sdp + c1 + j));
-            dst0[j / 4] = make_float4(__fmul_rn(s0.x, acc0[j]), __fmul_rn(s0.y, acc0[j + 1]),
-                                      __fmul_rn(s0.z, acc0[j + 2]), __fmul_rn(s0.w, acc0[j + 3]));
-            dst1[j / 4] = make_float4(__fmul_rn(s1.x, acc1[j]), __fmul_rn(s1.y, acc1[j + 1]),
-                                      __fmul_rn(s1.z, acc1[j + 2]), __fmul_rn(s1.w, acc1[j + 3]));
+            if (j < nr) {
+              const float4 s0 = __ldg(reinterpret_cast<const float4*>(sdp + c0 + j));
+              const float4 s1 = __ldg(reinterpret_cast<const float4*>(sdp + c1 + j));
+              dst0[j / 4] = make_float4(__fmul_rn(s0.x, acc0[j]), __fmul_rn(s0.y, acc0[j + 1]),
+                                        __fmul_rn(s0.z, acc0[j + 2]), __fmul_rn(s0.w, acc0[j + 3]));
+              dst1[j / 4] = make_float4(__fmul_rn(s1.x, acc1[j]), __fmul_rn(s1.y, acc1[j + 1]),
+                                        __fmul_rn(s1.z, acc1[j + 2]), __fmul_rn(s1.w, acc1[j + 3]));
+            }
           }
         }
       }
@@ -713,8 +770,9 @@ bool prefill_supported(int hidden, int inter) {
 namespace {
 
 // A 2D tensor map over `rows` int8 rows of `cols` bytes (row-major), box
-// 128 bytes x kM rows, 128-byte swizzle: the A operand tiles.
-cudaError_t make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int cols) {
+// 128 bytes x box_rows rows, 128-byte swizzle: the A operand tiles (kM rows,
+// or 32 for the quarters of a light item's tile).
+cudaError_t make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
     cudaDriverEntryPointQueryResult q{};
@@ -726,7 +784,7 @@ cudaError_t make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int co
   }
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols};
-  const cuuint32_t box[2] = {128, (cuuint32_t)kM};
+  const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -741,7 +799,8 @@ namespace {
 // The two GEMMs of one weight width; DBG: the capture instantiation.
 template <int BITS, bool DBG>
 cudaError_t prefill_pair(const GateUpTable& gu, const DownTable& dn, const CUtensorMap& map_x,
-                         const CUtensorMap& map_h, const Slot* slots, const Tile* t, const int32_t* n_tiles,
+                         const CUtensorMap& map_x32, const CUtensorMap& map_h, const CUtensorMap& map_h32,
+                         const Slot* slots, const Tile* t, const int32_t* n_tiles,
                          const int32_t* perm, int K, const float* xd, int hidden, int inter, int8_t* hri, float* hd,
                          float* y, int32_t* err, int grid, DbgArgs dbg, cudaStream_t st, cudaEvent_t ev_mid) {
   static int mask_gu[64] = {}, mask_dn[64] = {};
@@ -750,11 +809,11 @@ cudaError_t prefill_pair(const GateUpTable& gu, const DownTable& dn, const CUten
   if ((e = smem_opt_in(prefill_kernel<true, BITS, DBG, GateUpTable>, (int)smem, mask_gu)) != cudaSuccess) return e;
   if ((e = smem_opt_in(prefill_kernel<false, BITS, DBG, DownTable>, (int)smem, mask_dn)) != cudaSuccess) return e;
   prefill_kernel<true, BITS, DBG, GateUpTable><<<grid, kThreadsP, smem, st>>>(
-      gu, map_x, slots, t, n_tiles, perm, K, xd, hidden, inter, hri, hd, y, err, dbg);
+      gu, map_x, map_x32, slots, t, n_tiles, perm, K, xd, hidden, inter, hri, hd, y, err, dbg);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecordWithFlags(ev_mid, st, cudaEventRecordExternal)) != cudaSuccess) return e;
   prefill_kernel<false, BITS, DBG, DownTable><<<grid, kThreadsP, smem, st>>>(
-      dn, map_h, slots, t, n_tiles, perm, K, hd, hidden, inter, hri, hd, y, err, dbg);
+      dn, map_h, map_h32, slots, t, n_tiles, perm, K, hd, hidden, inter, hri, hd, y, err, dbg);
   return cudaGetLastError();
 }
 
@@ -777,9 +836,11 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
   build_tiles_kernel<<<1, 32, 0, st>>>(slots, n_slots, t, n_tiles);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap map_x, map_h;
-  if ((e = make_rows_map(&map_x, xr, rows, hidden)) != cudaSuccess) return e;
-  if ((e = make_rows_map(&map_h, hr, rows, inter)) != cudaSuccess) return e;
+  CUtensorMap map_x, map_h, map_x32, map_h32;
+  if ((e = make_rows_map(&map_x, xr, rows, hidden, kM)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&map_h, hr, rows, inter, kM)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&map_x32, xr, rows, hidden, 32)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&map_h32, hr, rows, inter, 32)) != cudaSuccess) return e;
   static int sms_cache[64] = {};
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -791,13 +852,13 @@ cudaError_t launch_prefill_experts(const GateUpTable& gu, const DownTable& dn, c
   int8_t* hri = reinterpret_cast<int8_t*>(hr);
   const DbgArgs dbg{dbg_buf, n_experts, n_shared};
   if (bits == 8)
-    return dbg_buf ? prefill_pair<8, true>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, hidden, inter, hri,
+    return dbg_buf ? prefill_pair<8, true>(gu, dn, map_x, map_x32, map_h, map_h32, slots, t, n_tiles, perm, K, xd, hidden, inter, hri,
                                            hd, y, err, grid, dbg, st, ev_mid)
-                   : prefill_pair<8, false>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, hidden, inter, hri,
+                   : prefill_pair<8, false>(gu, dn, map_x, map_x32, map_h, map_h32, slots, t, n_tiles, perm, K, xd, hidden, inter, hri,
                                             hd, y, err, grid, dbg, st, ev_mid);
-  return dbg_buf ? prefill_pair<4, true>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, hidden, inter, hri, hd,
+  return dbg_buf ? prefill_pair<4, true>(gu, dn, map_x, map_x32, map_h, map_h32, slots, t, n_tiles, perm, K, xd, hidden, inter, hri, hd,
                                          y, err, grid, dbg, st, ev_mid)
-                 : prefill_pair<4, false>(gu, dn, map_x, map_h, slots, t, n_tiles, perm, K, xd, hidden, inter, hri, hd,
+                 : prefill_pair<4, false>(gu, dn, map_x, map_x32, map_h, map_h32, slots, t, n_tiles, perm, K, xd, hidden, inter, hri, hd,
                                           y, err, grid, dbg, st, ev_mid);
 }
 
