@@ -72,8 +72,17 @@ constexpr int kM = 128;        // tokens per tile (MMA M, TMEM lanes)
 constexpr int kN = 128;        // output columns per item (MMA N): 64 gate + 64 up rows, or 128 down rows
 constexpr int kBS = 4;         // Q8 blocks per operand stage (K = 128)
 constexpr int kStages = 4;     // operand stages
-constexpr int kLookS = 2;      // stages the producers' copies run ahead
-constexpr int kPkSlots = kLookS + 2;  // packed-weight slots: a slot is rewritten only after every producer expanded it
+// The producers' packed-weight copies run kLookS stages ahead, into kPkSlots
+// = kLookS + 2 slots (a slot is rewritten only after every producer expanded
+// it) of kPk bytes: int4 rows (64 B per stage) 6 ahead in 8 slots of 8 KB,
+// int8 rows (128 B) 2 ahead in 4 slots of 16 KB -- the same 64 KB.
+template <int BITS>
+struct PkRing {
+  static constexpr int kLookS = BITS == 4 ? 6 : 2;
+  static constexpr int kPkSlots = kLookS + 2;
+  static constexpr int kPk = 128 * 4 * BITS * 4;
+};
+static_assert(PkRing<4>::kPkSlots * PkRing<4>::kPk == PkRing<8>::kPkSlots * PkRing<8>::kPk, "one ring size");
 constexpr int kHalf = 2;       // Q8 blocks per accumulator hand-off (MMA -> fold): 1 or 2
 constexpr int kTBufs = 4;      // TMEM accumulators (one per block), handed off in pairs
 constexpr int kProdWarps = 2;
@@ -95,9 +104,9 @@ struct PSmem {
   static constexpr int kStageA = kM * 128;          // A: 128 token rows x 128 int8 (4 blocks), 128B-swizzled
   static constexpr int kSubB = kN * 32;             // B, one block: 128 weight rows x 32 bytes
   static constexpr int kOpStage = kStageA + kBS * kSubB;
-  static constexpr int kPk = kN * kBS * 32;         // weights of one stage as copied (64 B per row int4, 128 B int8)
+  static constexpr int kPkRing = PkRing<8>::kPkSlots * PkRing<8>::kPk;  // packed-weight copies (either width)
   __host__ __device__ static constexpr size_t bytes() {
-    return 1024 + (size_t)kStages * kOpStage + (size_t)kPkSlots * kPk;
+    return 1024 + (size_t)kStages * kOpStage + (size_t)kPkRing;
   }
 };
 
@@ -286,7 +295,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
 
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1 KB aligned
   unsigned char* op_ring = smem;                                  // [kStages][A | B: kBS x kSubB]
-  unsigned char* pk_ring = op_ring + kStages * L::kOpStage;       // [kPkSlots][128 rows][64 B]
+  unsigned char* pk_ring = op_ring + kStages * L::kOpStage;       // [kPkSlots][128 rows][BITS * 16 B]
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -318,6 +327,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     // cursor (item ii, stage ji) moves ahead of the expansion.  (The A tiles
     // come from the TMA warp.)
     const int p = threadIdx.x;
+    constexpr int kLookS = PkRing<BITS>::kLookS, kPkSlots = PkRing<BITS>::kPkSlots, kPk = PkRing<BITS>::kPk;
     const size_t rb = (size_t)dim_in * BITS / 8;  // bytes per weight row
     constexpr int kChunks = BITS == 4 ? 4 : 8;      // 16-byte chunks per row per stage
     const int n_mine = blockIdx.x < n_items ? (n_items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
@@ -340,7 +350,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     auto issue = [&](int gj) {
       if (gj < total) {
         const int kb0 = ji * kBS;
-        unsigned char* pk = pk_ring + (gj % kPkSlots) * L::kPk;
+        unsigned char* pk = pk_ring + (gj % kPkSlots) * kPk;
 #pragma unroll
         for (int it = 0; it < kChunks * kN / kNProd; ++it) {  // row q / kChunks, chunk q % kChunks of the stage's bytes
           const int q = it * kNProd + p;
@@ -367,28 +377,45 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       const int s = gs % kStages;
       // the MMA is done with the operand stage's previous contents
       if (mbar_wait(&empty_bar[s], ((gs / kStages) & 1) ^ 1, abort, err, 10) && !*abort) {
-        const unsigned char* pk = pk_ring + (gs % kPkSlots) * L::kPk;
+        const unsigned char* pk = pk_ring + (gs % kPkSlots) * kPk;
         unsigned char* ob = op_ring + s * L::kOpStage + L::kStageA;
+        if constexpr (BITS == 4) {
+          // all of this thread's packed words first, then the expansion and
+          // the stores
+          uint4 w[kN / kNProd][kBS];
 #pragma unroll
-        for (int rr = 0; rr < kN / kNProd; ++rr) {
-        const int pr = p + rr * kNProd;  // the weight row this thread expands
+          for (int rr = 0; rr < kN / kNProd; ++rr)
 #pragma unroll
-        for (int c = 0; c < kBS; ++c) {
-          unsigned char* dst = ob + c * L::kSubB;
-          uint4 o0, o1;
-          if constexpr (BITS == 4) {
-            const uint4 w = *reinterpret_cast<const uint4*>(pk + pk_off<4>(pr, c));
-            expand_word(w.x, o0.x, o0.y);
-            expand_word(w.y, o0.z, o0.w);
-            expand_word(w.z, o1.x, o1.y);
-            expand_word(w.w, o1.z, o1.w);
-          } else {  // int8 rows are the operand as they are
-            o0 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(pr, 2 * c));
-            o1 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(pr, 2 * c + 1));
+            for (int c = 0; c < kBS; ++c)
+              w[rr][c] = *reinterpret_cast<const uint4*>(pk + pk_off<4>(p + rr * kNProd, c));
+#pragma unroll
+          for (int rr = 0; rr < kN / kNProd; ++rr) {
+            const int pr = p + rr * kNProd;  // the weight row this thread expands
+#pragma unroll
+            for (int c = 0; c < kBS; ++c) {
+              unsigned char* dst = ob + c * L::kSubB;
+              uint4 o0, o1;
+              expand_word(w[rr][c].x, o0.x, o0.y);
+              expand_word(w[rr][c].y, o0.z, o0.w);
+              expand_word(w[rr][c].z, o1.x, o1.y);
+              expand_word(w[rr][c].w, o1.z, o1.w);
+              *reinterpret_cast<uint4*>(dst + op_off(pr, 0)) = o0;
+              *reinterpret_cast<uint4*>(dst + op_off(pr, 1)) = o1;
+            }
           }
-          *reinterpret_cast<uint4*>(dst + op_off(pr, 0)) = o0;
-          *reinterpret_cast<uint4*>(dst + op_off(pr, 1)) = o1;
-        }
+        } else {  // int8 rows are the operand as they are
+#pragma unroll
+          for (int rr = 0; rr < kN / kNProd; ++rr) {
+            const int pr = p + rr * kNProd;
+#pragma unroll
+            for (int c = 0; c < kBS; ++c) {
+              unsigned char* dst = ob + c * L::kSubB;
+              const uint4 o0 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(pr, 2 * c));
+              const uint4 o1 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(pr, 2 * c + 1));
+              *reinterpret_cast<uint4*>(dst + op_off(pr, 0)) = o0;
+              *reinterpret_cast<uint4*>(dst + op_off(pr, 1)) = o1;
+            }
+          }
         }
       }
       fence_async_smem();  // this thread's operand writes (stores and cp.async) -> the tensor core
@@ -500,19 +527,11 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       if (lane == 0)
         for (int h = 0; h < kTBufs / kHalf; ++h) mbar_arrive(&tempty_bar[h]);
     }
-    // fold of nc (8 or 4) columns of each range from TMEM column col, block b
-    auto fold_cols = [&](auto ncw, uint32_t col, int c0, int c1, float dx, int b, float (&acc0)[16],
+    // fold of nc (8 or 4) loaded columns of each range (r0, r1), block b,
+    // into accumulators nc h ..
+    auto fold_cols = [&](auto ncw, const uint32_t* r0, const uint32_t* r1, float dx, int b, float (&acc0)[16],
                          float (&acc1)[16], int32_t* dbg0, int32_t* dbg1, bool valid, int h) {
       constexpr int nc = decltype(ncw)::value;
-      uint32_t r0[nc], r1[nc];
-      if constexpr (nc == 8) {
-        tmem_ld8(col + c0 + 8 * h, r0);
-        tmem_ld8(col + c1 + 8 * h, r1);
-      } else {
-        tmem_ld4(col + c0, r0);
-        tmem_ld4(col + c1, r1);
-      }
-      tmem_ld_wait();
 #pragma unroll
       for (int jj = 0; jj < nc; jj += 2) {
         // S + 0x4B400000 read as binary32 is 1.5 * 2^23 + S (|S| < 2^22)
@@ -600,17 +619,32 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           for (int i = 0; i < kHalf; ++i) {
             const int b = j * kBS + hs * kHalf + i;  // block of this item
             const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
-            if (active && ok) {
-              if (light) {
-                fold_cols(std::integral_constant<int, 4>{}, col, c0, c1, dcur[i], b, acc0, acc1, dbg0, dbg1, valid, 0);
-              } else {
-                // 8 columns of each range at a time (16 TMEM values live)
+            if (active && ok && !light) {
+              // 8 columns of each range at a time (16 TMEM values live)
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-                  fold_cols(std::integral_constant<int, 8>{}, col, c0, c1, dcur[i], b, acc0, acc1, dbg0, dbg1, valid,
-                            h);
+              for (int h = 0; h < 2; ++h) {
+                uint32_t r0[8], r1[8];
+                tmem_ld8(col + c0 + 8 * h, r0);
+                tmem_ld8(col + c1 + 8 * h, r1);
+                tmem_ld_wait();
+                fold_cols(std::integral_constant<int, 8>{}, r0, r1, dcur[i], b, acc0, acc1, dbg0, dbg1, valid, h);
               }
             }
+          }
+          if (active && ok && light) {
+            // 4 columns of each range per block: the hand-off's loads, then one wait
+            uint32_t r[kHalf][2][4];
+#pragma unroll
+            for (int i = 0; i < kHalf; ++i) {
+              const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
+              tmem_ld4(col + c0, r[i][0]);
+              tmem_ld4(col + c1, r[i][1]);
+            }
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < kHalf; ++i)
+              fold_cols(std::integral_constant<int, 4>{}, r[i][0], r[i][1], dcur[i], j * kBS + hs * kHalf + i, acc0,
+                        acc1, dbg0, dbg1, valid, 0);
           }
           fence_before_sync();
           __syncwarp();
