@@ -308,10 +308,12 @@ def run_suite(layers, cfg, dev, stream, peak_gbs, only=None, tokens=None):
         return len(torch.unique(idx)) + S
 
     def issued(layer, x):
-        """Experts streamed by the prepared decode path: once per launch of
-        at most 8 tokens (a 16-token batch is two launches)."""
+        """Expert reads of the prepared decode path (one launch of up to 16
+        tokens): a slot holds at most 8 tokens, so an expert with more of the
+        batch's tokens (the shared expert above 8 tokens) is read once per 8."""
         _, idx, _ = coli.moe_route(layer, x)
-        return sum(len(torch.unique(idx[i:i + 8])) + S for i in range(0, idx.shape[0], 8))
+        per_expert = torch.bincount(idx.flatten().long())
+        return int(((per_expert + 7) // 8).sum().item()) + S * ((x.shape[0] + 7) // 8)
 
     def time_steps(fn, n_steps, graph):
         if graph:

@@ -140,13 +140,12 @@ Workspace layout(const coli_moe_config& c, int64_t T) {
   L.hq = take(rows * I);  // h as int8 rows (Q8 of h; the tensor-core path's down operand)
   L.xr = take(tc ? rows * H : 0);
   L.hd = take(rows * (I / 32) * 4);
-  // the streaming decode kernel (prepared layers, up to kStreamChunked
-  // tokens in calls of <= kStreamMaxTok): (d, c16) of every h block of a
-  // call, its x planes' (d, c16), and its counters
-  const bool sm = T <= kStreamChunked;
-  const int64_t Tc = T < kStreamMaxTok ? T : kStreamMaxTok;
-  L.hdc = take(sm ? Tc * (K + S) * (I / 32) * 8 : 0);
-  L.xdc = take(sm ? Tc * (H / 32) * 8 : 0);  // with xq: the x planes the router kernel writes for > 2 tokens
+  // the streaming decode kernel (prepared layers, up to kStreamMaxTok
+  // tokens): (d, c16) of every h block of a call, its x planes' (d, c16),
+  // and its counters
+  const bool sm = T <= kStreamMaxTok;
+  L.hdc = take(sm ? T * (K + S) * (I / 32) * 8 : 0);
+  L.xdc = take(sm ? T * (H / 32) * 8 : 0);  // with xq: the x planes the router kernel writes for > 2 tokens
   L.ctr = take(sm ? (size_t)kStreamMaxSlots * 4 : 0);
   L.y = take(rows * H * 4);
   L.xn = take(T * H * 4);
@@ -218,46 +217,38 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   int32_t* status = at<int32_t>(ws, W.status);
   const int bits = bits_of(c);
   const bool aligned16 = ((uintptr_t)x & 15) == 0;
-  const int Tc = (int)(T < kStreamMaxTok ? T : kStreamMaxTok);
-  if (L->prepared != nullptr && aligned16 && T <= kStreamChunked && stream_supported(H, I, bits, Tc, K, S, E)) {
-    // decode on the streaming copy: per call of <= kStreamMaxTok tokens, 2
-    // kernels, the second launched with PDL (tokens are independent, so a
-    // larger batch is the same forward in pieces)
+  if (L->prepared != nullptr && aligned16 && T <= kStreamMaxTok && stream_supported(H, I, bits, (int)T, K, S, E)) {
+    // decode on the streaming copy: 2 kernels, the second launched with PDL
     int32_t* ctr = at<int32_t>(ws, W.ctr);
-    const size_t P = 2 * (size_t)I * (H / 32) + (size_t)H * (I / 32);  // capture words per (token, expert)
-    for (int64_t t0 = 0; t0 < T; t0 += kStreamMaxTok) {
-      const int Tn = (int)(T - t0 < kStreamMaxTok ? T - t0 : kStreamMaxTok);
-      // up to 2 tokens the streaming kernel quantises x itself (so that the
-      // shared expert starts before the router kernel ends); more tokens take
-      // the router kernel's planes
-      int8_t* xpl = Tn > 2 ? xq : nullptr;
-      float2* xdcp = Tn > 2 ? at<float2>(ws, W.xdc) : nullptr;
-      CHECK_LAUNCH(launch_router_decode(x + t0 * H, L->w_router, Tn, E, H, scores, nullptr, nullptr,
-                                        clear_status && t0 == 0 ? status : nullptr, ctr, kStreamMaxSlots, st, xpl,
-                                        xdcp));
-      if (t0 == 0) CHECK_LAUNCH(mark(0));
-      StreamArgs a{};
-      a.prep = static_cast<const unsigned char*>(L->prepared);
-      a.g = stream_geom(H, I, bits);
-      a.E = E;
-      a.K = K;
-      a.S = S;
-      a.T = Tn;
-      a.norm = c.norm_topk_prob;
-      a.rsf = c.routed_scaling_factor;
-      a.scores = scores;
-      a.bias = L->bias;
-      a.x = x + t0 * H;
-      a.xpl_g = xpl;
-      a.xdc_g = xdcp;
-      a.hpl = hq;
-      a.hdc = at<float2>(ws, W.hdc);
-      a.out = out + t0 * H;
-      a.h_ready = ctr;
-      a.status = status;
-      a.dbg = capture ? capture + (size_t)t0 * (K + S) * P : nullptr;
-      CHECK_LAUNCH(launch_expert_stream(a, st));
-    }
+    // up to 2 tokens the streaming kernel quantises x itself (so that the
+    // shared expert starts before the router kernel ends); more tokens take
+    // the router kernel's planes
+    int8_t* xpl = T > 2 ? xq : nullptr;
+    float2* xdcp = T > 2 ? at<float2>(ws, W.xdc) : nullptr;
+    CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, nullptr, nullptr,
+                                      clear_status ? status : nullptr, ctr, kStreamMaxSlots, st, xpl, xdcp));
+    CHECK_LAUNCH(mark(0));
+    StreamArgs a{};
+    a.prep = static_cast<const unsigned char*>(L->prepared);
+    a.g = stream_geom(H, I, bits);
+    a.E = E;
+    a.K = K;
+    a.S = S;
+    a.T = (int)T;
+    a.norm = c.norm_topk_prob;
+    a.rsf = c.routed_scaling_factor;
+    a.scores = scores;
+    a.bias = L->bias;
+    a.x = x;
+    a.xpl_g = xpl;
+    a.xdc_g = xdcp;
+    a.hpl = hq;
+    a.hdc = at<float2>(ws, W.hdc);
+    a.out = out;
+    a.h_ready = ctr;
+    a.status = status;
+    a.dbg = capture;
+    CHECK_LAUNCH(launch_expert_stream(a, st));
     CHECK_LAUNCH(mark(1));
     CHECK_LAUNCH(mark(2));
     return COLI_OK;
@@ -265,7 +256,7 @@ coli_status layer_forward(const coli_moe_layer* L, const float* x, int64_t T, fl
   if (bits == 4 && T <= kDecodeMaxTok && decode_supported(H, I)) {
     if (capture != nullptr)
       return fail(COLI_EINVAL, "%s: the partials capture covers the streaming (prepared layer, <= %d tokens) and "
-                  "tensor-core kernels, not this call's decode kernels", fn, kStreamChunked);
+                  "tensor-core kernels, not this call's decode kernels", fn, kStreamMaxTok);
     // decode: 5 kernels, the last four launched with PDL
     CHECK_LAUNCH(launch_router_decode(x, L->w_router, (int)T, E, H, scores, xq, xd, clear_status ? status : nullptr,
                                       nullptr, 0, st));

@@ -51,8 +51,16 @@ namespace coli {
 namespace {
 
 constexpr int kSW = 8;                               // warps per CTA (all compute; lane 0 also copies)
-constexpr int kMaxPairsS = kStreamMaxTok * kMaxTopK;  // (token, k) pairs of a batch
-constexpr int kMaxSlotsS = kStreamMaxSlots;          // slots: shared + distinct routed experts
+// Tokens, (token, k) pairs and slots of a launch of the instance for slots
+// of TT tokens: batches of up to TT tokens, except the largest TT, which
+// takes every batch up to kStreamMaxTok.
+template <int TT>
+struct StreamTables {
+  static constexpr int kTok = TT < kStreamSlotTok ? TT : kStreamMaxTok;
+  static constexpr int kPairs = kTok * kMaxTopK;
+  static constexpr int kSlots = ((kTok + TT - 1) / TT) * kMaxShared + kTok * kMaxTopK;
+};
+static_assert(StreamTables<kStreamSlotTok>::kSlots == kStreamMaxSlots, "the counters cover every slot");
 constexpr int kErrHReady = 25;                       // status: gave up waiting for a slot's h
 constexpr int kErrHStaged = 26;                      // status: gave up waiting for a slot's staged h
 constexpr int kErrHPair = 27;                        // status: gave up waiting for a pair's h buffer
@@ -83,10 +91,17 @@ struct StreamHRing {
   static constexpr bool value = TT == 4;
 };
 
+// Batches of more than kStreamSlotTok tokens read the x planes (the router
+// kernel's) from global memory through L1 instead of shared memory.
 template <int TT>
-__host__ __device__ inline size_t stream_smem_bytes(const StreamGeom& g, int n_sms, int n_rows) {
+__host__ __device__ inline int stream_x_staged(int n_tok) {
+  return n_tok <= kStreamSlotTok ? TT : 0;
+}
+
+template <int TT>
+__host__ __device__ inline size_t stream_smem_bytes(const StreamGeom& g, int n_sms, int n_tok, int n_rows) {
   const size_t ring = (size_t)kSW * kR * kStreamStageMax;  // 8 KB stages
-  const size_t xs = (size_t)TT * g.nbh * 40;               // x planes (32 B) + (d, c16) per block
+  const size_t xs = (size_t)stream_x_staged<TT>(n_tok) * g.nbh * 40;  // x planes (32 B) + (d, c16) per block
   const size_t hs = StreamHStaged<TT>::value ? (size_t)n_rows * g.nbi * 40              // h planes + (d, c16)
                     : StreamHRing<TT>::value  ? (size_t)kHRing * TT * g.nbi * 40 : 0;  // per slot buffer
   return 1024 + ring + xs + stream_y_bytes(g, n_sms, n_rows) + hs;
@@ -382,14 +397,19 @@ template <int TT, int BITS, bool DBG, int GC>
 __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid_constant__ StreamArgs a) {
   constexpr int R = kR;
   constexpr int kPairs = kSW / 2;
+  constexpr int kMaxPairsS = StreamTables<TT>::kPairs;
+  constexpr int kMaxSlotsS = StreamTables<TT>::kSlots;
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint64_t s_full[kSW][kR];  // one mbarrier per ring slot of each warp
   __shared__ int abort_s;
   __shared__ int s_idx[kMaxPairsS], s_row[kMaxPairsS];
   __shared__ float s_w[kMaxPairsS];
-  __shared__ int s_exp[kMaxSlotsS], s_cnt[kMaxSlotsS], s_base[kMaxSlotsS], s_tok[kMaxSlotsS][TT];
-  __shared__ uint32_t s_bits[kMaxExperts / 32], s_tm[kMaxExperts / 4];
-  __shared__ int s_bpre[kMaxExperts / 32];
+  // per slot: expert (table index), first y / h row, tokens, and the tokens
+  // (narrow types: the tables are sized for kStreamMaxSlots slots)
+  __shared__ short s_exp[kMaxSlotsS], s_base[kMaxSlotsS];
+  __shared__ unsigned char s_cnt[kMaxSlotsS], s_tok[kMaxSlotsS][TT];
+  __shared__ uint32_t s_bits[kMaxExperts / 32], s_tm[kMaxExperts / 2];
+  __shared__ short s_eslot[kMaxExperts];  // a chosen expert's first slot
   __shared__ int s_nslots;
   __shared__ int s_routed;      // the routing tables below are complete
   __shared__ int s_xready;      // the x planes are complete
@@ -401,7 +421,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   // units finished, and 1 + the last unit whose Q8 block of h is published
   __shared__ int s_arrive[kPairs][2];
   __shared__ int s_qdone[kPairs][2];
-  __shared__ int s_drow[DBG ? kMaxSlotsS : 1][TT];  // capture row of (slot, position): token * (K + S) + rank
+  __shared__ short s_drow[DBG ? kMaxSlotsS : 1][TT];  // capture row of (slot, position): token * (K + S) + rank
   constexpr bool HS = StreamHStaged<TT>::value;
   constexpr bool MMA = StreamMma<TT>::value;
   constexpr bool HR = StreamHRing<TT>::value;
@@ -414,17 +434,23 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = a.E, K = a.K, S = a.S, T = a.T;
   const int n_rows = T * (K + S);  // y rows of the batch (slot order)
+  // A slot holds at most TT of the batch's tokens: the shared experts (and
+  // any routed expert chosen by more than TT tokens) of a larger batch are
+  // several slots over the same weights, TT tokens each.
+  const int nsp = (T + TT - 1) / TT;  // slots of a shared expert
+  const int S2 = S * nsp;             // shared slots
+  const int XT = stream_x_staged<TT>(T);  // tokens of staged x planes (0: read from global)
   unsigned char* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   unsigned char* ring = smem + (size_t)warp * R * kStreamStageMax;
   uint4* xpl = reinterpret_cast<uint4*>(smem + (size_t)kSW * R * kStreamStageMax);
-  float2* xdc = reinterpret_cast<float2*>(xpl + 2 * TT * g.nbh);
-  float* s_y = reinterpret_cast<float*>(xdc + TT * g.nbh);  // [chunk of this CTA][y row][rpu_dn]
+  float2* xdc = reinterpret_cast<float2*>(xpl + 2 * XT * g.nbh);
+  float* s_y = reinterpret_cast<float*>(xdc + XT * g.nbh);  // [chunk of this CTA][y row][rpu_dn]
   // staged h (HS): the batch's rows in global order, planes then (d, c16)
   unsigned char* hst = reinterpret_cast<unsigned char*>(s_y) + stream_y_bytes(g, gridDim.x, n_rows);
   unsigned char* hst_dc = hst + (size_t)n_rows * g.nbi * 32;
   volatile int* abort_f = &abort_s;
 
-  for (int i = threadIdx.x; i < kMaxExperts / 4; i += blockDim.x) {
+  for (int i = threadIdx.x; i < kMaxExperts / 2; i += blockDim.x) {
     if (i < kMaxExperts / 32) s_bits[i] = 0u;
     s_tm[i] = 0u;
   }
@@ -439,15 +465,17 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     }
   if constexpr (HR)
     if (threadIdx.x < kHRing) s_hused[threadIdx.x] = 0;
-  // the shared slots come first and need no routing: slot s < S is shared
-  // expert s, with all T tokens (rows s T .. s T + T - 1)
-  for (int s = threadIdx.x; s < S; s += blockDim.x) {
-    s_exp[s] = E + s;
-    s_cnt[s] = T;
-    s_base[s] = s * T;
+  // the shared slots come first and need no routing: slot s2 < S2 is shared
+  // expert s2 / nsp with tokens TT j .. of the batch (j = s2 % nsp); shared
+  // expert s has rows s T .. s T + T - 1
+  for (int s2 = threadIdx.x; s2 < S2; s2 += blockDim.x) {
+    const int s = s2 / nsp, j = s2 - s * nsp;
+    s_exp[s2] = E + s;
+    s_cnt[s2] = min(TT, T - j * TT);
+    s_base[s2] = s * T + j * TT;
     for (int t = 0; t < TT; ++t) {
-      s_tok[s][t] = t;
-      if constexpr (DBG) s_drow[s][t] = t * (K + S) + K + s;
+      s_tok[s2][t] = j * TT + t;
+      if constexpr (DBG) s_drow[s2][t] = (j * TT + t) * (K + S) + K + s;
     }
   }
   if (threadIdx.x == 0) {
@@ -483,7 +511,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
   // pairs from the top warp down, so that the router warps form the last pairs
   const int pw = kSW - 1 - warp;
   const int pair = pw >> 1, half = pw & 1, gp = pair * G + blockIdx.x;
-  const int n_shared_gu = S * g.cpu_gu;
+  const int n_shared_gu = S2 * g.cpu_gu;
   const int c0 = (int)((int64_t)blockIdx.x * g.cpu_dn / G), c1 = (int)((int64_t)(blockIdx.x + 1) * g.cpu_dn / G);
   const int nch = c1 - c0;
   const bool shared_first = !router && gp < n_shared_gu;
@@ -507,7 +535,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     if (c.phase == 0) {
       const int u = gp + c.k * NP;
       const int slot = u / g.cpu_gu;
-      const int e = slot < S ? E + slot : s_exp[slot];
+      const int e = s_exp[slot];
       c.base = a.prep + (uint64_t)e * g.expert_bytes + (uint64_t)((u - slot * g.cpu_gu) * 2 + half) * g.ub_gu;
     } else if (c.phase == 1) {
       int id = 0;
@@ -520,7 +548,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       s_q[warp][c.k & (kQ - 1)] = id;
       if (id >= 0) {
         const int slot = id / nch, chunk = c0 + (id - slot * nch);
-        const int e = slot < S ? E + slot : s_exp[slot];
+        const int e = s_exp[slot];
         c.base = a.prep + (uint64_t)e * g.expert_bytes + g.dn_off + (uint64_t)chunk * g.ub_dn;
       }
     }
@@ -559,7 +587,16 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
     }
   };
 
-  if (!router && a.xpl_g != nullptr) {
+  if (!router && XT == 0) {
+    // the x planes stay in global memory (the router kernel's): every
+    // thread that reads them waits for that kernel first
+    pdl_wait();
+    asm volatile("bar.sync 2, %0;" ::"r"((kSW - n_router) * 32) : "memory");  // the non-router warps
+    if (threadIdx.x == n_router * 32) {
+      __threadfence_block();
+      *(volatile int*)&s_xready = 1;
+    }
+  } else if (!router && a.xpl_g != nullptr) {
     // the x planes from the router kernel: two bulk copies after the PDL wait
     if (threadIdx.x == n_router * 32) {
       pdl_wait();
@@ -645,11 +682,11 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
                                                  s_w + tr * K);
       __syncwarp();
       // the chosen experts (bit e of s_bits) and, per expert, the tokens that
-      // chose it (byte e & 3 of s_tm[e >> 2], bit t)
+      // chose it (half e & 1 of s_tm[e >> 1], bit t)
       if (lane < K) {
         const int e = s_idx[tr * K + lane];
         atomicOr(&s_bits[e >> 5], 1u << (e & 31));
-        atomicOr(&s_tm[e >> 2], 1u << ((e & 3) * 8 + tr));
+        atomicOr(&s_tm[e >> 1], 1u << ((e & 1) * 16 + tr));
       }
     }
     if (n_router > 1) asm volatile("bar.sync 1, %0;" ::"r"(n_router * 32) : "memory");  // the router warps
@@ -676,14 +713,18 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       }
     } else if (warp == 0) {
       __syncwarp();
-      auto tm_of = [&](int e) { return (s_tm[e >> 2] >> ((e & 3) * 8)) & 0xFFu; };
+      auto tm_of = [&](int e) { return (s_tm[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu; };
       // lane l: the experts 32l .. 32l+31; slots in ascending expert id after
-      // the shared ones, rows in slot order, a slot's rows in token order
+      // the shared ones (an expert of more than TT tokens: one slot per TT of
+      // them), rows in slot order, a slot's rows in token order
       const int nw = (E + 31) / 32;
       const uint32_t bits = lane < nw ? s_bits[lane] : 0u;
-      int rows = 0;
-      for (uint32_t bb = bits; bb; bb &= bb - 1) rows += __popc(tm_of(32 * lane + __ffs(bb) - 1));
-      const int c = __popc(bits);
+      int rows = 0, c = 0;
+      for (uint32_t bb = bits; bb; bb &= bb - 1) {
+        const int n = __popc(tm_of(32 * lane + __ffs(bb) - 1));
+        rows += n;
+        c += (n + TT - 1) / TT;
+      }
       int ci = c, ri = rows;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -693,30 +734,36 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
           ri += yr;
         }
       }
-      if (lane < nw) s_bpre[lane] = ci - c;
-      if (lane == 31) s_nslots = S + ci;
-      int r = S + ci - c, base = S * T + ri - rows;
+      if (lane == 31) s_nslots = S2 + ci;
+      int r = S2 + ci - c, base = S * T + ri - rows;
       for (uint32_t bb = bits; bb; bb &= bb - 1) {
         const int e = 32 * lane + __ffs(bb) - 1;
         const uint32_t m = tm_of(e);
-        s_exp[r] = e;
-        s_cnt[r] = __popc(m);
-        s_base[r] = base;
+        s_eslot[e] = r;
         int pos = 0;
-#pragma unroll
-        for (int t = 0; t < TT; ++t)
-          if ((m >> t) & 1u) s_tok[r][pos++] = t;
-        base += __popc(m);
+        for (int t = 0; t < kStreamMaxTok; ++t)
+          if ((m >> t) & 1u) {
+            if (pos % TT == 0) {  // the next slot of this expert
+              if (pos > 0) ++r;
+              s_exp[r] = e;
+              s_cnt[r] = 0;
+              s_base[r] = base + pos;
+            }
+            s_tok[r][pos % TT] = t;
+            ++s_cnt[r];
+            ++pos;
+          }
+        base += pos;
         ++r;
       }
       __syncwarp();
-      // each (token, rank) pair: the row of its expert's output
+      // each (token, rank) pair: the row of its expert's output (an expert's
+      // rows are contiguous over its slots)
       for (int p = lane; p < T * K; p += 32) {
-        const int e = s_idx[p], t = p / K, w32 = e >> 5;
-        const int slot = S + s_bpre[w32] + __popc(s_bits[w32] & ((1u << (e & 31)) - 1u));
+        const int e = s_idx[p], t = p / K;
         const int pos = __popc(tm_of(e) & ((1u << t) - 1u));
-        s_row[p] = s_base[slot] + pos;
-        if constexpr (DBG) s_drow[slot][pos] = t * (K + S) + (p - t * K);  // rank p - tK of token t
+        s_row[p] = s_base[s_eslot[e]] + pos;
+        if constexpr (DBG) s_drow[s_eslot[e] + pos / TT][pos % TT] = t * (K + S) + (p - t * K);  // rank p - tK of token t
       }
       __syncwarp();
       if (lane == 0) {
@@ -803,8 +850,8 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       Gs = g.g_gu;
       swz = g.swz_gu;
       nb = g.nbh;
-      ap = xpl;
-      adc = xdc;
+      ap = XT > 0 ? xpl : reinterpret_cast<const uint4*>(a.xpl_g);
+      adc = XT > 0 ? xdc : a.xdc_g;
       const int orow = chunk * 32 + 16 * half + (lane & 15);
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
@@ -987,12 +1034,12 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       if (!ok) break;
       const unsigned char* stg = ring + (size_t)(consumed % R) * kStreamStageMax;
       if constexpr (MMA) {
-        if (HS || HR || gu)
+        if (HS || HR || (gu && XT > 0))
           rows_stage_mma<BITS, DBG, GC, true>(Gs, stg, swz, s * span, nb, mmode, rB, rF0, rF1, ap, adc, accm, dbgm);
         else
           rows_stage_mma<BITS, DBG, GC, false>(Gs, stg, swz, s * span, nb, mmode, rB, rF0, rF1, ap, adc, accm, dbgm);
       } else {
-        if (HS || HR || gu)
+        if (HS || HR || (gu && XT > 0))
           rows_stage<TT, BITS, DBG, GC, true>(Gs, stg, swz, s * span + piece0, nb, nv, lpr == 2, tok, ap, adc, acc,
                                               dbg);
         else
@@ -1112,7 +1159,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) expert_stream_kernel(const __grid
       const float* yc = s_y + (size_t)cl * n_rows * rpu + rr;
       float accc = 0.0f;
       for (int kk = 0; kk < K; ++kk) accc = __fmaf_rn(s_w[t * K + kk], yc[(size_t)s_row[t * K + kk] * rpu], accc);
-      for (int s = 0; s < S; ++s) accc = __fadd_rn(accc, yc[(size_t)(s_base[s] + t) * rpu]);
+      for (int s = 0; s < S; ++s) accc = __fadd_rn(accc, yc[(size_t)(s * T + t) * rpu]);
       a.out[(size_t)t * g.H + (size_t)(c0 + cl) * rpu + rr] = accc;
     }
   }
@@ -1185,7 +1232,7 @@ cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
   int n_sms = 0;
   cudaError_t e = device_sms(&n_sms);
   if (e != cudaSuccess) return e;
-  const size_t smem = stream_smem_bytes<TT>(a.g, n_sms, a.T * (a.K + a.S));
+  const size_t smem = stream_smem_bytes<TT>(a.g, n_sms, a.T, a.T * (a.K + a.S));
   if (smem > kStreamDynMax) return cudaErrorInvalidConfiguration;
   if ((e = smem_opt_in(expert_stream_kernel<TT, BITS, DBG, GC>, (int)smem, granted)) != cudaSuccess) return e;
   // one CTA per SM, all resident at once (down units wait for gate/up units
@@ -1202,10 +1249,10 @@ bool stream_supported(int hidden, int inter, int bits, int n_tok, int top_k, int
   if (device_sms(&n_sms) != cudaSuccess) return false;
   const StreamGeom g = stream_geom(hidden, inter, bits);
   const int rows = n_tok * (top_k + n_shared);  // y (and h) rows of the batch
-  const size_t need = n_tok <= 1   ? stream_smem_bytes<1>(g, n_sms, rows)
-                      : n_tok <= 2 ? stream_smem_bytes<2>(g, n_sms, rows)
-                      : n_tok <= 4 ? stream_smem_bytes<4>(g, n_sms, rows)
-                                   : stream_smem_bytes<8>(g, n_sms, rows);
+  const size_t need = n_tok <= 1   ? stream_smem_bytes<1>(g, n_sms, n_tok, rows)
+                      : n_tok <= 2 ? stream_smem_bytes<2>(g, n_sms, n_tok, rows)
+                      : n_tok <= 4 ? stream_smem_bytes<4>(g, n_sms, n_tok, rows)
+                                   : stream_smem_bytes<8>(g, n_sms, n_tok, rows);
   (void)n_experts;
   return need <= kStreamDynMax;
 }

@@ -125,10 +125,14 @@ cudaError_t launch_down_decode(const DownTable& tbl, const Slot* slots, const in
 // Decode batches of <= kStreamMaxTok tokens on a prepared layer: one
 // persistent kernel (PDL launch after router_decode) that routes the batch
 // in every CTA, streams the layer's streaming copy stage by stage (gate/up,
-// SwiGLU, Q8_0 of h; down; combine) and writes `out`.
-constexpr int kStreamMaxTok = 8;   // tokens of one streaming kernel launch
-constexpr int kStreamChunked = 16;  // a prepared layer's batches up to this run as launches of <= kStreamMaxTok
-constexpr int kStreamMaxSlots = kMaxShared + kStreamMaxTok * kMaxTopK;
+// SwiGLU, Q8_0 of h; down; combine) and writes `out`.  Every expert the
+// batch chose is read once; an expert with more than kStreamSlotTok of the
+// batch's tokens (the shared experts of a batch above that size) is several
+// slots over the same weights.
+constexpr int kStreamMaxTok = 16;  // tokens of one streaming kernel launch
+constexpr int kStreamSlotTok = 8;  // tokens of one slot
+constexpr int kStreamMaxSlots =
+    ((kStreamMaxTok + kStreamSlotTok - 1) / kStreamSlotTok) * kMaxShared + kStreamMaxTok * kMaxTopK;
 struct StreamArgs {
   const unsigned char* prep;  // the layer's streaming copy (coli_moe_prepare)
   StreamGeom g;
