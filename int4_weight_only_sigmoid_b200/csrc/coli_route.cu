@@ -182,18 +182,18 @@ __global__ void __launch_bounds__(kRouteThreads) route_topk_kernel(const float* 
 // Decode batches (n_tok <= kDecodeMaxTok): two kernels.
 
 // Router scores.  A CTA of 8 warps owns 2 experts; their router rows and
-// (for up to kStageTok tokens) the token rows are copied to shared memory
-// with cp.async first, so the fold loop below reads only shared memory;
-// warp w folds expert (w & 1) for tokens t = w/2, w/2 + 4, ...  The CTAs
-// also write the Q8_0 of x for the expert kernels.
-constexpr int kStageTok = 2;
+// the token rows (kStageTok tokens at a time) are copied to shared memory
+// with cp.async, so the fold loop below reads only shared memory; in each
+// pass warp w folds expert (w & 1) for token w/2 of the pass.  The CTAs also
+// write the Q8_0 of x for the expert kernels.
+constexpr int kStageTok = 4;
 __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restrict__ x,
                                                             const float* __restrict__ wr, int n_tok, int E, int H,
                                                             float* __restrict__ scores, int8_t* __restrict__ xq,
                                                             float* __restrict__ xd, int8_t* __restrict__ xpl,
                                                             float2* __restrict__ xdc, int32_t* status_clear,
                                                             int32_t* zero, int n_zero) {
-  extern __shared__ __align__(16) float4 wsm[];  // [2][H/4] router rows, then [kStageTok][H/4] tokens
+  extern __shared__ __align__(16) float4 wsm[];  // [2][H/4] router rows, then [<= kStageTok][H/4] tokens
   // first kernel of a decode forward (launched without PDL, so everything
   // before it in the stream is complete): start the status word afresh
   if (status_clear && blockIdx.x == 0 && threadIdx.x == 0) *status_clear = 0;
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restr
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e0 = blockIdx.x * 2;
   const int nq = H / 4;
-  const bool stage_x = n_tok <= kStageTok;
+  const int G = n_tok < kStageTok ? n_tok : kStageTok;  // tokens per pass
   {
     // the router rows are read once per forward: first out of L2
     const uint64_t pol = l2_evict_first();
@@ -212,8 +212,7 @@ __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restr
       if (e0 + r < E) cp_async16_hint(wsm + i, wr + (size_t)(e0 + r) * H + 4 * j, pol);
     }
   }
-  if (stage_x)
-    for (int i = threadIdx.x; i < n_tok * nq; i += blockDim.x) cp_async16(wsm + 2 * nq + i, x + 4 * (size_t)i);
+  for (int i = threadIdx.x; i < G * nq; i += blockDim.x) cp_async16(wsm + 2 * nq + i, x + 4 * (size_t)i);
   // the Q8_0 of x for the expert kernels: one warp per 32-element block,
   // as rows (xq, xd) and / or as the streaming kernel's even / odd byte
   // planes with (d, -128 * sum of the even plane) (xpl, xdc)
@@ -234,25 +233,32 @@ __global__ void __launch_bounds__(256) router_decode_kernel(const float* __restr
       if (lane == 0) xdc[j] = make_float2(d, __int_as_float(-128 * se));
     }
   }
-  cp_async_wait_all();
-  __syncthreads();
   const int r = warp & 1, e = e0 + r;
-  if (e >= E) return;
   const float4* ws = wsm + r * nq;
-  for (int t = warp >> 1; t < n_tok; t += 4) {
-    const float4* xp = stage_x ? wsm + (2 + t) * nq : reinterpret_cast<const float4*>(x + (size_t)t * H);
-    float acc = 0.0f;
-#pragma unroll 8
-    for (int j = lane; j < nq; j += 32) {
-      const float4 a = xp[j];
-      const float4 b = ws[j];
-      acc = __fmaf_rn(a.x, b.x, acc);
-      acc = __fmaf_rn(a.y, b.y, acc);
-      acc = __fmaf_rn(a.z, b.z, acc);
-      acc = __fmaf_rn(a.w, b.w, acc);
+  for (int t0 = 0; t0 < n_tok; t0 += G) {
+    if (t0 > 0) {
+      __syncthreads();  // the previous pass's reads of the staged tokens are done
+      const int g = n_tok - t0 < G ? n_tok - t0 : G;
+      for (int i = threadIdx.x; i < g * nq; i += blockDim.x)
+        cp_async16(wsm + 2 * nq + i, x + (size_t)t0 * H + 4 * (size_t)i);
     }
-    const float logit = warp_sum_in_lane_order(acc);
-    if (lane == 0) scores[(size_t)t * E + e] = sigmoid_cw(logit);
+    cp_async_wait_all();
+    __syncthreads();
+    for (int tl = warp >> 1; e < E && tl < G && t0 + tl < n_tok; tl += 4) {
+      const float4* xp = wsm + (2 + tl) * nq;
+      float acc = 0.0f;
+#pragma unroll 8
+      for (int j = lane; j < nq; j += 32) {
+        const float4 a = xp[j];
+        const float4 b = ws[j];
+        acc = __fmaf_rn(a.x, b.x, acc);
+        acc = __fmaf_rn(a.y, b.y, acc);
+        acc = __fmaf_rn(a.z, b.z, acc);
+        acc = __fmaf_rn(a.w, b.w, acc);
+      }
+      const float logit = warp_sum_in_lane_order(acc);
+      if (lane == 0) scores[(size_t)(t0 + tl) * E + e] = sigmoid_cw(logit);
+    }
   }
 }
 
@@ -459,7 +465,7 @@ cudaError_t launch_topk(const float* scores, const float* bias, int n_tok, int E
 cudaError_t launch_router_decode(const float* x, const float* w_router, int n_tok, int E, int H, float* scores,
                                  int8_t* xq, float* xd, int32_t* status_clear, int32_t* zero, int n_zero,
                                  cudaStream_t st, int8_t* xpl, float2* xdc) {
-  const size_t smem = (size_t)(2 + (n_tok <= kStageTok ? n_tok : 0)) * H * sizeof(float);
+  const size_t smem = (size_t)(2 + (n_tok < kStageTok ? n_tok : kStageTok)) * H * sizeof(float);
   static int granted[64] = {};
   const cudaError_t e = smem_opt_in(router_decode_kernel, 200 * 1024, granted);
   if (e != cudaSuccess) return e;
