@@ -138,13 +138,6 @@ __device__ __forceinline__ void unpack_blk(const uint4& w, uint4& ue, uint4& so)
   so.w = w.w & 0xF0F0F0F0u;
 }
 
-__device__ __forceinline__ int even_plane_sum(const uint4& e) {
-  int s = __dp4a((int)e.x, 0x01010101, 0);
-  s = __dp4a((int)e.y, 0x01010101, s);
-  s = __dp4a((int)e.z, 0x01010101, s);
-  return __dp4a((int)e.w, 0x01010101, s);
-}
-
 __device__ __forceinline__ int warp_sum_int(int v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -1242,6 +1235,22 @@ cudaError_t stream_tt(const StreamArgs& a, cudaStream_t st) {
 
 }  // namespace
 
+// The instance's dynamic shared memory for this batch plus its static
+// shared memory (the capture instance's, the larger) within the device's
+// per-block limit.
+template <int TT>
+bool stream_fits(const StreamGeom& g, int n_sms, int n_tok, int rows) {
+  const size_t need = stream_smem_bytes<TT>(g, n_sms, n_tok, rows);
+  if (need > kStreamDynMax) return false;
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, expert_stream_kernel<TT, 4, true, 0>) != cudaSuccess) return false;
+  int dev = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return false;
+  return need + fa.sharedSizeBytes <= (size_t)optin;
+}
+
 bool stream_supported(int hidden, int inter, int bits, int n_tok, int top_k, int n_shared, int n_experts) {
   if (n_tok < 1 || n_tok > kStreamMaxTok || !stream_shape_ok(hidden, inter, bits)) return false;
   if (top_k < 1 || top_k > kMaxTopK || n_shared < 0 || n_shared > kMaxShared) return false;
@@ -1249,12 +1258,11 @@ bool stream_supported(int hidden, int inter, int bits, int n_tok, int top_k, int
   if (device_sms(&n_sms) != cudaSuccess) return false;
   const StreamGeom g = stream_geom(hidden, inter, bits);
   const int rows = n_tok * (top_k + n_shared);  // y (and h) rows of the batch
-  const size_t need = n_tok <= 1   ? stream_smem_bytes<1>(g, n_sms, n_tok, rows)
-                      : n_tok <= 2 ? stream_smem_bytes<2>(g, n_sms, n_tok, rows)
-                      : n_tok <= 4 ? stream_smem_bytes<4>(g, n_sms, n_tok, rows)
-                                   : stream_smem_bytes<8>(g, n_sms, n_tok, rows);
   (void)n_experts;
-  return need <= kStreamDynMax;
+  return n_tok <= 1   ? stream_fits<1>(g, n_sms, n_tok, rows)
+         : n_tok <= 2 ? stream_fits<2>(g, n_sms, n_tok, rows)
+         : n_tok <= 4 ? stream_fits<4>(g, n_sms, n_tok, rows)
+                      : stream_fits<8>(g, n_sms, n_tok, rows);
 }
 
 uint64_t stream_expert_bytes(int hidden, int inter, int bits) { return stream_geom(hidden, inter, bits).expert_bytes; }
