@@ -68,7 +68,7 @@ typedef enum {
  * Limits: hidden % 128 == 0; inter % 32 == 0; shared_inter % 32 == 0;
  * 1 <= top_k <= min(n_experts, 16); n_experts <= 512; 0 <= n_shared <= 4.
  * int8 weights need inter % 128 == 0 (they run on the streaming kernel of
- * a prepared layer for <= 8 tokens, else on the tensor-core kernels). */
+ * a prepared layer for <= 16 tokens, else on the tensor-core kernels). */
 typedef struct {
     int32_t hidden;
     int32_t inter;
@@ -95,7 +95,7 @@ typedef struct {
 /* One MoE layer.  `experts` and `shared` are HOST arrays (n_experts and
  * n_shared entries) of device-pointer sets; the router stays F32
  * ([W] "量化保留模块").  `prepared` is the layer's streaming copy
- * (coli_moe_prepare) or NULL: with it, decode batches of up to 8 tokens
+ * (coli_moe_prepare) or NULL: with it, decode batches of up to 16 tokens
  * read the experts from that copy (same results, bit for bit); without it,
  * or for other batch sizes, the kernels read the row-major weights. */
 typedef struct {
