@@ -85,6 +85,7 @@ struct PkRing {
 static_assert(PkRing<4>::kPkSlots * PkRing<4>::kPk == PkRing<8>::kPkSlots * PkRing<8>::kPk, "one ring size");
 constexpr int kHalf = 2;       // Q8 blocks per accumulator hand-off (MMA -> fold): 1 or 2
 constexpr int kTBufs = 4;      // TMEM accumulators (one per block), handed off in pairs
+constexpr int kNL = 32;        // light items (<= kNL tokens): the tokens are the MMA's N
 constexpr int kProdWarps = 2;
 constexpr int kEpiWarps = 16;  // 4 per TMEM lane quadrant, each a quarter of the columns
 // Warp w runs on scheduler w % 4 and, as a fold warp, reads TMEM lanes
@@ -260,6 +261,18 @@ __device__ __forceinline__ ItemInfo item_info(const Slot* slots, const Tile* til
   return f;
 }
 
+// Capture row of token n of the item's tile: token * (K + S) + rank (shared
+// expert s: rank K + s), and the capture's words per row.
+__device__ __forceinline__ int64_t dbg_row(const ItemInfo& f, const int32_t* perm, int top_k, const DbgArgs& dbg,
+                                           int n) {
+  if (f.slot.perm_base < 0) return (int64_t)(f.n0 + n) * (top_k + dbg.S) + top_k + (f.slot.table_idx - dbg.E);
+  const int pr = perm[f.slot.perm_base + f.n0 + n];
+  return (int64_t)(pr / top_k) * (top_k + dbg.S) + pr % top_k;
+}
+__device__ __forceinline__ int64_t dbg_words(int hidden, int inter) {
+  return 2 * (int64_t)inter * (hidden / 32) + (int64_t)hidden * (inter / 32);
+}
+
 // Row of token n of the item's tile in the per-token arrays: gate/up: the
 // token itself (x's scales and block sums); down: the (slot, token) row.
 __device__ __forceinline__ int64_t item_token_row(const ItemInfo& f, bool gu, const int32_t* perm, int top_k, int n) {
@@ -283,6 +296,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
   __shared__ float s_amax[2][kEpiWarps][32];  // gate/up fold: half-block absmax per (warp, token), by item parity
+  // gate/up fold of light items: the up rows' products per (c4, quadrant 2/3, lane, token), by item parity
+  __shared__ float s_up[GU ? 2 : 1][kEpiWarps / 4][64][8];
   extern __shared__ unsigned char smem_raw[];
 
   const int dim_in = GU ? hidden : inter;
@@ -429,7 +444,43 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       int gs = 0, gh = 0;
       bool ok = true;
       constexpr uint32_t idesc = idesc_i8_s32(kM, kN);
+      constexpr uint32_t idesc_l = idesc_i8_s32(kN, kNL);  // light: weights as M, tokens as N
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        if (item_info(slots, tiles, item, nm, kGroupRows).n_valid <= kNL) {
+          // light item: one hand-off per two stages (8 blocks of kNL
+          // columns in one 256-column pair of buffers)
+          for (int j = 0; j < nst && ok; ++j, ++gs) {
+            const int s = gs % kStages;
+            if (!mbar_wait(&full_bar[s], (gs / kStages) & 1, abort, err, 11)) {
+              ok = false;
+              break;
+            }
+            fence_after_sync();
+            const uint32_t opa = smem_u32(op_ring + s * L::kOpStage);
+            const uint32_t opb = opa + L::kStageA;
+            const int hb = gh % (kTBufs / kHalf);
+            if ((j & 1) == 0) {
+              if (!mbar_wait(&tempty_bar[hb], (gh / (kTBufs / kHalf)) & 1, abort, err, 12)) {
+                ok = false;
+                break;
+              }
+              fence_after_sync();
+            }
+#pragma unroll
+            for (int c = 0; c < kBS; ++c) {
+              const uint32_t d = tmem + hb * kHalf * kN + (j & 1) * kBS * kNL + c * kNL;
+              const uint64_t da = smem_desc_k_noswizzle(opb + c * L::kSubB, 128, 256);
+              const uint64_t db = smem_desc_k_sw128(opa + c * 32);
+              mma_i8(d, da, db, idesc_l);
+            }
+            if ((j & 1) == 1 || j == nst - 1) {
+              mma_commit(&tfull_bar[hb]);
+              ++gh;
+            }
+            mma_commit(&empty_bar[s]);
+          }
+          continue;
+        }
         for (int j = 0; j < nst && ok; ++j, ++gs) {
           const int s = gs % kStages;
           if (!mbar_wait(&full_bar[s], (gs / kStages) & 1, abort, err, 11)) {
@@ -474,15 +525,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     // expect_tx arrival on `full` and one TMA load of 128 rows x 128 bytes
     // (128-byte swizzle) of the row-ordered activations (gate/up) or h
     // (down), rows [row_base + n0, +128) of the item's slot; a light item (at
-    // most 32 tokens): rows [row_base + n0, +32) four times, into rows 0, 32,
-    // 64 and 96 of the tile (one per TMEM lane quadrant).
+    // most kNL tokens): rows [row_base + n0, +kNL) only.
     if (lane == 0) {
       int gs = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
         const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
         const int row0 = f.slot.row_base + f.n0;
-        const bool light = f.n_valid <= 32;
+        const bool light = f.n_valid <= kNL;
         for (int j = 0; j < nst; ++j, ++gs) {
           const int s = gs % kStages;
           if (!mbar_wait(&empty_bar[s], ((gs / kStages) & 1) ^ 1, abort, err, 16)) {
@@ -490,11 +540,11 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
             break;
           }
           unsigned char* oa = op_ring + s * L::kOpStage;
-          mbar_arrive_expect_tx(&full_bar[s], L::kStageA);
           if (light) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) tma_load_2d(oa + q * 32 * 128, &amap32, j * kBS * 32, row0, &full_bar[s]);
+            mbar_arrive_expect_tx(&full_bar[s], kNL * 128);
+            tma_load_2d(oa, &amap32, j * kBS * 32, row0, &full_bar[s]);
           } else {
+            mbar_arrive_expect_tx(&full_bar[s], L::kStageA);
             tma_load_2d(oa, &amap, j * kBS * 32, row0, &full_bar[s]);
           }
         }
@@ -506,14 +556,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
     // warp w: TMEM lanes 32*(w%4).. (tokens); columns c0.. and c1.. (16 each):
     // gate/up: gate rows [16 c4, 16 c4 + 16) of the group and the same up
     // rows (64 columns on); down: columns [32 c4, 32 c4 + 32).
-    // A light item (at most 32 tokens) holds its tokens in every lane
-    // quadrant (the A tile carries them four times), and the 16 warps split
-    // the columns instead: warp (quad q, c4) takes 4 of each range,
-    // c0 + 4 q and c1 + 4 q, so the fold runs on all four schedulers.
+    // A light item (at most kNL tokens) has the weight rows as the TMEM lanes
+    // and the tokens as columns (kNL per block): warp w folds weight rows
+    // 32 (w%4).. for tokens [8 c4, 8 c4 + 8).
     const int quad = warp & 3, c4 = (warp - kEpi0) >> 2;
-    const int c0n = GU ? 16 * c4 : 32 * c4;
-    const int c1n = GU ? kGroupRows + 16 * c4 : 32 * c4 + 16;
-    int n_done = 0;  // items this warp has folded (parity of the absmax exchange buffer)
+    const int c0 = GU ? 16 * c4 : 32 * c4;
+    const int c1 = GU ? kGroupRows + 16 * c4 : 32 * c4 + 16;
+    int n_done = 0;  // items this warp has folded (parity of the exchange buffers)
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     constexpr int kHandPerStage = kBS / kHalf;
     // isum from an accumulator read as binary32: int4 (B = 16 q): the value
@@ -527,168 +576,127 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
       if (lane == 0)
         for (int h = 0; h < kTBufs / kHalf; ++h) mbar_arrive(&tempty_bar[h]);
     }
-    // fold of nc (8 or 4) loaded columns of each range (r0, r1), block b,
-    // into accumulators nc h ..
-    auto fold_cols = [&](auto ncw, const uint32_t* r0, const uint32_t* r1, float dx, int b, float (&acc0)[16],
-                         float (&acc1)[16], int32_t* dbg0, int32_t* dbg1, bool valid, int h) {
-      constexpr int nc = decltype(ncw)::value;
-#pragma unroll
-      for (int jj = 0; jj < nc; jj += 2) {
-        // S + 0x4B400000 read as binary32 is 1.5 * 2^23 + S (|S| < 2^22)
-        float v0 = __uint_as_float(r0[jj] + kMagic), v1 = __uint_as_float(r0[jj + 1] + kMagic);
-        float u0 = __uint_as_float(r1[jj] + kMagic), u1 = __uint_as_float(r1[jj + 1] + kMagic);
-        fma2c(v0, v1, kIsumScale, kIsumOffset);  // exact: (float)isum
-        fma2c(u0, u1, kIsumScale, kIsumOffset);
-        const int colw = nc * h + jj;
-        if constexpr (DBG) {
-          if (valid) {
-            dbg0[(int64_t)colw * nb + b] = (int32_t)v0;
-            dbg0[(int64_t)(colw + 1) * nb + b] = (int32_t)v1;
-            dbg1[(int64_t)colw * nb + b] = (int32_t)u0;
-            dbg1[(int64_t)(colw + 1) * nb + b] = (int32_t)u1;
-          }
-        }
-        fma2(acc0[colw], acc0[colw + 1], dx, dx, v0, v1);
-        fma2(acc1[colw], acc1[colw + 1], dx, dx, u0, u1);
-      }
+    // (float)isum of two accumulator values (S + 0x4B400000 read as binary32
+    // is 1.5 * 2^23 + S, |S| < 2^22)
+    auto isum2 = [&](uint32_t a, uint32_t b, float& v0, float& v1) {
+      v0 = __uint_as_float(a + kMagic);
+      v1 = __uint_as_float(b + kMagic);
+      fma2c(v0, v1, kIsumScale, kIsumOffset);
     };
     int gh = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      bool active, valid, light;
-      int n, c0, c1;
-      const float* drow;  // the token's Q8 scales, one per block
+      const bool light = item_info(slots, tiles, item, nm, kGroupRows).n_valid <= kNL;  // CTA-uniform
       float acc0[16], acc1[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         acc0[j] = 0.0f;
         acc1[j] = 0.0f;
       }
-      // capture: this token's row and the first output row of each column range
-      int32_t* dbg0 = nullptr;
-      int32_t* dbg1 = nullptr;
-      {  // the item's description is read again for the epilogue: fewer live registers in the block loop
-        const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
-        light = f.n_valid <= 32;  // CTA-uniform
-        n = light ? lane : quad * 32 + lane;  // this thread's token within the tile
-        c0 = light ? c0n + 4 * quad : c0n;
-        c1 = light ? c1n + 4 * quad : c1n;
-        active = light || quad * 32 < f.n_valid;  // warp-uniform
-        valid = n < f.n_valid;
-        drow = ad + (valid ? item_token_row(f, GU, perm, top_k, n) : 0) * nb;
-      if constexpr (DBG) {
-        if (valid) {
-          const int nbh = hidden / 32, nbi = inter / 32;
-          const int64_t P = 2 * (int64_t)inter * nbh + (int64_t)hidden * nbi;
-          int64_t crow;
-          if (f.slot.perm_base < 0) {
-            crow = (int64_t)(f.n0 + n) * (top_k + dbg.S) + top_k + (f.slot.table_idx - dbg.E);
-          } else {
-            const int pr = perm[f.slot.perm_base + f.n0 + n];
-            crow = (int64_t)(pr / top_k) * (top_k + dbg.S) + pr % top_k;
-          }
-          int32_t* base = dbg.buf + crow * P;
-          if constexpr (GU) {
-            dbg0 = base + (int64_t)(f.m0 + c0) * nbh;                            // gate rows
-            dbg1 = base + (int64_t)inter * nbh + (int64_t)(f.m0 + c0) * nbh;     // up rows
-          } else {
-            dbg0 = base + 2 * (int64_t)inter * nbh + (int64_t)(f.m0 + c0) * nbi;
-            dbg1 = base + 2 * (int64_t)inter * nbh + (int64_t)(f.m0 + c1) * nbi;
-          }
-        }
-      }
-      }
-      // the token's Q8 scales of a hand-off (kHalf blocks), one hand-off ahead
-      float dnext[kHalf], dcur[kHalf];
-#pragma unroll
-      for (int i = 0; i < kHalf; ++i) dnext[i] = valid ? __ldg(drow + i) : 0.0f;
-      for (int j = 0; j < nst; ++j) {
-#pragma unroll
-        for (int hs = 0; hs < kHandPerStage; ++hs, ++gh) {
-          const int hn = j * kHandPerStage + hs + 1;  // next hand-off of this item
-#pragma unroll
-          for (int i = 0; i < kHalf; ++i) {
-            dcur[i] = dnext[i];
-            if (valid && hn < nst * kHandPerStage) dnext[i] = __ldg(drow + hn * kHalf + i);
-          }
-          const int hb = gh % (kTBufs / kHalf);
-          // warp-uniform: tcgen05.ld is a warp-wide instruction
-          const bool ok =
-              __all_sync(0xffffffffu, mbar_wait(&tfull_bar[hb], (gh / (kTBufs / kHalf)) & 1, abort, err, 13));
-          fence_after_sync();
-#pragma unroll
-          for (int i = 0; i < kHalf; ++i) {
-            const int b = j * kBS + hs * kHalf + i;  // block of this item
-            const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
-            if (active && ok && !light) {
-              // 8 columns of each range at a time (16 TMEM values live)
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                uint32_t r0[8], r1[8];
-                tmem_ld8(col + c0 + 8 * h, r0);
-                tmem_ld8(col + c1 + 8 * h, r1);
-                tmem_ld_wait();
-                fold_cols(std::integral_constant<int, 8>{}, r0, r1, dcur[i], b, acc0, acc1, dbg0, dbg1, valid, h);
+      if (!light) {
+        bool active, valid;
+        const int n = quad * 32 + lane;  // this thread's token within the tile
+        const float* drow;               // the token's Q8 scales, one per block
+        // capture: this token's row and the first output row of each column range
+        int32_t* dbg0 = nullptr;
+        int32_t* dbg1 = nullptr;
+        {  // the item's description is read again for the epilogue: fewer live registers in the block loop
+          const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
+          active = quad * 32 < f.n_valid;  // warp-uniform
+          valid = n < f.n_valid;
+          drow = ad + (valid ? item_token_row(f, GU, perm, top_k, n) : 0) * nb;
+          if constexpr (DBG) {
+            if (valid) {
+              int32_t* base = dbg.buf + dbg_row(f, perm, top_k, dbg, n) * dbg_words(hidden, inter);
+              const int nbh = hidden / 32, nbi = inter / 32;
+              if constexpr (GU) {
+                dbg0 = base + (int64_t)(f.m0 + c0) * nbh;                         // gate rows
+                dbg1 = base + (int64_t)inter * nbh + (int64_t)(f.m0 + c0) * nbh;  // up rows
+              } else {
+                dbg0 = base + 2 * (int64_t)inter * nbh + (int64_t)(f.m0 + c0) * nbi;
+                dbg1 = base + 2 * (int64_t)inter * nbh + (int64_t)(f.m0 + c1) * nbi;
               }
             }
           }
-          if (active && ok && light) {
-            // 4 columns of each range per block: the hand-off's loads, then one wait
-            uint32_t r[kHalf][2][4];
+        }
+        // the token's Q8 scales of a hand-off (kHalf blocks), one hand-off ahead
+        float dnext[kHalf], dcur[kHalf];
+#pragma unroll
+        for (int i = 0; i < kHalf; ++i) dnext[i] = valid ? __ldg(drow + i) : 0.0f;
+        for (int j = 0; j < nst; ++j) {
+#pragma unroll
+          for (int hs = 0; hs < kHandPerStage; ++hs, ++gh) {
+            const int hn = j * kHandPerStage + hs + 1;  // next hand-off of this item
 #pragma unroll
             for (int i = 0; i < kHalf; ++i) {
-              const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
-              tmem_ld4(col + c0, r[i][0]);
-              tmem_ld4(col + c1, r[i][1]);
+              dcur[i] = dnext[i];
+              if (valid && hn < nst * kHandPerStage) dnext[i] = __ldg(drow + hn * kHalf + i);
             }
-            tmem_ld_wait();
+            const int hb = gh % (kTBufs / kHalf);
+            // warp-uniform: tcgen05.ld is a warp-wide instruction
+            const bool ok =
+                __all_sync(0xffffffffu, mbar_wait(&tfull_bar[hb], (gh / (kTBufs / kHalf)) & 1, abort, err, 13));
+            fence_after_sync();
 #pragma unroll
-            for (int i = 0; i < kHalf; ++i)
-              fold_cols(std::integral_constant<int, 4>{}, r[i][0], r[i][1], dcur[i], j * kBS + hs * kHalf + i, acc0,
-                        acc1, dbg0, dbg1, valid, 0);
+            for (int i = 0; i < kHalf; ++i) {
+              const int b = j * kBS + hs * kHalf + i;  // block of this item
+              const uint32_t col = tmem + lane_base + (hb * kHalf + i) * kN;
+              if (active && ok) {
+                const float dx = dcur[i];
+                // 8 columns of each range at a time (16 TMEM values live)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  uint32_t r0[8], r1[8];
+                  tmem_ld8(col + c0 + 8 * h, r0);
+                  tmem_ld8(col + c1 + 8 * h, r1);
+                  tmem_ld_wait();
+#pragma unroll
+                  for (int jj = 0; jj < 8; jj += 2) {
+                    float v0, v1, u0, u1;
+                    isum2(r0[jj], r0[jj + 1], v0, v1);
+                    isum2(r1[jj], r1[jj + 1], u0, u1);
+                    const int colw = 8 * h + jj;
+                    if constexpr (DBG) {
+                      if (valid) {
+                        dbg0[(int64_t)colw * nb + b] = (int32_t)v0;
+                        dbg0[(int64_t)(colw + 1) * nb + b] = (int32_t)v1;
+                        dbg1[(int64_t)colw * nb + b] = (int32_t)u0;
+                        dbg1[(int64_t)(colw + 1) * nb + b] = (int32_t)u1;
+                      }
+                    }
+                    fma2(acc0[colw], acc0[colw + 1], dx, dx, v0, v1);
+                    fma2(acc1[colw], acc1[colw + 1], dx, dx, u0, u1);
+                  }
+                }
+              }
+            }
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[hb]);  // the hand-off's TMEM buffers may be rewritten now
           }
-          fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty_bar[hb]);  // the hand-off's TMEM buffers may be rewritten now
         }
-      }
-      if (active) {  // warp-uniform; the same for all warps that share a Q8 block of h
-        const bool go = !*abort;  // this warp's writes only: the warps meet the barrier regardless
-        const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
-        const int64_t row = (int64_t)f.slot.row_base + f.n0 + n;
-        const int nr = light ? 4 : 16;  // rows of each range this thread holds
-        if constexpr (GU) {
-          const int o = f.m0 + c0;  // this thread's first intermediate row
-          const float* sgp = tab.gate_s[f.slot.table_idx] + o;
-          const float* sup = tab.up_s[f.slot.table_idx] + o;
-          float amax = 0.0f;
+        if (active) {  // warp-uniform, and the same for both warps of a pair (one quadrant)
+          const bool go = !*abort;  // this warp's writes only: both warps meet the barrier regardless
+          const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
+          const int64_t row = (int64_t)f.slot.row_base + f.n0 + n;
+          if constexpr (GU) {
+            const int o = f.m0 + c0;  // this thread's 16 intermediate rows (half of a Q8 block of h)
+            const float* sgp = tab.gate_s[f.slot.table_idx] + o;
+            const float* sup = tab.up_s[f.slot.table_idx] + o;
+            float amax = 0.0f;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (j < nr) {
+            for (int j = 0; j < 16; ++j) {
               const float gv = __fmul_rn(__ldg(sgp + j), acc0[j]);
               const float u = __fmul_rn(__ldg(sup + j), acc1[j]);
               acc0[j] = __fmul_rn(__fmul_rn(gv, sigmoid_cw(gv)), u);
               amax = fmaxf(amax, fabsf(acc0[j]));
             }
-          }
-          // the block's absmax over the warps that hold its 32 rows: the
-          // partner warp (c4 ^ 1) of this quadrant, or (light) the 8 warps
-          // c4 in {c4 & ~1, c4 | 1} of all quadrants
-          float* xa = &s_amax[n_done & 1][0][0];
-          xa[(warp - kEpi0) * 32 + lane] = valid ? amax : 0.0f;
-          if (light) {
-            named_bar(10 + (c4 >> 1), 256);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int cc = (c4 & ~1) + (k >> 2), qq = k & 3;  // fold warp with c4 = cc in quadrant qq
-              amax = fmaxf(amax, xa[(4 * cc + ((qq - kEpi0) & 3)) * 32 + lane]);
-            }
-          } else {
+            // the block's absmax: this half's and the partner warp's (c4 ^ 1)
+            float* xa = &s_amax[n_done & 1][0][0];
+            xa[(warp - kEpi0) * 32 + lane] = valid ? amax : 0.0f;
             named_bar(2 + quad * 2 + (c4 >> 1), 64);
             amax = fmaxf(amax, xa[(warp - kEpi0 + 4 * ((c4 ^ 1) - c4)) * 32 + lane]);
-          }
-          const float d = __fdiv_rn(amax, 127.0f);
-          if (go && valid) {
-            if (!light) {
+            const float d = __fdiv_rn(amax, 127.0f);
+            if (go && valid) {
               // q in the operand order (int4 weights: per 8 elements 0,2,4,6,1,3,5,7;
               // int8: the elements' order)
               uint32_t pk[4];
@@ -710,33 +718,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
                 }
               }
               *reinterpret_cast<uint4*>(hr + row * inter + o) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            } else {
-              // 4 rows o.. (o % 8 is 0 or 4): int8 weights, 4 bytes in element
-              // order; int4 weights, element e of the group of 8 at byte
-              // e / 2 (even e) or 4 + e / 2 (odd e)
-              int8_t* hg = hr + row * inter + (o & ~7);
-              if constexpr (BITS == 4) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const int e = (o & 7) + j;
-                  hg[(e & 1) ? 4 + (e >> 1) : (e >> 1)] = (int8_t)q8_of(acc0[j], d);
-                }
-              } else {
-                uint32_t w = 0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) w |= ((uint32_t)q8_of(acc0[j], d) & 0xFFu) << (8 * j);
-                *reinterpret_cast<uint32_t*>(hr + row * inter + o) = w;
-              }
+              if ((c4 & 1) == 0) hd[row * (inter / 32) + (o >> 5)] = d;
             }
-            if ((c4 & 1) == 0 && (!light || quad == 0)) hd[row * (inter / 32) + (o >> 5)] = d;
-          }
-        } else if (go && valid) {
-          const float* sdp = tab.down_s[f.slot.table_idx] + f.m0;
-          float4* dst0 = reinterpret_cast<float4*>(y + row * hidden + f.m0 + c0);
-          float4* dst1 = reinterpret_cast<float4*>(y + row * hidden + f.m0 + c1);
+          } else if (go && valid) {
+            const float* sdp = tab.down_s[f.slot.table_idx] + f.m0;
+            float4* dst0 = reinterpret_cast<float4*>(y + row * hidden + f.m0 + c0);
+            float4* dst1 = reinterpret_cast<float4*>(y + row * hidden + f.m0 + c1);
 #pragma unroll
-          for (int j = 0; j < 16; j += 4) {
-            if (j < nr) {
+            for (int j = 0; j < 16; j += 4) {
               const float4 s0 = __ldg(reinterpret_cast<const float4*>(sdp + c0 + j));
               const float4 s1 = __ldg(reinterpret_cast<const float4*>(sdp + c1 + j));
               dst0[j / 4] = make_float4(__fmul_rn(s0.x, acc0[j]), __fmul_rn(s0.y, acc0[j + 1]),
@@ -744,6 +733,113 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
               dst1[j / 4] = make_float4(__fmul_rn(s1.x, acc1[j]), __fmul_rn(s1.y, acc1[j + 1]),
                                         __fmul_rn(s1.z, acc1[j + 2]), __fmul_rn(s1.w, acc1[j + 3]));
             }
+          }
+        }
+      } else {
+        // light item: this thread's weight row r (0..127 of the item's 128
+        // rows) for the warp's 8 tokens t0 + t; lane 4 t + c holds the Q8
+        // scale of token t0 + t for block c of the current stage
+        const int r = quad * 32 + lane, t0 = 8 * c4;
+        bool active;
+        const float* dl;  // lane's token's scales
+        int32_t* dbgt[8];
+        {
+          const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
+          active = t0 < f.n_valid;  // warp-uniform (the same for the four warps of this c4)
+          const int tl = t0 + (lane >> 2);
+          dl = tl < f.n_valid ? ad + item_token_row(f, GU, perm, top_k, tl) * nb : nullptr;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            dbgt[t] = nullptr;
+            if constexpr (DBG) {
+              if (t0 + t < f.n_valid) {
+                int32_t* base = dbg.buf + dbg_row(f, perm, top_k, dbg, t0 + t) * dbg_words(hidden, inter);
+                const int nbh = hidden / 32, nbi = inter / 32;
+                if constexpr (GU)
+                  dbgt[t] = r < kGroupRows ? base + (int64_t)(f.m0 + r) * nbh
+                                           : base + (int64_t)inter * nbh + (int64_t)(f.m0 + r - kGroupRows) * nbh;
+                else
+                  dbgt[t] = base + 2 * (int64_t)inter * nbh + (int64_t)(f.m0 + r) * nbi;
+              }
+            }
+          }
+        }
+        const int nh = (nst + 1) / 2;  // hand-offs: two stages each
+        for (int hh = 0; hh < nh; ++hh, ++gh) {
+          const int hb = gh % (kTBufs / kHalf);
+          const bool ok =
+              __all_sync(0xffffffffu, mbar_wait(&tfull_bar[hb], (gh / (kTBufs / kHalf)) & 1, abort, err, 13));
+          fence_after_sync();
+          if (active && ok) {
+            for (int jj = 0; jj < 2 && 2 * hh + jj < nst; ++jj) {
+              const int j = 2 * hh + jj;  // stage of this item
+              uint32_t rv[kBS][8];
+#pragma unroll
+              for (int c = 0; c < kBS; ++c)
+                tmem_ld8(tmem + lane_base + hb * kHalf * kN + jj * kBS * kNL + c * kNL + t0, rv[c]);
+              const float dxl = dl != nullptr ? __ldg(dl + j * kBS + (lane & 3)) : 0.0f;
+              tmem_ld_wait();
+#pragma unroll
+              for (int c = 0; c < kBS; ++c) {
+                const int b = j * kBS + c;
+#pragma unroll
+                for (int t = 0; t < 8; t += 2) {
+                  float v0, v1;
+                  isum2(rv[c][t], rv[c][t + 1], v0, v1);
+                  const float d0 = __shfl_sync(0xffffffffu, dxl, 4 * t + c);
+                  const float d1 = __shfl_sync(0xffffffffu, dxl, 4 * (t + 1) + c);
+                  if constexpr (DBG) {
+                    if (dbgt[t] != nullptr) dbgt[t][b] = (int32_t)v0;
+                    if (dbgt[t + 1] != nullptr) dbgt[t + 1][b] = (int32_t)v1;
+                  }
+                  fma2(acc0[t], acc0[t + 1], d0, d1, v0, v1);
+                }
+              }
+            }
+          }
+          fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty_bar[hb]);
+        }
+        if (active) {
+          const bool go = !*abort;
+          const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
+          if constexpr (GU) {
+            // up rows (quadrants 2, 3) hand their products to the gate rows'
+            // threads (quadrants 0, 1: same lane and c4) through shared memory
+            float* xu = &s_up[n_done & 1][c4][0][0];
+            const int o = f.m0 + (r & (kGroupRows - 1));  // intermediate row
+            if (r >= kGroupRows) {
+              const float su = __ldg(tab.up_s[f.slot.table_idx] + o);
+#pragma unroll
+              for (int t = 0; t < 8; ++t) xu[((quad - 2) * 32 + lane) * 8 + t] = __fmul_rn(su, acc0[t]);
+            }
+            named_bar(12 + c4, 128);  // the four warps of this c4
+            if (r < kGroupRows) {
+              const float sg = __ldg(tab.gate_s[f.slot.table_idx] + o);
+#pragma unroll
+              for (int t = 0; t < 8; ++t) {
+                const float gv = __fmul_rn(sg, acc0[t]);
+                const float u = xu[(quad * 32 + lane) * 8 + t];
+                const float h = __fmul_rn(__fmul_rn(gv, sigmoid_cw(gv)), u);
+                // Q8_0 block of h: the warp's 32 lanes are its 32 rows
+                const float d = __fdiv_rn(warp_max(fabsf(h)), 127.0f);
+                if (go && t0 + t < f.n_valid) {
+                  const int64_t row = (int64_t)f.slot.row_base + f.n0 + t0 + t;
+                  int pos = lane;  // int4 weights: element e of a group of 8 at e / 2 or 4 + e / 2
+                  if constexpr (BITS == 4) pos = (lane & ~7) + ((lane & 1) ? 4 + ((lane & 7) >> 1) : ((lane & 7) >> 1));
+                  hr[row * inter + (o & ~31) + pos] = (int8_t)q8_of(h, d);
+                  if (lane == 0) hd[row * (inter / 32) + (o >> 5)] = d;
+                }
+              }
+            }
+          } else if (go) {
+            const int o = f.m0 + r;  // output row
+            const float sd = __ldg(tab.down_s[f.slot.table_idx] + o);
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              if (t0 + t < f.n_valid)
+                y[((int64_t)f.slot.row_base + f.n0 + t0 + t) * hidden + o] = __fmul_rn(sd, acc0[t]);
           }
         }
       }
