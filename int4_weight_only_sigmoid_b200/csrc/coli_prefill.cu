@@ -34,22 +34,27 @@
 // applies contract F per block, so prefill equals the dp4a paths bit for
 // bit.
 //
-// Roles (640 threads): warps 0-1 producers (packed-weight copies; thread p
-// expands weight rows p and p + 64), warp 2 the A-tile TMA loads, warps 3-18
-// the fold (warp w reads TMEM lanes 32(w%4).. = 32 of the tile's tokens, and
-// a quarter of the item's columns: gate/up 16 gate rows and the same 16 up
-// rows, down 32 rows), warp 19 the MMA issuer (lane 0) and TMEM owner.  The
-// two fold warps that hold one Q8 block of h (32 intermediate rows) meet at
-// a named barrier to share the block's absmax.  (20 warps, 5 per scheduler,
-// leave 96 registers per thread.)
+// Roles (640 threads): warps 0-1 producers (each makes every other operand
+// stage on its own: packed-weight copies and the expansion of the stage's
+// 128 weight rows), warp 2 the A-tile TMA loads, warps 3-18 the fold, warp
+// 19 the MMA issuer (lane 0) and TMEM owner.  (20 warps, 5 per scheduler,
+// leave 96 registers per thread.)  Fold of an item of more than 32 tokens:
+// warp w reads TMEM lanes 32(w%4).. = 32 of the tile's tokens, and a quarter
+// of the item's columns (gate/up 16 gate rows and the same 16 up rows, down
+// 32 rows); the two warps that hold one Q8 block of h (32 intermediate rows)
+// meet at a named barrier to share the block's absmax.  An item of at most
+// 32 tokens is computed with the weights as the MMA's M (128 TMEM lanes) and
+// the tokens as its N (32 columns per block): warp w folds weight rows
+// 32(w%4).. for 8 of the tokens.
 // An operand stage holds 4 Q8 blocks (K = 128).  Per stage g: the TMA warp
 // loads its A tile into operand stage g % kStages once `empty` (the MMA's
-// commit) says the stage is free; the producers copy its packed weights
-// kLookS stages ahead (cp.async), expand them into the stage's B part and
-// arrive on `full`; the MMA issues one K=32 step per block onto a TMEM
-// accumulator per block (4 of them, handed to the fold kHalf blocks at a
-// time through `tfull` / `tempty`) and commits `empty`.  The fold reads a
-// buffer and releases it.  All waits are bounded (coli_tc.cuh).
+// commit) says the stage is free; a producer warp copies its packed weights
+// a few stages ahead (cp.async), expands them into the stage's B part and
+// arrives on `full`; the MMA issues one K=32 step per block onto a TMEM
+// accumulator per block (handed to the fold through `tfull` / `tempty`, two
+// blocks at a time, or eight for an item of at most 32 tokens) and commits
+// `empty`.  The fold reads a buffer and releases it.  All waits are bounded
+// (coli_tc.cuh).
 //
 // Sources: "Colibri：在笔记本上跑744B参数的AI模型", "关键特性" (integer dot
 // kernels, Q8_0 activations, packed int4); HN summary (hn.213312.xyz),
@@ -72,14 +77,14 @@ constexpr int kM = 128;        // tokens per tile (MMA M, TMEM lanes)
 constexpr int kN = 128;        // output columns per item (MMA N): 64 gate + 64 up rows, or 128 down rows
 constexpr int kBS = 4;         // Q8 blocks per operand stage (K = 128)
 constexpr int kStages = 4;     // operand stages
-// The producers' packed-weight copies run kLookS stages ahead, into kPkSlots
-// = kLookS + 2 slots (a slot is rewritten only after every producer expanded
-// it) of kPk bytes: int4 rows (64 B per stage) 6 ahead in 8 slots of 8 KB,
-// int8 rows (128 B) 2 ahead in 4 slots of 16 KB -- the same 64 KB.
+// The producers' packed-weight copies: kPkSlots slots of kPk bytes, int4
+// rows (64 B per stage) in 8 slots of 8 KB, int8 rows (128 B) in 4 slots of
+// 16 KB -- the same 64 KB.  Stage gs uses slot gs % kPkSlots; a producer
+// warp's stages are every kProdWarps-th, so a slot is reused only by the warp
+// that expanded its previous stage.
 template <int BITS>
 struct PkRing {
-  static constexpr int kLookS = BITS == 4 ? 6 : 2;
-  static constexpr int kPkSlots = kLookS + 2;
+  static constexpr int kPkSlots = BITS == 4 ? 8 : 4;
   static constexpr int kPk = 128 * 4 * BITS * 4;
 };
 static_assert(PkRing<4>::kPkSlots * PkRing<4>::kPk == PkRing<8>::kPkSlots * PkRing<8>::kPk, "one ring size");
@@ -95,8 +100,6 @@ constexpr int kTmaWarp = kProdWarps;                           // A-tile loads
 constexpr int kEpi0 = kProdWarps + 1;                          // first fold warp
 constexpr int kMmaWarp = kEpi0 + kEpiWarps;                    // MMA issuer, TMEM owner
 constexpr int kThreadsP = 32 * (kMmaWarp + 1);                 // 640
-constexpr int kNProd = 32 * kProdWarps;                        // producer threads
-static_assert(kN % kNProd == 0, "each producer thread expands whole weight rows");
 constexpr int kTmemCols = kTBufs * kN;                         // 512
 constexpr uint32_t kMagic = 0x4B400000u;                       // binary32 1.5 * 2^23
 constexpr float kMagicF = 12582912.0f;
@@ -314,7 +317,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_bar[s], kProdWarps + 1);  // + the TMA warp's expect_tx
+      mbar_init(&full_bar[s], 2);  // the stage's producer warp + the TMA warp's expect_tx
       mbar_init(&empty_bar[s], 1);
     }
     for (int b = 0; b < kTBufs / kHalf; ++b) {
@@ -334,106 +337,97 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
 
   if (warp < kProdWarps) {
     // ------------------------------------------------------------ producers
-    // A stage's packed weights (128 rows x 64 B) are copied 4 lanes per
-    // row, so that each warp instruction touches few cache lines; thread p
-    // then expands weight rows p, p + kNProd, ... of the stage's 4 blocks
-    // into the B operand.
-    // The copies run kLookS stages ahead across item boundaries: the issue
-    // cursor (item ii, stage ji) moves ahead of the expansion.  (The A tiles
-    // come from the TMA warp.)
-    const int p = threadIdx.x;
-    constexpr int kLookS = PkRing<BITS>::kLookS, kPkSlots = PkRing<BITS>::kPkSlots, kPk = PkRing<BITS>::kPk;
+    // Producer warp pw makes the operand stages gs = pw, pw + kProdWarps, ...
+    // of this CTA on its own: it copies the stage's packed weights (4 lanes
+    // per 64-byte int4 row, so that each instruction touches few cache lines)
+    // kLookW of its stages ahead with cp.async, and expands all 128 weight
+    // rows of the stage's 4 blocks into the B operand (lane l: rows l,
+    // l + 32, ...).  (The A tiles come from the TMA warp.)
+    constexpr int kPkSlots = PkRing<BITS>::kPkSlots, kPk = PkRing<BITS>::kPk;
+    constexpr int kLookW = kPkSlots / kProdWarps - 1;  // own stages in flight beyond the one expanded
+    const int pw = warp;
     const size_t rb = (size_t)dim_in * BITS / 8;  // bytes per weight row
     constexpr int kChunks = BITS == 4 ? 4 : 8;      // 16-byte chunks per row per stage
     const int n_mine = blockIdx.x < n_items ? (n_items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
     const int total = n_mine * nst;
-    int ii = blockIdx.x, ji = 0;
-    ItemInfo fi{};
-    auto enter_item = [&]() {
-      if (ii < n_items) fi = item_info(slots, tiles, ii, nm, kGroupRows);
-    };
-    // weight row r of the issue item: GU rows 0..63 gate, 64..127 up
-    auto wrow = [&](int r) -> const uint8_t* {
-      if constexpr (GU)
-        return (r < kGroupRows ? tab.gate_q[fi.slot.table_idx] : tab.up_q[fi.slot.table_idx]) +
-               (size_t)(fi.m0 + (r & (kGroupRows - 1))) * rb;
-      else
-        return tab.down_q[fi.slot.table_idx] + (size_t)(fi.m0 + r) * rb;
-    };
-    // packed-weight copies of the cursor's stage (global stage gj) into pk
-    // slot gj % kPkSlots; then the cursor moves on
+    // packed-weight copies of stage gj (the (gj / nst)-th item of this CTA)
+    // into pk slot gj % kPkSlots, as one commit group (empty past the end)
     auto issue = [&](int gj) {
       if (gj < total) {
+        const int k = gj / nst, ji = gj - k * nst;
+        const ItemInfo fi = item_info(slots, tiles, blockIdx.x + k * gridDim.x, nm, kGroupRows);
         const int kb0 = ji * kBS;
         unsigned char* pk = pk_ring + (gj % kPkSlots) * kPk;
-#pragma unroll
-        for (int it = 0; it < kChunks * kN / kNProd; ++it) {  // row q / kChunks, chunk q % kChunks of the stage's bytes
-          const int q = it * kNProd + p;
+#pragma unroll 4
+        for (int it = 0; it < kChunks * kN / 32; ++it) {  // row q / kChunks, chunk q % kChunks of the stage's bytes
+          const int q = it * 32 + lane;
           const int r = q / kChunks, c = q % kChunks;
-          cp_async16(pk + pk_off<BITS>(r, c), wrow(r) + (size_t)kb0 * (BITS * 4) + (size_t)c * 16);
+          const uint8_t* w;  // weight row r of the item: GU rows 0..63 gate, 64..127 up
+          if constexpr (GU)
+            w = (r < kGroupRows ? tab.gate_q[fi.slot.table_idx] : tab.up_q[fi.slot.table_idx]) +
+                (size_t)(fi.m0 + (r & (kGroupRows - 1))) * rb;
+          else
+            w = tab.down_q[fi.slot.table_idx] + (size_t)(fi.m0 + r) * rb;
+          cp_async16(pk + pk_off<BITS>(r, c), w + (size_t)kb0 * (BITS * 4) + (size_t)c * 16);
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        if (++ji == nst) {
-          ji = 0;
-          ii += gridDim.x;
-          enter_item();
-        }
-      } else {
-        asm volatile("cp.async.commit_group;" ::: "memory");
       }
+      asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    enter_item();
 #pragma unroll
-    for (int i = 0; i < kLookS; ++i) issue(i);
-    for (int gs = 0; gs < total; ++gs) {
-      issue(gs + kLookS);
-      asm volatile("cp.async.wait_group %0;" ::"n"(kLookS) : "memory");  // stage gs's copies (this thread's) are in
-      named_bar(1, kNProd);                                              // ... and every producer's
+    for (int u = 0; u < kLookW; ++u) issue(pw + u * kProdWarps);
+    for (int u = 0;; ++u) {
+      const int gs = pw + u * kProdWarps;
+      if (gs >= total) break;
+      issue(gs + kLookW * kProdWarps);
+      asm volatile("cp.async.wait_group %0;" ::"n"(kLookW) : "memory");  // stage gs's copies (this lane's) are in
+      __syncwarp();                                                       // ... and the warp's
       const int s = gs % kStages;
       // the MMA is done with the operand stage's previous contents
       if (mbar_wait(&empty_bar[s], ((gs / kStages) & 1) ^ 1, abort, err, 10) && !*abort) {
         const unsigned char* pk = pk_ring + (gs % kPkSlots) * kPk;
         unsigned char* ob = op_ring + s * L::kOpStage + L::kStageA;
-        if constexpr (BITS == 4) {
-          // all of this thread's packed words first, then the expansion and
-          // the stores
-          uint4 w[kN / kNProd][kBS];
+#pragma unroll 1
+        for (int rr = 0; rr < kN / 32; rr += 2) {
+          if constexpr (BITS == 4) {
+            // two rows' packed words first, then the expansion and the stores
+            uint4 w[2][kBS];
 #pragma unroll
-          for (int rr = 0; rr < kN / kNProd; ++rr)
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int c = 0; c < kBS; ++c)
-              w[rr][c] = *reinterpret_cast<const uint4*>(pk + pk_off<4>(p + rr * kNProd, c));
+              for (int c = 0; c < kBS; ++c)
+                w[h][c] = *reinterpret_cast<const uint4*>(pk + pk_off<4>(lane + (rr + h) * 32, c));
 #pragma unroll
-          for (int rr = 0; rr < kN / kNProd; ++rr) {
-            const int pr = p + rr * kNProd;  // the weight row this thread expands
+            for (int h = 0; h < 2; ++h) {
+              const int pr = lane + (rr + h) * 32;  // the weight row this lane expands
 #pragma unroll
-            for (int c = 0; c < kBS; ++c) {
-              unsigned char* dst = ob + c * L::kSubB;
-              uint4 o0, o1;
-              expand_word(w[rr][c].x, o0.x, o0.y);
-              expand_word(w[rr][c].y, o0.z, o0.w);
-              expand_word(w[rr][c].z, o1.x, o1.y);
-              expand_word(w[rr][c].w, o1.z, o1.w);
-              *reinterpret_cast<uint4*>(dst + op_off(pr, 0)) = o0;
-              *reinterpret_cast<uint4*>(dst + op_off(pr, 1)) = o1;
+              for (int c = 0; c < kBS; ++c) {
+                unsigned char* dst = ob + c * L::kSubB;
+                uint4 o0, o1;
+                expand_word(w[h][c].x, o0.x, o0.y);
+                expand_word(w[h][c].y, o0.z, o0.w);
+                expand_word(w[h][c].z, o1.x, o1.y);
+                expand_word(w[h][c].w, o1.z, o1.w);
+                *reinterpret_cast<uint4*>(dst + op_off(pr, 0)) = o0;
+                *reinterpret_cast<uint4*>(dst + op_off(pr, 1)) = o1;
+              }
             }
-          }
-        } else {  // int8 rows are the operand as they are
+          } else {  // int8 rows are the operand as they are
 #pragma unroll
-          for (int rr = 0; rr < kN / kNProd; ++rr) {
-            const int pr = p + rr * kNProd;
+            for (int h = 0; h < 2; ++h) {
+              const int pr = lane + (rr + h) * 32;
 #pragma unroll
-            for (int c = 0; c < kBS; ++c) {
-              unsigned char* dst = ob + c * L::kSubB;
-              const uint4 o0 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(pr, 2 * c));
-              const uint4 o1 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(pr, 2 * c + 1));
-              *reinterpret_cast<uint4*>(dst + op_off(pr, 0)) = o0;
-              *reinterpret_cast<uint4*>(dst + op_off(pr, 1)) = o1;
+              for (int c = 0; c < kBS; ++c) {
+                unsigned char* dst = ob + c * L::kSubB;
+                const uint4 o0 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(pr, 2 * c));
+                const uint4 o1 = *reinterpret_cast<const uint4*>(pk + pk_off<8>(pr, 2 * c + 1));
+                *reinterpret_cast<uint4*>(dst + op_off(pr, 0)) = o0;
+                *reinterpret_cast<uint4*>(dst + op_off(pr, 1)) = o1;
+              }
             }
           }
         }
       }
-      fence_async_smem();  // this thread's operand writes (stores and cp.async) -> the tensor core
+      fence_async_smem();  // this lane's operand writes -> the tensor core
       __syncwarp();
       if (lane == 0) mbar_arrive(&full_bar[s]);
     }
@@ -737,22 +731,26 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
         }
       } else {
         // light item: this thread's weight row r (0..127 of the item's 128
-        // rows) for the warp's 8 tokens t0 + t; lane 4 t + c holds the Q8
-        // scale of token t0 + t for block c of the current stage
-        const int r = quad * 32 + lane, t0 = 8 * c4;
+        // rows) for the warp's tw tokens t0 + t (the item's tokens split over
+        // the four warps of a quadrant, tw = 2, 4, 6 or 8); lane 4 t + c holds
+        // the Q8 scale of token t0 + t for block c of the current stage
+        const int r = quad * 32 + lane;
+        int tw, t0;
         bool active;
         const float* dl;  // lane's token's scales
         int32_t* dbgt[8];
         {
           const ItemInfo f = item_info(slots, tiles, item, nm, kGroupRows);
+          tw = 2 * ((f.n_valid + 7) / 8);  // tokens per warp
+          t0 = tw * c4;
           active = t0 < f.n_valid;  // warp-uniform (the same for the four warps of this c4)
           const int tl = t0 + (lane >> 2);
-          dl = tl < f.n_valid ? ad + item_token_row(f, GU, perm, top_k, tl) * nb : nullptr;
+          dl = (lane >> 2) < tw && tl < f.n_valid ? ad + item_token_row(f, GU, perm, top_k, tl) * nb : nullptr;
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
             dbgt[t] = nullptr;
             if constexpr (DBG) {
-              if (t0 + t < f.n_valid) {
+              if (t < tw && t0 + t < f.n_valid) {
                 int32_t* base = dbg.buf + dbg_row(f, perm, top_k, dbg, t0 + t) * dbg_words(hidden, inter);
                 const int nbh = hidden / 32, nbi = inter / 32;
                 if constexpr (GU)
@@ -765,6 +763,9 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
           }
         }
         const int nh = (nst + 1) / 2;  // hand-offs: two stages each
+        // the lane's Q8 scales for the next two stages, loaded two stages ahead
+        float dxn = dl != nullptr ? __ldg(dl + (lane & 3)) : 0.0f;
+        float dxn2 = dl != nullptr && nst > 1 ? __ldg(dl + kBS + (lane & 3)) : 0.0f;
         for (int hh = 0; hh < nh; ++hh, ++gh) {
           const int hb = gh % (kTBufs / kHalf);
           const bool ok =
@@ -777,13 +778,16 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
 #pragma unroll
               for (int c = 0; c < kBS; ++c)
                 tmem_ld8(tmem + lane_base + hb * kHalf * kN + jj * kBS * kNL + c * kNL + t0, rv[c]);
-              const float dxl = dl != nullptr ? __ldg(dl + j * kBS + (lane & 3)) : 0.0f;
+              const float dxl = dxn;
+              dxn = dxn2;
+              if (dl != nullptr && j + 2 < nst) dxn2 = __ldg(dl + (j + 2) * kBS + (lane & 3));
               tmem_ld_wait();
 #pragma unroll
               for (int c = 0; c < kBS; ++c) {
                 const int b = j * kBS + c;
 #pragma unroll
                 for (int t = 0; t < 8; t += 2) {
+                  if (t >= tw) break;  // warp-uniform
                   float v0, v1;
                   isum2(rv[c][t], rv[c][t + 1], v0, v1);
                   const float d0 = __shfl_sync(0xffffffffu, dxl, 4 * t + c);
@@ -812,13 +816,15 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
             if (r >= kGroupRows) {
               const float su = __ldg(tab.up_s[f.slot.table_idx] + o);
 #pragma unroll
-              for (int t = 0; t < 8; ++t) xu[((quad - 2) * 32 + lane) * 8 + t] = __fmul_rn(su, acc0[t]);
+              for (int t = 0; t < 8; ++t)
+                if (t < tw) xu[((quad - 2) * 32 + lane) * 8 + t] = __fmul_rn(su, acc0[t]);
             }
             named_bar(12 + c4, 128);  // the four warps of this c4
             if (r < kGroupRows) {
               const float sg = __ldg(tab.gate_s[f.slot.table_idx] + o);
 #pragma unroll
               for (int t = 0; t < 8; ++t) {
+                if (t >= tw) break;  // warp-uniform
                 const float gv = __fmul_rn(sg, acc0[t]);
                 const float u = xu[(quad * 32 + lane) * 8 + t];
                 const float h = __fmul_rn(__fmul_rn(gv, sigmoid_cw(gv)), u);
@@ -838,7 +844,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(
             const float sd = __ldg(tab.down_s[f.slot.table_idx] + o);
 #pragma unroll
             for (int t = 0; t < 8; ++t)
-              if (t0 + t < f.n_valid)
+              if (t < tw && t0 + t < f.n_valid)
                 y[((int64_t)f.slot.row_base + f.n0 + t0 + t) * hidden + o] = __fmul_rn(sd, acc0[t]);
           }
         }
