@@ -48,7 +48,10 @@ __global__ void __launch_bounds__(256) router_scores_kernel(const float* __restr
 // accumulator l of contract R (float4 number l + 32j of the row, ascending
 // j), and the 32 lane partials of each dot are summed left to right by one
 // lane after a transpose through shared memory.
-constexpr int kRtTok = 16, kRtExp = 16, kRtChunk = 128;  // chunk: float4 per row
+constexpr int kRtTok = 16, kRtExp = 16, kRtChunk = 64;  // chunk: float4 per row
+// the epilogue's per-warp transpose (8 warps x 32 dots x 33 floats) reuses
+// the staging buffers, which must hold it
+static_assert(2 * (kRtTok + kRtExp) * kRtChunk * 16 >= 8 * 32 * 33 * 4, "router tile staging too small");
 __global__ void __launch_bounds__(256) router_tiled_kernel(const float* __restrict__ x,
                                                            const float* __restrict__ wr, int n_tok, int E, int H,
                                                            float* __restrict__ scores) {
